@@ -1,0 +1,191 @@
+/*
+ * kvq.h -- single-token decode attention over a block-quantized KV cache with
+ * sparse V dequantization, for NVIDIA B200 (sm_100a).
+ *
+ * The method (tproger.ru, "Пропуск 90% работы по деквантизации ускорил
+ * декодирование LLM", sections "Решение — не ускорять, а пропускать" and
+ * "FAQ"): in a flash-attention decode kernel the softmax weights are known from
+ * K before any V work starts; every position whose weight exp(s_j - m_running)
+ * is below a threshold tau (the page uses 1e-6) has its V dequantization and
+ * accumulation skipped entirely.  K is always dequantized, because it produces
+ * the weights.  The page names q8_0, q4_0 and a Walsh-Hadamard-rotated
+ * codebook format (section "Почему это работает для любой квантизации").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All pointers named "device" are CUDA device pointers; "host" pointers are
+ *    ordinary CPU memory.  The caller owns every buffer; the library allocates
+ *    nothing and keeps no per-call state.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call that takes a stream is asynchronous on it.
+ *  - Return value: KVQ_OK or a negative KVQ_ERR_* code.  Argument checks run on
+ *    the host before anything is launched; on any error nothing is launched.
+ *    Faults detected inside a kernel (an out-of-range page index or sequence
+ *    length, a timed-out wait) set bits in the workspace's device flag word,
+ *    read back with kvq_read_device_flags(); outputs of such a call are
+ *    undefined.  No kernel traps.
+ *
+ * Cache layout (one "plane pair" for K, one for V)
+ * ------------------------------------------------
+ *  codes  plane: uint8  [num_pages][num_kv_heads][page_size][kvq_code_row_bytes(fmt, D)]
+ *  scales plane: fp16   [num_pages][num_kv_heads][page_size][kvq_scale_row_count(fmt, D)]
+ *  A "slot" is page * page_size + offset_in_page.  A contiguous cache is the
+ *  special case page_size = capacity, one page per sequence (page b for b).
+ *
+ *  q8_0  (32 int8 codes per block of 32 along head_dim, fp16 scale d):
+ *        d = absmax/127, q = round-half-away(x/d) in [-127, 127], x_hat = q*d.
+ *        codes row = D bytes (int8), scales row = D/32 fp16.
+ *  q4_0  (32 4-bit codes per block, fp16 scale d): m = the signed element of
+ *        largest |x|, d = m/-8, q = min(15, floor(x/d + 8.5)), x_hat = (q-8)*d.
+ *        codes row = D/2 bytes, element 2j in the low nibble of byte j and
+ *        element 2j+1 in the high nibble; scales row = D/32 fp16.
+ *  lut4  (rotated 4-bit codebook): y = c*H_D*(s .* x) with s the fixed random
+ *        signs, H_D the Sylvester Hadamard matrix and c = 1/sqrt(D); n = |y|;
+ *        idx = index of the codebook interval of y/n (thresholds at midpoints
+ *        of consecutive centroids); x_hat' = n*codebook[idx] in the rotated
+ *        domain.  codes row = D/2 bytes (nibbles as for q4_0); scales row = 1
+ *        fp16 (the norm n).  Attention runs in the rotated domain and the
+ *        output is rotated back (R^T = diag(s) c H_D), so every format returns
+ *        the same, unrotated, output.
+ *  All quantizer arithmetic is IEEE fp32 round-to-nearest-even, one operation
+ *  at a time (no fused multiply-add), so codes are fixed to the bit.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+#define KVQ_OK                0
+#define KVQ_ERR_INVALID_ARG  -1  /* null pointer, negative size, bad alignment, ... */
+#define KVQ_ERR_UNSUPPORTED  -2  /* format / head_dim / group size / page size not built */
+#define KVQ_ERR_CUDA         -3  /* a CUDA runtime call or launch failed */
+#define KVQ_ERR_WORKSPACE    -4  /* workspace too small */
+#define KVQ_ERR_DEVICE       -5  /* a kernel reported a fault through the flag word */
+
+/* ------------------------------------------------------------ formats */
+#define KVQ_FMT_Q8_0  0
+#define KVQ_FMT_Q4_0  1
+#define KVQ_FMT_LUT4  2
+
+/* Device flag bits (kvq_read_device_flags). */
+#define KVQ_FLAG_BAD_PAGE     1u  /* a page-table entry outside [0, num_pages) */
+#define KVQ_FLAG_BAD_SEQLEN   2u  /* seq_len < 0, > max_seq_len or > max_pages*page_size */
+#define KVQ_FLAG_TIMEOUT      4u  /* a bounded wait on an asynchronous copy gave up */
+
+/* Limits of this build. */
+#define KVQ_MAX_GROUP        8     /* query heads per KV head (num_q_heads / num_kv_heads) */
+#define KVQ_MAX_SPLIT_TOKENS 1024  /* positions per split-KV work unit */
+#define KVQ_MAX_BATCH        1024
+
+typedef struct kvq_cache_desc {
+    int32_t fmt;              /* KVQ_FMT_* */
+    int32_t head_dim;         /* 64 or 128 */
+    int32_t num_kv_heads;     /* >= 1 */
+    int32_t page_size;        /* tokens per page, a positive multiple of 64 */
+    int32_t num_pages;        /* physical pages held by each plane */
+    const uint16_t* codebook; /* lut4 only: device, 16 IEEE fp16 centroids, increasing */
+    const int8_t* signs;      /* lut4 only: device, head_dim entries, each +1 or -1 */
+} kvq_cache_desc;
+
+/* Bytes of one (token, KV head) row of the codes plane; 0 if (fmt, head_dim) is unsupported. */
+size_t kvq_code_row_bytes(int32_t fmt, int32_t head_dim);
+/* fp16 values in one row of the scales plane; 0 if unsupported. */
+size_t kvq_scale_row_count(int32_t fmt, int32_t head_dim);
+
+/*
+ * kvq_quantize -- write n_tokens K (or V) vectors into a cache plane pair.
+ *   x       device fp16 [n_tokens][num_kv_heads][head_dim]
+ *   slots   device int32 [n_tokens]: physical slot of token i (NULL: slot i);
+ *           every slot must lie in [0, num_pages*page_size) (not checked on device)
+ *   codes, scales  device planes (layout above), 16-byte aligned
+ * The block formulas are the ones in the header comment; the result is
+ * bit-identical to an IEEE fp32 evaluation of them.  lut4 needs desc->codebook
+ * and desc->signs.  n_tokens == 0 is a no-op.
+ */
+int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
+                 const int32_t* slots, void* codes, void* scales, void* stream);
+
+/*
+ * kvq_resolve_split -- the split length (positions per split-KV work unit) that
+ * kvq_decode_attn and kvq_combine use for a request.  split_tokens > 0 is
+ * rounded up to a multiple of 64 and capped at KVQ_MAX_SPLIT_TOKENS;
+ * split_tokens == 0 picks one from the problem size and the device's SM count
+ * (about one work unit per SM).  Returns the length (> 0) or a KVQ_ERR_* code.
+ * Sequence b is cut into splits [k*L, min((k+1)*L, seq_len_b)).
+ */
+int32_t kvq_resolve_split(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                          int32_t max_seq_len, int32_t split_tokens);
+
+/* Workspace bytes for a resolved split length L (> 0). */
+size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                          int32_t max_seq_len, int32_t split_tokens);
+
+/* Zero the workspace's device flag word (call once after allocating it). */
+int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronize `stream` and read the device flag word (KVQ_FLAG_* bits) into *flags (host). */
+int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
+
+/*
+ * kvq_decode_attn -- split-KV decode attention with sparse V, writing per-split
+ * partials (unnormalized o, running max m, denominator l) into the workspace.
+ *   q            device fp16 [batch][num_q_heads][head_dim]
+ *   k_codes, k_scales, v_codes, v_scales   device planes (layout above), 16-byte aligned
+ *   page_table   device int32 [batch][max_pages] (NULL: sequence b uses pages
+ *                b*max_pages .. b*max_pages + max_pages - 1)
+ *   seq_lens     device int32 [batch], each in [0, min(max_seq_len, max_pages*page_size)]
+ *   sm_scale     score scale (1/sqrt(head_dim) for standard attention)
+ *   tau          skip threshold, >= 0.  Position j of split s is skipped for
+ *                query head h when exp(s_hj - m_hs) < tau, with m_hs the running
+ *                maximum after all K tiles of the split are folded in; tau = 0
+ *                keeps everything (dense attention).  Skipped positions still
+ *                count in the softmax denominator.
+ *   split_tokens as for kvq_resolve_split (0 = auto)
+ *   stats        device uint64 [4] or NULL; ADDED to (caller zeroes):
+ *                [0] (position, query head) pairs scored, [1] pairs skipped,
+ *                [2] V rows read (positions kept by any head of the group),
+ *                [3] V rows skipped
+ * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
+ * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.
+ */
+int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
+                    int32_t num_q_heads, const void* k_codes, const void* k_scales,
+                    const void* v_codes, const void* v_scales, const int32_t* page_table,
+                    int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
+                    float sm_scale, float tau, int32_t split_tokens, void* workspace,
+                    size_t workspace_bytes, unsigned long long* stats, void* stream);
+
+/*
+ * kvq_combine -- log-sum-exp merge of the partials of kvq_decode_attn (same
+ * batch, num_q_heads, max_seq_len, split_tokens, seq_lens and workspace):
+ *   M = max_s m_s,  out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s,
+ * rotated back to the caller's basis for lut4.
+ *   out  device fp32 [batch][num_q_heads][head_dim]; a sequence of length 0
+ *        gets zeros.
+ */
+int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
+                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens,
+                const int32_t* seq_lens, float* out, void* stream);
+
+/*
+ * kvq_lloyd_max_codebook -- the minimum-MSE `levels`-entry scalar codebook for
+ * N(0, sigma^2) (Lloyd's iteration in fp64, symmetric), rounded to IEEE fp16
+ * (round-to-nearest-even) and written to out_fp16 (host, `levels` entries,
+ * increasing).  The lut4 format uses levels = 16, sigma = 1/sqrt(head_dim).
+ */
+int kvq_lloyd_max_codebook(int32_t levels, double sigma, uint16_t* out_fp16);
+
+/* A static, human-readable name for a status code. */
+const char* kvq_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

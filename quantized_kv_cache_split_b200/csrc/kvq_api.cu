@@ -1,0 +1,249 @@
+// C-ABI entry points of libkvq: argument validation, then one launch each.
+// Nothing here allocates device memory or keeps per-call state.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits) {
+  const size_t units = (size_t)batch * num_q_heads * max_splits;
+  return units * ((size_t)head_dim + 2) * sizeof(float);
+}
+
+int device_sm_count() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_desc(const kvq_cache_desc* d) {
+  if (!d) return KVQ_ERR_INVALID_ARG;
+  if (d->fmt != KVQ_FMT_Q8_0 && d->fmt != KVQ_FMT_Q4_0 && d->fmt != KVQ_FMT_LUT4)
+    return KVQ_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (d->num_kv_heads < 1 || d->num_pages < 1) return KVQ_ERR_INVALID_ARG;
+  if (d->page_size < 64 || d->page_size % 64 != 0) return KVQ_ERR_UNSUPPORTED;
+  if ((int64_t)d->num_pages * d->num_kv_heads * d->page_size > 0x7fffffffLL)
+    return KVQ_ERR_UNSUPPORTED;  // rows are addressed with 32-bit indices
+  if (d->fmt == KVQ_FMT_LUT4 && (!d->codebook || !d->signs)) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+int max_splits_for(int max_seq_len, int split_tokens) {
+  return (max_seq_len + split_tokens - 1) / split_tokens;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+size_t kvq_code_row_bytes(int32_t fmt, int32_t head_dim) {
+  if (head_dim != 64 && head_dim != 128) return 0;
+  if (fmt == KVQ_FMT_Q8_0) return (size_t)head_dim;
+  if (fmt == KVQ_FMT_Q4_0 || fmt == KVQ_FMT_LUT4) return (size_t)head_dim / 2;
+  return 0;
+}
+
+size_t kvq_scale_row_count(int32_t fmt, int32_t head_dim) {
+  if (head_dim != 64 && head_dim != 128) return 0;
+  if (fmt == KVQ_FMT_Q8_0 || fmt == KVQ_FMT_Q4_0) return (size_t)head_dim / 32;
+  if (fmt == KVQ_FMT_LUT4) return 1;
+  return 0;
+}
+
+int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
+                 const int32_t* slots, void* codes, void* scales, void* stream) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (n_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_tokens == 0) return KVQ_OK;
+  if (!x || !codes || !scales) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(x) & 1u))
+    return KVQ_ERR_INVALID_ARG;
+  if (!slots && (int64_t)n_tokens > (int64_t)desc->num_pages * desc->page_size)
+    return KVQ_ERR_INVALID_ARG;
+  return launch_quantize(*desc, x, n_tokens, slots, codes, scales,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int32_t kvq_resolve_split(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                          int32_t max_seq_len, int32_t split_tokens) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || max_seq_len < 0 || split_tokens < 0)
+    return KVQ_ERR_INVALID_ARG;
+  int L;
+  if (split_tokens > 0) {
+    L = split_tokens;
+  } else {
+    const int sms = device_sm_count();
+    if (sms <= 0) return KVQ_ERR_CUDA;
+    // about one work unit per SM if every sequence were max_seq_len long
+    const int64_t work = (int64_t)std::max(batch, 1) * desc->num_kv_heads * std::max(max_seq_len, 1);
+    L = (int)std::min<int64_t>((work + sms - 1) / sms, KVQ_MAX_SPLIT_TOKENS);
+  }
+  L = (L + kTile - 1) / kTile * kTile;
+  return std::max(kTile, std::min(L, KVQ_MAX_SPLIT_TOKENS));
+}
+
+size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                          int32_t max_seq_len, int32_t split_tokens) {
+  if (batch < 0 || num_q_heads < 0 || head_dim <= 0 || max_seq_len < 0 || split_tokens <= 0)
+    return 0;
+  return kWorkspaceHeader +
+         partials_bytes(batch, num_q_heads, head_dim, max_splits_for(max_seq_len, split_tokens));
+}
+
+int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes < kWorkspaceHeader) return KVQ_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, kWorkspaceHeader, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? KVQ_OK
+             : KVQ_ERR_CUDA;
+}
+
+int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream) {
+  if (!workspace || !flags) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaMemcpy(flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
+                    int32_t num_q_heads, const void* k_codes, const void* k_scales,
+                    const void* v_codes, const void* v_scales, const int32_t* page_table,
+                    int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
+                    float sm_scale, float tau, int32_t split_tokens, void* workspace,
+                    size_t workspace_bytes, unsigned long long* stats, void* stream) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || max_pages < 1 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (batch > KVQ_MAX_BATCH) return KVQ_ERR_UNSUPPORTED;
+  if (num_q_heads % desc->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  const int group = num_q_heads / desc->num_kv_heads;
+  if (group > KVQ_MAX_GROUP) return KVQ_ERR_UNSUPPORTED;
+  if (!(tau >= 0.0f) || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+  if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !seq_lens || !workspace)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_codes) || !aligned16(k_scales) || !aligned16(v_codes) || !aligned16(v_scales) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(q) & 1u))
+    return KVQ_ERR_INVALID_ARG;
+  if (!page_table && (int64_t)batch * max_pages > desc->num_pages) return KVQ_ERR_INVALID_ARG;
+  const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
+  if (L < 0) return L;
+  const size_t need = kvq_workspace_size(batch, num_q_heads, desc->head_dim, max_seq_len, L);
+  if (workspace_bytes < need) return KVQ_ERR_WORKSPACE;
+  if (batch == 0 || max_seq_len == 0) return KVQ_OK;
+  DecodeArgs a;
+  a.desc = *desc;
+  a.q = q;
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.group = group;
+  a.k_codes = k_codes;
+  a.k_scales = k_scales;
+  a.v_codes = v_codes;
+  a.v_scales = v_scales;
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.max_seq_len = max_seq_len;
+  a.sm_scale = sm_scale;
+  a.tau = tau;
+  a.split_tokens = L;
+  a.max_splits = max_splits_for(max_seq_len, L);
+  a.workspace = workspace;
+  a.stats = stats;
+  a.num_sms = device_sm_count();
+  if (a.num_sms <= 0) return KVQ_ERR_CUDA;
+  return launch_decode(a, static_cast<cudaStream_t>(stream));
+}
+
+int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
+                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens,
+                const int32_t* seq_lens, float* out, void* stream) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (!workspace || !seq_lens || !out) return KVQ_ERR_INVALID_ARG;
+  const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
+  if (L < 0) return L;
+  if (batch == 0) return KVQ_OK;
+  return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L,
+                        max_splits_for(max_seq_len, L), seq_lens, out,
+                        static_cast<cudaStream_t>(stream));
+}
+
+// Lloyd's iteration for N(0, sigma^2): thresholds at midpoints, centroids at the
+// conditional means sigma * (phi(a) - phi(b)) / (Phi(b) - Phi(a)).
+int kvq_lloyd_max_codebook(int32_t levels, double sigma, uint16_t* out_fp16) {
+  if (levels < 2 || levels > 256 || !(sigma > 0.0) || !out_fp16) return KVQ_ERR_INVALID_ARG;
+  const double inv_sqrt2pi = 0.3989422804014327;
+  auto pdf = [&](double z) { return isinf(z) ? 0.0 : inv_sqrt2pi * exp(-0.5 * z * z); };
+  auto cdf = [&](double z) {
+    if (isinf(z)) return z > 0 ? 1.0 : 0.0;
+    return 0.5 * erfc(-z * 0.7071067811865476);
+  };
+  std::vector<double> cen(levels), nxt(levels), edge(levels + 1);
+  for (int i = 0; i < levels; ++i) cen[i] = -2.0 + 4.0 * i / (levels - 1);  // unit-variance start
+  for (int iter = 0; iter < 200000; ++iter) {
+    edge[0] = -INFINITY;
+    edge[levels] = INFINITY;
+    for (int i = 1; i < levels; ++i) edge[i] = 0.5 * (cen[i - 1] + cen[i]);
+    for (int i = 0; i < levels; ++i) {
+      const double mass = cdf(edge[i + 1]) - cdf(edge[i]);
+      nxt[i] = (pdf(edge[i]) - pdf(edge[i + 1])) / mass;
+    }
+    double move = 0.0;
+    for (int i = 0; i < levels; ++i) {
+      const double v = 0.5 * (nxt[i] - nxt[levels - 1 - i]);  // keep it exactly symmetric
+      move = std::max(move, fabs(v - cen[i]));
+      cen[i] = v;
+    }
+    if (move < 1e-13) break;
+  }
+  for (int i = 0; i < levels; ++i) {
+    const __half h = __double2half(cen[i] * sigma);
+    out_fp16[i] = __half_as_ushort(h);
+  }
+  return KVQ_OK;
+}
+
+const char* kvq_status_string(int status) {
+  switch (status) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+    case KVQ_ERR_DEVICE: return "device-side fault reported";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle on
+the same seeded inputs.  Quantized planes must match bit for bit; attention
+outputs must satisfy the error bound of the method; skip counters must match
+the oracle's under the same split schedule within 0.1%."""
+import math
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+import workloads as W  # noqa: E402
+from oracle import quant as OQ  # noqa: E402
+from tests.gpu_helpers import check_parity, codebook_for, run_library, run_oracle  # noqa: E402
+
+
+# ------------------------------------------------------------------ quantizers: bit-exact
+
+def _special_vectors(rng, n, hkv, D):
+    x = (rng.standard_normal((n, hkv, D)) * rng.choice([0.01, 1.0, 30.0], (n, hkv, 1))).astype(np.float16)
+    x[0] = 0                                    # all-zero vector / blocks
+    x[1, :, :] = 1.5                            # |x| ties everywhere
+    x[1, :, 1::2] = -1.5
+    x[2, :, :32] = np.float16(6e-5)             # subnormal-range values
+    x[3, :, 5] = np.float16(-60000.0)           # one huge element
+    x[4, :, :] = np.arange(D, dtype=np.float16) - D // 2
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_quantize_bit_exact(fmt, D):
+    import quantized_kv_cache_split_b200 as K
+    rng = np.random.Generator(np.random.PCG64(77))
+    hkv, P, npages, n = 2, 64, 6, 333
+    x = _special_vectors(rng, n, hkv, D)
+    slots = rng.permutation(npages * P)[:n].astype(np.int32)
+    dev = torch.device("cuda")
+    cb16 = codebook_for(D) if fmt == "lut4" else None
+    signs = np.where(rng.random(D) < 0.5, -1, 1).astype(np.int8) if fmt == "lut4" else None
+    cache = K.QuantizedKVCache(fmt, D, hkv, P, npages, dev,
+                               None if cb16 is None else torch.from_numpy(cb16.view(np.int16).copy()),
+                               None if signs is None else torch.from_numpy(signs))
+    xt = torch.from_numpy(x).to(dev)
+    cache.write(xt, xt, torch.from_numpy(slots).to(dev))
+    torch.cuda.synchronize()
+    codes = cache.k_codes.cpu().numpy()
+    scales = cache.k_scales.cpu().numpy()
+    page, off = slots // P, slots % P
+    for h in range(hkv):
+        got_c = codes[page, h, off]
+        got_s = scales[page, h, off]
+        c, s = OQ.quantize(fmt, x[:, h], signs, cb16)
+        want_c = c.astype(np.int8).view(np.uint8) if fmt == "q8_0" else OQ.pack_nibbles(c)
+        assert np.array_equal(got_c, want_c), f"codes differ at {np.argwhere(got_c != want_c)[:5]}"
+        assert np.array_equal(got_s.view(np.uint16), s.astype(np.float16).view(np.uint16)), "scales"
+    assert np.array_equal(cache.v_codes.cpu().numpy(), codes)
+
+
+# ------------------------------------------------------------------ attention parity
+
+SMALL = [
+    ("tiny_q8_d64", 1e-6, 0), ("tiny_q8_d64", 0.0, 0), ("tiny_q8_d64", 1e-6, 64),
+    ("gqa_4k_q8", 1e-6, 0), ("gqa_4k_q8", 0.0, 0), ("gqa_4k_q8", 1e-6, 1024),
+    ("lut_4k", 1e-6, 0), ("lut_4k", 0.0, 0),
+]
+
+
+@pytest.mark.parametrize("name,tau,split", SMALL)
+def test_decode_parity_small(name, tau, split):
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
+    g = run_library(inp, tau, split, cb)
+    o = run_oracle(inp, tau, g["split"], cb)
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+
+
+RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("tau,split", [(0.0, 128), (1e-6, 0), (1e-4, 192), (1e-6, 1024)])
+def test_decode_parity_paged_ragged(fmt, tau, split):
+    base = W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt)
+    wl = W.shrink(base, RAGGED_LENS, n_planted=8)
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if fmt == "lut4" else None
+    g = run_library(inp, tau, split, cb)
+    o = run_oracle(inp, tau, g["split"], cb)
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (8, 1)])
+def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
+    wl = W.WORKLOADS["tiny_q8_d64"].with_(fmt=fmt, num_q_heads=hq, num_kv_heads=hkv,
+                                          seq_lens=(777, 300), batch=2, n_planted=6)
+    inp = W.generate(wl)
+    cb = codebook_for(64) if fmt == "lut4" else None
+    for tau, split in [(1e-6, 0), (0.0, 64)]:
+        g = run_library(inp, tau, split, cb)
+        o = run_oracle(inp, tau, g["split"], cb)
+        check_parity(inp, g, o, tau)
+
+
+# ------------------------------------------------------------------ full sizes
+
+@pytest.mark.parametrize("name", ["gqa_32k_q4", "lut_32k"])
+@pytest.mark.parametrize("tau", [1e-6, 0.0])
+def test_decode_parity_full_32k(name, tau):
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
+    g = run_library(inp, tau, 0, cb)
+    o = run_oracle(inp, tau, g["split"], cb)
+    check_parity(inp, g, o, tau)
+    if tau > 0:
+        # the workload's point: most weights are skipped
+        assert g["stats"][1] > 0.5 * g["stats"][0]
+
+
+@pytest.mark.parametrize("name", ["paged_b8_q4", "paged_b8_q8"])
+def test_decode_parity_full_paged(name):
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    g = run_library(inp, 1e-6, 0)
+    # full output on three (sequence, KV head) groups computed one by one by the oracle,
+    # plus the exact counters over everything
+    groups = [(3, 0), (0, 2), (7, 3)]
+    o = run_oracle(inp, 1e-6, g["split"], groups=groups)
+    check_parity(inp, g, o, 1e-6, groups=groups)
+    total = int(inp.seq_lens.sum())
+    assert g["stats"][0] == total * wl.num_q_heads
+    assert g["stats"][2] + g["stats"][3] == total * wl.num_kv_heads
+
+
+# ------------------------------------------------------------------ device-side fault reporting
+
+def test_bad_page_index_is_flagged_not_faulted():
+    import quantized_kv_cache_split_b200 as K
+    wl = W.shrink(W.WORKLOADS["paged_b8_q8"], [200, 100], n_planted=2)
+    inp = W.generate(wl)
+    inp.page_table[1, 0] = inp.num_pages + 5          # out of range: must not be read
+    g = run_library(inp, 1e-6, 0)
+    assert g["flags"] & K.KVQ_FLAG_BAD_PAGE
+
+
+def test_bad_seq_len_is_flagged_and_clamped():
+    import quantized_kv_cache_split_b200 as K
+    wl = W.shrink(W.WORKLOADS["gqa_4k_q8"], [300], n_planted=2)
+    inp = W.generate(wl)
+    dev = torch.device("cuda")
+    cache = K.QuantizedKVCache("q8_0", 128, 8, inp.page_size, inp.num_pages, dev)
+    cache.write(torch.from_numpy(inp.k).to(dev), torch.from_numpy(inp.v).to(dev),
+                torch.from_numpy(inp.slots).to(dev))
+    seq = torch.tensor([300 + 5000], dtype=torch.int32, device=dev)   # beyond max_seq_len
+    cache.attention(torch.from_numpy(inp.q).to(dev), seq, 300, None, 1, tau=1e-6)
+    assert cache.device_flags() & K.KVQ_FLAG_BAD_SEQLEN

@@ -1,0 +1,499 @@
+"""Benchmark: single-token decode attention over a block-quantized KV cache with
+sparse V dequantization, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa_32k_q4] [--tau 1e-6]
+
+One step = the whole decode-attention hot path for one decode token of every
+sequence in the workload: split-KV decode kernel (K tiles -> scores -> running
+max -> skip decision -> kept V only) + log-sum-exp combine.  Inputs are resident
+in HBM; the cache is replicated into enough copies that successive steps rotate
+through more than 3x the L2 size, so every step reads HBM.  Prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference available for
+this method) on bounded samples of the same workload.
+Multi-GPU (torchrun): every rank runs an independent replica (no collective on
+the data path; weak scaling); timings are reduced with MAX over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "decode-attn µs/token & achieved KV HBM GB/s at 32K ctx, sparse-V vs dense"
+UNIT = "us/token"
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
+DECODE_SRC = os.path.join(ROOT, "quantized_kv_cache_split_b200", "csrc", "kvq_decode.cu")
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as td
+    if world > 1 and not td.is_initialized():
+        import datetime
+        td.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return td
+
+
+def reduce_max(value: float, world: int, device="cpu") -> float:
+    """MAX over ranks of a per-rank float (timings)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as td
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    td.all_reduce(t, op=td.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as td
+        td.barrier()
+
+
+# ------------------------------------------------------------------ clocks (NVML, sampled during timing)
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, cuda_index: int):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(cuda_index)
+            try:
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            f = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self._reason_fn = f
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML here
+            self.err = str(e)
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        self.reasons |= int(self._reason_fn(self.h))
+
+    def start(self):
+        if not self.ok:
+            return
+        self._stop = False
+        self._sample()
+
+        def run():
+            while not self._stop:
+                self._sample()
+                time.sleep(0.001)
+        self.t = threading.Thread(target=run, daemon=True)
+        self.t.start()
+
+    def stop(self):
+        if not self.ok:
+            return
+        self._stop = True
+        self.t.join()
+        self._sample()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for b, n in _REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def traffic_from_profile(unit_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    try:
+        prof = json.load(open(PROFILE_TRAFFIC))
+        src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+        if prof.get("source_sha256_16") != src_hash:
+            return None
+        ent = prof["launches"].get(unit_key)
+        return None if ent is None else float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def measured_peaks():
+    try:
+        p = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class Replicas:
+    """R copies of the quantized cache so that successive steps miss in L2."""
+
+    def __init__(self, wl: W.Workload, inp: W.Inputs, device, min_bytes: int):
+        import torch
+        import quantized_kv_cache_split_b200 as K
+        self.wl, self.inp = wl, inp
+        D = wl.head_dim
+        cb = sg = None
+        if wl.fmt == "lut4":
+            cb = torch.from_numpy(K.kvq_lloyd_max_codebook(16, 1.0 / math.sqrt(D)).view(np.int16).copy())
+            sg = torch.from_numpy(inp.signs)
+        first = K.QuantizedKVCache(wl.fmt, D, wl.num_kv_heads, inp.page_size, inp.num_pages,
+                                   device, cb, sg)
+        first.write(torch.from_numpy(inp.k).to(device), torch.from_numpy(inp.v).to(device),
+                    torch.from_numpy(inp.slots).to(device))
+        plane_bytes = sum(t.numel() * t.element_size()
+                          for t in (first.k_codes, first.k_scales, first.v_codes, first.v_scales))
+        self.plane_bytes = plane_bytes
+        self.R = max(2, math.ceil(min_bytes / plane_bytes))
+        self.caches = [first]
+        for _ in range(self.R - 1):
+            c = K.QuantizedKVCache(wl.fmt, D, wl.num_kv_heads, inp.page_size, inp.num_pages,
+                                   device, first.codebook, first.signs)
+            for dst, src in ((c.k_codes, first.k_codes), (c.k_scales, first.k_scales),
+                             (c.v_codes, first.v_codes), (c.v_scales, first.v_scales)):
+                dst.copy_(src)
+            self.caches.append(c)
+        self.q = torch.from_numpy(inp.q).to(device)
+        self.seq = torch.from_numpy(inp.seq_lens).to(device)
+        self.pt = None if inp.page_table is None else torch.from_numpy(inp.page_table).to(device)
+        self.max_seq = int(inp.seq_lens.max())
+        self.B, self.Hq, self.D = wl.batch, wl.num_q_heads, D
+        self.L = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, 0)
+        self.ws_bytes = K.kvq_workspace_size(self.B, self.Hq, D, self.max_seq, self.L)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        K.kvq_workspace_init(self.ws, self.ws_bytes)
+        self.out = torch.empty((self.B, self.Hq, D), dtype=torch.float32, device=device)
+        self.sm = float(np.float32(1.0 / math.sqrt(D)))
+
+    def decode(self, i, tau, stats=None):
+        import quantized_kv_cache_split_b200 as K
+        c = self.caches[i % self.R]
+        K.kvq_decode_attn(c.desc, self.q, self.B, self.Hq, c.k_codes, c.k_scales, c.v_codes,
+                          c.v_scales, self.pt, self.inp.max_pages, self.seq, self.max_seq, self.sm,
+                          tau, self.L, self.ws, self.ws_bytes, stats)
+
+    def combine(self, i):
+        import quantized_kv_cache_split_b200 as K
+        c = self.caches[i % self.R]
+        K.kvq_combine(c.desc, self.ws, self.B, self.Hq, self.max_seq, self.L, self.seq, self.out)
+
+
+def capture(fn, n_steps, start):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n_steps):       # warm the capture-time host paths once
+            fn(start + i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i in range(n_steps):
+            fn(start + i)
+    return g
+
+
+class GraphRunner:
+    """Launch exactly n steps of `fn` through CUDA graphs: one graph of R steps
+    (copies 0..R-1) plus single-step graphs for the remainder."""
+
+    def __init__(self, fn, R):
+        self.R = R
+        self.full = capture(fn, R, 0)
+        self.single = [capture(fn, 1, i) for i in range(R)]
+
+    def run(self, n, offset=0):
+        """Steps offset .. offset + n - 1 (copy index = step % R)."""
+        i = offset
+        while i % self.R and n:
+            self.single[i % self.R].replay(); i += 1; n -= 1
+        while n >= self.R:
+            self.full.replay(); i += self.R; n -= self.R
+        while n:
+            self.single[i % self.R].replay(); i += 1; n -= 1
+
+
+def time_steps(runner, steps, warmup, world, sampler=None):
+    import torch
+    runner.run(warmup, 0)
+    torch.cuda.synchronize()
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.start()
+    start.record()
+    runner.run(steps, warmup)
+    end.record()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.stop()
+    barrier(world)
+    return start.elapsed_time(end)
+
+
+def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_splits_total: int):
+    """HBM bytes one decode launch must move: all K rows, the kept V rows,
+    Q, the page table, and the partials written."""
+    import quantized_kv_cache_split_b200 as K
+    wl = rep.wl
+    row = K.kvq_code_row_bytes(wl.fmt, wl.head_dim) + 2 * K.kvq_scale_row_count(wl.fmt, wl.head_dim)
+    tokens = int(rep.inp.seq_lens.sum())
+    k_bytes = tokens * wl.num_kv_heads * row
+    v_bytes = v_rows_read * row
+    q_bytes = wl.batch * wl.num_q_heads * wl.head_dim * 2
+    pt_bytes = 0 if rep.inp.page_table is None else sum(
+        (int(n) + rep.inp.page_size - 1) // rep.inp.page_size for n in rep.inp.seq_lens) * 4
+    part_bytes = n_splits_total * wl.group * (wl.head_dim + 2) * 4
+    return k_bytes + v_bytes + q_bytes + pt_bytes + part_bytes
+
+
+def gpu_arm(args, world, rank, local):
+    import torch
+    import quantized_kv_cache_split_b200 as K
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    wl = W.WORKLOADS[args.workload]
+    inp = W.generate(wl)
+    rep = Replicas(wl, inp, device, 3 * L2_BYTES)
+    n_splits_total = sum(wl.num_kv_heads * ((int(n) + rep.L - 1) // rep.L) for n in inp.seq_lens)
+
+    def counters(tau):
+        st = torch.zeros(4, dtype=torch.int64, device=device)
+        rep.decode(0, tau, st)
+        torch.cuda.synchronize()
+        return [int(x) for x in st.cpu()]
+
+    res = {}
+    hbm_peak, peak_kind = measured_peaks()
+    sampler = ClockSampler(local)
+    for tag, tau in (("sparse", args.tau), ("dense", 0.0)):
+        st = counters(tau)
+        step = GraphRunner(lambda i: (rep.decode(i, tau), rep.combine(i)), rep.R)
+        dec = GraphRunner(lambda i: rep.decode(i, tau), rep.R)
+        ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
+                                        sampler if tag == "sparse" else None), world, device)
+        ms_dec = reduce_max(time_steps(dec, args.steps, args.warmup, world), world, device)
+        abytes = algorithmic_bytes(rep, st[2], n_splits_total)
+        us_launch = ms_dec * 1e3 / args.steps
+        achieved = abytes / (us_launch * 1e-6) / 1e9
+        res[tag] = dict(tau=tau, ms_per_step=ms_step / args.steps,
+                        us_per_token=ms_step * 1e3 / args.steps / (wl.batch * world),
+                        decode_us_per_launch=us_launch, algorithmic_bytes=abytes,
+                        achieved_gbs=achieved, frac=achieved / hbm_peak,
+                        skipped_pair_frac=st[1] / max(st[0], 1),
+                        v_rows_read=st[2], v_rows_skipped=st[3],
+                        traffic=traffic_from_profile(f"{args.workload}:{tag}"))
+        del step, dec
+    e2e = None if args.skip_e2e else e2e_arm(args, rep, wl, inp, device, world)
+    sp = res["sparse"]
+    line = {
+        "metric": METRIC, "value": round(sp["us_per_token"], 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sp["ms_per_step"], 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": wl.batch, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
+                   "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
+                   "l2": f"inputs rotate over {rep.R} cache copies "
+                         f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "step": "kvq_decode_attn + kvq_combine (CUDA graph)"},
+        "roofline": {"bound": "hbm", "achieved": round(sp["achieved_gbs"], 1),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(sp["frac"], 4),
+                     "traffic": sp["traffic"], "peak_kind": peak_kind,
+                     "kernel": "kvq decode_kernel<q4_0,128>" if wl.fmt == "q4_0" else f"decode_kernel<{wl.fmt}>",
+                     "algorithmic_bytes_per_launch": sp["algorithmic_bytes"],
+                     "us_per_launch": round(sp["decode_us_per_launch"], 3)},
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "dense": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res["dense"].items()},
+        "sparse": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in sp.items()},
+        "clocks": sampler.report(),
+    }
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        line["cpu_baseline"] = cpu_baseline(wl, inp, rep.L, args.tau, budget_s=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as td
+        td.barrier()
+        td.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e_arm(args, rep, wl, inp, device, world):
+    """Same metric through the public API with host buffers: every step copies the new
+    token's q, k, v from pinned host memory, appends k/v to the cache (kvq_quantize),
+    runs decode + combine, and reads the output back to pinned host memory."""
+    import torch
+    B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+    h_q = torch.from_numpy(inp.q).pin_memory()
+    h_k = torch.from_numpy(inp.k[-B:]).pin_memory()      # the newest position of each sequence
+    h_v = torch.from_numpy(inp.v[-B:]).pin_memory()
+    last = torch.from_numpy(np.array([int(inp.slots[int(o) - 1]) for o in inp.seq_offsets()[1:]],
+                                     dtype=np.int32)).to(device)
+    h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
+    d_q = torch.empty_like(h_q, device=device)
+    d_k = torch.empty((B, Hkv, D), dtype=torch.float16, device=device)
+    d_v = torch.empty_like(d_k)
+    out = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
+
+    def step(i):
+        c = rep.caches[i % rep.R]
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        c.write(d_k, d_v, last)
+        c.attention(d_q, rep.seq, rep.max_seq, rep.pt, inp.max_pages, tau=args.tau,
+                    sm_scale=rep.sm, split_tokens=rep.L, out=out)
+        h_out.copy_(out, non_blocking=True)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    torch.cuda.synchronize()
+    el = reduce_max(time.perf_counter() - t0, world, device)
+    bi = h_q.numel() * 2 + h_k.numel() * 2 + h_v.numel() * 2
+    bo = h_out.numel() * 4
+    return {"value": round(el * 1e6 / args.steps / (B * world), 3), "unit": UNIT,
+            "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "how": "eager public API per step: H2D(q,k,v) + QuantizedKVCache.write + .attention + D2H(out)"}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+
+def _oracle_sample(wl, inp, split, tau, n_pos):
+    """One bounded sample: the oracle's sparse-V decode for the first KV head of the
+    first sequence, truncated to n_pos positions.  Returns (seconds, fraction of the
+    workload's (position, KV head) units it covers)."""
+    from oracle import attention as OA
+    from oracle import codebook as OC
+    cb = OC.lloyd_max_f16(16, 1.0 / math.sqrt(wl.head_dim)) if wl.fmt == "lut4" else None
+    seq = np.array([n_pos], dtype=np.int32)
+    t0 = time.perf_counter()
+    OA.decode_step(wl.fmt, inp.q[:1], inp.k[:n_pos], inp.v[:n_pos], seq, wl.num_kv_heads,
+                   1.0 / math.sqrt(wl.head_dim), tau, split, signs=inp.signs, codebook16=cb,
+                   with_dense=False, groups=[(0, 0)])
+    dt = time.perf_counter() - t0
+    frac = n_pos / (int(inp.seq_lens.sum()) * wl.num_kv_heads)
+    return dt, frac
+
+
+def cpu_baseline(wl, inp, split, tau, budget_s=15.0):
+    from threadpoolctl import threadpool_limits
+    n_pos = int(inp.seq_lens[0])
+    with threadpool_limits(limits=1):
+        times, frac = [], None
+        t_end = time.perf_counter() + budget_s
+        while time.perf_counter() < t_end or not times:
+            dt, frac = _oracle_sample(wl, inp, split, tau, n_pos)
+            times.append(dt)
+    us_per_step = statistics.median(times) / frac * 1e6
+    return {"value": round(us_per_step / wl.batch, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"fp64 numpy oracle (quantize + dequant + schedule-exact sparse-V attention) "
+                      f"on 1 of {wl.num_kv_heads} KV heads x {n_pos} positions, {len(times)} runs, "
+                      f"scaled to the whole workload"}
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    inp = W.generate(wl)
+    from threadpoolctl import threadpool_limits
+    # size one step so that warmup + steps finish in about args.ref_budget seconds
+    with threadpool_limits(limits=1):
+        pilot = 1024
+        dt, _ = _oracle_sample(wl, inp, 896, args.tau, pilot)
+        per_pos = dt / pilot
+        n_pos = int(args.ref_budget / max(args.steps + args.warmup, 1) / per_pos)
+        n_pos = max(64, min(n_pos, int(inp.seq_lens[0])))
+        for _ in range(args.warmup):
+            _oracle_sample(wl, inp, 896, args.tau, n_pos)
+        t = []
+        frac = None
+        for _ in range(args.steps):
+            dt, frac = _oracle_sample(wl, inp, 896, args.tau, n_pos)
+            t.append(dt)
+    us_step = sum(t) / len(t) / frac * 1e6
+    value = us_step / wl.batch
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(us_step / 1e3, 3), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "cache_format": wl.fmt, "tau": args.tau,
+                       "split_tokens": 896},
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: fp64 oracle on 1 KV head x {n_pos} positions, "
+                                       f"scaled to the whole workload"},
+            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gqa_32k_q4", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--tau", type=float, default=1e-6)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0)
+    ap.add_argument("--skip-e2e", action="store_true", help="(profiling runs) skip the e2e leg")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+    gpu_arm(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -82,6 +82,7 @@ extern "C" {
 #define KVQ_MAX_GROUP        8     /* query heads per KV head (num_q_heads / num_kv_heads) */
 #define KVQ_MAX_SPLIT_TOKENS 1024  /* positions per split-KV work unit */
 #define KVQ_MAX_BATCH        1024
+#define KVQ_MAX_SPLITS       4096  /* splits of one sequence: max_seq_len <= 4096 * split length */
 
 typedef struct kvq_cache_desc {
     int32_t fmt;              /* KVQ_FMT_* */

@@ -140,12 +140,12 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------- dequant (fp64)
 
 def dequantize_q8_0(codes: np.ndarray, scales16: np.ndarray) -> np.ndarray:
-    c = codes.astype(np.float64).reshape(codes.shape[:-1] + (-1, BLOCK))
+    c = codes.astype(np.float64).reshape(codes.shape[:-1] + (codes.shape[-1] // BLOCK, BLOCK))
     return (c * scales16.astype(np.float64)[..., None]).reshape(codes.shape)
 
 
 def dequantize_q4_0(codes: np.ndarray, scales16: np.ndarray) -> np.ndarray:
-    c = (codes.astype(np.float64) - 8.0).reshape(codes.shape[:-1] + (-1, BLOCK))
+    c = (codes.astype(np.float64) - 8.0).reshape(codes.shape[:-1] + (codes.shape[-1] // BLOCK, BLOCK))
     return (c * scales16.astype(np.float64)[..., None]).reshape(codes.shape)
 
 

@@ -35,6 +35,7 @@ KVQ_FLAG_TIMEOUT = 4
 KVQ_MAX_GROUP = 8
 KVQ_MAX_SPLIT_TOKENS = 1024
 KVQ_MAX_BATCH = 1024
+KVQ_MAX_SPLITS = 4096
 
 
 class KvqCacheDesc(ctypes.Structure):

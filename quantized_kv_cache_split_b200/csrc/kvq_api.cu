@@ -156,6 +156,7 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   if (!page_table && (int64_t)batch * max_pages > desc->num_pages) return KVQ_ERR_INVALID_ARG;
   const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
   if (L < 0) return L;
+  if (max_splits_for(max_seq_len, L) > KVQ_MAX_SPLITS) return KVQ_ERR_UNSUPPORTED;
   const size_t need = kvq_workspace_size(batch, num_q_heads, desc->head_dim, max_seq_len, L);
   if (workspace_bytes < need) return KVQ_ERR_WORKSPACE;
   if (batch == 0 || max_seq_len == 0) return KVQ_OK;
@@ -193,6 +194,7 @@ int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch
   if (!workspace || !seq_lens || !out) return KVQ_ERR_INVALID_ARG;
   const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
   if (L < 0) return L;
+  if (max_splits_for(max_seq_len, L) > KVQ_MAX_SPLITS) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;
   return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L,
                         max_splits_for(max_seq_len, L), seq_lens, out,

@@ -6,28 +6,31 @@
 // accumulation are skipped for every position whose weight exp(s - m_running)
 // is below tau.  Section "FAQ": K itself is always dequantized.
 //
-// One CTA (4 warps) per SM runs a persistent loop over work units
-// (sequence b, KV head, split of <= 1024 positions).  Per unit:
-//   K pass  64-position K tiles (codes + block scales) stream into a ring of
-//           shared-memory stages through TMA (2-D tensor copy with hardware
-//           swizzle for the codes, 1-D bulk copy for the scales), issued up to
-//           STAGES tiles ahead by one thread and running on into the next unit.
-//           Each warp dequantizes 16 positions in registers and multiplies them
-//           with the query group on the tensor cores (mma m16n8k16: positions x
-//           heads x head_dim); block scales / vector norms are applied to the
-//           fp32 score, so integer codes enter the MMA exactly.  Scores (log2
-//           units) go to shared memory; the running maximum is kept per head.
-//   weights Once every K tile of the unit is folded in, m_running is the unit's
-//           maximum.  p = 2^(s - m); l sums every p; (position, head) pairs with
-//           p < tau are dropped; positions kept by any head of the group are
-//           compacted (warp ballot + prefix) into a list, with their p values
-//           (fp16, pre-scaled by 2^14) transposed per head.
-//   V pass  Only listed positions are fetched (cp.async 16-byte gathers of their
-//           V rows and scales, four 64-row batches in flight), dequantized in
-//           registers and accumulated on the tensor cores (dims x heads x
-//           positions).  Skipped positions cost no HBM read, no dequant, no MMA.
-//   output  Unnormalized o, m (log2 units) and l of the unit go to the
-//           workspace; kvq_combine merges the units of a sequence.
+// Persistent CTAs (one per SM) loop over work units (sequence b, KV head,
+// split of <= 1024 positions).  Each CTA has 8 consumer warps and 1 producer
+// warp.
+//   producer  One lane streams 64-position K tiles (codes + block scales) into a
+//             ring of shared-memory stages with TMA: a 2-D tensor copy with
+//             hardware swizzle for the codes and a 1-D bulk copy for the scales,
+//             guarded by full/empty mbarriers, running ahead across work units.
+//   K pass    The unit's positions are cut into 16-position jobs dealt round-robin
+//             to the consumer warps.  A warp dequantizes its 16 rows in registers
+//             and multiplies them with the query group on the tensor cores (mma
+//             m16n8k16: positions x heads x head_dim); block scales / vector norms
+//             are applied to the fp32 score, so integer codes enter the MMA exactly.
+//             Scores (log2 units) go to shared memory; each warp keeps per-head maxima.
+//   weights   After one CTA barrier m_running is the unit's maximum.  Each warp
+//             revisits its own jobs: the skip test is s - m >= log2(tau) (no exp for
+//             it), the denominator l sums 2^(s - m) over every position, and positions
+//             kept by any head of the group are compacted (ballot + popcount) into the
+//             warp's private list, with their weights (fp16, x 2^14) per head.
+//   V pass    Each warp gathers only its kept V rows (cp.async 16-byte copies into a
+//             warp-private ring, 4 groups of 16 rows in flight), dequantizes them in
+//             registers and accumulates p^T V on the tensor cores (head_dim x heads x
+//             positions).  Skipped positions cost no HBM read, no dequant, no MMA.
+//   output    The 8 warps' accumulators are summed in shared memory; unnormalized o,
+//             m (log2 units) and l of the unit go to the workspace and kvq_combine
+//             merges the units of a sequence.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -38,15 +41,18 @@
 namespace kvq {
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kThreads = kConsumers + 32;  // + one producer warp
 constexpr int kLmax = KVQ_MAX_SPLIT_TOKENS;
 constexpr int kMaxTiles = kLmax / kTile;
+constexpr int kWarpSlots = kLmax / kConsumerWarps;  // kept-list slots owned by one warp
 constexpr int kPktStride = kLmax + 8;   // halves per head row of the compacted weights
 constexpr float kPScale = 16384.0f;     // p is stored in fp16 as p * 2^14
 constexpr float kPUnscale = 1.0f / 16384.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
+constexpr int kBarConsumers = 1;          // named barrier id shared by the consumer warps
 
 template <int FMT, int D>
 struct Cfg {
@@ -61,17 +67,18 @@ struct Cfg {
   static constexpr int STAGE_CODE = kTile * CROW;
   static constexpr int STAGE_SC = kTile * SROW;
   static constexpr int STAGE_BYTES = (STAGE_CODE + STAGE_SC + 1023) / 1024 * 1024;
-  static constexpr int STAGES = STAGE_BYTES <= 5120 ? 16 : 12;
+  static constexpr int STAGES = STAGE_BYTES <= 5120 ? 16 : 10;
   // TMA swizzle of the codes: 16-byte chunk index ^= (row >> SWZ_SHIFT) & SWZ_MASK
   static constexpr int SWZ_SHIFT = CROW == 128 ? 0 : CROW == 64 ? 1 : 2;
   static constexpr int SWZ_MASK = CROW / 16 - 1;
-  // V pass
-  static constexpr int VB = 64;               // positions per gather batch
-  static constexpr int NVB = 4;               // batches in flight
-  static constexpr int VSTRIDE = CROW + 16;   // padded row stride of the V staging buffer
-  static constexpr int VDW = D / kWarps;      // dims per warp
-  static constexpr int E = VDW / 8;           // dims per thread
-  static constexpr int MT = VDW / 16;         // m-tiles per warp
+  // V pass (warp-private): thread (r, c) owns dims E*r .. E*r + E - 1
+  static constexpr int E = D / 8;
+  static constexpr int MT = D / 16;                      // m-tiles (16 dims each)
+  static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
+  static constexpr int NWORD = RAWB / 4;
+  static constexpr int VSTRIDE = CROW + 16;              // padded staging row
+  static constexpr int NVS = kQ8 && D == 128 ? 3 : 4;    // groups of 16 rows in flight per warp
+  static constexpr int VGROUP = 16 * VSTRIDE + 16 * 8;   // one staged group: rows + scale records
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
 
@@ -82,18 +89,23 @@ struct Layout {
   static constexpr size_t S = stage + (size_t)C::STAGES * C::STAGE_BYTES;  // float [kLmax][8]
   static constexpr size_t pkt = S + (size_t)kLmax * 8 * 4;                  // half [8][kPktStride]
   static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;          // u16 [kLmax]
-  static constexpr size_t vbuf = list + (size_t)kLmax * 2;                  // [NVB][VB][VSTRIDE]
-  static constexpr size_t vsc = vbuf + (size_t)C::NVB * C::VB * C::VSTRIDE;  // [NVB][VB][8]
-  static constexpr size_t q = vsc + (size_t)C::NVB * C::VB * 8;             // float [8][D]
+  static constexpr size_t vst = list + (size_t)kLmax * 2;                   // [warps][NVS][VGROUP]
+  static constexpr size_t q = vst + (size_t)kConsumerWarps * C::NVS * C::VGROUP;  // float [8][D]
   static constexpr size_t rows = q + (size_t)8 * D * 4;                     // int [kMaxTiles]
   static constexpr size_t stage_row = rows + kMaxTiles * 4;                 // int [STAGES]
-  static constexpr size_t red = stage_row + C::STAGES * 4;                  // float [3][kWarps][8]
-  static constexpr size_t cnt = red + 3 * kWarps * 8 * 4;                   // int [8]
-  static constexpr size_t bars = (cnt + 8 * 4 + 7) / 8 * 8;                 // u64 [STAGES]
-  static constexpr size_t prefix = bars + C::STAGES * 8;                    // int [MAX_BATCH + 1]
+  static constexpr size_t red = stage_row + C::STAGES * 4;                  // float [2][warps][8]
+  static constexpr size_t cnt = red + 2 * kConsumerWarps * 8 * 4;           // int [2][warps]
+  static constexpr size_t bars = (cnt + 2 * kConsumerWarps * 4 + 7) / 8 * 8;  // u64 [2][STAGES]
+  static constexpr size_t prefix = bars + 2 * C::STAGES * 8;                // int [MAX_BATCH + 1]
   static constexpr size_t total = prefix + (KVQ_MAX_BATCH + 1) * 4;
   static constexpr size_t alloc = total + 1024;  // slack for aligning the base to 1024
+  // the 8 warps' V accumulators are reduced through the score buffer
+  static_assert((size_t)kConsumers * (D / 16) * 4 * 4 <= (size_t)kLmax * 8 * 4, "reduction space");
 };
+
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync %0, %1;" ::"n"(kBarConsumers), "n"(kConsumers) : "memory");
+}
 
 struct Item {
   int b, kvh, split, t0, n_tok;
@@ -275,121 +287,121 @@ __device__ __forceinline__ void k_tile_scores(const uint8_t* __restrict__ codes,
   }
 }
 
-// ------------------------------------------------------------------ V batch
-// Accumulate o[dims of this warp][8 heads] += v_hat^T p over one staged batch.
+// ------------------------------------------------------------------ V pass
+// Dequantize the raw bits of two positions (a, b) into half2 (a, b) pairs, one per
+// dim owned by this thread (E of them), in dim order.
 template <int FMT, int D>
-__device__ __forceinline__ void v_dequant_pair(uint32_t ra, uint32_t rb, const Lut& lut,
-                                               uint32_t (&e)[Cfg<FMT, D>::E]) {
+__device__ __forceinline__ void v_dequant_pair(const uint32_t (&ra)[Cfg<FMT, D>::NWORD],
+                                               const uint32_t (&rb)[Cfg<FMT, D>::NWORD],
+                                               const Lut& lut, uint32_t (&e)[Cfg<FMT, D>::E]) {
   using C = Cfg<FMT, D>;
-  if constexpr (C::kQ8) {
-    const __half2 bias = __half2half2(__ushort_as_half(0x6480));  // 1152
-    if constexpr (C::E == 4) {
-      const uint32_t wa = ra ^ 0x80808080u, wb = rb ^ 0x80808080u;
-      const uint32_t t01 = prmt(wa, wb, 0x5140u), t23 = prmt(wa, wb, 0x7362u);
-      e[0] = h2_as_u32(__hsub2(u32_as_h2(prmt(t01, 0x64646464u, 0x4140u)), bias));
-      e[1] = h2_as_u32(__hsub2(u32_as_h2(prmt(t01, 0x64646464u, 0x4342u)), bias));
-      e[2] = h2_as_u32(__hsub2(u32_as_h2(prmt(t23, 0x64646464u, 0x4140u)), bias));
-      e[3] = h2_as_u32(__hsub2(u32_as_h2(prmt(t23, 0x64646464u, 0x4342u)), bias));
+#pragma unroll
+  for (int k = 0; k < C::NWORD; ++k) {
+    const uint32_t wa = ra[k], wb = rb[k];
+    if constexpr (C::kQ8) {
+      // 4 int8 codes per word -> 4 dims
+      const __half2 bias = __half2half2(__ushort_as_half(0x6480));  // 1152
+      const uint32_t xa = wa ^ 0x80808080u, xb = wb ^ 0x80808080u;
+      const uint32_t t01 = prmt(xa, xb, 0x5140u), t23 = prmt(xa, xb, 0x7362u);
+      e[4 * k + 0] = h2_as_u32(__hsub2(u32_as_h2(prmt(t01, 0x64646464u, 0x4140u)), bias));
+      e[4 * k + 1] = h2_as_u32(__hsub2(u32_as_h2(prmt(t01, 0x64646464u, 0x4342u)), bias));
+      e[4 * k + 2] = h2_as_u32(__hsub2(u32_as_h2(prmt(t23, 0x64646464u, 0x4140u)), bias));
+      e[4 * k + 3] = h2_as_u32(__hsub2(u32_as_h2(prmt(t23, 0x64646464u, 0x4342u)), bias));
+    } else if constexpr (C::kQ4) {
+      // 8 nibbles per word -> 8 dims; x_lo holds dims 0-3 of both positions, x_hi dims 4-7
+      const __half2 b1032 = __half2half2(__ushort_as_half(0x6408));
+      const __half2 inv16 = __half2half2(__ushort_as_half(0x2C00));
+      const __half2 m72 = __half2half2(__ushort_as_half(0xD480));
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t x = hlf ? prmt(wa, wb, 0x7632u) : prmt(wa, wb, 0x5410u);
+        const uint32_t y = x >> 8;
+        e[8 * k + 4 * hlf + 0] = h2_as_u32(__hsub2(u32_as_h2((x & 0x000F000Fu) | kMagic), b1032));
+        e[8 * k + 4 * hlf + 1] =
+            h2_as_u32(__hfma2(u32_as_h2((x & 0x00F000F0u) | kMagic), inv16, m72));
+        e[8 * k + 4 * hlf + 2] = h2_as_u32(__hsub2(u32_as_h2((y & 0x000F000Fu) | kMagic), b1032));
+        e[8 * k + 4 * hlf + 3] =
+            h2_as_u32(__hfma2(u32_as_h2((y & 0x00F000F0u) | kMagic), inv16, m72));
+      }
     } else {
-      const uint32_t t = prmt(ra ^ 0x8080u, rb ^ 0x8080u, 0x5140u);
-      e[0] = h2_as_u32(__hsub2(u32_as_h2(prmt(t, 0x64646464u, 0x4140u)), bias));
-      e[1] = h2_as_u32(__hsub2(u32_as_h2(prmt(t, 0x64646464u, 0x4342u)), bias));
-    }
-  } else if constexpr (C::kQ4) {
-    const __half2 b1032 = __half2half2(__ushort_as_half(0x6408));
-    const __half2 inv16 = __half2half2(__ushort_as_half(0x2C00));
-    const __half2 m72 = __half2half2(__ushort_as_half(0xD480));
-    const uint32_t x = (C::E == 4) ? prmt(ra, rb, 0x5410u) : prmt(ra, rb, 0x0400u);
-    e[0] = h2_as_u32(__hsub2(u32_as_h2((x & 0x000F000Fu) | kMagic), b1032));
-    e[1] = h2_as_u32(__hfma2(u32_as_h2((x & 0x00F000F0u) | kMagic), inv16, m72));
-    if constexpr (C::E == 4) {
-      const uint32_t y = x >> 8;
-      e[2] = h2_as_u32(__hsub2(u32_as_h2((y & 0x000F000Fu) | kMagic), b1032));
-      e[3] = h2_as_u32(__hfma2(u32_as_h2((y & 0x00F000F0u) | kMagic), inv16, m72));
-    }
-  } else {
-    if constexpr (C::E == 4) {
-      const uint32_t x = prmt(ra, rb, 0x5410u);  // low half: a's 4 nibbles, high: b's
-      uint32_t La, Ha, Lb, Hb;
-      lut_lookup4(lut, x, nib_mask_lo(x), La, Ha);
-      lut_lookup4(lut, x >> 16, nib_mask_hi(x), Lb, Hb);
-      const uint32_t ta01 = prmt(La, Ha, 0x5140u), tb01 = prmt(Lb, Hb, 0x5140u);
-      const uint32_t ta23 = prmt(La, Ha, 0x7362u), tb23 = prmt(Lb, Hb, 0x7362u);
-      e[0] = prmt(ta01, tb01, 0x5410u);
-      e[1] = prmt(ta01, tb01, 0x7632u);
-      e[2] = prmt(ta23, tb23, 0x5410u);
-      e[3] = prmt(ta23, tb23, 0x7632u);
-    } else {
-      const uint32_t x = prmt(ra, rb, 0x0040u);  // nibbles: a0 a1 b0 b1
-      uint32_t L, H;
-      lut_lookup4(lut, x, nib_mask_lo(x), L, H);
-      e[0] = prmt(L, H, 0x6240u);
-      e[1] = prmt(L, H, 0x7351u);
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const uint32_t x = hlf ? prmt(wa, wb, 0x7632u) : prmt(wa, wb, 0x5410u);
+        uint32_t La, Ha, Lb, Hb;
+        lut_lookup4(lut, x, nib_mask_lo(x), La, Ha);
+        lut_lookup4(lut, x >> 16, nib_mask_hi(x), Lb, Hb);
+        const uint32_t ta01 = prmt(La, Ha, 0x5140u), tb01 = prmt(Lb, Hb, 0x5140u);
+        const uint32_t ta23 = prmt(La, Ha, 0x7362u), tb23 = prmt(Lb, Hb, 0x7362u);
+        e[8 * k + 4 * hlf + 0] = prmt(ta01, tb01, 0x5410u);
+        e[8 * k + 4 * hlf + 1] = prmt(ta01, tb01, 0x7632u);
+        e[8 * k + 4 * hlf + 2] = prmt(ta23, tb23, 0x5410u);
+        e[8 * k + 4 * hlf + 3] = prmt(ta23, tb23, 0x7632u);
+      }
     }
   }
 }
 
 template <int FMT, int D>
-__device__ __forceinline__ uint32_t v_raw(const uint8_t* row, int boff) {
+__device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D>::NWORD]) {
   using C = Cfg<FMT, D>;
-  if constexpr (C::kQ8) {
-    if constexpr (C::E == 4) return lds32(row + boff);
-    else return lds16(row + boff);
+  if constexpr (C::NWORD == 4) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+  } else if constexpr (C::NWORD == 2) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    w[0] = u.x; w[1] = u.y;
   } else {
-    if constexpr (C::E == 4) return lds16(row + boff);
-    else return lds8(row + boff);
+    w[0] = lds32(p);
   }
 }
 
+// Scale (q8_0 / q4_0 block scale of this thread's dims, or lut4 vector norm) of a
+// staged position; 0 for slots past the end so that stale rows contribute nothing.
 template <int FMT, int D>
-__device__ __forceinline__ __half v_scale(const uint8_t* vs, const uint16_t* list, int s_begin,
-                                          int slot, int n_in, int blk) {
+__device__ __forceinline__ __half v_scale(const uint8_t* rec, int slot, int n_valid, int blk,
+                                          const uint16_t* list_grp) {
   using C = Cfg<FMT, D>;
-  if (slot >= n_in) return __ushort_as_half(0);
+  if (slot >= n_valid) return __ushort_as_half(0);
   if constexpr (C::kLut) {
-    const int tok = list[s_begin + slot];
-    return *reinterpret_cast<const __half*>(vs + slot * 8 + 2 * (tok & 1));
+    const int tok = list_grp[slot];
+    return *reinterpret_cast<const __half*>(rec + slot * 8 + 2 * (tok & 1));
   } else {
-    return *reinterpret_cast<const __half*>(vs + slot * 8 + 2 * blk);
+    return *reinterpret_cast<const __half*>(rec + slot * 8 + 2 * blk);
   }
 }
 
+// One group of 16 staged positions: acc[dims x heads] += v_hat^T p.
 template <int FMT, int D>
-__device__ __forceinline__ void v_batch(const uint8_t* __restrict__ vb, const uint8_t* __restrict__ vs,
-                                        const __half* __restrict__ pkt,
-                                        const uint16_t* __restrict__ list, int s_begin, int n_in,
-                                        int warp, int lane, const Lut& lut,
-                                        float (&acc)[Cfg<FMT, D>::MT][4]) {
+__device__ __forceinline__ void v_group(const uint8_t* __restrict__ grp, const __half* __restrict__ prow,
+                                        const uint16_t* __restrict__ list_grp, int n_valid, int r,
+                                        int c, const Lut& lut, float (&acc)[Cfg<FMT, D>::MT][4]) {
   using C = Cfg<FMT, D>;
-  const int r = lane >> 2, c = lane & 3;
-  const int dim0 = warp * C::VDW + C::E * r;
-  const int boff = C::kQ8 ? dim0 : dim0 / 2;
-  const int blk = (warp * C::VDW) / 32;
-  const __half* prow = pkt + r * kPktStride + s_begin;
+  const uint8_t* rec = grp + 16 * C::VSTRIDE;
+  const int blk = (C::E * r) / 32;
+  const int sa = 2 * c, sc = sa + 8;
+  const uint32_t b0 = lds32(prow + sa);
+  const uint32_t b1 = lds32(prow + sc);
+  const __half2 dab = __halves2half2(v_scale<FMT, D>(rec, sa, n_valid, blk, list_grp),
+                                     v_scale<FMT, D>(rec, sa + 1, n_valid, blk, list_grp));
+  const __half2 dcd = __halves2half2(v_scale<FMT, D>(rec, sc, n_valid, blk, list_grp),
+                                     v_scale<FMT, D>(rec, sc + 1, n_valid, blk, list_grp));
+  uint32_t wa[C::NWORD], wb[C::NWORD], wc[C::NWORD], wd[C::NWORD];
+  const int boff = C::RAWB * r;
+  v_raw<FMT, D>(grp + sa * C::VSTRIDE + boff, wa);
+  v_raw<FMT, D>(grp + (sa + 1) * C::VSTRIDE + boff, wb);
+  v_raw<FMT, D>(grp + sc * C::VSTRIDE + boff, wc);
+  v_raw<FMT, D>(grp + (sc + 1) * C::VSTRIDE + boff, wd);
+  uint32_t eab[C::E], ecd[C::E];
+  v_dequant_pair<FMT, D>(wa, wb, lut, eab);
+  v_dequant_pair<FMT, D>(wc, wd, lut, ecd);
 #pragma unroll
-  for (int ks = 0; ks < C::VB / 16; ++ks) {
-    if (ks * 16 >= n_in) break;
-    const int sa = ks * 16 + 2 * c, sc = sa + 8;
-    const uint32_t b0 = lds32(prow + sa);
-    const uint32_t b1 = lds32(prow + sc);
-    const __half2 dab = __halves2half2(v_scale<FMT, D>(vs, list, s_begin, sa, n_in, blk),
-                                       v_scale<FMT, D>(vs, list, s_begin, sa + 1, n_in, blk));
-    const __half2 dcd = __halves2half2(v_scale<FMT, D>(vs, list, s_begin, sc, n_in, blk),
-                                       v_scale<FMT, D>(vs, list, s_begin, sc + 1, n_in, blk));
-    uint32_t eab[C::E], ecd[C::E];
-    v_dequant_pair<FMT, D>(v_raw<FMT, D>(vb + sa * C::VSTRIDE, boff),
-                           v_raw<FMT, D>(vb + (sa + 1) * C::VSTRIDE, boff), lut, eab);
-    v_dequant_pair<FMT, D>(v_raw<FMT, D>(vb + sc * C::VSTRIDE, boff),
-                           v_raw<FMT, D>(vb + (sc + 1) * C::VSTRIDE, boff), lut, ecd);
-#pragma unroll
-    for (int e = 0; e < C::E; ++e) {
-      eab[e] = h2_as_u32(__hmul2(u32_as_h2(eab[e]), dab));
-      ecd[e] = h2_as_u32(__hmul2(u32_as_h2(ecd[e]), dcd));
-    }
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt)
-      mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
+  for (int e = 0; e < C::E; ++e) {
+    eab[e] = h2_as_u32(__hmul2(u32_as_h2(eab[e]), dab));
+    ecd[e] = h2_as_u32(__hmul2(u32_as_h2(ecd[e]), dcd));
   }
+#pragma unroll
+  for (int mt = 0; mt < C::MT; ++mt)
+    mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -404,14 +416,16 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   float* S = reinterpret_cast<float*>(smem + LY::S);
   __half* pkt = reinterpret_cast<__half*>(smem + LY::pkt);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + LY::list);
-  uint8_t* vbuf = smem + LY::vbuf;
-  uint8_t* vsc = smem + LY::vsc;
+  uint8_t* vst = smem + LY::vst;
   float* qs = reinterpret_cast<float*>(smem + LY::q);
   int* item_rows = reinterpret_cast<int*>(smem + LY::rows);
   int* stage_row = reinterpret_cast<int*>(smem + LY::stage_row);
-  float* red = reinterpret_cast<float*>(smem + LY::red);
-  int* cnt = reinterpret_cast<int*>(smem + LY::cnt);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + LY::bars);
+  float* red_m = reinterpret_cast<float*>(smem + LY::red);
+  float* red_l = red_m + kConsumerWarps * 8;
+  int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
+  int* cnt_kept = cnt_skip + kConsumerWarps;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::bars);
+  uint64_t* empty = full + C::STAGES;
   int* prefix = reinterpret_cast<int*>(smem + LY::prefix);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -430,9 +444,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   }
   if (tid == 0) {
     prefix[0] = 0;
-    for (int i = 0; i < C::STAGES; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 4);  // the four warps that consume the tile's four 16-row jobs
+    }
     fence_mbar_init();
-    prefetch_tensormap(&tmap_k);
   }
   __syncthreads();
   if (warp == 0) {
@@ -453,7 +469,46 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   const int total_items = prefix[B] * hkv;
   if ((int)blockIdx.x >= total_items) return;
 
-  // ---- lut4 tables (registers)
+  // ================================================================ producer warp
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmap_k);
+      const uint8_t* ksc = static_cast<const uint8_t*>(a.k_scales);
+      int pg = 0;
+      for (int k = 0;; ++k) {
+        const int it = blockIdx.x + k * gridDim.x;
+        if (it >= total_items) break;
+        const Item I = decode_item(a, prefix, it);
+        const int ntiles = (I.n_tok + kTile - 1) / kTile;
+        for (int t = 0; t < ntiles; ++t, ++pg) {
+          const int stage = pg % C::STAGES, use = pg / C::STAGES;
+          if (use > 0 && !mbar_wait_bounded(&empty[stage], (uint32_t)(use - 1) & 1u)) {
+            set_flag(flags, KVQ_FLAG_TIMEOUT);
+            return;
+          }
+          uint8_t* dst = stages + (size_t)stage * C::STAGE_BYTES;
+          const int tok0 = I.t0 + t * kTile;
+          const int lp = tok0 / P, off = tok0 - lp * P;
+          const int page = a.page_table ? a.page_table[(size_t)I.b * a.max_pages + lp]
+                                        : I.b * a.max_pages + lp;
+          if (page >= 0 && page < a.desc.num_pages) {
+            const int row0 = (page * hkv + I.kvh) * P + off;
+            stage_row[stage] = row0;
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_CODE + C::STAGE_SC);
+            tma_load_2d(dst, &tmap_k, 0, row0, &full[stage]);
+            bulk_load(dst + C::STAGE_CODE, ksc + (size_t)row0 * C::SROW, C::STAGE_SC, &full[stage]);
+          } else {
+            set_flag(flags, KVQ_FLAG_BAD_PAGE);
+            stage_row[stage] = -1;
+            mbar_arrive(&full[stage]);  // completes the phase with no bytes
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ================================================================ consumer warps
   Lut lut;
   if constexpr (C::kLut) {
 #pragma unroll
@@ -472,44 +527,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
     for (int i = 0; i < 4; ++i) lut.lo[i] = lut.hi[i] = 0;
   }
 
-  // ---- producer state (thread 0): next tile to issue
-  int p_k = 0, p_t = 0, p_g = 0;
-  Item p_item;
-  p_item.n_tok = 0;
-  const uint8_t* ksc = static_cast<const uint8_t*>(a.k_scales);
-  auto producer_fill = [&](int limit) {
-    while (p_g < limit) {
-      if (p_t * kTile >= p_item.n_tok) {  // advance to the next work unit
-        const int it = blockIdx.x + p_k * gridDim.x;
-        if (it >= total_items) return;
-        p_item = decode_item(a, prefix, it);
-        ++p_k;
-        p_t = 0;
-      }
-      const int stage = p_g % C::STAGES;
-      uint8_t* dst = stages + (size_t)stage * C::STAGE_BYTES;
-      const int tok0 = p_item.t0 + p_t * kTile;
-      const int lp = tok0 / P, off = tok0 - lp * P;
-      const int page = a.page_table ? a.page_table[(size_t)p_item.b * a.max_pages + lp]
-                                    : p_item.b * a.max_pages + lp;
-      if (page >= 0 && page < a.desc.num_pages) {
-        const int row0 = (page * hkv + p_item.kvh) * P + off;
-        mbar_arrive_expect_tx(&bars[stage], C::STAGE_CODE + C::STAGE_SC);
-        tma_load_2d(dst, &tmap_k, 0, row0, &bars[stage]);
-        bulk_load(dst + C::STAGE_CODE, ksc + (size_t)row0 * C::SROW, C::STAGE_SC, &bars[stage]);
-        stage_row[stage] = row0;
-      } else {
-        set_flag(flags, KVQ_FLAG_BAD_PAGE);
-        stage_row[stage] = -1;
-        mbar_arrive(&bars[stage]);  // completes the phase with no bytes
-      }
-      ++p_t;
-      ++p_g;
-    }
-  };
-  if (tid == 0) producer_fill(C::STAGES);
-
   const float qk_scale = a.sm_scale * kLog2e;
+  const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
   const __half* qg = static_cast<const __half*>(a.q);
   const uint8_t* vcodes = static_cast<const uint8_t*>(a.v_codes);
   const uint8_t* vscales = static_cast<const uint8_t*>(a.v_scales);
@@ -517,56 +536,74 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   const size_t n_part = (size_t)B * Hq * a.max_splits;
   float* ws_m = ws_o + n_part * D;
   float* ws_l = ws_m + n_part;
+  const int wslot0 = warp * kWarpSlots;  // this warp's region of the kept list / weights
+  uint8_t* my_vst = vst + (size_t)warp * C::NVS * C::VGROUP;
 
-  int g = 0;  // K tiles consumed by this CTA
+  int g_base = 0;  // K tiles consumed by this CTA before the current unit
   for (int k = 0;; ++k) {
     const int it = blockIdx.x + k * gridDim.x;
     if (it >= total_items) break;
     const Item I = decode_item(a, prefix, it);
     const int ntiles = (I.n_tok + kTile - 1) / kTile;
+    const int njobs = 4 * ntiles;
 
     // ---- query group -> shared (fp32), rotated for lut4
-    for (int i = tid; i < 8 * D; i += kThreads) {
-      const int h = i / D, d = i - h * D;
-      qs[i] = (h < G) ? __half2float(qg[((size_t)I.b * Hq + I.kvh * G + h) * D + d]) : 0.f;
+    {
+      constexpr int kChunks = 8 * D / 8;  // 16-byte chunks of 8 heads x D fp16
+#pragma unroll
+      for (int j = 0; j < (kChunks + kConsumers - 1) / kConsumers; ++j) {
+        const int ch = tid + j * kConsumers;
+        if (ch < kChunks) {
+          const int h = ch / (D / 8), d0 = (ch - h * (D / 8)) * 8;
+          uint4 raw = make_uint4(0, 0, 0, 0);
+          if (h < G)
+            raw = *reinterpret_cast<const uint4*>(qg + ((size_t)I.b * Hq + I.kvh * G + h) * D + d0);
+          const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hp[e]);
+            qs[h * D + d0 + 2 * e] = f.x;
+            qs[h * D + d0 + 2 * e + 1] = f.y;
+          }
+        }
+      }
     }
-    __syncthreads();
+    consumer_sync();
     if constexpr (C::kLut) {
-      // q' = c * H * (s .* q), butterflies in fp32; warp w rotates heads w and w + 4
+      // q' = c * H * (s .* q), butterflies in fp32; warp w rotates head w
       constexpr int K = D / 32;
-      for (int h = warp; h < 8; h += kWarps) {
-        float y[K];
+      const int h = warp;
+      float y[K];
+#pragma unroll
+      for (int kk = 0; kk < K; ++kk) {
+        const int i = 32 * kk + lane;
+        y[kk] = qs[h * D + i] * (float)a.desc.signs[i];
+      }
+#pragma unroll
+      for (int hb = 1; hb < 32; hb <<= 1) {
+        const bool upper = (lane & hb) != 0;
 #pragma unroll
         for (int kk = 0; kk < K; ++kk) {
-          const int i = 32 * kk + lane;
-          y[kk] = qs[h * D + i] * (float)a.desc.signs[i];
+          const float o = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+          y[kk] = upper ? (o - y[kk]) : (y[kk] + o);
         }
-#pragma unroll
-        for (int hb = 1; hb < 32; hb <<= 1) {
-          const bool upper = (lane & hb) != 0;
-#pragma unroll
-          for (int kk = 0; kk < K; ++kk) {
-            const float o = __shfl_xor_sync(0xffffffffu, y[kk], hb);
-            y[kk] = upper ? (o - y[kk]) : (y[kk] + o);
-          }
-        }
-#pragma unroll
-        for (int kk = 0; kk + 1 < K; kk += 2) {
-          const float u = y[kk], v = y[kk + 1];
-          y[kk] = u + v; y[kk + 1] = u - v;
-        }
-        if (K == 4) {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const float u = y[kk], v = y[kk + 2];
-            y[kk] = u + v; y[kk + 2] = u - v;
-          }
-        }
-        const float cs = rsqrtf((float)D);
-#pragma unroll
-        for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
       }
-      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk + 1 < K; kk += 2) {
+        const float u = y[kk], v = y[kk + 1];
+        y[kk] = u + v; y[kk + 1] = u - v;
+      }
+      if (K == 4) {
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const float u = y[kk], v = y[kk + 2];
+          y[kk] = u + v; y[kk + 2] = u - v;
+        }
+      }
+      const float cs = rsqrtf((float)D);
+#pragma unroll
+      for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
+      consumer_sync();
     }
     uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
 #pragma unroll
@@ -586,219 +623,226 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       }
     }
 
-    // ---- K pass
+    // ---- K pass: this warp's 16-row jobs
     float mx0 = -INFINITY, mx1 = -INFINITY;
-    for (int t = 0; t < ntiles; ++t) {
+    bool timed_out = false;
+    for (int j = warp; j < njobs; j += kConsumerWarps) {
+      const int t = j >> 2, mt = j & 3;
+      const int g = g_base + t;
       const int stage = g % C::STAGES;
-      const bool ok = mbar_wait_bounded(&bars[stage], (uint32_t)(g / C::STAGES) & 1u);
-      if (ok) {
-        const uint8_t* base = stages + (size_t)stage * C::STAGE_BYTES;
-        const int row0 = 16 * warp + r;
-        float s[4];
-        k_tile_scores<FMT, D>(base, base + C::STAGE_CODE, row0, qf, ql, lut, c, s);
-        const int p0 = t * kTile + row0, p1 = p0 + 8;
-        const bool v0 = p0 < I.n_tok, v1 = p1 < I.n_tok;
-        const float s0 = v0 ? s[0] * qk_scale : -INFINITY, s1 = v0 ? s[1] * qk_scale : -INFINITY;
-        const float s2 = v1 ? s[2] * qk_scale : -INFINITY, s3 = v1 ? s[3] * qk_scale : -INFINITY;
-        *reinterpret_cast<float2*>(S + p0 * 8 + 2 * c) = make_float2(s0, s1);
-        *reinterpret_cast<float2*>(S + p1 * 8 + 2 * c) = make_float2(s2, s3);
-        mx0 = fmaxf(mx0, fmaxf(s0, s2));
-        mx1 = fmaxf(mx1, fmaxf(s1, s3));
+      if (!mbar_wait_bounded(&full[stage], (uint32_t)(g / C::STAGES) & 1u)) {
+        timed_out = true;
+        break;
       }
-      if (tid == 0) item_rows[t] = stage_row[stage];
-      if (__syncthreads_or(!ok)) {
-        if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-        return;
-      }
-      if (tid == 0) producer_fill(g + 1 + C::STAGES);
-      ++g;
+      const uint8_t* base = stages + (size_t)stage * C::STAGE_BYTES;
+      const int row0 = 16 * mt + r;
+      float s[4];
+      k_tile_scores<FMT, D>(base, base + C::STAGE_CODE, row0, qf, ql, lut, c, s);
+      if (mt == 0 && lane == 0) item_rows[t] = stage_row[stage];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      const int p0 = t * kTile + row0, p1 = p0 + 8;
+      const bool v0 = p0 < I.n_tok, v1 = p1 < I.n_tok;
+      const float s0 = v0 ? s[0] * qk_scale : -INFINITY, s1 = v0 ? s[1] * qk_scale : -INFINITY;
+      const float s2 = v1 ? s[2] * qk_scale : -INFINITY, s3 = v1 ? s[3] * qk_scale : -INFINITY;
+      *reinterpret_cast<float2*>(S + p0 * 8 + 2 * c) = make_float2(s0, s1);
+      *reinterpret_cast<float2*>(S + p1 * 8 + 2 * c) = make_float2(s2, s3);
+      mx0 = fmaxf(mx0, fmaxf(s0, s2));
+      mx1 = fmaxf(mx1, fmaxf(s1, s3));
     }
-
-    // ---- running maximum of the unit, per head
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
     if (r == 0) {
-      red[warp * 8 + 2 * c] = mx0;
-      red[warp * 8 + 2 * c + 1] = mx1;
+      red_m[warp * 8 + 2 * c] = mx0;
+      red_m[warp * 8 + 2 * c + 1] = mx1;
     }
-    __syncthreads();
-    float mh[8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      float v = red[h];
-#pragma unroll
-      for (int w = 1; w < kWarps; ++w) v = fmaxf(v, red[w * 8 + h]);
-      mh[h] = v;
-    }
-
-    // ---- weights, skip decision, compaction of kept positions
-    float lsum[8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) lsum[h] = 0.f;
-    int nskip = 0, kept_base = 0;
-    for (int base = 0; base < I.n_tok; base += kThreads) {
-      const int tok = base + tid;
-      bool any = false;
-      float pk[8];
-      if (tok < I.n_tok) {
-        const float4 sa = *reinterpret_cast<const float4*>(S + tok * 8);
-        const float4 sb = *reinterpret_cast<const float4*>(S + tok * 8 + 4);
-        const float sv[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          pk[h] = 0.f;
-          if (h < G) {
-            const float p = ex2(sv[h] - mh[h]);
-            lsum[h] += p;
-            const bool keep = p >= a.tau;
-            any |= keep;
-            nskip += keep ? 0 : 1;
-            pk[h] = keep ? p : 0.f;
-          }
-        }
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, any);
-      if (lane == 0) cnt[warp] = __popc(bal);
-      __syncthreads();
-      int wbase = kept_base;
-      for (int w = 0; w < warp; ++w) wbase += cnt[w];
-      int total = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) total += cnt[w];
-      if (any) {
-        const int slot = wbase + __popc(bal & ((1u << lane) - 1u));
-        list[slot] = (uint16_t)tok;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) pkt[h * kPktStride + slot] = __float2half_rn(pk[h] * kPScale);
-      }
-      kept_base += total;
-      __syncthreads();
-    }
-    const int n_kept = kept_base;
-    // zero the compacted weights up to the next multiple of 16 (partial MMA k-steps)
+    // barrier 1: every score of the unit and every warp's maximum are in shared memory
     {
-      const int pad_end = (n_kept + 15) & ~15;
-      for (int i = tid; i < 8 * 16; i += kThreads) {
-        const int h = i >> 4, sl = n_kept + (i & 15);
-        if (sl < pad_end) pkt[h * kPktStride + sl] = __ushort_as_half(0);
+      int bad = timed_out ? 1 : 0;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+          "bar.red.or.pred p, %2, %3, p;\n\tselp.s32 %0, 1, 0, p;\n\t}"
+          : "=r"(bad)
+          : "r"(bad), "n"(kBarConsumers), "n"(kConsumers)
+          : "memory");
+      if (bad) {
+        if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+        return;
       }
     }
-    // denominators
+    g_base += ntiles;
+
+    // ---- weights, skip test, compaction (own jobs); lane -> (row lane/2, heads 4*(lane&1)..+3)
+    const int hq0 = 4 * (lane & 1);
+    float mh[4];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      float v = lsum[h];
+    for (int i = 0; i < 4; ++i) {
+      float v = red_m[hq0 + i];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      lsum[h] = v;
+      for (int w = 1; w < kConsumerWarps; ++w) v = fmaxf(v, red_m[w * 8 + hq0 + i]);
+      mh[i] = v;
+    }
+    float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+    int nkept = 0, nskip = 0;
+    const unsigned lt_mask = (1u << (lane & ~1)) - 1u;
+    for (int j = warp; j < njobs; j += kConsumerWarps) {
+      const int pos = 16 * j + (lane >> 1);
+      const bool valid = pos < I.n_tok;
+      float sv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (valid) {
+        const float4 f = *reinterpret_cast<const float4*>(S + pos * 8 + hq0);
+        sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
+      }
+      bool keep[4];
+      bool any = false;
+      float p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool live = valid && (hq0 + i < G);
+        const float dlt = sv[i] - mh[i];
+        p[i] = live ? ex2(dlt) : 0.f;
+        lsum[i] += p[i];
+        keep[i] = live && dlt >= thr;
+        any |= keep[i];
+        nskip += (live && !keep[i]) ? 1 : 0;
+      }
+      any = any || (__shfl_xor_sync(0xffffffffu, any ? 1 : 0, 1) != 0);
+      const unsigned bal = __ballot_sync(0xffffffffu, any) & 0x55555555u;
+      if (any) {
+        const int slot = wslot0 + nkept + __popc(bal & lt_mask);
+        if ((lane & 1) == 0) list[slot] = (uint16_t)pos;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          pkt[(hq0 + i) * kPktStride + slot] = __float2half_rn(keep[i] ? p[i] * kPScale : 0.f);
+      }
+      nkept += __popc(bal);
+    }
+    // zero the weights of the padding slots of the last partial group of 16
+    {
+      const int pad = ((nkept + 15) & ~15) - nkept;
+      for (int i = lane; i < 8 * pad; i += 32)
+        pkt[(i / pad) * kPktStride + wslot0 + nkept + (i % pad)] = __ushort_as_half(0);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int o = 2; o < 32; o <<= 1) lsum[i] += __shfl_xor_sync(0xffffffffu, lsum[i], o);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
-    if (lane == 0) {
+    if (lane < 2) {
 #pragma unroll
-      for (int h = 0; h < 8; ++h) red[64 + warp * 8 + h] = lsum[h];
-      cnt[4 + warp] = nskip;
+      for (int i = 0; i < 4; ++i) red_l[warp * 8 + hq0 + i] = lsum[i];
     }
-    __syncthreads();
+    if (lane == 0) {
+      cnt_skip[warp] = nskip;
+      cnt_kept[warp] = nkept;
+    }
+    __syncwarp();
 
-    // ---- V pass over the kept positions only
+    // ---- V pass over this warp's kept positions only
     float acc[C::MT][4];
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    const int nb = (n_kept + C::VB - 1) / C::VB;
-    auto issue_v = [&](int bi) {
-      const int buf = bi % C::NVB;
-      const int s_begin = bi * C::VB;
-      uint8_t* vb = vbuf + (size_t)buf * C::VB * C::VSTRIDE;
-      uint8_t* vs = vsc + (size_t)buf * C::VB * 8;
+    const int ngroups = (nkept + 15) >> 4;
+    auto issue = [&](int gi) {
+      uint8_t* grp = my_vst + (size_t)(gi % C::NVS) * C::VGROUP;
       constexpr int CPR = C::CROW / 16;
-      for (int ch = tid; ch < C::VB * CPR; ch += kThreads) {
-        const int sl = ch / CPR, cc = ch - sl * CPR;
-        const int slot = s_begin + sl;
-        if (slot < n_kept) {
-          const int tok = list[slot];
+      for (int ch = lane; ch < 16 * CPR; ch += 32) {
+        const int rl = ch / CPR, cc = ch - rl * CPR;
+        const int slot = 16 * gi + rl;
+        if (slot < nkept) {
+          const int tok = list[wslot0 + slot];
           const int rb = item_rows[tok >> 6];
           if (rb >= 0) {
             const size_t row = (size_t)rb + (tok & 63);
-            cp_async16(vb + sl * C::VSTRIDE + cc * 16, vcodes + row * C::CROW + cc * 16);
+            cp_async16(grp + rl * C::VSTRIDE + cc * 16, vcodes + row * C::CROW + cc * 16);
           }
         }
       }
-      if (tid < C::VB) {
-        const int slot = s_begin + tid;
-        if (slot < n_kept) {
-          const int tok = list[slot];
+      if (lane < 16) {
+        const int slot = 16 * gi + lane;
+        if (slot < nkept) {
+          const int tok = list[wslot0 + slot];
           const int rb = item_rows[tok >> 6];
           if (rb >= 0) {
             const size_t row = (size_t)rb + (tok & 63);
-            if constexpr (C::kLut) cp_async4(vs + tid * 8, vscales + (row & ~(size_t)1) * 2);
-            else if constexpr (C::SROW == 8) cp_async8(vs + tid * 8, vscales + row * 8);
-            else cp_async4(vs + tid * 8, vscales + row * 4);
+            uint8_t* rec = grp + 16 * C::VSTRIDE + lane * 8;
+            if constexpr (C::kLut) cp_async4(rec, vscales + (row & ~(size_t)1) * 2);
+            else if constexpr (C::SROW == 8) cp_async8(rec, vscales + row * 8);
+            else cp_async4(rec, vscales + row * 4);
           }
         }
       }
+      cp_async_commit();
     };
 #pragma unroll
-    for (int i = 0; i < C::NVB; ++i) {
-      if (i < nb) issue_v(i);
-      cp_async_commit();
+    for (int i = 0; i < C::NVS; ++i) {
+      if (i < ngroups) issue(i);
+      else cp_async_commit();
     }
-    for (int bi = 0; bi < nb; ++bi) {
-      cp_async_wait<C::NVB - 1>();
-      __syncthreads();
-      const int buf = bi % C::NVB;
-      const int s_begin = bi * C::VB;
-      v_batch<FMT, D>(vbuf + (size_t)buf * C::VB * C::VSTRIDE, vsc + (size_t)buf * C::VB * 8, pkt,
-                      list, s_begin, min(C::VB, n_kept - s_begin), warp, lane, lut, acc);
-      __syncthreads();
-      if (bi + C::NVB < nb) issue_v(bi + C::NVB);
-      cp_async_commit();
+    for (int gi = 0; gi < ngroups; ++gi) {
+      cp_async_wait<C::NVS - 1>();
+      __syncwarp();
+      v_group<FMT, D>(my_vst + (size_t)(gi % C::NVS) * C::VGROUP,
+                      pkt + r * kPktStride + wslot0 + 16 * gi, list + wslot0 + 16 * gi,
+                      min(16, nkept - 16 * gi), r, c, lut, acc);
+      __syncwarp();
+      if (gi + C::NVS < ngroups) issue(gi + C::NVS);
+      else cp_async_commit();
     }
     cp_async_wait<0>();
 
-    // ---- unit epilogue: o (unnormalized), m (log2 units), l
+    // ---- sum the warps' accumulators (through the score buffer) and write the unit
+    consumer_sync();  // barrier 2: no warp still reads scores
+    float* ored = S;  // [warp][accumulator register][lane]
+    constexpr int NE = C::MT * 4;  // accumulator registers per thread
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ored[(warp * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
+    consumer_sync();  // barrier 3
     {
       const size_t unit0 = ((size_t)I.b * Hq + (size_t)I.kvh * G) * a.max_splits + I.split;
-      const int dim0 = warp * C::VDW + C::E * r;
+      for (int q = tid; q < 32 * NE; q += kConsumers) {
+        const int ln = q & 31, e = q >> 5;
+        float v = 0.f;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int h = 2 * c + hh;
-        if (h < G) {
-          float* dst = ws_o + (unit0 + (size_t)h * a.max_splits) * D + dim0;
-          if constexpr (C::E == 4) {
-            *reinterpret_cast<float4*>(dst) =
-                make_float4(acc[0][hh] * kPUnscale, acc[0][2 + hh] * kPUnscale,
-                            acc[1][hh] * kPUnscale, acc[1][2 + hh] * kPUnscale);
-          } else {
-            *reinterpret_cast<float2*>(dst) =
-                make_float2(acc[0][hh] * kPUnscale, acc[0][2 + hh] * kPUnscale);
-          }
-        }
+        for (int w = 0; w < kConsumerWarps; ++w) v += ored[(w * NE + e) * 32 + ln];
+        const int mt = e >> 2, i = e & 3;
+        const int rr = ln >> 2, cc = ln & 3;
+        const int h = 2 * cc + (i & 1);
+        const int dim = C::E * rr + 2 * mt + (i >> 1);
+        if (h < G) ws_o[(unit0 + (size_t)h * a.max_splits) * D + dim] = v * kPUnscale;
       }
       if (tid < G) {
-        float l = 0.f;
+        float m = red_m[tid], l = red_l[tid];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) l += red[64 + w * 8 + tid];
-        float mt = red[tid];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) mt = fmaxf(mt, red[w * 8 + tid]);
+        for (int w = 1; w < kConsumerWarps; ++w) {
+          m = fmaxf(m, red_m[w * 8 + tid]);
+          l += red_l[w * 8 + tid];
+        }
         const size_t u = unit0 + (size_t)tid * a.max_splits;
-        ws_m[u] = mt;
+        ws_m[u] = m;
         ws_l[u] = l;
       }
       if (tid == 0 && a.stats) {
-        int ns = 0;
+        int ns = 0, nk = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) ns += cnt[4 + w];
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          ns += cnt_skip[w];
+          nk += cnt_kept[w];
+        }
         atomicAdd(&a.stats[0], (unsigned long long)I.n_tok * G);
         atomicAdd(&a.stats[1], (unsigned long long)ns);
-        atomicAdd(&a.stats[2], (unsigned long long)n_kept);
-        atomicAdd(&a.stats[3], (unsigned long long)(I.n_tok - n_kept));
+        atomicAdd(&a.stats[2], (unsigned long long)nk);
+        atomicAdd(&a.stats[3], (unsigned long long)(I.n_tok - nk));
       }
     }
-    __syncthreads();
+    consumer_sync();  // barrier 4: shared buffers free for the next unit
   }
 }
 
@@ -837,9 +881,21 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return KVQ_ERR_CUDA;
   auto kern = decode_kernel<FMT, D>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::alloc) !=
-      cudaSuccess)
-    return KVQ_ERR_CUDA;
+  // The shared-memory opt-in is set once per device (so that later calls, including
+  // ones made while a stream is being captured into a graph, issue no attribute call).
+  static std::mutex mu;
+  static uint64_t done_mask = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return KVQ_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!(done_mask >> dev & 1)) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)LY::alloc) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+      done_mask |= 1ull << dev;
+    }
+  }
   // upper bound on work units: every sequence as long as max_seq_len
   const int64_t units = (int64_t)a.batch * a.desc.num_kv_heads * a.max_splits;
   const int grid = (int)std::min<int64_t>(units, a.num_sms);

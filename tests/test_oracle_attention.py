@@ -184,3 +184,19 @@ def test_planted_scores_concentrate_attention():
     w = np.exp(s - s.max(1, keepdims=True))
     w /= w.sum(1, keepdims=True)
     assert (w < 1e-6).mean() > 0.9
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+def test_decode_step_empty_and_single_position(fmt):
+    wl = W.shrink(W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt), [0, 1, 65], n_planted=1)
+    inp = W.generate(wl)
+    cb = CB.lloyd_max_f16(16, 1 / math.sqrt(128)) if fmt == "lut4" else None
+    res = A.decode_step(fmt, inp.q, inp.k, inp.v, inp.seq_lens, wl.num_kv_heads,
+                        1 / math.sqrt(128), 1e-6, 64, signs=inp.signs, codebook16=cb)
+    assert np.all(res["out_sparse"][0] == 0) and np.all(res["out_dense"][0] == 0)
+    # one position: the output is that position's dequantized V
+    kc, ks = Q.quantize(fmt, inp.v[0:1, 0], inp.signs, cb)
+    v1 = Q.dequantize(fmt, kc, ks, cb)
+    if fmt == "lut4":
+        v1 = Q.unrotate_f64(v1, inp.signs)
+    np.testing.assert_allclose(res["out_sparse"][1, 0], v1[0], rtol=1e-12, atol=1e-12)

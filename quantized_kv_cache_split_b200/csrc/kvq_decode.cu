@@ -95,13 +95,19 @@ struct Layout {
   static constexpr size_t stage_row = rows + kMaxTiles * 4;                 // int [STAGES]
   static constexpr size_t red = stage_row + C::STAGES * 4;                  // float [2][warps][8]
   static constexpr size_t cnt = red + 2 * kConsumerWarps * 8 * 4;           // int [2][warps]
-  static constexpr size_t bars = (cnt + 2 * kConsumerWarps * 4 + 7) / 8 * 8;  // u64 [2][STAGES]
+  static constexpr size_t bars = (cnt + (2 * kConsumerWarps + 2) * 4 + 7) / 8 * 8;  // u64 [2][STAGES]
   static constexpr size_t prefix = bars + 2 * C::STAGES * 8;                // int [MAX_BATCH + 1]
   static constexpr size_t total = prefix + (KVQ_MAX_BATCH + 1) * 4;
   static constexpr size_t alloc = total + 1024;  // slack for aligning the base to 1024
   // the 8 warps' V accumulators are reduced through the score buffer
   static_assert((size_t)kConsumers * (D / 16) * 4 * 4 <= (size_t)kLmax * 8 * 4, "reduction space");
 };
+
+// Final CTA-wide barrier, reached by the producer warp and by the consumer warps from
+// different code paths: the non-aligned form permits that.
+__device__ __forceinline__ void cta_final_sync() {
+  asm volatile("barrier.sync 0;" ::: "memory");
+}
 
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync %0, %1;" ::"n"(kBarConsumers), "n"(kConsumers) : "memory");
@@ -444,6 +450,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   }
   if (tid == 0) {
     prefix[0] = 0;
+    cnt_skip[2 * kConsumerWarps] = 0;  // consumer timeout flag
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);  // the four warps that consume the tile's four 16-row jobs
@@ -475,7 +482,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       prefetch_tensormap(&tmap_k);
       const uint8_t* ksc = static_cast<const uint8_t*>(a.k_scales);
       int pg = 0;
-      for (int k = 0;; ++k) {
+      for (int k = 0; k < (1 << 30); ++k) {
         const int it = blockIdx.x + k * gridDim.x;
         if (it >= total_items) break;
         const Item I = decode_item(a, prefix, it);
@@ -484,7 +491,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
           const int stage = pg % C::STAGES, use = pg / C::STAGES;
           if (use > 0 && !mbar_wait_bounded(&empty[stage], (uint32_t)(use - 1) & 1u)) {
             set_flag(flags, KVQ_FLAG_TIMEOUT);
-            return;
+            k = 1 << 30;  // stop producing; consumers time out on the missing tiles
+            break;
           }
           uint8_t* dst = stages + (size_t)stage * C::STAGE_BYTES;
           const int tok0 = I.t0 + t * kTile;
@@ -505,6 +513,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         }
       }
     }
+    // stay resident until every consumer is done: nothing issued here is left unwaited
+    __syncwarp();
+    cta_final_sync();
     return;
   }
 
@@ -660,18 +671,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       red_m[warp * 8 + 2 * c + 1] = mx1;
     }
     // barrier 1: every score of the unit and every warp's maximum are in shared memory
-    {
-      int bad = timed_out ? 1 : 0;
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tsetp.ne.s32 p, %1, 0;\n\t"
-          "bar.red.or.pred p, %2, %3, p;\n\tselp.s32 %0, 1, 0, p;\n\t}"
-          : "=r"(bad)
-          : "r"(bad), "n"(kBarConsumers), "n"(kConsumers)
-          : "memory");
-      if (bad) {
-        if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-        return;
-      }
+    if (timed_out && lane == 0) atomicOr(cnt_skip + 2 * kConsumerWarps, 1);
+    consumer_sync();
+    if (cnt_skip[2 * kConsumerWarps] != 0) {
+      if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+      break;  // leave the unit loop; all consumer warps see the same flag
     }
     g_base += ntiles;
 
@@ -709,7 +713,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         any |= keep[i];
         nskip += (live && !keep[i]) ? 1 : 0;
       }
-      any = any || (__shfl_xor_sync(0xffffffffu, any ? 1 : 0, 1) != 0);
+      // (the shuffle must run on every lane: never inside a short-circuit)
+      const int partner_any = __shfl_xor_sync(0xffffffffu, any ? 1 : 0, 1);
+      any = any || (partner_any != 0);
       const unsigned bal = __ballot_sync(0xffffffffu, any) & 0x55555555u;
       if (any) {
         const int slot = wslot0 + nkept + __popc(bal & lt_mask);
@@ -844,6 +850,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
     }
     consumer_sync();  // barrier 4: shared buffers free for the next unit
   }
+  cta_final_sync();  // with the producer warp
 }
 
 // ------------------------------------------------------------------ host side

@@ -7,28 +7,28 @@
 // is below tau.  Section "FAQ": K itself is always dequantized.
 //
 // Persistent CTAs (one per SM) loop over work units (sequence b, KV head,
-// split of <= 1024 positions).  Each CTA has 8 consumer warps and 1 producer
-// warp.
+// split of <= 1024 positions).  Each CTA has 16 consumer warps and 1 producer warp.
 //   producer  One lane streams 64-position K tiles (codes + block scales) into a
-//             ring of shared-memory stages with TMA: a 2-D tensor copy with
-//             hardware swizzle for the codes and a 1-D bulk copy for the scales,
-//             guarded by full/empty mbarriers, running ahead across work units.
-//   K pass    The unit's positions are cut into 16-position jobs dealt round-robin
-//             to the consumer warps.  A warp dequantizes its 16 rows in registers
-//             and multiplies them with the query group on the tensor cores (mma
-//             m16n8k16: positions x heads x head_dim); block scales / vector norms
-//             are applied to the fp32 score, so integer codes enter the MMA exactly.
-//             Scores (log2 units) go to shared memory; each warp keeps per-head maxima.
-//   weights   After one CTA barrier m_running is the unit's maximum.  Each warp
-//             revisits its own jobs: the skip test is s - m >= log2(tau) (no exp for
-//             it), the denominator l sums 2^(s - m) over every position, and positions
-//             kept by any head of the group are compacted (ballot + popcount) into the
-//             warp's private list, with their weights (fp16, x 2^14) per head.
-//   V pass    Each warp gathers only its kept V rows (cp.async 16-byte copies into a
-//             warp-private ring, 4 groups of 16 rows in flight), dequantizes them in
+//             ring of shared-memory stages with TMA: a 2-D tensor copy with hardware
+//             swizzle for the codes and a 1-D bulk copy for the scales, guarded by
+//             full/empty mbarriers, running ahead across work units.
+//   K pass    The unit's positions are cut into 16-position jobs dealt round-robin to
+//             the consumer warps.  Codes go into the tensor cores (mma m16n8k16:
+//             positions x heads x head_dim) as magic-number fp16 values (code + a
+//             fixed offset); the offset's contribution, a per-(head, block) constant of
+//             the query, is preloaded into the accumulator, and the block scale /
+//             vector norm is applied to the fp32 score.  Scores stay in registers.
+//   weights   After one CTA barrier m_running is the unit's maximum.  Each warp tests
+//             its scores: keep iff s - m >= log2(tau) (no exp for the test); the
+//             denominator l sums 2^(s - m) over every position; positions kept by any
+//             head of the group are compacted (ballot + popcount) into the warp's
+//             private list, with their weights (fp16, x 2^14) per head.
+//   V pass    Each warp fetches only its kept V rows (one bulk copy of the codes and
+//             one of an aligned scale window per row, completing on a per-warp
+//             mbarrier, several groups of 16 rows in flight), dequantizes them in
 //             registers and accumulates p^T V on the tensor cores (head_dim x heads x
 //             positions).  Skipped positions cost no HBM read, no dequant, no MMA.
-//   output    The 8 warps' accumulators are summed in shared memory; unnormalized o,
+//   output    The warps' accumulators are summed in shared memory; unnormalized o,
 //             m (log2 units) and l of the unit go to the workspace and kvq_combine
 //             merges the units of a sequence.
 #include <cudaTypedefs.h>
@@ -41,18 +41,21 @@
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kThreads = kConsumers + 32;  // + one producer warp
 constexpr int kLmax = KVQ_MAX_SPLIT_TOKENS;
 constexpr int kMaxTiles = kLmax / kTile;
-constexpr int kWarpSlots = kLmax / kConsumerWarps;  // kept-list slots owned by one warp
+constexpr int kJobsPerWarp = kLmax / 16 / kConsumerWarps;  // 16-row jobs per warp per unit (max)
+constexpr int kWarpSlots = 16 * kJobsPerWarp;             // kept-list slots owned by one warp
 constexpr int kPktStride = kLmax + 8;   // halves per head row of the compacted weights
 constexpr float kPScale = 16384.0f;     // p is stored in fp16 as p * 2^14
 constexpr float kPUnscale = 1.0f / 16384.0f;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 in both halves
-constexpr int kBarConsumers = 1;          // named barrier id shared by the consumer warps
+constexpr uint32_t kMagic = 0x64006400u;    // fp16 1024 in both halves (unit mantissa step 1)
+constexpr uint32_t kMagic64 = 0x54005400u;  // fp16 64: mantissa bits 4..7 then count in units of 1
+constexpr int kBarConsumers = 1;            // named barrier shared by the consumer warps
+static_assert(kJobsPerWarp * kConsumerWarps * 16 == kLmax, "job split");
 
 template <int FMT, int D>
 struct Cfg {
@@ -62,12 +65,13 @@ struct Cfg {
   static constexpr int CROW = kQ8 ? D : D / 2;          // code bytes per row
   static constexpr int NSC = kLut ? 1 : D / 32;          // fp16 per scale row
   static constexpr int SROW = 2 * NSC;                   // scale bytes per row
+  static constexpr int RPW = 16 / SROW;                  // rows per 16-byte scale window
   static constexpr int NBLK = D / 32;
   static constexpr int KSTEPS = D / 16;
   static constexpr int STAGE_CODE = kTile * CROW;
   static constexpr int STAGE_SC = kTile * SROW;
   static constexpr int STAGE_BYTES = (STAGE_CODE + STAGE_SC + 1023) / 1024 * 1024;
-  static constexpr int STAGES = STAGE_BYTES <= 5120 ? 16 : 10;
+  static constexpr int STAGES = STAGE_BYTES <= 5120 ? 16 : 8;
   // TMA swizzle of the codes: 16-byte chunk index ^= (row >> SWZ_SHIFT) & SWZ_MASK
   static constexpr int SWZ_SHIFT = CROW == 128 ? 0 : CROW == 64 ? 1 : 2;
   static constexpr int SWZ_MASK = CROW / 16 - 1;
@@ -76,9 +80,9 @@ struct Cfg {
   static constexpr int MT = D / 16;                      // m-tiles (16 dims each)
   static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
   static constexpr int NWORD = RAWB / 4;
-  static constexpr int VSTRIDE = CROW + 16;              // padded staging row
-  static constexpr int NVS = kQ8 && D == 128 ? 3 : 4;    // groups of 16 rows in flight per warp
-  static constexpr int VGROUP = 16 * VSTRIDE + 16 * 8;   // one staged group: rows + scale records
+  static constexpr int VSTRIDE = CROW + 16;              // staged row: codes + scale window
+  static constexpr int NVS = CROW == 128 ? 2 : 3;        // groups of 16 rows in flight per warp
+  static constexpr int VGROUP = 16 * VSTRIDE;
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
 
@@ -86,21 +90,22 @@ template <int FMT, int D>
 struct Layout {
   using C = Cfg<FMT, D>;
   static constexpr size_t stage = 0;
-  static constexpr size_t S = stage + (size_t)C::STAGES * C::STAGE_BYTES;  // float [kLmax][8]
-  static constexpr size_t pkt = S + (size_t)kLmax * 8 * 4;                  // half [8][kPktStride]
-  static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;          // u16 [kLmax]
-  static constexpr size_t vst = list + (size_t)kLmax * 2;                   // [warps][NVS][VGROUP]
+  static constexpr size_t ored = stage + (size_t)C::STAGES * C::STAGE_BYTES;  // float [8][NE][32]
+  static constexpr size_t pkt = ored + (size_t)8 * (D / 16) * 4 * 32 * 4;     // half [8][kPktStride]
+  static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;            // u16 [kLmax]
+  static constexpr size_t vst = list + (size_t)kLmax * 2;                     // [warps][NVS][VGROUP]
   static constexpr size_t q = vst + (size_t)kConsumerWarps * C::NVS * C::VGROUP;  // float [8][D]
-  static constexpr size_t rows = q + (size_t)8 * D * 4;                     // int [kMaxTiles]
-  static constexpr size_t stage_row = rows + kMaxTiles * 4;                 // int [STAGES]
-  static constexpr size_t red = stage_row + C::STAGES * 4;                  // float [2][warps][8]
-  static constexpr size_t cnt = red + 2 * kConsumerWarps * 8 * 4;           // int [2][warps]
-  static constexpr size_t bars = (cnt + (2 * kConsumerWarps + 2) * 4 + 7) / 8 * 8;  // u64 [2][STAGES]
-  static constexpr size_t prefix = bars + 2 * C::STAGES * 8;                // int [MAX_BATCH + 1]
+  static constexpr size_t corr = q + (size_t)8 * D * 4;                       // float [8][NBLK]
+  static constexpr size_t rows = corr + (size_t)8 * C::NBLK * 4;              // int [kMaxTiles]
+  static constexpr size_t stage_row = rows + kMaxTiles * 4;                   // int [STAGES]
+  static constexpr size_t red = stage_row + C::STAGES * 4;                    // float [2][warps][8]
+  static constexpr size_t cnt = red + 2 * kConsumerWarps * 8 * 4;             // int [2][warps] + flags
+  static constexpr size_t bars = (cnt + (2 * kConsumerWarps + 2) * 4 + 7) / 8 * 8;
+  static constexpr size_t nbars = 2 * C::STAGES + kConsumerWarps * C::NVS;    // full, empty, V groups
+  static constexpr size_t prefix = bars + nbars * 8;                          // int [MAX_BATCH + 1]
   static constexpr size_t total = prefix + (KVQ_MAX_BATCH + 1) * 4;
   static constexpr size_t alloc = total + 1024;  // slack for aligning the base to 1024
-  // the 8 warps' V accumulators are reduced through the score buffer
-  static_assert((size_t)kConsumers * (D / 16) * 4 * 4 <= (size_t)kLmax * 8 * 4, "reduction space");
+  static_assert(alloc <= 232448, "shared memory");
 };
 
 // Final CTA-wide barrier, reached by the producer warp and by the consumer warps from
@@ -183,14 +188,18 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return h2_as_u32(__floats2half2_rn(lo, hi));
 }
 
-// ------------------------------------------------------------------ K tile
-// Scores of 16 positions (rows row0, row0 + 8 of this lane) x 8 heads.
+// ------------------------------------------------------------------ K job
+// Raw scores (before sm_scale) of 16 positions (rows row0, row0 + 8 of this lane)
+// x 8 heads.  q8_0 / q4_0: codes enter the MMA as fp16 (code + offset); the
+// accumulator starts at -corr (the offset's contribution for this lane's heads) so
+// each block's sum is exactly sum_d q_d * code_d, then the block scale multiplies it.
 template <int FMT, int D>
-__device__ __forceinline__ void k_tile_scores(const uint8_t* __restrict__ codes,
-                                              const uint8_t* __restrict__ sc, int row0,
-                                              const uint32_t (&qf)[D / 16][2],
-                                              const uint32_t (&ql)[D / 16][2], const Lut& lut,
-                                              int c, float (&s)[4]) {
+__device__ __forceinline__ void k_job_scores(const uint8_t* __restrict__ codes,
+                                             const uint8_t* __restrict__ sc, int row0,
+                                             const uint32_t (&qf)[D / 16][2],
+                                             const uint32_t (&ql)[D / 16][2],
+                                             const float (&corr)[D / 32][2], const Lut& lut,
+                                             int c, float (&s)[4]) {
   using C = Cfg<FMT, D>;
   const int row1 = row0 + 8;
   const uint8_t* p0 = codes + row0 * C::CROW + (c << 2);
@@ -198,71 +207,45 @@ __device__ __forceinline__ void k_tile_scores(const uint8_t* __restrict__ codes,
   const int sw0 = (row0 >> C::SWZ_SHIFT) & C::SWZ_MASK;
   const int sw1 = (row1 >> C::SWZ_SHIFT) & C::SWZ_MASK;
   s[0] = s[1] = s[2] = s[3] = 0.f;
-  if constexpr (C::kQ8) {
-    // scales of the two rows: NBLK fp16 each
-    uint32_t d0w[2], d1w[2];
+  if constexpr (!C::kLut) {
+    float2 d0f[C::NBLK / 2 > 0 ? C::NBLK / 2 : 1], d1f[C::NBLK / 2 > 0 ? C::NBLK / 2 : 1];
     if constexpr (C::NBLK == 4) {
       const uint2 u0 = *reinterpret_cast<const uint2*>(sc + row0 * C::SROW);
       const uint2 u1 = *reinterpret_cast<const uint2*>(sc + row1 * C::SROW);
-      d0w[0] = u0.x; d0w[1] = u0.y; d1w[0] = u1.x; d1w[1] = u1.y;
+      d0f[0] = __half22float2(u32_as_h2(u0.x)); d0f[1] = __half22float2(u32_as_h2(u0.y));
+      d1f[0] = __half22float2(u32_as_h2(u1.x)); d1f[1] = __half22float2(u32_as_h2(u1.y));
     } else {
-      d0w[0] = lds32(sc + row0 * C::SROW); d1w[0] = lds32(sc + row1 * C::SROW);
-      d0w[1] = d1w[1] = 0;
+      d0f[0] = __half22float2(u32_as_h2(lds32(sc + row0 * C::SROW)));
+      d1f[0] = __half22float2(u32_as_h2(lds32(sc + row1 * C::SROW)));
     }
-    const __half2 bias = __half2half2(__ushort_as_half(0x6480));  // 1152
 #pragma unroll
     for (int m = 0; m < C::NBLK; ++m) {
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      float t[4] = {-corr[m][0], -corr[m][1], -corr[m][0], -corr[m][1]};
+      if constexpr (C::kQ8) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int ks = 2 * m + j;  // chunk ks of the row holds dims 16 ks .. 16 ks + 15
-        const uint32_t x0 = lds32(p0 + ((ks ^ sw0) << 4)) ^ 0x80808080u;
-        const uint32_t x1 = lds32(p1 + ((ks ^ sw1) << 4)) ^ 0x80808080u;
-        const uint32_t a0 = h2_as_u32(__hsub2(u32_as_h2(prmt(x0, 0x64646464u, 0x4240u)), bias));
-        const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2(prmt(x1, 0x64646464u, 0x4240u)), bias));
-        const uint32_t a2 = h2_as_u32(__hsub2(u32_as_h2(prmt(x0, 0x64646464u, 0x4341u)), bias));
-        const uint32_t a3 = h2_as_u32(__hsub2(u32_as_h2(prmt(x1, 0x64646464u, 0x4341u)), bias));
-        mma16816(t, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        for (int j = 0; j < 2; ++j) {
+          const int ks = 2 * m + j;  // chunk ks of the row holds dims 16 ks .. 16 ks + 15
+          const uint32_t x0 = lds32(p0 + ((ks ^ sw0) << 4)) ^ 0x80808080u;
+          const uint32_t x1 = lds32(p1 + ((ks ^ sw1) << 4)) ^ 0x80808080u;
+          // (byte + 128) | fp16(1024): code + 1152, exact
+          mma16816(t, prmt(x0, 0x64646464u, 0x4240u), prmt(x1, 0x64646464u, 0x4240u),
+                   prmt(x0, 0x64646464u, 0x4341u), prmt(x1, 0x64646464u, 0x4341u), qf[ks][0],
+                   qf[ks][1]);
+        }
+      } else {
+        const uint32_t x0 = lds32(p0 + ((m ^ sw0) << 4));
+        const uint32_t x1 = lds32(p1 + ((m ^ sw1) << 4));
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t y0 = x0 >> (8 * j), y1 = x1 >> (8 * j);
+          // even nibbles: 1024 + n; odd nibbles (bits 4..7): 64 + n
+          mma16816(t, (y0 & 0x000F000Fu) | kMagic, (y1 & 0x000F000Fu) | kMagic,
+                   (y0 & 0x00F000F0u) | kMagic64, (y1 & 0x00F000F0u) | kMagic64,
+                   qf[2 * m + j][0], qf[2 * m + j][1]);
+        }
       }
-      const uint32_t w0 = d0w[m >> 1], w1 = d1w[m >> 1];
-      const float d0 = __half2float(__ushort_as_half((uint16_t)((m & 1) ? (w0 >> 16) : w0)));
-      const float d1 = __half2float(__ushort_as_half((uint16_t)((m & 1) ? (w1 >> 16) : w1)));
-      s[0] = fmaf(d0, t[0], s[0]); s[1] = fmaf(d0, t[1], s[1]);
-      s[2] = fmaf(d1, t[2], s[2]); s[3] = fmaf(d1, t[3], s[3]);
-    }
-  } else if constexpr (C::kQ4) {
-    uint32_t d0w[2], d1w[2];
-    if constexpr (C::NBLK == 4) {
-      const uint2 u0 = *reinterpret_cast<const uint2*>(sc + row0 * C::SROW);
-      const uint2 u1 = *reinterpret_cast<const uint2*>(sc + row1 * C::SROW);
-      d0w[0] = u0.x; d0w[1] = u0.y; d1w[0] = u1.x; d1w[1] = u1.y;
-    } else {
-      d0w[0] = lds32(sc + row0 * C::SROW); d1w[0] = lds32(sc + row1 * C::SROW);
-      d0w[1] = d1w[1] = 0;
-    }
-    const __half2 b1032 = __half2half2(__ushort_as_half(0x6408));       // 1032
-    const __half2 inv16 = __half2half2(__ushort_as_half(0x2C00));       // 1/16
-    const __half2 m72 = __half2half2(__ushort_as_half(0xD480));         // -72
-#pragma unroll
-    for (int m = 0; m < C::NBLK; ++m) {
-      const uint32_t x0 = lds32(p0 + ((m ^ sw0) << 4));
-      const uint32_t x1 = lds32(p1 + ((m ^ sw1) << 4));
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint32_t y0 = x0 >> (8 * j), y1 = x1 >> (8 * j);
-        // (n_{2j}, n_{2j+4}) and 16 * (n_{2j+1}, n_{2j+5}) as fp16, then minus 8
-        const uint32_t a0 = h2_as_u32(__hsub2(u32_as_h2((y0 & 0x000F000Fu) | kMagic), b1032));
-        const uint32_t a1 = h2_as_u32(__hsub2(u32_as_h2((y1 & 0x000F000Fu) | kMagic), b1032));
-        const uint32_t a2 =
-            h2_as_u32(__hfma2(u32_as_h2((y0 & 0x00F000F0u) | kMagic), inv16, m72));
-        const uint32_t a3 =
-            h2_as_u32(__hfma2(u32_as_h2((y1 & 0x00F000F0u) | kMagic), inv16, m72));
-        mma16816(t, a0, a1, a2, a3, qf[2 * m + j][0], qf[2 * m + j][1]);
-      }
-      const uint32_t w0 = d0w[m >> 1], w1 = d1w[m >> 1];
-      const float d0 = __half2float(__ushort_as_half((uint16_t)((m & 1) ? (w0 >> 16) : w0)));
-      const float d1 = __half2float(__ushort_as_half((uint16_t)((m & 1) ? (w1 >> 16) : w1)));
+      const float d0 = (m & 1) ? d0f[m >> 1].y : d0f[m >> 1].x;
+      const float d1 = (m & 1) ? d1f[m >> 1].y : d1f[m >> 1].x;
       s[0] = fmaf(d0, t[0], s[0]); s[1] = fmaf(d0, t[1], s[1]);
       s[2] = fmaf(d1, t[2], s[2]); s[3] = fmaf(d1, t[3], s[3]);
     }
@@ -277,7 +260,6 @@ __device__ __forceinline__ void k_tile_scores(const uint8_t* __restrict__ codes,
       lut_lookup4(lut, x0 >> 16, nib_mask_hi(x0), L1, H1);    // row0 dims +4..7
       lut_lookup4(lut, x1, nib_mask_lo(x1), L2, H2);          // row1 dims +0..3
       lut_lookup4(lut, x1 >> 16, nib_mask_hi(x1), L3, H3);    // row1 dims +4..7
-      // k-step 2m: dims +0..3, k-step 2m+1: dims +4..7
       const uint32_t a0 = prmt(L0, H0, 0x5140u), a2 = prmt(L0, H0, 0x7362u);
       const uint32_t a1 = prmt(L2, H2, 0x5140u), a3 = prmt(L2, H2, 0x7362u);
       mma16816(s, a0, a1, a2, a3, qf[2 * m][0], qf[2 * m][1]);
@@ -315,19 +297,16 @@ __device__ __forceinline__ void v_dequant_pair(const uint32_t (&ra)[Cfg<FMT, D>:
       e[4 * k + 3] = h2_as_u32(__hsub2(u32_as_h2(prmt(t23, 0x64646464u, 0x4342u)), bias));
     } else if constexpr (C::kQ4) {
       // 8 nibbles per word -> 8 dims; x_lo holds dims 0-3 of both positions, x_hi dims 4-7
-      const __half2 b1032 = __half2half2(__ushort_as_half(0x6408));
-      const __half2 inv16 = __half2half2(__ushort_as_half(0x2C00));
-      const __half2 m72 = __half2half2(__ushort_as_half(0xD480));
+      const __half2 b1032 = __half2half2(__ushort_as_half(0x6408));  // 1032
+      const __half2 b72 = __half2half2(__ushort_as_half(0x5480));    // 72
 #pragma unroll
       for (int hlf = 0; hlf < 2; ++hlf) {
         const uint32_t x = hlf ? prmt(wa, wb, 0x7632u) : prmt(wa, wb, 0x5410u);
         const uint32_t y = x >> 8;
         e[8 * k + 4 * hlf + 0] = h2_as_u32(__hsub2(u32_as_h2((x & 0x000F000Fu) | kMagic), b1032));
-        e[8 * k + 4 * hlf + 1] =
-            h2_as_u32(__hfma2(u32_as_h2((x & 0x00F000F0u) | kMagic), inv16, m72));
+        e[8 * k + 4 * hlf + 1] = h2_as_u32(__hsub2(u32_as_h2((x & 0x00F000F0u) | kMagic64), b72));
         e[8 * k + 4 * hlf + 2] = h2_as_u32(__hsub2(u32_as_h2((y & 0x000F000Fu) | kMagic), b1032));
-        e[8 * k + 4 * hlf + 3] =
-            h2_as_u32(__hfma2(u32_as_h2((y & 0x00F000F0u) | kMagic), inv16, m72));
+        e[8 * k + 4 * hlf + 3] = h2_as_u32(__hsub2(u32_as_h2((y & 0x00F000F0u) | kMagic64), b72));
       }
     } else {
 #pragma unroll
@@ -361,19 +340,17 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
   }
 }
 
-// Scale (q8_0 / q4_0 block scale of this thread's dims, or lut4 vector norm) of a
-// staged position; 0 for slots past the end so that stale rows contribute nothing.
+// Scale of a staged position (q8_0 / q4_0 block scale of this thread's dims, or the
+// lut4 vector norm), read from the row's 16-byte scale window; 0 past the end so
+// that stale rows contribute nothing.
 template <int FMT, int D>
-__device__ __forceinline__ __half v_scale(const uint8_t* rec, int slot, int n_valid, int blk,
+__device__ __forceinline__ __half v_scale(const uint8_t* grp, int slot, int n_valid, int blk,
                                           const uint16_t* list_grp) {
   using C = Cfg<FMT, D>;
   if (slot >= n_valid) return __ushort_as_half(0);
-  if constexpr (C::kLut) {
-    const int tok = list_grp[slot];
-    return *reinterpret_cast<const __half*>(rec + slot * 8 + 2 * (tok & 1));
-  } else {
-    return *reinterpret_cast<const __half*>(rec + slot * 8 + 2 * blk);
-  }
+  const int tok = list_grp[slot];
+  const int off = C::CROW + (tok & (C::RPW - 1)) * C::SROW + (C::kLut ? 0 : 2 * blk);
+  return *reinterpret_cast<const __half*>(grp + slot * C::VSTRIDE + off);
 }
 
 // One group of 16 staged positions: acc[dims x heads] += v_hat^T p.
@@ -382,15 +359,14 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ grp, const _
                                         const uint16_t* __restrict__ list_grp, int n_valid, int r,
                                         int c, const Lut& lut, float (&acc)[Cfg<FMT, D>::MT][4]) {
   using C = Cfg<FMT, D>;
-  const uint8_t* rec = grp + 16 * C::VSTRIDE;
   const int blk = (C::E * r) / 32;
   const int sa = 2 * c, sc = sa + 8;
   const uint32_t b0 = lds32(prow + sa);
   const uint32_t b1 = lds32(prow + sc);
-  const __half2 dab = __halves2half2(v_scale<FMT, D>(rec, sa, n_valid, blk, list_grp),
-                                     v_scale<FMT, D>(rec, sa + 1, n_valid, blk, list_grp));
-  const __half2 dcd = __halves2half2(v_scale<FMT, D>(rec, sc, n_valid, blk, list_grp),
-                                     v_scale<FMT, D>(rec, sc + 1, n_valid, blk, list_grp));
+  const __half2 dab = __halves2half2(v_scale<FMT, D>(grp, sa, n_valid, blk, list_grp),
+                                     v_scale<FMT, D>(grp, sa + 1, n_valid, blk, list_grp));
+  const __half2 dcd = __halves2half2(v_scale<FMT, D>(grp, sc, n_valid, blk, list_grp),
+                                     v_scale<FMT, D>(grp, sc + 1, n_valid, blk, list_grp));
   uint32_t wa[C::NWORD], wb[C::NWORD], wc[C::NWORD], wd[C::NWORD];
   const int boff = C::RAWB * r;
   v_raw<FMT, D>(grp + sa * C::VSTRIDE + boff, wa);
@@ -410,6 +386,13 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ grp, const _
     mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
 }
 
+// bit 4r set iff any of bits 4r .. 4r+3 of a ballot is set (one row per 4-lane group)
+__device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
+  uint32_t x = bal | (bal >> 1);
+  x |= x >> 2;
+  return x & 0x11111111u;
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -419,19 +402,22 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* stages = smem + LY::stage;
-  float* S = reinterpret_cast<float*>(smem + LY::S);
+  float* ored = reinterpret_cast<float*>(smem + LY::ored);
   __half* pkt = reinterpret_cast<__half*>(smem + LY::pkt);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + LY::list);
   uint8_t* vst = smem + LY::vst;
   float* qs = reinterpret_cast<float*>(smem + LY::q);
+  float* corr_s = reinterpret_cast<float*>(smem + LY::corr);
   int* item_rows = reinterpret_cast<int*>(smem + LY::rows);
   int* stage_row = reinterpret_cast<int*>(smem + LY::stage_row);
   float* red_m = reinterpret_cast<float*>(smem + LY::red);
   float* red_l = red_m + kConsumerWarps * 8;
   int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
   int* cnt_kept = cnt_skip + kConsumerWarps;
+  int* abort_flag = cnt_skip + 2 * kConsumerWarps;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::bars);
   uint64_t* empty = full + C::STAGES;
+  uint64_t* vbar = empty + C::STAGES;
   int* prefix = reinterpret_cast<int*>(smem + LY::prefix);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -450,11 +436,12 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   }
   if (tid == 0) {
     prefix[0] = 0;
-    cnt_skip[2 * kConsumerWarps] = 0;  // consumer timeout flag
+    *abort_flag = 0;
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 4);  // the four warps that consume the tile's four 16-row jobs
     }
+    for (int i = 0; i < kConsumerWarps * C::NVS; ++i) mbar_init(&vbar[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -549,8 +536,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   float* ws_l = ws_m + n_part;
   const int wslot0 = warp * kWarpSlots;  // this warp's region of the kept list / weights
   uint8_t* my_vst = vst + (size_t)warp * C::NVS * C::VGROUP;
+  uint64_t* my_vbar = vbar + warp * C::NVS;
+  const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;  // this lane's two heads exist
 
   int g_base = 0;  // K tiles consumed by this CTA before the current unit
+  int vg = 0;      // V groups fetched by this warp so far (mbarrier phase bookkeeping)
   for (int k = 0;; ++k) {
     const int it = blockIdx.x + k * gridDim.x;
     if (it >= total_items) break;
@@ -558,64 +548,74 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
     const int ntiles = (I.n_tok + kTile - 1) / kTile;
     const int njobs = 4 * ntiles;
 
-    // ---- query group -> shared (fp32), rotated for lut4
+    // ---- query group -> shared (fp32)
     {
       constexpr int kChunks = 8 * D / 8;  // 16-byte chunks of 8 heads x D fp16
+      if (tid < kChunks) {
+        const int h = tid / (D / 8), d0 = (tid - h * (D / 8)) * 8;
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (h < G)
+          raw = *reinterpret_cast<const uint4*>(qg + ((size_t)I.b * Hq + I.kvh * G + h) * D + d0);
+        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
-      for (int j = 0; j < (kChunks + kConsumers - 1) / kConsumers; ++j) {
-        const int ch = tid + j * kConsumers;
-        if (ch < kChunks) {
-          const int h = ch / (D / 8), d0 = (ch - h * (D / 8)) * 8;
-          uint4 raw = make_uint4(0, 0, 0, 0);
-          if (h < G)
-            raw = *reinterpret_cast<const uint4*>(qg + ((size_t)I.b * Hq + I.kvh * G + h) * D + d0);
-          const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(hp[e]);
-            qs[h * D + d0 + 2 * e] = f.x;
-            qs[h * D + d0 + 2 * e + 1] = f.y;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(hp[e]);
+          qs[h * D + d0 + 2 * e] = f.x;
+          qs[h * D + d0 + 2 * e + 1] = f.y;
         }
       }
     }
     consumer_sync();
-    if constexpr (C::kLut) {
-      // q' = c * H * (s .* q), butterflies in fp32; warp w rotates head w
-      constexpr int K = D / 32;
+    if (warp < 8) {
       const int h = warp;
-      float y[K];
-#pragma unroll
-      for (int kk = 0; kk < K; ++kk) {
-        const int i = 32 * kk + lane;
-        y[kk] = qs[h * D + i] * (float)a.desc.signs[i];
-      }
-#pragma unroll
-      for (int hb = 1; hb < 32; hb <<= 1) {
-        const bool upper = (lane & hb) != 0;
+      constexpr int K = D / 32;
+      if constexpr (C::kLut) {
+        // q' = c * H * (s .* q), butterflies in fp32; warp h rotates head h
+        float y[K];
 #pragma unroll
         for (int kk = 0; kk < K; ++kk) {
-          const float o = __shfl_xor_sync(0xffffffffu, y[kk], hb);
-          y[kk] = upper ? (o - y[kk]) : (y[kk] + o);
+          const int i = 32 * kk + lane;
+          y[kk] = qs[h * D + i] * (float)a.desc.signs[i];
+        }
+#pragma unroll
+        for (int hb = 1; hb < 32; hb <<= 1) {
+          const bool upper = (lane & hb) != 0;
+#pragma unroll
+          for (int kk = 0; kk < K; ++kk) {
+            const float o = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+            y[kk] = upper ? (o - y[kk]) : (y[kk] + o);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk + 1 < K; kk += 2) {
+          const float u = y[kk], v = y[kk + 1];
+          y[kk] = u + v; y[kk + 1] = u - v;
+        }
+        if (K == 4) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const float u = y[kk], v = y[kk + 2];
+            y[kk] = u + v; y[kk + 2] = u - v;
+          }
+        }
+        const float cs = rsqrtf((float)D);
+#pragma unroll
+        for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
+      } else {
+        // offset contribution per (head, block): sum_d q_d * (offset_d + 8) for q4_0
+        // (offset 1024 on even dims, 64 on odd dims), sum_d q_d * 1152 for q8_0; fp64 sums
+#pragma unroll
+        for (int m = 0; m < K; ++m) {
+          const int d = 32 * m + lane;
+          const double w = C::kQ8 ? 1152.0 : ((d & 1) ? 72.0 : 1032.0);
+          double v = (double)qs[h * D + d] * w;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) corr_s[h * C::NBLK + m] = (float)v;
         }
       }
-#pragma unroll
-      for (int kk = 0; kk + 1 < K; kk += 2) {
-        const float u = y[kk], v = y[kk + 1];
-        y[kk] = u + v; y[kk + 1] = u - v;
-      }
-      if (K == 4) {
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const float u = y[kk], v = y[kk + 2];
-          y[kk] = u + v; y[kk + 2] = u - v;
-        }
-      }
-      const float cs = rsqrtf((float)D);
-#pragma unroll
-      for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
-      consumer_sync();
     }
+    consumer_sync();
     uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
 #pragma unroll
     for (int ks = 0; ks < C::KSTEPS; ++ks) {
@@ -633,33 +633,44 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         ql[ks][0] = ql[ks][1] = 0;
       }
     }
+    float corr[C::NBLK][2];
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      corr[m][0] = C::kLut ? 0.f : corr_s[(2 * c) * C::NBLK + m];
+      corr[m][1] = C::kLut ? 0.f : corr_s[(2 * c + 1) * C::NBLK + m];
+    }
 
-    // ---- K pass: this warp's 16-row jobs
+    // ---- K pass: this warp's 16-row jobs; scores stay in registers
+    float sreg[kJobsPerWarp][4];
     float mx0 = -INFINITY, mx1 = -INFINITY;
-    bool timed_out = false;
-    for (int j = warp; j < njobs; j += kConsumerWarps) {
-      const int t = j >> 2, mt = j & 3;
-      const int g = g_base + t;
-      const int stage = g % C::STAGES;
-      if (!mbar_wait_bounded(&full[stage], (uint32_t)(g / C::STAGES) & 1u)) {
-        timed_out = true;
-        break;
+    bool ok_all = true;
+#pragma unroll
+    for (int jj = 0; jj < kJobsPerWarp; ++jj) {
+      sreg[jj][0] = sreg[jj][1] = sreg[jj][2] = sreg[jj][3] = -INFINITY;
+      const int j = warp + kConsumerWarps * jj;
+      if (j < njobs && ok_all) {
+        const int t = j >> 2, mt = j & 3;
+        const int g = g_base + t;
+        const int stage = g % C::STAGES;
+        ok_all = __all_sync(0xffffffffu, mbar_wait_bounded(&full[stage], (uint32_t)(g / C::STAGES) & 1u));
+        if (ok_all) {
+          const uint8_t* base = stages + (size_t)stage * C::STAGE_BYTES;
+          const int row0 = 16 * mt + r;
+          float s[4];
+          k_job_scores<FMT, D>(base, base + C::STAGE_CODE, row0, qf, ql, corr, lut, c, s);
+          if (mt == 0 && lane == 0) item_rows[t] = stage_row[stage];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stage]);
+          const int p0 = 16 * j + r;
+          const bool v0 = p0 < I.n_tok, v1 = p0 + 8 < I.n_tok;
+          sreg[jj][0] = v0 ? s[0] * qk_scale : -INFINITY;
+          sreg[jj][1] = v0 ? s[1] * qk_scale : -INFINITY;
+          sreg[jj][2] = v1 ? s[2] * qk_scale : -INFINITY;
+          sreg[jj][3] = v1 ? s[3] * qk_scale : -INFINITY;
+          mx0 = fmaxf(mx0, fmaxf(sreg[jj][0], sreg[jj][2]));
+          mx1 = fmaxf(mx1, fmaxf(sreg[jj][1], sreg[jj][3]));
+        }
       }
-      const uint8_t* base = stages + (size_t)stage * C::STAGE_BYTES;
-      const int row0 = 16 * mt + r;
-      float s[4];
-      k_tile_scores<FMT, D>(base, base + C::STAGE_CODE, row0, qf, ql, lut, c, s);
-      if (mt == 0 && lane == 0) item_rows[t] = stage_row[stage];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-      const int p0 = t * kTile + row0, p1 = p0 + 8;
-      const bool v0 = p0 < I.n_tok, v1 = p1 < I.n_tok;
-      const float s0 = v0 ? s[0] * qk_scale : -INFINITY, s1 = v0 ? s[1] * qk_scale : -INFINITY;
-      const float s2 = v1 ? s[2] * qk_scale : -INFINITY, s3 = v1 ? s[3] * qk_scale : -INFINITY;
-      *reinterpret_cast<float2*>(S + p0 * 8 + 2 * c) = make_float2(s0, s1);
-      *reinterpret_cast<float2*>(S + p1 * 8 + 2 * c) = make_float2(s2, s3);
-      mx0 = fmaxf(mx0, fmaxf(s0, s2));
-      mx1 = fmaxf(mx1, fmaxf(s1, s3));
     }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
@@ -670,61 +681,57 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       red_m[warp * 8 + 2 * c] = mx0;
       red_m[warp * 8 + 2 * c + 1] = mx1;
     }
-    // barrier 1: every score of the unit and every warp's maximum are in shared memory
-    if (timed_out && lane == 0) atomicOr(cnt_skip + 2 * kConsumerWarps, 1);
-    consumer_sync();
-    if (cnt_skip[2 * kConsumerWarps] != 0) {
+    if (!ok_all && lane == 0) atomicOr(abort_flag, 1);
+    consumer_sync();  // barrier 1: every warp's maxima are in shared memory
+    if (*abort_flag) {
       if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-      break;  // leave the unit loop; all consumer warps see the same flag
+      break;  // all consumer warps see the same flag
     }
     g_base += ntiles;
 
-    // ---- weights, skip test, compaction (own jobs); lane -> (row lane/2, heads 4*(lane&1)..+3)
-    const int hq0 = 4 * (lane & 1);
-    float mh[4];
+    // ---- weights, skip test, compaction, from the registers (rows r, r+8; heads 2c, 2c+1)
+    float mh0 = red_m[2 * c], mh1 = red_m[2 * c + 1];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float v = red_m[hq0 + i];
-#pragma unroll
-      for (int w = 1; w < kConsumerWarps; ++w) v = fmaxf(v, red_m[w * 8 + hq0 + i]);
-      mh[i] = v;
+    for (int w = 1; w < kConsumerWarps; ++w) {
+      mh0 = fmaxf(mh0, red_m[w * 8 + 2 * c]);
+      mh1 = fmaxf(mh1, red_m[w * 8 + 2 * c + 1]);
     }
-    float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+    float l0 = 0.f, l1 = 0.f;
     int nkept = 0, nskip = 0;
-    const unsigned lt_mask = (1u << (lane & ~1)) - 1u;
-    for (int j = warp; j < njobs; j += kConsumerWarps) {
-      const int pos = 16 * j + (lane >> 1);
-      const bool valid = pos < I.n_tok;
-      float sv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (valid) {
-        const float4 f = *reinterpret_cast<const float4*>(S + pos * 8 + hq0);
-        sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
-      }
-      bool keep[4];
-      bool any = false;
-      float p[4];
+    const uint32_t below = (1u << (4 * r)) - 1u;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool live = valid && (hq0 + i < G);
-        const float dlt = sv[i] - mh[i];
-        p[i] = live ? ex2(dlt) : 0.f;
-        lsum[i] += p[i];
-        keep[i] = live && dlt >= thr;
-        any |= keep[i];
-        nskip += (live && !keep[i]) ? 1 : 0;
+    for (int jj = 0; jj < kJobsPerWarp; ++jj) {
+      const int j = warp + kConsumerWarps * jj;
+      if (j < njobs) {
+        const int p0 = 16 * j + r;
+        const bool va = p0 < I.n_tok, vb = p0 + 8 < I.n_tok;
+        const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
+        const float da0 = sreg[jj][0] - mh0, da1 = sreg[jj][1] - mh1;
+        const float db0 = sreg[jj][2] - mh0, db1 = sreg[jj][3] - mh1;
+        const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
+        const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
+        l0 += ea0 + eb0;
+        l1 += ea1 + eb1;
+        const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
+        const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
+        nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
+        const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
+        const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
+        const int na = __popc(rows_a);
+        if ((rows_a >> (4 * r)) & 1u) {
+          const int slot = wslot0 + nkept + __popc(rows_a & below);
+          if (c == 0) list[slot] = (uint16_t)p0;
+          pkt[(2 * c) * kPktStride + slot] = __float2half_rn(ka0 ? ea0 * kPScale : 0.f);
+          pkt[(2 * c + 1) * kPktStride + slot] = __float2half_rn(ka1 ? ea1 * kPScale : 0.f);
+        }
+        if ((rows_b >> (4 * r)) & 1u) {
+          const int slot = wslot0 + nkept + na + __popc(rows_b & below);
+          if (c == 0) list[slot] = (uint16_t)(p0 + 8);
+          pkt[(2 * c) * kPktStride + slot] = __float2half_rn(kb0 ? eb0 * kPScale : 0.f);
+          pkt[(2 * c + 1) * kPktStride + slot] = __float2half_rn(kb1 ? eb1 * kPScale : 0.f);
+        }
+        nkept += na + __popc(rows_b);
       }
-      // (the shuffle must run on every lane: never inside a short-circuit)
-      const int partner_any = __shfl_xor_sync(0xffffffffu, any ? 1 : 0, 1);
-      any = any || (partner_any != 0);
-      const unsigned bal = __ballot_sync(0xffffffffu, any) & 0x55555555u;
-      if (any) {
-        const int slot = wslot0 + nkept + __popc(bal & lt_mask);
-        if ((lane & 1) == 0) list[slot] = (uint16_t)pos;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          pkt[(hq0 + i) * kPktStride + slot] = __float2half_rn(keep[i] ? p[i] * kPScale : 0.f);
-      }
-      nkept += __popc(bal);
     }
     // zero the weights of the padding slots of the last partial group of 16
     {
@@ -733,15 +740,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         pkt[(i / pad) * kPktStride + wslot0 + nkept + (i % pad)] = __ushort_as_half(0);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int o = 2; o < 32; o <<= 1) lsum[i] += __shfl_xor_sync(0xffffffffu, lsum[i], o);
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
-    if (lane < 2) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) red_l[warp * 8 + hq0 + i] = lsum[i];
+    if (r == 0) {
+      red_l[warp * 8 + 2 * c] = l0;
+      red_l[warp * 8 + 2 * c + 1] = l1;
     }
     if (lane == 0) {
       cnt_skip[warp] = nskip;
@@ -755,69 +762,74 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
     for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     const int ngroups = (nkept + 15) >> 4;
     auto issue = [&](int gi) {
-      uint8_t* grp = my_vst + (size_t)(gi % C::NVS) * C::VGROUP;
-      constexpr int CPR = C::CROW / 16;
-      for (int ch = lane; ch < 16 * CPR; ch += 32) {
-        const int rl = ch / CPR, cc = ch - rl * CPR;
-        const int slot = 16 * gi + rl;
-        if (slot < nkept) {
-          const int tok = list[wslot0 + slot];
-          const int rb = item_rows[tok >> 6];
-          if (rb >= 0) {
-            const size_t row = (size_t)rb + (tok & 63);
-            cp_async16(grp + rl * C::VSTRIDE + cc * 16, vcodes + row * C::CROW + cc * 16);
-          }
-        }
+      const int stage = (vg + gi) % C::NVS;
+      uint8_t* grp = my_vst + (size_t)stage * C::VGROUP;
+      const int slot = 16 * gi + lane;
+      const bool valid = lane < 16 && slot < nkept;
+      const int tok = valid ? list[wslot0 + slot] : 0;
+      const int rb = valid ? item_rows[tok >> 6] : -1;
+      const bool go = valid && rb >= 0;
+      const int nrows = __popc(__ballot_sync(0xffffffffu, go));
+      if (lane == 0) {
+        if (nrows) mbar_arrive_expect_tx(&my_vbar[stage], nrows * (C::CROW + 16));
+        else mbar_arrive(&my_vbar[stage]);
       }
-      if (lane < 16) {
-        const int slot = 16 * gi + lane;
-        if (slot < nkept) {
-          const int tok = list[wslot0 + slot];
-          const int rb = item_rows[tok >> 6];
-          if (rb >= 0) {
-            const size_t row = (size_t)rb + (tok & 63);
-            uint8_t* rec = grp + 16 * C::VSTRIDE + lane * 8;
-            if constexpr (C::kLut) cp_async4(rec, vscales + (row & ~(size_t)1) * 2);
-            else if constexpr (C::SROW == 8) cp_async8(rec, vscales + row * 8);
-            else cp_async4(rec, vscales + row * 4);
-          }
-        }
+      __syncwarp();
+      if (go) {
+        const size_t row = (size_t)rb + (tok & 63);
+        bulk_load(grp + lane * C::VSTRIDE, vcodes + row * C::CROW, C::CROW, &my_vbar[stage]);
+        bulk_load(grp + lane * C::VSTRIDE + C::CROW,
+                  vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW, 16, &my_vbar[stage]);
       }
-      cp_async_commit();
     };
 #pragma unroll
-    for (int i = 0; i < C::NVS; ++i) {
+    for (int i = 0; i < C::NVS; ++i)
       if (i < ngroups) issue(i);
-      else cp_async_commit();
-    }
+    bool vok = true;
     for (int gi = 0; gi < ngroups; ++gi) {
-      cp_async_wait<C::NVS - 1>();
-      __syncwarp();
-      v_group<FMT, D>(my_vst + (size_t)(gi % C::NVS) * C::VGROUP,
-                      pkt + r * kPktStride + wslot0 + 16 * gi, list + wslot0 + 16 * gi,
-                      min(16, nkept - 16 * gi), r, c, lut, acc);
+      const int stage = (vg + gi) % C::NVS;
+      vok = __all_sync(0xffffffffu,
+                       mbar_wait_bounded(&my_vbar[stage], (uint32_t)((vg + gi) / C::NVS) & 1u));
+      if (!vok) break;
+      v_group<FMT, D>(my_vst + (size_t)stage * C::VGROUP, pkt + r * kPktStride + wslot0 + 16 * gi,
+                      list + wslot0 + 16 * gi, min(16, nkept - 16 * gi), r, c, lut, acc);
       __syncwarp();
       if (gi + C::NVS < ngroups) issue(gi + C::NVS);
-      else cp_async_commit();
     }
-    cp_async_wait<0>();
+    vg += ngroups;
+    if (!vok && lane == 0) atomicOr(abort_flag, 1);
 
-    // ---- sum the warps' accumulators (through the score buffer) and write the unit
-    consumer_sync();  // barrier 2: no warp still reads scores
-    float* ored = S;  // [warp][accumulator register][lane]
+    // ---- sum the warps' accumulators and write the unit
     constexpr int NE = C::MT * 4;  // accumulator registers per thread
+    consumer_sync();  // barrier 2
+    if (*abort_flag) {
+      if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+      break;
+    }
+    if (warp >= 8) {
 #pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt)
+      for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ored[(warp * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
+        for (int i = 0; i < 4; ++i) ored[((warp - 8) * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
+    }
     consumer_sync();  // barrier 3
+    if (warp < 8) {
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float* p = ored + (warp * NE + mt * 4 + i) * 32 + lane;
+          *p = *p + acc[mt][i];
+        }
+    }
+    consumer_sync();  // barrier 4
     {
       const size_t unit0 = ((size_t)I.b * Hq + (size_t)I.kvh * G) * a.max_splits + I.split;
       for (int q = tid; q < 32 * NE; q += kConsumers) {
         const int ln = q & 31, e = q >> 5;
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) v += ored[(w * NE + e) * 32 + ln];
+        for (int w = 0; w < 8; ++w) v += ored[(w * NE + e) * 32 + ln];
         const int mt = e >> 2, i = e & 3;
         const int rr = ln >> 2, cc = ln & 3;
         const int h = 2 * cc + (i & 1);
@@ -848,7 +860,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         atomicAdd(&a.stats[3], (unsigned long long)(I.n_tok - nk));
       }
     }
-    consumer_sync();  // barrier 4: shared buffers free for the next unit
+    // the next unit's first barrier (after its query staging) keeps every buffer read
+    // above ahead of that unit's writes
   }
   cta_final_sync();  // with the producer warp
 }

@@ -93,7 +93,9 @@ struct Layout {
   static constexpr size_t ored = stage + (size_t)C::STAGES * C::STAGE_BYTES;  // float [8][NE][32]
   static constexpr size_t pkt = ored + (size_t)8 * (D / 16) * 4 * 32 * 4;     // half [8][kPktStride]
   static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;            // u16 [kLmax]
-  static constexpr size_t vst = list + (size_t)kLmax * 2;                     // [warps][NVS][VGROUP]
+  static constexpr size_t pktg = list + (size_t)kLmax * 2;                    // half [8][kPktStride]
+  static constexpr size_t listg = pktg + (size_t)8 * kPktStride * 2;          // u16 [kLmax]
+  static constexpr size_t vst = listg + (size_t)kLmax * 2;                    // [warps][NVS][VGROUP]
   static constexpr size_t q = vst + (size_t)kConsumerWarps * C::NVS * C::VGROUP;  // float [8][D]
   static constexpr size_t corr = q + (size_t)8 * D * 4;                       // float [8][NBLK]
   static constexpr size_t rows = corr + (size_t)8 * C::NBLK * 4;              // int [kMaxTiles]
@@ -405,6 +407,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   float* ored = reinterpret_cast<float*>(smem + LY::ored);
   __half* pkt = reinterpret_cast<__half*>(smem + LY::pkt);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + LY::list);
+  __half* pktg = reinterpret_cast<__half*>(smem + LY::pktg);        // CTA-wide compacted weights
+  uint16_t* listg = reinterpret_cast<uint16_t*>(smem + LY::listg);  // CTA-wide kept list
   uint8_t* vst = smem + LY::vst;
   float* qs = reinterpret_cast<float*>(smem + LY::q);
   float* corr_s = reinterpret_cast<float*>(smem + LY::corr);
@@ -733,12 +737,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         nkept += na + __popc(rows_b);
       }
     }
-    // zero the weights of the padding slots of the last partial group of 16
-    {
-      const int pad = ((nkept + 15) & ~15) - nkept;
-      for (int i = lane; i < 8 * pad; i += 32)
-        pkt[(i / pad) * kPktStride + wslot0 + nkept + (i % pad)] = __ushort_as_half(0);
-    }
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -754,19 +752,39 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       cnt_skip[warp] = nskip;
       cnt_kept[warp] = nkept;
     }
-    __syncwarp();
+    consumer_sync();  // barrier 2: every warp's kept count is known
+    // ---- concatenate the warps' lists in warp order (deterministic) into the CTA list
+    int gbase = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const int n = cnt_kept[w];
+      gbase += (w < warp) ? n : 0;
+      total += n;
+    }
+    for (int i = lane; i < nkept; i += 32) listg[gbase + i] = list[wslot0 + i];
+    for (int i = lane; i < 8 * nkept; i += 32) {
+      const int h = i / nkept, sl = i - h * nkept;
+      pktg[h * kPktStride + gbase + sl] = pkt[h * kPktStride + wslot0 + sl];
+    }
+    if (warp == kConsumerWarps - 1) {  // zero the padding slots of the last partial group
+      const int pad = ((total + 15) & ~15) - total;
+      for (int i = lane; i < 8 * pad; i += 32)
+        pktg[(i / pad) * kPktStride + total + (i % pad)] = __ushort_as_half(0);
+    }
+    consumer_sync();  // barrier 3: the CTA list is complete
 
-    // ---- V pass over this warp's kept positions only
+    // ---- V pass: kept positions only, 16-row groups dealt round-robin to the warps
     float acc[C::MT][4];
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    const int ngroups = (nkept + 15) >> 4;
-    auto issue = [&](int gi) {
+    const int ngroups_all = (total + 15) >> 4;
+    const int ngroups = ngroups_all > warp ? (ngroups_all - warp + kConsumerWarps - 1) / kConsumerWarps : 0;
+    auto issue = [&](int gi) {  // gi: this warp's gi-th group = CTA group warp + 16 gi
       const int stage = (vg + gi) % C::NVS;
       uint8_t* grp = my_vst + (size_t)stage * C::VGROUP;
-      const int slot = 16 * gi + lane;
-      const bool valid = lane < 16 && slot < nkept;
-      const int tok = valid ? list[wslot0 + slot] : 0;
+      const int slot = 16 * (warp + kConsumerWarps * gi) + lane;
+      const bool valid = lane < 16 && slot < total;
+      const int tok = valid ? listg[slot] : 0;
       const int rb = valid ? item_rows[tok >> 6] : -1;
       const bool go = valid && rb >= 0;
       const int nrows = __popc(__ballot_sync(0xffffffffu, go));
@@ -791,8 +809,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       vok = __all_sync(0xffffffffu,
                        mbar_wait_bounded(&my_vbar[stage], (uint32_t)((vg + gi) / C::NVS) & 1u));
       if (!vok) break;
-      v_group<FMT, D>(my_vst + (size_t)stage * C::VGROUP, pkt + r * kPktStride + wslot0 + 16 * gi,
-                      list + wslot0 + 16 * gi, min(16, nkept - 16 * gi), r, c, lut, acc);
+      const int s0 = 16 * (warp + kConsumerWarps * gi);
+      v_group<FMT, D>(my_vst + (size_t)stage * C::VGROUP, pktg + r * kPktStride + s0, listg + s0,
+                      min(16, total - s0), r, c, lut, acc);
       __syncwarp();
       if (gi + C::NVS < ngroups) issue(gi + C::NVS);
     }
@@ -801,7 +820,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
 
     // ---- sum the warps' accumulators and write the unit
     constexpr int NE = C::MT * 4;  // accumulator registers per thread
-    consumer_sync();  // barrier 2
+    consumer_sync();  // barrier 4: every warp's V accumulation is done
     if (*abort_flag) {
       if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
       break;
@@ -812,7 +831,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) ored[((warp - 8) * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
-    consumer_sync();  // barrier 3
+    consumer_sync();  // barrier 5
     if (warp < 8) {
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt)
@@ -822,7 +841,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
           *p = *p + acc[mt][i];
         }
     }
-    consumer_sync();  // barrier 4
+    consumer_sync();  // barrier 6
     {
       const size_t unit0 = ((size_t)I.b * Hq + (size_t)I.kvh * G) * a.max_splits + I.split;
       for (int q = tid; q < 32 * NE; q += kConsumers) {

@@ -6,33 +6,33 @@
 // accumulation are skipped for every position whose weight exp(s - m_running)
 // is below tau.  Section "FAQ": K itself is always dequantized.
 //
-// Persistent CTAs (one per SM) loop over work units (sequence b, KV head,
-// split of <= 1024 positions).  Each CTA has 16 consumer warps and 1 producer warp.
-//   producer  One lane streams 64-position K tiles (codes + block scales) into a
-//             ring of shared-memory stages with TMA: a 2-D tensor copy with hardware
-//             swizzle for the codes and a 1-D bulk copy for the scales, guarded by
-//             full/empty mbarriers, running ahead across work units.
-//   K pass    The unit's positions are cut into 16-position jobs dealt round-robin to
-//             the consumer warps.  Codes go into the tensor cores (mma m16n8k16:
-//             positions x heads x head_dim) as magic-number fp16 values (code + a
-//             fixed offset); the offset's contribution, a per-(head, block) constant of
-//             the query, is preloaded into the accumulator, and the block scale /
-//             vector norm is applied to the fp32 score.  Scores stay in registers.
+// Persistent CTAs (one per SM, 16 warps) loop over work units (sequence b, KV
+// head, split of <= 1024 positions = at most 16 tiles of 64 positions).
+//   K fetch   Warp w owns tile w of the unit.  At the start of the unit it streams
+//             the tile's codes and block scales into its private shared buffer with
+//             16-byte cp.async copies (an XOR swizzle on the codes keeps the MMA
+//             fragment reads free of bank conflicts); nothing waits on another warp.
+//             (Measured on B200: per-operation costs make 4 KB bulk/TMA copies run at
+//             a fraction of what many 16-byte async copies reach.)
+//   K pass    Once its copies land, the warp scores its 64 positions x 8 query heads
+//             on the tensor cores (mma m16n8k16: positions x heads x head_dim).  Codes
+//             enter the MMA as magic-number fp16 values (code + a fixed offset); the
+//             offset's contribution, a per-(head, block) constant of the query, is
+//             preloaded into the accumulator, and the block scale / vector norm is
+//             applied to the fp32 score.
 //   weights   After one CTA barrier m_running is the unit's maximum.  Each warp tests
 //             its scores: keep iff s - m >= log2(tau) (no exp for the test); the
 //             denominator l sums 2^(s - m) over every position; positions kept by any
 //             head of the group are compacted (ballot + popcount) into the warp's
-//             private list, with their weights (fp16, x 2^14) per head.
-//   V pass    Each warp fetches only its kept V rows (one bulk copy of the codes and
-//             one of an aligned scale window per row, completing on a per-warp
-//             mbarrier, several groups of 16 rows in flight), dequantizes them in
-//             registers and accumulates p^T V on the tensor cores (head_dim x heads x
-//             positions).  Skipped positions cost no HBM read, no dequant, no MMA.
+//             list, and the lists are concatenated in warp order into one CTA list.
+//   V pass    16-row groups of the CTA list are dealt round-robin to the warps.  A warp
+//             gathers only those kept V rows (cp.async 16-byte copies into its buffer,
+//             three groups in flight), dequantizes them in registers and accumulates
+//             p^T V on the tensor cores (head_dim x heads x positions).  Skipped
+//             positions cost no HBM read, no dequant, no MMA.
 //   output    The warps' accumulators are summed in shared memory; unnormalized o,
 //             m (log2 units) and l of the unit go to the workspace and kvq_combine
 //             merges the units of a sequence.
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "kvq_device.cuh"
@@ -41,21 +41,18 @@
 namespace kvq {
 namespace {
 
-constexpr int kConsumerWarps = 16;
-constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kThreads = kConsumers + 32;  // + one producer warp
+constexpr int kWarps = 16;
+constexpr int kThreads = 32 * kWarps;
 constexpr int kLmax = KVQ_MAX_SPLIT_TOKENS;
 constexpr int kMaxTiles = kLmax / kTile;
-constexpr int kJobsPerWarp = kLmax / 16 / kConsumerWarps;  // 16-row jobs per warp per unit (max)
-constexpr int kWarpSlots = 16 * kJobsPerWarp;             // kept-list slots owned by one warp
-constexpr int kPktStride = kLmax + 8;   // halves per head row of the compacted weights
-constexpr float kPScale = 16384.0f;     // p is stored in fp16 as p * 2^14
+static_assert(kMaxTiles == kWarps, "one K tile per warp per unit");
+constexpr int kWarpSlots = kTile;        // kept-list slots owned by one warp (its tile)
+constexpr int kPktStride = kLmax + 8;    // halves per head row of the compacted weights
+constexpr float kPScale = 16384.0f;      // p is stored in fp16 as p * 2^14
 constexpr float kPUnscale = 1.0f / 16384.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kMagic = 0x64006400u;    // fp16 1024 in both halves (unit mantissa step 1)
 constexpr uint32_t kMagic64 = 0x54005400u;  // fp16 64: mantissa bits 4..7 then count in units of 1
-constexpr int kBarConsumers = 1;            // named barrier shared by the consumer warps
-static_assert(kJobsPerWarp * kConsumerWarps * 16 == kLmax, "job split");
 
 template <int FMT, int D>
 struct Cfg {
@@ -68,57 +65,49 @@ struct Cfg {
   static constexpr int RPW = 16 / SROW;                  // rows per 16-byte scale window
   static constexpr int NBLK = D / 32;
   static constexpr int KSTEPS = D / 16;
-  static constexpr int STAGE_CODE = kTile * CROW;
-  static constexpr int STAGE_SC = kTile * SROW;
-  static constexpr int STAGE_BYTES = (STAGE_CODE + STAGE_SC + 1023) / 1024 * 1024;
-  static constexpr int STAGES = STAGE_BYTES <= 5120 ? 16 : 8;
-  // TMA swizzle of the codes: 16-byte chunk index ^= (row >> SWZ_SHIFT) & SWZ_MASK
+  static constexpr int STAGE_CODE = kTile * CROW;        // one K tile: codes ...
+  static constexpr int STAGE_SC = kTile * SROW;          // ... then scales
+  // XOR swizzle of 16-byte chunks within a code row: chunk ^= (row >> SWZ_SHIFT) & SWZ_MASK
   static constexpr int SWZ_SHIFT = CROW == 128 ? 0 : CROW == 64 ? 1 : 2;
   static constexpr int SWZ_MASK = CROW / 16 - 1;
-  // V pass (warp-private): thread (r, c) owns dims E*r .. E*r + E - 1
+  // V pass: thread (r, c) owns dims E*r .. E*r + E - 1
   static constexpr int E = D / 8;
   static constexpr int MT = D / 16;                      // m-tiles (16 dims each)
   static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
   static constexpr int NWORD = RAWB / 4;
   static constexpr int VSTRIDE = CROW + 16;              // staged row: codes + scale window
-  static constexpr int NVS = CROW == 128 ? 2 : 3;        // groups of 16 rows in flight per warp
+  static constexpr int NVS = 3;                          // V groups of 16 rows in flight per warp
   static constexpr int VGROUP = 16 * VSTRIDE;
+  // one buffer per warp: its K tile, then its V groups
+  static constexpr int WBUF = ((STAGE_CODE + STAGE_SC > NVS * VGROUP ? STAGE_CODE + STAGE_SC
+                                                                      : NVS * VGROUP) + 127) / 128 * 128;
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
 
 template <int FMT, int D>
 struct Layout {
   using C = Cfg<FMT, D>;
-  static constexpr size_t stage = 0;
-  static constexpr size_t ored = stage + (size_t)C::STAGES * C::STAGE_BYTES;  // float [8][NE][32]
-  static constexpr size_t pkt = ored + (size_t)8 * (D / 16) * 4 * 32 * 4;     // half [8][kPktStride]
+  static constexpr size_t wbuf = 0;                                           // [warps][WBUF]
+  // reduction buffer float [8][NE][32]; before the epilogue it holds the per-lane score
+  // slots (4 float4 per lane per warp)
+  static constexpr size_t ORED = (size_t)8 * (D / 16) * 4 * 32 * 4 > (size_t)kWarps * 4 * 32 * 16
+                                     ? (size_t)8 * (D / 16) * 4 * 32 * 4
+                                     : (size_t)kWarps * 4 * 32 * 16;
+  static constexpr size_t ored = wbuf + (size_t)kWarps * C::WBUF;
+  static constexpr size_t pkt = ored + ORED;                                  // half [8][kPktStride]
   static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;            // u16 [kLmax]
   static constexpr size_t pktg = list + (size_t)kLmax * 2;                    // half [8][kPktStride]
   static constexpr size_t listg = pktg + (size_t)8 * kPktStride * 2;          // u16 [kLmax]
-  static constexpr size_t vst = listg + (size_t)kLmax * 2;                    // [warps][NVS][VGROUP]
-  static constexpr size_t q = vst + (size_t)kConsumerWarps * C::NVS * C::VGROUP;  // float [8][D]
+  static constexpr size_t q = listg + (size_t)kLmax * 2;                      // float [8][D]
   static constexpr size_t corr = q + (size_t)8 * D * 4;                       // float [8][NBLK]
   static constexpr size_t rows = corr + (size_t)8 * C::NBLK * 4;              // int [kMaxTiles]
-  static constexpr size_t stage_row = rows + kMaxTiles * 4;                   // int [STAGES]
-  static constexpr size_t red = stage_row + C::STAGES * 4;                    // float [2][warps][8]
-  static constexpr size_t cnt = red + 2 * kConsumerWarps * 8 * 4;             // int [2][warps] + flags
-  static constexpr size_t bars = (cnt + (2 * kConsumerWarps + 2) * 4 + 7) / 8 * 8;
-  static constexpr size_t nbars = 2 * C::STAGES + kConsumerWarps * C::NVS;    // full, empty, V groups
-  static constexpr size_t prefix = bars + nbars * 8;                          // int [MAX_BATCH + 1]
+  static constexpr size_t red = rows + kMaxTiles * 4;                         // float [2][warps][8]
+  static constexpr size_t cnt = red + 2 * kWarps * 8 * 4;                     // int [2][warps]
+  static constexpr size_t prefix = cnt + 2 * kWarps * 4;                      // int [MAX_BATCH + 1]
   static constexpr size_t total = prefix + (KVQ_MAX_BATCH + 1) * 4;
-  static constexpr size_t alloc = total + 1024;  // slack for aligning the base to 1024
+  static constexpr size_t alloc = total + 128;  // slack for aligning the base to 128
   static_assert(alloc <= 232448, "shared memory");
 };
-
-// Final CTA-wide barrier, reached by the producer warp and by the consumer warps from
-// different code paths: the non-aligned form permits that.
-__device__ __forceinline__ void cta_final_sync() {
-  asm volatile("barrier.sync 0;" ::: "memory");
-}
-
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync %0, %1;" ::"n"(kBarConsumers), "n"(kConsumers) : "memory");
-}
 
 struct Item {
   int b, kvh, split, t0, n_tok;
@@ -398,30 +387,23 @@ __device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
+decode_kernel(const DecodeArgs a) {
   using C = Cfg<FMT, D>;
   using LY = Layout<FMT, D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* stages = smem + LY::stage;
+  uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
   float* ored = reinterpret_cast<float*>(smem + LY::ored);
   __half* pkt = reinterpret_cast<__half*>(smem + LY::pkt);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + LY::list);
   __half* pktg = reinterpret_cast<__half*>(smem + LY::pktg);        // CTA-wide compacted weights
   uint16_t* listg = reinterpret_cast<uint16_t*>(smem + LY::listg);  // CTA-wide kept list
-  uint8_t* vst = smem + LY::vst;
   float* qs = reinterpret_cast<float*>(smem + LY::q);
   float* corr_s = reinterpret_cast<float*>(smem + LY::corr);
   int* item_rows = reinterpret_cast<int*>(smem + LY::rows);
-  int* stage_row = reinterpret_cast<int*>(smem + LY::stage_row);
   float* red_m = reinterpret_cast<float*>(smem + LY::red);
-  float* red_l = red_m + kConsumerWarps * 8;
+  float* red_l = red_m + kWarps * 8;
   int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
-  int* cnt_kept = cnt_skip + kConsumerWarps;
-  int* abort_flag = cnt_skip + 2 * kConsumerWarps;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::bars);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* vbar = empty + C::STAGES;
+  int* cnt_kept = cnt_skip + kWarps;
   int* prefix = reinterpret_cast<int*>(smem + LY::prefix);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -429,6 +411,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   uint32_t* flags = reinterpret_cast<uint32_t*>(a.workspace);
   const int hkv = a.desc.num_kv_heads, G = a.group, P = a.desc.page_size, Ls = a.split_tokens;
   const int B = a.batch, Hq = a.num_q_heads;
+  uint8_t* my_buf = smem + LY::wbuf + (size_t)warp * C::WBUF;
 
   // ---- work list: splits per sequence, exclusive prefix
   for (int b = tid; b < B; b += kThreads) {
@@ -438,16 +421,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
     const int nc = max(0, min(n, cap));
     prefix[b + 1] = (nc + Ls - 1) / Ls;
   }
-  if (tid == 0) {
-    prefix[0] = 0;
-    *abort_flag = 0;
-    for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 4);  // the four warps that consume the tile's four 16-row jobs
-    }
-    for (int i = 0; i < kConsumerWarps * C::NVS; ++i) mbar_init(&vbar[i], 1);
-    fence_mbar_init();
-  }
+  if (tid == 0) prefix[0] = 0;
   __syncthreads();
   if (warp == 0) {
     int run = 0;
@@ -467,50 +441,6 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   const int total_items = prefix[B] * hkv;
   if ((int)blockIdx.x >= total_items) return;
 
-  // ================================================================ producer warp
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      prefetch_tensormap(&tmap_k);
-      const uint8_t* ksc = static_cast<const uint8_t*>(a.k_scales);
-      int pg = 0;
-      for (int k = 0; k < (1 << 30); ++k) {
-        const int it = blockIdx.x + k * gridDim.x;
-        if (it >= total_items) break;
-        const Item I = decode_item(a, prefix, it);
-        const int ntiles = (I.n_tok + kTile - 1) / kTile;
-        for (int t = 0; t < ntiles; ++t, ++pg) {
-          const int stage = pg % C::STAGES, use = pg / C::STAGES;
-          if (use > 0 && !mbar_wait_bounded(&empty[stage], (uint32_t)(use - 1) & 1u)) {
-            set_flag(flags, KVQ_FLAG_TIMEOUT);
-            k = 1 << 30;  // stop producing; consumers time out on the missing tiles
-            break;
-          }
-          uint8_t* dst = stages + (size_t)stage * C::STAGE_BYTES;
-          const int tok0 = I.t0 + t * kTile;
-          const int lp = tok0 / P, off = tok0 - lp * P;
-          const int page = a.page_table ? a.page_table[(size_t)I.b * a.max_pages + lp]
-                                        : I.b * a.max_pages + lp;
-          if (page >= 0 && page < a.desc.num_pages) {
-            const int row0 = (page * hkv + I.kvh) * P + off;
-            stage_row[stage] = row0;
-            mbar_arrive_expect_tx(&full[stage], C::STAGE_CODE + C::STAGE_SC);
-            tma_load_2d(dst, &tmap_k, 0, row0, &full[stage]);
-            bulk_load(dst + C::STAGE_CODE, ksc + (size_t)row0 * C::SROW, C::STAGE_SC, &full[stage]);
-          } else {
-            set_flag(flags, KVQ_FLAG_BAD_PAGE);
-            stage_row[stage] = -1;
-            mbar_arrive(&full[stage]);  // completes the phase with no bytes
-          }
-        }
-      }
-    }
-    // stay resident until every consumer is done: nothing issued here is left unwaited
-    __syncwarp();
-    cta_final_sync();
-    return;
-  }
-
-  // ================================================================ consumer warps
   Lut lut;
   if constexpr (C::kLut) {
 #pragma unroll
@@ -532,6 +462,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   const float qk_scale = a.sm_scale * kLog2e;
   const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
   const __half* qg = static_cast<const __half*>(a.q);
+  const uint8_t* kcodes = static_cast<const uint8_t*>(a.k_codes);
+  const uint8_t* kscales = static_cast<const uint8_t*>(a.k_scales);
   const uint8_t* vcodes = static_cast<const uint8_t*>(a.v_codes);
   const uint8_t* vscales = static_cast<const uint8_t*>(a.v_scales);
   float* ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + kWorkspaceHeader);
@@ -539,18 +471,44 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
   float* ws_m = ws_o + n_part * D;
   float* ws_l = ws_m + n_part;
   const int wslot0 = warp * kWarpSlots;  // this warp's region of the kept list / weights
-  uint8_t* my_vst = vst + (size_t)warp * C::NVS * C::VGROUP;
-  uint64_t* my_vbar = vbar + warp * C::NVS;
   const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;  // this lane's two heads exist
 
-  int g_base = 0;  // K tiles consumed by this CTA before the current unit
-  int vg = 0;      // V groups fetched by this warp so far (mbarrier phase bookkeeping)
+#pragma unroll 1
   for (int k = 0;; ++k) {
     const int it = blockIdx.x + k * gridDim.x;
     if (it >= total_items) break;
     const Item I = decode_item(a, prefix, it);
     const int ntiles = (I.n_tok + kTile - 1) / kTile;
-    const int njobs = 4 * ntiles;
+    const bool has_tile = warp < ntiles;
+
+    // ---- K fetch: this warp's tile (positions 64 w .. 64 w + 63 of the unit)
+    if (has_tile) {
+      const int tok0 = I.t0 + warp * kTile;
+      const int lp = tok0 / P, off = tok0 - lp * P;  // tiles never straddle pages (P % 64 == 0)
+      const int page = a.page_table ? a.page_table[(size_t)I.b * a.max_pages + lp]
+                                    : I.b * a.max_pages + lp;
+      const bool ok = page >= 0 && page < a.desc.num_pages;
+      const int row0 = ok ? (page * hkv + I.kvh) * P + off : -1;
+      if (lane == 0) {
+        item_rows[warp] = row0;
+        if (!ok) set_flag(flags, KVQ_FLAG_BAD_PAGE);
+      }
+      if (ok) {
+        constexpr int CPR = C::CROW / 16;
+        const uint8_t* src = kcodes + (size_t)row0 * C::CROW;
+#pragma unroll
+        for (int i = lane; i < kTile * CPR; i += 32) {
+          const int row = i / CPR, cc = i - row * CPR;
+          const int sc = cc ^ ((row >> C::SWZ_SHIFT) & C::SWZ_MASK);
+          cp_async16(my_buf + row * C::CROW + (sc << 4), src + (size_t)i * 16);
+        }
+        const uint8_t* ssrc = kscales + (size_t)row0 * C::SROW;
+#pragma unroll
+        for (int i = lane; i < C::STAGE_SC / 16; i += 32)
+          cp_async16(my_buf + C::STAGE_CODE + i * 16, ssrc + (size_t)i * 16);
+      }
+    }
+    cp_async_commit();
 
     // ---- query group -> shared (fp32)
     {
@@ -569,7 +527,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         }
       }
     }
-    consumer_sync();
+    __syncthreads();
     if (warp < 8) {
       const int h = warp;
       constexpr int K = D / 32;
@@ -607,19 +565,19 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
       } else {
         // offset contribution per (head, block): sum_d q_d * (offset_d + 8) for q4_0
-        // (offset 1024 on even dims, 64 on odd dims), sum_d q_d * 1152 for q8_0; fp64 sums
+        // (offset 1024 on even dims, 64 on odd dims), sum_d q_d * 1152 for q8_0
 #pragma unroll
         for (int m = 0; m < K; ++m) {
           const int d = 32 * m + lane;
-          const double w = C::kQ8 ? 1152.0 : ((d & 1) ? 72.0 : 1032.0);
-          double v = (double)qs[h * D + d] * w;
+          const float w = C::kQ8 ? 1152.f : ((d & 1) ? 72.f : 1032.f);
+          float v = qs[h * D + d] * w;
 #pragma unroll
           for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) corr_s[h * C::NBLK + m] = (float)v;
+          if (lane == 0) corr_s[h * C::NBLK + m] = v;
         }
       }
     }
-    consumer_sync();
+    __syncthreads();
     uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
 #pragma unroll
     for (int ks = 0; ks < C::KSTEPS; ++ks) {
@@ -644,36 +602,24 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       corr[m][1] = C::kLut ? 0.f : corr_s[(2 * c + 1) * C::NBLK + m];
     }
 
-    // ---- K pass: this warp's 16-row jobs; scores stay in registers
-    float sreg[kJobsPerWarp][4];
+    // ---- K pass: the warp's tile, four 16-row jobs; scores to per-lane shared slots
+    float4* sbuf = reinterpret_cast<float4*>(ored) + (size_t)warp * 4 * 32 + lane;
     float mx0 = -INFINITY, mx1 = -INFINITY;
-    bool ok_all = true;
-#pragma unroll
-    for (int jj = 0; jj < kJobsPerWarp; ++jj) {
-      sreg[jj][0] = sreg[jj][1] = sreg[jj][2] = sreg[jj][3] = -INFINITY;
-      const int j = warp + kConsumerWarps * jj;
-      if (j < njobs && ok_all) {
-        const int t = j >> 2, mt = j & 3;
-        const int g = g_base + t;
-        const int stage = g % C::STAGES;
-        ok_all = __all_sync(0xffffffffu, mbar_wait_bounded(&full[stage], (uint32_t)(g / C::STAGES) & 1u));
-        if (ok_all) {
-          const uint8_t* base = stages + (size_t)stage * C::STAGE_BYTES;
-          const int row0 = 16 * mt + r;
-          float s[4];
-          k_job_scores<FMT, D>(base, base + C::STAGE_CODE, row0, qf, ql, corr, lut, c, s);
-          if (mt == 0 && lane == 0) item_rows[t] = stage_row[stage];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[stage]);
-          const int p0 = 16 * j + r;
-          const bool v0 = p0 < I.n_tok, v1 = p0 + 8 < I.n_tok;
-          sreg[jj][0] = v0 ? s[0] * qk_scale : -INFINITY;
-          sreg[jj][1] = v0 ? s[1] * qk_scale : -INFINITY;
-          sreg[jj][2] = v1 ? s[2] * qk_scale : -INFINITY;
-          sreg[jj][3] = v1 ? s[3] * qk_scale : -INFINITY;
-          mx0 = fmaxf(mx0, fmaxf(sreg[jj][0], sreg[jj][2]));
-          mx1 = fmaxf(mx1, fmaxf(sreg[jj][1], sreg[jj][3]));
-        }
+    cp_async_wait<0>();
+    __syncwarp();
+    if (has_tile) {
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        const int row0 = 16 * mt + r;
+        float s[4];
+        k_job_scores<FMT, D>(my_buf, my_buf + C::STAGE_CODE, row0, qf, ql, corr, lut, c, s);
+        const int p0 = warp * kTile + row0;
+        const bool v0 = p0 < I.n_tok, v1 = p0 + 8 < I.n_tok;
+        const float4 sv = make_float4(v0 ? s[0] * qk_scale : -INFINITY, v0 ? s[1] * qk_scale : -INFINITY,
+                                      v1 ? s[2] * qk_scale : -INFINITY, v1 ? s[3] * qk_scale : -INFINITY);
+        sbuf[mt * 32] = sv;
+        mx0 = fmaxf(mx0, fmaxf(sv.x, sv.z));
+        mx1 = fmaxf(mx1, fmaxf(sv.y, sv.w));
       }
     }
 #pragma unroll
@@ -685,33 +631,27 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       red_m[warp * 8 + 2 * c] = mx0;
       red_m[warp * 8 + 2 * c + 1] = mx1;
     }
-    if (!ok_all && lane == 0) atomicOr(abort_flag, 1);
-    consumer_sync();  // barrier 1: every warp's maxima are in shared memory
-    if (*abort_flag) {
-      if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-      break;  // all consumer warps see the same flag
-    }
-    g_base += ntiles;
+    __syncthreads();  // barrier 1: every warp's maxima are in shared memory
 
-    // ---- weights, skip test, compaction, from the registers (rows r, r+8; heads 2c, 2c+1)
+    // ---- weights, skip test, compaction (rows r, r+8 of each job; heads 2c, 2c+1)
     float mh0 = red_m[2 * c], mh1 = red_m[2 * c + 1];
 #pragma unroll
-    for (int w = 1; w < kConsumerWarps; ++w) {
+    for (int w = 1; w < kWarps; ++w) {
       mh0 = fmaxf(mh0, red_m[w * 8 + 2 * c]);
       mh1 = fmaxf(mh1, red_m[w * 8 + 2 * c + 1]);
     }
     float l0 = 0.f, l1 = 0.f;
     int nkept = 0, nskip = 0;
     const uint32_t below = (1u << (4 * r)) - 1u;
-#pragma unroll
-    for (int jj = 0; jj < kJobsPerWarp; ++jj) {
-      const int j = warp + kConsumerWarps * jj;
-      if (j < njobs) {
-        const int p0 = 16 * j + r;
+    if (has_tile) {
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        const float4 sv = sbuf[mt * 32];
+        const int p0 = warp * kTile + 16 * mt + r;
         const bool va = p0 < I.n_tok, vb = p0 + 8 < I.n_tok;
         const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
-        const float da0 = sreg[jj][0] - mh0, da1 = sreg[jj][1] - mh1;
-        const float db0 = sreg[jj][2] - mh0, db1 = sreg[jj][3] - mh1;
+        const float da0 = sv.x - mh0, da1 = sv.y - mh1;
+        const float db0 = sv.z - mh0, db1 = sv.w - mh1;
         const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
         const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
         l0 += ea0 + eb0;
@@ -752,86 +692,82 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       cnt_skip[warp] = nskip;
       cnt_kept[warp] = nkept;
     }
-    consumer_sync();  // barrier 2: every warp's kept count is known
+    __syncthreads();  // barrier 2: every warp's kept count is known
     // ---- concatenate the warps' lists in warp order (deterministic) into the CTA list
     int gbase = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       const int n = cnt_kept[w];
       gbase += (w < warp) ? n : 0;
       total += n;
     }
-    for (int i = lane; i < nkept; i += 32) listg[gbase + i] = list[wslot0 + i];
-    for (int i = lane; i < 8 * nkept; i += 32) {
-      const int h = i / nkept, sl = i - h * nkept;
-      pktg[h * kPktStride + gbase + sl] = pkt[h * kPktStride + wslot0 + sl];
+    for (int i = lane; i < nkept; i += 32) {
+      listg[gbase + i] = list[wslot0 + i];
+#pragma unroll
+      for (int h = 0; h < 8; ++h) pktg[h * kPktStride + gbase + i] = pkt[h * kPktStride + wslot0 + i];
     }
-    if (warp == kConsumerWarps - 1) {  // zero the padding slots of the last partial group
+    if (warp == kWarps - 1) {  // zero the padding slots of the last partial group
       const int pad = ((total + 15) & ~15) - total;
       for (int i = lane; i < 8 * pad; i += 32)
         pktg[(i / pad) * kPktStride + total + (i % pad)] = __ushort_as_half(0);
     }
-    consumer_sync();  // barrier 3: the CTA list is complete
+    __syncthreads();  // barrier 3: the CTA list is complete
 
     // ---- V pass: kept positions only, 16-row groups dealt round-robin to the warps
     float acc[C::MT][4];
 #pragma unroll
     for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     const int ngroups_all = (total + 15) >> 4;
-    const int ngroups = ngroups_all > warp ? (ngroups_all - warp + kConsumerWarps - 1) / kConsumerWarps : 0;
-    auto issue = [&](int gi) {  // gi: this warp's gi-th group = CTA group warp + 16 gi
-      const int stage = (vg + gi) % C::NVS;
-      uint8_t* grp = my_vst + (size_t)stage * C::VGROUP;
-      const int slot = 16 * (warp + kConsumerWarps * gi) + lane;
-      const bool valid = lane < 16 && slot < total;
-      const int tok = valid ? listg[slot] : 0;
-      const int rb = valid ? item_rows[tok >> 6] : -1;
-      const bool go = valid && rb >= 0;
-      const int nrows = __popc(__ballot_sync(0xffffffffu, go));
-      if (lane == 0) {
-        if (nrows) mbar_arrive_expect_tx(&my_vbar[stage], nrows * (C::CROW + 16));
-        else mbar_arrive(&my_vbar[stage]);
+    const int ngroups = ngroups_all > warp ? (ngroups_all - warp + kWarps - 1) / kWarps : 0;
+    auto issue = [&](int gi) {  // this warp's gi-th group = CTA group warp + 16 gi
+      uint8_t* grp = my_buf + (size_t)(gi % C::NVS) * C::VGROUP;
+      const int s0 = 16 * (warp + kWarps * gi);
+      constexpr int CPR = C::CROW / 16 + 1;  // code chunks + the scale window
+#pragma unroll
+      for (int i = lane; i < 16 * CPR; i += 32) {
+        const int rl = i / CPR, cc = i - rl * CPR;
+        const int slot = s0 + rl;
+        if (slot < total) {
+          const int tok = listg[slot];
+          const int rb = item_rows[tok >> 6];
+          if (rb >= 0) {
+            const size_t row = (size_t)rb + (tok & 63);
+            const uint8_t* src = cc < CPR - 1 ? vcodes + row * C::CROW + cc * 16
+                                              : vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW;
+            cp_async16(grp + rl * C::VSTRIDE + cc * 16, src);
+          }
+        }
       }
-      __syncwarp();
-      if (go) {
-        const size_t row = (size_t)rb + (tok & 63);
-        bulk_load(grp + lane * C::VSTRIDE, vcodes + row * C::CROW, C::CROW, &my_vbar[stage]);
-        bulk_load(grp + lane * C::VSTRIDE + C::CROW,
-                  vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW, 16, &my_vbar[stage]);
-      }
+      cp_async_commit();
     };
 #pragma unroll
-    for (int i = 0; i < C::NVS; ++i)
+    for (int i = 0; i < C::NVS; ++i) {
       if (i < ngroups) issue(i);
-    bool vok = true;
+      else cp_async_commit();
+    }
+#pragma unroll 1
     for (int gi = 0; gi < ngroups; ++gi) {
-      const int stage = (vg + gi) % C::NVS;
-      vok = __all_sync(0xffffffffu,
-                       mbar_wait_bounded(&my_vbar[stage], (uint32_t)((vg + gi) / C::NVS) & 1u));
-      if (!vok) break;
-      const int s0 = 16 * (warp + kConsumerWarps * gi);
-      v_group<FMT, D>(my_vst + (size_t)stage * C::VGROUP, pktg + r * kPktStride + s0, listg + s0,
-                      min(16, total - s0), r, c, lut, acc);
+      cp_async_wait<C::NVS - 1>();
+      __syncwarp();
+      const int s0 = 16 * (warp + kWarps * gi);
+      v_group<FMT, D>(my_buf + (size_t)(gi % C::NVS) * C::VGROUP, pktg + r * kPktStride + s0,
+                      listg + s0, min(16, total - s0), r, c, lut, acc);
       __syncwarp();
       if (gi + C::NVS < ngroups) issue(gi + C::NVS);
+      else cp_async_commit();
     }
-    vg += ngroups;
-    if (!vok && lane == 0) atomicOr(abort_flag, 1);
+    cp_async_wait<0>();
 
     // ---- sum the warps' accumulators and write the unit
     constexpr int NE = C::MT * 4;  // accumulator registers per thread
-    consumer_sync();  // barrier 4: every warp's V accumulation is done
-    if (*abort_flag) {
-      if (tid == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-      break;
-    }
+    __syncthreads();  // barrier 4: every warp's V accumulation is done; score slots free
     if (warp >= 8) {
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) ored[((warp - 8) * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
-    consumer_sync();  // barrier 5
+    __syncthreads();  // barrier 5
     if (warp < 8) {
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt)
@@ -841,10 +777,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
           *p = *p + acc[mt][i];
         }
     }
-    consumer_sync();  // barrier 6
+    __syncthreads();  // barrier 6
     {
       const size_t unit0 = ((size_t)I.b * Hq + (size_t)I.kvh * G) * a.max_splits + I.split;
-      for (int q = tid; q < 32 * NE; q += kConsumers) {
+      for (int q = tid; q < 32 * NE; q += kThreads) {
         const int ln = q & 31, e = q >> 5;
         float v = 0.f;
 #pragma unroll
@@ -858,7 +794,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       if (tid < G) {
         float m = red_m[tid], l = red_l[tid];
 #pragma unroll
-        for (int w = 1; w < kConsumerWarps; ++w) {
+        for (int w = 1; w < kWarps; ++w) {
           m = fmaxf(m, red_m[w * 8 + tid]);
           l += red_l[w * 8 + tid];
         }
@@ -869,7 +805,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
       if (tid == 0 && a.stats) {
         int ns = 0, nk = 0;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) {
+        for (int w = 0; w < kWarps; ++w) {
           ns += cnt_skip[w];
           nk += cnt_kept[w];
         }
@@ -879,46 +815,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap_k, const DecodeArgs a) {
         atomicAdd(&a.stats[3], (unsigned long long)(I.n_tok - nk));
       }
     }
-    // the next unit's first barrier (after its query staging) keeps every buffer read
-    // above ahead of that unit's writes
+    __syncthreads();  // barrier 7: shared buffers free for the next unit
   }
-  cta_final_sync();  // with the producer warp
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 template <int FMT, int D>
 int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
-  using C = Cfg<FMT, D>;
   using LY = Layout<FMT, D>;
-  auto encode = tensor_map_encoder();
-  if (!encode) return KVQ_ERR_CUDA;
-  CUtensorMap tmap;
-  const uint64_t rows = (uint64_t)a.desc.num_pages * a.desc.num_kv_heads * a.desc.page_size;
-  cuuint64_t dims[2] = {(cuuint64_t)C::CROW, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)C::CROW};
-  cuuint32_t box[2] = {(cuuint32_t)C::CROW, (cuuint32_t)kTile};
-  cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle swz = C::CROW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                 : C::CROW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k_codes), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return KVQ_ERR_CUDA;
   auto kern = decode_kernel<FMT, D>;
   // The shared-memory opt-in is set once per device (so that later calls, including
   // ones made while a stream is being captured into a graph, issue no attribute call).
@@ -939,7 +843,7 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   const int64_t units = (int64_t)a.batch * a.desc.num_kv_heads * a.max_splits;
   const int grid = (int)std::min<int64_t>(units, a.num_sms);
   if (grid <= 0) return KVQ_OK;
-  kern<<<grid, kThreads, LY::alloc, stream>>>(tmap, a);
+  kern<<<grid, kThreads, LY::alloc, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -83,6 +83,7 @@ extern "C" {
 #define KVQ_MAX_SPLIT_TOKENS 1024  /* positions per split-KV work unit */
 #define KVQ_MAX_BATCH        1024
 #define KVQ_MAX_SPLITS       4096  /* splits of one sequence: max_seq_len <= 4096 * split length */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)  /* static scratch of kvq_decode_attn_noalloc */
 
 typedef struct kvq_cache_desc {
     int32_t fmt;              /* KVQ_FMT_* */
@@ -173,6 +174,30 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
 int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
                 int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens,
                 const int32_t* seq_lens, float* out, void* stream);
+
+/*
+ * kvq_decode_attn_noalloc -- kvq_decode_attn followed by kvq_combine, for callers that
+ * cannot allocate device memory while decoding (a serving runtime that plans every
+ * buffer up front, a process confined to a fixed memory pool, or code running where
+ * cudaMalloc is not allowed).  The paper has no counterpart: this is packaging.
+ *   The per-split partials live in a library-owned static device array of
+ *   KVQ_NOALLOC_SCRATCH_BYTES (8 MiB); every GPU that loads the library keeps it until
+ *   the process exits.  Nothing is allocated or freed by the call.
+ *   Arguments are those of kvq_decode_attn (no workspace) plus
+ *   out  device fp32 [batch][num_q_heads][head_dim], as written by kvq_combine.
+ *   Returns KVQ_ERR_WORKSPACE when kvq_workspace_size(...) for the request exceeds
+ *   KVQ_NOALLOC_SCRATCH_BYTES.
+ *   The first call on each device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.  All calls share
+ *   the one array and each call clears its fault-flag word first, so calls whose
+ *   execution overlaps on the GPU (different streams, or another thread) race.
+ */
+int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q, int32_t batch,
+                            int32_t num_q_heads, const void* k_codes, const void* k_scales,
+                            const void* v_codes, const void* v_scales, const int32_t* page_table,
+                            int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
+                            float sm_scale, float tau, int32_t split_tokens,
+                            unsigned long long* stats, float* out, void* stream);
 
 /*
  * kvq_lloyd_max_codebook -- the minimum-MSE `levels`-entry scalar codebook for

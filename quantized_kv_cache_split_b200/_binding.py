@@ -36,6 +36,7 @@ KVQ_MAX_GROUP = 8
 KVQ_MAX_SPLIT_TOKENS = 1024
 KVQ_MAX_BATCH = 1024
 KVQ_MAX_SPLITS = 4096
+KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class KvqCacheDesc(ctypes.Structure):
@@ -59,7 +60,7 @@ class KvqError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m quantized_kv_cache_split_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python quantized_kv_cache_split_b200/build.py` "
             "(the CUDA library is required; there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
@@ -75,6 +76,8 @@ def _load():
         "kvq_decode_attn": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32, F32,
                                            I32, P, SZ, P, P]),
         "kvq_combine": (ctypes.c_int, [D, P, I32, I32, I32, I32, P, P, P]),
+        "kvq_decode_attn_noalloc": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32,
+                                                   F32, I32, P, P, P]),
         "kvq_lloyd_max_codebook": (ctypes.c_int, [I32, ctypes.c_double,
                                                   ctypes.POINTER(ctypes.c_uint16)]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -198,3 +201,18 @@ def kvq_lloyd_max_codebook(levels: int = 16, sigma: float = 1.0) -> np.ndarray:
     buf = (ctypes.c_uint16 * levels)()
     _check("kvq_lloyd_max_codebook", _lib.kvq_lloyd_max_codebook(levels, float(sigma), buf))
     return np.frombuffer(bytes(buf), dtype=np.float16).copy()
+
+
+def kvq_decode_attn_noalloc(desc: KvqCacheDesc, q, batch: int, num_q_heads: int, k_codes,
+                            k_scales, v_codes, v_scales, page_table, max_pages: int, seq_lens,
+                            max_seq_len: int, sm_scale: float, tau: float, split_tokens: int, out,
+                            stats=None, stream=None, check: bool = True) -> int:
+    """Decode + merge using the library's static scratch (no device allocation)."""
+    st = _lib.kvq_decode_attn_noalloc(ctypes.byref(desc), _ptr(q), batch, num_q_heads,
+                                      _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                                      _ptr(page_table), max_pages, _ptr(seq_lens), max_seq_len,
+                                      float(sm_scale), float(tau), split_tokens, _ptr(stats),
+                                      _ptr(out), _stream(stream))
+    if check:
+        _check("kvq_decode_attn_noalloc", st)
+    return st

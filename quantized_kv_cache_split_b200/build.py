@@ -1,6 +1,8 @@
 """Build libkvq.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m quantized_kv_cache_split_b200.build [--force] [--checked]
+    python quantized_kv_cache_split_b200/build.py [--force] [--ptxas-info]
+
+(run by path: importing the package loads the library, which this script produces)
 
 The library is plain CUDA C++ with a C ABI; it does not link against PyTorch.
 """

@@ -1,0 +1,66 @@
+// kvq_decode_attn_noalloc: decode attention + merge with a fixed, library-owned scratch.
+//
+// Some callers cannot allocate device memory at decode time: an inference runtime that
+// pre-plans every buffer before serving, a process running under a memory pool that
+// forbids new allocations, or a host that calls in from a context where cudaMalloc is
+// not permitted.  This entry point runs the same split-KV kernel and merge as
+// kvq_decode_attn + kvq_combine, but keeps the per-split partials in a static device
+// array owned by the library, so the caller passes only inputs and outputs.
+#include <mutex>
+
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the scratch array, looked up once per device with that device current.
+// (In host code the symbol name is only a host-side stand-in, never a device address.)
+int scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return KVQ_OK;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q, int32_t batch,
+                                       int32_t num_q_heads, const void* k_codes,
+                                       const void* k_scales, const void* v_codes,
+                                       const void* v_scales, const int32_t* page_table,
+                                       int32_t max_pages, const int32_t* seq_lens,
+                                       int32_t max_seq_len, float sm_scale, float tau,
+                                       int32_t split_tokens, unsigned long long* stats,
+                                       float* out, void* stream) {
+  if (!desc || !out) return KVQ_ERR_INVALID_ARG;
+  const int32_t L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
+  if (L < 0) return L;
+  const size_t need = kvq_workspace_size(batch, num_q_heads, desc->head_dim, max_seq_len, L);
+  if (need == 0 || need > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
+  void* ws = nullptr;
+  int st = scratch_address(&ws);
+  if (st != KVQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the flag word must start at zero for every call (no allocation involved)
+  if (cudaMemsetAsync(ws, 0, kWorkspaceHeader, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  st = kvq_decode_attn(desc, q, batch, num_q_heads, k_codes, k_scales, v_codes, v_scales,
+                       page_table, max_pages, seq_lens, max_seq_len, sm_scale, tau, L, ws, need,
+                       stats, stream);
+  if (st != KVQ_OK) return st;
+  return kvq_combine(desc, ws, batch, num_q_heads, max_seq_len, L, seq_lens, out, stream);
+}

@@ -19,6 +19,12 @@ positions, [0, L), [L, 2L), ...; each split is one flash-decoding work unit:
        position, skipped or not (only V work is skipped);
     3. V pass: position j contributes p_j v_hat_j iff p_j >= tau; otherwise its
        V is neither dequantized nor accumulated.
+Optionally (``share`` > 1) the running maximum that decides the skips is the
+one over a group of ``share`` consecutive splits of the same (sequence, KV head)
+whose K passes have all finished before V work starts: every split of the group
+uses m = max over the group's scores for its weights, its l and its skip test.
+This is still a maximum over already-scored K, so m <= M and the skipped-mass
+bound below holds unchanged.
 Splits are merged by the log-sum-exp rule:
     M = max_s m_s,  out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s.
 With tau = 0 every position is kept and the result equals dense attention.
@@ -65,8 +71,11 @@ def combine(o: np.ndarray, m: np.ndarray, l: np.ndarray) -> np.ndarray:
     return num / den[:, None]
 
 
-def sparse_v_attention(q, k_hat, v_hat, sm_scale, tau, split_len):
+def sparse_v_attention(q, k_hat, v_hat, sm_scale, tau, split_len, share=1):
     """Schedule-exact sparse-V attention for one (sequence, KV head) group.
+
+    ``share``: number of consecutive splits whose K passes share one running
+    maximum for the skip test (1 = each split uses its own).
 
     Returns a dict: out [G, D]; per-split o, m, l; keep [G, N] (bool);
     n_skipped (pairs); v_rows_read / v_rows_skipped (positions); skipped_mass [G]
@@ -80,10 +89,16 @@ def sparse_v_attention(q, k_hat, v_hat, sm_scale, tau, split_len):
     keep = np.zeros((G, N), dtype=bool)
     s_all = np.zeros((G, N))
     os_, ms, ls = [], [], []
-    for a, b in split_bounds(N, split_len):
-        # 1. K pass over the split: scores and the running maximum.
+    bounds = split_bounds(N, split_len)
+    group_max = []
+    for g0 in range(0, len(bounds), share):
+        a0, b0 = bounds[g0][0], bounds[min(g0 + share, len(bounds)) - 1][1]
+        group_max.append(scores(q, k_hat[a0:b0], sm_scale).max(axis=1))
+    for si, (a, b) in enumerate(bounds):
+        # 1. K pass over the split: scores and the running maximum (over the
+        #    split, or over its group of splits when they share it).
         s = scores(q, k_hat[a:b], sm_scale)
-        m = s.max(axis=1)
+        m = group_max[si // share]
         # 2. weights relative to the running maximum; all of them enter l.
         p = np.exp(s - m[:, None])
         l = p.sum(axis=1)
@@ -118,7 +133,7 @@ def sparse_v_attention(q, k_hat, v_hat, sm_scale, tau, split_len):
 
 
 def decode_step(fmt, q16, k16, v16, seq_lens, num_kv_heads, sm_scale, tau, split_len,
-                signs=None, codebook16=None, with_dense=True, groups=None):
+                signs=None, codebook16=None, with_dense=True, groups=None, share=1):
     """Whole decode step on the logical (unpaged) cache.
 
     q16 [B, Hq, D] fp16; k16, v16 [T, Hkv, D] fp16 (sequences concatenated).
@@ -127,6 +142,7 @@ def decode_step(fmt, q16, k16, v16, seq_lens, num_kv_heads, sm_scale, tau, split
     rotated with R = c H diag(s) in fp64) and the output is rotated back with R^T.
 
     ``groups``: optional list of (b, kv_head) to evaluate (others left as NaN).
+    ``share``: splits per shared running maximum (see ``sparse_v_attention``).
     Returns dict with out_sparse [B, Hq, D], out_dense [B, Hq, D] (if asked),
     skipped_mass [B, Hq], vmax [B, Hkv] (max |v_hat|), and summed counters.
     """
@@ -151,7 +167,7 @@ def decode_step(fmt, q16, k16, v16, seq_lens, num_kv_heads, sm_scale, tau, split
         qg = q16[b, h * G:(h + 1) * G].astype(np.float64)
         if fmt == "lut4":
             qg = Q.rotate_f64(qg, signs)
-        r = sparse_v_attention(qg, k_hat, v_hat, sm_scale, tau, split_len)
+        r = sparse_v_attention(qg, k_hat, v_hat, sm_scale, tau, split_len, share)
         o = r["out"]
         if with_dense:
             od, _ = dense_attention(qg, k_hat, v_hat, sm_scale)

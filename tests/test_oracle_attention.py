@@ -200,3 +200,54 @@ def test_decode_step_empty_and_single_position(fmt):
     if fmt == "lut4":
         v1 = Q.unrotate_f64(v1, inp.signs)
     np.testing.assert_allclose(res["out_sparse"][1, 0], v1[0], rtol=1e-12, atol=1e-12)
+
+
+def _keep_brute_force(q, k, scale, tau, split_len, share):
+    """Keep flags by plain loops: position j of split s is kept for head g iff
+    exp(s_gj - m) >= tau, m the maximum over the splits of s's sharing group."""
+    G, N = len(q), len(k)
+    span = split_len * share
+    keep = [[False] * N for _ in range(G)]
+    for g in range(G):
+        s = [sum(float(q[g][d]) * float(k[j][d]) for d in range(len(q[g]))) * scale for j in range(N)]
+        for a in range(0, N, span):
+            m = max(s[a:a + span])
+            for j in range(a, min(a + span, N)):
+                keep[g][j] = math.exp(s[j] - m) >= tau
+    return np.array(keep)
+
+
+@pytest.mark.parametrize("split_len,share", [(8, 1), (8, 3), (5, 4), (16, 100)])
+def test_shared_running_max_keep_set_brute_force(split_len, share):
+    r = _rng(11)
+    q = r.standard_normal((3, 16))
+    k = r.standard_normal((90, 16)) * 3
+    k[[7, 41, 77]] = q.mean(0) * 6  # a few strong keys so groups differ
+    v = r.standard_normal((90, 16))
+    res = A.sparse_v_attention(q, k, v, 0.25, 1e-3, split_len, share)
+    np.testing.assert_array_equal(res["keep"], _keep_brute_force(q, k, 0.25, 1e-3, split_len, share))
+    dense, w = A.dense_attention(q, k, v, 0.25)
+    np.testing.assert_allclose(res["skipped_mass"], (w * ~res["keep"]).sum(1), rtol=1e-10, atol=1e-18)
+    assert (res["skipped_mass"] <= 1e-3 * (~res["keep"]).sum(1) + 1e-15).all()
+    err = np.abs(res["out"] - dense)
+    assert (err <= res["skipped_mass"][:, None] * np.abs(v).max() * (1 + 1e-9) + 1e-14).all()
+
+
+def test_shared_running_max_special_cases():
+    r = _rng(12)
+    q = r.standard_normal((2, 16))
+    k = r.standard_normal((70, 16)) * 3
+    v = r.standard_normal((70, 16))
+    dense, w = A.dense_attention(q, k, v, 0.25)
+    # tau = 0 keeps everything whatever the sharing
+    np.testing.assert_allclose(A.sparse_v_attention(q, k, v, 0.25, 0.0, 9, 4)["out"], dense,
+                               rtol=1e-12, atol=1e-14)
+    # one group covering every split: the skip test uses the final maximum M
+    res = A.sparse_v_attention(q, k, v, 0.25, 1e-2, 9, 8)
+    s = (q @ k.T) * 0.25
+    np.testing.assert_array_equal(res["keep"], np.exp(s - s.max(1, keepdims=True)) >= 1e-2)
+    # nested groups only raise the maximum, so they skip at least as much
+    n1 = A.sparse_v_attention(q, k, v, 0.25, 1e-2, 9, 1)["n_skipped"]
+    n2 = A.sparse_v_attention(q, k, v, 0.25, 1e-2, 9, 2)["n_skipped"]
+    n4 = A.sparse_v_attention(q, k, v, 0.25, 1e-2, 9, 4)["n_skipped"]
+    assert n1 <= n2 <= n4 <= res["n_skipped"]

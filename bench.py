@@ -5,8 +5,9 @@ sparse V dequantization, on B200.
                     [--workload gqa_32k_q4] [--tau 1e-6]
 
 One step = the whole decode-attention hot path for one decode token of every
-sequence in the workload: split-KV decode kernel (K tiles -> scores -> running
-max -> skip decision -> kept V only) + log-sum-exp combine.  Inputs are resident
+sequence in the workload: one split-KV decode launch (K tiles -> scores -> running
+max -> skip decision -> kept V only -> cluster merge -> log-sum-exp merge of the
+partials by the last cluster of each (sequence, KV head)).  Inputs are resident
 in HBM; the cache is replicated into enough copies that successive steps rotate
 through more than 3x the L2 size, so every step reads HBM.  Prints one JSON line.
 
@@ -195,19 +196,29 @@ class Replicas:
         self.pt = None if inp.page_table is None else torch.from_numpy(inp.page_table).to(device)
         self.max_seq = int(inp.seq_lens.max())
         self.B, self.Hq, self.D = wl.batch, wl.num_q_heads, D
+        # the schedule: L positions per split; the shared-maximum option runs clusters of
+        # CS splits (its own L and CS)
         self.L = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, 0)
-        self.ws_bytes = K.kvq_workspace_size(self.B, self.Hq, D, self.max_seq, self.L)
+        self.L_sh = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, 0,
+                                        K.KVQ_OPT_SHARED_MAX)
+        self.CS_sh = K.kvq_resolve_cluster(first.desc, self.B, self.Hq, self.max_seq, 0,
+                                           K.KVQ_OPT_SHARED_MAX)
+        self.ws_bytes = max(K.kvq_workspace_size(self.B, self.Hq, D, self.max_seq, L)
+                            for L in (self.L, self.L_sh))
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
         K.kvq_workspace_init(self.ws, self.ws_bytes)
         self.out = torch.empty((self.B, self.Hq, D), dtype=torch.float32, device=device)
         self.sm = float(np.float32(1.0 / math.sqrt(D)))
 
-    def decode(self, i, tau, stats=None):
+    def decode(self, i, tau, stats=None, shared_max=False, fused=True):
+        """One decode step on cache copy i % R; ``fused``: the merge runs in the same
+        kernel and writes ``self.out``."""
         import quantized_kv_cache_split_b200 as K
         c = self.caches[i % self.R]
         K.kvq_decode_attn(c.desc, self.q, self.B, self.Hq, c.k_codes, c.k_scales, c.v_codes,
                           c.v_scales, self.pt, self.inp.max_pages, self.seq, self.max_seq, self.sm,
-                          tau, self.L, self.ws, self.ws_bytes, stats)
+                          tau, self.L_sh if shared_max else self.L, self.ws, self.ws_bytes, stats,
+                          self.out if fused else None, K.KVQ_OPT_SHARED_MAX if shared_max else 0)
 
     def combine(self, i):
         import quantized_kv_cache_split_b200 as K
@@ -269,9 +280,10 @@ def time_steps(runner, steps, warmup, world, sampler=None):
     return start.elapsed_time(end)
 
 
-def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_splits_total: int):
-    """HBM bytes one decode launch must move: all K rows, the kept V rows,
-    Q, the page table, and the partials written."""
+def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int):
+    """HBM bytes one fused decode launch must move: every K row, the kept V rows, Q,
+    the page table, the partials (one per cluster of splits, written once and read
+    once by the in-kernel merge) and the output."""
     import quantized_kv_cache_split_b200 as K
     wl = rep.wl
     row = K.kvq_code_row_bytes(wl.fmt, wl.head_dim) + 2 * K.kvq_scale_row_count(wl.fmt, wl.head_dim)
@@ -281,48 +293,53 @@ def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_splits_total: int):
     q_bytes = wl.batch * wl.num_q_heads * wl.head_dim * 2
     pt_bytes = 0 if rep.inp.page_table is None else sum(
         (int(n) + rep.inp.page_size - 1) // rep.inp.page_size for n in rep.inp.seq_lens) * 4
-    part_bytes = n_splits_total * wl.group * (wl.head_dim + 2) * 4
-    return k_bytes + v_bytes + q_bytes + pt_bytes + part_bytes
+    part_bytes = 2 * n_partials * wl.group * (wl.head_dim + 2) * 4
+    out_bytes = wl.batch * wl.num_q_heads * wl.head_dim * 4
+    return k_bytes + v_bytes + q_bytes + pt_bytes + part_bytes + out_bytes
 
 
 def gpu_arm(args, world, rank, local):
     import torch
-    import quantized_kv_cache_split_b200 as K
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
     wl = W.WORKLOADS[args.workload]
     inp = W.generate(wl)
     rep = Replicas(wl, inp, device, 3 * L2_BYTES)
-    n_splits_total = sum(wl.num_kv_heads * ((int(n) + rep.L - 1) // rep.L) for n in inp.seq_lens)
+    def n_partials(L, CS):
+        return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
 
-    def counters(tau):
+    def counters(tau, shared):
         st = torch.zeros(4, dtype=torch.int64, device=device)
-        rep.decode(0, tau, st)
+        rep.decode(0, tau, st, shared_max=shared)
         torch.cuda.synchronize()
         return [int(x) for x in st.cpu()]
 
     res = {}
     hbm_peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
-    for tag, tau in (("sparse", args.tau), ("dense", 0.0)):
-        st = counters(tau)
-        step = GraphRunner(lambda i: (rep.decode(i, tau), rep.combine(i)), rep.R)
-        dec = GraphRunner(lambda i: rep.decode(i, tau), rep.R)
+    variants = (("sparse", args.tau, False), ("dense", 0.0, False), ("sparse_shared_max", args.tau, True))
+    for tag, tau, shared in variants:
+        st = counters(tau, shared)
+        step = GraphRunner(lambda i: rep.decode(i, tau, shared_max=shared), rep.R)
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)
-        ms_dec = reduce_max(time_steps(dec, args.steps, args.warmup, world), world, device)
-        abytes = algorithmic_bytes(rep, st[2], n_splits_total)
-        us_launch = ms_dec * 1e3 / args.steps
+        abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if shared
+                                   else n_partials(rep.L, 1))
+        us_launch = ms_step * 1e3 / args.steps
         achieved = abytes / (us_launch * 1e-6) / 1e9
-        res[tag] = dict(tau=tau, ms_per_step=ms_step / args.steps,
+        res[tag] = dict(tau=tau, shared_max=shared, ms_per_step=ms_step / args.steps,
                         us_per_token=ms_step * 1e3 / args.steps / (wl.batch * world),
-                        decode_us_per_launch=us_launch, algorithmic_bytes=abytes,
+                        us_per_launch=us_launch, algorithmic_bytes=abytes,
                         achieved_gbs=achieved, frac=achieved / hbm_peak,
                         skipped_pair_frac=st[1] / max(st[0], 1),
                         v_rows_read=st[2], v_rows_skipped=st[3],
                         traffic=traffic_from_profile(f"{args.workload}:{tag}"))
-        del step, dec
+        del step
+    # the two-launch path (partials, then kvq_combine) for comparison
+    two = GraphRunner(lambda i: (rep.decode(i, args.tau, fused=False), rep.combine(i)), rep.R)
+    ms_two = reduce_max(time_steps(two, args.steps, args.warmup, world), world, device)
+    del two
     e2e = None if args.skip_e2e else e2e_arm(args, rep, wl, inp, device, world)
     sp = res["sparse"]
     line = {
@@ -334,20 +351,24 @@ def gpu_arm(args, world, rank, local):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
+                   "shared_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
                    "l2": f"inputs rotate over {rep.R} cache copies "
                          f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": "kvq_decode_attn + kvq_combine (CUDA graph)"},
+                   "step": "one kvq_decode_attn launch with the in-kernel merge (CUDA graph)"},
         "roofline": {"bound": "hbm", "achieved": round(sp["achieved_gbs"], 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(sp["frac"], 4),
                      "traffic": sp["traffic"], "peak_kind": peak_kind,
-                     "kernel": "kvq decode_kernel<q4_0,128>" if wl.fmt == "q4_0" else f"decode_kernel<{wl.fmt}>",
+                     "kernel": f"decode_kernel<{wl.fmt},{wl.head_dim}>",
                      "algorithmic_bytes_per_launch": sp["algorithmic_bytes"],
-                     "us_per_launch": round(sp["decode_us_per_launch"], 3)},
+                     "us_per_launch": round(sp["us_per_launch"], 3)},
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": args.steps,
         "dense": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res["dense"].items()},
         "sparse": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in sp.items()},
+        "sparse_shared_max": {k: (round(v, 6) if isinstance(v, float) else v)
+                              for k, v in res["sparse_shared_max"].items()},
+        "two_launch_us_per_token": round(ms_two * 1e3 / args.steps / (wl.batch * world), 4),
         "clocks": sampler.report(),
     }
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
@@ -363,7 +384,8 @@ def gpu_arm(args, world, rank, local):
 def e2e_arm(args, rep, wl, inp, device, world):
     """Same metric through the public API with host buffers: every step copies the new
     token's q, k, v from pinned host memory, appends k/v to the cache (kvq_quantize),
-    runs decode + combine, and reads the output back to pinned host memory."""
+    runs the decode (with its in-kernel merge), and reads the output back to pinned host
+    memory."""
     import torch
     B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     h_q = torch.from_numpy(inp.q).pin_memory()
@@ -400,7 +422,8 @@ def e2e_arm(args, rep, wl, inp, device, world):
     bo = h_out.numel() * 4
     return {"value": round(el * 1e6 / args.steps / (B * world), 3), "unit": UNIT,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-            "how": "eager public API per step: H2D(q,k,v) + QuantizedKVCache.write + .attention + D2H(out)"}
+            "how": "eager public API per step: H2D(q,k,v) + QuantizedKVCache.write + .attention + D2H(out)",
+            "gpu_launches_per_step": 3}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)

@@ -73,6 +73,9 @@ extern "C" {
 #define KVQ_FMT_Q4_0  1
 #define KVQ_FMT_LUT4  2
 
+/* Option bits of kvq_decode_attn. */
+#define KVQ_OPT_SHARED_MAX 1u  /* the splits of one cluster share one running maximum (below) */
+
 /* Device flag bits (kvq_read_device_flags). */
 #define KVQ_FLAG_BAD_PAGE     1u  /* a page-table entry outside [0, num_pages) */
 #define KVQ_FLAG_BAD_SEQLEN   2u  /* seq_len < 0, > max_seq_len or > max_pages*page_size */
@@ -114,45 +117,68 @@ int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
                  const int32_t* slots, void* codes, void* scales, void* stream);
 
 /*
- * kvq_resolve_split -- the split length (positions per split-KV work unit) that
- * kvq_decode_attn and kvq_combine use for a request.  split_tokens > 0 is
- * rounded up to a multiple of 64 and capped at KVQ_MAX_SPLIT_TOKENS;
- * split_tokens == 0 picks one from the problem size and the device's SM count
- * (about one work unit per SM).  Returns the length (> 0) or a KVQ_ERR_* code.
- * Sequence b is cut into splits [k*L, min((k+1)*L, seq_len_b)).
+ * kvq_resolve_split -- the split length L (positions per split-KV work unit) that
+ * kvq_decode_attn and kvq_combine use for a request (same split_tokens and
+ * options).  split_tokens > 0 is capped at KVQ_MAX_SPLIT_TOKENS and rounded up to a
+ * multiple of 64; split_tokens == 0 picks one from the problem size and how many
+ * CTAs (or CTA clusters) of the decode kernel fit on the current device (about one
+ * split per CTA slot).
+ * Returns L (> 0) or a KVQ_ERR_* code.
+ * Sequence b is cut into splits [k*L, min((k+1)*L, seq_len_b)), k = 0, 1, ...
  */
 int32_t kvq_resolve_split(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
-                          int32_t max_seq_len, int32_t split_tokens);
+                          int32_t max_seq_len, int32_t split_tokens, uint32_t options);
+
+/*
+ * kvq_resolve_cluster -- CS, the number of consecutive splits of one (sequence, KV
+ * head) that one thread-block cluster processes together (same arguments as
+ * kvq_resolve_split).  CS = 1 without KVQ_OPT_SHARED_MAX; with it CS is 2 or 4
+ * (when sequences are long enough), splits kCS .. kCS + CS - 1 form cluster group k,
+ * and the CTAs of a group share one running maximum and merge their partials on
+ * chip, so the workspace holds one partial per group.
+ */
+int32_t kvq_resolve_cluster(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                            int32_t max_seq_len, int32_t split_tokens, uint32_t options);
 
 /* Workspace bytes for a resolved split length L (> 0). */
 size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                           int32_t max_seq_len, int32_t split_tokens);
 
-/* Zero the workspace's device flag word (call once after allocating it). */
+/* Zero the workspace (its device flag word and the merge counters); call once after
+ * allocating it.  A workspace whose call to kvq_decode_attn completed is ready for
+ * the next call without another init. */
 int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronize `stream` and read the device flag word (KVQ_FLAG_* bits) into *flags (host). */
 int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
 
 /*
- * kvq_decode_attn -- split-KV decode attention with sparse V, writing per-split
- * partials (unnormalized o, running max m, denominator l) into the workspace.
- *   q            device fp16 [batch][num_q_heads][head_dim]
+ * kvq_decode_attn -- split-KV decode attention with sparse V.
+ *   q            device fp16 [batch][num_q_heads][head_dim], 16-byte aligned
  *   k_codes, k_scales, v_codes, v_scales   device planes (layout above), 16-byte aligned
  *   page_table   device int32 [batch][max_pages] (NULL: sequence b uses pages
  *                b*max_pages .. b*max_pages + max_pages - 1)
  *   seq_lens     device int32 [batch], each in [0, min(max_seq_len, max_pages*page_size)]
  *   sm_scale     score scale (1/sqrt(head_dim) for standard attention)
  *   tau          skip threshold, >= 0.  Position j of split s is skipped for
- *                query head h when exp(s_hj - m_hs) < tau, with m_hs the running
- *                maximum after all K tiles of the split are folded in; tau = 0
- *                keeps everything (dense attention).  Skipped positions still
- *                count in the softmax denominator.
+ *                query head h when exp(s_hj - m_hs) < tau, where m_hs is the running
+ *                maximum once all K tiles of the split are folded in (with
+ *                KVQ_OPT_SHARED_MAX: of all splits of its cluster group, see
+ *                kvq_resolve_cluster).  tau = 0 keeps everything (dense attention).
+ *                Skipped positions still count in the softmax denominator.
  *   split_tokens as for kvq_resolve_split (0 = auto)
+ *   options      0 or KVQ_OPT_SHARED_MAX; other bits are an error
+ *   workspace    device, kvq_workspace_size(...) bytes, 16-byte aligned, initialized
+ *                once with kvq_workspace_init.  Receives one partial (unnormalized o,
+ *                running maximum m, denominator l) per cluster group.
  *   stats        device uint64 [4] or NULL; ADDED to (caller zeroes):
  *                [0] (position, query head) pairs scored, [1] pairs skipped,
  *                [2] V rows read (positions kept by any head of the group),
  *                [3] V rows skipped
+ *   out          device fp32 [batch][num_q_heads][head_dim], 16-byte aligned, or NULL.  When given, the
+ *                same kernel also merges the partials (as kvq_combine does: the last
+ *                cluster to finish a (sequence, KV head) merges it) and writes the
+ *                output; calls that share a workspace must not overlap on the GPU.
  * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
  * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.
  */
@@ -160,43 +186,44 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
                     int32_t num_q_heads, const void* k_codes, const void* k_scales,
                     const void* v_codes, const void* v_scales, const int32_t* page_table,
                     int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
-                    float sm_scale, float tau, int32_t split_tokens, void* workspace,
-                    size_t workspace_bytes, unsigned long long* stats, void* stream);
+                    float sm_scale, float tau, int32_t split_tokens, uint32_t options,
+                    void* workspace, size_t workspace_bytes, unsigned long long* stats,
+                    float* out, void* stream);
 
 /*
  * kvq_combine -- log-sum-exp merge of the partials of kvq_decode_attn (same
- * batch, num_q_heads, max_seq_len, split_tokens, seq_lens and workspace):
+ * batch, num_q_heads, max_seq_len, split_tokens, options, seq_lens and workspace), for callers
+ * that passed no output pointer to it (or that merge partials from elsewhere):
  *   M = max_s m_s,  out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s,
  * rotated back to the caller's basis for lut4.
  *   out  device fp32 [batch][num_q_heads][head_dim]; a sequence of length 0
  *        gets zeros.
  */
 int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
-                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens,
+                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens, uint32_t options,
                 const int32_t* seq_lens, float* out, void* stream);
 
 /*
- * kvq_decode_attn_noalloc -- kvq_decode_attn followed by kvq_combine, for callers that
+ * kvq_decode_attn_noalloc -- kvq_decode_attn with an output pointer, for callers that
  * cannot allocate device memory while decoding (a serving runtime that plans every
  * buffer up front, a process confined to a fixed memory pool, or code running where
  * cudaMalloc is not allowed).  The paper has no counterpart: this is packaging.
  *   The per-split partials live in a library-owned static device array of
  *   KVQ_NOALLOC_SCRATCH_BYTES (8 MiB); every GPU that loads the library keeps it until
  *   the process exits.  Nothing is allocated or freed by the call.
- *   Arguments are those of kvq_decode_attn (no workspace) plus
- *   out  device fp32 [batch][num_q_heads][head_dim], as written by kvq_combine.
+ *   Arguments are those of kvq_decode_attn without the workspace; `out` is required.
  *   Returns KVQ_ERR_WORKSPACE when kvq_workspace_size(...) for the request exceeds
  *   KVQ_NOALLOC_SCRATCH_BYTES.
  *   The first call on each device looks up the array's device address (with that
  *   device current); make that first call before any stream capture.  All calls share
- *   the one array and each call clears its fault-flag word first, so calls whose
+ *   the one array and each call clears its fault-flag word and merge counters first, so calls whose
  *   execution overlaps on the GPU (different streams, or another thread) race.
  */
 int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q, int32_t batch,
                             int32_t num_q_heads, const void* k_codes, const void* k_scales,
                             const void* v_codes, const void* v_scales, const int32_t* page_table,
                             int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
-                            float sm_scale, float tau, int32_t split_tokens,
+                            float sm_scale, float tau, int32_t split_tokens, uint32_t options,
                             unsigned long long* stats, float* out, void* stream);
 
 /*

@@ -28,6 +28,8 @@ KVQ_FMT_Q4_0 = 1
 KVQ_FMT_LUT4 = 2
 FORMATS = {"q8_0": KVQ_FMT_Q8_0, "q4_0": KVQ_FMT_Q4_0, "lut4": KVQ_FMT_LUT4}
 
+KVQ_OPT_SHARED_MAX = 1
+
 KVQ_FLAG_BAD_PAGE = 1
 KVQ_FLAG_BAD_SEQLEN = 2
 KVQ_FLAG_TIMEOUT = 4
@@ -64,20 +66,22 @@ def _load():
             "(the CUDA library is required; there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    U32 = ctypes.c_uint32
     D = ctypes.POINTER(KvqCacheDesc)
     sig = {
         "kvq_code_row_bytes": (SZ, [I32, I32]),
         "kvq_scale_row_count": (SZ, [I32, I32]),
         "kvq_quantize": (ctypes.c_int, [D, P, I32, P, P, P, P]),
-        "kvq_resolve_split": (I32, [D, I32, I32, I32, I32]),
+        "kvq_resolve_split": (I32, [D, I32, I32, I32, I32, U32]),
+        "kvq_resolve_cluster": (I32, [D, I32, I32, I32, I32, U32]),
         "kvq_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
         "kvq_workspace_init": (ctypes.c_int, [P, SZ, P]),
         "kvq_read_device_flags": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
         "kvq_decode_attn": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32, F32,
-                                           I32, P, SZ, P, P]),
-        "kvq_combine": (ctypes.c_int, [D, P, I32, I32, I32, I32, P, P, P]),
+                                           I32, U32, P, SZ, P, P, P]),
+        "kvq_combine": (ctypes.c_int, [D, P, I32, I32, I32, I32, U32, P, P, P]),
         "kvq_decode_attn_noalloc": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32,
-                                                   F32, I32, P, P, P]),
+                                                   F32, I32, U32, P, P, P]),
         "kvq_lloyd_max_codebook": (ctypes.c_int, [I32, ctypes.c_double,
                                                   ctypes.POINTER(ctypes.c_uint16)]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -151,10 +155,20 @@ def kvq_quantize(desc: KvqCacheDesc, x, n_tokens: int, slots, codes, scales, str
 
 
 def kvq_resolve_split(desc: KvqCacheDesc, batch: int, num_q_heads: int, max_seq_len: int,
-                      split_tokens: int = 0, check: bool = True) -> int:
-    v = _lib.kvq_resolve_split(ctypes.byref(desc), batch, num_q_heads, max_seq_len, split_tokens)
+                      split_tokens: int = 0, options: int = 0, check: bool = True) -> int:
+    v = _lib.kvq_resolve_split(ctypes.byref(desc), batch, num_q_heads, max_seq_len, split_tokens,
+                               int(options))
     if check and v < 0:
         raise KvqError("kvq_resolve_split", v)
+    return v
+
+
+def kvq_resolve_cluster(desc: KvqCacheDesc, batch: int, num_q_heads: int, max_seq_len: int,
+                        split_tokens: int = 0, options: int = 0, check: bool = True) -> int:
+    v = _lib.kvq_resolve_cluster(ctypes.byref(desc), batch, num_q_heads, max_seq_len, split_tokens,
+                                 int(options))
+    if check and v < 0:
+        raise KvqError("kvq_resolve_cluster", v)
     return v
 
 
@@ -177,21 +191,22 @@ def kvq_read_device_flags(workspace, stream=None) -> int:
 def kvq_decode_attn(desc: KvqCacheDesc, q, batch: int, num_q_heads: int, k_codes, k_scales,
                     v_codes, v_scales, page_table, max_pages: int, seq_lens, max_seq_len: int,
                     sm_scale: float, tau: float, split_tokens: int, workspace, workspace_bytes: int,
-                    stats=None, stream=None, check: bool = True) -> int:
+                    stats=None, out=None, options: int = 0, stream=None, check: bool = True) -> int:
     st = _lib.kvq_decode_attn(ctypes.byref(desc), _ptr(q), batch, num_q_heads, _ptr(k_codes),
                               _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), _ptr(page_table),
                               max_pages, _ptr(seq_lens), max_seq_len, float(sm_scale), float(tau),
-                              split_tokens, _ptr(workspace), workspace_bytes, _ptr(stats),
-                              _stream(stream))
+                              split_tokens, int(options), _ptr(workspace), workspace_bytes,
+                              _ptr(stats), _ptr(out), _stream(stream))
     if check:
         _check("kvq_decode_attn", st)
     return st
 
 
 def kvq_combine(desc: KvqCacheDesc, workspace, batch: int, num_q_heads: int, max_seq_len: int,
-                split_tokens: int, seq_lens, out, stream=None, check: bool = True) -> int:
+                split_tokens: int, seq_lens, out, options: int = 0, stream=None,
+                check: bool = True) -> int:
     st = _lib.kvq_combine(ctypes.byref(desc), _ptr(workspace), batch, num_q_heads, max_seq_len,
-                          split_tokens, _ptr(seq_lens), _ptr(out), _stream(stream))
+                          split_tokens, int(options), _ptr(seq_lens), _ptr(out), _stream(stream))
     if check:
         _check("kvq_combine", st)
     return st
@@ -206,13 +221,13 @@ def kvq_lloyd_max_codebook(levels: int = 16, sigma: float = 1.0) -> np.ndarray:
 def kvq_decode_attn_noalloc(desc: KvqCacheDesc, q, batch: int, num_q_heads: int, k_codes,
                             k_scales, v_codes, v_scales, page_table, max_pages: int, seq_lens,
                             max_seq_len: int, sm_scale: float, tau: float, split_tokens: int, out,
-                            stats=None, stream=None, check: bool = True) -> int:
+                            stats=None, options: int = 0, stream=None, check: bool = True) -> int:
     """Decode + merge using the library's static scratch (no device allocation)."""
     st = _lib.kvq_decode_attn_noalloc(ctypes.byref(desc), _ptr(q), batch, num_q_heads,
                                       _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
                                       _ptr(page_table), max_pages, _ptr(seq_lens), max_seq_len,
-                                      float(sm_scale), float(tau), split_tokens, _ptr(stats),
-                                      _ptr(out), _stream(stream))
+                                      float(sm_scale), float(tau), split_tokens, int(options),
+                                      _ptr(stats), _ptr(out), _stream(stream))
     if check:
         _check("kvq_decode_attn_noalloc", st)
     return st

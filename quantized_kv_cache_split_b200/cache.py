@@ -65,30 +65,41 @@ class QuantizedKVCache:
         kb.kvq_quantize(self.desc, v, n, slots, self.v_codes, self.v_scales, stream)
 
     # ---------------------------------------------------------------- decode
-    def workspace(self, batch: int, num_q_heads: int, max_seq_len: int, split_tokens: int):
-        L = kb.kvq_resolve_split(self.desc, batch, num_q_heads, max_seq_len, split_tokens)
+    def workspace(self, batch: int, num_q_heads: int, max_seq_len: int, split_tokens: int,
+                  options: int = 0):
+        L = kb.kvq_resolve_split(self.desc, batch, num_q_heads, max_seq_len, split_tokens, options)
         nbytes = kb.kvq_workspace_size(batch, num_q_heads, self.head_dim, max_seq_len, L)
+        key = (batch, num_q_heads)
         if self._ws is None or self._ws.numel() < nbytes:
             self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-            kb.kvq_workspace_init(self._ws, nbytes)
+            self._ws_key = None
+        if self._ws_key != key:  # the merge counters move with (batch, heads): zero them
+            kb.kvq_workspace_init(self._ws, self._ws.numel())
+            self._ws_key = key
         return self._ws, nbytes, L
 
     def attention(self, q: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
                   page_table: Optional[torch.Tensor] = None, max_pages: int = 1,
                   tau: float = 1e-6, sm_scale: Optional[float] = None, split_tokens: int = 0,
                   out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-                  stream=None) -> torch.Tensor:
-        """Decode attention of q [batch, num_q_heads, head_dim] (fp16) -> fp32 output."""
+                  shared_max: bool = False, fused: bool = True, stream=None) -> torch.Tensor:
+        """Decode attention of q [batch, num_q_heads, head_dim] (fp16) -> fp32 output.
+
+        ``fused``: merge the split partials inside the decode kernel (one launch);
+        otherwise kvq_combine merges them in a second launch.  ``shared_max``: the
+        splits of a cluster share one running maximum for the skip test."""
         B, Hq, D = q.shape
         if sm_scale is None:
             sm_scale = 1.0 / math.sqrt(D)
-        ws, nbytes, L = self.workspace(B, Hq, max_seq_len, split_tokens)
+        opts = kb.KVQ_OPT_SHARED_MAX if shared_max else 0
+        ws, nbytes, L = self.workspace(B, Hq, max_seq_len, split_tokens, opts)
         if out is None:
             out = torch.empty((B, Hq, D), dtype=torch.float32, device=self.device)
         kb.kvq_decode_attn(self.desc, q, B, Hq, self.k_codes, self.k_scales, self.v_codes,
                            self.v_scales, page_table, max_pages, seq_lens, max_seq_len, sm_scale,
-                           tau, L, ws, nbytes, stats, stream)
-        kb.kvq_combine(self.desc, ws, B, Hq, max_seq_len, L, seq_lens, out, stream)
+                           tau, L, ws, nbytes, stats, out if fused else None, opts, stream)
+        if not fused:
+            kb.kvq_combine(self.desc, ws, B, Hq, max_seq_len, L, seq_lens, out, opts, stream)
         return out
 
     def device_flags(self) -> int:

@@ -46,11 +46,63 @@ int check_desc(const kvq_cache_desc* d) {
   if ((int64_t)d->num_pages * d->num_kv_heads * d->page_size > 0x7fffffffLL)
     return KVQ_ERR_UNSUPPORTED;  // rows are addressed with 32-bit indices
   if (d->fmt == KVQ_FMT_LUT4 && (!d->codebook || !d->signs)) return KVQ_ERR_INVALID_ARG;
+  if (d->fmt == KVQ_FMT_LUT4 && (reinterpret_cast<uintptr_t>(d->signs) & 7u)) return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
 
 int max_splits_for(int max_seq_len, int split_tokens) {
   return (max_seq_len + split_tokens - 1) / split_tokens;
+}
+
+int cluster_for(int max_splits) { return max_splits >= 4 ? 4 : max_splits >= 2 ? 2 : 1; }
+
+// Split length L of a request (the device is queried only when split_tokens == 0).
+int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, int max_seq_len,
+                      int split_tokens, uint32_t options, int* L_out) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (batch < 0 || num_q_heads < 1 || max_seq_len < 0 || split_tokens < 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (options & ~KVQ_OPT_SHARED_MAX) return KVQ_ERR_INVALID_ARG;
+  int L;
+  if (split_tokens > 0) {
+    L = std::min(split_tokens, KVQ_MAX_SPLIT_TOKENS);
+  } else {
+    // about one split per CTA slot of the device if every sequence were max_seq_len
+    // long (clusters of 4 CTAs when the splits share their running maximum)
+    const int64_t pairs = (int64_t)std::max(batch, 1) * desc->num_kv_heads;
+    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode_cluster_capacity(desc->fmt, desc->head_dim, 4) : 0;
+    int64_t ctas_per_pair;  // splits of one (sequence, KV head) that run at once
+    if (cap4 > 0) {
+      ctas_per_pair = 4 * std::max<int64_t>(1, cap4 / pairs);
+    } else {
+      const int cap1 = decode_cluster_capacity(desc->fmt, desc->head_dim, 1);
+      if (cap1 <= 0) return KVQ_ERR_CUDA;
+      ctas_per_pair = std::max<int64_t>(1, cap1 / pairs);
+    }
+    L = (int)std::min<int64_t>((std::max(max_seq_len, 1) + ctas_per_pair - 1) / ctas_per_pair,
+                               KVQ_MAX_SPLIT_TOKENS);
+  }
+  L = (L + kTile - 1) / kTile * kTile;
+  *L_out = std::max(kTile, std::min(L, KVQ_MAX_SPLIT_TOKENS));
+  return KVQ_OK;
+}
+
+// Splits per thread-block cluster: 1 unless the splits share their running maximum;
+// then 4 when a sequence can have 4 or more splits, else 2 (smaller when the device
+// cannot hold such clusters).  Also the clusters that fit on the device at once.
+int resolve_cluster(const kvq_cache_desc* desc, int max_seq_len, int L, uint32_t options,
+                    int* cs_out, int* cap_out) {
+  int CS = (options & KVQ_OPT_SHARED_MAX) ? cluster_for(max_splits_for(std::max(max_seq_len, 1), L)) : 1;
+  for (; CS >= 1; CS >>= 1) {
+    const int cap = decode_cluster_capacity(desc->fmt, desc->head_dim, CS);
+    if (cap > 0) {
+      *cs_out = CS;
+      *cap_out = cap;
+      return KVQ_OK;
+    }
+  }
+  return KVQ_ERR_CUDA;
 }
 
 }  // namespace
@@ -90,36 +142,32 @@ int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
 }
 
 int32_t kvq_resolve_split(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
-                          int32_t max_seq_len, int32_t split_tokens) {
-  int st = check_desc(desc);
+                          int32_t max_seq_len, int32_t split_tokens, uint32_t options) {
+  int L = 0;
+  const int st = resolve_split_len(desc, batch, num_q_heads, max_seq_len, split_tokens, options, &L);
+  return st != KVQ_OK ? st : L;
+}
+
+int32_t kvq_resolve_cluster(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                            int32_t max_seq_len, int32_t split_tokens, uint32_t options) {
+  int L = 0, CS = 0, cap = 0;
+  int st = resolve_split_len(desc, batch, num_q_heads, max_seq_len, split_tokens, options, &L);
   if (st != KVQ_OK) return st;
-  if (batch < 0 || num_q_heads < 1 || max_seq_len < 0 || split_tokens < 0)
-    return KVQ_ERR_INVALID_ARG;
-  int L;
-  if (split_tokens > 0) {
-    L = split_tokens;
-  } else {
-    const int sms = device_sm_count();
-    if (sms <= 0) return KVQ_ERR_CUDA;
-    // about one work unit per SM if every sequence were max_seq_len long
-    const int64_t work = (int64_t)std::max(batch, 1) * desc->num_kv_heads * std::max(max_seq_len, 1);
-    L = (int)std::min<int64_t>((work + sms - 1) / sms, KVQ_MAX_SPLIT_TOKENS);
-  }
-  L = (L + kTile - 1) / kTile * kTile;
-  return std::max(kTile, std::min(L, KVQ_MAX_SPLIT_TOKENS));
+  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &cap);
+  return st != KVQ_OK ? st : CS;
 }
 
 size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                           int32_t max_seq_len, int32_t split_tokens) {
   if (batch < 0 || num_q_heads < 0 || head_dim <= 0 || max_seq_len < 0 || split_tokens <= 0)
     return 0;
-  return kWorkspaceHeader +
+  return kWorkspaceHeader + counters_bytes(batch, num_q_heads) +
          partials_bytes(batch, num_q_heads, head_dim, max_splits_for(max_seq_len, split_tokens));
 }
 
 int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < kWorkspaceHeader) return KVQ_ERR_WORKSPACE;
-  return cudaMemsetAsync(workspace, 0, kWorkspaceHeader, static_cast<cudaStream_t>(stream)) ==
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? KVQ_OK
              : KVQ_ERR_CUDA;
@@ -138,8 +186,9 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
                     int32_t num_q_heads, const void* k_codes, const void* k_scales,
                     const void* v_codes, const void* v_scales, const int32_t* page_table,
                     int32_t max_pages, const int32_t* seq_lens, int32_t max_seq_len,
-                    float sm_scale, float tau, int32_t split_tokens, void* workspace,
-                    size_t workspace_bytes, unsigned long long* stats, void* stream) {
+                    float sm_scale, float tau, int32_t split_tokens, uint32_t options,
+                    void* workspace, size_t workspace_bytes, unsigned long long* stats,
+                    float* out, void* stream) {
   int st = check_desc(desc);
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads < 1 || max_pages < 1 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
@@ -151,15 +200,25 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   if (!q || !k_codes || !k_scales || !v_codes || !v_scales || !seq_lens || !workspace)
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k_codes) || !aligned16(k_scales) || !aligned16(v_codes) || !aligned16(v_scales) ||
-      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(q) & 1u))
+      !aligned16(workspace) || !aligned16(q) || !aligned16(out))
     return KVQ_ERR_INVALID_ARG;
   if (!page_table && (int64_t)batch * max_pages > desc->num_pages) return KVQ_ERR_INVALID_ARG;
-  const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
-  if (L < 0) return L;
+  int L = 0;
+  st = resolve_split_len(desc, batch, num_q_heads, max_seq_len, split_tokens, options, &L);
+  if (st != KVQ_OK) return st;
   if (max_splits_for(max_seq_len, L) > KVQ_MAX_SPLITS) return KVQ_ERR_UNSUPPORTED;
   const size_t need = kvq_workspace_size(batch, num_q_heads, desc->head_dim, max_seq_len, L);
   if (workspace_bytes < need) return KVQ_ERR_WORKSPACE;
-  if (batch == 0 || max_seq_len == 0) return KVQ_OK;
+  if (batch == 0) return KVQ_OK;
+  if (max_seq_len == 0) {  // no positions anywhere: the output is zero
+    if (out && cudaMemsetAsync(out, 0, (size_t)batch * num_q_heads * desc->head_dim * sizeof(float),
+                               static_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+    return KVQ_OK;
+  }
+  int CS = 1, capacity = 0;
+  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
+  if (st != KVQ_OK) return st;
   DecodeArgs a;
   a.desc = *desc;
   a.q = q;
@@ -179,24 +238,42 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.split_tokens = L;
   a.max_splits = max_splits_for(max_seq_len, L);
   a.workspace = workspace;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.counters = reinterpret_cast<int*>(ws + kWorkspaceHeader);
+  a.generations = reinterpret_cast<uint32_t*>(a.counters + (size_t)batch * num_q_heads);
+  a.group_merge = 0;  // decided at launch
+  const size_t n_part = (size_t)batch * num_q_heads * a.max_splits;
+  a.part_o = reinterpret_cast<float*>(ws + kWorkspaceHeader + counters_bytes(batch, num_q_heads));
+  a.part_m = a.part_o + n_part * desc->head_dim;
+  a.part_l = a.part_m + n_part;
   a.stats = stats;
-  a.num_sms = device_sm_count();
-  if (a.num_sms <= 0) return KVQ_ERR_CUDA;
+  a.out = out;
+  a.cluster = CS;
+  a.shared_max = (options & KVQ_OPT_SHARED_MAX) ? 1 : 0;
+  // clusters: at most one per (sequence, KV head, group of CS splits), at most what fits
+  a.units_per_seq = (a.max_splits + CS - 1) / CS;
+  const int64_t groups = (int64_t)batch * desc->num_kv_heads * a.units_per_seq;
+  a.grid = (int)std::min<int64_t>(groups, capacity) * CS;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 
 int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
-                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens,
+                int32_t num_q_heads, int32_t max_seq_len, int32_t split_tokens, uint32_t options,
                 const int32_t* seq_lens, float* out, void* stream) {
   int st = check_desc(desc);
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads < 1 || max_seq_len < 0) return KVQ_ERR_INVALID_ARG;
   if (!workspace || !seq_lens || !out) return KVQ_ERR_INVALID_ARG;
-  const int L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
-  if (L < 0) return L;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return KVQ_ERR_INVALID_ARG;
+  int L = 0;
+  st = resolve_split_len(desc, batch, num_q_heads, max_seq_len, split_tokens, options, &L);
+  if (st != KVQ_OK) return st;
   if (max_splits_for(max_seq_len, L) > KVQ_MAX_SPLITS) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;
-  return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L,
+  int CS = 1, capacity = 0;
+  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
+  if (st != KVQ_OK) return st;
+  return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L, CS,
                         max_splits_for(max_seq_len, L), seq_lens, out,
                         static_cast<cudaStream_t>(stream));
 }

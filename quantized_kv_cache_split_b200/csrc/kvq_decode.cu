@@ -6,33 +6,43 @@
 // accumulation are skipped for every position whose weight exp(s - m_running)
 // is below tau.  Section "FAQ": K itself is always dequantized.
 //
-// Persistent CTAs (one per SM, 16 warps) loop over work units (sequence b, KV
-// head, split of <= 1024 positions = at most 16 tiles of 64 positions).
-//   K fetch   Warp w owns tile w of the unit.  At the start of the unit it streams
-//             the tile's codes and block scales into its private shared buffer with
-//             16-byte cp.async copies (an XOR swizzle on the codes keeps the MMA
-//             fragment reads free of bank conflicts); nothing waits on another warp.
-//             (Measured on B200: per-operation costs make 4 KB bulk/TMA copies run at
-//             a fraction of what many 16-byte async copies reach.)
-//   K pass    Once its copies land, the warp scores its 64 positions x 8 query heads
-//             on the tensor cores (mma m16n8k16: positions x heads x head_dim).  Codes
-//             enter the MMA as magic-number fp16 values (code + a fixed offset); the
-//             offset's contribution, a per-(head, block) constant of the query, is
-//             preloaded into the accumulator, and the block scale / vector norm is
-//             applied to the fp32 score.
-//   weights   After one CTA barrier m_running is the unit's maximum.  Each warp tests
-//             its scores: keep iff s - m >= log2(tau) (no exp for the test); the
-//             denominator l sums 2^(s - m) over every position; positions kept by any
-//             head of the group are compacted (ballot + popcount) into the warp's
-//             list, and the lists are concatenated in warp order into one CTA list.
-//   V pass    16-row groups of the CTA list are dealt round-robin to the warps.  A warp
-//             gathers only those kept V rows (cp.async 16-byte copies into its buffer,
-//             three groups in flight), dequantizes them in registers and accumulates
-//             p^T V on the tensor cores (head_dim x heads x positions).  Skipped
-//             positions cost no HBM read, no dequant, no MMA.
-//   output    The warps' accumulators are summed in shared memory; unnormalized o,
-//             m (log2 units) and l of the unit go to the workspace and kvq_combine
-//             merges the units of a sequence.
+// Work unit: one split (<= 1024 positions = at most 16 tiles of 64) of one
+// (sequence, KV head).  A thread-block cluster of CS CTAs (CS = 1, 2 or 4) takes CS
+// consecutive splits of the same (sequence, KV head); clusters loop persistently
+// over such groups.  Each CTA has 16 warps; warp w owns tile w of its split.
+//   Q         Every warp builds its own query fragments straight from global memory
+//             (lut4: rotates the query with butterflies in registers and shuffles),
+//             while its K copies are in flight; no block-wide step.
+//   K fetch   The warp streams its tile's codes and block scales into its private
+//             shared buffer with 16-byte cp.async copies, one copy group per 16-row
+//             job (an XOR swizzle of the 16-byte chunks keeps the MMA fragment reads
+//             free of bank conflicts).  With tau = 0 (nothing can be skipped) it also
+//             prefetches its V tile at once, when shared memory allows.
+//   K pass    As each job's copies land, the warp scores its 16 positions x 8 query
+//             heads on the tensor cores (mma m16n8k16: positions x heads x head_dim).
+//             Codes enter the MMA as magic-number fp16 values (code + a fixed
+//             offset); the offset's contribution, a per-(head, block) constant of the
+//             query, is preloaded into the accumulator, and the block scale / vector
+//             norm is applied to the fp32 score.  Scores stay in registers.
+//   max       One CTA barrier gives the split's maximum per head; with the shared
+//             maximum option, one cluster barrier and a read of the other CTAs'
+//             maxima (distributed shared memory) give the cluster's.
+//   weights   Each warp tests its scores: keep iff s - m >= log2(tau) (no exp needed
+//             for the test); l sums 2^(s - m) over every position; positions kept by
+//             any head of the group are compacted (ballot + popcount) into the warp's
+//             own list.  No block-wide step.
+//   V pass    The warp gathers only its kept V rows (16-byte cp.async copies of the
+//             codes plus a 16-byte window holding the row's scales), dequantizes them
+//             in registers and accumulates p^T V on the tensor cores (head_dim x
+//             heads x positions).  Skipped positions cost no HBM read, no dequant and
+//             no MMA.  A warp with nothing kept does nothing.
+//   output    The warps' accumulators (only those of warps that kept something) are
+//             summed through shared memory.  The CTAs of a cluster merge their (o, m,
+//             l) through distributed shared memory into one partial per cluster,
+//             which goes to the workspace.  When an output pointer is given, the last
+//             cluster to finish a (sequence, KV head) (an arrival counter in the
+//             workspace) merges that pair's partials by the log-sum-exp rule and
+//             writes the output (lut4: rotated back), so no second kernel runs.
 #include <mutex>
 
 #include "kvq_device.cuh"
@@ -45,14 +55,18 @@ constexpr int kWarps = 16;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kLmax = KVQ_MAX_SPLIT_TOKENS;
 constexpr int kMaxTiles = kLmax / kTile;
-static_assert(kMaxTiles == kWarps, "one K tile per warp per unit");
-constexpr int kWarpSlots = kTile;        // kept-list slots owned by one warp (its tile)
-constexpr int kPktStride = kLmax + 8;    // halves per head row of the compacted weights
+static_assert(kMaxTiles == kWarps, "one K tile per warp per split");
+constexpr int kPkStride = kTile + 8;     // halves per head row of a warp's compacted weights
 constexpr float kPScale = 16384.0f;      // p is stored in fp16 as p * 2^14
 constexpr float kPUnscale = 1.0f / 16384.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kMagic = 0x64006400u;    // fp16 1024 in both halves (unit mantissa step 1)
 constexpr uint32_t kMagic64 = 0x54005400u;  // fp16 64: mantissa bits 4..7 then count in units of 1
+constexpr size_t kSmemLimit = 232448;       // dynamic shared memory per CTA on sm_100a
+constexpr int kMergeCap = 256;              // partials per (sequence, head) whose weights the merge keeps
+
+constexpr int round128(int x) { return (x + 127) / 128 * 128; }
+constexpr int cmax3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
 
 template <int FMT, int D>
 struct Cfg {
@@ -65,75 +79,70 @@ struct Cfg {
   static constexpr int RPW = 16 / SROW;                  // rows per 16-byte scale window
   static constexpr int NBLK = D / 32;
   static constexpr int KSTEPS = D / 16;
-  static constexpr int STAGE_CODE = kTile * CROW;        // one K tile: codes ...
+  static constexpr int STAGE_CODE = kTile * CROW;        // one tile: codes ...
   static constexpr int STAGE_SC = kTile * SROW;          // ... then scales
-  // XOR swizzle of 16-byte chunks within a code row: chunk ^= (row >> SWZ_SHIFT) & SWZ_MASK
+  static constexpr int TILE = STAGE_CODE + STAGE_SC;
+  // XOR swizzle of 16-byte chunks within a K code row: chunk ^= (row >> SWZ_SHIFT) & SWZ_MASK
   static constexpr int SWZ_SHIFT = CROW == 128 ? 0 : CROW == 64 ? 1 : 2;
   static constexpr int SWZ_MASK = CROW / 16 - 1;
   // V pass: thread (r, c) owns dims E*r .. E*r + E - 1
   static constexpr int E = D / 8;
   static constexpr int MT = D / 16;                      // m-tiles (16 dims each)
+  static constexpr int NE = MT * 4;                      // accumulator registers per thread
   static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
   static constexpr int NWORD = RAWB / 4;
-  static constexpr int VSTRIDE = CROW + 16;              // staged row: codes + scale window
-  static constexpr int NVS = 3;                          // V groups of 16 rows in flight per warp
-  static constexpr int VGROUP = 16 * VSTRIDE;
-  // one buffer per warp: its K tile, then its V groups
-  static constexpr int WBUF = ((STAGE_CODE + STAGE_SC > NVS * VGROUP ? STAGE_CODE + STAGE_SC
-                                                                      : NVS * VGROUP) + 127) / 128 * 128;
+  static constexpr int VSTRIDE = CROW + 16;              // gathered row: codes + scale window
+  static constexpr int VGROUP = 16 * VSTRIDE;            // one group of 16 gathered rows
+  // per-warp buffer: its K tile, then its gathered V rows (all 4 groups), then its
+  // accumulators for the block-wide sum
+  static constexpr int KBUF = round128(cmax3(TILE, 4 * VGROUP, NE * 32 * 4));
+  static constexpr int VT = round128(TILE);              // per-warp prefetched V tile (tau = 0)
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
 
 template <int FMT, int D>
 struct Layout {
   using C = Cfg<FMT, D>;
-  static constexpr size_t wbuf = 0;                                           // [warps][WBUF]
-  // reduction buffer float [8][NE][32]; before the epilogue it holds the per-lane score
-  // slots (4 float4 per lane per warp)
-  static constexpr size_t ORED = (size_t)8 * (D / 16) * 4 * 32 * 4 > (size_t)kWarps * 4 * 32 * 16
-                                     ? (size_t)8 * (D / 16) * 4 * 32 * 4
-                                     : (size_t)kWarps * 4 * 32 * 16;
-  static constexpr size_t ored = wbuf + (size_t)kWarps * C::WBUF;
-  static constexpr size_t pkt = ored + ORED;                                  // half [8][kPktStride]
-  static constexpr size_t list = pkt + (size_t)8 * kPktStride * 2;            // u16 [kLmax]
-  static constexpr size_t pktg = list + (size_t)kLmax * 2;                    // half [8][kPktStride]
-  static constexpr size_t listg = pktg + (size_t)8 * kPktStride * 2;          // u16 [kLmax]
-  static constexpr size_t q = listg + (size_t)kLmax * 2;                      // float [8][D]
-  static constexpr size_t corr = q + (size_t)8 * D * 4;                       // float [8][NBLK]
-  static constexpr size_t rows = corr + (size_t)8 * C::NBLK * 4;              // int [kMaxTiles]
-  static constexpr size_t red = rows + kMaxTiles * 4;                         // float [2][warps][8]
+  static constexpr size_t kbuf = 0;                                            // [warps][KBUF]
+  static constexpr size_t pk = kbuf + (size_t)kWarps * C::KBUF;               // half [warps][8][kPkStride]
+  static constexpr size_t list = pk + (size_t)kWarps * 8 * kPkStride * 2;     // u8 [warps][64]
+  static constexpr size_t red = list + (size_t)kWarps * kTile;                // float [2][warps][8]
   static constexpr size_t cnt = red + 2 * kWarps * 8 * 4;                     // int [2][warps]
-  static constexpr size_t prefix = cnt + 2 * kWarps * 4;                      // int [MAX_BATCH + 1]
-  static constexpr size_t total = prefix + (KVQ_MAX_BATCH + 1) * 4;
+  static constexpr size_t cmx = cnt + 2 * kWarps * 4;                         // float [8] CTA maxima
+  static constexpr size_t mpart = cmx + 8 * 4;                                // float [8]
+  static constexpr size_t lpart = mpart + 8 * 4;                              // float [8]
+  static constexpr size_t octa = lpart + 8 * 4;                               // float [8][D]
+  static constexpr size_t slen = octa + (size_t)8 * D * 4;                    // int [MAX_BATCH]
+  static constexpr size_t misc = slen + KVQ_MAX_BATCH * 4;                     // int [4]
+  static constexpr size_t mrg = misc + 16;                                     // float [2][8]
+  static constexpr size_t scr = mrg + 64;                                      // float4 [warps][4][32] scores
+  static constexpr size_t base_total = scr + (size_t)kWarps * 4 * 32 * 16;
+  // tau = 0 prefetches the V tile alongside K when shared memory allows
+  static constexpr size_t vtile = (base_total + 127) / 128 * 128;             // [warps][VT]
+  static constexpr bool kPrefetchV = vtile + (size_t)kWarps * C::VT + 128 <= kSmemLimit;
+  static constexpr size_t total = kPrefetchV ? vtile + (size_t)kWarps * C::VT : base_total;
   static constexpr size_t alloc = total + 128;  // slack for aligning the base to 128
-  static_assert(alloc <= 232448, "shared memory");
+  static_assert(alloc <= kSmemLimit, "shared memory");
+  // cp.async destinations need 16-byte alignment; vector loads need 8 or 16
+  static_assert(kbuf % 128 == 0 && C::KBUF % 128 == 0 && vtile % 128 == 0 && C::VT % 128 == 0,
+                "staging buffers");
+  static_assert(pk % 16 == 0 && red % 16 == 0 && octa % 16 == 0 && slen % 16 == 0 && scr % 16 == 0,
+                "alignment");
+  // the merges' scratch reuses the staging buffers
+  static_assert((size_t)kWarps * C::KBUF >= (size_t)8 * kMergeCap * 4, "merge weights");
+  static_assert((size_t)kWarps * C::KBUF >= (size_t)kThreads * 16 + 2 * kMergeCap * 4 + D * 4 + 16,
+                "group merge scratch");
 };
 
-struct Item {
-  int b, kvh, split, t0, n_tok;
-};
-
-__device__ __forceinline__ int clamp_len(const DecodeArgs& a, int b) {
-  const int cap = min(a.max_seq_len, a.max_pages * a.desc.page_size);
-  const int n = a.seq_lens[b];
-  return max(0, min(n, cap));
-}
-
-__device__ __forceinline__ Item decode_item(const DecodeArgs& a, const int* prefix, int it) {
-  const int hkv = a.desc.num_kv_heads;
-  Item I;
-  const int sg = it / hkv;
-  I.kvh = it - sg * hkv;
-  int lo = 0, hi = a.batch;  // largest b with prefix[b] <= sg
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (prefix[mid] <= sg) lo = mid; else hi = mid;
+// cp.async.wait_group with a count known only after unrolling
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    default: cp_async_wait<4>(); break;
   }
-  I.b = lo;
-  I.split = sg - prefix[lo];
-  I.t0 = I.split * a.split_tokens;
-  I.n_tok = min(a.split_tokens, clamp_len(a, lo) - I.t0);
-  return I;
 }
 
 // ------------------------------------------------------------------ LUT lookups
@@ -156,24 +165,6 @@ __device__ __forceinline__ void lut_lookup4(const Lut& t, uint32_t sel, uint32_t
 // byte masks for nibbles 0-3 / 4-7 of x: replicate bit 3 of each nibble
 __device__ __forceinline__ uint32_t nib_mask_lo(uint32_t x) { return prmt(x << 4, x, 0xD9C8u); }
 __device__ __forceinline__ uint32_t nib_mask_hi(uint32_t x) { return prmt(x << 4, x, 0xFBEAu); }
-
-// ------------------------------------------------------------------ query fragments
-// Physical dims feeding the B fragment of k-step ks for tid-in-group c, in the
-// order (reg0.lo, reg0.hi, reg1.lo, reg1.hi).  They mirror how each format's
-// A fragment is unpacked from one 32-bit word of codes.
-template <int FMT>
-__device__ __forceinline__ void k_dims(int ks, int c, int (&d)[4]) {
-  if (FMT == KVQ_FMT_Q8_0) {
-    const int base = 16 * ks + 4 * c;  // bytes b0..b3 -> (b0, b2) and (b1, b3)
-    d[0] = base; d[1] = base + 2; d[2] = base + 1; d[3] = base + 3;
-  } else if (FMT == KVQ_FMT_Q4_0) {
-    const int base = 32 * (ks >> 1) + 8 * c + 2 * (ks & 1);  // nibble pairs (n, n+4)
-    d[0] = base; d[1] = base + 4; d[2] = base + 1; d[3] = base + 5;
-  } else {
-    const int base = 32 * (ks >> 1) + 8 * c + 4 * (ks & 1);  // consecutive nibbles
-    d[0] = base; d[1] = base + 1; d[2] = base + 2; d[3] = base + 3;
-  }
-}
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return h2_as_u32(__floats2half2_rn(lo, hi));
@@ -331,39 +322,173 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
   }
 }
 
-// Scale of a staged position (q8_0 / q4_0 block scale of this thread's dims, or the
-// lut4 vector norm), read from the row's 16-byte scale window; 0 past the end so
-// that stale rows contribute nothing.
-template <int FMT, int D>
-__device__ __forceinline__ __half v_scale(const uint8_t* grp, int slot, int n_valid, int blk,
-                                          const uint16_t* list_grp) {
-  using C = Cfg<FMT, D>;
-  if (slot >= n_valid) return __ushort_as_half(0);
-  const int tok = list_grp[slot];
-  const int off = C::CROW + (tok & (C::RPW - 1)) * C::SROW + (C::kLut ? 0 : 2 * blk);
-  return *reinterpret_cast<const __half*>(grp + slot * C::VSTRIDE + off);
+// bit 4r set iff any of bits 4r .. 4r+3 of a ballot is set (one row per 4-lane group)
+__device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
+  uint32_t x = bal | (bal >> 1);
+  x |= x >> 2;
+  return x & 0x11111111u;
 }
 
-// One group of 16 staged positions: acc[dims x heads] += v_hat^T p.
+// ------------------------------------------------------------------ query fragments
+// Lane (r, c) of every warp builds, straight from the fp16 query in global memory, the
+// B fragments of the K pass for query head r of the group (null qh: a head the group
+// does not have), plus the offset correction of its accumulator heads 2c, 2c + 1
+// (q8_0 / q4_0) or the fp16 low parts of the rotated query (lut4).  The dims a lane
+// needs mirror how each format's A fragment is unpacked from one 32-bit word of codes:
+//   q8_0  k-step ks: dims 16 ks + 4c + {0, 2 | 1, 3}
+//   q4_0  k-step 2m + j: dims 32m + 8c + 2j + {0, 4 | 1, 5}
+//   lut4  k-step 2m + j: dims 32m + 8c + 4j + {0, 1 | 2, 3}
 template <int FMT, int D>
-__device__ __forceinline__ void v_group(const uint8_t* __restrict__ grp, const __half* __restrict__ prow,
-                                        const uint16_t* __restrict__ list_grp, int n_valid, int r,
-                                        int c, const Lut& lut, float (&acc)[Cfg<FMT, D>::MT][4]) {
+__device__ __forceinline__ void build_query(const __half* __restrict__ qh,
+                                            const int8_t* __restrict__ signs, int c,
+                                            uint32_t (&qf)[D / 16][2], uint32_t (&ql)[D / 16][2],
+                                            float (&corr)[D / 32][2]) {
+  using C = Cfg<FMT, D>;
+  if constexpr (!C::kLut) {
+    float part[C::NBLK];
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      if constexpr (C::kQ4) {
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (qh) u = __ldg(reinterpret_cast<const uint4*>(qh + 32 * m + 8 * c));
+        qf[2 * m][0] = prmt(u.x, u.z, 0x5410u);
+        qf[2 * m][1] = prmt(u.x, u.z, 0x7632u);
+        qf[2 * m + 1][0] = prmt(u.y, u.w, 0x5410u);
+        qf[2 * m + 1][1] = prmt(u.y, u.w, 0x7632u);
+        // dims 32m + 8c + i: even i enter the MMA as 1024 + n, odd i as 64 + n; both
+        // decode as n - 8, so the offsets are 1032 and 72
+        const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
+        const float2 f2 = __half22float2(u32_as_h2(u.z)), f3 = __half22float2(u32_as_h2(u.w));
+        part[m] = 1032.f * ((f0.x + f1.x) + (f2.x + f3.x)) + 72.f * ((f0.y + f1.y) + (f2.y + f3.y));
+      } else {
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int ks = 2 * m + j;
+          uint2 u = make_uint2(0, 0);
+          if (qh) u = __ldg(reinterpret_cast<const uint2*>(qh + 16 * ks + 4 * c));
+          qf[ks][0] = prmt(u.x, u.y, 0x5410u);
+          qf[ks][1] = prmt(u.x, u.y, 0x7632u);
+          const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
+          s += (f0.x + f0.y) + (f1.x + f1.y);
+        }
+        part[m] = 1152.f * s;  // codes enter as 1152 + q
+      }
+      ql[2 * m][0] = ql[2 * m][1] = ql[2 * m + 1][0] = ql[2 * m + 1][1] = 0;
+    }
+    // sum over the four lanes of head r, then fetch heads 2c, 2c + 1
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      float v = part[m];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      corr[m][0] = __shfl_sync(0xffffffffu, v, 8 * c);
+      corr[m][1] = __shfl_sync(0xffffffffu, v, 8 * c + 4);
+    }
+  } else {
+    // q' = (1/sqrt(D)) H (s .* q), Sylvester H.  Lane c of head r holds dims
+    // 32m + 8c + i: index bits 0-2 are i (in the lane), bits 3-4 are c (lanes c ^ 1,
+    // c ^ 2), bits 5-6 are m (in the lane).
+    float y[C::NBLK][8];
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (qh) u = __ldg(reinterpret_cast<const uint4*>(qh + 32 * m + 8 * c));
+      const uint2 sg = __ldg(reinterpret_cast<const uint2*>(signs + 32 * m + 8 * c));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float2 f = __half22float2(u32_as_h2(w[i >> 1]));
+        const int8_t sgn = static_cast<int8_t>(((i < 4 ? sg.x : sg.y) >> (8 * (i & 3))) & 0xffu);
+        y[m][i] = ((i & 1) ? f.y : f.x) * (float)sgn;
+      }
+    }
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+      for (int m = 0; m < C::NBLK; ++m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (!(i & h)) {
+            const float p = y[m][i], q = y[m][i + h];
+            y[m][i] = p + q;
+            y[m][i + h] = p - q;
+          }
+#pragma unroll
+    for (int bit = 1; bit < 4; bit <<= 1) {
+      const bool upper = (c & bit) != 0;
+#pragma unroll
+      for (int m = 0; m < C::NBLK; ++m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float o = __shfl_xor_sync(0xffffffffu, y[m][i], bit);
+          y[m][i] = upper ? (o - y[m][i]) : (y[m][i] + o);
+        }
+    }
+#pragma unroll
+    for (int h = 1; h < C::NBLK; h <<= 1)
+#pragma unroll
+      for (int m = 0; m < C::NBLK; ++m)
+        if (!(m & h)) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float p = y[m][i], q = y[m + h][i];
+            y[m][i] = p + q;
+            y[m + h][i] = p - q;
+          }
+        }
+    const float cs = D == 64 ? 0.125f : 0.08838834764831845f;  // 1/sqrt(D)
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float v0 = y[m][4 * j] * cs, v1 = y[m][4 * j + 1] * cs;
+        const float v2 = y[m][4 * j + 2] * cs, v3 = y[m][4 * j + 3] * cs;
+        const __half2 h01 = __floats2half2_rn(v0, v1), h23 = __floats2half2_rn(v2, v3);
+        qf[2 * m + j][0] = h2_as_u32(h01);
+        qf[2 * m + j][1] = h2_as_u32(h23);
+        ql[2 * m + j][0] = pack_h2(v0 - __low2float(h01), v1 - __high2float(h01));
+        ql[2 * m + j][1] = pack_h2(v2 - __low2float(h23), v3 - __high2float(h23));
+      }
+      corr[m][0] = corr[m][1] = 0.f;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ V groups
+// One group of 16 staged V positions: acc[dims x heads] += v_hat^T p.  TILE: the
+// positions are rows s0 .. s0 + 15 of a staged tile (codes rows, then scale rows);
+// otherwise they are gathered rows, each its codes followed by the 16-byte window of
+// the scales plane that holds its scales (trow: the row's index in its tile).  Slots
+// at or past n_valid get scale 0, so whatever bytes they hold contribute nothing
+// (every format decodes any bit pattern to a finite value).
+template <int FMT, int D, bool TILE>
+__device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const __half* __restrict__ prow,
+                                        const uint8_t* __restrict__ trow, int s0, int n_valid,
+                                        int r, int c, const Lut& lut,
+                                        float (&acc)[Cfg<FMT, D>::MT][4]) {
   using C = Cfg<FMT, D>;
   const int blk = (C::E * r) / 32;
   const int sa = 2 * c, sc = sa + 8;
   const uint32_t b0 = lds32(prow + sa);
   const uint32_t b1 = lds32(prow + sc);
-  const __half2 dab = __halves2half2(v_scale<FMT, D>(grp, sa, n_valid, blk, list_grp),
-                                     v_scale<FMT, D>(grp, sa + 1, n_valid, blk, list_grp));
-  const __half2 dcd = __halves2half2(v_scale<FMT, D>(grp, sc, n_valid, blk, list_grp),
-                                     v_scale<FMT, D>(grp, sc + 1, n_valid, blk, list_grp));
+  auto code = [&](int slot) -> const uint8_t* {
+    return TILE ? buf + (s0 + slot) * C::CROW + C::RAWB * r : buf + slot * C::VSTRIDE + C::RAWB * r;
+  };
+  auto scale = [&](int slot) -> __half {
+    if (slot >= n_valid) return __ushort_as_half(0);
+    const int off = C::kLut ? 0 : 2 * blk;
+    const uint8_t* p = TILE ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW + off
+                            : buf + slot * C::VSTRIDE + C::CROW + (trow[slot] & (C::RPW - 1)) * C::SROW + off;
+    return *reinterpret_cast<const __half*>(p);
+  };
+  const __half2 dab = __halves2half2(scale(sa), scale(sa + 1));
+  const __half2 dcd = __halves2half2(scale(sc), scale(sc + 1));
   uint32_t wa[C::NWORD], wb[C::NWORD], wc[C::NWORD], wd[C::NWORD];
-  const int boff = C::RAWB * r;
-  v_raw<FMT, D>(grp + sa * C::VSTRIDE + boff, wa);
-  v_raw<FMT, D>(grp + (sa + 1) * C::VSTRIDE + boff, wb);
-  v_raw<FMT, D>(grp + sc * C::VSTRIDE + boff, wc);
-  v_raw<FMT, D>(grp + (sc + 1) * C::VSTRIDE + boff, wd);
+  v_raw<FMT, D>(code(sa), wa);
+  v_raw<FMT, D>(code(sa + 1), wb);
+  v_raw<FMT, D>(code(sc), wc);
+  v_raw<FMT, D>(code(sc + 1), wd);
   uint32_t eab[C::E], ecd[C::E];
   v_dequant_pair<FMT, D>(wa, wb, lut, eab);
   v_dequant_pair<FMT, D>(wc, wd, lut, ecd);
@@ -377,11 +502,112 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ grp, const _
     mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
 }
 
-// bit 4r set iff any of bits 4r .. 4r+3 of a ballot is set (one row per 4-lane group)
-__device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
-  uint32_t x = bal | (bal >> 1);
-  x |= x >> 2;
-  return x & 0x11111111u;
+// ------------------------------------------------------------------ merge of one head
+// Log-sum-exp merge of the n partials of one query head (partial u at slot uh + u):
+//   M = max_u m_u,  out = sum_u 2^(m_u - M) o_u / sum_u 2^(m_u - M) l_u
+// (lut4: rotated back, out = s .* (c H out')), written to out_row.  The whole CTA takes
+// part: thread t handles float4 column t % (D/4) of partials t / (D/4), t / (D/4) + NG,
+// ...; every load is issued before the first wait.  Scratch: wm, wl [kMergeCap] floats,
+// red [kThreads] float4, hv [D] floats, den [1].
+template <int FMT, int D>
+__device__ __forceinline__ void merge_head(const DecodeArgs& a, size_t uh, int n, float* out_row,
+                                        float* wm, float* wl, float4* red, float* hv, float* den_s) {
+  using C = Cfg<FMT, D>;
+  constexpr int NC = D / 4;           // float4 columns of a head
+  constexpr int NG = kThreads / NC;   // groups of partials
+  constexpr int kPer = 4;             // partials per thread loaded together
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d4 = tid % NC, ug = tid / NC;
+  if (tid < n) {
+    wm[tid] = __ldcg(a.part_m + uh + tid);
+    wl[tid] = __ldcg(a.part_l + uh + tid);
+  }
+  float4 o4[kPer];
+#pragma unroll
+  for (int t = 0; t < kPer; ++t) {
+    const int u = ug + t * NG;
+    o4[t] = u < n ? __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
+  if (warp == 0) {  // maximum, weights (in place of the maxima) and denominator
+    float M = -INFINITY;
+    for (int u = lane; u < n; u += 32) M = fmaxf(M, wm[u]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int u = lane; u < n; u += 32) {
+      const float w = ex2(wm[u] - M);
+      wm[u] = w;
+      den = fmaf(w, wl[u], den);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) den_s[0] = den;
+  }
+  __syncthreads();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int t = 0; t < kPer; ++t) {
+    const int u = ug + t * NG;
+    if (u < n) {
+      const float w = wm[u];
+      acc.x = fmaf(w, o4[t].x, acc.x); acc.y = fmaf(w, o4[t].y, acc.y);
+      acc.z = fmaf(w, o4[t].z, acc.z); acc.w = fmaf(w, o4[t].w, acc.w);
+    }
+  }
+  for (int u = ug + kPer * NG; u < n; u += NG) {  // more partials than one batch
+    const float w = wm[u];
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4);
+    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+  }
+  red[ug * NC + d4] = acc;
+  __syncthreads();
+  if (tid < NC) {
+    float4 v = red[tid];
+#pragma unroll 4
+    for (int g = 1; g < NG; ++g) {
+      const float4 x = red[g * NC + tid];
+      v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
+    }
+    const float inv = 1.f / den_s[0];
+    v = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
+    if constexpr (C::kLut) reinterpret_cast<float4*>(hv)[tid] = v;
+    else reinterpret_cast<float4*>(out_row)[tid] = v;
+  }
+  if constexpr (C::kLut) {
+    __syncthreads();
+    if (warp == 0) {  // out = s .* (c H out')
+      constexpr int K = D / 32;
+      float y[K];
+#pragma unroll
+      for (int kk = 0; kk < K; ++kk) y[kk] = hv[32 * kk + lane];
+#pragma unroll
+      for (int hb = 1; hb < 32; hb <<= 1) {
+        const bool upper = (lane & hb) != 0;
+#pragma unroll
+        for (int kk = 0; kk < K; ++kk) {
+          const float t = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+          y[kk] = upper ? (t - y[kk]) : (y[kk] + t);
+        }
+      }
+#pragma unroll
+      for (int hb = 1; hb < K; hb <<= 1)
+#pragma unroll
+        for (int kk = 0; kk < K; ++kk)
+          if (!(kk & hb)) {
+            const float u = y[kk], v = y[kk + hb];
+            y[kk] = u + v;
+            y[kk + hb] = u - v;
+          }
+      const float cs = D == 64 ? 0.125f : 0.08838834764831845f;
+#pragma unroll
+      for (int kk = 0; kk < K; ++kk)
+        out_row[32 * kk + lane] = y[kk] * cs * (float)a.desc.signs[32 * kk + lane];
+    }
+  }
+  __syncthreads();  // scratch free again
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -392,54 +618,46 @@ decode_kernel(const DecodeArgs a) {
   using LY = Layout<FMT, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
-  float* ored = reinterpret_cast<float*>(smem + LY::ored);
-  __half* pkt = reinterpret_cast<__half*>(smem + LY::pkt);
-  uint16_t* list = reinterpret_cast<uint16_t*>(smem + LY::list);
-  __half* pktg = reinterpret_cast<__half*>(smem + LY::pktg);        // CTA-wide compacted weights
-  uint16_t* listg = reinterpret_cast<uint16_t*>(smem + LY::listg);  // CTA-wide kept list
-  float* qs = reinterpret_cast<float*>(smem + LY::q);
-  float* corr_s = reinterpret_cast<float*>(smem + LY::corr);
-  int* item_rows = reinterpret_cast<int*>(smem + LY::rows);
   float* red_m = reinterpret_cast<float*>(smem + LY::red);
   float* red_l = red_m + kWarps * 8;
   int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
   int* cnt_kept = cnt_skip + kWarps;
-  int* prefix = reinterpret_cast<int*>(smem + LY::prefix);
+  float* cmx = reinterpret_cast<float*>(smem + LY::cmx);       // this CTA's maxima (log2)
+  float* mpart = reinterpret_cast<float*>(smem + LY::mpart);   // m of this CTA's partial
+  float* lpart = reinterpret_cast<float*>(smem + LY::lpart);   // l of this CTA's partial
+  float* octa = reinterpret_cast<float*>(smem + LY::octa);     // o of this CTA's partial [8][D]
+  int* slen = reinterpret_cast<int*>(smem + LY::slen);         // clamped sequence lengths
+  int* misc = reinterpret_cast<int*>(smem + LY::misc);
+  float* mrg_m = reinterpret_cast<float*>(smem + LY::mrg);     // merge: per-head maximum ...
+  float* mrg_d = mrg_m + 8;                                    // ... and denominator
+  float* mrg_w = reinterpret_cast<float*>(smem + LY::kbuf);    // merge: weights [8][kMergeCap]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
   uint32_t* flags = reinterpret_cast<uint32_t*>(a.workspace);
   const int hkv = a.desc.num_kv_heads, G = a.group, P = a.desc.page_size, Ls = a.split_tokens;
-  const int B = a.batch, Hq = a.num_q_heads;
-  uint8_t* my_buf = smem + LY::wbuf + (size_t)warp * C::WBUF;
+  const int B = a.batch, Hq = a.num_q_heads, CS = a.cluster;
+  const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
+  const int cid = CS > 1 ? (int)cluster_index() : (int)blockIdx.x;
+  const int ncl = CS > 1 ? (int)cluster_count() : (int)gridDim.x;
+  uint8_t* kbuf = smem + LY::kbuf + (size_t)warp * C::KBUF;
+  uint8_t* vtile = smem + LY::vtile + (size_t)warp * C::VT;   // used only when kPrefetchV
+  __half* pk_w = reinterpret_cast<__half*>(smem + LY::pk) + (size_t)warp * 8 * kPkStride;
+  uint8_t* list_w = smem + LY::list + (size_t)warp * kTile;
+  // Work units form a static list over (group of CS splits cu, sequence b, KV head),
+  // cu-major, as if every sequence were max_seq_len long; a unit past its sequence's
+  // end is skipped.  cu-major order puts the units that exist for every sequence first.
+  const int NCU = a.units_per_seq;
+  const int total = B * NCU * hkv;
+  const int cap = min(a.max_seq_len, a.max_pages * P);  // positions that exist in memory
 
-  // ---- work list: splits per sequence, exclusive prefix
-  for (int b = tid; b < B; b += kThreads) {
-    const int n = a.seq_lens[b];
-    const int cap = min(a.max_seq_len, a.max_pages * P);
-    if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
-    const int nc = max(0, min(n, cap));
-    prefix[b + 1] = (nc + Ls - 1) / Ls;
-  }
-  if (tid == 0) prefix[0] = 0;
-  __syncthreads();
-  if (warp == 0) {
-    int run = 0;
-    for (int base = 1; base <= B; base += 32) {
-      const int i = base + lane;
-      int v = (i <= B) ? prefix[i] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-      }
-      if (i <= B) prefix[i] = v + run;
-      run += __shfl_sync(0xffffffffu, v, 31);
-    }
-  }
-  __syncthreads();
-  const int total_items = prefix[B] * hkv;
-  if ((int)blockIdx.x >= total_items) return;
+  // compacted weights of pad slots must be finite: start from zeros
+  for (int i = lane; i < 8 * kPkStride / 2; i += 32) reinterpret_cast<uint32_t*>(pk_w)[i] = 0u;
+  // Programmatic dependent launch: the next kernel on the stream may be scheduled now
+  // (it waits for this grid to finish before reading anything), and this one reads no
+  // input before the preceding grid has finished and its writes are visible.
+  grid_dependents_launch();
+  grid_dependency_wait();
 
   Lut lut;
   if constexpr (C::kLut) {
@@ -461,167 +679,131 @@ decode_kernel(const DecodeArgs a) {
 
   const float qk_scale = a.sm_scale * kLog2e;
   const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
+  const bool prefetch_v = LY::kPrefetchV && !(a.tau > 0.f);  // tau = 0: every row is kept
   const __half* qg = static_cast<const __half*>(a.q);
   const uint8_t* kcodes = static_cast<const uint8_t*>(a.k_codes);
   const uint8_t* kscales = static_cast<const uint8_t*>(a.k_scales);
   const uint8_t* vcodes = static_cast<const uint8_t*>(a.v_codes);
   const uint8_t* vscales = static_cast<const uint8_t*>(a.v_scales);
-  float* ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + kWorkspaceHeader);
-  const size_t n_part = (size_t)B * Hq * a.max_splits;
-  float* ws_m = ws_o + n_part * D;
-  float* ws_l = ws_m + n_part;
-  const int wslot0 = warp * kWarpSlots;  // this warp's region of the kept list / weights
-  const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;  // this lane's two heads exist
+  const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;  // this lane's two accumulator heads exist
+  const uint32_t below = (1u << (4 * r)) - 1u;
 
 #pragma unroll 1
   for (int k = 0;; ++k) {
-    const int it = blockIdx.x + k * gridDim.x;
-    if (it >= total_items) break;
-    const Item I = decode_item(a, prefix, it);
-    const int ntiles = (I.n_tok + kTile - 1) / kTile;
-    const bool has_tile = warp < ntiles;
+    const int it = cid + k * ncl;
+    if (it >= total) break;
+    // ---- the cluster's (group of splits, sequence, KV head) and this CTA's split
+    const int kvh = it % hkv;
+    const int bu = it / hkv;
+    const int b = bu % B;
+    const int cu = bu / B;
+    const int t0 = (cu * CS + (int)rank) * Ls;
+    // The first unit reads its sequence length from global memory while its K copies
+    // are already in flight (they cover what exists in memory, up to cap); later
+    // units know the length before copying anything.
+    int nb;
+    if (k == 0) {
+      nb = __shfl_sync(0xffffffffu, lane == 0 ? __ldg(a.seq_lens + b) : 0, 0);
+      nb = max(0, min(nb, cap));
+    } else {
+      __syncthreads();  // the lengths in shared memory are visible (the first unit may have had no barrier)
+      nb = slen[b];
+      if (cu * CS * Ls >= nb) continue;  // no such unit (uniform over the cluster)
+    }
+    const int avail = k == 0 ? cap : nb;  // positions the copies may cover
 
-    // ---- K fetch: this warp's tile (positions 64 w .. 64 w + 63 of the unit)
-    if (has_tile) {
-      const int tok0 = I.t0 + warp * kTile;
+    // ---- K fetch (and, for tau = 0, the V tile): one copy group per 16-row job
+    int row0 = -1;
+    const int ncopy = min(kTile, avail - t0 - warp * kTile);
+    if (ncopy > 0) {
+      const int tok0 = t0 + warp * kTile;
       const int lp = tok0 / P, off = tok0 - lp * P;  // tiles never straddle pages (P % 64 == 0)
-      const int page = a.page_table ? a.page_table[(size_t)I.b * a.max_pages + lp]
-                                    : I.b * a.max_pages + lp;
-      const bool ok = page >= 0 && page < a.desc.num_pages;
-      const int row0 = ok ? (page * hkv + I.kvh) * P + off : -1;
-      if (lane == 0) {
-        item_rows[warp] = row0;
-        if (!ok) set_flag(flags, KVQ_FLAG_BAD_PAGE);
-      }
-      if (ok) {
+      const int page = a.page_table ? __ldg(a.page_table + (size_t)b * a.max_pages + lp)
+                                    : b * a.max_pages + lp;
+      if (page >= 0 && page < a.desc.num_pages) {
+        row0 = (page * hkv + kvh) * P + off;
         constexpr int CPR = C::CROW / 16;
         const uint8_t* src = kcodes + (size_t)row0 * C::CROW;
-#pragma unroll
-        for (int i = lane; i < kTile * CPR; i += 32) {
-          const int row = i / CPR, cc = i - row * CPR;
-          const int sc = cc ^ ((row >> C::SWZ_SHIFT) & C::SWZ_MASK);
-          cp_async16(my_buf + row * C::CROW + (sc << 4), src + (size_t)i * 16);
-        }
         const uint8_t* ssrc = kscales + (size_t)row0 * C::SROW;
 #pragma unroll
-        for (int i = lane; i < C::STAGE_SC / 16; i += 32)
-          cp_async16(my_buf + C::STAGE_CODE + i * 16, ssrc + (size_t)i * 16);
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int i = lane; i < 16 * CPR; i += 32) {
+            const int row = 16 * j + i / CPR, cc = i % CPR;
+            const int sw = cc ^ ((row >> C::SWZ_SHIFT) & C::SWZ_MASK);
+            cp_async16(kbuf + row * C::CROW + (sw << 4), src + (size_t)row * C::CROW + cc * 16);
+          }
+          if (lane < C::SROW)  // 16 rows of scales = SROW 16-byte chunks
+            cp_async16(kbuf + C::STAGE_CODE + 16 * j * C::SROW + lane * 16,
+                       ssrc + 16 * j * C::SROW + lane * 16);
+          cp_async_commit();
+        }
+        if (prefetch_v) {
+          const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
+#pragma unroll 4
+          for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(vtile + i * 16, vsrc + i * 16);
+          const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
+#pragma unroll
+          for (int i = lane; i < C::STAGE_SC / 16; i += 32)
+            cp_async16(vtile + C::STAGE_CODE + i * 16, vssrc + i * 16);
+          cp_async_commit();
+        }
       }
     }
-    cp_async_commit();
+    if (k == 0) {
+      // clamped sequence lengths for later units and the final zero fill (read once,
+      // behind the first copies; visible after the next barrier)
+      for (int bb = tid; bb < B; bb += kThreads) {
+        const int n = a.seq_lens[bb];
+        if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
+        slen[bb] = max(0, min(n, cap));
+      }
+    }
+    if (k == 0 && cu * CS * Ls >= nb) {  // a speculative unit past the sequence's end
+      cp_async_wait<0>();
+      continue;
+    }
+    const int n_tok = max(0, min(Ls, nb - t0));
+    int nvalid = min(kTile, n_tok - warp * kTile);  // positions of this warp's tile
+    if (nvalid > 0 && row0 < 0) {
+      if (lane == 0) set_flag(flags, KVQ_FLAG_BAD_PAGE);
+      nvalid = 0;
+    }
 
-    // ---- query group -> shared (fp32)
-    {
-      constexpr int kChunks = 8 * D / 8;  // 16-byte chunks of 8 heads x D fp16
-      if (tid < kChunks) {
-        const int h = tid / (D / 8), d0 = (tid - h * (D / 8)) * 8;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (h < G)
-          raw = *reinterpret_cast<const uint4*>(qg + ((size_t)I.b * Hq + I.kvh * G + h) * D + d0);
-        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __half22float2(hp[e]);
-          qs[h * D + d0 + 2 * e] = f.x;
-          qs[h * D + d0 + 2 * e + 1] = f.y;
-        }
-      }
-    }
-    __syncthreads();
-    if (warp < 8) {
-      const int h = warp;
-      constexpr int K = D / 32;
-      if constexpr (C::kLut) {
-        // q' = c * H * (s .* q), butterflies in fp32; warp h rotates head h
-        float y[K];
-#pragma unroll
-        for (int kk = 0; kk < K; ++kk) {
-          const int i = 32 * kk + lane;
-          y[kk] = qs[h * D + i] * (float)a.desc.signs[i];
-        }
-#pragma unroll
-        for (int hb = 1; hb < 32; hb <<= 1) {
-          const bool upper = (lane & hb) != 0;
-#pragma unroll
-          for (int kk = 0; kk < K; ++kk) {
-            const float o = __shfl_xor_sync(0xffffffffu, y[kk], hb);
-            y[kk] = upper ? (o - y[kk]) : (y[kk] + o);
-          }
-        }
-#pragma unroll
-        for (int kk = 0; kk + 1 < K; kk += 2) {
-          const float u = y[kk], v = y[kk + 1];
-          y[kk] = u + v; y[kk + 1] = u - v;
-        }
-        if (K == 4) {
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const float u = y[kk], v = y[kk + 2];
-            y[kk] = u + v; y[kk + 2] = u - v;
-          }
-        }
-        const float cs = rsqrtf((float)D);
-#pragma unroll
-        for (int kk = 0; kk < K; ++kk) qs[h * D + 32 * kk + lane] = y[kk] * cs;
-      } else {
-        // offset contribution per (head, block): sum_d q_d * (offset_d + 8) for q4_0
-        // (offset 1024 on even dims, 64 on odd dims), sum_d q_d * 1152 for q8_0
-#pragma unroll
-        for (int m = 0; m < K; ++m) {
-          const int d = 32 * m + lane;
-          const float w = C::kQ8 ? 1152.f : ((d & 1) ? 72.f : 1032.f);
-          float v = qs[h * D + d] * w;
-#pragma unroll
-          for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if (lane == 0) corr_s[h * C::NBLK + m] = v;
-        }
-      }
-    }
-    __syncthreads();
+    // ---- query fragments (overlap the copies in flight)
     uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
-#pragma unroll
-    for (int ks = 0; ks < C::KSTEPS; ++ks) {
-      int d[4];
-      k_dims<FMT>(ks, c, d);
-      const float v0 = qs[r * D + d[0]], v1 = qs[r * D + d[1]];
-      const float v2 = qs[r * D + d[2]], v3 = qs[r * D + d[3]];
-      const __half2 h01 = __floats2half2_rn(v0, v1), h23 = __floats2half2_rn(v2, v3);
-      qf[ks][0] = h2_as_u32(h01);
-      qf[ks][1] = h2_as_u32(h23);
-      if constexpr (C::kLut) {
-        ql[ks][0] = pack_h2(v0 - __low2float(h01), v1 - __high2float(h01));
-        ql[ks][1] = pack_h2(v2 - __low2float(h23), v3 - __high2float(h23));
-      } else {
-        ql[ks][0] = ql[ks][1] = 0;
-      }
-    }
     float corr[C::NBLK][2];
-#pragma unroll
-    for (int m = 0; m < C::NBLK; ++m) {
-      corr[m][0] = C::kLut ? 0.f : corr_s[(2 * c) * C::NBLK + m];
-      corr[m][1] = C::kLut ? 0.f : corr_s[(2 * c + 1) * C::NBLK + m];
-    }
+    build_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr,
+                        a.desc.signs, c, qf, ql, corr);
 
-    // ---- K pass: the warp's tile, four 16-row jobs; scores to per-lane shared slots
-    float4* sbuf = reinterpret_cast<float4*>(ored) + (size_t)warp * 4 * 32 + lane;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-    cp_async_wait<0>();
-    __syncwarp();
-    if (has_tile) {
+    // ---- K pass: four 16-row jobs as their copies land.  Scores stay in registers;
+    //      each lane keeps a running maximum and sum 2^(s - m) for its two heads, so
+    //      the denominator needs no pass of its own.
+    float4* scw = reinterpret_cast<float4*>(smem + LY::scr) + (size_t)warp * 4 * 32 + lane;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        const int row0 = 16 * mt + r;
-        float s[4];
-        k_job_scores<FMT, D>(my_buf, my_buf + C::STAGE_CODE, row0, qf, ql, corr, lut, c, s);
-        const int p0 = warp * kTile + row0;
-        const bool v0 = p0 < I.n_tok, v1 = p0 + 8 < I.n_tok;
-        const float4 sv = make_float4(v0 ? s[0] * qk_scale : -INFINITY, v0 ? s[1] * qk_scale : -INFINITY,
-                                      v1 ? s[2] * qk_scale : -INFINITY, v1 ? s[3] * qk_scale : -INFINITY);
-        sbuf[mt * 32] = sv;
-        mx0 = fmaxf(mx0, fmaxf(sv.x, sv.z));
-        mx1 = fmaxf(mx1, fmaxf(sv.y, sv.w));
+    for (int j = 0; j < 4; ++j) {
+      if (16 * j >= nvalid) break;
+      cp_async_wait_n(3 - j + (prefetch_v ? 1 : 0));
+      __syncwarp();
+      float s[4];
+      k_job_scores<FMT, D>(kbuf, kbuf + C::STAGE_CODE, 16 * j + r, qf, ql, corr, lut, c, s);
+      const bool v0 = 16 * j + r < nvalid, v1 = 16 * j + r + 8 < nvalid;
+      const float4 sv = make_float4(v0 ? s[0] * qk_scale : -INFINITY, v0 ? s[1] * qk_scale : -INFINITY,
+                                    v1 ? s[2] * qk_scale : -INFINITY, v1 ? s[3] * qk_scale : -INFINITY);
+      scw[j * 32] = sv;
+      const float n0 = fmaxf(m0, fmaxf(sv.x, sv.z));
+      const float n1 = fmaxf(m1, fmaxf(sv.y, sv.w));
+      if (n0 != -INFINITY) {
+        l0 = l0 * ex2(m0 - n0) + ex2(sv.x - n0) + ex2(sv.z - n0);
+        m0 = n0;
+      }
+      if (n1 != -INFINITY) {
+        l1 = l1 * ex2(m1 - n1) + ex2(sv.y - n1) + ex2(sv.w - n1);
+        m1 = n1;
       }
     }
+    float mx0 = m0, mx1 = m1;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
@@ -631,31 +813,47 @@ decode_kernel(const DecodeArgs a) {
       red_m[warp * 8 + 2 * c] = mx0;
       red_m[warp * 8 + 2 * c + 1] = mx1;
     }
-    __syncthreads();  // barrier 1: every warp's maxima are in shared memory
-
-    // ---- weights, skip test, compaction (rows r, r+8 of each job; heads 2c, 2c+1)
-    float mh0 = red_m[2 * c], mh1 = red_m[2 * c + 1];
+    __syncthreads();  // every warp's maxima are in shared memory
+    if (tid < 8) {
+      float m = red_m[tid];
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) {
-      mh0 = fmaxf(mh0, red_m[w * 8 + 2 * c]);
-      mh1 = fmaxf(mh1, red_m[w * 8 + 2 * c + 1]);
+      for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red_m[w * 8 + tid]);
+      cmx[tid] = m;
     }
-    float l0 = 0.f, l1 = 0.f;
+    if (CS > 1) cluster_sync(); else __syncthreads();  // CTA maxima visible (cluster-wide)
+    float mh0 = cmx[2 * c], mh1 = cmx[2 * c + 1];
+    if (CS > 1 && a.shared_max) {
+      for (int rk = 0; rk < CS; ++rk) {
+        if (rk == (int)rank) continue;
+        mh0 = fmaxf(mh0, dsmem_ld(dsmem_addr(cmx + 2 * c, rk)));
+        mh1 = fmaxf(mh1, dsmem_ld(dsmem_addr(cmx + 2 * c + 1, rk)));
+      }
+    }
+    if (warp == 0 && r == 0) {
+      mpart[2 * c] = mh0;
+      mpart[2 * c + 1] = mh1;
+    }
+    // denominator: each lane's running sum rescaled to the decision maximum
+    l0 = (m0 != -INFINITY) ? l0 * ex2(m0 - mh0) : 0.f;
+    l1 = (m1 != -INFINITY) ? l1 * ex2(m1 - mh1) : 0.f;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+
+    // ---- skip test and compaction into this warp's list (rows r, r + 8 of each job;
+    //      heads 2c, 2c + 1); weights are computed for kept pairs only
     int nkept = 0, nskip = 0;
-    const uint32_t below = (1u << (4 * r)) - 1u;
-    if (has_tile) {
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        const float4 sv = sbuf[mt * 32];
-        const int p0 = warp * kTile + 16 * mt + r;
-        const bool va = p0 < I.n_tok, vb = p0 + 8 < I.n_tok;
+    for (int j = 0; j < 4; ++j) {
+      if (16 * j < nvalid) {
+        const int ra = 16 * j + r, rb = ra + 8;
+        const bool va = ra < nvalid, vb = rb < nvalid;
         const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
+        const float4 sv = scw[j * 32];
         const float da0 = sv.x - mh0, da1 = sv.y - mh1;
         const float db0 = sv.z - mh0, db1 = sv.w - mh1;
-        const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
-        const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
-        l0 += ea0 + eb0;
-        l1 += ea1 + eb1;
         const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
         const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
         nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
@@ -663,24 +861,19 @@ decode_kernel(const DecodeArgs a) {
         const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
         const int na = __popc(rows_a);
         if ((rows_a >> (4 * r)) & 1u) {
-          const int slot = wslot0 + nkept + __popc(rows_a & below);
-          if (c == 0) list[slot] = (uint16_t)p0;
-          pkt[(2 * c) * kPktStride + slot] = __float2half_rn(ka0 ? ea0 * kPScale : 0.f);
-          pkt[(2 * c + 1) * kPktStride + slot] = __float2half_rn(ka1 ? ea1 * kPScale : 0.f);
+          const int slot = nkept + __popc(rows_a & below);
+          if (c == 0) list_w[slot] = (uint8_t)ra;
+          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(ka0 ? ex2(da0) * kPScale : 0.f);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(ka1 ? ex2(da1) * kPScale : 0.f);
         }
         if ((rows_b >> (4 * r)) & 1u) {
-          const int slot = wslot0 + nkept + na + __popc(rows_b & below);
-          if (c == 0) list[slot] = (uint16_t)(p0 + 8);
-          pkt[(2 * c) * kPktStride + slot] = __float2half_rn(kb0 ? eb0 * kPScale : 0.f);
-          pkt[(2 * c + 1) * kPktStride + slot] = __float2half_rn(kb1 ? eb1 * kPScale : 0.f);
+          const int slot = nkept + na + __popc(rows_b & below);
+          if (c == 0) list_w[slot] = (uint8_t)rb;
+          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(kb0 ? ex2(db0) * kPScale : 0.f);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(kb1 ? ex2(db1) * kPScale : 0.f);
         }
         nkept += na + __popc(rows_b);
       }
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
@@ -692,158 +885,408 @@ decode_kernel(const DecodeArgs a) {
       cnt_skip[warp] = nskip;
       cnt_kept[warp] = nkept;
     }
-    __syncthreads();  // barrier 2: every warp's kept count is known
-    // ---- concatenate the warps' lists in warp order (deterministic) into the CTA list
-    int gbase = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      const int n = cnt_kept[w];
-      gbase += (w < warp) ? n : 0;
-      total += n;
-    }
-    for (int i = lane; i < nkept; i += 32) {
-      listg[gbase + i] = list[wslot0 + i];
-#pragma unroll
-      for (int h = 0; h < 8; ++h) pktg[h * kPktStride + gbase + i] = pkt[h * kPktStride + wslot0 + i];
-    }
-    if (warp == kWarps - 1) {  // zero the padding slots of the last partial group
-      const int pad = ((total + 15) & ~15) - total;
-      for (int i = lane; i < 8 * pad; i += 32)
-        pktg[(i / pad) * kPktStride + total + (i % pad)] = __ushort_as_half(0);
-    }
-    __syncthreads();  // barrier 3: the CTA list is complete
+    __syncwarp();  // the warp's list and weights are complete
 
-    // ---- V pass: kept positions only, 16-row groups dealt round-robin to the warps
-    float acc[C::MT][4];
+    // ---- V pass: this warp's kept positions only
+    if (nkept > 0) {
+      float acc[C::MT][4];
 #pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-    const int ngroups_all = (total + 15) >> 4;
-    const int ngroups = ngroups_all > warp ? (ngroups_all - warp + kWarps - 1) / kWarps : 0;
-    auto issue = [&](int gi) {  // this warp's gi-th group = CTA group warp + 16 gi
-      uint8_t* grp = my_buf + (size_t)(gi % C::NVS) * C::VGROUP;
-      const int s0 = 16 * (warp + kWarps * gi);
-      constexpr int CPR = C::CROW / 16 + 1;  // code chunks + the scale window
+      for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      const int ng = (nkept + 15) >> 4;
+      if (prefetch_v || nkept == nvalid) {
+        // every valid row is kept, so slot s is tile row s; without the prefetched tile,
+        // one contiguous copy of the V tile into the (now free) K buffer
+        const uint8_t* vt = vtile;
+        if (!prefetch_v) {
+          __syncwarp();  // every lane is done reading the K tile
+          const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
+#pragma unroll 4
+          for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(kbuf + i * 16, vsrc + i * 16);
+          const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
 #pragma unroll
-      for (int i = lane; i < 16 * CPR; i += 32) {
-        const int rl = i / CPR, cc = i - rl * CPR;
-        const int slot = s0 + rl;
-        if (slot < total) {
-          const int tok = listg[slot];
-          const int rb = item_rows[tok >> 6];
-          if (rb >= 0) {
-            const size_t row = (size_t)rb + (tok & 63);
+          for (int i = lane; i < C::STAGE_SC / 16; i += 32)
+            cp_async16(kbuf + C::STAGE_CODE + i * 16, vssrc + i * 16);
+          cp_async_commit();
+          vt = kbuf;
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+#pragma unroll 1
+        for (int g = 0; g < ng; ++g)
+          v_group<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
+                                min(16, nkept - 16 * g), r, c, lut, acc);
+      } else {
+        // gather the kept rows into the (now free) K buffer: codes + the scale window
+        constexpr int CPR = C::CROW / 16 + 1;
+        for (int i = lane; i < 16 * ng * CPR; i += 32) {
+          const int s = i / CPR, cc = i - s * CPR;
+          if (s < nkept) {
+            const size_t row = (size_t)row0 + list_w[s];
             const uint8_t* src = cc < CPR - 1 ? vcodes + row * C::CROW + cc * 16
                                               : vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW;
-            cp_async16(grp + rl * C::VSTRIDE + cc * 16, src);
+            cp_async16(kbuf + (s >> 4) * C::VGROUP + (s & 15) * C::VSTRIDE + cc * 16, src);
           }
         }
-      }
-      cp_async_commit();
-    };
-#pragma unroll
-    for (int i = 0; i < C::NVS; ++i) {
-      if (i < ngroups) issue(i);
-      else cp_async_commit();
-    }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
 #pragma unroll 1
-    for (int gi = 0; gi < ngroups; ++gi) {
-      cp_async_wait<C::NVS - 1>();
-      __syncwarp();
-      const int s0 = 16 * (warp + kWarps * gi);
-      v_group<FMT, D>(my_buf + (size_t)(gi % C::NVS) * C::VGROUP, pktg + r * kPktStride + s0,
-                      listg + s0, min(16, total - s0), r, c, lut, acc);
-      __syncwarp();
-      if (gi + C::NVS < ngroups) issue(gi + C::NVS);
-      else cp_async_commit();
+        for (int g = 0; g < ng; ++g)
+          v_group<FMT, D, false>(kbuf + g * C::VGROUP, pk_w + r * kPkStride + 16 * g, list_w + 16 * g,
+                                 0, min(16, nkept - 16 * g), r, c, lut, acc);
+      }
+      __syncwarp();  // staged V fully read before the accumulators overwrite the buffer
+      float* accw = reinterpret_cast<float*>(kbuf);
+#pragma unroll
+      for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accw[(mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
-    cp_async_wait<0>();
+    cp_async_wait<0>();  // nothing of this split stays in flight
+    __syncthreads();     // every warp's accumulators, l and counts are in shared memory
 
-    // ---- sum the warps' accumulators and write the unit
-    constexpr int NE = C::MT * 4;  // accumulator registers per thread
-    __syncthreads();  // barrier 4: every warp's V accumulation is done; score slots free
-    if (warp >= 8) {
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) ored[((warp - 8) * NE + mt * 4 + i) * 32 + lane] = acc[mt][i];
-    }
-    __syncthreads();  // barrier 5
-    if (warp < 8) {
-#pragma unroll
-      for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float* p = ored + (warp * NE + mt * 4 + i) * 32 + lane;
-          *p = *p + acc[mt][i];
-        }
-    }
-    __syncthreads();  // barrier 6
-    {
-      const size_t unit0 = ((size_t)I.b * Hq + (size_t)I.kvh * G) * a.max_splits + I.split;
-      for (int q = tid; q < 32 * NE; q += kThreads) {
-        const int ln = q & 31, e = q >> 5;
+    // ---- this CTA's partial: sum the accumulators of the warps that kept something.
+    //      A lone CTA writes it straight to the workspace; a cluster merges first.
+    const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
+    for (int q = tid; q < 32 * C::NE; q += kThreads) {
+      const int ln = q & 31, e = q >> 5;
+      const int mt = e >> 2, i = e & 3;
+      const int h = 2 * (ln & 3) + (i & 1);
+      const int dim = C::E * (ln >> 2) + 2 * mt + (i >> 1);
+      if (h < G) {
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += ored[(w * NE + e) * 32 + ln];
-        const int mt = e >> 2, i = e & 3;
-        const int rr = ln >> 2, cc = ln & 3;
-        const int h = 2 * cc + (i & 1);
-        const int dim = C::E * rr + 2 * mt + (i >> 1);
-        if (h < G) ws_o[(unit0 + (size_t)h * a.max_splits) * D + dim] = v * kPUnscale;
-      }
-      if (tid < G) {
-        float m = red_m[tid], l = red_l[tid];
-#pragma unroll
-        for (int w = 1; w < kWarps; ++w) {
-          m = fmaxf(m, red_m[w * 8 + tid]);
-          l += red_l[w * 8 + tid];
-        }
-        const size_t u = unit0 + (size_t)tid * a.max_splits;
-        ws_m[u] = m;
-        ws_l[u] = l;
-      }
-      if (tid == 0 && a.stats) {
-        int ns = 0, nk = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          ns += cnt_skip[w];
-          nk += cnt_kept[w];
-        }
-        atomicAdd(&a.stats[0], (unsigned long long)I.n_tok * G);
-        atomicAdd(&a.stats[1], (unsigned long long)ns);
-        atomicAdd(&a.stats[2], (unsigned long long)nk);
-        atomicAdd(&a.stats[3], (unsigned long long)(I.n_tok - nk));
+        for (int w = 0; w < kWarps; ++w)
+          if (cnt_kept[w] > 0) v += reinterpret_cast<const float*>(smem + LY::kbuf + (size_t)w * C::KBUF)[q];
+        v *= kPUnscale;
+        if (CS > 1) octa[h * D + dim] = v;
+        else a.part_o[(slot0 + (size_t)h * a.max_splits) * D + dim] = v;
       }
     }
-    __syncthreads();  // barrier 7: shared buffers free for the next unit
+    if (tid < G) {
+      float l = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
+      if (CS > 1) {
+        lpart[tid] = l;
+      } else {
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mpart[tid];
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+      }
+    }
+    if (tid == 32 && a.stats && n_tok > 0) {
+      int ns = 0, nk = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        ns += cnt_skip[w];
+        nk += cnt_kept[w];
+      }
+      atomicAdd(&a.stats[0], (unsigned long long)n_tok * G);
+      atomicAdd(&a.stats[1], (unsigned long long)ns);
+      atomicAdd(&a.stats[2], (unsigned long long)nk);
+      atomicAdd(&a.stats[3], (unsigned long long)(n_tok - nk));
+    }
+
+    if (CS > 1) {
+      // one partial per cluster: merge the CTAs' (o, m, l), each CTA a slice of dims
+      cluster_sync();  // every CTA's partial is complete
+      const int per = (G * D + CS - 1) / CS;
+      for (int e = tid; e < per; e += kThreads) {
+        const int idx = (int)rank * per + e;
+        if (idx < G * D) {
+          const int h = idx / D, d = idx - h * D;
+          float mr[4], Mc = -INFINITY;
+#pragma unroll
+          for (int rk = 0; rk < 4; ++rk) {
+            mr[rk] = rk < CS ? dsmem_ld(dsmem_addr(mpart + h, rk)) : -INFINITY;
+            Mc = fmaxf(Mc, mr[rk]);
+          }
+          float o = 0.f;
+#pragma unroll
+          for (int rk = 0; rk < 4; ++rk)
+            if (rk < CS && mr[rk] != -INFINITY) o += ex2(mr[rk] - Mc) * dsmem_ld(dsmem_addr(octa + idx, rk));
+          a.part_o[(slot0 + (size_t)h * a.max_splits) * D + d] = o;
+        }
+      }
+      if (rank == 0 && tid < G) {
+        float mr[4], Mc = -INFINITY;
+#pragma unroll
+        for (int rk = 0; rk < 4; ++rk) {
+          mr[rk] = rk < CS ? dsmem_ld(dsmem_addr(mpart + tid, rk)) : -INFINITY;
+          Mc = fmaxf(Mc, mr[rk]);
+        }
+        float l = 0.f;
+#pragma unroll
+        for (int rk = 0; rk < 4; ++rk)
+          if (rk < CS && mr[rk] != -INFINITY) l += ex2(mr[rk] - Mc) * dsmem_ld(dsmem_addr(lpart + tid, rk));
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = Mc;
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+      }
+      if (a.out) __threadfence();
+      cluster_sync();  // no CTA reuses its shared partial before the others have read it
+    } else if (a.out) {
+      __threadfence();
+      __syncthreads();
+    }
+
+    // ---- in-kernel merge.  When every unit has its own CTA, the CTAs of this
+    //      (sequence, KV head) meet at a barrier and CTA s merges heads s, s + n, ...;
+    //      otherwise the last cluster to finish the pair merges all of its heads.
+    if (a.out && a.group_merge) {
+      const int n = (nb + Ls - 1) / Ls;  // splits (CTAs) of this (sequence, KV head)
+      if (tid == 0)
+        misc[0] = cta_group_barrier(a.counters + (size_t)b * hkv + kvh,
+                                    a.generations + (size_t)b * hkv + kvh, n);
+      __syncthreads();
+      if (misc[0]) {
+        __threadfence();
+        uint8_t* scratch = smem + LY::kbuf;  // free: every warp's accumulators are summed
+        for (int h = cu; h < G; h += n)
+          merge_head<FMT, D>(a, ((size_t)b * Hq + (size_t)kvh * G + h) * a.max_splits, n,
+                             a.out + ((size_t)b * Hq + (size_t)kvh * G + h) * D,
+                             reinterpret_cast<float*>(scratch + kThreads * 16),
+                             reinterpret_cast<float*>(scratch + kThreads * 16 + kMergeCap * 4),
+                             reinterpret_cast<float4*>(scratch),
+                             reinterpret_cast<float*>(scratch + kThreads * 16 + 2 * kMergeCap * 4),
+                             reinterpret_cast<float*>(scratch + kThreads * 16 + 2 * kMergeCap * 4 + D * 4));
+      } else if (tid == 0) {
+        set_flag(flags, KVQ_FLAG_TIMEOUT);
+      }
+    } else if (a.out && rank == 0) {
+      const int ncu = ((nb + Ls - 1) / Ls + CS - 1) / CS;  // partials of sequence b
+      if (tid == 0) {
+        __threadfence();
+        const int old = atomicAdd(&a.counters[(size_t)b * hkv + kvh], 1);
+        misc[0] = old == ncu - 1;
+      }
+      __syncthreads();
+      if (misc[0]) {
+        __threadfence();
+        const size_t u0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits;
+        const bool keep_m = ncu <= kMergeCap;
+        // Two threads per (head, 4 dims), each taking every other partial; the second
+        // half hands its sum over in shared memory.  The partial outputs are requested
+        // first so that they are in flight while the maxima are reduced.
+        const int nq = G * (D / 4);
+        const int half = tid >= nq ? 1 : 0;
+        const int qq = tid - half * nq;
+        const bool act = tid < 2 * nq;
+        const int h = qq / (D / 4), d4 = qq - h * (D / 4);
+        const size_t uh = u0 + (size_t)h * a.max_splits;
+        constexpr int kBatch = 20;  // partials per thread whose loads are in flight together
+        float4 o4[kBatch];
+#pragma unroll
+        for (int t = 0; t < kBatch; ++t) {
+          const int u = half + 2 * t;
+          o4[t] = act && u < ncu ? __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (warp < G) {  // head `warp`: maximum and denominator, 64 partials per round
+          const size_t uw = u0 + (size_t)warp * a.max_splits;
+          float M = -INFINITY, den = 0.f;
+          for (int ub = 0; ub < ncu; ub += 64) {
+            const int ua = ub + lane, uc = ub + 32 + lane;
+            const float ma = ua < ncu ? __ldcg(a.part_m + uw + ua) : -INFINITY;
+            const float mc = uc < ncu ? __ldcg(a.part_m + uw + uc) : -INFINITY;
+            const float la = ua < ncu ? __ldcg(a.part_l + uw + ua) : 0.f;
+            const float lc = uc < ncu ? __ldcg(a.part_l + uw + uc) : 0.f;
+            if (keep_m) {
+              if (ua < ncu) mrg_w[warp * kMergeCap + ua] = ma;
+              if (uc < ncu) mrg_w[warp * kMergeCap + uc] = mc;
+            }
+            float bm = fmaxf(ma, mc);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float nm = fmaxf(M, bm);
+            float ds = (ma == -INFINITY ? 0.f : ex2(ma - nm) * la) + (mc == -INFINITY ? 0.f : ex2(mc - nm) * lc);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+            den = (M == -INFINITY ? 0.f : den * ex2(M - nm)) + ds;
+            M = nm;
+          }
+          if (lane == 0) {
+            mrg_m[warp] = M;
+            mrg_d[warp] = den;
+          }
+        }
+        __syncthreads();
+        float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (act) {
+          const float Mh = mrg_m[h];
+          auto weight = [&](int u) {
+            return ex2((keep_m ? mrg_w[h * kMergeCap + u] : __ldcg(a.part_m + uh + u)) - Mh);
+          };
+#pragma unroll
+          for (int t = 0; t < kBatch; ++t) {
+            const int u = half + 2 * t;
+            if (u < ncu) {
+              const float w = weight(u);
+              acc4.x = fmaf(w, o4[t].x, acc4.x);
+              acc4.y = fmaf(w, o4[t].y, acc4.y);
+              acc4.z = fmaf(w, o4[t].z, acc4.z);
+              acc4.w = fmaf(w, o4[t].w, acc4.w);
+            }
+          }
+          for (int u = half + 2 * kBatch; u < ncu; u += 2) {  // more partials than one batch
+            const float w = weight(u);
+            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4);
+            acc4.x = fmaf(w, v4.x, acc4.x);
+            acc4.y = fmaf(w, v4.y, acc4.y);
+            acc4.z = fmaf(w, v4.z, acc4.z);
+            acc4.w = fmaf(w, v4.w, acc4.w);
+          }
+          if (half) reinterpret_cast<float4*>(octa)[qq] = acc4;
+        }
+        __syncthreads();
+        if (act && !half) {
+          const float4 o4 = reinterpret_cast<const float4*>(octa)[qq];
+          const float inv = 1.f / mrg_d[h];
+          const float4 v = make_float4((acc4.x + o4.x) * inv, (acc4.y + o4.y) * inv,
+                                       (acc4.z + o4.z) * inv, (acc4.w + o4.w) * inv);
+          if constexpr (C::kLut) reinterpret_cast<float4*>(octa)[qq] = v;
+          else reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D)[qq] = v;
+        }
+        if constexpr (C::kLut) {
+          __syncthreads();
+          if (warp < G) {  // out = s .* (c H out'), one warp per head
+            constexpr int K = D / 32;
+            float y[K];
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk) y[kk] = octa[warp * D + 32 * kk + lane];
+#pragma unroll
+            for (int hb = 1; hb < 32; hb <<= 1) {
+              const bool upper = (lane & hb) != 0;
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk) {
+                const float t = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+                y[kk] = upper ? (t - y[kk]) : (y[kk] + t);
+              }
+            }
+#pragma unroll
+            for (int hb = 1; hb < K; hb <<= 1)
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk)
+                if (!(kk & hb)) {
+                  const float u = y[kk], v = y[kk + hb];
+                  y[kk] = u + v;
+                  y[kk + hb] = u - v;
+                }
+            const float cs = D == 64 ? 0.125f : 0.08838834764831845f;
+            float* dst = a.out + ((size_t)b * Hq + (size_t)kvh * G + warp) * D;
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk)
+              dst[32 * kk + lane] = y[kk] * cs * (float)a.desc.signs[32 * kk + lane];
+          }
+        }
+        if (tid == 0) a.counters[(size_t)b * hkv + kvh] = 0;  // ready for the next call
+      }
+    }
+  }
+
+  // sequences with no positions get a zero output (they have no units)
+  if (a.out && blockIdx.x == 0) {
+    __syncthreads();  // the lengths in shared memory are visible
+    for (int b = 0; b < B; ++b)
+      if (slen[b] == 0)
+        for (int i = tid; i < Hq * D; i += kThreads) a.out[(size_t)b * Hq * D + i] = 0.f;
   }
 }
 
 // ------------------------------------------------------------------ host side
+std::mutex g_mu;
+
+template <int FMT, int D>
+int configure(int dev) {
+  using LY = Layout<FMT, D>;
+  static uint64_t done_mask = 0;  // guarded by g_mu
+  if (!(done_mask >> dev & 1)) {
+    auto kern = decode_kernel<FMT, D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)LY::alloc) !=
+        cudaSuccess)
+      return KVQ_ERR_CUDA;
+    done_mask |= 1ull << dev;
+  }
+  return KVQ_OK;
+}
+
+template <int FMT, int D>
+int capacity_t(int cluster) {
+  using LY = Layout<FMT, D>;
+  static int cache[64][3] = {};  // [device][log2 cluster] = clusters + 1; guarded by g_mu
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int ci = cluster == 4 ? 2 : cluster == 2 ? 1 : 0;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (cache[dev][ci] == 0) {
+    if (configure<FMT, D>(dev) != KVQ_OK) return 0;
+    int n = 0;
+    if (cluster == 1) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<FMT, D>, kThreads, LY::alloc) !=
+          cudaSuccess)
+        return 0;
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+      n *= sms;
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(cluster * 64, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = LY::alloc;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<FMT, D>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+    }
+    cache[dev][ci] = n + 1;
+  }
+  return cache[dev][ci] - 1;
+}
+
 template <int FMT, int D>
 int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   using LY = Layout<FMT, D>;
-  auto kern = decode_kernel<FMT, D>;
-  // The shared-memory opt-in is set once per device (so that later calls, including
-  // ones made while a stream is being captured into a graph, issue no attribute call).
-  static std::mutex mu;
-  static uint64_t done_mask = 0;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return KVQ_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
   {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!(done_mask >> dev & 1)) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)LY::alloc) != cudaSuccess)
-        return KVQ_ERR_CUDA;
-      done_mask |= 1ull << dev;
-    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (configure<FMT, D>(dev) != KVQ_OK) return KVQ_ERR_CUDA;
   }
-  // upper bound on work units: every sequence as long as max_seq_len
-  const int64_t units = (int64_t)a.batch * a.desc.num_kv_heads * a.max_splits;
-  const int grid = (int)std::min<int64_t>(units, a.num_sms);
-  if (grid <= 0) return KVQ_OK;
-  kern<<<grid, kThreads, LY::alloc, stream>>>(a);
+  if (a.grid <= 0) return KVQ_OK;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(a.grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = LY::alloc;
+  cfg.stream = stream;
+  DecodeArgs b = a;
+  // every unit with its own CTA (a single round): the in-kernel merge may use a barrier
+  // among the CTAs of a (sequence, KV head), so all CTAs must be resident together
+  b.group_merge = a.out && a.cluster == 1 && a.max_splits <= kMergeCap &&
+                  (int64_t)a.batch * a.units_per_seq * a.desc.num_kv_heads <= a.grid;
+  int na = 0;
+  if (a.cluster > 1) attr[na++] = attr[0];
+  if (b.group_merge) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+  } else {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+  }
+  ++na;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, decode_kernel<FMT, D>, b) != cudaSuccess) return KVQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -851,13 +1294,25 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int f = a.desc.fmt, d = a.desc.head_dim;
-  if (f == KVQ_FMT_Q8_0 && d == 128) return launch_decode_t<KVQ_FMT_Q8_0, 128>(a, stream);
-  if (f == KVQ_FMT_Q8_0 && d == 64) return launch_decode_t<KVQ_FMT_Q8_0, 64>(a, stream);
-  if (f == KVQ_FMT_Q4_0 && d == 128) return launch_decode_t<KVQ_FMT_Q4_0, 128>(a, stream);
-  if (f == KVQ_FMT_Q4_0 && d == 64) return launch_decode_t<KVQ_FMT_Q4_0, 64>(a, stream);
-  if (f == KVQ_FMT_LUT4 && d == 128) return launch_decode_t<KVQ_FMT_LUT4, 128>(a, stream);
-  if (f == KVQ_FMT_LUT4 && d == 64) return launch_decode_t<KVQ_FMT_LUT4, 64>(a, stream);
+#define KVQ_CALL_LAUNCH(F, DD) launch_decode_t<F, DD>(a, stream)
+  if (f == KVQ_FMT_Q8_0 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_Q8_0, 128);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_Q8_0, 64);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_Q4_0, 128);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_Q4_0, 64);
+  if (f == KVQ_FMT_LUT4 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_LUT4, 128);
+  if (f == KVQ_FMT_LUT4 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_LUT4, 64);
+#undef KVQ_CALL_LAUNCH
   return KVQ_ERR_UNSUPPORTED;
+}
+
+int decode_cluster_capacity(int f, int d, int cluster) {
+  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity_t<KVQ_FMT_Q8_0, 128>(cluster);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity_t<KVQ_FMT_Q8_0, 64>(cluster);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity_t<KVQ_FMT_Q4_0, 128>(cluster);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity_t<KVQ_FMT_Q4_0, 64>(cluster);
+  if (f == KVQ_FMT_LUT4 && d == 128) return capacity_t<KVQ_FMT_LUT4, 128>(cluster);
+  if (f == KVQ_FMT_LUT4 && d == 64) return capacity_t<KVQ_FMT_LUT4, 64>(cluster);
+  return 0;
 }
 
 }  // namespace kvq

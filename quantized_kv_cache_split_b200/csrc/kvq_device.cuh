@@ -139,6 +139,78 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// ------------------------------------------------------------------ thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster arrives (release) and waits (acquire).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ------------------------------------------------------------------ inter-CTA signalling
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// A barrier among the `n` CTAs that share (counter, generation), called by one thread
+// of each CTA after its writes are fenced.  The last to arrive resets the counter and
+// advances the generation; the others wait for the generation to change, for at most
+// kWaitCycles.  Returns false if the wait gave up.
+__device__ __forceinline__ bool cta_group_barrier(int* counter, uint32_t* generation, int n) {
+  const uint32_t g0 = ld_acquire_gpu(generation);
+  const int old = atomicAdd(counter, 1);
+  if (old == n - 1) {
+    atomicExch(counter, 0);
+    __threadfence();
+    atomicAdd(generation, 1u);
+    return true;
+  }
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(generation) == g0) {
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(64);
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// Block until the grids this one depends on have completed and their memory is visible
+// (a no-op when the launch has no programmatic dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the dependent grid to be scheduled before this one completes.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ bit tricks
 // prmt in its default mode: selector nibble bit 3 replicates the sign of the chosen byte.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {

@@ -27,21 +27,40 @@ struct DecodeArgs {
   int split_tokens;   // resolved, multiple of kTile
   int max_splits;     // ceil(max_seq_len / split_tokens)
   void* workspace;
+  int* counters;      // [batch][num_kv_heads] arrival counters of the in-kernel merge
+  float* part_o;      // partials, see below
+  float* part_m;
+  float* part_l;
   unsigned long long* stats;
-  int num_sms;
+  float* out;         // non-null: merge in the same kernel and write the output
+  int cluster;        // consecutive splits per thread-block cluster (1, 2 or 4)
+  int shared_max;     // the splits of a cluster share one running maximum
+  int grid;           // CTAs launched (a multiple of cluster)
+  int units_per_seq;  // cluster groups of one (sequence, KV head) at max_seq_len
+  int group_merge;    // every unit has its own CTA: the CTAs of a (sequence, KV head) meet
+                      // at a barrier and each merges some of its heads
+  uint32_t* generations;  // [batch][num_kv_heads] barrier generations (group_merge)
 };
 
-// Partials inside the workspace (after the 256-byte header):
+// Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits); the merge counters and the
+// barrier generations (int32 [batch][num_q_heads] each reserved, together rounded up to
+// 256 bytes); then the partials, one slot per cluster of splits:
 //   o [batch][num_q_heads][max_splits][head_dim] fp32 (unnormalized)
 //   m [batch][num_q_heads][max_splits] fp32 (running maximum, log2 units)
 //   l [batch][num_q_heads][max_splits] fp32
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits);
+__host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
+  return ((size_t)2 * batch * num_q_heads * sizeof(int32_t) + 255) / 256 * 256;
+}
 
 int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,
                     void* codes, void* scales, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Clusters of `cluster` CTAs of the decode kernel for (fmt, head_dim) that fit on the
+// current device at once (0 if none); cached per device.
+int decode_cluster_capacity(int fmt, int head_dim, int cluster);
 int launch_combine(const kvq_cache_desc& desc, const void* workspace, int batch, int num_q_heads,
-                   int max_seq_len, int split_tokens, int max_splits, const int32_t* seq_lens,
+                   int max_seq_len, int split_tokens, int cluster, int max_splits, const int32_t* seq_lens,
                    float* out, cudaStream_t stream);
 
 int device_sm_count();

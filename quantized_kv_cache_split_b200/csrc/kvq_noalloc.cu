@@ -3,9 +3,10 @@
 // Some callers cannot allocate device memory at decode time: an inference runtime that
 // pre-plans every buffer before serving, a process running under a memory pool that
 // forbids new allocations, or a host that calls in from a context where cudaMalloc is
-// not permitted.  This entry point runs the same split-KV kernel and merge as
-// kvq_decode_attn + kvq_combine, but keeps the per-split partials in a static device
-// array owned by the library, so the caller passes only inputs and outputs.
+// not permitted.  This entry point runs the same split-KV kernel, with its in-kernel
+// merge, as kvq_decode_attn given an output pointer, but keeps the partials and merge
+// counters in a static device array owned by the library, so the caller passes only
+// inputs and outputs.
 #include <mutex>
 
 #include "kvq_device.cuh"
@@ -45,10 +46,10 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q
                                        const void* v_scales, const int32_t* page_table,
                                        int32_t max_pages, const int32_t* seq_lens,
                                        int32_t max_seq_len, float sm_scale, float tau,
-                                       int32_t split_tokens, unsigned long long* stats,
-                                       float* out, void* stream) {
+                                       int32_t split_tokens, uint32_t options,
+                                       unsigned long long* stats, float* out, void* stream) {
   if (!desc || !out) return KVQ_ERR_INVALID_ARG;
-  const int32_t L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens);
+  const int32_t L = kvq_resolve_split(desc, batch, num_q_heads, max_seq_len, split_tokens, options);
   if (L < 0) return L;
   const size_t need = kvq_workspace_size(batch, num_q_heads, desc->head_dim, max_seq_len, L);
   if (need == 0 || need > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
@@ -56,11 +57,11 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q
   int st = scratch_address(&ws);
   if (st != KVQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the flag word must start at zero for every call (no allocation involved)
-  if (cudaMemsetAsync(ws, 0, kWorkspaceHeader, s) != cudaSuccess) return KVQ_ERR_CUDA;
-  st = kvq_decode_attn(desc, q, batch, num_q_heads, k_codes, k_scales, v_codes, v_scales,
-                       page_table, max_pages, seq_lens, max_seq_len, sm_scale, tau, L, ws, need,
-                       stats, stream);
-  if (st != KVQ_OK) return st;
-  return kvq_combine(desc, ws, batch, num_q_heads, max_seq_len, L, seq_lens, out, stream);
+  // the flag word and the merge counters must start at zero for every call
+  if (cudaMemsetAsync(ws, 0, kWorkspaceHeader + counters_bytes(batch, num_q_heads), s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  // the merge runs inside the decode kernel (output pointer given)
+  return kvq_decode_attn(desc, q, batch, num_q_heads, k_codes, k_scales, v_codes, v_scales,
+                         page_table, max_pages, seq_lens, max_seq_len, sm_scale, tau, L, options,
+                         ws, need, stats, out, stream);
 }

@@ -18,7 +18,11 @@ def codebook_for(D: int) -> np.ndarray:
     return OC.lloyd_max_f16(16, 1.0 / math.sqrt(D))
 
 
-def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=None):
+def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=None,
+                shared_max: bool = False, fused: bool = True):
+    """One decode step through the C ABI.  ``fused``: the merge runs inside the decode
+    kernel; otherwise kvq_combine runs it.  ``shared_max``: the splits of a cluster
+    share one running maximum (the oracle replays it with share = the cluster size)."""
     import quantized_kv_cache_split_b200 as K
     wl = inp.wl
     D, Hkv = wl.head_dim, wl.num_kv_heads
@@ -38,19 +42,22 @@ def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=Non
     max_seq = int(max(inp.seq_lens.max(), 1))
     out = cache.attention(q, seq, max_seq, pt, inp.max_pages, tau=tau,
                           sm_scale=float(np.float32(1.0 / math.sqrt(D))),
-                          split_tokens=split_tokens, stats=stats)
+                          split_tokens=split_tokens, stats=stats, shared_max=shared_max,
+                          fused=fused)
     torch.cuda.synchronize()
-    L = K.kvq_resolve_split(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens)
+    opts = K.KVQ_OPT_SHARED_MAX if shared_max else 0
+    L = K.kvq_resolve_split(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens, opts)
+    CS = K.kvq_resolve_cluster(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens, opts)
     flags = cache.device_flags()
     return dict(out=out.cpu().numpy().astype(np.float64), stats=stats.cpu().numpy(), split=L,
-                flags=flags, cache=cache)
+                cluster=CS, share=CS if shared_max else 1, flags=flags, cache=cache)
 
 
-def run_oracle(inp: W.Inputs, tau: float, split: int, codebook16=None, groups=None):
+def run_oracle(inp: W.Inputs, tau: float, split: int, codebook16=None, groups=None, share: int = 1):
     wl = inp.wl
     return OA.decode_step(wl.fmt, inp.q, inp.k, inp.v, inp.seq_lens, wl.num_kv_heads,
                           float(np.float32(1.0 / math.sqrt(wl.head_dim))), float(np.float32(tau)),
-                          split, signs=inp.signs, codebook16=codebook16, groups=groups)
+                          split, signs=inp.signs, codebook16=codebook16, groups=groups, share=share)
 
 
 def check_parity(inp: W.Inputs, g: dict, o: dict, tau: float, groups=None):

@@ -73,7 +73,8 @@ def test_split_resolution_and_workspace_size():
     assert K.kvq_resolve_split(d, 1, 32, 4096, 5000) == K.KVQ_MAX_SPLIT_TOKENS
     assert K.kvq_resolve_split(d, 1, 32, 4096, 1) == 64
     ws = K.kvq_workspace_size(2, 32, 128, 1000, 128)
-    assert ws == 256 + 2 * 32 * 8 * (128 + 2) * 4
+    assert ws == 256 + 512 + 2 * 32 * 8 * (128 + 2) * 4      # header, merge counters, partials
+    assert K.kvq_workspace_size(3, 32, 128, 1000, 128) == 256 + 768 + 3 * 32 * 8 * (128 + 2) * 4
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -91,19 +92,19 @@ def test_quantize_rejects_bad_descriptors(kw, code):
 
 def test_quantize_rejects_bad_pointers():
     d = _desc()
-    assert K.kvq_quantize(d, None, 4, None, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_quantize(d, None, 4, None, FAKE, FAKE, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
     assert K.kvq_quantize(d, FAKE, 4, None, FAKE + 8, FAKE, 0, check=False) == K.KVQ_ERR_INVALID_ARG
-    assert K.kvq_quantize(d, FAKE, -1, None, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_INVALID_ARG
-    assert K.kvq_quantize(d, FAKE, 0, None, FAKE, FAKE, 0, check=False) == K.KVQ_OK
+    assert K.kvq_quantize(d, FAKE, -1, None, FAKE, FAKE, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_quantize(d, FAKE, 0, None, FAKE, FAKE, stream=0, check=False) == K.KVQ_OK
     # more tokens than the cache holds, with identity slots
-    assert K.kvq_quantize(d, FAKE, 8 * 64 + 1, None, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_quantize(d, FAKE, 8 * 64 + 1, None, FAKE, FAKE, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
 
 
 def _decode(d, **kw):
     a = dict(q=FAKE, batch=1, num_q_heads=32, k_codes=FAKE, k_scales=FAKE, v_codes=FAKE,
              v_scales=FAKE, page_table=None, max_pages=1, seq_lens=FAKE, max_seq_len=256,
              sm_scale=0.088, tau=1e-6, split_tokens=64, workspace=FAKE, workspace_bytes=1 << 30,
-             stats=None, stream=0)
+             stats=None, out=None, options=0, stream=0)
     a.update(kw)
     return K.kvq_decode_attn(d, check=False, **a)
 
@@ -120,6 +121,10 @@ def _decode(d, **kw):
     (dict(batch=K.KVQ_MAX_BATCH + 1, max_pages=1), K.KVQ_ERR_UNSUPPORTED),
     (dict(batch=9, max_pages=1), K.KVQ_ERR_INVALID_ARG),  # identity pages beyond num_pages
     (dict(batch=0), K.KVQ_OK),
+    (dict(options=2), K.KVQ_ERR_INVALID_ARG),           # unknown option bit
+    (dict(q=FAKE + 8), K.KVQ_ERR_INVALID_ARG),          # query not 16-byte aligned
+    (dict(out=FAKE + 2), K.KVQ_ERR_INVALID_ARG),        # output not 4-byte aligned
+    (dict(workspace=FAKE + 8), K.KVQ_ERR_INVALID_ARG),  # workspace not 16-byte aligned
 ])
 def test_decode_rejects_bad_arguments(kw, code):
     assert _decode(_desc(), **kw) == code
@@ -127,9 +132,9 @@ def test_decode_rejects_bad_arguments(kw, code):
 
 def test_combine_rejects_bad_arguments():
     d = _desc()
-    assert K.kvq_combine(d, None, 1, 32, 256, 64, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_INVALID_ARG
-    assert K.kvq_combine(d, FAKE, 1, 32, 256, 64, FAKE, None, 0, check=False) == K.KVQ_ERR_INVALID_ARG
-    assert K.kvq_combine(d, FAKE, 0, 32, 256, 64, FAKE, FAKE, 0, check=False) == K.KVQ_OK
+    assert K.kvq_combine(d, None, 1, 32, 256, 64, FAKE, FAKE, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_combine(d, FAKE, 1, 32, 256, 64, FAKE, None, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_combine(d, FAKE, 0, 32, 256, 64, FAKE, FAKE, stream=0, check=False) == K.KVQ_OK
 
 
 def test_product_code_never_imports_the_oracle():

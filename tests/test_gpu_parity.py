@@ -79,18 +79,70 @@ def test_decode_parity_small(name, tau, split):
     assert g["flags"] == 0
 
 
+@pytest.mark.parametrize("name,tau,split", [
+    ("tiny_q8_d64", 1e-6, 64), ("gqa_4k_q8", 1e-6, 0), ("gqa_4k_q8", 1e-6, 256), ("lut_4k", 1e-6, 0),
+    ("lut_4k", 1e-2, 128)])
+def test_decode_parity_shared_max(name, tau, split):
+    # the splits of a cluster share one running maximum for the skip test
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
+    g = run_library(inp, tau, split, cb, shared_max=True)
+    assert g["share"] > 1
+    o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+
+
+@pytest.mark.parametrize("name,tau", [("gqa_4k_q8", 1e-6), ("lut_4k", 0.0), ("tiny_q8_d64", 1e-6)])
+def test_combine_kernel_matches_in_kernel_merge(name, tau):
+    # kvq_combine over the workspace partials gives what the in-kernel merge gives
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
+    g1 = run_library(inp, tau, 0, cb, fused=True)
+    g2 = run_library(inp, tau, 0, cb, fused=False)
+    o = run_oracle(inp, tau, g1["split"], cb)
+    check_parity(inp, g2, o, tau)
+    vmax = np.abs(inp.v.astype(np.float32)).max()
+    assert np.max(np.abs(g1["out"] - g2["out"])) <= 1e-5 * vmax
+
+
+def test_in_kernel_merge_resets_its_counters():
+    # back-to-back calls on one workspace: each must merge exactly once and agree bitwise
+    import quantized_kv_cache_split_b200 as K
+    wl = W.shrink(W.WORKLOADS["paged_b8_q4"], [3000, 64, 0, 1500, 777], n_planted=8)
+    inp = W.generate(wl)
+    g = run_library(inp, 1e-6, 128)
+    cache = g["cache"]
+    dev = torch.device("cuda")
+    q = torch.from_numpy(inp.q).to(dev)
+    seq = torch.from_numpy(inp.seq_lens).to(dev)
+    pt = torch.from_numpy(inp.page_table).to(dev)
+    outs = []
+    for _ in range(3):
+        o = torch.full((wl.batch, wl.num_q_heads, wl.head_dim), float("nan"), device=dev)
+        cache.attention(q, seq, int(inp.seq_lens.max()), pt, inp.max_pages, tau=1e-6,
+                        sm_scale=float(np.float32(1 / math.sqrt(128))), split_tokens=128, out=o)
+        outs.append(o.cpu().numpy())
+    assert not np.isnan(outs[0]).any()
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2])
+    np.testing.assert_array_equal(outs[0], g["out"].astype(np.float32))
+
+
 RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 
 
 @pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
-@pytest.mark.parametrize("tau,split", [(0.0, 128), (1e-6, 0), (1e-4, 192), (1e-6, 1024)])
-def test_decode_parity_paged_ragged(fmt, tau, split):
+@pytest.mark.parametrize("tau,split,shared", [(0.0, 128, False), (1e-6, 0, False), (1e-4, 192, False),
+                                              (1e-6, 1024, False), (1e-6, 128, True)])
+def test_decode_parity_paged_ragged(fmt, tau, split, shared):
     base = W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt)
     wl = W.shrink(base, RAGGED_LENS, n_planted=8)
     inp = W.generate(wl)
     cb = codebook_for(wl.head_dim) if fmt == "lut4" else None
-    g = run_library(inp, tau, split, cb)
-    o = run_oracle(inp, tau, g["split"], cb)
+    g = run_library(inp, tau, split, cb, shared_max=shared)
+    o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
     check_parity(inp, g, o, tau)
     assert g["flags"] == 0
 
@@ -111,13 +163,13 @@ def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
 # ------------------------------------------------------------------ full sizes
 
 @pytest.mark.parametrize("name", ["gqa_32k_q4", "lut_32k"])
-@pytest.mark.parametrize("tau", [1e-6, 0.0])
-def test_decode_parity_full_32k(name, tau):
+@pytest.mark.parametrize("tau,shared", [(1e-6, False), (0.0, False), (1e-6, True)])
+def test_decode_parity_full_32k(name, tau, shared):
     wl = W.WORKLOADS[name]
     inp = W.generate(wl)
     cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
-    g = run_library(inp, tau, 0, cb)
-    o = run_oracle(inp, tau, g["split"], cb)
+    g = run_library(inp, tau, 0, cb, shared_max=shared)
+    o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
     check_parity(inp, g, o, tau)
     if tau > 0:
         # the workload's point: most weights are skipped

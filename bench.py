@@ -210,15 +210,17 @@ class Replicas:
         self.out = torch.empty((self.B, self.Hq, D), dtype=torch.float32, device=device)
         self.sm = float(np.float32(1.0 / math.sqrt(D)))
 
-    def decode(self, i, tau, stats=None, shared_max=False, fused=True):
+    def decode(self, i, tau, stats=None, scope="split", fused=True):
         """One decode step on cache copy i % R; ``fused``: the merge runs in the same
-        kernel and writes ``self.out``."""
+        kernel and writes ``self.out``; ``scope``: the running maximum of the skip test
+        ("split", "cluster" or "sequence")."""
         import quantized_kv_cache_split_b200 as K
         c = self.caches[i % self.R]
+        opts = {"split": 0, "cluster": K.KVQ_OPT_SHARED_MAX, "sequence": K.KVQ_OPT_GLOBAL_MAX}[scope]
         K.kvq_decode_attn(c.desc, self.q, self.B, self.Hq, c.k_codes, c.k_scales, c.v_codes,
                           c.v_scales, self.pt, self.inp.max_pages, self.seq, self.max_seq, self.sm,
-                          tau, self.L_sh if shared_max else self.L, self.ws, self.ws_bytes, stats,
-                          self.out if fused else None, K.KVQ_OPT_SHARED_MAX if shared_max else 0)
+                          tau, self.L_sh if scope == "cluster" else self.L, self.ws, self.ws_bytes,
+                          stats, self.out if fused else None, opts)
 
     def combine(self, i):
         import quantized_kv_cache_split_b200 as K
@@ -309,26 +311,27 @@ def gpu_arm(args, world, rank, local):
     def n_partials(L, CS):
         return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
 
-    def counters(tau, shared):
+    def counters(tau, scope):
         st = torch.zeros(4, dtype=torch.int64, device=device)
-        rep.decode(0, tau, st, shared_max=shared)
+        rep.decode(0, tau, st, scope=scope)
         torch.cuda.synchronize()
         return [int(x) for x in st.cpu()]
 
     res = {}
     hbm_peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
-    variants = (("sparse", args.tau, False), ("dense", 0.0, False), ("sparse_shared_max", args.tau, True))
-    for tag, tau, shared in variants:
-        st = counters(tau, shared)
-        step = GraphRunner(lambda i: rep.decode(i, tau, shared_max=shared), rep.R)
+    variants = (("sparse", args.tau, "split"), ("dense", 0.0, "split"),
+                ("sparse_cluster_max", args.tau, "cluster"), ("sparse_sequence_max", args.tau, "sequence"))
+    for tag, tau, scope in variants:
+        st = counters(tau, scope)
+        step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope), rep.R)
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)
-        abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if shared
+        abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if scope == "cluster"
                                    else n_partials(rep.L, 1))
         us_launch = ms_step * 1e3 / args.steps
         achieved = abytes / (us_launch * 1e-6) / 1e9
-        res[tag] = dict(tau=tau, shared_max=shared, ms_per_step=ms_step / args.steps,
+        res[tag] = dict(tau=tau, max_scope=scope, ms_per_step=ms_step / args.steps,
                         us_per_token=ms_step * 1e3 / args.steps / (wl.batch * world),
                         us_per_launch=us_launch, algorithmic_bytes=abytes,
                         achieved_gbs=achieved, frac=achieved / hbm_peak,
@@ -351,7 +354,7 @@ def gpu_arm(args, world, rank, local):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
-                   "shared_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
+                   "cluster_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
                    "l2": f"inputs rotate over {rep.R} cache copies "
                          f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -366,8 +369,10 @@ def gpu_arm(args, world, rank, local):
         "gpu_launches": args.steps,
         "dense": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res["dense"].items()},
         "sparse": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in sp.items()},
-        "sparse_shared_max": {k: (round(v, 6) if isinstance(v, float) else v)
-                              for k, v in res["sparse_shared_max"].items()},
+        "sparse_cluster_max": {k: (round(v, 6) if isinstance(v, float) else v)
+                               for k, v in res["sparse_cluster_max"].items()},
+        "sparse_sequence_max": {k: (round(v, 6) if isinstance(v, float) else v)
+                                for k, v in res["sparse_sequence_max"].items()},
         "two_launch_us_per_token": round(ms_two * 1e3 / args.steps / (wl.batch * world), 4),
         "clocks": sampler.report(),
     }

@@ -75,6 +75,7 @@ extern "C" {
 
 /* Option bits of kvq_decode_attn. */
 #define KVQ_OPT_SHARED_MAX 1u  /* the splits of one cluster share one running maximum (below) */
+#define KVQ_OPT_GLOBAL_MAX 2u  /* every split uses the maximum over all splits of its sequence (below) */
 
 /* Device flag bits (kvq_read_device_flags). */
 #define KVQ_FLAG_BAD_PAGE     1u  /* a page-table entry outside [0, num_pages) */
@@ -164,10 +165,16 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                query head h when exp(s_hj - m_hs) < tau, where m_hs is the running
  *                maximum once all K tiles of the split are folded in (with
  *                KVQ_OPT_SHARED_MAX: of all splits of its cluster group, see
- *                kvq_resolve_cluster).  tau = 0 keeps everything (dense attention).
+ *                kvq_resolve_cluster; with KVQ_OPT_GLOBAL_MAX: of all splits of the
+ *                (sequence, KV head), i.e. the final maximum of the whole K pass).
+ *                tau = 0 keeps everything (dense attention).
  *                Skipped positions still count in the softmax denominator.
  *   split_tokens as for kvq_resolve_split (0 = auto)
- *   options      0 or KVQ_OPT_SHARED_MAX; other bits are an error
+ *   options      0, KVQ_OPT_SHARED_MAX or KVQ_OPT_GLOBAL_MAX; other bits or both are an
+ *                error.  KVQ_OPT_GLOBAL_MAX needs every split of the request on its own
+ *                CTA at once (KVQ_ERR_UNSUPPORTED otherwise): the CTAs of a (sequence, KV
+ *                head) exchange their maxima through the workspace between the K pass
+ *                and the V pass (a bounded wait; KVQ_FLAG_TIMEOUT if it gives up).
  *   workspace    device, kvq_workspace_size(...) bytes, 16-byte aligned, initialized
  *                once with kvq_workspace_init.  Receives one partial (unnormalized o,
  *                running maximum m, denominator l) per cluster group.

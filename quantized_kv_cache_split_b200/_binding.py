@@ -29,6 +29,7 @@ KVQ_FMT_LUT4 = 2
 FORMATS = {"q8_0": KVQ_FMT_Q8_0, "q4_0": KVQ_FMT_Q4_0, "lut4": KVQ_FMT_LUT4}
 
 KVQ_OPT_SHARED_MAX = 1
+KVQ_OPT_GLOBAL_MAX = 2
 
 KVQ_FLAG_BAD_PAGE = 1
 KVQ_FLAG_BAD_SEQLEN = 2

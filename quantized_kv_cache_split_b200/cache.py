@@ -82,16 +82,18 @@ class QuantizedKVCache:
                   page_table: Optional[torch.Tensor] = None, max_pages: int = 1,
                   tau: float = 1e-6, sm_scale: Optional[float] = None, split_tokens: int = 0,
                   out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-                  shared_max: bool = False, fused: bool = True, stream=None) -> torch.Tensor:
+                  max_scope: str = "split", fused: bool = True, stream=None) -> torch.Tensor:
         """Decode attention of q [batch, num_q_heads, head_dim] (fp16) -> fp32 output.
 
         ``fused``: merge the split partials inside the decode kernel (one launch);
-        otherwise kvq_combine merges them in a second launch.  ``shared_max``: the
-        splits of a cluster share one running maximum for the skip test."""
+        otherwise kvq_combine merges them in a second launch.  ``max_scope``: the running
+        maximum the skip test uses: "split" (each split's own), "cluster" (shared by the
+        splits of a thread-block cluster) or "sequence" (over all splits of the
+        sequence and KV head)."""
         B, Hq, D = q.shape
         if sm_scale is None:
             sm_scale = 1.0 / math.sqrt(D)
-        opts = kb.KVQ_OPT_SHARED_MAX if shared_max else 0
+        opts = {"split": 0, "cluster": kb.KVQ_OPT_SHARED_MAX, "sequence": kb.KVQ_OPT_GLOBAL_MAX}[max_scope]
         ws, nbytes, L = self.workspace(B, Hq, max_seq_len, split_tokens, opts)
         if out is None:
             out = torch.empty((B, Hq, D), dtype=torch.float32, device=self.device)

@@ -63,7 +63,8 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads < 1 || max_seq_len < 0 || split_tokens < 0)
     return KVQ_ERR_INVALID_ARG;
-  if (options & ~KVQ_OPT_SHARED_MAX) return KVQ_ERR_INVALID_ARG;
+  if (options & ~(KVQ_OPT_SHARED_MAX | KVQ_OPT_GLOBAL_MAX)) return KVQ_ERR_INVALID_ARG;
+  if ((options & KVQ_OPT_SHARED_MAX) && (options & KVQ_OPT_GLOBAL_MAX)) return KVQ_ERR_INVALID_ARG;
   int L;
   if (split_tokens > 0) {
     L = std::min(split_tokens, KVQ_MAX_SPLIT_TOKENS);
@@ -240,7 +241,7 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.workspace = workspace;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.counters = reinterpret_cast<int*>(ws + kWorkspaceHeader);
-  a.generations = reinterpret_cast<uint32_t*>(a.counters + (size_t)batch * num_q_heads);
+  a.tallies = a.counters + (size_t)batch * num_q_heads;
   a.group_merge = 0;  // decided at launch
   const size_t n_part = (size_t)batch * num_q_heads * a.max_splits;
   a.part_o = reinterpret_cast<float*>(ws + kWorkspaceHeader + counters_bytes(batch, num_q_heads));
@@ -250,9 +251,12 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.out = out;
   a.cluster = CS;
   a.shared_max = (options & KVQ_OPT_SHARED_MAX) ? 1 : 0;
+  a.global_max = (options & KVQ_OPT_GLOBAL_MAX) ? 1 : 0;
   // clusters: at most one per (sequence, KV head, group of CS splits), at most what fits
   a.units_per_seq = (a.max_splits + CS - 1) / CS;
   const int64_t groups = (int64_t)batch * desc->num_kv_heads * a.units_per_seq;
+  // the maximum over all splits needs every split on its own CTA at once
+  if (a.global_max && groups > capacity) return KVQ_ERR_UNSUPPORTED;
   a.grid = (int)std::min<int64_t>(groups, capacity) * CS;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }

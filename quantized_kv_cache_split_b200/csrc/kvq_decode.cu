@@ -108,15 +108,18 @@ struct Layout {
   static constexpr size_t list = pk + (size_t)kWarps * 8 * kPkStride * 2;     // u8 [warps][64]
   static constexpr size_t red = list + (size_t)kWarps * kTile;                // float [2][warps][8]
   static constexpr size_t cnt = red + 2 * kWarps * 8 * 4;                     // int [2][warps]
-  static constexpr size_t cmx = cnt + 2 * kWarps * 4;                         // float [8] CTA maxima
-  static constexpr size_t mpart = cmx + 8 * 4;                                // float [8]
+  static constexpr size_t cmx = cnt + 2 * kWarps * 4;                         // float [2][8] maxima
+  static constexpr size_t mpart = cmx + 16 * 4;                               // float [8]
   static constexpr size_t lpart = mpart + 8 * 4;                              // float [8]
   static constexpr size_t octa = lpart + 8 * 4;                               // float [8][D]
   static constexpr size_t slen = octa + (size_t)8 * D * 4;                    // int [MAX_BATCH]
   static constexpr size_t misc = slen + KVQ_MAX_BATCH * 4;                     // int [4]
   static constexpr size_t mrg = misc + 16;                                     // float [2][8]
   static constexpr size_t scr = mrg + 64;                                      // float4 [warps][4][32] scores
-  static constexpr size_t base_total = scr + (size_t)kWarps * 4 * 32 * 16;
+  // query fragments shared by the warps: [words][32 lanes]
+  static constexpr int kQfWords = 2 * C::KSTEPS + (C::kLut ? 2 * C::KSTEPS : 0) + 2 * C::NBLK;
+  static constexpr size_t qfr = scr + (size_t)kWarps * 4 * 32 * 16;
+  static constexpr size_t base_total = qfr + (size_t)kQfWords * 32 * 4;
   // tau = 0 prefetches the V tile alongside K when shared memory allows
   static constexpr size_t vtile = (base_total + 127) / 128 * 128;             // [warps][VT]
   static constexpr bool kPrefetchV = vtile + (size_t)kWarps * C::VT + 128 <= kSmemLimit;
@@ -330,17 +333,57 @@ __device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
 }
 
 // ------------------------------------------------------------------ query fragments
-// Lane (r, c) of every warp builds, straight from the fp16 query in global memory, the
-// B fragments of the K pass for query head r of the group (null qh: a head the group
-// does not have), plus the offset correction of its accumulator heads 2c, 2c + 1
+// Lane (r, c) of every warp builds, from the fp16 query words it loaded (zeros for a
+// head the group does not have), the B fragments of the K pass for query head r, plus the offset correction of its accumulator heads 2c, 2c + 1
 // (q8_0 / q4_0) or the fp16 low parts of the rotated query (lut4).  The dims a lane
 // needs mirror how each format's A fragment is unpacked from one 32-bit word of codes:
 //   q8_0  k-step ks: dims 16 ks + 4c + {0, 2 | 1, 3}
 //   q4_0  k-step 2m + j: dims 32m + 8c + 2j + {0, 4 | 1, 5}
 //   lut4  k-step 2m + j: dims 32m + 8c + 4j + {0, 1 | 2, 3}
+// The raw query words a lane needs (loaded early, so that they lead the copy queue),
+// and for lut4 the rotation signs of its dims.
+template <int D>
+struct QRaw {
+  uint32_t w[D / 8];
+  uint32_t sg[D / 16];
+};
+
 template <int FMT, int D>
-__device__ __forceinline__ void build_query(const __half* __restrict__ qh,
-                                            const int8_t* __restrict__ signs, int c,
+__device__ __forceinline__ void load_query(const __half* __restrict__ qh,
+                                           const int8_t* __restrict__ signs, int c, QRaw<D>& q) {
+  using C = Cfg<FMT, D>;
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) q.w[i] = 0u;
+#pragma unroll
+  for (int i = 0; i < D / 16; ++i) q.sg[i] = 0u;
+  if (qh) {
+    if constexpr (C::kQ8) {
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(qh + 16 * ks + 4 * c));
+        q.w[2 * ks] = u.x;
+        q.w[2 * ks + 1] = u.y;
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < C::NBLK; ++m) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(qh + 32 * m + 8 * c));
+        q.w[4 * m] = u.x; q.w[4 * m + 1] = u.y; q.w[4 * m + 2] = u.z; q.w[4 * m + 3] = u.w;
+      }
+    }
+  }
+  if constexpr (C::kLut) {
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(signs + 32 * m + 8 * c));
+      q.sg[2 * m] = u.x;
+      q.sg[2 * m + 1] = u.y;
+    }
+  }
+}
+
+template <int FMT, int D>
+__device__ __forceinline__ void build_query(const QRaw<D>& q, int c,
                                             uint32_t (&qf)[D / 16][2], uint32_t (&ql)[D / 16][2],
                                             float (&corr)[D / 32][2]) {
   using C = Cfg<FMT, D>;
@@ -349,8 +392,7 @@ __device__ __forceinline__ void build_query(const __half* __restrict__ qh,
 #pragma unroll
     for (int m = 0; m < C::NBLK; ++m) {
       if constexpr (C::kQ4) {
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (qh) u = __ldg(reinterpret_cast<const uint4*>(qh + 32 * m + 8 * c));
+        const uint4 u = make_uint4(q.w[4 * m], q.w[4 * m + 1], q.w[4 * m + 2], q.w[4 * m + 3]);
         qf[2 * m][0] = prmt(u.x, u.z, 0x5410u);
         qf[2 * m][1] = prmt(u.x, u.z, 0x7632u);
         qf[2 * m + 1][0] = prmt(u.y, u.w, 0x5410u);
@@ -365,8 +407,7 @@ __device__ __forceinline__ void build_query(const __half* __restrict__ qh,
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const int ks = 2 * m + j;
-          uint2 u = make_uint2(0, 0);
-          if (qh) u = __ldg(reinterpret_cast<const uint2*>(qh + 16 * ks + 4 * c));
+          const uint2 u = make_uint2(q.w[2 * ks], q.w[2 * ks + 1]);
           qf[ks][0] = prmt(u.x, u.y, 0x5410u);
           qf[ks][1] = prmt(u.x, u.y, 0x7632u);
           const float2 f0 = __half22float2(u32_as_h2(u.x)), f1 = __half22float2(u32_as_h2(u.y));
@@ -392,10 +433,8 @@ __device__ __forceinline__ void build_query(const __half* __restrict__ qh,
     float y[C::NBLK][8];
 #pragma unroll
     for (int m = 0; m < C::NBLK; ++m) {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (qh) u = __ldg(reinterpret_cast<const uint4*>(qh + 32 * m + 8 * c));
-      const uint2 sg = __ldg(reinterpret_cast<const uint2*>(signs + 32 * m + 8 * c));
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      const uint2 sg = make_uint2(q.sg[2 * m], q.sg[2 * m + 1]);
+      const uint32_t w[4] = {q.w[4 * m], q.w[4 * m + 1], q.w[4 * m + 2], q.w[4 * m + 3]};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float2 f = __half22float2(u32_as_h2(w[i >> 1]));
@@ -622,7 +661,7 @@ decode_kernel(const DecodeArgs a) {
   float* red_l = red_m + kWarps * 8;
   int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
   int* cnt_kept = cnt_skip + kWarps;
-  float* cmx = reinterpret_cast<float*>(smem + LY::cmx);       // this CTA's maxima (log2)
+  float* cmx = reinterpret_cast<float*>(smem + LY::cmx);       // this CTA's maxima, then the sequence's (log2)
   float* mpart = reinterpret_cast<float*>(smem + LY::mpart);   // m of this CTA's partial
   float* lpart = reinterpret_cast<float*>(smem + LY::lpart);   // l of this CTA's partial
   float* octa = reinterpret_cast<float*>(smem + LY::octa);     // o of this CTA's partial [8][D]
@@ -712,6 +751,12 @@ decode_kernel(const DecodeArgs a) {
     }
     const int avail = k == 0 ? cap : nb;  // positions the copies may cover
 
+    // ---- warp 0 loads the query words first, ahead of the copies in the load queue
+    QRaw<D> qraw;
+    if (warp == 0)
+      load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr,
+                         a.desc.signs, c, qraw);
+
     // ---- K fetch (and, for tau = 0, the V tile): one copy group per 16-row job
     int row0 = -1;
     const int ncopy = min(kTile, avail - t0 - warp * kTile);
@@ -770,18 +815,51 @@ decode_kernel(const DecodeArgs a) {
       nvalid = 0;
     }
 
-    // ---- query fragments (overlap the copies in flight)
+    // ---- query fragments: warp 0 builds them once for the CTA while the copies are
+    //      in flight; every warp then reads its lane's words
     uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
     float corr[C::NBLK][2];
-    build_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr,
-                        a.desc.signs, c, qf, ql, corr);
+    uint32_t* qfr = reinterpret_cast<uint32_t*>(smem + LY::qfr);
+    constexpr int kQl = 2 * C::KSTEPS, kCorr = C::kLut ? 4 * C::KSTEPS : 2 * C::KSTEPS;
+    if (warp == 0) {
+      build_query<FMT, D>(qraw, c, qf, ql, corr);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        qfr[(2 * ks) * 32 + lane] = qf[ks][0];
+        qfr[(2 * ks + 1) * 32 + lane] = qf[ks][1];
+        if constexpr (C::kLut) {
+          qfr[(kQl + 2 * ks) * 32 + lane] = ql[ks][0];
+          qfr[(kQl + 2 * ks + 1) * 32 + lane] = ql[ks][1];
+        }
+      }
+      if constexpr (!C::kLut) {
+#pragma unroll
+        for (int m = 0; m < C::NBLK; ++m) {
+          qfr[(kCorr + 2 * m) * 32 + lane] = __float_as_uint(corr[m][0]);
+          qfr[(kCorr + 2 * m + 1) * 32 + lane] = __float_as_uint(corr[m][1]);
+        }
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+      qf[ks][0] = qfr[(2 * ks) * 32 + lane];
+      qf[ks][1] = qfr[(2 * ks + 1) * 32 + lane];
+      ql[ks][0] = C::kLut ? qfr[(kQl + 2 * ks) * 32 + lane] : 0u;
+      ql[ks][1] = C::kLut ? qfr[(kQl + 2 * ks + 1) * 32 + lane] : 0u;
+    }
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      corr[m][0] = C::kLut ? 0.f : __uint_as_float(qfr[(kCorr + 2 * m) * 32 + lane]);
+      corr[m][1] = C::kLut ? 0.f : __uint_as_float(qfr[(kCorr + 2 * m + 1) * 32 + lane]);
+    }
 
-    // ---- K pass: four 16-row jobs as their copies land.  Scores stay in registers;
-    //      each lane keeps a running maximum and sum 2^(s - m) for its two heads, so
-    //      the denominator needs no pass of its own.
+    // ---- K pass: four 16-row jobs as their copies land; scores to this lane's slots,
+    //      with the lane's largest and smallest valid score per head
     float4* scw = reinterpret_cast<float4*>(smem + LY::scr) + (size_t)warp * 4 * 32 + lane;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-#pragma unroll 1
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    float mn0 = INFINITY, mn1 = INFINITY;
+#pragma unroll
     for (int j = 0; j < 4; ++j) {
       if (16 * j >= nvalid) break;
       cp_async_wait_n(3 - j + (prefetch_v ? 1 : 0));
@@ -792,18 +870,11 @@ decode_kernel(const DecodeArgs a) {
       const float4 sv = make_float4(v0 ? s[0] * qk_scale : -INFINITY, v0 ? s[1] * qk_scale : -INFINITY,
                                     v1 ? s[2] * qk_scale : -INFINITY, v1 ? s[3] * qk_scale : -INFINITY);
       scw[j * 32] = sv;
-      const float n0 = fmaxf(m0, fmaxf(sv.x, sv.z));
-      const float n1 = fmaxf(m1, fmaxf(sv.y, sv.w));
-      if (n0 != -INFINITY) {
-        l0 = l0 * ex2(m0 - n0) + ex2(sv.x - n0) + ex2(sv.z - n0);
-        m0 = n0;
-      }
-      if (n1 != -INFINITY) {
-        l1 = l1 * ex2(m1 - n1) + ex2(sv.y - n1) + ex2(sv.w - n1);
-        m1 = n1;
-      }
+      mx0 = fmaxf(mx0, fmaxf(sv.x, sv.z));
+      mx1 = fmaxf(mx1, fmaxf(sv.y, sv.w));
+      mn0 = fminf(mn0, fminf(v0 ? sv.x : INFINITY, v1 ? sv.z : INFINITY));
+      mn1 = fminf(mn1, fminf(v0 ? sv.y : INFINITY, v1 ? sv.w : INFINITY));
     }
-    float mx0 = m0, mx1 = m1;
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
@@ -821,7 +892,43 @@ decode_kernel(const DecodeArgs a) {
       cmx[tid] = m;
     }
     if (CS > 1) cluster_sync(); else __syncthreads();  // CTA maxima visible (cluster-wide)
+    const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
+    int nbar = 0;  // group barriers this unit has passed (barrier k waits for k * n arrivals)
+    if (a.global_max) {
+      // every split of this (sequence, KV head) publishes its maxima in its partial's m
+      // slot; after a barrier among them, each reads all and takes the largest
+      const int n = (nb + Ls - 1) / Ls;
+      if (tid < G) a.part_m[slot0 + (size_t)tid * a.max_splits] = cmx[tid];
+      __syncthreads();
+      ++nbar;
+      if (tid == 0) {
+        misc[1] = cta_group_arrive_wait(a.counters + (size_t)b * hkv + kvh, nbar * n);
+        if (!(a.out && a.group_merge))  // no second barrier follows
+          cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
+      }
+      __syncthreads();
+      if (misc[1]) {
+        __threadfence();
+        if (warp < G) {
+          const size_t uw = ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits;
+          float M = -INFINITY;
+          for (int u = lane; u < n; u += 32) M = fmaxf(M, __ldcg(a.part_m + uw + u));
+#pragma unroll
+          for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          if (lane == 0) cmx[8 + warp] = M;
+        }
+      } else if (tid == 0) {
+        set_flag(flags, KVQ_FLAG_TIMEOUT);
+      }
+      __syncthreads();
+    }
+    // (with the maximum over all splits, a fast CTA may already have replaced its
+    // published maxima by the final one in its m slot: the same largest value)
     float mh0 = cmx[2 * c], mh1 = cmx[2 * c + 1];
+    if (a.global_max && misc[1]) {
+      mh0 = cmx[8 + 2 * c];
+      mh1 = cmx[8 + 2 * c + 1];
+    }
     if (CS > 1 && a.shared_max) {
       for (int rk = 0; rk < CS; ++rk) {
         if (rk == (int)rank) continue;
@@ -833,27 +940,58 @@ decode_kernel(const DecodeArgs a) {
       mpart[2 * c] = mh0;
       mpart[2 * c + 1] = mh1;
     }
-    // denominator: each lane's running sum rescaled to the decision maximum
-    l0 = (m0 != -INFINITY) ? l0 * ex2(m0 - mh0) : 0.f;
-    l1 = (m1 != -INFINITY) ? l1 * ex2(m1 - mh1) : 0.f;
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    }
 
-    // ---- skip test and compaction into this warp's list (rows r, r + 8 of each job;
-    //      heads 2c, 2c + 1); weights are computed for kept pairs only
+    // ---- skip test.  When every valid pair of the warp's tile is kept (the smallest
+    //      scores pass), the V tile is copied at once and the weights go to row
+    //      positions; otherwise kept positions are compacted into this warp's list (rows
+    //      r, r + 8 of each job; heads 2c, 2c + 1).  Weights only for kept pairs.
+    const bool all_kept = nvalid > 0 &&
+                          __all_sync(0xffffffffu, (!hl0 || mn0 - mh0 >= thr) && (!hl1 || mn1 - mh1 >= thr));
+    if (all_kept && !prefetch_v) {
+      __syncwarp();  // every lane is done reading the K tile
+      const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
+#pragma unroll 4
+      for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(kbuf + i * 16, vsrc + i * 16);
+      const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
+#pragma unroll
+      for (int i = lane; i < C::STAGE_SC / 16; i += 32)
+        cp_async16(kbuf + C::STAGE_CODE + i * 16, vssrc + i * 16);
+      cp_async_commit();
+    }
+    // the weights 2^(s - m) of every valid pair also give the denominator l
     int nkept = 0, nskip = 0;
-#pragma unroll 1
+    float l0 = 0.f, l1 = 0.f;
+    if (all_kept) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (16 * j >= nvalid) break;
+        const float4 sv = scw[j * 32];
+        const int ra = 16 * j + r, rb = ra + 8;
+        const bool va = ra < nvalid, vb = rb < nvalid;
+        const float ea0 = va && hl0 ? ex2(sv.x - mh0) : 0.f, ea1 = va && hl1 ? ex2(sv.y - mh1) : 0.f;
+        const float eb0 = vb && hl0 ? ex2(sv.z - mh0) : 0.f, eb1 = vb && hl1 ? ex2(sv.w - mh1) : 0.f;
+        l0 += ea0 + eb0;
+        l1 += ea1 + eb1;
+        pk_w[(2 * c) * kPkStride + ra] = __float2half_rn(ea0 * kPScale);
+        pk_w[(2 * c + 1) * kPkStride + ra] = __float2half_rn(ea1 * kPScale);
+        pk_w[(2 * c) * kPkStride + rb] = __float2half_rn(eb0 * kPScale);
+        pk_w[(2 * c + 1) * kPkStride + rb] = __float2half_rn(eb1 * kPScale);
+      }
+      nkept = nvalid;
+    }
+#pragma unroll
     for (int j = 0; j < 4; ++j) {
-      if (16 * j < nvalid) {
+      if (!all_kept && 16 * j < nvalid) {
         const int ra = 16 * j + r, rb = ra + 8;
         const bool va = ra < nvalid, vb = rb < nvalid;
         const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
         const float4 sv = scw[j * 32];
         const float da0 = sv.x - mh0, da1 = sv.y - mh1;
         const float db0 = sv.z - mh0, db1 = sv.w - mh1;
+        const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
+        const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
+        l0 += ea0 + eb0;
+        l1 += ea1 + eb1;
         const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
         const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
         nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
@@ -863,20 +1001,25 @@ decode_kernel(const DecodeArgs a) {
         if ((rows_a >> (4 * r)) & 1u) {
           const int slot = nkept + __popc(rows_a & below);
           if (c == 0) list_w[slot] = (uint8_t)ra;
-          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(ka0 ? ex2(da0) * kPScale : 0.f);
-          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(ka1 ? ex2(da1) * kPScale : 0.f);
+          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(ka0 ? ea0 * kPScale : 0.f);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(ka1 ? ea1 * kPScale : 0.f);
         }
         if ((rows_b >> (4 * r)) & 1u) {
           const int slot = nkept + na + __popc(rows_b & below);
           if (c == 0) list_w[slot] = (uint8_t)rb;
-          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(kb0 ? ex2(db0) * kPScale : 0.f);
-          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(kb1 ? ex2(db1) * kPScale : 0.f);
+          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(kb0 ? eb0 * kPScale : 0.f);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(kb1 ? eb1 * kPScale : 0.f);
         }
         nkept += na + __popc(rows_b);
       }
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
     if (r == 0) {
       red_l[warp * 8 + 2 * c] = l0;
       red_l[warp * 8 + 2 * c + 1] = l1;
@@ -896,8 +1039,8 @@ decode_kernel(const DecodeArgs a) {
       if (prefetch_v || nkept == nvalid) {
         // every valid row is kept, so slot s is tile row s; without the prefetched tile,
         // one contiguous copy of the V tile into the (now free) K buffer
-        const uint8_t* vt = vtile;
-        if (!prefetch_v) {
+        const uint8_t* vt = prefetch_v ? vtile : kbuf;
+        if (!prefetch_v && !all_kept) {
           __syncwarp();  // every lane is done reading the K tile
           const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
 #pragma unroll 4
@@ -907,11 +1050,10 @@ decode_kernel(const DecodeArgs a) {
           for (int i = lane; i < C::STAGE_SC / 16; i += 32)
             cp_async16(kbuf + C::STAGE_CODE + i * 16, vssrc + i * 16);
           cp_async_commit();
-          vt = kbuf;
         }
         cp_async_wait<0>();
         __syncwarp();
-#pragma unroll 1
+#pragma unroll 2
         for (int g = 0; g < ng; ++g)
           v_group<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
                                 min(16, nkept - 16 * g), r, c, lut, acc);
@@ -930,7 +1072,7 @@ decode_kernel(const DecodeArgs a) {
         cp_async_commit();
         cp_async_wait<0>();
         __syncwarp();
-#pragma unroll 1
+#pragma unroll 2
         for (int g = 0; g < ng; ++g)
           v_group<FMT, D, false>(kbuf + g * C::VGROUP, pk_w + r * kPkStride + 16 * g, list_w + 16 * g,
                                  0, min(16, nkept - 16 * g), r, c, lut, acc);
@@ -947,7 +1089,6 @@ decode_kernel(const DecodeArgs a) {
 
     // ---- this CTA's partial: sum the accumulators of the warps that kept something.
     //      A lone CTA writes it straight to the workspace; a cluster merges first.
-    const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
     for (int q = tid; q < 32 * C::NE; q += kThreads) {
       const int ln = q & 31, e = q >> 5;
       const int mt = e >> 2, i = e & 3;
@@ -1025,8 +1166,7 @@ decode_kernel(const DecodeArgs a) {
       if (a.out) __threadfence();
       cluster_sync();  // no CTA reuses its shared partial before the others have read it
     } else if (a.out) {
-      __threadfence();
-      __syncthreads();
+      __syncthreads();  // the partial is written (the arrival below publishes it)
     }
 
     // ---- in-kernel merge.  When every unit has its own CTA, the CTAs of this
@@ -1034,9 +1174,11 @@ decode_kernel(const DecodeArgs a) {
     //      otherwise the last cluster to finish the pair merges all of its heads.
     if (a.out && a.group_merge) {
       const int n = (nb + Ls - 1) / Ls;  // splits (CTAs) of this (sequence, KV head)
-      if (tid == 0)
-        misc[0] = cta_group_barrier(a.counters + (size_t)b * hkv + kvh,
-                                    a.generations + (size_t)b * hkv + kvh, n);
+      ++nbar;
+      if (tid == 0) {
+        misc[0] = cta_group_arrive_wait(a.counters + (size_t)b * hkv + kvh, nbar * n);
+        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
+      }
       __syncthreads();
       if (misc[0]) {
         __threadfence();
@@ -1073,7 +1215,7 @@ decode_kernel(const DecodeArgs a) {
         const bool act = tid < 2 * nq;
         const int h = qq / (D / 4), d4 = qq - h * (D / 4);
         const size_t uh = u0 + (size_t)h * a.max_splits;
-        constexpr int kBatch = 20;  // partials per thread whose loads are in flight together
+        constexpr int kBatch = C::kLut ? 12 : 20;  // partials per thread whose loads are in flight together
         float4 o4[kBatch];
 #pragma unroll
         for (int t = 0; t < kBatch; ++t) {
@@ -1276,7 +1418,7 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
                   (int64_t)a.batch * a.units_per_seq * a.desc.num_kv_heads <= a.grid;
   int na = 0;
   if (a.cluster > 1) attr[na++] = attr[0];
-  if (b.group_merge) {
+  if (b.group_merge || a.global_max) {  // CTAs wait for one another: all resident together
     attr[na].id = cudaLaunchAttributeCooperative;
     attr[na].val.cooperative = 1;
   } else {

@@ -179,25 +179,35 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-// A barrier among the `n` CTAs that share (counter, generation), called by one thread
-// of each CTA after its writes are fenced.  The last to arrive resets the counter and
-// advances the generation; the others wait for the generation to change, for at most
-// kWaitCycles.  Returns false if the wait gave up.
-__device__ __forceinline__ bool cta_group_barrier(int* counter, uint32_t* generation, int n) {
-  const uint32_t g0 = ld_acquire_gpu(generation);
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier k (k = 1, 2, ...) among the CTAs that share `counter`, called by one thread of
+// each CTA after a block barrier: a fenced increment (publishing every write the CTA
+// made before that block barrier), then a wait until all `target` = k * n arrivals are
+// in, for at most kWaitCycles.  Returns false if the wait gave up.
+__device__ __forceinline__ bool cta_group_arrive_wait(int* counter, int target) {
+  __threadfence();
   const int old = atomicAdd(counter, 1);
-  if (old == n - 1) {
-    atomicExch(counter, 0);
-    __threadfence();
-    atomicAdd(generation, 1u);
-    return true;
-  }
+  if (old + 1 >= target) return true;
   const long long t0 = clock64();
-  while (ld_acquire_gpu(generation) == g0) {
+  while (ld_acquire_gpu(counter) < target) {
     if (clock64() - t0 > kWaitCycles) return false;
-    __nanosleep(64);
+    __nanosleep(32);
   }
   return true;
+}
+
+// Called by one thread of each of the `n` CTAs once it no longer waits on `counter`:
+// the last of them zeroes the counter (and this tally) for the next launch.
+__device__ __forceinline__ void cta_group_done(int* counter, int* tally, int n) {
+  if (atomicAdd(tally, 1) == n - 1) {
+    atomicExch(counter, 0);
+    atomicExch(tally, 0);
+  }
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -35,16 +35,17 @@ struct DecodeArgs {
   float* out;         // non-null: merge in the same kernel and write the output
   int cluster;        // consecutive splits per thread-block cluster (1, 2 or 4)
   int shared_max;     // the splits of a cluster share one running maximum
+  int global_max;     // every split of a (sequence, KV head) uses the maximum over all of them
   int grid;           // CTAs launched (a multiple of cluster)
   int units_per_seq;  // cluster groups of one (sequence, KV head) at max_seq_len
   int group_merge;    // every unit has its own CTA: the CTAs of a (sequence, KV head) meet
                       // at a barrier and each merges some of its heads
-  uint32_t* generations;  // [batch][num_kv_heads] barrier generations (group_merge)
+  int* tallies;       // [batch][num_kv_heads] CTAs done with the group barriers
 };
 
-// Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits); the merge counters and the
-// barrier generations (int32 [batch][num_q_heads] each reserved, together rounded up to
-// 256 bytes); then the partials, one slot per cluster of splits:
+// Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits); the merge / barrier counters
+// and the barrier tallies (int32 [batch][num_q_heads] each reserved, together rounded up
+// to 256 bytes); then the partials, one slot per cluster of splits:
 //   o [batch][num_q_heads][max_splits][head_dim] fp32 (unnormalized)
 //   m [batch][num_q_heads][max_splits] fp32 (running maximum, log2 units)
 //   l [batch][num_q_heads][max_splits] fp32

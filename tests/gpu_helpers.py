@@ -19,10 +19,11 @@ def codebook_for(D: int) -> np.ndarray:
 
 
 def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=None,
-                shared_max: bool = False, fused: bool = True):
+                max_scope: str = "split", fused: bool = True):
     """One decode step through the C ABI.  ``fused``: the merge runs inside the decode
-    kernel; otherwise kvq_combine runs it.  ``shared_max``: the splits of a cluster
-    share one running maximum (the oracle replays it with share = the cluster size)."""
+    kernel; otherwise kvq_combine runs it.  ``max_scope``: "split", "cluster" (the
+    splits of a cluster share one running maximum; the oracle replays it with share =
+    the cluster size) or "sequence" (share = every split)."""
     import quantized_kv_cache_split_b200 as K
     wl = inp.wl
     D, Hkv = wl.head_dim, wl.num_kv_heads
@@ -42,15 +43,16 @@ def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=Non
     max_seq = int(max(inp.seq_lens.max(), 1))
     out = cache.attention(q, seq, max_seq, pt, inp.max_pages, tau=tau,
                           sm_scale=float(np.float32(1.0 / math.sqrt(D))),
-                          split_tokens=split_tokens, stats=stats, shared_max=shared_max,
+                          split_tokens=split_tokens, stats=stats, max_scope=max_scope,
                           fused=fused)
     torch.cuda.synchronize()
-    opts = K.KVQ_OPT_SHARED_MAX if shared_max else 0
+    opts = {"split": 0, "cluster": K.KVQ_OPT_SHARED_MAX, "sequence": K.KVQ_OPT_GLOBAL_MAX}[max_scope]
     L = K.kvq_resolve_split(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens, opts)
     CS = K.kvq_resolve_cluster(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens, opts)
     flags = cache.device_flags()
     return dict(out=out.cpu().numpy().astype(np.float64), stats=stats.cpu().numpy(), split=L,
-                cluster=CS, share=CS if shared_max else 1, flags=flags, cache=cache)
+                cluster=CS, share={"split": 1, "cluster": CS, "sequence": 1 << 30}[max_scope],
+                flags=flags, cache=cache)
 
 
 def run_oracle(inp: W.Inputs, tau: float, split: int, codebook16=None, groups=None, share: int = 1):

@@ -87,11 +87,35 @@ def test_decode_parity_shared_max(name, tau, split):
     wl = W.WORKLOADS[name]
     inp = W.generate(wl)
     cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
-    g = run_library(inp, tau, split, cb, shared_max=True)
+    g = run_library(inp, tau, split, cb, max_scope="cluster")
     assert g["share"] > 1
     o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
     check_parity(inp, g, o, tau)
     assert g["flags"] == 0
+
+
+@pytest.mark.parametrize("name,tau,split", [
+    ("tiny_q8_d64", 1e-6, 64), ("gqa_4k_q8", 1e-6, 0), ("lut_4k", 1e-6, 0), ("lut_4k", 1e-2, 512),
+    ("gqa_4k_q8", 0.0, 256)])
+def test_decode_parity_sequence_max(name, tau, split):
+    # every split uses the maximum over all splits of its sequence (the final maximum)
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
+    g = run_library(inp, tau, split, cb, max_scope="sequence")
+    o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+
+
+def test_sequence_max_rejects_requests_beyond_one_round():
+    # more splits than CTAs that run at once: the maxima cannot be exchanged in one launch
+    import quantized_kv_cache_split_b200 as K
+    desc = K.make_desc("q8_0", 128, 8, 4096, 64)
+    fake = 1 << 20  # never dereferenced: the call is refused before any launch
+    st = K.kvq_decode_attn(desc, fake, 64, 32, fake, fake, fake, fake, None, 1, fake, 4096, 0.088,
+                           1e-6, 64, fake, 1 << 40, options=K.KVQ_OPT_GLOBAL_MAX, check=False)
+    assert st == K.KVQ_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("name,tau", [("gqa_4k_q8", 1e-6), ("lut_4k", 0.0), ("tiny_q8_d64", 1e-6)])
@@ -134,14 +158,15 @@ RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 
 
 @pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
-@pytest.mark.parametrize("tau,split,shared", [(0.0, 128, False), (1e-6, 0, False), (1e-4, 192, False),
-                                              (1e-6, 1024, False), (1e-6, 128, True)])
-def test_decode_parity_paged_ragged(fmt, tau, split, shared):
+@pytest.mark.parametrize("tau,split,scope", [(0.0, 128, "split"), (1e-6, 0, "split"), (1e-4, 192, "split"),
+                                             (1e-6, 1024, "split"), (1e-6, 128, "cluster"),
+                                             (1e-6, 0, "sequence")])
+def test_decode_parity_paged_ragged(fmt, tau, split, scope):
     base = W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt)
     wl = W.shrink(base, RAGGED_LENS, n_planted=8)
     inp = W.generate(wl)
     cb = codebook_for(wl.head_dim) if fmt == "lut4" else None
-    g = run_library(inp, tau, split, cb, shared_max=shared)
+    g = run_library(inp, tau, split, cb, max_scope=scope)
     o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
     check_parity(inp, g, o, tau)
     assert g["flags"] == 0
@@ -163,12 +188,13 @@ def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
 # ------------------------------------------------------------------ full sizes
 
 @pytest.mark.parametrize("name", ["gqa_32k_q4", "lut_32k"])
-@pytest.mark.parametrize("tau,shared", [(1e-6, False), (0.0, False), (1e-6, True)])
-def test_decode_parity_full_32k(name, tau, shared):
+@pytest.mark.parametrize("tau,scope", [(1e-6, "split"), (0.0, "split"), (1e-6, "cluster"),
+                                       (1e-6, "sequence")])
+def test_decode_parity_full_32k(name, tau, scope):
     wl = W.WORKLOADS[name]
     inp = W.generate(wl)
     cb = codebook_for(wl.head_dim) if wl.fmt == "lut4" else None
-    g = run_library(inp, tau, 0, cb, shared_max=shared)
+    g = run_library(inp, tau, 0, cb, max_scope=scope)
     o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
     check_parity(inp, g, o, tau)
     if tau > 0:

@@ -177,15 +177,20 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                and the V pass (a bounded wait; KVQ_FLAG_TIMEOUT if it gives up).
  *   workspace    device, kvq_workspace_size(...) bytes, 16-byte aligned, initialized
  *                once with kvq_workspace_init.  Receives one partial (unnormalized o,
- *                running maximum m, denominator l) per cluster group.
+ *                running maximum m, denominator l) per cluster group (with `out` given,
+ *                o may be left unwritten).
  *   stats        device uint64 [4] or NULL; ADDED to (caller zeroes):
  *                [0] (position, query head) pairs scored, [1] pairs skipped,
  *                [2] V rows read (positions kept by any head of the group),
  *                [3] V rows skipped
- *   out          device fp32 [batch][num_q_heads][head_dim], 16-byte aligned, or NULL.  When given, the
- *                same kernel also merges the partials (as kvq_combine does: the last
- *                cluster to finish a (sequence, KV head) merges it) and writes the
- *                output; calls that share a workspace must not overlap on the GPU.
+ *   out          device fp32 [batch][num_q_heads][head_dim], 16-byte aligned, or NULL.
+ *                When given, the same kernel also merges the splits and writes the
+ *                output (the log-sum-exp rule of kvq_combine): when every split of the
+ *                request runs on its own CTA at once, each split adds its normalized
+ *                share into the output with floating-point atomics (so the last bits of
+ *                the output may differ from run to run); otherwise the last cluster to
+ *                finish a (sequence, KV head) merges it.  Calls that share a workspace
+ *                must not overlap on the GPU.
  * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
  * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.
  */

@@ -133,8 +133,6 @@ struct Layout {
                 "alignment");
   // the merges' scratch reuses the staging buffers
   static_assert((size_t)kWarps * C::KBUF >= (size_t)8 * kMergeCap * 4, "merge weights");
-  static_assert((size_t)kWarps * C::KBUF >= (size_t)kThreads * 16 + 2 * kMergeCap * 4 + D * 4 + 16,
-                "group merge scratch");
 };
 
 // cp.async.wait_group with a count known only after unrolling
@@ -541,114 +539,6 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const _
     mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
 }
 
-// ------------------------------------------------------------------ merge of one head
-// Log-sum-exp merge of the n partials of one query head (partial u at slot uh + u):
-//   M = max_u m_u,  out = sum_u 2^(m_u - M) o_u / sum_u 2^(m_u - M) l_u
-// (lut4: rotated back, out = s .* (c H out')), written to out_row.  The whole CTA takes
-// part: thread t handles float4 column t % (D/4) of partials t / (D/4), t / (D/4) + NG,
-// ...; every load is issued before the first wait.  Scratch: wm, wl [kMergeCap] floats,
-// red [kThreads] float4, hv [D] floats, den [1].
-template <int FMT, int D>
-__device__ __forceinline__ void merge_head(const DecodeArgs& a, size_t uh, int n, float* out_row,
-                                        float* wm, float* wl, float4* red, float* hv, float* den_s) {
-  using C = Cfg<FMT, D>;
-  constexpr int NC = D / 4;           // float4 columns of a head
-  constexpr int NG = kThreads / NC;   // groups of partials
-  constexpr int kPer = 4;             // partials per thread loaded together
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int d4 = tid % NC, ug = tid / NC;
-  if (tid < n) {
-    wm[tid] = __ldcg(a.part_m + uh + tid);
-    wl[tid] = __ldcg(a.part_l + uh + tid);
-  }
-  float4 o4[kPer];
-#pragma unroll
-  for (int t = 0; t < kPer; ++t) {
-    const int u = ug + t * NG;
-    o4[t] = u < n ? __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4)
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  __syncthreads();
-  if (warp == 0) {  // maximum, weights (in place of the maxima) and denominator
-    float M = -INFINITY;
-    for (int u = lane; u < n; u += 32) M = fmaxf(M, wm[u]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
-    for (int u = lane; u < n; u += 32) {
-      const float w = ex2(wm[u] - M);
-      wm[u] = w;
-      den = fmaf(w, wl[u], den);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) den_s[0] = den;
-  }
-  __syncthreads();
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-  for (int t = 0; t < kPer; ++t) {
-    const int u = ug + t * NG;
-    if (u < n) {
-      const float w = wm[u];
-      acc.x = fmaf(w, o4[t].x, acc.x); acc.y = fmaf(w, o4[t].y, acc.y);
-      acc.z = fmaf(w, o4[t].z, acc.z); acc.w = fmaf(w, o4[t].w, acc.w);
-    }
-  }
-  for (int u = ug + kPer * NG; u < n; u += NG) {  // more partials than one batch
-    const float w = wm[u];
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(a.part_o + (uh + u) * D) + d4);
-    acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-    acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-  }
-  red[ug * NC + d4] = acc;
-  __syncthreads();
-  if (tid < NC) {
-    float4 v = red[tid];
-#pragma unroll 4
-    for (int g = 1; g < NG; ++g) {
-      const float4 x = red[g * NC + tid];
-      v.x += x.x; v.y += x.y; v.z += x.z; v.w += x.w;
-    }
-    const float inv = 1.f / den_s[0];
-    v = make_float4(v.x * inv, v.y * inv, v.z * inv, v.w * inv);
-    if constexpr (C::kLut) reinterpret_cast<float4*>(hv)[tid] = v;
-    else reinterpret_cast<float4*>(out_row)[tid] = v;
-  }
-  if constexpr (C::kLut) {
-    __syncthreads();
-    if (warp == 0) {  // out = s .* (c H out')
-      constexpr int K = D / 32;
-      float y[K];
-#pragma unroll
-      for (int kk = 0; kk < K; ++kk) y[kk] = hv[32 * kk + lane];
-#pragma unroll
-      for (int hb = 1; hb < 32; hb <<= 1) {
-        const bool upper = (lane & hb) != 0;
-#pragma unroll
-        for (int kk = 0; kk < K; ++kk) {
-          const float t = __shfl_xor_sync(0xffffffffu, y[kk], hb);
-          y[kk] = upper ? (t - y[kk]) : (y[kk] + t);
-        }
-      }
-#pragma unroll
-      for (int hb = 1; hb < K; hb <<= 1)
-#pragma unroll
-        for (int kk = 0; kk < K; ++kk)
-          if (!(kk & hb)) {
-            const float u = y[kk], v = y[kk + hb];
-            y[kk] = u + v;
-            y[kk + hb] = u - v;
-          }
-      const float cs = D == 64 ? 0.125f : 0.08838834764831845f;
-#pragma unroll
-      for (int kk = 0; kk < K; ++kk)
-        out_row[32 * kk + lane] = y[kk] * cs * (float)a.desc.signs[32 * kk + lane];
-    }
-  }
-  __syncthreads();  // scratch free again
-}
-
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1030,6 +920,27 @@ decode_kernel(const DecodeArgs a) {
     }
     __syncwarp();  // the warp's list and weights are complete
 
+    // ---- additive in-kernel merge (every split on its own CTA): the split publishes its
+    //      (m, l) and arrives at its (sequence, KV head) barrier now, so that the wait
+    //      overlaps its V work; split 0 clears the output rows that the splits add into
+    const bool add_merge = a.out && a.group_merge;
+    const int nsplit = (nb + Ls - 1) / Ls;
+    if (add_merge) {
+      __syncthreads();  // every warp's l is in shared memory
+      if (tid < G) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mpart[tid];
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+      }
+      if (cu == 0)
+        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
+      __syncthreads();
+      ++nbar;
+      if (tid == 0) cta_group_arrive(a.counters + (size_t)b * hkv + kvh);
+    }
+
     // ---- V pass: this warp's kept positions only
     if (nkept > 0) {
       float acc[C::MT][4];
@@ -1100,11 +1011,11 @@ decode_kernel(const DecodeArgs a) {
         for (int w = 0; w < kWarps; ++w)
           if (cnt_kept[w] > 0) v += reinterpret_cast<const float*>(smem + LY::kbuf + (size_t)w * C::KBUF)[q];
         v *= kPUnscale;
-        if (CS > 1) octa[h * D + dim] = v;
+        if (CS > 1 || add_merge) octa[h * D + dim] = v;
         else a.part_o[(slot0 + (size_t)h * a.max_splits) * D + dim] = v;
       }
     }
-    if (tid < G) {
+    if (tid < G && !add_merge) {
       float l = 0.f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
@@ -1169,30 +1080,82 @@ decode_kernel(const DecodeArgs a) {
       __syncthreads();  // the partial is written (the arrival below publishes it)
     }
 
-    // ---- in-kernel merge.  When every unit has its own CTA, the CTAs of this
-    //      (sequence, KV head) meet at a barrier and CTA s merges heads s, s + n, ...;
-    //      otherwise the last cluster to finish the pair merges all of its heads.
-    if (a.out && a.group_merge) {
-      const int n = (nb + Ls - 1) / Ls;  // splits (CTAs) of this (sequence, KV head)
-      ++nbar;
+    // ---- in-kernel merge.  When every split has its own CTA, each adds its share
+    //      o_s 2^(m_s - M) / L (M, L over all splits, read once every split has
+    //      published its (m, l)) into the output; otherwise the last cluster to finish
+    //      the (sequence, KV head) merges the written partials by the log-sum-exp rule.
+    if (add_merge) {
       if (tid == 0) {
-        misc[0] = cta_group_arrive_wait(a.counters + (size_t)b * hkv + kvh, nbar * n);
-        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
+        misc[0] = cta_group_wait(a.counters + (size_t)b * hkv + kvh, nbar * nsplit);
+        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, nsplit);
       }
       __syncthreads();
       if (misc[0]) {
         __threadfence();
-        uint8_t* scratch = smem + LY::kbuf;  // free: every warp's accumulators are summed
-        for (int h = cu; h < G; h += n)
-          merge_head<FMT, D>(a, ((size_t)b * Hq + (size_t)kvh * G + h) * a.max_splits, n,
-                             a.out + ((size_t)b * Hq + (size_t)kvh * G + h) * D,
-                             reinterpret_cast<float*>(scratch + kThreads * 16),
-                             reinterpret_cast<float*>(scratch + kThreads * 16 + kMergeCap * 4),
-                             reinterpret_cast<float4*>(scratch),
-                             reinterpret_cast<float*>(scratch + kThreads * 16 + 2 * kMergeCap * 4),
-                             reinterpret_cast<float*>(scratch + kThreads * 16 + 2 * kMergeCap * 4 + D * 4));
+        if (warp < G) {  // this split's share of head `warp`: 2^(m_s - M) / L
+          const size_t uw = ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits;
+          float M = -INFINITY, L = 0.f;
+          for (int ub = 0; ub < nsplit; ub += 64) {
+            const int ua = ub + lane, uc = ub + 32 + lane;
+            const float ma = ua < nsplit ? __ldcg(a.part_m + uw + ua) : -INFINITY;
+            const float mc = uc < nsplit ? __ldcg(a.part_m + uw + uc) : -INFINITY;
+            const float la = ua < nsplit ? __ldcg(a.part_l + uw + ua) : 0.f;
+            const float lc = uc < nsplit ? __ldcg(a.part_l + uw + uc) : 0.f;
+            float bm = fmaxf(ma, mc);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float nm = fmaxf(M, bm);
+            float ds = (ma == -INFINITY ? 0.f : ex2(ma - nm) * la) + (mc == -INFINITY ? 0.f : ex2(mc - nm) * lc);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + ds;
+            M = nm;
+          }
+          if (lane == 0) cmx[8 + warp] = ex2(mpart[warp] - M) / L;
+        }
       } else if (tid == 0) {
         set_flag(flags, KVQ_FLAG_TIMEOUT);
+      }
+      __syncthreads();  // the coefficients (and this CTA's o) are in shared memory
+      if (misc[0]) {
+        if constexpr (C::kLut) {  // rotate the scaled rows back: s .* (c H (coef * o'))
+          if (warp < G) {
+            constexpr int K = D / 32;
+            const float coef = cmx[8 + warp] * (D == 64 ? 0.125f : 0.08838834764831845f);
+            float y[K];
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk) y[kk] = octa[warp * D + 32 * kk + lane] * coef;
+#pragma unroll
+            for (int hb = 1; hb < 32; hb <<= 1) {
+              const bool upper = (lane & hb) != 0;
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk) {
+                const float t = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+                y[kk] = upper ? (t - y[kk]) : (y[kk] + t);
+              }
+            }
+#pragma unroll
+            for (int hb = 1; hb < K; hb <<= 1)
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk)
+                if (!(kk & hb)) {
+                  const float u = y[kk], v = y[kk + hb];
+                  y[kk] = u + v;
+                  y[kk + hb] = u - v;
+                }
+#pragma unroll
+            for (int kk = 0; kk < K; ++kk)
+              octa[warp * D + 32 * kk + lane] = y[kk] * (float)a.desc.signs[32 * kk + lane];
+          }
+          __syncthreads();
+        }
+        float* orow = a.out + ((size_t)b * Hq + (size_t)kvh * G) * D;
+        for (int q4 = tid; q4 < G * D / 4; q4 += kThreads) {
+          const int h = q4 / (D / 4);
+          const float coef = C::kLut ? 1.f : cmx[8 + h];
+          const float4 v = reinterpret_cast<const float4*>(octa)[q4];
+          red_add_f32x4(orow + 4 * q4, make_float4(v.x * coef, v.y * coef, v.z * coef, v.w * coef));
+        }
       }
     } else if (a.out && rank == 0) {
       const int ncu = ((nb + Ls - 1) / Ls + CS - 1) / CS;  // partials of sequence b

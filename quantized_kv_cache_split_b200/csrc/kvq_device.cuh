@@ -201,6 +201,27 @@ __device__ __forceinline__ bool cta_group_arrive_wait(int* counter, int target) 
   return true;
 }
 
+// The two halves of cta_group_arrive_wait, for work that overlaps the wait.
+__device__ __forceinline__ void cta_group_arrive(int* counter) {
+  __threadfence();
+  atomicAdd(counter, 1);
+}
+__device__ __forceinline__ bool cta_group_wait(const int* counter, int target) {
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(counter) < target) {
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// out[0..3] += v, one vector reduction in global memory (16-byte aligned address).
+__device__ __forceinline__ void red_add_f32x4(float* out, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 // Called by one thread of each of the `n` CTAs once it no longer waits on `counter`:
 // the last of them zeroes the counter (and this tally) for the next launch.
 __device__ __forceinline__ void cta_group_done(int* counter, int* tally, int n) {

@@ -282,10 +282,11 @@ def time_steps(runner, steps, warmup, world, sampler=None):
     return start.elapsed_time(end)
 
 
-def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int):
+def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int, with_o: bool):
     """HBM bytes one fused decode launch must move: every K row, the kept V rows, Q,
     the page table, the partials (one per cluster of splits, written once and read
-    once by the in-kernel merge) and the output."""
+    once by the in-kernel merge: (m, l) only when each split adds its share into the
+    output itself, also o when a last cluster merges) and the output."""
     import quantized_kv_cache_split_b200 as K
     wl = rep.wl
     row = K.kvq_code_row_bytes(wl.fmt, wl.head_dim) + 2 * K.kvq_scale_row_count(wl.fmt, wl.head_dim)
@@ -295,7 +296,7 @@ def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int):
     q_bytes = wl.batch * wl.num_q_heads * wl.head_dim * 2
     pt_bytes = 0 if rep.inp.page_table is None else sum(
         (int(n) + rep.inp.page_size - 1) // rep.inp.page_size for n in rep.inp.seq_lens) * 4
-    part_bytes = 2 * n_partials * wl.group * (wl.head_dim + 2) * 4
+    part_bytes = 2 * n_partials * wl.group * ((wl.head_dim if with_o else 0) + 2) * 4
     out_bytes = wl.batch * wl.num_q_heads * wl.head_dim * 4
     return k_bytes + v_bytes + q_bytes + pt_bytes + part_bytes + out_bytes
 
@@ -328,7 +329,7 @@ def gpu_arm(args, world, rank, local):
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)
         abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if scope == "cluster"
-                                   else n_partials(rep.L, 1))
+                                   else n_partials(rep.L, 1), with_o=scope == "cluster")
         us_launch = ms_step * 1e3 / args.steps
         achieved = abytes / (us_launch * 1e-6) / 1e9
         res[tag] = dict(tau=tau, max_scope=scope, ms_per_step=ms_step / args.steps,

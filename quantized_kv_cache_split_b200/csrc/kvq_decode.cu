@@ -780,6 +780,7 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red_m[w * 8 + tid]);
       cmx[tid] = m;
+      if (tid == 0) misc[2] = 0;  // warps done with their V pass (read after the next barrier)
     }
     if (CS > 1) cluster_sync(); else __syncthreads();  // CTA maxima visible (cluster-wide)
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
@@ -995,6 +996,60 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) accw[(mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
+    if (add_merge) {
+      // the first warp done with its V pass waits for every split of this (sequence, KV
+      // head) to publish, then computes this split's share of each head, 2^(m_s - M) / L,
+      // while the other warps are still accumulating
+      int first = 0;
+      if (lane == 0) first = atomicAdd(&misc[2], 1) == 0;
+      first = __shfl_sync(0xffffffffu, first, 0);
+      if (first) {
+        int ok = 0;
+        if (lane == 0) {
+          ok = cta_group_wait(a.counters + (size_t)b * hkv + kvh, nbar * nsplit);
+          cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, nsplit);
+          if (!ok) set_flag(flags, KVQ_FLAG_TIMEOUT);
+          misc[0] = ok;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+          __threadfence();
+          // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads in flight
+          // together for up to 64 partials), then combine across the four lanes
+          const int h = lane >> 2, j = lane & 3;
+          const size_t uh = ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits;
+          float M = -INFINITY, L = 0.f;
+          for (int ub = 0; ub < nsplit; ub += 64) {
+            float mv[16], lv[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const int u = ub + j + 4 * t;
+              const bool v = h < G && u < nsplit;
+              mv[t] = v ? __ldcg(a.part_m + uh + u) : -INFINITY;
+              lv[t] = v ? __ldcg(a.part_l + uh + u) : 0.f;
+            }
+            float bm = M;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) bm = fmaxf(bm, mv[t]);
+            float ds = (M == -INFINITY) ? 0.f : L * ex2(M - bm);
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              if (mv[t] != -INFINITY) ds = fmaf(ex2(mv[t] - bm), lv[t], ds);
+            M = bm;
+            L = ds;
+          }
+#pragma unroll
+          for (int o = 1; o < 4; o <<= 1) {  // combine (M, L) of the four lanes of head h
+            const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
+            const float Lo = __shfl_xor_sync(0xffffffffu, L, o);
+            const float nm = fmaxf(M, Mo);
+            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + (Mo == -INFINITY ? 0.f : Lo * ex2(Mo - nm));
+            M = nm;
+          }
+          if (j == 0 && h < G) cmx[8 + h] = ex2(mpart[h] - M) / L;
+        }
+      }
+    }
     cp_async_wait<0>();  // nothing of this split stays in flight
     __syncthreads();     // every warp's accumulators, l and counts are in shared memory
 
@@ -1085,38 +1140,7 @@ decode_kernel(const DecodeArgs a) {
     //      published its (m, l)) into the output; otherwise the last cluster to finish
     //      the (sequence, KV head) merges the written partials by the log-sum-exp rule.
     if (add_merge) {
-      if (tid == 0) {
-        misc[0] = cta_group_wait(a.counters + (size_t)b * hkv + kvh, nbar * nsplit);
-        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, nsplit);
-      }
-      __syncthreads();
-      if (misc[0]) {
-        __threadfence();
-        if (warp < G) {  // this split's share of head `warp`: 2^(m_s - M) / L
-          const size_t uw = ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits;
-          float M = -INFINITY, L = 0.f;
-          for (int ub = 0; ub < nsplit; ub += 64) {
-            const int ua = ub + lane, uc = ub + 32 + lane;
-            const float ma = ua < nsplit ? __ldcg(a.part_m + uw + ua) : -INFINITY;
-            const float mc = uc < nsplit ? __ldcg(a.part_m + uw + uc) : -INFINITY;
-            const float la = ua < nsplit ? __ldcg(a.part_l + uw + ua) : 0.f;
-            const float lc = uc < nsplit ? __ldcg(a.part_l + uw + uc) : 0.f;
-            float bm = fmaxf(ma, mc);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-            const float nm = fmaxf(M, bm);
-            float ds = (ma == -INFINITY ? 0.f : ex2(ma - nm) * la) + (mc == -INFINITY ? 0.f : ex2(mc - nm) * lc);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + ds;
-            M = nm;
-          }
-          if (lane == 0) cmx[8 + warp] = ex2(mpart[warp] - M) / L;
-        }
-      } else if (tid == 0) {
-        set_flag(flags, KVQ_FLAG_TIMEOUT);
-      }
-      __syncthreads();  // the coefficients (and this CTA's o) are in shared memory
+      __syncthreads();  // this CTA's o is in shared memory
       if (misc[0]) {
         if constexpr (C::kLut) {  // rotate the scaled rows back: s .* (c H (coef * o'))
           if (warp < G) {

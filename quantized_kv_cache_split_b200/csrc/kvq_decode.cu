@@ -108,8 +108,8 @@ struct Layout {
   static constexpr size_t list = pk + (size_t)kWarps * 8 * kPkStride * 2;     // u8 [warps][64]
   static constexpr size_t red = list + (size_t)kWarps * kTile;                // float [2][warps][8]
   static constexpr size_t cnt = red + 2 * kWarps * 8 * 4;                     // int [2][warps]
-  static constexpr size_t cmx = cnt + 2 * kWarps * 4;                         // float [2][8] maxima
-  static constexpr size_t mpart = cmx + 16 * 4;                               // float [8]
+  static constexpr size_t cmx = cnt + 2 * kWarps * 4;                         // float [3][8]
+  static constexpr size_t mpart = cmx + 24 * 4;                               // float [8]
   static constexpr size_t lpart = mpart + 8 * 4;                              // float [8]
   static constexpr size_t octa = lpart + 8 * 4;                               // float [8][D]
   static constexpr size_t slen = octa + (size_t)8 * D * 4;                    // int [MAX_BATCH]
@@ -551,7 +551,8 @@ decode_kernel(const DecodeArgs a) {
   float* red_l = red_m + kWarps * 8;
   int* cnt_skip = reinterpret_cast<int*>(smem + LY::cnt);
   int* cnt_kept = cnt_skip + kWarps;
-  float* cmx = reinterpret_cast<float*>(smem + LY::cmx);       // this CTA's maxima, then the sequence's (log2)
+  // this CTA's maxima, the sequence's (log2), and this split's share of each head
+  float* cmx = reinterpret_cast<float*>(smem + LY::cmx);
   float* mpart = reinterpret_cast<float*>(smem + LY::mpart);   // m of this CTA's partial
   float* lpart = reinterpret_cast<float*>(smem + LY::lpart);   // l of this CTA's partial
   float* octa = reinterpret_cast<float*>(smem + LY::octa);     // o of this CTA's partial [8][D]
@@ -786,35 +787,73 @@ decode_kernel(const DecodeArgs a) {
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
     int nbar = 0;  // group barriers this unit has passed (barrier k waits for k * n arrivals)
     if (a.global_max) {
-      // every split of this (sequence, KV head) publishes its maxima in its partial's m
-      // slot; after a barrier among them, each reads all and takes the largest
+      // every split publishes its maxima and its denominators relative to them; after one
+      // barrier among the splits of this (sequence, KV head) each derives the final
+      // maximum M and denominator L of every head (split 0 first clears the output rows
+      // that the splits add their shares into)
       const int n = (nb + Ls - 1) / Ls;
-      if (tid < G) a.part_m[slot0 + (size_t)tid * a.max_splits] = cmx[tid];
+      float lo0 = 0.f, lo1 = 0.f;
+      const float c0 = cmx[2 * c], c1 = cmx[2 * c + 1];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (16 * j >= nvalid) break;
+        const float4 sv = scw[j * 32];  // invalid rows hold -inf
+        lo0 += ex2(sv.x - c0) + ex2(sv.z - c0);
+        lo1 += ex2(sv.y - c1) + ex2(sv.w - c1);
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lo0 += __shfl_xor_sync(0xffffffffu, lo0, o);
+        lo1 += __shfl_xor_sync(0xffffffffu, lo1, o);
+      }
+      if (r == 0) {
+        red_l[warp * 8 + 2 * c] = lo0;
+        red_l[warp * 8 + 2 * c + 1] = lo1;
+      }
+      __syncthreads();
+      if (tid < G) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
+        a.xch[slot0 + (size_t)tid * a.max_splits] = make_float2(cmx[tid], l);
+      }
+      if (a.out && a.group_merge && cu == 0)
+        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
       __syncthreads();
       ++nbar;
       if (tid == 0) {
         misc[1] = cta_group_arrive_wait(a.counters + (size_t)b * hkv + kvh, nbar * n);
-        if (!(a.out && a.group_merge))  // no second barrier follows
-          cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
+        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
+        misc[0] = misc[1];
+        if (!misc[1]) set_flag(flags, KVQ_FLAG_TIMEOUT);
       }
       __syncthreads();
       if (misc[1]) {
         __threadfence();
-        if (warp < G) {
+        if (warp < G) {  // M and L of head `warp` over all splits
           const size_t uw = ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits;
-          float M = -INFINITY;
-          for (int u = lane; u < n; u += 32) M = fmaxf(M, __ldcg(a.part_m + uw + u));
+          float M = -INFINITY, L = 0.f;
+          for (int ub = 0; ub < n; ub += 32) {
+            const int u = ub + lane;
+            const float2 e = u < n ? __ldcg(a.xch + uw + u) : make_float2(-INFINITY, 0.f);
+            float bm = e.x;
 #pragma unroll
-          for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-          if (lane == 0) cmx[8 + warp] = M;
+            for (int o = 16; o; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+            const float nm = fmaxf(M, bm);
+            float ds = e.x == -INFINITY ? 0.f : ex2(e.x - nm) * e.y;
+#pragma unroll
+            for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + ds;
+            M = nm;
+          }
+          if (lane == 0) {
+            cmx[8 + warp] = M;
+            cmx[16 + warp] = 1.f / L;  // this split's share: 2^(M - M) / L
+          }
         }
-      } else if (tid == 0) {
-        set_flag(flags, KVQ_FLAG_TIMEOUT);
       }
       __syncthreads();
     }
-    // (with the maximum over all splits, a fast CTA may already have replaced its
-    // published maxima by the final one in its m slot: the same largest value)
     float mh0 = cmx[2 * c], mh1 = cmx[2 * c + 1];
     if (a.global_max && misc[1]) {
       mh0 = cmx[8 + 2 * c];
@@ -923,17 +962,17 @@ decode_kernel(const DecodeArgs a) {
 
     // ---- additive in-kernel merge (every split on its own CTA): the split publishes its
     //      (m, l) and arrives at its (sequence, KV head) barrier now, so that the wait
-    //      overlaps its V work; split 0 clears the output rows that the splits add into
+    //      overlaps its V work; split 0 clears the output rows that the splits add into.
+    //      (With the sequence-wide maximum this exchange already happened.)
     const bool add_merge = a.out && a.group_merge;
     const int nsplit = (nb + Ls - 1) / Ls;
-    if (add_merge) {
+    if (add_merge && !a.global_max) {
       __syncthreads();  // every warp's l is in shared memory
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        a.part_m[slot0 + (size_t)tid * a.max_splits] = mpart[tid];
-        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+        a.xch[slot0 + (size_t)tid * a.max_splits] = make_float2(mpart[tid], l);
       }
       if (cu == 0)
         for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
@@ -996,7 +1035,7 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) accw[(mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
-    if (add_merge) {
+    if (add_merge && !a.global_max) {
       // the first warp done with its V pass waits for every split of this (sequence, KV
       // head) to publish, then computes this split's share of each head, 2^(m_s - M) / L,
       // while the other warps are still accumulating
@@ -1024,9 +1063,9 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int u = ub + j + 4 * t;
-              const bool v = h < G && u < nsplit;
-              mv[t] = v ? __ldcg(a.part_m + uh + u) : -INFINITY;
-              lv[t] = v ? __ldcg(a.part_l + uh + u) : 0.f;
+              const float2 e = h < G && u < nsplit ? __ldcg(a.xch + uh + u) : make_float2(-INFINITY, 0.f);
+              mv[t] = e.x;
+              lv[t] = e.y;
             }
             float bm = M;
 #pragma unroll
@@ -1046,7 +1085,7 @@ decode_kernel(const DecodeArgs a) {
             L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + (Mo == -INFINITY ? 0.f : Lo * ex2(Mo - nm));
             M = nm;
           }
-          if (j == 0 && h < G) cmx[8 + h] = ex2(mpart[h] - M) / L;
+          if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
         }
       }
     }
@@ -1145,7 +1184,7 @@ decode_kernel(const DecodeArgs a) {
         if constexpr (C::kLut) {  // rotate the scaled rows back: s .* (c H (coef * o'))
           if (warp < G) {
             constexpr int K = D / 32;
-            const float coef = cmx[8 + warp] * (D == 64 ? 0.125f : 0.08838834764831845f);
+            const float coef = cmx[16 + warp] * (D == 64 ? 0.125f : 0.08838834764831845f);
             float y[K];
 #pragma unroll
             for (int kk = 0; kk < K; ++kk) y[kk] = octa[warp * D + 32 * kk + lane] * coef;
@@ -1176,7 +1215,7 @@ decode_kernel(const DecodeArgs a) {
         float* orow = a.out + ((size_t)b * Hq + (size_t)kvh * G) * D;
         for (int q4 = tid; q4 < G * D / 4; q4 += kThreads) {
           const int h = q4 / (D / 4);
-          const float coef = C::kLut ? 1.f : cmx[8 + h];
+          const float coef = C::kLut ? 1.f : cmx[16 + h];
           const float4 v = reinterpret_cast<const float4*>(octa)[q4];
           red_add_f32x4(orow + 4 * q4, make_float4(v.x * coef, v.y * coef, v.z * coef, v.w * coef));
         }

@@ -31,6 +31,7 @@ struct DecodeArgs {
   float* part_o;      // partials, see below
   float* part_m;
   float* part_l;
+  float2* xch;        // (m, l) each split publishes for the others [batch][num_q_heads][max_splits]
   unsigned long long* stats;
   float* out;         // non-null: merge in the same kernel and write the output
   int cluster;        // consecutive splits per thread-block cluster (1, 2 or 4)
@@ -49,6 +50,8 @@ struct DecodeArgs {
 //   o [batch][num_q_heads][max_splits][head_dim] fp32 (unnormalized)
 //   m [batch][num_q_heads][max_splits] fp32 (running maximum, log2 units)
 //   l [batch][num_q_heads][max_splits] fp32
+//   (m, l) exchange [batch][num_q_heads][max_splits] fp32 x 2 (what the splits of a
+//   (sequence, KV head) publish to one another at their group barrier)
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits);
 __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
   return ((size_t)2 * batch * num_q_heads * sizeof(int32_t) + 255) / 256 * 256;

@@ -27,6 +27,19 @@ lut4   rotated 4-bit codebook (TurboQuant-style, Walsh-Hadamard rotation named i
        idx_i = #{k : u_i > t_k};  stored norm = fp16_rne(n);
        x_hat' = n16 * c16[idx]  (in the rotated domain).
 
+nvfp4  (named in the tproger page's opening summary among the schemes the method
+       works with; the page gives no arithmetic).  Blocks of 16 along the head
+       dimension, E2M1 codes with an E4M3 block scale and a per-vector fp32 scale:
+       amax = max |x_i| over the vector;  g = fp32(amax / 2688)  (2688 = 6 * 448, the
+       largest E2M1 value times the largest E4M3 value);  per block
+       s = e4m3(fp32(amax_b / fp32(6 * g)))  (0 when g == 0);
+       code_i = e2m1(fp32(x_i / fp32(g * s)))  (0 when g * s == 0);
+       x_hat = e2m1_value(code) * s * g.  e4m3 / e2m1 round to nearest with ties to
+       the even code and saturate at the largest finite value (448 / 6); e2m1 keeps
+       the sign (a negative value that rounds to zero gives the code of -0).
+       Scale row (little-endian bytes): the D/16 E4M3 codes, the 4 bytes of g, zero
+       padding to a multiple of 8 bytes.
+
 Packing of 4-bit codes: element 2j in the low nibble of byte j, element 2j+1 in
 the high nibble.
 """
@@ -181,6 +194,102 @@ def unrotate_f64(y: np.ndarray, signs: np.ndarray) -> np.ndarray:
     return (np.asarray(y, dtype=np.float64) @ H.T / np.sqrt(D)) * signs.astype(np.float64)
 
 
+# ---------------------------------------------------------------- nvfp4
+
+NV_BLOCK = 16
+E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # codes 0..7; bit 3 = sign
+
+
+def _e4m3_magnitudes() -> np.ndarray:
+    """Value of every non-negative E4M3 code 0..126 (code 127 is NaN): exponent bits 3..6
+    with bias 7, three mantissa bits; exponent 0 is subnormal (m / 8) 2^-6."""
+    vals = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        vals.append((m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+E4M3_MAGNITUDES = _e4m3_magnitudes()
+
+
+def _nearest_even(mag: np.ndarray, table: np.ndarray) -> np.ndarray:
+    """Index of the nearest entry of the increasing `table` (ties -> the even index);
+    values beyond the last entry saturate to it."""
+    mag = np.asarray(mag, dtype=np.float64)
+    dist = np.abs(mag[..., None] - table)            # exact: float32 inputs, exact table
+    best = dist.min(axis=-1, keepdims=True)
+    cand = dist == best
+    idx = np.arange(len(table))
+    # among the (at most two, adjacent) nearest entries take the even index
+    even = np.where(cand & (idx % 2 == 0), idx, len(table))
+    pick = even.min(axis=-1)
+    first = np.where(cand, idx, len(table)).min(axis=-1)
+    return np.where(pick < len(table), pick, first)
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float32)
+    code = _nearest_even(np.abs(v), E2M1_MAGNITUDES).astype(np.uint8)
+    return np.where(np.signbit(v), code | 8, code).astype(np.uint8)
+
+
+def e2m1_decode(code: np.ndarray) -> np.ndarray:
+    code = np.asarray(code).astype(np.int64)
+    mag = E2M1_MAGNITUDES[code & 7]
+    return np.where(code & 8, -mag, mag)
+
+
+def e4m3_encode(t: np.ndarray) -> np.ndarray:
+    """Non-negative float32 -> E4M3 code (nearest, ties to even, saturating at 448)."""
+    return _nearest_even(np.asarray(t, dtype=np.float32), E4M3_MAGNITUDES).astype(np.uint8)
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    return E4M3_MAGNITUDES[np.asarray(code).astype(np.int64) & 127]
+
+
+def nvfp4_scale_row_words(D: int) -> int:
+    return (D // NV_BLOCK + 4 + 7) // 8 * 4
+
+
+def quantize_nvfp4(x16: np.ndarray):
+    """Returns (codes [..., D] E2M1 bit patterns, scale rows [..., nvfp4_scale_row_words(D)]
+    as uint16 words)."""
+    x = np.asarray(x16).astype(np.float32)
+    D = x.shape[-1]
+    assert D % NV_BLOCK == 0
+    xb = x.reshape(x.shape[:-1] + (D // NV_BLOCK, NV_BLOCK))
+    amax = np.abs(x).max(axis=-1)                                   # [...]
+    g = (amax / F32(2688.0)).astype(np.float32)
+    six_g = (F32(6.0) * g).astype(np.float32)
+    amax_b = np.abs(xb).max(axis=-1)                                # [..., B]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.where(six_g[..., None] > 0, amax_b / six_g[..., None], F32(0.0)).astype(np.float32)
+    sc = e4m3_encode(t)                                             # [..., B]
+    s = e4m3_decode(sc).astype(np.float32)
+    den = (g[..., None] * s).astype(np.float32)                     # [..., B]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(den[..., None] > 0, xb / den[..., None], F32(0.0)).astype(np.float32)
+    codes = np.where(den[..., None] > 0, e2m1_encode(v), np.uint8(0)).reshape(x.shape)
+    nw = nvfp4_scale_row_words(D)
+    row = np.zeros(x.shape[:-1] + (2 * nw,), dtype=np.uint8)
+    row[..., : D // NV_BLOCK] = sc
+    row[..., D // NV_BLOCK: D // NV_BLOCK + 4] = g[..., None].view(np.uint8)
+    return codes.astype(np.int64), row.view(np.uint16)
+
+
+def dequantize_nvfp4(codes: np.ndarray, words: np.ndarray) -> np.ndarray:
+    codes = np.asarray(codes)
+    D = codes.shape[-1]
+    raw = np.ascontiguousarray(np.asarray(words, dtype=np.uint16)).view(np.uint8)
+    sc = raw[..., : D // NV_BLOCK]
+    g = np.ascontiguousarray(raw[..., D // NV_BLOCK: D // NV_BLOCK + 4]).view(np.float32)[..., 0]
+    s = e4m3_decode(sc).astype(np.float64)
+    vals = e2m1_decode(codes).reshape(codes.shape[:-1] + (D // NV_BLOCK, NV_BLOCK))
+    return (vals * s[..., None] * g.astype(np.float64)[..., None, None]).reshape(codes.shape)
+
+
 # ---------------------------------------------------------------- whole cache
 
 def quantize(fmt: str, x16: np.ndarray, signs=None, codebook16=None):
@@ -192,6 +301,8 @@ def quantize(fmt: str, x16: np.ndarray, signs=None, codebook16=None):
     if fmt == "lut4":
         idx, n = quantize_lut4(x16, signs, codebook16)
         return idx, n[..., None]
+    if fmt == "nvfp4":
+        return quantize_nvfp4(x16)
     raise ValueError(fmt)
 
 
@@ -202,4 +313,6 @@ def dequantize(fmt: str, codes, scales16, codebook16=None) -> np.ndarray:
         return dequantize_q4_0(codes, scales16)
     if fmt == "lut4":
         return dequantize_lut4(codes, scales16[..., 0], codebook16)
+    if fmt == "nvfp4":
+        return dequantize_nvfp4(codes, scales16)
     raise ValueError(fmt)

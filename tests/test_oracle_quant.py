@@ -203,3 +203,105 @@ def test_lut4_bitexact_against_fp64_where_unambiguous():
     ambiguous = np.min(np.abs(u[..., None] - t), axis=-1) < 1e-6
     assert ((idx == ref) | ambiguous).all()
     assert (n == nn.astype(np.float16)).mean() > 0.95
+
+
+# ---------------------------------------------------------------- nvfp4
+
+def _e2m1_table_from_bits():
+    """E2M1 magnitudes from the bit layout (2 exponent bits, bias 1, 1 mantissa bit;
+    exponent 0 is subnormal), independent of the oracle's table."""
+    out = []
+    for code in range(8):
+        e, m = code >> 1, code & 1
+        out.append(Fraction(m, 2) if e == 0 else (1 + Fraction(m, 2)) * Fraction(2) ** (e - 1))
+    return out
+
+
+def _nearest_even_brute(x: Fraction, table):
+    best = None
+    for i, v in enumerate(table):
+        d = abs(x - v)
+        if best is None or d < best[0] or (d == best[0] and i % 2 == 0):
+            best = (d, i)
+    return best[1]
+
+
+def test_e4m3_encoding_matches_torch_float8():
+    # independent reference: PyTorch's float8_e4m3fn cast (round to nearest even)
+    import torch
+    rng = np.random.Generator(np.random.PCG64(21))
+    t = np.concatenate([rng.random(2000) * 448, np.exp(rng.uniform(-12, 6, 2000)),
+                        Q.E4M3_MAGNITUDES, (Q.E4M3_MAGNITUDES[1:] + Q.E4M3_MAGNITUDES[:-1]) / 2])
+    t = t[t <= 448].astype(np.float32)
+    ref = torch.from_numpy(t).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(Q.e4m3_encode(t), ref)
+    assert np.array_equal(Q.e4m3_decode(np.arange(127)),
+                          torch.arange(127, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy())
+    assert Q.e4m3_encode(np.float32([1e4]))[0] == 126           # saturates at 448
+
+
+def test_e2m1_encoding_brute_force():
+    table = _e2m1_table_from_bits()
+    assert [float(v) for v in table] == list(Q.E2M1_MAGNITUDES)
+    rng = np.random.Generator(np.random.PCG64(22))
+    mids = [float((a + b) / 2) for a, b in zip(table[:-1], table[1:])]
+    vals = np.concatenate([rng.uniform(-8, 8, 3000), mids, [-m for m in mids], [0.0, -0.0, 6.0, 7.0, -9.0]])
+    vals = vals.astype(np.float32)
+    got = Q.e2m1_encode(vals)
+    for v, c in zip(vals, got):
+        mag = _nearest_even_brute(abs(Fraction(float(v))), table)
+        want = mag | (8 if np.signbit(v) else 0)
+        assert c == want, (v, c, want)
+
+
+def test_nvfp4_quantizer_steps_exact():
+    rng = np.random.Generator(np.random.PCG64(23))
+    x = (rng.standard_normal((40, 128)) * rng.choice([0.01, 1.0, 50.0], (40, 1))).astype(np.float16)
+    codes, words = Q.quantize_nvfp4(x)
+    raw = words.view(np.uint8)
+    table = _e2m1_table_from_bits()
+    e4 = {i: Fraction(float(v)) for i, v in enumerate(Q.E4M3_MAGNITUDES)}
+    for i in range(len(x)):
+        xf = [Fraction(float(v)) for v in x[i].astype(np.float32)]
+        amax = max(abs(v) for v in xf)
+        g = np.float32(raw[i, 8:12].view(np.float32)[0])
+        assert abs(Fraction(float(g)) - amax / 2688) <= _ulp32(float(g)) / 2     # fp32(amax / 2688)
+        six_g = np.float32(np.float32(6.0) * g)
+        for b in range(8):
+            blk = xf[16 * b:16 * b + 16]
+            t = np.float32(np.float32(max(abs(v) for v in blk)) / six_g)
+            sc = raw[i, b]
+            assert sc == _nearest_even_brute(Fraction(float(t)), [e4[k] for k in range(127)])
+            den = np.float32(g * np.float32(float(e4[sc])))
+            for j in range(16):
+                v = np.float32(np.float32(float(blk[j])) / den) if den > 0 else np.float32(0.0)
+                c = codes[i, 16 * b + j]
+                want = _nearest_even_brute(abs(Fraction(float(v))), table) | (8 if np.signbit(v) else 0)
+                assert den == 0 or c == want
+
+
+def test_nvfp4_special_vectors_and_error_bound():
+    D = 64
+    zero = np.zeros((1, D), dtype=np.float16)
+    c, w = Q.quantize_nvfp4(zero)
+    assert not c.any() and not w.any()
+    # values exactly representable as e2m1 * e4m3 * g round-trip exactly
+    x = np.zeros((1, D), dtype=np.float16)
+    x[0, :8] = [6, 4, 3, 2, 1.5, 1, 0.5, -6]
+    c, w = Q.quantize_nvfp4(x)
+    xh = Q.dequantize_nvfp4(c, w)
+    assert np.allclose(xh[0, :8], x[0, :8].astype(np.float64), rtol=1e-6)
+    # tiny negatives keep their sign bit; reconstruction error within half an e2m1 step
+    rng = np.random.Generator(np.random.PCG64(24))
+    x = (rng.standard_normal((50, D)) * 2).astype(np.float16)
+    c, w = Q.quantize_nvfp4(x)
+    xh = Q.dequantize_nvfp4(c, w)
+    raw = w.view(np.uint8)
+    g = raw[:, 4:8].copy().view(np.float32)[:, 0].astype(np.float64)
+    s = Q.e4m3_decode(raw[:, :4]).astype(np.float64)                      # [50, 4]
+    unit = (s * g[:, None])[:, :, None]                                     # value of 1.0 per block
+    err = np.abs(xh - x.astype(np.float64)).reshape(50, 4, 16)
+    mag = np.abs(x.astype(np.float64)).reshape(50, 4, 16) / unit
+    step = np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0))              # e2m1 spacing there
+    assert (err <= (step / 2) * unit * (1 + 1e-6) + 1e-12).all()
+    assert Q.nvfp4_scale_row_words(128) == 8 and Q.nvfp4_scale_row_words(64) == 4

@@ -9,7 +9,8 @@
  * is below a threshold tau (the page uses 1e-6) has its V dequantization and
  * accumulation skipped entirely.  K is always dequantized, because it produces
  * the weights.  The page names q8_0, q4_0 and a Walsh-Hadamard-rotated
- * codebook format (section "Почему это работает для любой квантизации").
+ * codebook format (section "Почему это работает для любой квантизации"); its opening
+ * summary also names NVFP4.
  *
  * Conventions shared by every call
  * --------------------------------
@@ -29,6 +30,7 @@
  * ------------------------------------------------
  *  codes  plane: uint8  [num_pages][num_kv_heads][page_size][kvq_code_row_bytes(fmt, D)]
  *  scales plane: fp16   [num_pages][num_kv_heads][page_size][kvq_scale_row_count(fmt, D)]
+ *  (the scales plane is addressed in fp16 slots; for nvfp4 they hold raw bytes)
  *  A "slot" is page * page_size + offset_in_page.  A contiguous cache is the
  *  special case page_size = capacity, one page per sequence (page b for b).
  *
@@ -47,6 +49,13 @@
  *        fp16 (the norm n).  Attention runs in the rotated domain and the
  *        output is rotated back (R^T = diag(s) c H_D), so every format returns
  *        the same, unrotated, output.
+ *  nvfp4 (E2M1 codes, blocks of 16 along head_dim): g = amax/2688 over the vector
+ *        (fp32); per block s = e4m3(amax_b / (6 g)); code = e2m1(x / (g s));
+ *        x_hat = e2m1_value(code) * s * g.  e4m3 / e2m1 round to nearest, ties to
+ *        the even code, saturating at 448 / 6; e2m1 keeps the sign of x.  codes row =
+ *        D/2 bytes (nibbles as for q4_0, E2M1 bit patterns); scales row = the D/16
+ *        E4M3 bytes, the fp32 g (little-endian), zero padding to a multiple of 8
+ *        bytes: 8 fp16 slots for D = 128, 4 for D = 64.
  *  All quantizer arithmetic is IEEE fp32 round-to-nearest-even, one operation
  *  at a time (no fused multiply-add), so codes are fixed to the bit.
  */
@@ -72,6 +81,7 @@ extern "C" {
 #define KVQ_FMT_Q8_0  0
 #define KVQ_FMT_Q4_0  1
 #define KVQ_FMT_LUT4  2
+#define KVQ_FMT_NVFP4 3
 
 /* Option bits of kvq_decode_attn. */
 #define KVQ_OPT_SHARED_MAX 1u  /* the splits of one cluster share one running maximum (below) */

@@ -26,7 +26,8 @@ KVQ_ERR_DEVICE = -5
 KVQ_FMT_Q8_0 = 0
 KVQ_FMT_Q4_0 = 1
 KVQ_FMT_LUT4 = 2
-FORMATS = {"q8_0": KVQ_FMT_Q8_0, "q4_0": KVQ_FMT_Q4_0, "lut4": KVQ_FMT_LUT4}
+KVQ_FMT_NVFP4 = 3
+FORMATS = {"q8_0": KVQ_FMT_Q8_0, "q4_0": KVQ_FMT_Q4_0, "lut4": KVQ_FMT_LUT4, "nvfp4": KVQ_FMT_NVFP4}
 
 KVQ_OPT_SHARED_MAX = 1
 KVQ_OPT_GLOBAL_MAX = 2

@@ -38,7 +38,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int check_desc(const kvq_cache_desc* d) {
   if (!d) return KVQ_ERR_INVALID_ARG;
-  if (d->fmt != KVQ_FMT_Q8_0 && d->fmt != KVQ_FMT_Q4_0 && d->fmt != KVQ_FMT_LUT4)
+  if (d->fmt != KVQ_FMT_Q8_0 && d->fmt != KVQ_FMT_Q4_0 && d->fmt != KVQ_FMT_LUT4 &&
+      d->fmt != KVQ_FMT_NVFP4)
     return KVQ_ERR_UNSUPPORTED;
   if (d->head_dim != 64 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (d->num_kv_heads < 1 || d->num_pages < 1) return KVQ_ERR_INVALID_ARG;
@@ -116,7 +117,7 @@ extern "C" {
 size_t kvq_code_row_bytes(int32_t fmt, int32_t head_dim) {
   if (head_dim != 64 && head_dim != 128) return 0;
   if (fmt == KVQ_FMT_Q8_0) return (size_t)head_dim;
-  if (fmt == KVQ_FMT_Q4_0 || fmt == KVQ_FMT_LUT4) return (size_t)head_dim / 2;
+  if (fmt == KVQ_FMT_Q4_0 || fmt == KVQ_FMT_LUT4 || fmt == KVQ_FMT_NVFP4) return (size_t)head_dim / 2;
   return 0;
 }
 
@@ -124,6 +125,7 @@ size_t kvq_scale_row_count(int32_t fmt, int32_t head_dim) {
   if (head_dim != 64 && head_dim != 128) return 0;
   if (fmt == KVQ_FMT_Q8_0 || fmt == KVQ_FMT_Q4_0) return (size_t)head_dim / 32;
   if (fmt == KVQ_FMT_LUT4) return 1;
+  if (fmt == KVQ_FMT_NVFP4) return ((size_t)head_dim / 16 + 4 + 7) / 8 * 4;  // bytes / 2
   return 0;
 }
 

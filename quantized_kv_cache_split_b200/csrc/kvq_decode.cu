@@ -45,6 +45,8 @@
 //             writes the output (lut4: rotated back), so no second kernel runs.
 #include <mutex>
 
+#include <cuda_fp8.h>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -73,8 +75,10 @@ struct Cfg {
   static constexpr bool kQ8 = FMT == KVQ_FMT_Q8_0;
   static constexpr bool kQ4 = FMT == KVQ_FMT_Q4_0;
   static constexpr bool kLut = FMT == KVQ_FMT_LUT4;
+  static constexpr bool kNv = FMT == KVQ_FMT_NVFP4;      // E2M1 codes, E4M3 scales per 16
   static constexpr int CROW = kQ8 ? D : D / 2;          // code bytes per row
-  static constexpr int NSC = kLut ? 1 : D / 32;          // fp16 per scale row
+  // fp16 slots per scale row (nvfp4: E4M3 bytes, fp32 vector scale, padding)
+  static constexpr int NSC = kLut ? 1 : kNv ? (D / 16 + 4 + 7) / 8 * 4 : D / 32;
   static constexpr int SROW = 2 * NSC;                   // scale bytes per row
   static constexpr int RPW = 16 / SROW;                  // rows per 16-byte scale window
   static constexpr int NBLK = D / 32;
@@ -167,6 +171,16 @@ __device__ __forceinline__ void lut_lookup4(const Lut& t, uint32_t sel, uint32_t
 __device__ __forceinline__ uint32_t nib_mask_lo(uint32_t x) { return prmt(x << 4, x, 0xD9C8u); }
 __device__ __forceinline__ uint32_t nib_mask_hi(uint32_t x) { return prmt(x << 4, x, 0xFBEAu); }
 
+// An E4M3 byte as an fp16 pair (s, s) (exact).
+__device__ __forceinline__ __half2 e4m3_pair(uint32_t b) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(b | (b << 8)), __NV_E4M3);
+  return *reinterpret_cast<const __half2*>(&h);
+}
+__device__ __forceinline__ float e4m3_float(uint32_t b) { return __low2float(e4m3_pair(b)); }
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, __half2 b) {
+  return h2_as_u32(__hmul2(u32_as_h2(a), b));
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return h2_as_u32(__floats2half2_rn(lo, hi));
 }
@@ -190,7 +204,7 @@ __device__ __forceinline__ void k_job_scores(const uint8_t* __restrict__ codes,
   const int sw0 = (row0 >> C::SWZ_SHIFT) & C::SWZ_MASK;
   const int sw1 = (row1 >> C::SWZ_SHIFT) & C::SWZ_MASK;
   s[0] = s[1] = s[2] = s[3] = 0.f;
-  if constexpr (!C::kLut) {
+  if constexpr (C::kQ8 || C::kQ4) {
     float2 d0f[C::NBLK / 2 > 0 ? C::NBLK / 2 : 1], d1f[C::NBLK / 2 > 0 ? C::NBLK / 2 : 1];
     if constexpr (C::NBLK == 4) {
       const uint2 u0 = *reinterpret_cast<const uint2*>(sc + row0 * C::SROW);
@@ -232,7 +246,7 @@ __device__ __forceinline__ void k_job_scores(const uint8_t* __restrict__ codes,
       s[0] = fmaf(d0, t[0], s[0]); s[1] = fmaf(d0, t[1], s[1]);
       s[2] = fmaf(d1, t[2], s[2]); s[3] = fmaf(d1, t[3], s[3]);
     }
-  } else {
+  } else if constexpr (C::kLut) {
     // lut4: centroid lookups; the query carries hi + lo fp16 parts.
 #pragma unroll
     for (int m = 0; m < C::NBLK; ++m) {
@@ -255,6 +269,33 @@ __device__ __forceinline__ void k_job_scores(const uint8_t* __restrict__ codes,
     const float n0 = __half2float(*reinterpret_cast<const __half*>(sc + row0 * 2));
     const float n1 = __half2float(*reinterpret_cast<const __half*>(sc + row1 * 2));
     s[0] *= n0; s[1] *= n0; s[2] *= n1; s[3] *= n1;
+  } else {
+    // nvfp4: E2M1 values from the table; the lane's 8 dims of chunk m lie in 16-block
+    // 2m + c/2, whose E4M3 scale multiplies them in fp16 (exact: an E2M1 value times an
+    // E4M3 value is representable); the fp32 vector scale multiplies the score.
+    const uint8_t* s0p = sc + row0 * C::SROW;
+    const uint8_t* s1p = sc + row1 * C::SROW;
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      const uint32_t x0 = lds32(p0 + ((m ^ sw0) << 4));
+      const uint32_t x1 = lds32(p1 + ((m ^ sw1) << 4));
+      const int blk = 2 * m + (c >> 1);
+      const __half2 sc0 = e4m3_pair(s0p[blk]), sc1 = e4m3_pair(s1p[blk]);
+      uint32_t L0, H0, L1, H1, L2, H2, L3, H3;
+      lut_lookup4(lut, x0, nib_mask_lo(x0), L0, H0);          // row0 dims +0..3
+      lut_lookup4(lut, x0 >> 16, nib_mask_hi(x0), L1, H1);    // row0 dims +4..7
+      lut_lookup4(lut, x1, nib_mask_lo(x1), L2, H2);          // row1 dims +0..3
+      lut_lookup4(lut, x1 >> 16, nib_mask_hi(x1), L3, H3);    // row1 dims +4..7
+      const uint32_t a0 = hmul2u(prmt(L0, H0, 0x5140u), sc0), a2 = hmul2u(prmt(L0, H0, 0x7362u), sc0);
+      const uint32_t a1 = hmul2u(prmt(L2, H2, 0x5140u), sc1), a3 = hmul2u(prmt(L2, H2, 0x7362u), sc1);
+      mma16816(s, a0, a1, a2, a3, qf[2 * m][0], qf[2 * m][1]);
+      const uint32_t b0 = hmul2u(prmt(L1, H1, 0x5140u), sc0), b2 = hmul2u(prmt(L1, H1, 0x7362u), sc0);
+      const uint32_t b1 = hmul2u(prmt(L3, H3, 0x5140u), sc1), b3 = hmul2u(prmt(L3, H3, 0x7362u), sc1);
+      mma16816(s, b0, b1, b2, b3, qf[2 * m + 1][0], qf[2 * m + 1][1]);
+    }
+    const float g0 = *reinterpret_cast<const float*>(s0p + D / 16);
+    const float g1 = *reinterpret_cast<const float*>(s1p + D / 16);
+    s[0] *= g0; s[1] *= g0; s[2] *= g1; s[3] *= g1;
   }
 }
 
@@ -385,7 +426,19 @@ __device__ __forceinline__ void build_query(const QRaw<D>& q, int c,
                                             uint32_t (&qf)[D / 16][2], uint32_t (&ql)[D / 16][2],
                                             float (&corr)[D / 32][2]) {
   using C = Cfg<FMT, D>;
-  if constexpr (!C::kLut) {
+  if constexpr (C::kNv) {
+    // the query as it is (no rotation, no offset): k-step 2m + j takes halves 4j .. 4j + 3
+    // of the lane's 8 dims 32m + 8c .. 32m + 8c + 7
+#pragma unroll
+    for (int m = 0; m < C::NBLK; ++m) {
+      qf[2 * m][0] = q.w[4 * m];
+      qf[2 * m][1] = q.w[4 * m + 1];
+      qf[2 * m + 1][0] = q.w[4 * m + 2];
+      qf[2 * m + 1][1] = q.w[4 * m + 3];
+      ql[2 * m][0] = ql[2 * m][1] = ql[2 * m + 1][0] = ql[2 * m + 1][1] = 0u;
+      corr[m][0] = corr[m][1] = 0.f;
+    }
+  } else if constexpr (!C::kLut) {
     float part[C::NBLK];
 #pragma unroll
     for (int m = 0; m < C::NBLK; ++m) {
@@ -514,10 +567,12 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const _
   };
   auto scale = [&](int slot) -> __half {
     if (slot >= n_valid) return __ushort_as_half(0);
-    const int off = C::kLut ? 0 : 2 * blk;
-    const uint8_t* p = TILE ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW + off
-                            : buf + slot * C::VSTRIDE + C::CROW + (trow[slot] & (C::RPW - 1)) * C::SROW + off;
-    return *reinterpret_cast<const __half*>(p);
+    const uint8_t* srow = TILE ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW
+                               : buf + slot * C::VSTRIDE + C::CROW + (trow[slot] & (C::RPW - 1)) * C::SROW;
+    if constexpr (C::kNv)  // E4M3 block scale of this thread's dims times the vector scale
+      return __float2half_rn(e4m3_float(srow[(C::E * r) / 16]) *
+                             *reinterpret_cast<const float*>(srow + D / 16));
+    return *reinterpret_cast<const __half*>(srow + (C::kLut ? 0 : 2 * blk));
   };
   const __half2 dab = __halves2half2(scale(sa), scale(sa + 1));
   const __half2 dcd = __halves2half2(scale(sc), scale(sc + 1));
@@ -601,6 +656,15 @@ decode_kernel(const DecodeArgs a) {
         hi |= (e >> 8) << (8 * j);
       }
       lut.lo[i] = lo; lut.hi[i] = hi;
+    }
+  } else if constexpr (C::kNv) {
+    // E2M1 code -> fp16: 0, 0.5, 1, 1.5, 2, 3, 4, 6, then the same with the sign bit;
+    // every low byte is zero
+    const uint32_t hi[4] = {0x3E3C3800u, 0x46444240u, 0xBEBCB880u, 0xC6C4C2C0u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lut.lo[i] = 0u;
+      lut.hi[i] = hi[i];
     }
   } else {
 #pragma unroll
@@ -1468,6 +1532,8 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (f == KVQ_FMT_Q4_0 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_Q4_0, 128);
   if (f == KVQ_FMT_Q4_0 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_Q4_0, 64);
   if (f == KVQ_FMT_LUT4 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_LUT4, 128);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_NVFP4, 64);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return KVQ_CALL_LAUNCH(KVQ_FMT_NVFP4, 128);
   if (f == KVQ_FMT_LUT4 && d == 64) return KVQ_CALL_LAUNCH(KVQ_FMT_LUT4, 64);
 #undef KVQ_CALL_LAUNCH
   return KVQ_ERR_UNSUPPORTED;
@@ -1479,6 +1545,8 @@ int decode_cluster_capacity(int f, int d, int cluster) {
   if (f == KVQ_FMT_Q4_0 && d == 128) return capacity_t<KVQ_FMT_Q4_0, 128>(cluster);
   if (f == KVQ_FMT_Q4_0 && d == 64) return capacity_t<KVQ_FMT_Q4_0, 64>(cluster);
   if (f == KVQ_FMT_LUT4 && d == 128) return capacity_t<KVQ_FMT_LUT4, 128>(cluster);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity_t<KVQ_FMT_NVFP4, 64>(cluster);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity_t<KVQ_FMT_NVFP4, 128>(cluster);
   if (f == KVQ_FMT_LUT4 && d == 64) return capacity_t<KVQ_FMT_LUT4, 64>(cluster);
   return 0;
 }

@@ -186,12 +186,17 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
 }
 
 // Barrier k (k = 1, 2, ...) among the CTAs that share `counter`, called by one thread of
-// each CTA after a block barrier: a fenced increment (publishing every write the CTA
-// made before that block barrier), then a wait until all `target` = k * n arrivals are
-// in, for at most kWaitCycles.  Returns false if the wait gave up.
+// each CTA after a block barrier: an increment with release semantics (publishing every
+// write the CTA made before that block barrier), then a wait until all `target` = k * n
+// arrivals are in, for at most kWaitCycles.  Returns false if the wait gave up.
+__device__ __forceinline__ int atom_add_release_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ bool cta_group_arrive_wait(int* counter, int target) {
-  __threadfence();
-  const int old = atomicAdd(counter, 1);
+  const int old = atom_add_release_gpu(counter, 1);
   if (old + 1 >= target) return true;
   const long long t0 = clock64();
   while (ld_acquire_gpu(counter) < target) {
@@ -203,8 +208,7 @@ __device__ __forceinline__ bool cta_group_arrive_wait(int* counter, int target) 
 
 // The two halves of cta_group_arrive_wait, for work that overlaps the wait.
 __device__ __forceinline__ void cta_group_arrive(int* counter) {
-  __threadfence();
-  atomicAdd(counter, 1);
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
 }
 __device__ __forceinline__ bool cta_group_wait(const int* counter, int target) {
   const long long t0 = clock64();

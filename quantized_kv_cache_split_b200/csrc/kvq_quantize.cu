@@ -1,4 +1,4 @@
-// Cache writers: fp16 K/V vectors -> q8_0 / q4_0 / rotated lut4 blocks.
+// Cache writers: fp16 K/V vectors -> q8_0 / q4_0 / rotated lut4 / nvfp4 blocks.
 //
 // One warp per (token, KV head) vector.  Lane l holds elements l, l+32, l+64,
 // l+96 (head_dim 128) or l, l+32 (head_dim 64), so a 32-element block is one
@@ -187,6 +187,91 @@ quant_lut4_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_
   if (lane == 0) norms[row] = __float2half_rn(n);
 }
 
+// ------------------------------------------------------------------ nvfp4
+// E2M1 magnitude code of |v|: the number of decision points passed, where the points
+// are the midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 between the values 0, 0.5, 1,
+// 1.5, 2, 3, 4, 6, and a value on a midpoint goes to the even code (round to nearest
+// even); above 6 it stays at 6 (saturation).  The sign bit follows the sign of v.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  const float mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  uint32_t c = 0;
+#pragma unroll
+  for (int k = 0; k < 7; ++k) c += (a > mid[k] || (a == mid[k] && (k & 1))) ? 1u : 0u;
+  return c | (signbit(v) ? 8u : 0u);
+}
+
+// E4M3 code of t >= 0: round to nearest even on the 3-bit mantissa, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_code(float t) {
+  if (!(t < 448.0f)) return 126u;                    // 448 and beyond (also NaN): 448
+  if (t < 0.015625f) {                               // below 2^-6: subnormal steps of 2^-9
+    const int m = __float2int_rn(__fmul_rn(t, 512.0f));  // exact scaling, ties to even
+    return (uint32_t)m;                              // m == 8 is the smallest normal, code 8
+  }
+  const uint32_t bits = __float_as_uint(t);
+  int e = (int)((bits >> 23) & 0xffu) - 127 + 7;     // biased E4M3 exponent, 1 .. 15
+  uint32_t q = (bits >> 20) & 7u;
+  const uint32_t rem = bits & 0xfffffu, half = 0x80000u;
+  if (rem > half || (rem == half && (q & 1u))) ++q;
+  if (q == 8u) { q = 0; ++e; }
+  if (e > 15 || (e == 15 && q == 7u)) return 126u;
+  return ((uint32_t)e << 3) | q;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const int e = (int)(code >> 3) & 15, m = (int)(code & 7u);
+  return e ? ldexpf((float)(8 + m), e - 10) : ldexpf((float)m, -9);
+}
+
+__device__ __forceinline__ float half_warp_max(float v) {
+#pragma unroll
+  for (int o = 8; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// nvfp4: g = amax/2688 over the vector; per 16-element block s = e4m3(amax_b / (6 g));
+// code = e2m1(x / (g s)).  Lane l holds elements l + 32 m, so block 2m + (l >> 4) is a
+// half-warp.  Scale row: the E4M3 bytes, then g (fp32), then zero padding.
+template <int D>
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+quant_nvfp4_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_t* __restrict__ slots,
+                   int page_size, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int NM = D / 32;
+  constexpr int SROWB = (D / 16 + 4 + 7) / 8 * 8;  // scale row bytes
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
+  if (vec >= (int64_t)n_tok * hkv) return;
+  const int64_t tok = vec / hkv;
+  const int h = (int)(vec - tok * hkv);
+  const int64_t slot = slots ? (int64_t)slots[tok] : tok;
+  const int64_t row = slot_row(slot, page_size, hkv, h);
+  const __half* xv = x + vec * D;
+  float v[NM];
+  float amax = 0.f;
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    v[m] = __half2float(xv[32 * m + lane]);
+    amax = fmaxf(amax, fabsf(v[m]));
+  }
+  amax = warp_max(amax);
+  const float g = __fdiv_rn(amax, 2688.0f);
+  const float six_g = __fmul_rn(6.0f, g);
+  uint8_t* srow = scales + row * SROWB;
+#pragma unroll
+  for (int m = 0; m < NM; ++m) {
+    const float amax_b = half_warp_max(fabsf(v[m]));
+    const float t = six_g > 0.f ? __fdiv_rn(amax_b, six_g) : 0.f;
+    const uint32_t sc = e4m3_code(t);
+    const float den = __fmul_rn(g, e4m3_value(sc));
+    const uint32_t q = den > 0.f ? e2m1_code(__fdiv_rn(v[m], den)) : 0u;
+    const uint32_t hi = __shfl_down_sync(0xffffffffu, q, 1);
+    if ((lane & 1) == 0) codes[row * (D / 2) + 16 * m + (lane >> 1)] = (uint8_t)(q | (hi << 4));
+    if ((lane & 15) == 0) srow[2 * m + (lane >> 4)] = (uint8_t)sc;
+  }
+  if (lane == 0) *reinterpret_cast<float*>(srow + D / 16) = g;
+  if (lane == 1 && SROWB > D / 16 + 4) *reinterpret_cast<uint32_t*>(srow + D / 16 + 4) = 0u;
+}
+
 }  // namespace
 
 int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,
@@ -210,6 +295,8 @@ int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const 
                  (__half*)scales)
   KVQ_QUANT_CASE(KVQ_FMT_LUT4, 128, quant_lut4_kernel, desc.codebook, desc.signs,
                  (uint8_t*)codes, (__half*)scales)
+  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 64, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales)
+  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 128, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales)
 #undef KVQ_QUANT_CASE
   return KVQ_ERR_UNSUPPORTED;
 }

@@ -42,6 +42,9 @@ def test_row_sizes():
     assert K.kvq_code_row_bytes("lut4", 64) == 32
     assert K.kvq_scale_row_count("q8_0", 128) == 4
     assert K.kvq_scale_row_count("lut4", 128) == 1
+    assert K.kvq_code_row_bytes("nvfp4", 128) == 64
+    # nvfp4 scale rows: D/16 E4M3 bytes + fp32 vector scale, padded to 8 bytes (fp16 slots)
+    assert K.kvq_scale_row_count("nvfp4", 128) == 8 and K.kvq_scale_row_count("nvfp4", 64) == 4
     assert K.kvq_code_row_bytes("q8_0", 96) == 0
 
 

@@ -29,7 +29,7 @@ def _special_vectors(rng, n, hkv, D):
     return x
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
 @pytest.mark.parametrize("D", [64, 128])
 def test_quantize_bit_exact(fmt, D):
     import quantized_kv_cache_split_b200 as K
@@ -55,7 +55,8 @@ def test_quantize_bit_exact(fmt, D):
         c, s = OQ.quantize(fmt, x[:, h], signs, cb16)
         want_c = c.astype(np.int8).view(np.uint8) if fmt == "q8_0" else OQ.pack_nibbles(c)
         assert np.array_equal(got_c, want_c), f"codes differ at {np.argwhere(got_c != want_c)[:5]}"
-        assert np.array_equal(got_s.view(np.uint16), s.astype(np.float16).view(np.uint16)), "scales"
+        want_s = s if fmt == "nvfp4" else s.astype(np.float16).view(np.uint16)  # nvfp4: raw words
+        assert np.array_equal(got_s.view(np.uint16), want_s), "scales"
     assert np.array_equal(cache.v_codes.cpu().numpy(), codes)
 
 
@@ -159,7 +160,7 @@ def test_in_kernel_merge_resets_its_counters():
 RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
 @pytest.mark.parametrize("tau,split,scope", [(0.0, 128, "split"), (1e-6, 0, "split"), (1e-4, 192, "split"),
                                              (1e-6, 1024, "split"), (1e-6, 128, "cluster"),
                                              (1e-6, 0, "sequence")])
@@ -174,7 +175,7 @@ def test_decode_parity_paged_ragged(fmt, tau, split, scope):
     assert g["flags"] == 0
 
 
-@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4"])
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (8, 1)])
 def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
     wl = W.WORKLOADS["tiny_q8_d64"].with_(fmt=fmt, num_q_heads=hq, num_kv_heads=hkv,
@@ -189,7 +190,7 @@ def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
 
 # ------------------------------------------------------------------ full sizes
 
-@pytest.mark.parametrize("name", ["gqa_32k_q4", "lut_32k"])
+@pytest.mark.parametrize("name", ["gqa_32k_q4", "lut_32k", "nvfp4_32k"])
 @pytest.mark.parametrize("tau,scope", [(1e-6, "split"), (0.0, "split"), (1e-6, "cluster"),
                                        (1e-6, "sequence")])
 def test_decode_parity_full_32k(name, tau, scope):

@@ -40,6 +40,7 @@ import numpy as np
 FMT_Q8_0 = "q8_0"
 FMT_Q4_0 = "q4_0"
 FMT_LUT4 = "lut4"
+FMT_NVFP4 = "nvfp4"
 
 
 @dataclasses.dataclass(frozen=True)
@@ -87,6 +88,9 @@ WORKLOADS = {
                        FMT_LUT4, (0.0, 1e-6), 1004),
     "lut_32k": Workload("lut_32k", 1, 32, 4, 128, (32768,), 64, 10.0, 20.0,
                         FMT_LUT4, (0.0, 1e-6), 1014),
+    # NVFP4 (E2M1 + E4M3 block scales) at the 32K GQA-8 shape.
+    "nvfp4_32k": Workload("nvfp4_32k", 1, 32, 4, 128, (32768,), 64, 10.0, 20.0,
+                          FMT_NVFP4, (0.0, 1e-6), 1023),
     # 8 concurrent streams, paged 64-token pages, mixed context lengths.
     "paged_b8_q8": Workload("paged_b8_q8", 8, 32, 4, 128, _PAGED_LENS, 64, 10.0, 20.0,
                             FMT_Q8_0, (0.0, 1e-6, 1e-4), 1005, page_size=64),

@@ -303,6 +303,7 @@ def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int, with_o: 
 
 def gpu_arm(args, world, rank, local):
     import torch
+    import quantized_kv_cache_split_b200 as K
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     init_dist(world, "nccl")
@@ -324,7 +325,11 @@ def gpu_arm(args, world, rank, local):
     variants = (("sparse", args.tau, "split"), ("dense", 0.0, "split"),
                 ("sparse_cluster_max", args.tau, "cluster"), ("sparse_sequence_max", args.tau, "sequence"))
     for tag, tau, scope in variants:
-        st = counters(tau, scope)
+        try:
+            st = counters(tau, scope)
+        except K.KvqError as e:  # the sequence-wide maximum needs every split on its own CTA
+            res[tag] = {"max_scope": scope, "unavailable": str(e)}
+            continue
         step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope), rep.R)
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)

@@ -155,9 +155,10 @@ int32_t kvq_resolve_cluster(const kvq_cache_desc* desc, int32_t batch, int32_t n
 size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                           int32_t max_seq_len, int32_t split_tokens);
 
-/* Zero the workspace (its device flag word and the merge counters); call once after
- * allocating it.  A workspace whose call to kvq_decode_attn completed is ready for
- * the next call without another init. */
+/* Zero the workspace (its device flag word, the launch counter that tags the (m, l)
+ * exchange and the merge counters); call once after allocating it.  A workspace whose
+ * call to kvq_decode_attn completed is ready for the next call without another init,
+ * whatever the next call's shape; after KVQ_FLAG_TIMEOUT, init it again. */
 int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronize `stream` and read the device flag word (KVQ_FLAG_* bits) into *flags (host). */

@@ -54,7 +54,6 @@ class QuantizedKVCache:
         self.desc = kb.make_desc(fmt, head_dim, num_kv_heads, page_size, num_pages,
                                  self.codebook, self.signs)
         self._ws = None
-        self._ws_key = None
 
     # ---------------------------------------------------------------- writes
     def write(self, k: torch.Tensor, v: torch.Tensor, slots: Optional[torch.Tensor] = None,
@@ -69,13 +68,9 @@ class QuantizedKVCache:
                   options: int = 0):
         L = kb.kvq_resolve_split(self.desc, batch, num_q_heads, max_seq_len, split_tokens, options)
         nbytes = kb.kvq_workspace_size(batch, num_q_heads, self.head_dim, max_seq_len, L)
-        key = (batch, num_q_heads)
         if self._ws is None or self._ws.numel() < nbytes:
             self._ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
-            self._ws_key = None
-        if self._ws_key != key:  # the merge counters move with (batch, heads): zero them
-            kb.kvq_workspace_init(self._ws, self._ws.numel())
-            self._ws_key = key
+            kb.kvq_workspace_init(self._ws, self._ws.numel())  # once; any later shape reuses it
         return self._ws, nbytes, L
 
     def attention(self, q: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,

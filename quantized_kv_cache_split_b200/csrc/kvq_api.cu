@@ -14,7 +14,7 @@ namespace kvq {
 
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits) {
   const size_t units = (size_t)batch * num_q_heads * max_splits;
-  return units * ((size_t)head_dim + 2 + 2) * sizeof(float);  // o, m, l, then the (m, l) exchange
+  return units * (16 + ((size_t)head_dim + 2) * sizeof(float));  // (m, l) exchange, o, m, l
 }
 
 int device_sm_count() {
@@ -243,13 +243,13 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.workspace = workspace;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.counters = reinterpret_cast<int*>(ws + kWorkspaceHeader);
-  a.tallies = a.counters + (size_t)batch * num_q_heads;
+  a.epoch = reinterpret_cast<unsigned long long*>(ws + kEpochOffset);
   a.group_merge = 0;  // decided at launch
   const size_t n_part = (size_t)batch * num_q_heads * a.max_splits;
-  a.part_o = reinterpret_cast<float*>(ws + kWorkspaceHeader + counters_bytes(batch, num_q_heads));
+  a.xch = reinterpret_cast<ulonglong2*>(ws + kWorkspaceHeader + counters_bytes(batch, num_q_heads));
+  a.part_o = reinterpret_cast<float*>(a.xch + n_part);
   a.part_m = a.part_o + n_part * desc->head_dim;
   a.part_l = a.part_m + n_part;
-  a.xch = reinterpret_cast<float2*>(a.part_l + n_part);
   a.stats = stats;
   a.out = out;
   a.cluster = CS;

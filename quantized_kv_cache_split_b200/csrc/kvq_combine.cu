@@ -29,8 +29,10 @@ combine_kernel(const uint8_t* __restrict__ ws, int batch, int hq, int max_seq_le
   const int bh = blockIdx.x;
   const int b = bh / hq;
   const int tid = threadIdx.x;
-  const float* o = reinterpret_cast<const float*>(ws + kWorkspaceHeader + counters_bytes(batch, hq));
   const size_t n_part = (size_t)batch * hq * max_splits;
+  // the partials follow the header, the merge counters and the (m, l) exchange entries
+  const float* o = reinterpret_cast<const float*>(ws + kWorkspaceHeader + counters_bytes(batch, hq) +
+                                                  16 * n_part);
   const float* m = o + n_part * D;
   const float* l = m + n_part;
   const int n = max(0, min(seq_lens[b], max_seq_len));

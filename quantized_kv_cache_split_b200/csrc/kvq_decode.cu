@@ -364,6 +364,56 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
   }
 }
 
+// (M, L) of the exchange entries e[u] this lane takes: u = first + step * t (t < T) in
+// every pass of T * step entries, u < n, none when !active; M is their maximum and L
+// their denominators rescaled to it.  Each pass waits until all its entries carry this
+// launch's tag (its loads all in flight together); false if that took longer than
+// kWaitCycles.  Warp-uniform: every lane of the warp calls it with the same n.
+template <int T>
+__device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int step, int n,
+                                           bool active, uint32_t tag, float& M, float& L) {
+  M = -INFINITY;
+  L = 0.f;
+  for (int ub = 0; ub < n; ub += T * step) {
+    float mv[T], lv[T];
+    const long long t0 = clock64();
+    for (;;) {
+      bool all = true;
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        const int u = ub + first + step * t;
+        mv[t] = -INFINITY;
+        lv[t] = 0.f;
+        if (active && u < n) all &= xch_load(e + u, tag, mv[t], lv[t]);
+      }
+      if (__all_sync(0xffffffffu, all)) break;
+      if (__any_sync(0xffffffffu, clock64() - t0 > kWaitCycles)) return false;
+      __nanosleep(32);
+    }
+    float bm = M;
+#pragma unroll
+    for (int t = 0; t < T; ++t) bm = fmaxf(bm, mv[t]);
+    float ds = (M == -INFINITY) ? 0.f : L * ex2(M - bm);
+#pragma unroll
+    for (int t = 0; t < T; ++t)
+      if (mv[t] != -INFINITY) ds = fmaf(ex2(mv[t] - bm), lv[t], ds);
+    M = bm;
+    L = ds;
+  }
+  return true;
+}
+
+// Combine (M, L) across the lanes that differ in bits 1 .. max_off of the lane index.
+__device__ __forceinline__ void xch_combine(float& M, float& L, int max_off) {
+  for (int o = 1; o <= max_off; o <<= 1) {
+    const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
+    const float Lo = __shfl_xor_sync(0xffffffffu, L, o);
+    const float nm = fmaxf(M, Mo);
+    L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + (Mo == -INFINITY ? 0.f : Lo * ex2(Mo - nm));
+    M = nm;
+  }
+}
+
 // bit 4r set iff any of bits 4r .. 4r+3 of a ballot is set (one row per 4-lane group)
 __device__ __forceinline__ uint32_t rows_of(uint32_t bal) {
   uint32_t x = bal | (bal >> 1);
@@ -643,6 +693,18 @@ decode_kernel(const DecodeArgs a) {
   // input before the preceding grid has finished and its writes are visible.
   grid_dependents_launch();
   grid_dependency_wait();
+  // Every CTA takes part in the launch count that tags the (m, l) exchange.  A CTA with
+  // work has its last warp read the counter and the first 32 sequence lengths here, ahead
+  // of the first copies (a load issued behind them waits for them), and store what it
+  // read behind them.
+  unsigned long long ep_raw = 0;
+  int len_raw = 0;
+  if (cid >= total) {
+    if (tid == 0) epoch_advance(a.epoch);  // no work: only the count
+  } else if (warp == kWarps - 1) {
+    if (lane == 0) ep_raw = epoch_read(a.epoch);
+    if (lane < B) len_raw = __ldg(a.seq_lens + lane);
+  }
 
   Lut lut;
   if constexpr (C::kLut) {
@@ -697,8 +759,7 @@ decode_kernel(const DecodeArgs a) {
     // units know the length before copying anything.
     int nb;
     if (k == 0) {
-      nb = __shfl_sync(0xffffffffu, lane == 0 ? __ldg(a.seq_lens + b) : 0, 0);
-      nb = max(0, min(nb, cap));
+      nb = __ldg(a.seq_lens + b);  // in flight while the copies are issued
     } else {
       __syncthreads();  // the lengths in shared memory are visible (the first unit may have had no barrier)
       nb = slen[b];
@@ -751,12 +812,20 @@ decode_kernel(const DecodeArgs a) {
       }
     }
     if (k == 0) {
-      // clamped sequence lengths for later units and the final zero fill (read once,
-      // behind the first copies; visible after the next barrier)
-      for (int bb = tid; bb < B; bb += kThreads) {
-        const int n = a.seq_lens[bb];
-        if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
-        slen[bb] = max(0, min(n, cap));
+      nb = max(0, min(nb, cap));
+      // this launch's exchange tag, and the clamped sequence lengths for later units and
+      // the final zero fill, stored by the last warp (which builds no query fragments)
+      // from what it read before the copies; visible after the next barrier
+      if (warp == kWarps - 1) {
+        if (lane == 0) {
+          epoch_advance(a.epoch);
+          misc[3] = (int)epoch_tag(ep_raw);  // read after the next barrier
+        }
+        for (int bb = lane; bb < B; bb += 32) {
+          const int n = bb < 32 ? len_raw : a.seq_lens[bb];
+          if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
+          slen[bb] = max(0, min(n, cap));
+        }
       }
     }
     if (k == 0 && cu * CS * Ls >= nb) {  // a speculative unit past the sequence's end
@@ -845,11 +914,14 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red_m[w * 8 + tid]);
       cmx[tid] = m;
-      if (tid == 0) misc[2] = 0;  // warps done with their V pass (read after the next barrier)
+      if (tid == 0) {
+        misc[0] = misc[1] = 1;  // exchanges not failed (yet)
+        misc[2] = 0;            // warps done with their V pass (read after the next barrier)
+      }
     }
     if (CS > 1) cluster_sync(); else __syncthreads();  // CTA maxima visible (cluster-wide)
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
-    int nbar = 0;  // group barriers this unit has passed (barrier k waits for k * n arrivals)
+    const uint32_t tag = (uint32_t)misc[3];
     if (a.global_max) {
       // every split publishes its maxima and its denominators relative to them; after one
       // barrier among the splits of this (sequence, KV head) each derives the final
@@ -874,47 +946,32 @@ decode_kernel(const DecodeArgs a) {
         red_l[warp * 8 + 2 * c] = lo0;
         red_l[warp * 8 + 2 * c + 1] = lo1;
       }
-      __syncthreads();
+      const bool zero_out = a.out && a.group_merge && cu == 0;
+      if (zero_out)
+        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
+      __syncthreads();  // every warp's l is in shared memory, the output rows are cleared
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        a.xch[slot0 + (size_t)tid * a.max_splits] = make_float2(cmx[tid], l);
+        if (zero_out) __threadfence();  // the cleared rows are visible before this entry
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, cmx[tid], l);
       }
-      if (a.out && a.group_merge && cu == 0)
-        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
-      __syncthreads();
-      ++nbar;
-      if (tid == 0) {
-        misc[1] = cta_group_arrive_wait(a.counters + (size_t)b * hkv + kvh, nbar * n);
-        cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, n);
-        misc[0] = misc[1];
-        if (!misc[1]) set_flag(flags, KVQ_FLAG_TIMEOUT);
-      }
-      __syncthreads();
-      if (misc[1]) {
-        __threadfence();
-        if (warp < G) {  // M and L of head `warp` over all splits
-          const size_t uw = ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits;
-          float M = -INFINITY, L = 0.f;
-          for (int ub = 0; ub < n; ub += 32) {
-            const int u = ub + lane;
-            const float2 e = u < n ? __ldcg(a.xch + uw + u) : make_float2(-INFINITY, 0.f);
-            float bm = e.x;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-            const float nm = fmaxf(M, bm);
-            float ds = e.x == -INFINITY ? 0.f : ex2(e.x - nm) * e.y;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + ds;
-            M = nm;
-          }
+      if (warp < G) {  // M and L of head `warp` over all splits, once every entry is in
+        float M, L;
+        const bool ok = xch_reduce<4>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits,
+                                      lane, 32, n, true, tag, M, L);
+        if (ok) {
+          xch_combine(M, L, 16);
           if (lane == 0) {
             cmx[8 + warp] = M;
             cmx[16 + warp] = 1.f / L;  // this split's share: 2^(M - M) / L
           }
+        } else if (lane == 0) {
+          set_flag(flags, KVQ_FLAG_TIMEOUT);
+          misc[0] = misc[1] = 0;
         }
+        __threadfence();  // what the other splits wrote before their entries is visible
       }
       __syncthreads();
     }
@@ -1031,18 +1088,16 @@ decode_kernel(const DecodeArgs a) {
     const bool add_merge = a.out && a.group_merge;
     const int nsplit = (nb + Ls - 1) / Ls;
     if (add_merge && !a.global_max) {
-      __syncthreads();  // every warp's l is in shared memory
+      if (cu == 0)
+        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
+      __syncthreads();  // every warp's l is in shared memory, the output rows are cleared
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        a.xch[slot0 + (size_t)tid * a.max_splits] = make_float2(mpart[tid], l);
+        if (cu == 0) __threadfence();  // the cleared rows are visible before this entry
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mpart[tid], l);
       }
-      if (cu == 0)
-        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
-      __syncthreads();
-      ++nbar;
-      if (tid == 0) cta_group_arrive(a.counters + (size_t)b * hkv + kvh);
     }
 
     // ---- V pass: this warp's kept positions only
@@ -1107,50 +1162,20 @@ decode_kernel(const DecodeArgs a) {
       if (lane == 0) first = atomicAdd(&misc[2], 1) == 0;
       first = __shfl_sync(0xffffffffu, first, 0);
       if (first) {
-        int ok = 0;
-        if (lane == 0) {
-          ok = cta_group_wait(a.counters + (size_t)b * hkv + kvh, nbar * nsplit);
-          cta_group_done(a.counters + (size_t)b * hkv + kvh, a.tallies + (size_t)b * hkv + kvh, nsplit);
-          if (!ok) set_flag(flags, KVQ_FLAG_TIMEOUT);
-          misc[0] = ok;
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
+        // partials in flight together), then combine across the four lanes
+        const int h = lane >> 2, j = lane & 3;
+        float M, L;
+        const bool ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
+                                       j, 4, nsplit, h < G, tag, M, L);
         if (ok) {
-          __threadfence();
-          // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads in flight
-          // together for up to 64 partials), then combine across the four lanes
-          const int h = lane >> 2, j = lane & 3;
-          const size_t uh = ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits;
-          float M = -INFINITY, L = 0.f;
-          for (int ub = 0; ub < nsplit; ub += 64) {
-            float mv[16], lv[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t) {
-              const int u = ub + j + 4 * t;
-              const float2 e = h < G && u < nsplit ? __ldcg(a.xch + uh + u) : make_float2(-INFINITY, 0.f);
-              mv[t] = e.x;
-              lv[t] = e.y;
-            }
-            float bm = M;
-#pragma unroll
-            for (int t = 0; t < 16; ++t) bm = fmaxf(bm, mv[t]);
-            float ds = (M == -INFINITY) ? 0.f : L * ex2(M - bm);
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-              if (mv[t] != -INFINITY) ds = fmaf(ex2(mv[t] - bm), lv[t], ds);
-            M = bm;
-            L = ds;
-          }
-#pragma unroll
-          for (int o = 1; o < 4; o <<= 1) {  // combine (M, L) of the four lanes of head h
-            const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
-            const float Lo = __shfl_xor_sync(0xffffffffu, L, o);
-            const float nm = fmaxf(M, Mo);
-            L = (M == -INFINITY ? 0.f : L * ex2(M - nm)) + (Mo == -INFINITY ? 0.f : Lo * ex2(Mo - nm));
-            M = nm;
-          }
+          xch_combine(M, L, 2);
           if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
+        } else if (lane == 0) {
+          set_flag(flags, KVQ_FLAG_TIMEOUT);
+          misc[0] = 0;
         }
+        __threadfence();  // what the other splits wrote before their entries is visible
       }
     }
     cp_async_wait<0>();  // nothing of this split stays in flight
@@ -1492,7 +1517,7 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
   }
   if (a.grid <= 0) return KVQ_OK;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.cluster;
   attr[0].val.clusterDim.y = 1;
@@ -1508,17 +1533,27 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
                   (int64_t)a.batch * a.units_per_seq * a.desc.num_kv_heads <= a.grid;
   int na = 0;
   if (a.cluster > 1) attr[na++] = attr[0];
-  if (b.group_merge || a.global_max) {  // CTAs wait for one another: all resident together
+  const bool coop = b.group_merge || a.global_max;
+  if (coop) {  // CTAs wait for one another: all resident together
     attr[na].id = cudaLaunchAttributeCooperative;
     attr[na].val.cooperative = 1;
-  } else {
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
   }
+  // Programmatic dependent launch: this grid may be set up while the previous kernel on
+  // the stream finishes (every CTA waits for that kernel before reading anything, so a
+  // cooperative grid still has all its CTAs resident once it proceeds).
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
   ++na;
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, decode_kernel<FMT, D>, b) != cudaSuccess) return KVQ_ERR_CUDA;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<FMT, D>, b);
+  if (e != cudaSuccess && coop) {  // a driver that does not take both: cooperative alone
+    (void)cudaGetLastError();
+    cfg.numAttrs = na - 1;
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<FMT, D>, b);
+  }
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 

@@ -172,51 +172,61 @@ __device__ __forceinline__ float dsmem_ld(uint32_t addr) {
   return v;
 }
 
-// ------------------------------------------------------------------ inter-CTA signalling
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+// ------------------------------------------------------------------ tagged exchange
+// The splits of one (sequence, KV head) publish their (m, l) to one another through
+// 64-bit words that each carry a launch tag in the high half, so a reader needs no
+// separate arrival counter: an entry is this launch's once its tag matches.  A 64-bit
+// access is single-copy atomic, so value and tag are always seen together.
+//
+// The tag comes from a launch counter in the workspace header.  Every CTA reads it at
+// its start and then adds its share of kEpochStep (CTA 0: kEpochStep - (grid - 1), the
+// others 1), so each launch adds exactly kEpochStep; a CTA's read sees the previous
+// launches' total plus less than kEpochStep of this launch's own adds, so
+// read / kEpochStep is the same launch number e for every CTA, and the tag is e + 1.
+constexpr int kEpochShift = 16;
+constexpr unsigned long long kEpochStep = 1ull << kEpochShift;  // > any grid
+constexpr size_t kEpochOffset = 8;                               // byte offset in the header
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Barrier k (k = 1, 2, ...) among the CTAs that share `counter`, called by one thread of
-// each CTA after a block barrier: an increment with release semantics (publishing every
-// write the CTA made before that block barrier), then a wait until all `target` = k * n
-// arrivals are in, for at most kWaitCycles.  Returns false if the wait gave up.
-__device__ __forceinline__ int atom_add_release_gpu(int* p, int v) {
-  int old;
-  asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
+// One thread of every CTA: read the counter (epoch_read), then add this CTA's share
+// (epoch_advance, after the read); the tag is epoch_tag of what was read.
+__device__ __forceinline__ unsigned long long epoch_read(const unsigned long long* epoch) {
+  return ld_relaxed_u64(epoch);
+}
+__device__ __forceinline__ void epoch_advance(unsigned long long* epoch) {
+  red_add_u64(epoch, blockIdx.x == 0 ? kEpochStep - (gridDim.x - 1) : 1ull);
+}
+__device__ __forceinline__ uint32_t epoch_tag(unsigned long long read) {
+  return (uint32_t)(read >> kEpochShift) + 1u;
 }
 
-__device__ __forceinline__ bool cta_group_arrive_wait(int* counter, int target) {
-  const int old = atom_add_release_gpu(counter, 1);
-  if (old + 1 >= target) return true;
-  const long long t0 = clock64();
-  while (ld_acquire_gpu(counter) < target) {
-    if (clock64() - t0 > kWaitCycles) return false;
-    __nanosleep(32);
-  }
-  return true;
+__device__ __forceinline__ unsigned long long tag_word(uint32_t tag, float v) {
+  return ((unsigned long long)tag << 32) | __float_as_uint(v);
 }
 
-// The two halves of cta_group_arrive_wait, for work that overlaps the wait.
-__device__ __forceinline__ void cta_group_arrive(int* counter) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
+// One entry: (m, l) of one head of one split, each word tagged.
+__device__ __forceinline__ void xch_store(ulonglong2* p, uint32_t tag, float m, float l) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(tag_word(tag, m)),
+               "l"(tag_word(tag, l))
+               : "memory");
 }
-__device__ __forceinline__ bool cta_group_wait(const int* counter, int target) {
-  const long long t0 = clock64();
-  while (ld_acquire_gpu(counter) < target) {
-    if (clock64() - t0 > kWaitCycles) return false;
-    __nanosleep(32);
-  }
-  return true;
+
+// Read an entry; false while it is not this launch's (tag mismatch in either word).
+__device__ __forceinline__ bool xch_load(const ulonglong2* p, uint32_t tag, float& m, float& l) {
+  unsigned long long a, b;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+  m = __uint_as_float((uint32_t)a);
+  l = __uint_as_float((uint32_t)b);
+  return (uint32_t)(a >> 32) == tag && (uint32_t)(b >> 32) == tag;
 }
 
 // out[0..3] += v, one vector reduction in global memory (16-byte aligned address).
@@ -224,15 +234,6 @@ __device__ __forceinline__ void red_add_f32x4(float* out, float4 v) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(out), "f"(v.x), "f"(v.y),
                "f"(v.z), "f"(v.w)
                : "memory");
-}
-
-// Called by one thread of each of the `n` CTAs once it no longer waits on `counter`:
-// the last of them zeroes the counter (and this tally) for the next launch.
-__device__ __forceinline__ void cta_group_done(int* counter, int* tally, int n) {
-  if (atomicAdd(tally, 1) == n - 1) {
-    atomicExch(counter, 0);
-    atomicExch(tally, 0);
-  }
 }
 
 // ------------------------------------------------------------------ programmatic dependent launch

@@ -27,11 +27,13 @@ struct DecodeArgs {
   int split_tokens;   // resolved, multiple of kTile
   int max_splits;     // ceil(max_seq_len / split_tokens)
   void* workspace;
-  int* counters;      // [batch][num_kv_heads] arrival counters of the in-kernel merge
+  int* counters;      // [batch][num_kv_heads] arrival counters of the last-arrival merge
+  unsigned long long* epoch;  // launch counter in the workspace header (exchange tags)
   float* part_o;      // partials, see below
   float* part_m;
   float* part_l;
-  float2* xch;        // (m, l) each split publishes for the others [batch][num_q_heads][max_splits]
+  ulonglong2* xch;    // tagged (m, l) each split publishes for the others
+                      // [batch][num_q_heads][max_splits]
   unsigned long long* stats;
   float* out;         // non-null: merge in the same kernel and write the output
   int cluster;        // consecutive splits per thread-block cluster (1, 2 or 4)
@@ -39,22 +41,23 @@ struct DecodeArgs {
   int global_max;     // every split of a (sequence, KV head) uses the maximum over all of them
   int grid;           // CTAs launched (a multiple of cluster)
   int units_per_seq;  // cluster groups of one (sequence, KV head) at max_seq_len
-  int group_merge;    // every unit has its own CTA: the CTAs of a (sequence, KV head) meet
-                      // at a barrier and each merges some of its heads
-  int* tallies;       // [batch][num_kv_heads] CTAs done with the group barriers
+  int group_merge;    // every unit has its own CTA: the splits of a (sequence, KV head)
+                      // exchange (m, l) and each adds its share into the output
 };
 
-// Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits); the merge / barrier counters
-// and the barrier tallies (int32 [batch][num_q_heads] each reserved, together rounded up
-// to 256 bytes); then the partials, one slot per cluster of splits:
+// Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch
+// counter that tags the exchange entries); the last-arrival merge counters (int32
+// [batch][num_q_heads] reserved, rounded up to 256 bytes); then, one slot per cluster of
+// splits:
+//   (m, l) exchange [batch][num_q_heads][max_splits] 2 x u64, each word a fp32 value
+//   under a 32-bit launch tag (what the splits of a (sequence, KV head) publish to one
+//   another)
 //   o [batch][num_q_heads][max_splits][head_dim] fp32 (unnormalized)
 //   m [batch][num_q_heads][max_splits] fp32 (running maximum, log2 units)
 //   l [batch][num_q_heads][max_splits] fp32
-//   (m, l) exchange [batch][num_q_heads][max_splits] fp32 x 2 (what the splits of a
-//   (sequence, KV head) publish to one another at their group barrier)
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits);
 __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
-  return ((size_t)2 * batch * num_q_heads * sizeof(int32_t) + 255) / 256 * 256;
+  return ((size_t)batch * num_q_heads * sizeof(int32_t) + 255) / 256 * 256;
 }
 
 int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,

@@ -57,8 +57,12 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q
   int st = scratch_address(&ws);
   if (st != KVQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the flag word and the merge counters must start at zero for every call
-  if (cudaMemsetAsync(ws, 0, kWorkspaceHeader + counters_bytes(batch, num_q_heads), s) != cudaSuccess)
+  // the flag word and the merge counters start at zero for every call; the launch
+  // counter in the header (bytes 8..15) keeps counting, so that no exchange entry left
+  // by an earlier call carries the tag of this one
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess ||
+      cudaMemsetAsync(static_cast<uint8_t*>(ws) + kWorkspaceHeader, 0, counters_bytes(batch, num_q_heads),
+                      s) != cudaSuccess)
     return KVQ_ERR_CUDA;
   // the merge runs inside the decode kernel (output pointer given)
   return kvq_decode_attn(desc, q, batch, num_q_heads, k_codes, k_scales, v_codes, v_scales,

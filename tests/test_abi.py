@@ -76,9 +76,9 @@ def test_split_resolution_and_workspace_size():
     assert K.kvq_resolve_split(d, 1, 32, 4096, 5000) == K.KVQ_MAX_SPLIT_TOKENS
     assert K.kvq_resolve_split(d, 1, 32, 4096, 1) == 64
     ws = K.kvq_workspace_size(2, 32, 128, 1000, 128)
-    # header, barrier counters, partials (o, m, l) and the (m, l) exchange
-    assert ws == 256 + 512 + 2 * 32 * 8 * (128 + 4) * 4
-    assert K.kvq_workspace_size(3, 32, 128, 1000, 128) == 256 + 768 + 3 * 32 * 8 * (128 + 4) * 4
+    # header, merge counters, then per partial the tagged (m, l) exchange entry and (o, m, l)
+    assert ws == 256 + 256 + 2 * 32 * 8 * (16 + (128 + 2) * 4)
+    assert K.kvq_workspace_size(3, 32, 128, 1000, 128) == 256 + 512 + 3 * 32 * 8 * (16 + (128 + 2) * 4)
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -157,6 +157,38 @@ def test_in_kernel_merge_resets_its_counters():
         np.testing.assert_allclose(o, outs[0], rtol=0, atol=1e-5 * vmax)
 
 
+def test_exchange_across_request_shapes_on_one_workspace():
+    # The splits of a (sequence, KV head) find one another's (m, l) by a launch tag, not by
+    # counters at shape-dependent places: requests of different batch sizes alternate on one
+    # workspace with no re-init, and each must give what the full request gives for the
+    # same sequences.  Every launch adds exactly 2^16 to the launch counter (header bytes
+    # 8..15), whatever its grid.
+    wl = W.shrink(W.WORKLOADS["paged_b8_q4"], [3000, 64, 0, 1500, 777], n_planted=8)
+    inp = W.generate(wl)
+    g = run_library(inp, 1e-6, 512)  # every split on its own CTA: the exchange path
+    cache = g["cache"]
+    dev = torch.device("cuda")
+    q = torch.from_numpy(inp.q).to(dev)
+    seq = torch.from_numpy(inp.seq_lens).to(dev)
+    pt = torch.from_numpy(inp.page_table).to(dev)
+    sel = torch.tensor([3, 0], device=dev)
+    sm = float(np.float32(1 / math.sqrt(128)))
+    vmax = float(np.abs(inp.v.astype(np.float32)).max())
+    launches = 1  # run_library's call initialized the workspace and launched once
+    for scope in ("split", "sequence", "split"):
+        full = cache.attention(q, seq, 3000, pt, inp.max_pages, tau=1e-6, sm_scale=sm,
+                               split_tokens=512, max_scope=scope)
+        sub = cache.attention(q[sel].contiguous(), seq[sel].contiguous(), 3000, pt[sel].contiguous(),
+                              inp.max_pages, tau=1e-6, sm_scale=sm, split_tokens=512, max_scope=scope)
+        launches += 2
+        np.testing.assert_allclose(sub.cpu().numpy(), full[sel].cpu().numpy(), rtol=0, atol=1e-5 * vmax)
+        if scope == "split":
+            np.testing.assert_allclose(full.cpu().numpy(), g["out"], rtol=0, atol=1e-5 * vmax)
+    assert cache.device_flags() == 0
+    header = cache._ws[:16].cpu().numpy()
+    assert int(header[8:16].view(np.uint64)[0]) == launches * (1 << 16)
+
+
 RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 
 

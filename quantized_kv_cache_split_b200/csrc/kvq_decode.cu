@@ -95,11 +95,16 @@ struct Cfg {
   static constexpr int NE = MT * 4;                      // accumulator registers per thread
   static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
   static constexpr int NWORD = RAWB / 4;
-  static constexpr int VSTRIDE = CROW + 16;              // gathered row: codes + scale window
-  static constexpr int VGROUP = 16 * VSTRIDE;            // one group of 16 gathered rows
-  // per-warp buffer: its K tile, then its gathered V rows (all 4 groups), then its
-  // accumulators for the block-wide sum
-  static constexpr int KBUF = round128(cmax3(TILE, 4 * VGROUP, NE * 32 * 4));
+  // q8_0 / q4_0 V pass: codes enter the MMA as magic-number fp16 (code + offset) read
+  // with transposing matrix loads, the scale rides on the weights (see v_group_mag)
+  static constexpr bool kMag = kQ8 || kQ4;
+  // V staging (a whole tile or gathered rows): codes at row stride CROW with the same
+  // chunk swizzle as K, then a tile's scale rows (SROW each) or, for gathered rows, the
+  // 16-byte window of the scales plane that holds each row's scales
+  static constexpr int GSC = STAGE_CODE;                  // gathered rows' scale windows
+  // per-warp buffer: its K tile, then its staged V rows, then its accumulators for the
+  // block-wide sum
+  static constexpr int KBUF = round128(cmax3(TILE, STAGE_CODE + kTile * 16, NE * 32 * 4));
   static constexpr int VT = round128(TILE);              // per-warp prefetched V tile (tau = 0)
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
@@ -596,12 +601,39 @@ __device__ __forceinline__ void build_query(const QRaw<D>& q, int c,
 }
 
 // ------------------------------------------------------------------ V groups
-// One group of 16 staged V positions: acc[dims x heads] += v_hat^T p.  TILE: the
-// positions are rows s0 .. s0 + 15 of a staged tile (codes rows, then scale rows);
-// otherwise they are gathered rows, each its codes followed by the 16-byte window of
-// the scales plane that holds its scales (trow: the row's index in its tile).  Slots
-// at or past n_valid get scale 0, so whatever bytes they hold contribute nothing
-// (every format decodes any bit pattern to a finite value).
+// Chunk swizzle of a staged row (K tiles and V rows alike): 16-byte chunk cc of row `row`
+// sits at chunk position cc ^ swz(row).
+template <int FMT, int D>
+__device__ __forceinline__ int swz(int row) {
+  using C = Cfg<FMT, D>;
+  return (row >> C::SWZ_SHIFT) & C::SWZ_MASK;
+}
+
+// Stage the whole 64-row V tile that starts at plane row row0: codes swizzled, then the
+// scale rows (one copy group).
+template <int FMT, int D>
+__device__ __forceinline__ void copy_v_tile(uint8_t* dst, const uint8_t* vcodes, const uint8_t* vscales,
+                                            size_t row0, int lane) {
+  using C = Cfg<FMT, D>;
+  constexpr int CPR = C::CROW / 16;
+  const uint8_t* src = vcodes + row0 * C::CROW;
+#pragma unroll 4
+  for (int i = lane; i < kTile * CPR; i += 32) {
+    const int row = i / CPR, cc = i % CPR;
+    cp_async16(dst + row * C::CROW + ((cc ^ swz<FMT, D>(row)) << 4), src + (size_t)row * C::CROW + cc * 16);
+  }
+  const uint8_t* ssrc = vscales + row0 * C::SROW;
+#pragma unroll
+  for (int i = lane; i < C::STAGE_SC / 16; i += 32) cp_async16(dst + C::STAGE_CODE + i * 16, ssrc + i * 16);
+  cp_async_commit();
+}
+
+// lut4 / nvfp4: one group of 16 staged V positions (slots s0 .. s0 + 15 of the staging
+// buffer): acc[dims x heads] += v_hat^T p.  TILE: slot s is row s of a staged tile;
+// otherwise a gathered row whose scales sit in its window at (trow & (RPW - 1)) * SROW
+// (trow: the row's index in its tile).  Slots at or past n_valid (counted from s0) get
+// scale 0, so whatever bytes they hold contribute nothing (every format decodes any bit
+// pattern to a finite value).  Thread (r, c) owns dims E*r .. E*r + E - 1.
 template <int FMT, int D, bool TILE>
 __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const __half* __restrict__ prow,
                                         const uint8_t* __restrict__ trow, int s0, int n_valid,
@@ -613,12 +645,13 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const _
   const uint32_t b0 = lds32(prow + sa);
   const uint32_t b1 = lds32(prow + sc);
   auto code = [&](int slot) -> const uint8_t* {
-    return TILE ? buf + (s0 + slot) * C::CROW + C::RAWB * r : buf + slot * C::VSTRIDE + C::RAWB * r;
+    const int row = s0 + slot, o = C::RAWB * r;
+    return buf + row * C::CROW + (((o >> 4) ^ swz<FMT, D>(row)) << 4) + (o & 15);
   };
   auto scale = [&](int slot) -> __half {
     if (slot >= n_valid) return __ushort_as_half(0);
     const uint8_t* srow = TILE ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW
-                               : buf + slot * C::VSTRIDE + C::CROW + (trow[slot] & (C::RPW - 1)) * C::SROW;
+                               : buf + C::GSC + (s0 + slot) * 16 + (trow[slot] & (C::RPW - 1)) * C::SROW;
     if constexpr (C::kNv)  // E4M3 block scale of this thread's dims times the vector scale
       return __float2half_rn(e4m3_float(srow[(C::E * r) / 16]) *
                              *reinterpret_cast<const float*>(srow + D / 16));
@@ -642,6 +675,149 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const _
 #pragma unroll
   for (int mt = 0; mt < C::MT; ++mt)
     mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], b0, b1);
+}
+// q8_0 / q4_0 V pass.  Codes become fp16 by the magic-number bits (fp16 value = code +
+// offset, exact) and one fp16 subtraction of the offset (exact: a small integer), read
+// with transposing matrix loads so that one register already pairs two positions; the
+// scale d of each (position, block) rides on the weights instead of the codes: B = p d'
+// per block, with d' = d 2^-k, k >= 0 per block for the whole staged buffer, so that p d'
+// (p stored as p 2^14) stays inside fp16; v_mag_finish undoes 2^-k.  The MMA pipe is the
+// scarce unit here (mma.sync), so the offset is removed on the ALU rather than by an extra
+// MMA.  Thread (r, c) ends up with, per m-tile mt and heads 2c, 2c + 1 (accumulator pairs
+// 0, 1 and 2, 3):
+//   q4_0: chunk b = block b, m-tile 2b + s: dims 32b + 4r + 2s (low nibble: 1024 + n,
+//         minus 1032) and 32b + 4r + 2s + 1 (bits 4..7 in place: 64 + n, minus 72);
+//   q8_0: chunk ch = dims 16ch .. 16ch + 15, m-tile ch: dims 16ch + 2r and 16ch + 2r + 1
+//         ((byte ^ 0x80) | fp16 1024 = 1152 + code, minus 1152).
+template <int FMT, int D>
+__device__ __forceinline__ int v_dim(int r, int mt, int i) {
+  using C = Cfg<FMT, D>;
+  if constexpr (C::kQ4) return 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + (i >> 1);
+  else if constexpr (C::kQ8) return 16 * mt + 2 * r + (i >> 1);
+  else return C::E * r + 2 * mt + (i >> 1);
+}
+
+// The scale row of staged slot `slot` (TILE: a tile's scale rows; otherwise the row's
+// place in its gathered 16-byte window).
+template <int FMT, int D, bool TILE>
+__device__ __forceinline__ uint8_t* v_scale_row(uint8_t* buf, const uint8_t* list, int slot) {
+  using C = Cfg<FMT, D>;
+  return TILE ? buf + C::STAGE_CODE + slot * C::SROW
+              : buf + C::GSC + slot * 16 + (list[slot] & (C::RPW - 1)) * C::SROW;
+}
+
+// Per block, k = the smallest exponent >= 0 with d 2^-k < 2 for every staged slot
+// 0 .. n - 1, and those scales multiplied by 2^-k in place (exact).  Warp-wide.
+template <int FMT, int D, bool TILE>
+__device__ __forceinline__ void v_mag_normalize(uint8_t* buf, const uint8_t* list, int n, int lane,
+                                                int (&k)[Cfg<FMT, D>::NBLK]) {
+  using C = Cfg<FMT, D>;
+  constexpr int NW = C::NBLK / 2;  // 32-bit words (two blocks' scales) per scale row
+  uint32_t mx[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mx[w] = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int slot = lane + 32 * h;
+    if (slot < n) {
+      const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, slot));
+#pragma unroll
+      for (int w = 0; w < NW; ++w)  // |d| (scales are >= 0 but may be -0)
+        mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(sr[w] & 0x7FFF7FFFu)));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(__shfl_xor_sync(0xffffffffu, mx[w], o))));
+  uint32_t f[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int e0 = (mx[w] >> 10) & 31, e1 = (mx[w] >> 26) & 31;  // fp16 exponent fields
+    k[2 * w] = min(14, max(0, e0 - 15));
+    k[2 * w + 1] = min(14, max(0, e1 - 15));
+    f[w] = ((uint32_t)(15 - k[2 * w]) << 10) | ((uint32_t)(15 - k[2 * w + 1]) << 26);  // 2^-k
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int slot = lane + 32 * h;
+    if (slot < n) {
+      uint32_t* sr = reinterpret_cast<uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, slot));
+#pragma unroll
+      for (int w = 0; w < NW; ++w) sr[w] = h2_as_u32(__hmul2(u32_as_h2(sr[w]), u32_as_h2(f[w])));
+    }
+  }
+  __syncwarp();
+}
+
+// One group of 16 staged positions (slots s0 .. s0 + 15; slots at or past n_valid,
+// counted from s0, get weight 0).
+template <int FMT, int D, bool TILE>
+__device__ __forceinline__ void v_group_mag(uint8_t* __restrict__ buf, const __half* __restrict__ prow,
+                                            const uint8_t* __restrict__ list, int s0, int n_valid,
+                                            int lane, int r, int c, float (&acc)[Cfg<FMT, D>::MT][4]) {
+  using C = Cfg<FMT, D>;
+  constexpr int NCH = C::CROW / 16;  // 16-byte chunks per row
+  constexpr int NW = C::NBLK / 2;
+  // weights times scales: slots 2c, 2c + 1 (B rows k = 2c, 2c + 1) and 2c + 8, 2c + 9
+  uint32_t ws[4][NW];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int slot = 2 * c + (q & 1) + 8 * (q >> 1);
+    const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, s0 + slot));
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ws[q][w] = slot < n_valid ? sr[w] : 0u;
+  }
+  const uint32_t p01 = lds32(prow + 2 * c), p89 = lds32(prow + 2 * c + 8);
+  uint32_t b0[C::NBLK], b1[C::NBLK];
+#pragma unroll
+  for (int blk = 0; blk < C::NBLK; ++blk) {
+    const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
+    b0[blk] = h2_as_u32(__hmul2(u32_as_h2(p01), u32_as_h2(prmt(ws[0][blk >> 1], ws[1][blk >> 1], sel))));
+    b1[blk] = h2_as_u32(__hmul2(u32_as_h2(p89), u32_as_h2(prmt(ws[2][blk >> 1], ws[3][blk >> 1], sel))));
+  }
+  auto sub = [](uint32_t x, uint32_t neg) { return h2_as_u32(__hadd2(u32_as_h2(x), u32_as_h2(neg))); };
+  constexpr uint32_t kM1032 = 0xE408E408u, kM72 = 0xD480D480u, kM1152 = 0xE480E480u;  // fp16 pairs
+  // codes, two chunks per matrix load: matrix i = (positions s0 + 8 (i & 1) .., chunk
+  // cb + (i >> 1)), so R[j][h] = chunk cb + j, positions 2c, 2c + 1 (+ 8 h)
+  const int mi = lane >> 3;
+  const int row = s0 + 8 * (mi & 1) + (lane & 7);
+  const uint8_t* rp = buf + row * C::CROW;
+  const int sw = swz<FMT, D>(row);
+#pragma unroll
+  for (int cb = 0; cb < NCH; cb += 2) {
+    uint32_t R[2][2];
+    ldsm_x4_trans(rp + (((cb + (mi >> 1)) ^ sw) << 4), R[0][0], R[0][1], R[1][0], R[1][1]);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int ch = cb + j;
+      if constexpr (C::kQ4) {
+        const uint32_t x0 = R[j][0], x1 = R[j][1], y0 = x0 >> 8, y1 = x1 >> 8;
+        mma16816(acc[2 * ch], sub((x0 & 0x000F000Fu) | kMagic, kM1032), sub((x0 & 0x00F000F0u) | kMagic64, kM72),
+                 sub((x1 & 0x000F000Fu) | kMagic, kM1032), sub((x1 & 0x00F000F0u) | kMagic64, kM72), b0[ch], b1[ch]);
+        mma16816(acc[2 * ch + 1], sub((y0 & 0x000F000Fu) | kMagic, kM1032), sub((y0 & 0x00F000F0u) | kMagic64, kM72),
+                 sub((y1 & 0x000F000Fu) | kMagic, kM1032), sub((y1 & 0x00F000F0u) | kMagic64, kM72), b0[ch], b1[ch]);
+      } else {
+        const uint32_t x0 = R[j][0] ^ 0x80808080u, x1 = R[j][1] ^ 0x80808080u;
+        mma16816(acc[ch], sub(prmt(x0, 0x64646464u, 0x4240u), kM1152), sub(prmt(x0, 0x64646464u, 0x4341u), kM1152),
+                 sub(prmt(x1, 0x64646464u, 0x4240u), kM1152), sub(prmt(x1, 0x64646464u, 0x4341u), kM1152),
+                 b0[ch >> 1], b1[ch >> 1]);
+      }
+    }
+  }
+}
+
+// acc *= 2^k, per block (undoes the scale normalization).
+template <int FMT, int D>
+__device__ __forceinline__ void v_mag_finish(float (&acc)[Cfg<FMT, D>::MT][4], const int (&k)[Cfg<FMT, D>::NBLK]) {
+  using C = Cfg<FMT, D>;
+#pragma unroll
+  for (int mt = 0; mt < C::MT; ++mt) {
+    const float f = __int_as_float((127 + k[mt >> 1]) << 23);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[mt][i] *= f;
+  }
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -799,16 +975,7 @@ decode_kernel(const DecodeArgs a) {
                        ssrc + 16 * j * C::SROW + lane * 16);
           cp_async_commit();
         }
-        if (prefetch_v) {
-          const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
-#pragma unroll 4
-          for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(vtile + i * 16, vsrc + i * 16);
-          const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
-#pragma unroll
-          for (int i = lane; i < C::STAGE_SC / 16; i += 32)
-            cp_async16(vtile + C::STAGE_CODE + i * 16, vssrc + i * 16);
-          cp_async_commit();
-        }
+        if (prefetch_v) copy_v_tile<FMT, D>(vtile, vcodes, vscales, (size_t)row0, lane);
       }
     }
     if (k == 0) {
@@ -1000,14 +1167,7 @@ decode_kernel(const DecodeArgs a) {
                           __all_sync(0xffffffffu, (!hl0 || mn0 - mh0 >= thr) && (!hl1 || mn1 - mh1 >= thr));
     if (all_kept && !prefetch_v) {
       __syncwarp();  // every lane is done reading the K tile
-      const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
-#pragma unroll 4
-      for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(kbuf + i * 16, vsrc + i * 16);
-      const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
-#pragma unroll
-      for (int i = lane; i < C::STAGE_SC / 16; i += 32)
-        cp_async16(kbuf + C::STAGE_CODE + i * 16, vssrc + i * 16);
-      cp_async_commit();
+      copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, lane);
     }
     // the weights 2^(s - m) of every valid pair also give the denominator l
     int nkept = 0, nskip = 0;
@@ -1108,44 +1268,59 @@ decode_kernel(const DecodeArgs a) {
       const int ng = (nkept + 15) >> 4;
       if (prefetch_v || nkept == nvalid) {
         // every valid row is kept, so slot s is tile row s; without the prefetched tile,
-        // one contiguous copy of the V tile into the (now free) K buffer
-        const uint8_t* vt = prefetch_v ? vtile : kbuf;
+        // one copy of the V tile into the (now free) K buffer
+        uint8_t* vt = prefetch_v ? vtile : kbuf;
         if (!prefetch_v && !all_kept) {
           __syncwarp();  // every lane is done reading the K tile
-          const uint8_t* vsrc = vcodes + (size_t)row0 * C::CROW;
-#pragma unroll 4
-          for (int i = lane; i < C::STAGE_CODE / 16; i += 32) cp_async16(kbuf + i * 16, vsrc + i * 16);
-          const uint8_t* vssrc = vscales + (size_t)row0 * C::SROW;
-#pragma unroll
-          for (int i = lane; i < C::STAGE_SC / 16; i += 32)
-            cp_async16(kbuf + C::STAGE_CODE + i * 16, vssrc + i * 16);
-          cp_async_commit();
+          copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, lane);
         }
         cp_async_wait<0>();
         __syncwarp();
+        if constexpr (C::kMag) {
+          int kx[C::NBLK];
+          v_mag_normalize<FMT, D, true>(vt, list_w, nkept, lane, kx);
 #pragma unroll 2
-        for (int g = 0; g < ng; ++g)
-          v_group<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
-                                min(16, nkept - 16 * g), r, c, lut, acc);
+          for (int g = 0; g < ng; ++g)
+            v_group_mag<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
+                                      min(16, nkept - 16 * g), lane, r, c, acc);
+          v_mag_finish<FMT, D>(acc, kx);
+        } else {
+#pragma unroll 2
+          for (int g = 0; g < ng; ++g)
+            v_group<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
+                                  min(16, nkept - 16 * g), r, c, lut, acc);
+        }
       } else {
-        // gather the kept rows into the (now free) K buffer: codes + the scale window
-        constexpr int CPR = C::CROW / 16 + 1;
-        for (int i = lane; i < 16 * ng * CPR; i += 32) {
-          const int s = i / CPR, cc = i - s * CPR;
-          if (s < nkept) {
-            const size_t row = (size_t)row0 + list_w[s];
-            const uint8_t* src = cc < CPR - 1 ? vcodes + row * C::CROW + cc * 16
-                                              : vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW;
-            cp_async16(kbuf + (s >> 4) * C::VGROUP + (s & 15) * C::VSTRIDE + cc * 16, src);
+        // gather the kept rows into the (now free) K buffer: slot s gets its codes (chunk
+        // swizzle of row s) and the 16-byte window of the scales plane holding its scales
+        constexpr int CPR = C::CROW / 16;
+        for (int i = lane; i < 16 * ng * (CPR + 1); i += 32) {
+          const int sl = i / (CPR + 1), cc = i - sl * (CPR + 1);
+          if (sl < nkept) {
+            const size_t row = (size_t)row0 + list_w[sl];
+            if (cc < CPR)
+              cp_async16(kbuf + sl * C::CROW + ((cc ^ swz<FMT, D>(sl)) << 4), vcodes + row * C::CROW + cc * 16);
+            else
+              cp_async16(kbuf + C::GSC + sl * 16, vscales + (row & ~(size_t)(C::RPW - 1)) * C::SROW);
           }
         }
         cp_async_commit();
         cp_async_wait<0>();
         __syncwarp();
+        if constexpr (C::kMag) {
+          int kx[C::NBLK];
+          v_mag_normalize<FMT, D, false>(kbuf, list_w, nkept, lane, kx);
 #pragma unroll 2
-        for (int g = 0; g < ng; ++g)
-          v_group<FMT, D, false>(kbuf + g * C::VGROUP, pk_w + r * kPkStride + 16 * g, list_w + 16 * g,
-                                 0, min(16, nkept - 16 * g), r, c, lut, acc);
+          for (int g = 0; g < ng; ++g)
+            v_group_mag<FMT, D, false>(kbuf, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
+                                       min(16, nkept - 16 * g), lane, r, c, acc);
+          v_mag_finish<FMT, D>(acc, kx);
+        } else {
+#pragma unroll 2
+          for (int g = 0; g < ng; ++g)
+            v_group<FMT, D, false>(kbuf, pk_w + r * kPkStride + 16 * g, list_w + 16 * g, 16 * g,
+                                   min(16, nkept - 16 * g), r, c, lut, acc);
+        }
       }
       __syncwarp();  // staged V fully read before the accumulators overwrite the buffer
       float* accw = reinterpret_cast<float*>(kbuf);
@@ -1187,7 +1362,7 @@ decode_kernel(const DecodeArgs a) {
       const int ln = q & 31, e = q >> 5;
       const int mt = e >> 2, i = e & 3;
       const int h = 2 * (ln & 3) + (i & 1);
-      const int dim = C::E * (ln >> 2) + 2 * mt + (i >> 1);
+      const int dim = v_dim<FMT, D>(ln >> 2, mt, i);
       if (h < G) {
         float v = 0.f;
 #pragma unroll

@@ -132,11 +132,22 @@ __device__ __forceinline__ void cp_async_wait() {
 // D += A * B, m16n8k16, f16 inputs, f32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 matrices of 16-bit elements from shared memory, transposed: lane l gives the
+// address of row l % 8 of matrix l / 8; register i of lane (r = l / 4, c = l % 4) holds
+// elements (row 2c, column r) and (row 2c + 1, column r) of matrix i (low half first).
+__device__ __forceinline__ void ldsm_x4_trans(const void* p, uint32_t& d0, uint32_t& d1, uint32_t& d2,
+                                              uint32_t& d3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
+               : "r"(smem_u32(p))
+               : "memory");
 }
 
 // ------------------------------------------------------------------ thread-block clusters

@@ -993,8 +993,19 @@ decode_kernel(const DecodeArgs a) {
           if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
           slen[bb] = max(0, min(n, cap));
         }
+        // Every split adds its share into the output rows of its (sequence, KV head)
+        // (single round only).  Split 0 clears them here, long before any share is
+        // added, and raises the rows' flag with release semantics; whoever adds waits
+        // for the flag with acquire semantics (a wait that is long over by then).
+        if (a.out && a.group_merge && cu == 0 && nb > 0) {
+          float4* orow = reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D);
+          for (int i = lane; i < G * D / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          __syncwarp();
+          if (lane == 0) flag_set_release(a.zflag + (size_t)b * hkv + kvh, epoch_tag(ep_raw));
+        }
       }
     }
+    const bool add_merge = a.out && a.group_merge;
     if (k == 0 && cu * CS * Ls >= nb) {  // a speculative unit past the sequence's end
       cp_async_wait<0>();
       continue;
@@ -1113,15 +1124,11 @@ decode_kernel(const DecodeArgs a) {
         red_l[warp * 8 + 2 * c] = lo0;
         red_l[warp * 8 + 2 * c + 1] = lo1;
       }
-      const bool zero_out = a.out && a.group_merge && cu == 0;
-      if (zero_out)
-        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
-      __syncthreads();  // every warp's l is in shared memory, the output rows are cleared
+      __syncthreads();  // every warp's l is in shared memory
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        if (zero_out) __threadfence();  // the cleared rows are visible before this entry
         xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, cmx[tid], l);
       }
       if (warp < G) {  // M and L of head `warp` over all splits, once every entry is in
@@ -1138,7 +1145,6 @@ decode_kernel(const DecodeArgs a) {
           set_flag(flags, KVQ_FLAG_TIMEOUT);
           misc[0] = misc[1] = 0;
         }
-        __threadfence();  // what the other splits wrote before their entries is visible
       }
       __syncthreads();
     }
@@ -1245,17 +1251,13 @@ decode_kernel(const DecodeArgs a) {
     //      (m, l) and arrives at its (sequence, KV head) barrier now, so that the wait
     //      overlaps its V work; split 0 clears the output rows that the splits add into.
     //      (With the sequence-wide maximum this exchange already happened.)
-    const bool add_merge = a.out && a.group_merge;
     const int nsplit = (nb + Ls - 1) / Ls;
     if (add_merge && !a.global_max) {
-      if (cu == 0)
-        for (int i = tid; i < G * D; i += kThreads) a.out[((size_t)b * Hq + (size_t)kvh * G) * D + i] = 0.f;
-      __syncthreads();  // every warp's l is in shared memory, the output rows are cleared
+      __syncthreads();  // every warp's l is in shared memory
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        if (cu == 0) __threadfence();  // the cleared rows are visible before this entry
         xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mpart[tid], l);
       }
     }
@@ -1329,28 +1331,42 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) accw[(mt * 4 + i) * 32 + lane] = acc[mt][i];
     }
-    if (add_merge && !a.global_max) {
-      // the first warp done with its V pass waits for every split of this (sequence, KV
-      // head) to publish, then computes this split's share of each head, 2^(m_s - M) / L,
-      // while the other warps are still accumulating
+    if (add_merge) {
+      // One warp (the last when it has no tile, so it gets here right after the publish,
+      // otherwise the first warp done with its V pass) waits, while the other warps are
+      // still accumulating, for split 0's flag that the output rows are cleared (acquire:
+      // the shares are added after it) and, without the sequence-wide maximum, for every
+      // split of this (sequence, KV head) to publish, and computes this split's share of
+      // each head, 2^(m_s - M) / L.
       int first = 0;
-      if (lane == 0) first = atomicAdd(&misc[2], 1) == 0;
-      first = __shfl_sync(0xffffffffu, first, 0);
+      if (n_tok <= (kWarps - 1) * kTile) {
+        first = warp == kWarps - 1;
+      } else {
+        if (lane == 0) first = atomicAdd(&misc[2], 1) == 0;
+        first = __shfl_sync(0xffffffffu, first, 0);
+      }
       if (first) {
-        // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
-        // partials in flight together), then combine across the four lanes
-        const int h = lane >> 2, j = lane & 3;
-        float M, L;
-        const bool ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
-                                       j, 4, nsplit, h < G, tag, M, L);
-        if (ok) {
-          xch_combine(M, L, 2);
-          if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
-        } else if (lane == 0) {
-          set_flag(flags, KVQ_FLAG_TIMEOUT);
-          misc[0] = 0;
+        bool ok = true;
+        if (!a.global_max) {
+          // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
+          // partials in flight together), then combine across the four lanes
+          const int h = lane >> 2, j = lane & 3;
+          float M, L;
+          ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
+                              j, 4, nsplit, h < G, tag, M, L);
+          if (ok) {
+            xch_combine(M, L, 2);
+            if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
+          }
         }
-        __threadfence();  // what the other splits wrote before their entries is visible
+        if (lane == 0) {
+          if (ok) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
+          if (!ok) {
+            set_flag(flags, KVQ_FLAG_TIMEOUT);
+            misc[0] = 0;
+          }
+        }
+        __syncwarp();
       }
     }
     cp_async_wait<0>();  // nothing of this split stays in flight

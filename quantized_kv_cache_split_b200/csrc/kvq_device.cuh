@@ -220,6 +220,24 @@ __device__ __forceinline__ uint32_t epoch_tag(unsigned long long read) {
   return (uint32_t)(read >> kEpochShift) + 1u;
 }
 
+// A flag word that holds the tag of the launch that last set it.  set: every write of
+// the calling thread (and of the threads ordered before it by a barrier) made before it
+// is visible to whoever reads the tag with flag_wait.
+__device__ __forceinline__ void flag_set_release(unsigned long long* p, uint32_t tag) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"((unsigned long long)tag) : "memory");
+}
+// Wait (at most kWaitCycles) until the flag holds `tag`, with acquire semantics.
+__device__ __forceinline__ bool flag_wait_acquire(const unsigned long long* p, uint32_t tag) {
+  unsigned long long v;
+  const long long t0 = clock64();
+  for (;;) {
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    if ((uint32_t)v == tag) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+    __nanosleep(32);
+  }
+}
+
 __device__ __forceinline__ unsigned long long tag_word(uint32_t tag, float v) {
   return ((unsigned long long)tag << 32) | __float_as_uint(v);
 }

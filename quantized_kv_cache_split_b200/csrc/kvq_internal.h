@@ -28,6 +28,7 @@ struct DecodeArgs {
   int max_splits;     // ceil(max_seq_len / split_tokens)
   void* workspace;
   int* counters;      // [batch][num_kv_heads] arrival counters of the last-arrival merge
+  unsigned long long* zflag;  // [batch][num_kv_heads] output rows cleared (launch tag)
   unsigned long long* epoch;  // launch counter in the workspace header (exchange tags)
   float* part_o;      // partials, see below
   float* part_m;
@@ -46,8 +47,9 @@ struct DecodeArgs {
 };
 
 // Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch
-// counter that tags the exchange entries); the last-arrival merge counters (int32
-// [batch][num_q_heads] reserved, rounded up to 256 bytes); then, one slot per cluster of
+// counter that tags the exchange entries); the merge flags and counters (u64 flags
+// "output rows cleared" [batch][num_q_heads], then int32 last-arrival counters
+// [batch][num_q_heads], together rounded up to 256 bytes); then, one slot per cluster of
 // splits:
 //   (m, l) exchange [batch][num_q_heads][max_splits] 2 x u64, each word a fp32 value
 //   under a 32-bit launch tag (what the splits of a (sequence, KV head) publish to one
@@ -57,7 +59,7 @@ struct DecodeArgs {
 //   l [batch][num_q_heads][max_splits] fp32
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits);
 __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
-  return ((size_t)batch * num_q_heads * sizeof(int32_t) + 255) / 256 * 256;
+  return ((size_t)batch * num_q_heads * (sizeof(uint64_t) + sizeof(int32_t)) + 255) / 256 * 256;
 }
 
 int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,

@@ -408,33 +408,6 @@ __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int s
   return true;
 }
 
-// Maximum (W = 0, the published m) or sum (W = 1, the published l) of one word of the
-// entries this lane takes (as in xch_reduce), waiting for this launch's tag.
-template <int T, int W>
-__device__ __forceinline__ bool xch_fold(const ulonglong2* e, int first, int step, int n, bool active,
-                                         uint32_t tag, float& acc) {
-  acc = W == 0 ? -INFINITY : 0.f;
-  for (int ub = 0; ub < n; ub += T * step) {
-    float v[T];
-    const long long t0 = clock64();
-    for (;;) {
-      bool all = true;
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        const int u = ub + first + step * t;
-        v[t] = W == 0 ? -INFINITY : 0.f;
-        if (active && u < n) all &= xch_load_word(e + u, W, tag, v[t]);
-      }
-      if (__all_sync(0xffffffffu, all)) break;
-      if (__any_sync(0xffffffffu, clock64() - t0 > kWaitCycles)) return false;
-      __nanosleep(32);
-    }
-#pragma unroll
-    for (int t = 0; t < T; ++t) acc = W == 0 ? fmaxf(acc, v[t]) : acc + v[t];
-  }
-  return true;
-}
-
 // Combine (M, L) across the lanes that differ in bits 1 .. max_off of the lane index.
 __device__ __forceinline__ void xch_combine(float& M, float& L, int max_off) {
   for (int o = 1; o <= max_off; o <<= 1) {
@@ -1128,19 +1101,46 @@ decode_kernel(const DecodeArgs a) {
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;  // head 0 of the group
     const uint32_t tag = (uint32_t)misc[3];
     if (a.global_max) {
-      // every split publishes its maxima; each derives the maximum M of every head over
-      // all splits of this (sequence, KV head) once every split's is in (the denominators,
-      // relative to M, are exchanged after the skip test)
+      // every split publishes its maxima and its denominators relative to them; after one
+      // barrier among the splits of this (sequence, KV head) each derives the final
+      // maximum M and denominator L of every head (split 0 first clears the output rows
+      // that the splits add their shares into)
       const int n = (nb + Ls - 1) / Ls;
-      if (tid < G) xch_store_word(a.xch + slot0 + (size_t)tid * a.max_splits, 0, tag, cmx[tid]);
-      if (warp < G) {  // M of head `warp` over all splits
-        float M;
-        const bool ok = xch_fold<4, 0>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits,
-                                       lane, 32, n, true, tag, M);
-        if (ok) {
+      float lo0 = 0.f, lo1 = 0.f;
+      const float c0 = cmx[2 * c], c1 = cmx[2 * c + 1];
 #pragma unroll
-          for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-          if (lane == 0) cmx[8 + warp] = M;
+      for (int j = 0; j < 4; ++j) {
+        if (16 * j >= nvalid) break;
+        const float4 sv = scw[j * 32];  // invalid rows hold -inf
+        lo0 += ex2(sv.x - c0) + ex2(sv.z - c0);
+        lo1 += ex2(sv.y - c1) + ex2(sv.w - c1);
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lo0 += __shfl_xor_sync(0xffffffffu, lo0, o);
+        lo1 += __shfl_xor_sync(0xffffffffu, lo1, o);
+      }
+      if (r == 0) {
+        red_l[warp * 8 + 2 * c] = lo0;
+        red_l[warp * 8 + 2 * c + 1] = lo1;
+      }
+      __syncthreads();  // every warp's l is in shared memory
+      if (tid < G) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, cmx[tid], l);
+      }
+      if (warp < G) {  // M and L of head `warp` over all splits, once every entry is in
+        float M, L;
+        const bool ok = xch_reduce<4>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + warp) * a.max_splits,
+                                      lane, 32, n, true, tag, M, L);
+        if (ok) {
+          xch_combine(M, L, 16);
+          if (lane == 0) {
+            cmx[8 + warp] = M;
+            cmx[16 + warp] = 1.f / L;  // this split's share: 2^(M - M) / L
+          }
         } else if (lane == 0) {
           set_flag(flags, KVQ_FLAG_TIMEOUT);
           misc[0] = misc[1] = 0;
@@ -1248,18 +1248,17 @@ decode_kernel(const DecodeArgs a) {
     __syncwarp();  // the warp's list and weights are complete
 
     // ---- additive in-kernel merge (every split on its own CTA): the split publishes its
-    //      (m, l) now (with the sequence-wide maximum, m went out before the skip test
-    //      and l, relative to it, goes now), so that the wait overlaps its V work
+    //      (m, l) and arrives at its (sequence, KV head) barrier now, so that the wait
+    //      overlaps its V work; split 0 clears the output rows that the splits add into.
+    //      (With the sequence-wide maximum this exchange already happened.)
     const int nsplit = (nb + Ls - 1) / Ls;
-    if (add_merge) {
+    if (add_merge && !a.global_max) {
       __syncthreads();  // every warp's l is in shared memory
       if (tid < G) {
         float l = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) l += red_l[w * 8 + tid];
-        ulonglong2* e = a.xch + slot0 + (size_t)tid * a.max_splits;
-        if (a.global_max) xch_store_word(e, 1, tag, l);
-        else xch_store(e, tag, mpart[tid], l);
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mpart[tid], l);
       }
     }
 
@@ -1347,25 +1346,17 @@ decode_kernel(const DecodeArgs a) {
         first = __shfl_sync(0xffffffffu, first, 0);
       }
       if (first) {
-        // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
-        // partials in flight together), then combine across the four lanes
-        const int h = lane >> 2, j = lane & 3;
-        const ulonglong2* eh = a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits;
-        bool ok;
+        bool ok = true;
         if (!a.global_max) {
+          // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
+          // partials in flight together), then combine across the four lanes
+          const int h = lane >> 2, j = lane & 3;
           float M, L;
-          ok = xch_reduce<16>(eh, j, 4, nsplit, h < G, tag, M, L);
+          ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
+                              j, 4, nsplit, h < G, tag, M, L);
           if (ok) {
             xch_combine(M, L, 2);
             if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
-          }
-        } else {  // every l is relative to the same maximum: L is their sum
-          float L;
-          ok = xch_fold<16, 1>(eh, j, 4, nsplit, h < G, tag, L);
-          if (ok) {
-            L += __shfl_xor_sync(0xffffffffu, L, 1);
-            L += __shfl_xor_sync(0xffffffffu, L, 2);
-            if (j == 0 && h < G) cmx[16 + h] = 1.f / L;
           }
         }
         if (lane == 0) {

@@ -249,20 +249,6 @@ __device__ __forceinline__ void xch_store(ulonglong2* p, uint32_t tag, float m, 
                : "memory");
 }
 
-// One word of an entry (w = 0: m, w = 1: l) on its own, for exchanges that publish the two
-// at different times.
-__device__ __forceinline__ void xch_store_word(ulonglong2* p, int w, uint32_t tag, float v) {
-  unsigned long long* q = reinterpret_cast<unsigned long long*>(p) + w;
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(q), "l"(tag_word(tag, v)) : "memory");
-}
-__device__ __forceinline__ bool xch_load_word(const ulonglong2* p, int w, uint32_t tag, float& v) {
-  const unsigned long long* q = reinterpret_cast<const unsigned long long*>(p) + w;
-  unsigned long long a;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(a) : "l"(q) : "memory");
-  v = __uint_as_float((uint32_t)a);
-  return (uint32_t)(a >> 32) == tag;
-}
-
 // Read an entry; false while it is not this launch's (tag mismatch in either word).
 __device__ __forceinline__ bool xch_load(const ulonglong2* p, uint32_t tag, float& m, float& l) {
   unsigned long long a, b;

@@ -820,6 +820,53 @@ __device__ __forceinline__ void v_mag_finish(float (&acc)[Cfg<FMT, D>::MT][4], c
   }
 }
 
+// ------------------------------------------------------------------ unit schedule
+// Units after the first round, for batches that fit one warp's ballot: the existing units
+// (cu, b, kvh) (cu * span < len_b) whose place in the static list (cu-major, then b, then
+// kvh) is `first` or later, in that order; CTA c takes the c-th, (c + ncl)-th, ... of them,
+// so every CTA gets the same number of units (the static list, with its holes where
+// sequences are shorter, gives some CTAs many more).  The cursor (lvl, base: the ranks
+// before level lvl) only moves forward.  Warp-uniform; lens = clamped lengths.
+struct UnitCursor {
+  int lvl, base;
+};
+
+__device__ __forceinline__ bool next_dense_unit(int rank, const int* lens, int B, int hkv, int span,
+                                                int levels, int first, int lane, UnitCursor& uc, int& cu,
+                                                int& b, int& kvh) {
+  const int per = B * hkv;
+  const int l0 = first / per, s0 = first % per;  // where the remainder starts
+  while (uc.lvl < levels) {
+    const unsigned m = __ballot_sync(0xffffffffu, lane < B && lens[lane] > uc.lvl * span);
+    unsigned mb = m;   // sequences whose every KV head counts at this level
+    int part = 0, bs = 0, ks = 0;
+    if (uc.lvl == l0) {  // the first level counts from static place s0 on
+      bs = s0 / hkv;
+      ks = s0 % hkv;
+      part = ((m >> bs) & 1u) ? hkv - ks : 0;
+      mb = m & ~((2u << bs) - 1u);
+    }
+    const int n = part + __popc(mb) * hkv;
+    if (rank < uc.base + n) {
+      int j = rank - uc.base;
+      if (j < part) {
+        b = bs;
+        kvh = ks + j;
+      } else {
+        j -= part;
+        b = (int)__fns(mb, 0, j / hkv + 1);
+        kvh = j % hkv;
+      }
+      cu = uc.lvl;
+      return true;
+    }
+    if (m == 0u) return false;  // no sequence reaches this level or any later one
+    uc.base += n;
+    ++uc.lvl;
+  }
+  return false;
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -920,15 +967,25 @@ decode_kernel(const DecodeArgs a) {
   const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;  // this lane's two accumulator heads exist
   const uint32_t below = (1u << (4 * r)) - 1u;
 
+  // after the first round, batches of up to 32 sequences take the existing units evenly
+  const bool dense = B <= 32 && total > ncl;
+  UnitCursor ucur{ncl / (B * hkv), 0};
 #pragma unroll 1
   for (int k = 0;; ++k) {
-    const int it = cid + k * ncl;
-    if (it >= total) break;
     // ---- the cluster's (group of splits, sequence, KV head) and this CTA's split
-    const int kvh = it % hkv;
-    const int bu = it / hkv;
-    const int b = bu % B;
-    const int cu = bu / B;
+    int kvh, b, cu;
+    if (k > 0 && dense) {
+      __syncthreads();  // the lengths in shared memory are visible (the first unit may have had no barrier)
+      if (!next_dense_unit(cid + (k - 1) * ncl, slen, B, hkv, CS * Ls, NCU, ncl, lane, ucur, cu, b, kvh)) break;
+    } else {
+      const int it = cid + k * ncl;
+      if (it >= total) break;
+      kvh = it % hkv;
+      const int bu = it / hkv;
+      b = bu % B;
+      cu = bu / B;
+      if (k > 0) __syncthreads();  // as above
+    }
     const int t0 = (cu * CS + (int)rank) * Ls;
     // The first unit reads its sequence length from global memory while its K copies
     // are already in flight (they cover what exists in memory, up to cap); later
@@ -937,7 +994,6 @@ decode_kernel(const DecodeArgs a) {
     if (k == 0) {
       nb = __ldg(a.seq_lens + b);  // in flight while the copies are issued
     } else {
-      __syncthreads();  // the lengths in shared memory are visible (the first unit may have had no barrier)
       nb = slen[b];
       if (cu * CS * Ls >= nb) continue;  // no such unit (uniform over the cluster)
     }

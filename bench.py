@@ -182,7 +182,11 @@ class Replicas:
         plane_bytes = sum(t.numel() * t.element_size()
                           for t in (first.k_codes, first.k_scales, first.v_codes, first.v_scales))
         self.plane_bytes = plane_bytes
-        self.R = max(2, math.ceil(min_bytes / plane_bytes))
+        # rotate over enough copies to exceed 3x L2, at most 512 (a tiny cache cannot reach
+        # it with any sensible number of copies: it is then timed with its copies in L2,
+        # which the config's "l2" field says)
+        self.R = max(2, min(512, math.ceil(min_bytes / plane_bytes)))
+        self.l2_cold = self.R * plane_bytes >= min_bytes
         self.caches = [first]
         for _ in range(self.R - 1):
             c = K.QuantizedKVCache(wl.fmt, D, wl.num_kv_heads, inp.page_size, inp.num_pages,
@@ -361,8 +365,10 @@ def gpu_arm(args, world, rank, local):
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
                    "cluster_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
-                   "l2": f"inputs rotate over {rep.R} cache copies "
-                         f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)",
+                   "l2": (f"inputs rotate over {rep.R} cache copies "
+                          f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)" if rep.l2_cold else
+                          f"inputs rotate over {rep.R} cache copies "
+                          f"({rep.R * rep.plane_bytes / 2**20:.1f} MiB < L2: timed with the cache in L2)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "step": "one kvq_decode_attn launch with the in-kernel merge (CUDA graph)"},
         "roofline": {"bound": "hbm", "achieved": round(sp["achieved_gbs"], 1),

@@ -400,47 +400,58 @@ def gpu_arm(args, world, rank, local):
 
 def e2e_arm(args, rep, wl, inp, device, world):
     """Same metric through the public API with host buffers: every step copies the new
-    token's q, k, v from pinned host memory, appends k/v to the cache (kvq_quantize),
-    runs the decode (with its in-kernel merge), and reads the output back to pinned host
-    memory."""
+    token's q, k, v (one packed pinned host buffer) to the device, appends k/v to the
+    cache (kvq_quantize_kv), runs the decode (with its in-kernel merge) and reads the
+    output back to pinned host memory.  The step is captured once per cache copy as a
+    CUDA graph of those public-API calls (how a serving loop issues it) and replayed;
+    the eager form (every call from Python each step) is reported beside it."""
     import torch
     B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
-    h_q = torch.from_numpy(inp.q).pin_memory()
-    h_k = torch.from_numpy(inp.k[-B:]).pin_memory()      # the newest position of each sequence
-    h_v = torch.from_numpy(inp.v[-B:]).pin_memory()
+    nq, nkv = B * Hq * D, B * Hkv * D
+    h_in = torch.cat([torch.from_numpy(inp.q).reshape(-1),
+                      torch.from_numpy(inp.k[-B:]).reshape(-1),     # the newest position of each sequence
+                      torch.from_numpy(inp.v[-B:]).reshape(-1)]).pin_memory()
     last = torch.from_numpy(np.array([int(inp.slots[int(o) - 1]) for o in inp.seq_offsets()[1:]],
                                      dtype=np.int32)).to(device)
     h_out = torch.empty((B, Hq, D), dtype=torch.float32).pin_memory()
-    d_q = torch.empty_like(h_q, device=device)
-    d_k = torch.empty((B, Hkv, D), dtype=torch.float16, device=device)
-    d_v = torch.empty_like(d_k)
+    d_in = torch.empty_like(h_in, device=device)
+    d_q = d_in[:nq].view(B, Hq, D)
+    d_k = d_in[nq:nq + nkv].view(B, Hkv, D)
+    d_v = d_in[nq + nkv:].view(B, Hkv, D)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
 
     def step(i):
         c = rep.caches[i % rep.R]
-        d_q.copy_(h_q, non_blocking=True)
-        d_k.copy_(h_k, non_blocking=True)
-        d_v.copy_(h_v, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
         c.write(d_k, d_v, last)
         c.attention(d_q, rep.seq, rep.max_seq, rep.pt, inp.max_pages, tau=args.tau,
                     sm_scale=rep.sm, split_tokens=rep.L, out=out)
         h_out.copy_(out, non_blocking=True)
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    barrier(world)
-    t0 = time.perf_counter()
-    for i in range(args.steps):
-        step(args.warmup + i)
-    torch.cuda.synchronize()
-    el = reduce_max(time.perf_counter() - t0, world, device)
-    bi = h_q.numel() * 2 + h_k.numel() * 2 + h_v.numel() * 2
+    def timed(run):
+        for i in range(args.warmup):
+            run(i)
+        torch.cuda.synchronize()
+        barrier(world)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            run(args.warmup + i)
+        torch.cuda.synchronize()
+        return reduce_max(time.perf_counter() - t0, world, device)
+
+    el_eager = timed(step)
+    R = min(rep.R, args.steps)  # one graph per cache copy the timed steps use
+    graphs = [capture(step, 1, i) for i in range(R)]
+    el = timed(lambda i: graphs[i % R].replay())
+    bi = h_in.numel() * 2
     bo = h_out.numel() * 4
-    return {"value": round(el * 1e6 / args.steps / (B * world), 3), "unit": UNIT,
+    per = lambda e: round(e * 1e6 / args.steps / (B * world), 3)  # noqa: E731
+    return {"value": per(el), "unit": UNIT,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
-            "how": "eager public API per step: H2D(q,k,v) + QuantizedKVCache.write + .attention + D2H(out)",
-            "gpu_launches_per_step": 3}
+            "how": "public API per step: H2D(q, k, v) + QuantizedKVCache.write + .attention + "
+                   "D2H(out), captured as one CUDA graph per cache copy and replayed",
+            "eager_value": per(el_eager),
+            "gpu_launches_per_step": 2}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)

@@ -128,6 +128,16 @@ int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
                  const int32_t* slots, void* codes, void* scales, void* stream);
 
 /*
+ * kvq_quantize_kv -- kvq_quantize of the K vectors k into (k_codes, k_scales) and of the
+ * V vectors v into (v_codes, v_scales), same slots, in one launch (the append of a
+ * decode step).  Arguments, layout, results and errors are those of two kvq_quantize
+ * calls.
+ */
+int kvq_quantize_kv(const kvq_cache_desc* desc, const void* k, const void* v, int32_t n_tokens,
+                    const int32_t* slots, void* k_codes, void* k_scales, void* v_codes,
+                    void* v_scales, void* stream);
+
+/*
  * kvq_resolve_split -- the split length L (positions per split-KV work unit) that
  * kvq_decode_attn and kvq_combine use for a request (same split_tokens and
  * options).  split_tokens > 0 is capped at KVQ_MAX_SPLIT_TOKENS and rounded up to a

@@ -74,6 +74,7 @@ def _load():
         "kvq_code_row_bytes": (SZ, [I32, I32]),
         "kvq_scale_row_count": (SZ, [I32, I32]),
         "kvq_quantize": (ctypes.c_int, [D, P, I32, P, P, P, P]),
+        "kvq_quantize_kv": (ctypes.c_int, [D, P, P, I32, P, P, P, P, P, P]),
         "kvq_resolve_split": (I32, [D, I32, I32, I32, I32, U32]),
         "kvq_resolve_cluster": (I32, [D, I32, I32, I32, I32, U32]),
         "kvq_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
@@ -153,6 +154,16 @@ def kvq_quantize(desc: KvqCacheDesc, x, n_tokens: int, slots, codes, scales, str
                            _ptr(scales), _stream(stream))
     if check:
         _check("kvq_quantize", st)
+    return st
+
+
+def kvq_quantize_kv(desc: KvqCacheDesc, k, v, n_tokens: int, slots, k_codes, k_scales, v_codes,
+                    v_scales, stream=None, check: bool = True) -> int:
+    st = _lib.kvq_quantize_kv(ctypes.byref(desc), _ptr(k), _ptr(v), int(n_tokens), _ptr(slots),
+                              _ptr(k_codes), _ptr(k_scales), _ptr(v_codes), _ptr(v_scales),
+                              _stream(stream))
+    if check:
+        _check("kvq_quantize_kv", st)
     return st
 
 

@@ -60,8 +60,8 @@ class QuantizedKVCache:
               stream=None):
         """Quantize fp16 K/V [n_tokens, num_kv_heads, head_dim] into physical ``slots``."""
         n = k.shape[0]
-        kb.kvq_quantize(self.desc, k, n, slots, self.k_codes, self.k_scales, stream)
-        kb.kvq_quantize(self.desc, v, n, slots, self.v_codes, self.v_scales, stream)
+        kb.kvq_quantize_kv(self.desc, k, v, n, slots, self.k_codes, self.k_scales, self.v_codes,
+                           self.v_scales, stream)
 
     # ---------------------------------------------------------------- decode
     def workspace(self, batch: int, num_q_heads: int, max_seq_len: int, split_tokens: int,

@@ -140,7 +140,24 @@ int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
     return KVQ_ERR_INVALID_ARG;
   if (!slots && (int64_t)n_tokens > (int64_t)desc->num_pages * desc->page_size)
     return KVQ_ERR_INVALID_ARG;
-  return launch_quantize(*desc, x, n_tokens, slots, codes, scales,
+  return launch_quantize(*desc, x, nullptr, n_tokens, slots, codes, scales, nullptr, nullptr,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int kvq_quantize_kv(const kvq_cache_desc* desc, const void* k, const void* v, int32_t n_tokens,
+                    const int32_t* slots, void* k_codes, void* k_scales, void* v_codes,
+                    void* v_scales, void* stream) {
+  int st = check_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (n_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (n_tokens == 0) return KVQ_OK;
+  if (!k || !v || !k_codes || !k_scales || !v_codes || !v_scales) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k_codes) || !aligned16(k_scales) || !aligned16(v_codes) || !aligned16(v_scales) ||
+      (reinterpret_cast<uintptr_t>(k) & 1u) || (reinterpret_cast<uintptr_t>(v) & 1u))
+    return KVQ_ERR_INVALID_ARG;
+  if (!slots && (int64_t)n_tokens > (int64_t)desc->num_pages * desc->page_size)
+    return KVQ_ERR_INVALID_ARG;
+  return launch_quantize(*desc, k, v, n_tokens, slots, k_codes, k_scales, v_codes, v_scales,
                          static_cast<cudaStream_t>(stream));
 }
 

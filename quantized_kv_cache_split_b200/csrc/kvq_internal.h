@@ -62,8 +62,11 @@ __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
   return ((size_t)batch * num_q_heads * (sizeof(uint64_t) + sizeof(int32_t)) + 255) / 256 * 256;
 }
 
-int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,
-                    void* codes, void* scales, cudaStream_t stream);
+// x2 == nullptr: one plane pair; otherwise the second pair (x2, codes2, scales2) in the
+// same launch.
+int launch_quantize(const kvq_cache_desc& desc, const void* x, const void* x2, int n_tok,
+                    const int32_t* slots, void* codes, void* scales, void* codes2, void* scales2,
+                    cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Clusters of `cluster` CTAs of the decode kernel for (fmt, head_dim) that fit on the
 // current device at once (0 if none); cached per device.

@@ -29,8 +29,14 @@ __device__ __forceinline__ int64_t slot_row(int64_t slot, int page_size, int hkv
 // q8_0: d = amax/127, q = round-half-away(x/d) clamped to [-127, 127].
 template <int D>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
-quant_q8_0_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_t* __restrict__ slots,
-                  int page_size, int8_t* __restrict__ codes, __half* __restrict__ scales) {
+quant_q8_0_kernel(const __half* __restrict__ x, const __half* __restrict__ x2, int n_tok, int hkv,
+                  const int32_t* __restrict__ slots, int page_size, int8_t* __restrict__ codes,
+                  __half* __restrict__ scales, int8_t* __restrict__ codes2, __half* __restrict__ scales2) {
+  if (blockIdx.y) {  // the second plane pair (V of a K + V write)
+    x = x2;
+    codes = codes2;
+    scales = scales2;
+  }
   constexpr int NB = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t vec = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -61,8 +67,14 @@ quant_q8_0_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_
 // q = min(15, floor(x/d + 8.5)); q = 8 when d == 0.
 template <int D>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
-quant_q4_0_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_t* __restrict__ slots,
-                  int page_size, uint8_t* __restrict__ codes, __half* __restrict__ scales) {
+quant_q4_0_kernel(const __half* __restrict__ x, const __half* __restrict__ x2, int n_tok, int hkv,
+                  const int32_t* __restrict__ slots, int page_size, uint8_t* __restrict__ codes,
+                  __half* __restrict__ scales, uint8_t* __restrict__ codes2, __half* __restrict__ scales2) {
+  if (blockIdx.y) {  // the second plane pair (V of a K + V write)
+    x = x2;
+    codes = codes2;
+    scales = scales2;
+  }
   constexpr int NB = D / 32;
   const int lane = threadIdx.x & 31;
   const int64_t vec = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
@@ -104,10 +116,15 @@ quant_q4_0_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_
 // t_k = (c_k + c_{k+1}) * 0.5 from the fp16 codebook.
 template <int D>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
-quant_lut4_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_t* __restrict__ slots,
-                  int page_size, const uint16_t* __restrict__ codebook,
+quant_lut4_kernel(const __half* __restrict__ x, const __half* __restrict__ x2, int n_tok, int hkv,
+                  const int32_t* __restrict__ slots, int page_size, const uint16_t* __restrict__ codebook,
                   const int8_t* __restrict__ signs, uint8_t* __restrict__ codes,
-                  __half* __restrict__ norms) {
+                  __half* __restrict__ norms, uint8_t* __restrict__ codes2, __half* __restrict__ norms2) {
+  if (blockIdx.y) {  // the second plane pair (V of a K + V write)
+    x = x2;
+    codes = codes2;
+    norms = norms2;
+  }
   constexpr int K = D / 32;  // elements per lane
   __shared__ float thr[15];
   if (threadIdx.x < 15) {
@@ -234,8 +251,14 @@ __device__ __forceinline__ float half_warp_max(float v) {
 // half-warp.  Scale row: the E4M3 bytes, then g (fp32), then zero padding.
 template <int D>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
-quant_nvfp4_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32_t* __restrict__ slots,
-                   int page_size, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+quant_nvfp4_kernel(const __half* __restrict__ x, const __half* __restrict__ x2, int n_tok, int hkv,
+                   const int32_t* __restrict__ slots, int page_size, uint8_t* __restrict__ codes,
+                   uint8_t* __restrict__ scales, uint8_t* __restrict__ codes2, uint8_t* __restrict__ scales2) {
+  if (blockIdx.y) {  // the second plane pair (V of a K + V write)
+    x = x2;
+    codes = codes2;
+    scales = scales2;
+  }
   constexpr int NM = D / 32;
   constexpr int SROWB = (D / 16 + 4 + 7) / 8 * 8;  // scale row bytes
   const int lane = threadIdx.x & 31;
@@ -274,29 +297,38 @@ quant_nvfp4_kernel(const __half* __restrict__ x, int n_tok, int hkv, const int32
 
 }  // namespace
 
-int launch_quantize(const kvq_cache_desc& desc, const void* x, int n_tok, const int32_t* slots,
-                    void* codes, void* scales, cudaStream_t stream) {
+int launch_quantize(const kvq_cache_desc& desc, const void* x, const void* x2, int n_tok,
+                    const int32_t* slots, void* codes, void* scales, void* codes2, void* scales2,
+                    cudaStream_t stream) {
   const int64_t vecs = (int64_t)n_tok * desc.num_kv_heads;
   const int64_t blocks = (vecs + kWarpsPerBlock - 1) / kWarpsPerBlock;
   if (blocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)blocks), block(32 * kWarpsPerBlock);
+  // y = 0: the first plane pair; y = 1: the second (K and V in one launch)
+  const dim3 grid((unsigned)blocks, x2 ? 2u : 1u), block(32 * kWarpsPerBlock);
   const __half* xh = static_cast<const __half*>(x);
+  const __half* xh2 = static_cast<const __half*>(x2);
   const int hkv = desc.num_kv_heads, ps = desc.page_size;
-#define KVQ_QUANT_CASE(FMT, DIM, KERNEL, ...)                                     \
-  if (desc.fmt == FMT && desc.head_dim == DIM) {                                  \
-    KERNEL<DIM><<<grid, block, 0, stream>>>(xh, n_tok, hkv, slots, ps, __VA_ARGS__); \
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;             \
+#define KVQ_QUANT_CASE(FMT, DIM, KERNEL, ...)                                            \
+  if (desc.fmt == FMT && desc.head_dim == DIM) {                                         \
+    KERNEL<DIM><<<grid, block, 0, stream>>>(xh, xh2, n_tok, hkv, slots, ps, __VA_ARGS__); \
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;                    \
   }
-  KVQ_QUANT_CASE(KVQ_FMT_Q8_0, 64, quant_q8_0_kernel, (int8_t*)codes, (__half*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_Q8_0, 128, quant_q8_0_kernel, (int8_t*)codes, (__half*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_Q4_0, 64, quant_q4_0_kernel, (uint8_t*)codes, (__half*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_Q4_0, 128, quant_q4_0_kernel, (uint8_t*)codes, (__half*)scales)
+  KVQ_QUANT_CASE(KVQ_FMT_Q8_0, 64, quant_q8_0_kernel, (int8_t*)codes, (__half*)scales, (int8_t*)codes2,
+                 (__half*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_Q8_0, 128, quant_q8_0_kernel, (int8_t*)codes, (__half*)scales, (int8_t*)codes2,
+                 (__half*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_Q4_0, 64, quant_q4_0_kernel, (uint8_t*)codes, (__half*)scales, (uint8_t*)codes2,
+                 (__half*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_Q4_0, 128, quant_q4_0_kernel, (uint8_t*)codes, (__half*)scales, (uint8_t*)codes2,
+                 (__half*)scales2)
   KVQ_QUANT_CASE(KVQ_FMT_LUT4, 64, quant_lut4_kernel, desc.codebook, desc.signs, (uint8_t*)codes,
-                 (__half*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_LUT4, 128, quant_lut4_kernel, desc.codebook, desc.signs,
-                 (uint8_t*)codes, (__half*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 64, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales)
-  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 128, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales)
+                 (__half*)scales, (uint8_t*)codes2, (__half*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_LUT4, 128, quant_lut4_kernel, desc.codebook, desc.signs, (uint8_t*)codes,
+                 (__half*)scales, (uint8_t*)codes2, (__half*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 64, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales, (uint8_t*)codes2,
+                 (uint8_t*)scales2)
+  KVQ_QUANT_CASE(KVQ_FMT_NVFP4, 128, quant_nvfp4_kernel, (uint8_t*)codes, (uint8_t*)scales, (uint8_t*)codes2,
+                 (uint8_t*)scales2)
 #undef KVQ_QUANT_CASE
   return KVQ_ERR_UNSUPPORTED;
 }

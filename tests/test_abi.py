@@ -105,6 +105,21 @@ def test_quantize_rejects_bad_pointers():
     assert K.kvq_quantize(d, FAKE, 8 * 64 + 1, None, FAKE, FAKE, stream=0, check=False) == K.KVQ_ERR_INVALID_ARG
 
 
+def test_quantize_kv_rejects_bad_pointers():
+    # the K + V append: the checks of two kvq_quantize calls, before any launch
+    d = _desc()
+    q = lambda *a: K.kvq_quantize_kv(d, *a, stream=0, check=False)  # noqa: E731
+    assert q(FAKE, None, 4, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert q(None, FAKE, 4, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, 4, None, FAKE, FAKE, FAKE + 8, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE + 1, 4, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, -1, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert q(FAKE, FAKE, 0, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_OK
+    assert q(FAKE, FAKE, 8 * 64 + 1, None, FAKE, FAKE, FAKE, FAKE) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_quantize_kv(K.KvqCacheDesc(7, 128, 4, 64, 8, None, None),
+                             FAKE, FAKE, 4, None, FAKE, FAKE, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_UNSUPPORTED
+
+
 def _decode(d, **kw):
     a = dict(q=FAKE, batch=1, num_q_heads=32, k_codes=FAKE, k_scales=FAKE, v_codes=FAKE,
              v_scales=FAKE, page_table=None, max_pages=1, seq_lens=FAKE, max_seq_len=256,

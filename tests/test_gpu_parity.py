@@ -57,7 +57,9 @@ def test_quantize_bit_exact(fmt, D):
         assert np.array_equal(got_c, want_c), f"codes differ at {np.argwhere(got_c != want_c)[:5]}"
         want_s = s if fmt == "nvfp4" else s.astype(np.float16).view(np.uint16)  # nvfp4: raw words
         assert np.array_equal(got_s.view(np.uint16), want_s), "scales"
+    # the writer quantizes K and V in one launch (the second plane pair): same bytes
     assert np.array_equal(cache.v_codes.cpu().numpy(), codes)
+    assert np.array_equal(cache.v_scales.cpu().numpy().view(np.uint16), scales.view(np.uint16))
 
 
 # ------------------------------------------------------------------ attention parity
@@ -187,6 +189,21 @@ def test_exchange_across_request_shapes_on_one_workspace():
     assert cache.device_flags() == 0
     header = cache._ws[:16].cpu().numpy()
     assert int(header[8:16].view(np.uint64)[0]) == launches * (1 << 16)
+
+
+@pytest.mark.parametrize("fmt,tau", [("q4_0", 1e-6), ("q8_0", 0.0)])
+def test_decode_parity_many_sequences(fmt, tau):
+    # 40 sequences (more than one warp ballot): after the first round the units follow
+    # the static list; 64-position splits make several rounds on any device
+    rng = np.random.Generator(np.random.PCG64(4040))
+    lens = [int(x) for x in rng.integers(0, 600, size=40)]
+    lens[3], lens[17] = 0, 1
+    wl = W.shrink(W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt), lens, n_planted=4)
+    inp = W.generate(wl)
+    g = run_library(inp, tau, 64)
+    o = run_oracle(inp, tau, g["split"])
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
 
 
 RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]

@@ -240,7 +240,7 @@ int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch
  * kvq_decode_attn_noalloc -- kvq_decode_attn with an output pointer, for callers that
  * cannot allocate device memory while decoding (a serving runtime that plans every
  * buffer up front, a process confined to a fixed memory pool, or code running where
- * cudaMalloc is not allowed).  The paper has no counterpart: this is packaging.
+ * cudaMalloc is not allowed).  The method's pages have no counterpart: this is packaging.
  *   The per-split partials live in a library-owned static device array of
  *   KVQ_NOALLOC_SCRATCH_BYTES (8 MiB); every GPU that loads the library keeps it until
  *   the process exits.  Nothing is allocated or freed by the call.

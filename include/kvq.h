@@ -90,7 +90,7 @@ extern "C" {
 /* Device flag bits (kvq_read_device_flags). */
 #define KVQ_FLAG_BAD_PAGE     1u  /* a page-table entry outside [0, num_pages) */
 #define KVQ_FLAG_BAD_SEQLEN   2u  /* seq_len < 0, > max_seq_len or > max_pages*page_size */
-#define KVQ_FLAG_TIMEOUT      4u  /* a bounded wait on an asynchronous copy gave up */
+#define KVQ_FLAG_TIMEOUT      4u  /* a bounded wait (cross-CTA exchange, flag) gave up */
 
 /* Limits of this build. */
 #define KVQ_MAX_GROUP        8     /* query heads per KV head (num_q_heads / num_kv_heads) */
@@ -170,6 +170,16 @@ size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
  * call to kvq_decode_attn completed is ready for the next call without another init,
  * whatever the next call's shape; after KVQ_FLAG_TIMEOUT, init it again. */
 int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kvq_selftest_wait -- diagnostic: runs the decode kernel's bounded waits (the (m, l)
+ * exchange poll and the cleared-rows flag wait) against entries in the workspace header
+ * that never become ready, each giving up after max_cycles SM cycles (> 0) and setting
+ * KVQ_FLAG_TIMEOUT in the workspace's flag word, as a decode whose splits could not all
+ * meet would.  It reads the header's spare bytes only; the GPU context stays usable.
+ *   workspace  device, >= 256 bytes (the header), 16-byte aligned
+ */
+int kvq_selftest_wait(void* workspace, size_t workspace_bytes, long long max_cycles, void* stream);
 
 /* Synchronize `stream` and read the device flag word (KVQ_FLAG_* bits) into *flags (host). */
 int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);

@@ -80,6 +80,7 @@ def _load():
         "kvq_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
         "kvq_workspace_init": (ctypes.c_int, [P, SZ, P]),
         "kvq_read_device_flags": (ctypes.c_int, [P, ctypes.POINTER(ctypes.c_uint32), P]),
+        "kvq_selftest_wait": (ctypes.c_int, [P, ctypes.c_size_t, ctypes.c_longlong, P]),
         "kvq_decode_attn": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32, F32,
                                            I32, U32, P, SZ, P, P, P]),
         "kvq_combine": (ctypes.c_int, [D, P, I32, I32, I32, I32, U32, P, P, P]),
@@ -199,6 +200,14 @@ def kvq_read_device_flags(workspace, stream=None) -> int:
     _check("kvq_read_device_flags",
            _lib.kvq_read_device_flags(_ptr(workspace), ctypes.byref(out), _stream(stream)))
     return out.value
+
+
+def kvq_selftest_wait(workspace, workspace_bytes: int, max_cycles: int, stream=None,
+                      check: bool = True) -> int:
+    st = _lib.kvq_selftest_wait(_ptr(workspace), int(workspace_bytes), int(max_cycles), _stream(stream))
+    if check:
+        _check("kvq_selftest_wait", st)
+    return st
 
 
 def kvq_decode_attn(desc: KvqCacheDesc, q, batch: int, num_q_heads: int, k_codes, k_scales,

@@ -193,6 +193,12 @@ int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
              : KVQ_ERR_CUDA;
 }
 
+int kvq_selftest_wait(void* workspace, size_t workspace_bytes, long long max_cycles, void* stream) {
+  if (!workspace || max_cycles <= 0 || !aligned16(workspace)) return KVQ_ERR_INVALID_ARG;
+  if (workspace_bytes < kWorkspaceHeader) return KVQ_ERR_WORKSPACE;
+  return launch_selftest_wait(workspace, max_cycles, static_cast<cudaStream_t>(stream));
+}
+
 int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream) {
   if (!workspace || !flags) return KVQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

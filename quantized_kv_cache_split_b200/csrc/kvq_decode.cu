@@ -373,10 +373,11 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
 // every pass of T * step entries, u < n, none when !active; M is their maximum and L
 // their denominators rescaled to it.  Each pass waits until all its entries carry this
 // launch's tag (its loads all in flight together); false if that took longer than
-// kWaitCycles.  Warp-uniform: every lane of the warp calls it with the same n.
+// `limit` SM cycles.  Warp-uniform: every lane of the warp calls it with the same n.
 template <int T>
 __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int step, int n,
-                                           bool active, uint32_t tag, float& M, float& L) {
+                                           bool active, uint32_t tag, float& M, float& L,
+                                           long long limit = kWaitCycles) {
   M = -INFINITY;
   L = 0.f;
   for (int ub = 0; ub < n; ub += T * step) {
@@ -392,7 +393,7 @@ __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int s
         if (active && u < n) all &= xch_load(e + u, tag, mv[t], lv[t]);
       }
       if (__all_sync(0xffffffffu, all)) break;
-      if (__any_sync(0xffffffffu, clock64() - t0 > kWaitCycles)) return false;
+      if (__any_sync(0xffffffffu, clock64() - t0 > limit)) return false;
       __nanosleep(32);
     }
     float bm = M;
@@ -1805,6 +1806,29 @@ int launch_decode_t(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+namespace {
+// The exchange's bounded waits against entries that never become this launch's: the
+// (m, l) poll and the cleared-rows flag wait each give up after `limit` cycles and set
+// KVQ_FLAG_TIMEOUT, as a decode that lost a split would.  The entries are four exchange
+// entries and one flag word in the workspace header's spare bytes (64..143), read only.
+__global__ void selftest_wait_kernel(uint8_t* ws, long long limit) {
+  uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
+  const ulonglong2* e = reinterpret_cast<const ulonglong2*>(ws + 64);
+  const unsigned long long* f = reinterpret_cast<const unsigned long long*>(ws + 128);
+  const uint32_t never = 0xffffffffu;  // no launch reaches this tag
+  float M, L;
+  const bool ok1 = xch_reduce<4>(e, threadIdx.x & 31, 32, 4, true, never, M, L, limit);
+  bool ok2 = true;
+  if ((threadIdx.x & 31) == 0) ok2 = flag_wait_acquire(f, never, limit);
+  if ((threadIdx.x & 31) == 0 && (!ok1 || !ok2)) set_flag(flags, KVQ_FLAG_TIMEOUT);
+}
+}  // namespace
+
+int launch_selftest_wait(void* workspace, long long max_cycles, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint8_t*>(workspace), max_cycles);
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
 
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const int f = a.desc.fmt, d = a.desc.head_dim;

@@ -145,14 +145,15 @@ __device__ __forceinline__ uint32_t epoch_tag(unsigned long long read) {
 __device__ __forceinline__ void flag_set_release(unsigned long long* p, uint32_t tag) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"((unsigned long long)tag) : "memory");
 }
-// Wait (at most kWaitCycles) until the flag holds `tag`, with acquire semantics.
-__device__ __forceinline__ bool flag_wait_acquire(const unsigned long long* p, uint32_t tag) {
+// Wait (at most `limit` SM cycles) until the flag holds `tag`, with acquire semantics.
+__device__ __forceinline__ bool flag_wait_acquire(const unsigned long long* p, uint32_t tag,
+                                                  long long limit = kWaitCycles) {
   unsigned long long v;
   const long long t0 = clock64();
   for (;;) {
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     if ((uint32_t)v == tag) return true;
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
     __nanosleep(32);
   }
 }

@@ -68,6 +68,7 @@ int launch_quantize(const kvq_cache_desc& desc, const void* x, const void* x2, i
                     const int32_t* slots, void* codes, void* scales, void* codes2, void* scales2,
                     cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+int launch_selftest_wait(void* workspace, long long max_cycles, cudaStream_t stream);
 // Clusters of `cluster` CTAs of the decode kernel for (fmt, head_dim) that fit on the
 // current device at once (0 if none); cached per device.
 int decode_cluster_capacity(int fmt, int head_dim, int cluster);

@@ -120,6 +120,13 @@ def test_quantize_kv_rejects_bad_pointers():
                              FAKE, FAKE, 4, None, FAKE, FAKE, FAKE, FAKE, 0, check=False) == K.KVQ_ERR_UNSUPPORTED
 
 
+def test_selftest_wait_rejects_bad_arguments():
+    assert K.kvq_selftest_wait(None, 256, 1000, 0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_selftest_wait(FAKE, 256, 0, 0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_selftest_wait(FAKE + 8, 256, 1000, 0, check=False) == K.KVQ_ERR_INVALID_ARG
+    assert K.kvq_selftest_wait(FAKE, 255, 1000, 0, check=False) == K.KVQ_ERR_WORKSPACE
+
+
 def _decode(d, **kw):
     a = dict(q=FAKE, batch=1, num_q_heads=32, k_codes=FAKE, k_scales=FAKE, v_codes=FAKE,
              v_scales=FAKE, page_table=None, max_pages=1, seq_lens=FAKE, max_seq_len=256,

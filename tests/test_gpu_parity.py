@@ -206,6 +206,22 @@ def test_decode_parity_many_sequences(fmt, tau):
     assert g["flags"] == 0
 
 
+def test_bounded_waits_give_up_and_leave_the_context_usable():
+    # The exchange poll and the flag wait of the decode kernel, run against entries that
+    # never become ready with a 2M-cycle bound: KVQ_FLAG_TIMEOUT, no hang, and the next
+    # decode on a fresh workspace is correct.
+    import quantized_kv_cache_split_b200 as K
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    K.kvq_workspace_init(ws, ws.numel())
+    K.kvq_selftest_wait(ws, ws.numel(), 2_000_000)
+    assert K.kvq_read_device_flags(ws) & K.KVQ_FLAG_TIMEOUT
+    wl = W.WORKLOADS["tiny_q8_d64"]
+    inp = W.generate(wl)
+    g = run_library(inp, 1e-6, 64)
+    check_parity(inp, g, run_oracle(inp, 1e-6, g["split"]), 1e-6)
+    assert g["flags"] == 0
+
+
 RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 
 

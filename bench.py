@@ -214,13 +214,14 @@ class Replicas:
         self.out = torch.empty((self.B, self.Hq, D), dtype=torch.float32, device=device)
         self.sm = float(np.float32(1.0 / math.sqrt(D)))
 
-    def decode(self, i, tau, stats=None, scope="split", fused=True):
+    def decode(self, i, tau, stats=None, scope="split", fused=True, v_opt=0):
         """One decode step on cache copy i % R; ``fused``: the merge runs in the same
         kernel and writes ``self.out``; ``scope``: the running maximum of the skip test
-        ("split", "cluster" or "sequence")."""
+        ("split", "cluster" or "sequence"); ``v_opt``: a V fetch option bit (0: the
+        library's choice)."""
         import quantized_kv_cache_split_b200 as K
         c = self.caches[i % self.R]
-        opts = {"split": 0, "cluster": K.KVQ_OPT_SHARED_MAX, "sequence": K.KVQ_OPT_GLOBAL_MAX}[scope]
+        opts = {"split": 0, "cluster": K.KVQ_OPT_SHARED_MAX, "sequence": K.KVQ_OPT_GLOBAL_MAX}[scope] | v_opt
         K.kvq_decode_attn(c.desc, self.q, self.B, self.Hq, c.k_codes, c.k_scales, c.v_codes,
                           c.v_scales, self.pt, self.inp.max_pages, self.seq, self.max_seq, self.sm,
                           tau, self.L_sh if scope == "cluster" else self.L, self.ws, self.ws_bytes,
@@ -317,31 +318,38 @@ def gpu_arm(args, world, rank, local):
     def n_partials(L, CS):
         return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
 
-    def counters(tau, scope):
+    def counters(tau, scope, v_opt):
         st = torch.zeros(4, dtype=torch.int64, device=device)
-        rep.decode(0, tau, st, scope=scope)
+        rep.decode(0, tau, st, scope=scope, v_opt=v_opt)
         torch.cuda.synchronize()
         return [int(x) for x in st.cpu()]
 
     res = {}
     hbm_peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
-    variants = (("sparse", args.tau, "split"), ("dense", 0.0, "split"),
-                ("sparse_cluster_max", args.tau, "cluster"), ("sparse_sequence_max", args.tau, "sequence"))
-    for tag, tau, scope in variants:
+    # the headline leaves the V fetch to the library (V with K in a single-round launch,
+    # kept rows only otherwise); the two policies are also timed on their own
+    variants = (("sparse", args.tau, "split", 0), ("dense", 0.0, "split", 0),
+                ("sparse_v_kept_only", args.tau, "split", K.KVQ_OPT_V_KEPT_ONLY),
+                ("sparse_v_with_k", args.tau, "split", K.KVQ_OPT_V_WITH_K),
+                ("sparse_cluster_max", args.tau, "cluster", 0), ("sparse_sequence_max", args.tau, "sequence", 0),
+                ("sparse_sequence_max_v_kept_only", args.tau, "sequence", K.KVQ_OPT_V_KEPT_ONLY))
+    for tag, tau, scope, v_opt in variants:
         try:
-            st = counters(tau, scope)
+            st = counters(tau, scope, v_opt)
         except K.KvqError as e:  # the sequence-wide maximum needs every split on its own CTA
             res[tag] = {"max_scope": scope, "unavailable": str(e)}
             continue
-        step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope), rep.R)
+        step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope, v_opt=v_opt), rep.R)
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)
         abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if scope == "cluster"
                                    else n_partials(rep.L, 1), with_o=scope == "cluster")
         us_launch = ms_step * 1e3 / args.steps
         achieved = abytes / (us_launch * 1e-6) / 1e9
-        res[tag] = dict(tau=tau, max_scope=scope, ms_per_step=ms_step / args.steps,
+        res[tag] = dict(tau=tau, max_scope=scope, v_fetch={0: "auto", K.KVQ_OPT_V_KEPT_ONLY: "kept_only",
+                                                           K.KVQ_OPT_V_WITH_K: "with_k"}[v_opt],
+                        ms_per_step=ms_step / args.steps,
                         us_per_token=ms_step * 1e3 / args.steps / (wl.batch * world),
                         us_per_launch=us_launch, algorithmic_bytes=abytes,
                         achieved_gbs=achieved, frac=achieved / hbm_peak,
@@ -364,6 +372,7 @@ def gpu_arm(args, world, rank, local):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
+                   "v_fetch": "library's choice: V tiles with K in a single-round launch, else kept rows only",
                    "cluster_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
                    "l2": (f"inputs rotate over {rep.R} cache copies "
                           f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)" if rep.l2_cold else
@@ -385,6 +394,8 @@ def gpu_arm(args, world, rank, local):
                                for k, v in res["sparse_cluster_max"].items()},
         "sparse_sequence_max": {k: (round(v, 6) if isinstance(v, float) else v)
                                 for k, v in res["sparse_sequence_max"].items()},
+        **{tag: {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res[tag].items()}
+           for tag in ("sparse_v_kept_only", "sparse_v_with_k", "sparse_sequence_max_v_kept_only")},
         "two_launch_us_per_token": round(ms_two * 1e3 / args.steps / (wl.batch * world), 4),
         "clocks": sampler.report(),
     }

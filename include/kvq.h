@@ -86,6 +86,8 @@ extern "C" {
 /* Option bits of kvq_decode_attn. */
 #define KVQ_OPT_SHARED_MAX 1u  /* the splits of one cluster share one running maximum (below) */
 #define KVQ_OPT_GLOBAL_MAX 2u  /* every split uses the maximum over all splits of its sequence (below) */
+#define KVQ_OPT_V_KEPT_ONLY 4u /* tau > 0: copy only the kept V rows, after the skip test (below) */
+#define KVQ_OPT_V_WITH_K    8u /* tau > 0: copy every V tile together with its K tile (below) */
 
 /* Device flag bits (kvq_read_device_flags). */
 #define KVQ_FLAG_BAD_PAGE     1u  /* a page-table entry outside [0, num_pages) */
@@ -201,8 +203,19 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                tau = 0 keeps everything (dense attention).
  *                Skipped positions still count in the softmax denominator.
  *   split_tokens as for kvq_resolve_split (0 = auto)
- *   options      0, KVQ_OPT_SHARED_MAX or KVQ_OPT_GLOBAL_MAX; other bits or both are an
- *                error.  KVQ_OPT_GLOBAL_MAX needs every split of the request on its own
+ *   options      at most one of KVQ_OPT_SHARED_MAX and KVQ_OPT_GLOBAL_MAX, at most one
+ *                of KVQ_OPT_V_KEPT_ONLY and KVQ_OPT_V_WITH_K; other bits or both of a
+ *                pair are an error.
+ *                How V reaches the SM (results are the same either way): with
+ *                KVQ_OPT_V_KEPT_ONLY a split copies only its kept V rows, once its
+ *                skip test is done (fewest bytes; a second DRAM round trip); with
+ *                KVQ_OPT_V_WITH_K every V tile is copied together with its K tile and
+ *                the skipped rows are left out of the contraction only (more bytes, no
+ *                second round trip).  Neither: V_WITH_K when every split of the request
+ *                runs on its own CTA at once (a single-round launch, bound by latency),
+ *                else V_KEPT_ONLY.  tau = 0 always copies V with K.  Formats whose
+ *                staging does not fit shared memory twice copy kept rows only.
+ *                KVQ_OPT_GLOBAL_MAX needs every split of the request on its own
  *                CTA at once (KVQ_ERR_UNSUPPORTED otherwise): the CTAs of a (sequence, KV
  *                head) exchange their maxima through the workspace between the K pass
  *                and the V pass (a bounded wait; KVQ_FLAG_TIMEOUT if it gives up).
@@ -212,7 +225,8 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                o may be left unwritten).
  *   stats        device uint64 [4] or NULL; ADDED to (caller zeroes):
  *                [0] (position, query head) pairs scored, [1] pairs skipped,
- *                [2] V rows read (positions kept by any head of the group),
+ *                [2] V rows needed (positions kept by any head of the group; the
+ *                rows copied, unless V tiles are copied with K),
  *                [3] V rows skipped
  *   out          device fp32 [batch][num_q_heads][head_dim], 16-byte aligned, or NULL.
  *                When given, the same kernel also merges the splits and writes the

@@ -31,6 +31,8 @@ FORMATS = {"q8_0": KVQ_FMT_Q8_0, "q4_0": KVQ_FMT_Q4_0, "lut4": KVQ_FMT_LUT4, "nv
 
 KVQ_OPT_SHARED_MAX = 1
 KVQ_OPT_GLOBAL_MAX = 2
+KVQ_OPT_V_KEPT_ONLY = 4
+KVQ_OPT_V_WITH_K = 8
 
 KVQ_FLAG_BAD_PAGE = 1
 KVQ_FLAG_BAD_SEQLEN = 2

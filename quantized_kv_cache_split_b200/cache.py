@@ -77,19 +77,24 @@ class QuantizedKVCache:
                   page_table: Optional[torch.Tensor] = None, max_pages: int = 1,
                   tau: float = 1e-6, sm_scale: Optional[float] = None, split_tokens: int = 0,
                   out: Optional[torch.Tensor] = None, stats: Optional[torch.Tensor] = None,
-                  max_scope: str = "split", fused: bool = True, stream=None) -> torch.Tensor:
+                  max_scope: str = "split", fused: bool = True, v_fetch: str = "auto",
+                  stream=None) -> torch.Tensor:
         """Decode attention of q [batch, num_q_heads, head_dim] (fp16) -> fp32 output.
 
         ``fused``: merge the split partials inside the decode kernel (one launch);
         otherwise kvq_combine merges them in a second launch.  ``max_scope``: the running
         maximum the skip test uses: "split" (each split's own), "cluster" (shared by the
         splits of a thread-block cluster) or "sequence" (over all splits of the
-        sequence and KV head)."""
+        sequence and KV head).  ``v_fetch``: how V rows reach the SM when tau > 0:
+        "kept" (only the kept rows, after the skip test), "with_k" (every V tile with its
+        K tile; skipped rows are left out of the contraction only) or "auto" (with_k for
+        a single-round launch, else kept); the result is the same."""
         B, Hq, D = q.shape
         if sm_scale is None:
             sm_scale = 1.0 / math.sqrt(D)
         opts = {"split": 0, "cluster": kb.KVQ_OPT_SHARED_MAX, "sequence": kb.KVQ_OPT_GLOBAL_MAX}[max_scope]
         ws, nbytes, L = self.workspace(B, Hq, max_seq_len, split_tokens, opts)
+        opts |= {"auto": 0, "kept": kb.KVQ_OPT_V_KEPT_ONLY, "with_k": kb.KVQ_OPT_V_WITH_K}[v_fetch]
         if out is None:
             out = torch.empty((B, Hq, D), dtype=torch.float32, device=self.device)
         kb.kvq_decode_attn(self.desc, q, B, Hq, self.k_codes, self.k_scales, self.v_codes,

@@ -64,8 +64,10 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
   if (st != KVQ_OK) return st;
   if (batch < 0 || num_q_heads < 1 || max_seq_len < 0 || split_tokens < 0)
     return KVQ_ERR_INVALID_ARG;
-  if (options & ~(KVQ_OPT_SHARED_MAX | KVQ_OPT_GLOBAL_MAX)) return KVQ_ERR_INVALID_ARG;
+  if (options & ~(KVQ_OPT_SHARED_MAX | KVQ_OPT_GLOBAL_MAX | KVQ_OPT_V_KEPT_ONLY | KVQ_OPT_V_WITH_K))
+    return KVQ_ERR_INVALID_ARG;
   if ((options & KVQ_OPT_SHARED_MAX) && (options & KVQ_OPT_GLOBAL_MAX)) return KVQ_ERR_INVALID_ARG;
+  if ((options & KVQ_OPT_V_KEPT_ONLY) && (options & KVQ_OPT_V_WITH_K)) return KVQ_ERR_INVALID_ARG;
   int L;
   if (split_tokens > 0) {
     L = std::min(split_tokens, KVQ_MAX_SPLIT_TOKENS);
@@ -285,6 +287,8 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   // the maximum over all splits needs every split on its own CTA at once
   if (a.global_max && groups > capacity) return KVQ_ERR_UNSUPPORTED;
   a.grid = (int)std::min<int64_t>(groups, capacity) * CS;
+  // a single round is latency-bound: V comes with K unless the caller says otherwise
+  a.v_early = (options & KVQ_OPT_V_WITH_K) ? 1 : (options & KVQ_OPT_V_KEPT_ONLY) ? 0 : groups <= capacity;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -602,6 +602,18 @@ __device__ __forceinline__ void build_query(const QRaw<D>& q, int c,
 }
 
 // ------------------------------------------------------------------ V groups
+// Where the V rows of a group sit in the staging buffer: kVGathered: slot s holds the s-th
+// kept row (codes) and the 16-byte window of the scales plane holding its scales;
+// kVTile: slot s is row s of a staged 64-row tile; kVTileList: a staged tile whose kept
+// rows are named by the warp's list (slot s is tile row list[s]; rows are masked into the
+// tile, so a stale entry past the kept count still names a row of the tile).
+enum VSrc { kVGathered = 0, kVTile = 1, kVTileList = 2 };
+
+template <int SRC>
+__device__ __forceinline__ int v_row(const uint8_t* list, int slot) {
+  return SRC == kVTileList ? (list[slot] & (kTile - 1)) : slot;
+}
+
 // Chunk swizzle of a staged row (K tiles and V rows alike): 16-byte chunk cc of row `row`
 // sits at chunk position cc ^ swz(row).
 template <int FMT, int D>
@@ -630,12 +642,12 @@ __device__ __forceinline__ void copy_v_tile(uint8_t* dst, const uint8_t* vcodes,
 }
 
 // lut4 / nvfp4: one group of 16 staged V positions (slots s0 .. s0 + 15 of the staging
-// buffer): acc[dims x heads] += v_hat^T p.  TILE: slot s is row s of a staged tile;
-// otherwise a gathered row whose scales sit in its window at (trow & (RPW - 1)) * SROW
-// (trow: the row's index in its tile).  Slots at or past n_valid (counted from s0) get
-// scale 0, so whatever bytes they hold contribute nothing (every format decodes any bit
-// pattern to a finite value).  Thread (r, c) owns dims E*r .. E*r + E - 1.
-template <int FMT, int D, bool TILE>
+// buffer, placed as SRC says): acc[dims x heads] += v_hat^T p.  A gathered row's scales
+// sit in its window at (trow & (RPW - 1)) * SROW (trow: the row's index in its tile;
+// the list entries of the group).  Slots at or past n_valid (counted from s0) get scale
+// 0, so whatever bytes they hold contribute nothing (every format decodes any bit pattern
+// to a finite value).  Thread (r, c) owns dims E*r .. E*r + E - 1.
+template <int FMT, int D, int SRC>
 __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const __half* __restrict__ prow,
                                         const uint8_t* __restrict__ trow, int s0, int n_valid,
                                         int r, int c, const Lut& lut,
@@ -646,13 +658,15 @@ __device__ __forceinline__ void v_group(const uint8_t* __restrict__ buf, const _
   const uint32_t b0 = lds32(prow + sa);
   const uint32_t b1 = lds32(prow + sc);
   auto code = [&](int slot) -> const uint8_t* {
-    const int row = s0 + slot, o = C::RAWB * r;
+    const int row = SRC == kVTileList ? v_row<SRC>(trow, slot) : s0 + slot, o = C::RAWB * r;
     return buf + row * C::CROW + (((o >> 4) ^ swz<FMT, D>(row)) << 4) + (o & 15);
   };
   auto scale = [&](int slot) -> __half {
     if (slot >= n_valid) return __ushort_as_half(0);
-    const uint8_t* srow = TILE ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW
-                               : buf + C::GSC + (s0 + slot) * 16 + (trow[slot] & (C::RPW - 1)) * C::SROW;
+    const uint8_t* srow =
+        SRC == kVTile       ? buf + C::STAGE_CODE + (s0 + slot) * C::SROW
+        : SRC == kVTileList ? buf + C::STAGE_CODE + v_row<SRC>(trow, slot) * C::SROW
+                           : buf + C::GSC + (s0 + slot) * 16 + (trow[slot] & (C::RPW - 1)) * C::SROW;
     if constexpr (C::kNv)  // E4M3 block scale of this thread's dims times the vector scale
       return __float2half_rn(e4m3_float(srow[(C::E * r) / 16]) *
                              *reinterpret_cast<const float*>(srow + D / 16));
@@ -698,18 +712,18 @@ __device__ __forceinline__ int v_dim(int r, int mt, int i) {
   else return C::E * r + 2 * mt + (i >> 1);
 }
 
-// The scale row of staged slot `slot` (TILE: a tile's scale rows; otherwise the row's
-// place in its gathered 16-byte window).
-template <int FMT, int D, bool TILE>
+// The scale row of staged slot `slot` (a tile's scale rows, or the row's place in its
+// gathered 16-byte window).
+template <int FMT, int D, int SRC>
 __device__ __forceinline__ uint8_t* v_scale_row(uint8_t* buf, const uint8_t* list, int slot) {
   using C = Cfg<FMT, D>;
-  return TILE ? buf + C::STAGE_CODE + slot * C::SROW
-              : buf + C::GSC + slot * 16 + (list[slot] & (C::RPW - 1)) * C::SROW;
+  if constexpr (SRC == kVGathered) return buf + C::GSC + slot * 16 + (list[slot] & (C::RPW - 1)) * C::SROW;
+  return buf + C::STAGE_CODE + v_row<SRC>(list, slot) * C::SROW;
 }
 
 // Per block, k = the smallest exponent >= 0 with d 2^-k < 2 for every staged slot
 // 0 .. n - 1, and those scales multiplied by 2^-k in place (exact).  Warp-wide.
-template <int FMT, int D, bool TILE>
+template <int FMT, int D, int SRC>
 __device__ __forceinline__ void v_mag_normalize(uint8_t* buf, const uint8_t* list, int n, int lane,
                                                 int (&k)[Cfg<FMT, D>::NBLK]) {
   using C = Cfg<FMT, D>;
@@ -721,7 +735,7 @@ __device__ __forceinline__ void v_mag_normalize(uint8_t* buf, const uint8_t* lis
   for (int h = 0; h < 2; ++h) {
     const int slot = lane + 32 * h;
     if (slot < n) {
-      const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, slot));
+      const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, SRC>(buf, list, slot));
 #pragma unroll
       for (int w = 0; w < NW; ++w)  // |d| (scales are >= 0 but may be -0)
         mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(sr[w] & 0x7FFF7FFFu)));
@@ -744,7 +758,7 @@ __device__ __forceinline__ void v_mag_normalize(uint8_t* buf, const uint8_t* lis
   for (int h = 0; h < 2; ++h) {
     const int slot = lane + 32 * h;
     if (slot < n) {
-      uint32_t* sr = reinterpret_cast<uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, slot));
+      uint32_t* sr = reinterpret_cast<uint32_t*>(v_scale_row<FMT, D, SRC>(buf, list, slot));
 #pragma unroll
       for (int w = 0; w < NW; ++w) sr[w] = h2_as_u32(__hmul2(u32_as_h2(sr[w]), u32_as_h2(f[w])));
     }
@@ -754,7 +768,7 @@ __device__ __forceinline__ void v_mag_normalize(uint8_t* buf, const uint8_t* lis
 
 // One group of 16 staged positions (slots s0 .. s0 + 15; slots at or past n_valid,
 // counted from s0, get weight 0).
-template <int FMT, int D, bool TILE>
+template <int FMT, int D, int SRC>
 __device__ __forceinline__ void v_group_mag(uint8_t* __restrict__ buf, const __half* __restrict__ prow,
                                             const uint8_t* __restrict__ list, int s0, int n_valid,
                                             int lane, int r, int c, float (&acc)[Cfg<FMT, D>::MT][4]) {
@@ -766,7 +780,7 @@ __device__ __forceinline__ void v_group_mag(uint8_t* __restrict__ buf, const __h
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int slot = 2 * c + (q & 1) + 8 * (q >> 1);
-    const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, TILE>(buf, list, s0 + slot));
+    const uint32_t* sr = reinterpret_cast<const uint32_t*>(v_scale_row<FMT, D, SRC>(buf, list, s0 + slot));
 #pragma unroll
     for (int w = 0; w < NW; ++w) ws[q][w] = slot < n_valid ? sr[w] : 0u;
   }
@@ -783,7 +797,7 @@ __device__ __forceinline__ void v_group_mag(uint8_t* __restrict__ buf, const __h
   // codes, two chunks per matrix load: matrix i = (positions s0 + 8 (i & 1) .., chunk
   // cb + (i >> 1)), so R[j][h] = chunk cb + j, positions 2c, 2c + 1 (+ 8 h)
   const int mi = lane >> 3;
-  const int row = s0 + 8 * (mi & 1) + (lane & 7);
+  const int row = v_row<SRC>(list, s0 + 8 * (mi & 1) + (lane & 7));
   const uint8_t* rp = buf + row * C::CROW;
   const int sw = swz<FMT, D>(row);
 #pragma unroll
@@ -959,7 +973,9 @@ decode_kernel(const DecodeArgs a) {
 
   const float qk_scale = a.sm_scale * kLog2e;
   const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
-  const bool prefetch_v = LY::kPrefetchV && !(a.tau > 0.f);  // tau = 0: every row is kept
+  // V tiles copied with K (tau = 0: every row is kept; otherwise when the launch asks,
+  // so that kept rows wait for no second DRAM round trip and skipped rows cost bytes only)
+  const bool prefetch_v = LY::kPrefetchV && (!(a.tau > 0.f) || a.v_early);
   const __half* qg = static_cast<const __half*>(a.q);
   const uint8_t* kcodes = static_cast<const uint8_t*>(a.k_codes);
   const uint8_t* kscales = static_cast<const uint8_t*>(a.k_scales);
@@ -1325,7 +1341,7 @@ decode_kernel(const DecodeArgs a) {
 #pragma unroll
       for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       const int ng = (nkept + 15) >> 4;
-      if (prefetch_v || nkept == nvalid) {
+      if (nkept == nvalid) {
         // every valid row is kept, so slot s is tile row s; without the prefetched tile,
         // one copy of the V tile into the (now free) K buffer
         uint8_t* vt = prefetch_v ? vtile : kbuf;
@@ -1337,17 +1353,35 @@ decode_kernel(const DecodeArgs a) {
         __syncwarp();
         if constexpr (C::kMag) {
           int kx[C::NBLK];
-          v_mag_normalize<FMT, D, true>(vt, list_w, nkept, lane, kx);
+          v_mag_normalize<FMT, D, kVTile>(vt, list_w, nkept, lane, kx);
 #pragma unroll 2
           for (int g = 0; g < ng; ++g)
-            v_group_mag<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
-                                      min(16, nkept - 16 * g), lane, r, c, acc);
+            v_group_mag<FMT, D, kVTile>(vt, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
+                                       min(16, nkept - 16 * g), lane, r, c, acc);
           v_mag_finish<FMT, D>(acc, kx);
         } else {
 #pragma unroll 2
           for (int g = 0; g < ng; ++g)
-            v_group<FMT, D, true>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
-                                  min(16, nkept - 16 * g), r, c, lut, acc);
+            v_group<FMT, D, kVTile>(vt, pk_w + r * kPkStride + 16 * g, nullptr, 16 * g,
+                                   min(16, nkept - 16 * g), r, c, lut, acc);
+        }
+      } else if (prefetch_v) {
+        // the tile is staged already: only its kept rows (the list) enter the contraction
+        cp_async_wait<0>();
+        __syncwarp();
+        if constexpr (C::kMag) {
+          int kx[C::NBLK];
+          v_mag_normalize<FMT, D, kVTileList>(vtile, list_w, nkept, lane, kx);
+#pragma unroll 2
+          for (int g = 0; g < ng; ++g)
+            v_group_mag<FMT, D, kVTileList>(vtile, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
+                                           min(16, nkept - 16 * g), lane, r, c, acc);
+          v_mag_finish<FMT, D>(acc, kx);
+        } else {
+#pragma unroll 2
+          for (int g = 0; g < ng; ++g)
+            v_group<FMT, D, kVTileList>(vtile, pk_w + r * kPkStride + 16 * g, list_w + 16 * g, 16 * g,
+                                       min(16, nkept - 16 * g), r, c, lut, acc);
         }
       } else {
         // gather the kept rows into the (now free) K buffer: slot s gets its codes (chunk
@@ -1368,17 +1402,17 @@ decode_kernel(const DecodeArgs a) {
         __syncwarp();
         if constexpr (C::kMag) {
           int kx[C::NBLK];
-          v_mag_normalize<FMT, D, false>(kbuf, list_w, nkept, lane, kx);
+          v_mag_normalize<FMT, D, kVGathered>(kbuf, list_w, nkept, lane, kx);
 #pragma unroll 2
           for (int g = 0; g < ng; ++g)
-            v_group_mag<FMT, D, false>(kbuf, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
-                                       min(16, nkept - 16 * g), lane, r, c, acc);
+            v_group_mag<FMT, D, kVGathered>(kbuf, pk_w + r * kPkStride + 16 * g, list_w, 16 * g,
+                                           min(16, nkept - 16 * g), lane, r, c, acc);
           v_mag_finish<FMT, D>(acc, kx);
         } else {
 #pragma unroll 2
           for (int g = 0; g < ng; ++g)
-            v_group<FMT, D, false>(kbuf, pk_w + r * kPkStride + 16 * g, list_w + 16 * g, 16 * g,
-                                   min(16, nkept - 16 * g), r, c, lut, acc);
+            v_group<FMT, D, kVGathered>(kbuf, pk_w + r * kPkStride + 16 * g, list_w + 16 * g, 16 * g,
+                                       min(16, nkept - 16 * g), r, c, lut, acc);
         }
       }
       __syncwarp();  // staged V fully read before the accumulators overwrite the buffer

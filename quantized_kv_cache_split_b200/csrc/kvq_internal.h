@@ -44,6 +44,8 @@ struct DecodeArgs {
   int units_per_seq;  // cluster groups of one (sequence, KV head) at max_seq_len
   int group_merge;    // every unit has its own CTA: the splits of a (sequence, KV head)
                       // exchange (m, l) and each adds its share into the output
+  int v_early;        // tau > 0: copy each V tile together with its K tile (every row,
+                      // kept or not) instead of only the kept rows after the skip test
 };
 
 // Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch

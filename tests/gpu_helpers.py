@@ -19,11 +19,12 @@ def codebook_for(D: int) -> np.ndarray:
 
 
 def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=None,
-                max_scope: str = "split", fused: bool = True):
+                max_scope: str = "split", fused: bool = True, v_fetch: str = "auto"):
     """One decode step through the C ABI.  ``fused``: the merge runs inside the decode
     kernel; otherwise kvq_combine runs it.  ``max_scope``: "split", "cluster" (the
     splits of a cluster share one running maximum; the oracle replays it with share =
-    the cluster size) or "sequence" (share = every split)."""
+    the cluster size) or "sequence" (share = every split).  ``v_fetch``: the V copy
+    policy ("auto", "kept", "with_k"), which must not change the result."""
     import quantized_kv_cache_split_b200 as K
     wl = inp.wl
     D, Hkv = wl.head_dim, wl.num_kv_heads
@@ -44,7 +45,7 @@ def run_library(inp: W.Inputs, tau: float, split_tokens: int = 0, codebook16=Non
     out = cache.attention(q, seq, max_seq, pt, inp.max_pages, tau=tau,
                           sm_scale=float(np.float32(1.0 / math.sqrt(D))),
                           split_tokens=split_tokens, stats=stats, max_scope=max_scope,
-                          fused=fused)
+                          fused=fused, v_fetch=v_fetch)
     torch.cuda.synchronize()
     opts = {"split": 0, "cluster": K.KVQ_OPT_SHARED_MAX, "sequence": K.KVQ_OPT_GLOBAL_MAX}[max_scope]
     L = K.kvq_resolve_split(cache.desc, wl.batch, wl.num_q_heads, max_seq, split_tokens, opts)

@@ -148,8 +148,9 @@ def _decode(d, **kw):
     (dict(batch=K.KVQ_MAX_BATCH + 1, max_pages=1), K.KVQ_ERR_UNSUPPORTED),
     (dict(batch=9, max_pages=1), K.KVQ_ERR_INVALID_ARG),  # identity pages beyond num_pages
     (dict(batch=0), K.KVQ_OK),
-    (dict(options=4), K.KVQ_ERR_INVALID_ARG),           # unknown option bit
+    (dict(options=16), K.KVQ_ERR_INVALID_ARG),          # unknown option bit
     (dict(options=3), K.KVQ_ERR_INVALID_ARG),           # two maximum scopes at once
+    (dict(options=12), K.KVQ_ERR_INVALID_ARG),          # two V fetch policies at once
     (dict(q=FAKE + 8), K.KVQ_ERR_INVALID_ARG),          # query not 16-byte aligned
     (dict(out=FAKE + 2), K.KVQ_ERR_INVALID_ARG),        # output not 4-byte aligned
     (dict(workspace=FAKE + 8), K.KVQ_ERR_INVALID_ARG),  # workspace not 16-byte aligned

@@ -241,6 +241,24 @@ def test_decode_parity_paged_ragged(fmt, tau, split, scope):
 
 
 @pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
+@pytest.mark.parametrize("v_fetch", ["kept", "with_k"])
+@pytest.mark.parametrize("tau,split,scope", [(1e-6, 0, "split"), (1e-4, 128, "split"), (1e-6, 0, "sequence"),
+                                             (1e-2, 64, "cluster")])
+def test_decode_parity_v_fetch_policies(fmt, v_fetch, tau, split, scope):
+    # V rows copied after the skip test (kept rows only) or together with K (skipped
+    # rows left out of the contraction): the same result, the same skip counts, in
+    # single-round (split 0) and multi-round (split 128, 64) launches
+    base = W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt)
+    wl = W.shrink(base, RAGGED_LENS, n_planted=8)
+    inp = W.generate(wl)
+    cb = codebook_for(wl.head_dim) if fmt == "lut4" else None
+    g = run_library(inp, tau, split, cb, max_scope=scope, v_fetch=v_fetch)
+    o = run_oracle(inp, tau, g["split"], cb, share=g["share"])
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+
+
+@pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
 @pytest.mark.parametrize("hq,hkv", [(4, 4), (4, 2), (8, 1)])
 def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
     wl = W.WORKLOADS["tiny_q8_d64"].with_(fmt=fmt, num_q_heads=hq, num_kv_heads=hkv,
@@ -268,6 +286,16 @@ def test_decode_parity_full_32k(name, tau, scope):
     if tau > 0:
         # the workload's point: most weights are skipped
         assert g["stats"][1] > 0.5 * g["stats"][0]
+
+
+@pytest.mark.parametrize("v_fetch,scope", [("kept", "split"), ("kept", "sequence"), ("with_k", "cluster")])
+def test_decode_parity_full_32k_v_fetch(v_fetch, scope):
+    # the single-round 32K launch copies V with K by default: the other policy too
+    wl = W.WORKLOADS["gqa_32k_q4"]
+    inp = W.generate(wl)
+    g = run_library(inp, 1e-6, 0, None, max_scope=scope, v_fetch=v_fetch)
+    o = run_oracle(inp, 1e-6, g["split"], None, share=g["share"])
+    check_parity(inp, g, o, 1e-6)
 
 
 @pytest.mark.parametrize("name", ["paged_b8_q4", "paged_b8_q8"])

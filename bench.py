@@ -327,8 +327,8 @@ def gpu_arm(args, world, rank, local):
     res = {}
     hbm_peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
-    # the headline leaves the V fetch to the library (V with K in a single-round launch,
-    # kept rows only otherwise); the two policies are also timed on their own
+    # the headline leaves the V fetch to the library (V with K; nvfp4: kept rows only);
+    # the two policies are also timed on their own
     variants = (("sparse", args.tau, "split", 0), ("dense", 0.0, "split", 0),
                 ("sparse_v_kept_only", args.tau, "split", K.KVQ_OPT_V_KEPT_ONLY),
                 ("sparse_v_with_k", args.tau, "split", K.KVQ_OPT_V_WITH_K),
@@ -372,7 +372,7 @@ def gpu_arm(args, world, rank, local):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
-                   "v_fetch": "library's choice: V tiles with K in a single-round launch, else kept rows only",
+                   "v_fetch": "library's choice: V tiles with K (nvfp4: kept rows only)",
                    "cluster_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
                    "l2": (f"inputs rotate over {rep.R} cache copies "
                           f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)" if rep.l2_cold else

@@ -211,10 +211,11 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                skip test is done (fewest bytes; a second DRAM round trip); with
  *                KVQ_OPT_V_WITH_K every V tile is copied together with its K tile and
  *                the skipped rows are left out of the contraction only (more bytes, no
- *                second round trip).  Neither: V_WITH_K when every split of the request
- *                runs on its own CTA at once (a single-round launch, bound by latency),
- *                else V_KEPT_ONLY.  tau = 0 always copies V with K.  Formats whose
- *                staging does not fit shared memory twice copy kept rows only.
+ *                second round trip).  Neither: V_WITH_K, except KVQ_FMT_NVFP4 (kept rows
+ *                only); both measured on B200, where these steps are bound by latency
+ *                and the MMA pipe rather than by HBM bytes.  tau = 0 always copies V
+ *                with K.  Formats whose staging does not fit shared memory twice
+ *                (q8_0 at head_dim 128) copy kept rows only.
  *                KVQ_OPT_GLOBAL_MAX needs every split of the request on its own
  *                CTA at once (KVQ_ERR_UNSUPPORTED otherwise): the CTAs of a (sequence, KV
  *                head) exchange their maxima through the workspace between the K pass

@@ -87,8 +87,8 @@ class QuantizedKVCache:
         splits of a thread-block cluster) or "sequence" (over all splits of the
         sequence and KV head).  ``v_fetch``: how V rows reach the SM when tau > 0:
         "kept" (only the kept rows, after the skip test), "with_k" (every V tile with its
-        K tile; skipped rows are left out of the contraction only) or "auto" (with_k for
-        a single-round launch, else kept); the result is the same."""
+        K tile; skipped rows are left out of the contraction only) or "auto" (with_k,
+        except nvfp4: kept); the result is the same."""
         B, Hq, D = q.shape
         if sm_scale is None:
             sm_scale = 1.0 / math.sqrt(D)

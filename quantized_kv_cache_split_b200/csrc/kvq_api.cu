@@ -287,8 +287,12 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   // the maximum over all splits needs every split on its own CTA at once
   if (a.global_max && groups > capacity) return KVQ_ERR_UNSUPPORTED;
   a.grid = (int)std::min<int64_t>(groups, capacity) * CS;
-  // a single round is latency-bound: V comes with K unless the caller says otherwise
-  a.v_early = (options & KVQ_OPT_V_WITH_K) ? 1 : (options & KVQ_OPT_V_KEPT_ONLY) ? 0 : groups <= capacity;
+  // At these sizes the step is bound by latency and the legacy MMA pipe, not by bytes, so
+  // by default V comes with K (no second DRAM round trip); nvfp4 gathers its kept rows
+  // instead (its V pass over a partly kept staged tile measured slower than the gather)
+  a.v_early = (options & KVQ_OPT_V_WITH_K)      ? 1
+              : (options & KVQ_OPT_V_KEPT_ONLY) ? 0
+                                                : desc->fmt != KVQ_FMT_NVFP4;
   return launch_decode(a, static_cast<cudaStream_t>(stream));
 }
 

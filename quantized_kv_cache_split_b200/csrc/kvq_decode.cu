@@ -10,14 +10,16 @@
 // (sequence, KV head).  A thread-block cluster of CS CTAs (CS = 1, 2 or 4) takes CS
 // consecutive splits of the same (sequence, KV head); clusters loop persistently
 // over such groups.  Each CTA has 16 warps; warp w owns tile w of its split.
-//   Q         Every warp builds its own query fragments straight from global memory
-//             (lut4: rotates the query with butterflies in registers and shuffles),
-//             while its K copies are in flight; no block-wide step.
+//   Q         Warp 0 builds the query fragments (lut4: rotates the query with
+//             butterflies in registers and shuffles) while the K copies are in flight
+//             and shares them through shared memory.
 //   K fetch   The warp streams its tile's codes and block scales into its private
 //             shared buffer with 16-byte cp.async copies, one copy group per 16-row
 //             job (an XOR swizzle of the 16-byte chunks keeps the MMA fragment reads
-//             free of bank conflicts).  With tau = 0 (nothing can be skipped) it also
-//             prefetches its V tile at once, when shared memory allows.
+//             free of bank conflicts).  With V fetched early (tau = 0, or when the
+//             launch asks: the library's default except for nvfp4, since these steps
+//             are bound by latency rather than bytes) it also copies its V tile at
+//             once, when shared memory allows.
 //   K pass    As each job's copies land, the warp scores its 16 positions x 8 query
 //             heads on the tensor cores (mma m16n8k16: positions x heads x head_dim).
 //             Codes enter the MMA as magic-number fp16 values (code + a fixed
@@ -26,23 +28,29 @@
 //             norm is applied to the fp32 score.  Scores stay in registers.
 //   max       One CTA barrier gives the split's maximum per head; with the shared
 //             maximum option, one cluster barrier and a read of the other CTAs'
-//             maxima (distributed shared memory) give the cluster's.
+//             maxima (distributed shared memory) give the cluster's; with the
+//             sequence-wide option, a tagged exchange through the workspace gives the
+//             maximum over every split of the (sequence, KV head).
 //   weights   Each warp tests its scores: keep iff s - m >= log2(tau) (no exp needed
 //             for the test); l sums 2^(s - m) over every position; positions kept by
 //             any head of the group are compacted (ballot + popcount) into the warp's
 //             own list.  No block-wide step.
-//   V pass    The warp gathers only its kept V rows (16-byte cp.async copies of the
-//             codes plus a 16-byte window holding the row's scales), dequantizes them
-//             in registers and accumulates p^T V on the tensor cores (head_dim x
-//             heads x positions).  Skipped positions cost no HBM read, no dequant and
-//             no MMA.  A warp with nothing kept does nothing.
+//   V pass    Only the kept rows enter the contraction: p^T V on the tensor cores
+//             (head_dim x heads x positions), the rows dequantized in registers.
+//             Without the early copy the warp gathers just those rows (16-byte
+//             cp.async copies of the codes plus a 16-byte window holding the row's
+//             scales), so skipped positions cost no HBM read, no dequant and no MMA;
+//             with it, the list addresses the kept rows inside the staged tile.  A
+//             warp with nothing kept does nothing.
 //   output    The warps' accumulators (only those of warps that kept something) are
 //             summed through shared memory.  The CTAs of a cluster merge their (o, m,
-//             l) through distributed shared memory into one partial per cluster,
-//             which goes to the workspace.  When an output pointer is given, the last
-//             cluster to finish a (sequence, KV head) (an arrival counter in the
-//             workspace) merges that pair's partials by the log-sum-exp rule and
-//             writes the output (lut4: rotated back), so no second kernel runs.
+//             l) through distributed shared memory into one partial per cluster.
+//             When an output pointer is given the merge runs in this kernel: if every
+//             unit has its own CTA, the splits of a (sequence, KV head) exchange their
+//             (m, l) and each adds its normalized share into the output; otherwise
+//             the last cluster to finish the pair (an arrival counter in the
+//             workspace) merges the written partials by the log-sum-exp rule (lut4:
+//             the output is rotated back), so no second kernel runs.
 #include <mutex>
 
 #include <cuda_fp8.h>
@@ -105,7 +113,7 @@ struct Cfg {
   // per-warp buffer: its K tile, then its staged V rows, then its accumulators for the
   // block-wide sum
   static constexpr int KBUF = round128(cmax3(TILE, STAGE_CODE + kTile * 16, NE * 32 * 4));
-  static constexpr int VT = round128(TILE);              // per-warp prefetched V tile (tau = 0)
+  static constexpr int VT = round128(TILE);              // per-warp V tile copied with K
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
 
@@ -129,7 +137,7 @@ struct Layout {
   static constexpr int kQfWords = 2 * C::KSTEPS + (C::kLut ? 2 * C::KSTEPS : 0) + 2 * C::NBLK;
   static constexpr size_t qfr = scr + (size_t)kWarps * 4 * 32 * 16;
   static constexpr size_t base_total = qfr + (size_t)kQfWords * 32 * 4;
-  // tau = 0 prefetches the V tile alongside K when shared memory allows
+  // the V tiles copied with K (tau = 0, or when the launch asks) when shared memory allows
   static constexpr size_t vtile = (base_total + 127) / 128 * 128;             // [warps][VT]
   static constexpr bool kPrefetchV = vtile + (size_t)kWarps * C::VT + 128 <= kSmemLimit;
   static constexpr size_t total = kPrefetchV ? vtile + (size_t)kWarps * C::VT : base_total;
@@ -1022,7 +1030,7 @@ decode_kernel(const DecodeArgs a) {
       load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr,
                          a.desc.signs, c, qraw);
 
-    // ---- K fetch (and, for tau = 0, the V tile): one copy group per 16-row job
+    // ---- K fetch (and, when V is fetched early, the V tile): one copy group per 16-row job
     int row0 = -1;
     const int ncopy = min(kTile, avail - t0 - warp * kTile);
     if (ncopy > 0) {
@@ -1262,10 +1270,13 @@ decode_kernel(const DecodeArgs a) {
         const float eb0 = vb && hl0 ? ex2(sv.z - mh0) : 0.f, eb1 = vb && hl1 ? ex2(sv.w - mh1) : 0.f;
         l0 += ea0 + eb0;
         l1 += ea1 + eb1;
-        pk_w[(2 * c) * kPkStride + ra] = __float2half_rn(ea0 * kPScale);
-        pk_w[(2 * c + 1) * kPkStride + ra] = __float2half_rn(ea1 * kPScale);
-        pk_w[(2 * c) * kPkStride + rb] = __float2half_rn(eb0 * kPScale);
-        pk_w[(2 * c + 1) * kPkStride + rb] = __float2half_rn(eb1 * kPScale);
+        // two weights per conversion (the conversion pipe is the scarce unit here)
+        const __half2 pa = __floats2half2_rn(ea0 * kPScale, ea1 * kPScale);
+        const __half2 pb = __floats2half2_rn(eb0 * kPScale, eb1 * kPScale);
+        pk_w[(2 * c) * kPkStride + ra] = __low2half(pa);
+        pk_w[(2 * c + 1) * kPkStride + ra] = __high2half(pa);
+        pk_w[(2 * c) * kPkStride + rb] = __low2half(pb);
+        pk_w[(2 * c + 1) * kPkStride + rb] = __high2half(pb);
       }
       nkept = nvalid;
     }
@@ -1288,17 +1299,19 @@ decode_kernel(const DecodeArgs a) {
         const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
         const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
         const int na = __popc(rows_a);
+        const __half2 pa = __floats2half2_rn(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f);
+        const __half2 pb = __floats2half2_rn(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f);
         if ((rows_a >> (4 * r)) & 1u) {
           const int slot = nkept + __popc(rows_a & below);
           if (c == 0) list_w[slot] = (uint8_t)ra;
-          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(ka0 ? ea0 * kPScale : 0.f);
-          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(ka1 ? ea1 * kPScale : 0.f);
+          pk_w[(2 * c) * kPkStride + slot] = __low2half(pa);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __high2half(pa);
         }
         if ((rows_b >> (4 * r)) & 1u) {
           const int slot = nkept + na + __popc(rows_b & below);
           if (c == 0) list_w[slot] = (uint8_t)rb;
-          pk_w[(2 * c) * kPkStride + slot] = __float2half_rn(kb0 ? eb0 * kPScale : 0.f);
-          pk_w[(2 * c + 1) * kPkStride + slot] = __float2half_rn(kb1 ? eb1 * kPScale : 0.f);
+          pk_w[(2 * c) * kPkStride + slot] = __low2half(pb);
+          pk_w[(2 * c + 1) * kPkStride + slot] = __high2half(pb);
         }
         nkept += na + __popc(rows_b);
       }
@@ -1437,8 +1450,12 @@ decode_kernel(const DecodeArgs a) {
         first = __shfl_sync(0xffffffffu, first, 0);
       }
       if (first) {
+        // the cleared-rows flag (raised early) first, so that its round trip overlaps
+        // the wait for the last split's (m, l) rather than following it
         bool ok = true;
-        if (!a.global_max) {
+        if (lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok && !a.global_max) {
           // lanes 4h .. 4h + 3 take head h, partials j, j + 4, ... (all loads of up to 64
           // partials in flight together), then combine across the four lanes
           const int h = lane >> 2, j = lane & 3;
@@ -1450,12 +1467,9 @@ decode_kernel(const DecodeArgs a) {
             if (j == 0 && h < G) cmx[16 + h] = ex2(mpart[h] - M) / L;
           }
         }
-        if (lane == 0) {
-          if (ok) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
-          if (!ok) {
-            set_flag(flags, KVQ_FLAG_TIMEOUT);
-            misc[0] = 0;
-          }
+        if (lane == 0 && !ok) {
+          set_flag(flags, KVQ_FLAG_TIMEOUT);
+          misc[0] = 0;
         }
         __syncwarp();
       }
@@ -1465,19 +1479,34 @@ decode_kernel(const DecodeArgs a) {
 
     // ---- this CTA's partial: sum the accumulators of the warps that kept something.
     //      A lone CTA writes it straight to the workspace; a cluster merges first.
-    for (int q = tid; q < 32 * C::NE; q += kThreads) {
-      const int ln = q & 31, e = q >> 5;
-      const int mt = e >> 2, i = e & 3;
-      const int h = 2 * (ln & 3) + (i & 1);
-      const int dim = v_dim<FMT, D>(ln >> 2, mt, i);
-      if (h < G) {
-        float v = 0.f;
+    //      Four consecutive entries per thread (one 16-byte load per warp), the warps
+    //      in index order.
+    uint32_t wk = 0;  // warps whose accumulators hold something
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
-          if (cnt_kept[w] > 0) v += reinterpret_cast<const float*>(smem + LY::kbuf + (size_t)w * C::KBUF)[q];
-        v *= kPUnscale;
-        if (CS > 1 || add_merge) octa[h * D + dim] = v;
-        else a.part_o[(slot0 + (size_t)h * a.max_splits) * D + dim] = v;
+    for (int w = 0; w < kWarps; ++w) wk |= (cnt_kept[w] > 0 ? 1u : 0u) << w;
+    for (int q4 = tid; q4 < 8 * C::NE; q4 += kThreads) {
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        if ((wk >> w) & 1u) {
+          const float4 x = reinterpret_cast<const float4*>(smem + LY::kbuf + (size_t)w * C::KBUF)[q4];
+          v[0] += x.x;
+          v[1] += x.y;
+          v[2] += x.z;
+          v[3] += x.w;
+        }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int q = 4 * q4 + t;
+        const int ln = q & 31, e = q >> 5;
+        const int mt = e >> 2, i = e & 3;
+        const int h = 2 * (ln & 3) + (i & 1);
+        const int dim = v_dim<FMT, D>(ln >> 2, mt, i);
+        if (h < G) {
+          const float o = v[t] * kPUnscale;
+          if (CS > 1 || add_merge) octa[h * D + dim] = o;
+          else a.part_o[(slot0 + (size_t)h * a.max_splits) * D + dim] = o;
+        }
       }
     }
     if (tid < G && !add_merge) {

@@ -288,10 +288,10 @@ def time_steps(runner, steps, warmup, world, sampler=None):
 
 
 def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int, with_o: bool):
-    """HBM bytes one fused decode launch must move: every K row, the kept V rows, Q,
-    the page table, the partials (one per cluster of splits, written once and read
-    once by the in-kernel merge: (m, l) only when each split adds its share into the
-    output itself, also o when a last cluster merges) and the output."""
+    """HBM bytes one decode step must move: every K row, the kept V rows, Q, the page
+    table, the partials (one per cluster of splits, written once and read once by the
+    merge: (m, l) only when each split adds its share into the output itself, also o
+    when a last cluster or the combine kernel merges) and the output."""
     import quantized_kv_cache_split_b200 as K
     wl = rep.wl
     row = K.kvq_code_row_bytes(wl.fmt, wl.head_dim) + 2 * K.kvq_scale_row_count(wl.fmt, wl.head_dim)
@@ -343,8 +343,10 @@ def gpu_arm(args, world, rank, local):
         step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope, v_opt=v_opt), rep.R)
         ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
                                         sampler if tag == "sparse" else None), world, device)
+        # o partials cross HBM when clusters merge them or the combine kernel does
         abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if scope == "cluster"
-                                   else n_partials(rep.L, 1), with_o=scope == "cluster")
+                                   else n_partials(rep.L, 1),
+                                   with_o=scope == "cluster" or decode_launches_per_call(rep, device) == 2)
         us_launch = ms_step * 1e3 / args.steps
         achieved = abytes / (us_launch * 1e-6) / 1e9
         res[tag] = dict(tau=tau, max_scope=scope, v_fetch={0: "auto", K.KVQ_OPT_V_KEPT_ONLY: "kept_only",
@@ -379,7 +381,9 @@ def gpu_arm(args, world, rank, local):
                           f"inputs rotate over {rep.R} cache copies "
                           f"({rep.R * rep.plane_bytes / 2**20:.1f} MiB < L2: timed with the cache in L2)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": "one kvq_decode_attn launch with the in-kernel merge (CUDA graph)"},
+                   "step": ("one kvq_decode_attn call (CUDA graph): "
+                            + ("one launch, merge in the kernel" if decode_launches_per_call(rep, device) == 1
+                               else "decode launch + combine launch"))},
         "roofline": {"bound": "hbm", "achieved": round(sp["achieved_gbs"], 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(sp["frac"], 4),
                      "traffic": sp["traffic"], "peak_kind": peak_kind,
@@ -387,7 +391,7 @@ def gpu_arm(args, world, rank, local):
                      "algorithmic_bytes_per_launch": sp["algorithmic_bytes"],
                      "us_per_launch": round(sp["us_per_launch"], 3)},
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * decode_launches_per_call(rep, device),
         "dense": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res["dense"].items()},
         "sparse": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in sp.items()},
         "sparse_cluster_max": {k: (round(v, 6) if isinstance(v, float) else v)
@@ -407,6 +411,15 @@ def gpu_arm(args, world, rank, local):
         td.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def decode_launches_per_call(rep, device):
+    """Kernels one kvq_decode_attn call with an output launches: the decode kernel, plus the
+    combine kernel when the request has more (split, sequence, KV head) units than CTAs
+    that run at once (one per SM), as the library decides."""
+    import torch
+    units = rep.wl.batch * rep.wl.num_kv_heads * -(-max(rep.max_seq, 1) // rep.L)
+    return 1 if units <= torch.cuda.get_device_properties(device).multi_processor_count else 2
 
 
 def e2e_arm(args, rep, wl, inp, device, world):
@@ -462,7 +475,7 @@ def e2e_arm(args, rep, wl, inp, device, world):
             "how": "public API per step: H2D(q, k, v) + QuantizedKVCache.write + .attention + "
                    "D2H(out), captured as one CUDA graph per cache copy and replayed",
             "eager_value": per(el_eager),
-            "gpu_launches_per_step": 2}
+            "gpu_launches_per_step": 1 + decode_launches_per_call(rep, device)}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)

@@ -230,12 +230,14 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                rows copied, unless V tiles are copied with K),
  *                [3] V rows skipped
  *   out          device fp32 [batch][num_q_heads][head_dim], 16-byte aligned, or NULL.
- *                When given, the same kernel also merges the splits and writes the
- *                output (the log-sum-exp rule of kvq_combine): when every split of the
- *                request runs on its own CTA at once, each split adds its normalized
- *                share into the output with floating-point atomics (so the last bits of
- *                the output may differ from run to run); otherwise the last cluster to
- *                finish a (sequence, KV head) merges it.  Calls that share a workspace
+ *                When given, the call also merges the splits and writes the output (the
+ *                log-sum-exp rule of kvq_combine): when every split of the request runs
+ *                on its own CTA at once, inside the decode kernel, each split adding its
+ *                normalized share into the output with floating-point atomics (so the
+ *                last bits of the output may differ from run to run); with
+ *                KVQ_OPT_SHARED_MAX, inside the kernel too, the last cluster to finish a
+ *                (sequence, KV head) merging it; otherwise by a second launch on the same
+ *                stream, the combine kernel of kvq_combine.  Calls that share a workspace
  *                must not overlap on the GPU.
  * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
  * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.

@@ -293,7 +293,17 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.v_early = (options & KVQ_OPT_V_WITH_K)      ? 1
               : (options & KVQ_OPT_V_KEPT_ONLY) ? 0
                                                 : desc->fmt != KVQ_FMT_NVFP4;
-  return launch_decode(a, static_cast<cudaStream_t>(stream));
+  // The merge: inside the decode kernel when every split has its own CTA (the splits add
+  // their shares) or splits share a cluster (the cluster merges, the last one to finish
+  // a (sequence, KV head) merges the clusters' partials); otherwise the partials go to the
+  // workspace and the combine kernel merges them, one CTA per (sequence, query head),
+  // which measured faster than the last finisher of each (sequence, KV head) merging alone.
+  const bool combine_after = out && CS == 1 && groups > capacity;
+  if (combine_after) a.out = nullptr;
+  st = launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (st != KVQ_OK || !combine_after) return st;
+  return launch_combine(*desc, workspace, batch, num_q_heads, max_seq_len, L, CS, a.max_splits, seq_lens,
+                        out, static_cast<cudaStream_t>(stream));
 }
 
 int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,

@@ -135,13 +135,15 @@ def test_combine_kernel_matches_in_kernel_merge(name, tau):
     assert np.max(np.abs(g1["out"] - g2["out"])) <= 1e-5 * vmax
 
 
-def test_in_kernel_merge_resets_its_counters():
-    # back-to-back calls on one workspace: each must merge exactly once (the additive
-    # merge may change the last bits from run to run)
+@pytest.mark.parametrize("scope", ["split", "cluster"])
+def test_in_kernel_merge_resets_its_counters(scope):
+    # back-to-back multi-round calls on one workspace: each must merge exactly once (the
+    # clusters' last finisher counts arrivals in the workspace; split scope merges with the
+    # combine kernel after the decode; the additive merge may change the last bits)
     import quantized_kv_cache_split_b200 as K
     wl = W.shrink(W.WORKLOADS["paged_b8_q4"], [3000, 64, 0, 1500, 777], n_planted=8)
     inp = W.generate(wl)
-    g = run_library(inp, 1e-6, 128)
+    g = run_library(inp, 1e-6, 128, max_scope=scope)
     cache = g["cache"]
     dev = torch.device("cuda")
     q = torch.from_numpy(inp.q).to(dev)
@@ -151,7 +153,8 @@ def test_in_kernel_merge_resets_its_counters():
     for _ in range(3):
         o = torch.full((wl.batch, wl.num_q_heads, wl.head_dim), float("nan"), device=dev)
         cache.attention(q, seq, int(inp.seq_lens.max()), pt, inp.max_pages, tau=1e-6,
-                        sm_scale=float(np.float32(1 / math.sqrt(128))), split_tokens=128, out=o)
+                        sm_scale=float(np.float32(1 / math.sqrt(128))), split_tokens=128, out=o,
+                        max_scope=scope)
         outs.append(o.cpu().numpy())
     assert not np.isnan(outs[0]).any()
     vmax = float(np.abs(inp.v.astype(np.float32)).max())
@@ -265,8 +268,9 @@ def test_decode_parity_head_dim_64_and_groups(fmt, hq, hkv):
                                           seq_lens=(777, 300), batch=2, n_planted=6)
     inp = W.generate(wl)
     cb = codebook_for(64) if fmt == "lut4" else None
-    for tau, split in [(1e-6, 0), (0.0, 64)]:
-        g = run_library(inp, tau, split, cb)
+    # the library's V fetch, both explicit policies (tau > 0), and dense
+    for tau, split, v_fetch in [(1e-6, 0, "auto"), (1e-6, 0, "kept"), (1e-4, 128, "with_k"), (0.0, 64, "auto")]:
+        g = run_library(inp, tau, split, cb, v_fetch=v_fetch)
         o = run_oracle(inp, tau, g["split"], cb)
         check_parity(inp, g, o, tau)
 

@@ -630,22 +630,21 @@ __device__ __forceinline__ int swz(int row) {
   return (row >> C::SWZ_SHIFT) & C::SWZ_MASK;
 }
 
-// Stage the whole 64-row V tile that starts at plane row row0: codes swizzled, then the
-// scale rows (one copy group).
+// Stage the V rows row0 .. row0 + rows - 1 of a tile (rows = 64, or 32 for a half tile):
+// codes swizzled, then the scale rows (one copy group).
 template <int FMT, int D>
 __device__ __forceinline__ void copy_v_tile(uint8_t* dst, const uint8_t* vcodes, const uint8_t* vscales,
-                                            size_t row0, int lane) {
+                                            size_t row0, int rows, int lane) {
   using C = Cfg<FMT, D>;
   constexpr int CPR = C::CROW / 16;
   const uint8_t* src = vcodes + row0 * C::CROW;
 #pragma unroll 4
-  for (int i = lane; i < kTile * CPR; i += 32) {
+  for (int i = lane; i < rows * CPR; i += 32) {
     const int row = i / CPR, cc = i % CPR;
     cp_async16(dst + row * C::CROW + ((cc ^ swz<FMT, D>(row)) << 4), src + (size_t)row * C::CROW + cc * 16);
   }
   const uint8_t* ssrc = vscales + row0 * C::SROW;
-#pragma unroll
-  for (int i = lane; i < C::STAGE_SC / 16; i += 32) cp_async16(dst + C::STAGE_CODE + i * 16, ssrc + i * 16);
+  for (int i = lane; i < rows * C::SROW / 16; i += 32) cp_async16(dst + C::STAGE_CODE + i * 16, ssrc + i * 16);
   cp_async_commit();
 }
 
@@ -994,6 +993,19 @@ decode_kernel(const DecodeArgs a) {
 
   // after the first round, batches of up to 32 sequences take the existing units evenly
   const bool dense = B <= 32 && total > ncl;
+  // Positions [seg0, seg0 + seg_len) of each split are this warp's: tile w for warp w.  A
+  // split of kWarps - 2 tiles leaves two warps idle; for lut4 and nvfp4 its last two tiles
+  // are then halved with them, so that each SM sub-partition (warp w runs on w % 4) holds
+  // 3.5 tiles of the K and V passes instead of 4 on two of them and 3 on the others.
+  // (Measured: this pays where the V pass dequantizes on the ALU; the q8_0 / q4_0 kernels,
+  // whose V codes go to the MMA nearly as loaded, lose more to the extra live registers.)
+  constexpr bool kHalfTiles = !C::kMag;
+  const bool halves = kHalfTiles && Ls == (kWarps - 2) * kTile;
+  int seg0 = warp * kTile, seg_len = kTile;
+  if (halves && warp >= kWarps - 4) {
+    seg_len = kTile / 2;
+    if (warp >= kWarps - 2) seg0 = (warp - 2) * kTile + kTile / 2;
+  }
   UnitCursor ucur{ncl / (B * hkv), 0};
 #pragma unroll 1
   for (int k = 0;; ++k) {
@@ -1032,9 +1044,9 @@ decode_kernel(const DecodeArgs a) {
 
     // ---- K fetch (and, when V is fetched early, the V tile): one copy group per 16-row job
     int row0 = -1;
-    const int ncopy = min(kTile, avail - t0 - warp * kTile);
+    const int ncopy = min(seg_len, avail - t0 - seg0);
     if (ncopy > 0) {
-      const int tok0 = t0 + warp * kTile;
+      const int tok0 = t0 + seg0;
       const int lp = tok0 / P, off = tok0 - lp * P;  // tiles never straddle pages (P % 64 == 0)
       const int page = a.page_table ? __ldg(a.page_table + (size_t)b * a.max_pages + lp)
                                     : b * a.max_pages + lp;
@@ -1045,18 +1057,20 @@ decode_kernel(const DecodeArgs a) {
         const uint8_t* ssrc = kscales + (size_t)row0 * C::SROW;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+          if (16 * j < seg_len) {  // a half tile copies two jobs; every warp commits four groups
 #pragma unroll
-          for (int i = lane; i < 16 * CPR; i += 32) {
-            const int row = 16 * j + i / CPR, cc = i % CPR;
-            const int sw = cc ^ ((row >> C::SWZ_SHIFT) & C::SWZ_MASK);
-            cp_async16(kbuf + row * C::CROW + (sw << 4), src + (size_t)row * C::CROW + cc * 16);
+            for (int i = lane; i < 16 * CPR; i += 32) {
+              const int row = 16 * j + i / CPR, cc = i % CPR;
+              const int sw = cc ^ ((row >> C::SWZ_SHIFT) & C::SWZ_MASK);
+              cp_async16(kbuf + row * C::CROW + (sw << 4), src + (size_t)row * C::CROW + cc * 16);
+            }
+            if (lane < C::SROW)  // 16 rows of scales = SROW 16-byte chunks
+              cp_async16(kbuf + C::STAGE_CODE + 16 * j * C::SROW + lane * 16,
+                         ssrc + 16 * j * C::SROW + lane * 16);
           }
-          if (lane < C::SROW)  // 16 rows of scales = SROW 16-byte chunks
-            cp_async16(kbuf + C::STAGE_CODE + 16 * j * C::SROW + lane * 16,
-                       ssrc + 16 * j * C::SROW + lane * 16);
           cp_async_commit();
         }
-        if (prefetch_v) copy_v_tile<FMT, D>(vtile, vcodes, vscales, (size_t)row0, lane);
+        if (prefetch_v) copy_v_tile<FMT, D>(vtile, vcodes, vscales, (size_t)row0, seg_len, lane);
       }
     }
     if (k == 0) {
@@ -1092,7 +1106,7 @@ decode_kernel(const DecodeArgs a) {
       continue;
     }
     const int n_tok = max(0, min(Ls, nb - t0));
-    int nvalid = min(kTile, n_tok - warp * kTile);  // positions of this warp's tile
+    int nvalid = min(seg_len, n_tok - seg0);  // positions of this warp's tile
     if (nvalid > 0 && row0 < 0) {
       if (lane == 0) set_flag(flags, KVQ_FLAG_BAD_PAGE);
       nvalid = 0;
@@ -1254,7 +1268,7 @@ decode_kernel(const DecodeArgs a) {
                           __all_sync(0xffffffffu, (!hl0 || mn0 - mh0 >= thr) && (!hl1 || mn1 - mh1 >= thr));
     if (all_kept && !prefetch_v) {
       __syncwarp();  // every lane is done reading the K tile
-      copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, lane);
+      copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, seg_len, lane);
     }
     // the weights 2^(s - m) of every valid pair also give the denominator l
     int nkept = 0, nskip = 0;
@@ -1360,7 +1374,7 @@ decode_kernel(const DecodeArgs a) {
         uint8_t* vt = prefetch_v ? vtile : kbuf;
         if (!prefetch_v && !all_kept) {
           __syncwarp();  // every lane is done reading the K tile
-          copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, lane);
+          copy_v_tile<FMT, D>(kbuf, vcodes, vscales, (size_t)row0, seg_len, lane);
         }
         cp_async_wait<0>();
         __syncwarp();
@@ -1443,7 +1457,7 @@ decode_kernel(const DecodeArgs a) {
       // split of this (sequence, KV head) to publish, and computes this split's share of
       // each head, 2^(m_s - M) / L.
       int first = 0;
-      if (n_tok <= (kWarps - 1) * kTile) {
+      if (!halves && n_tok <= (kWarps - 1) * kTile) {
         first = warp == kWarps - 1;
       } else {
         if (lane == 0) first = atomicAdd(&misc[2], 1) == 0;

@@ -231,8 +231,9 @@ RAGGED_LENS = [1000, 70, 1, 0, 2049, 64, 130, 3001]
 @pytest.mark.parametrize("fmt", ["q8_0", "q4_0", "lut4", "nvfp4"])
 @pytest.mark.parametrize("tau,split,scope", [(0.0, 128, "split"), (1e-6, 0, "split"), (1e-4, 192, "split"),
                                              (1e-6, 1024, "split"), (1e-6, 128, "cluster"),
-                                             (1e-6, 0, "sequence")])
+                                             (1e-6, 0, "sequence"), (1e-6, 896, "split"), (0.0, 896, "split")])
 def test_decode_parity_paged_ragged(fmt, tau, split, scope):
+    # split 896 = 14 tiles: the last two tiles are halved between four warps
     base = W.WORKLOADS["paged_b8_q4"].with_(fmt=fmt)
     wl = W.shrink(base, RAGGED_LENS, n_planted=8)
     inp = W.generate(wl)

@@ -166,7 +166,7 @@ def measured_peaks():
 class Replicas:
     """R copies of the quantized cache so that successive steps miss in L2."""
 
-    def __init__(self, wl: W.Workload, inp: W.Inputs, device, min_bytes: int):
+    def __init__(self, wl: W.Workload, inp: W.Inputs, device, min_bytes: int, split_tokens: int = 0):
         import torch
         import quantized_kv_cache_split_b200 as K
         self.wl, self.inp = wl, inp
@@ -202,7 +202,7 @@ class Replicas:
         self.B, self.Hq, self.D = wl.batch, wl.num_q_heads, D
         # the schedule: L positions per split; the shared-maximum option runs clusters of
         # CS splits (its own L and CS)
-        self.L = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, 0)
+        self.L = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, split_tokens)
         self.L_sh = K.kvq_resolve_split(first.desc, self.B, self.Hq, self.max_seq, 0,
                                         K.KVQ_OPT_SHARED_MAX)
         self.CS_sh = K.kvq_resolve_cluster(first.desc, self.B, self.Hq, self.max_seq, 0,
@@ -314,7 +314,7 @@ def gpu_arm(args, world, rank, local):
     init_dist(world, "nccl")
     wl = W.WORKLOADS[args.workload]
     inp = W.generate(wl)
-    rep = Replicas(wl, inp, device, 3 * L2_BYTES)
+    rep = Replicas(wl, inp, device, 3 * L2_BYTES, args.split_tokens)
     def n_partials(L, CS):
         return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
 
@@ -560,6 +560,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=120.0)
     ap.add_argument("--skip-e2e", action="store_true", help="(profiling runs) skip the e2e leg")
+    ap.add_argument("--split-tokens", type=int, default=0,
+                    help="positions per split (0: the library's choice, kvq_resolve_split)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -234,10 +234,11 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                log-sum-exp rule of kvq_combine): when every split of the request runs
  *                on its own CTA at once, inside the decode kernel, each split adding its
  *                normalized share into the output with floating-point atomics (so the
- *                last bits of the output may differ from run to run); with
- *                KVQ_OPT_SHARED_MAX, inside the kernel too, the last cluster to finish a
- *                (sequence, KV head) merging it; otherwise by a second launch on the same
- *                stream, the combine kernel of kvq_combine.  Calls that share a workspace
+ *                last bits of the output may differ from run to run); otherwise, with
+ *                clusters of splits (KVQ_OPT_SHARED_MAX and kvq_resolve_cluster > 1),
+ *                inside the kernel too, the last cluster to finish a (sequence, KV head)
+ *                merging it; otherwise by a second launch on the same stream, the
+ *                combine kernel of kvq_combine.  Calls that share a workspace
  *                must not overlap on the GPU.
  * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
  * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.

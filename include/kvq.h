@@ -94,7 +94,7 @@ extern "C" {
 #define KVQ_FLAG_BAD_SEQLEN   2u  /* seq_len < 0, > max_seq_len or > max_pages*page_size */
 #define KVQ_FLAG_TIMEOUT      4u  /* a bounded wait (cross-CTA exchange, flag) gave up */
 
-/* Limits of this build. */
+/* Compile-time limits of the library. */
 #define KVQ_MAX_GROUP        8     /* query heads per KV head (num_q_heads / num_kv_heads) */
 #define KVQ_MAX_SPLIT_TOKENS 1024  /* positions per split-KV work unit */
 #define KVQ_MAX_BATCH        1024

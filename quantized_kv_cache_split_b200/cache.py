@@ -89,12 +89,18 @@ class QuantizedKVCache:
         "kept" (only the kept rows, after the skip test), "with_k" (every V tile with its
         K tile; skipped rows are left out of the contraction only) or "auto" (with_k,
         except nvfp4: kept); the result is the same."""
+        scopes = {"split": 0, "cluster": kb.KVQ_OPT_SHARED_MAX, "sequence": kb.KVQ_OPT_GLOBAL_MAX}
+        fetches = {"auto": 0, "kept": kb.KVQ_OPT_V_KEPT_ONLY, "with_k": kb.KVQ_OPT_V_WITH_K}
+        if max_scope not in scopes:
+            raise ValueError(f"max_scope must be one of {sorted(scopes)}, not {max_scope!r}")
+        if v_fetch not in fetches:
+            raise ValueError(f"v_fetch must be one of {sorted(fetches)}, not {v_fetch!r}")
         B, Hq, D = q.shape
         if sm_scale is None:
             sm_scale = 1.0 / math.sqrt(D)
-        opts = {"split": 0, "cluster": kb.KVQ_OPT_SHARED_MAX, "sequence": kb.KVQ_OPT_GLOBAL_MAX}[max_scope]
+        opts = scopes[max_scope]
         ws, nbytes, L = self.workspace(B, Hq, max_seq_len, split_tokens, opts)
-        opts |= {"auto": 0, "kept": kb.KVQ_OPT_V_KEPT_ONLY, "with_k": kb.KVQ_OPT_V_WITH_K}[v_fetch]
+        opts |= fetches[v_fetch]
         if out is None:
             out = torch.empty((B, Hq, D), dtype=torch.float32, device=self.device)
         kb.kvq_decode_attn(self.desc, q, B, Hq, self.k_codes, self.k_scales, self.v_codes,

@@ -174,3 +174,15 @@ def test_product_code_never_imports_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle", text, re.M), f
                 assert "oracle/" not in text, f
+
+
+def test_cache_attention_rejects_unknown_scope_and_fetch_policy():
+    # checked before any device call: a CPU-resident cache is enough
+    import torch
+    cache = K.QuantizedKVCache("q4_0", 128, 4, 64, 2, "cpu")
+    q = torch.zeros((1, 32, 128), dtype=torch.float16)
+    lens = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="max_scope"):
+        cache.attention(q, lens, 64, max_scope="global")
+    with pytest.raises(ValueError, match="v_fetch"):
+        cache.attention(q, lens, 64, v_fetch="all")

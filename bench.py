@@ -2,14 +2,19 @@
 sparse V dequantization, on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload gqa_32k_q4] [--tau 1e-6]
+                    [--workload gqa_32k_q4] [--tau 1e-6] [--headline-only]
 
 One step = the whole decode-attention hot path for one decode token of every
-sequence in the workload: one split-KV decode launch (K tiles -> scores -> running
-max -> skip decision -> kept V only -> cluster merge -> log-sum-exp merge of the
-partials by the last cluster of each (sequence, KV head)).  Inputs are resident
-in HBM; the cache is replicated into enough copies that successive steps rotate
-through more than 3x the L2 size, so every step reads HBM.  Prints one JSON line.
+sequence in the workload: one kvq_decode_attn call (K tiles -> scores -> running
+maximum -> skip decision -> V of the kept rows -> merge of the splits into the
+output).  Inputs are resident in HBM; the cache is replicated into enough copies
+that successive steps rotate through more than 3x the L2 size, so every step
+reads HBM.  The W warm-up steps and the K timed steps are each captured as one
+CUDA graph; the timed region is one replay, bracketed by CUDA events.  Prints one
+JSON line: the headline workload (every variant of the skip test and V fetch, the
+two-launch path, the end-to-end path through the Python API with host buffers),
+then, unless --headline-only, a table of every workload (dense and sparse at each
+of its tau values).
 
 --impl reference times the fp64 CPU oracle (the only reference available for
 this method) on bounded samples of the same workload.
@@ -234,12 +239,14 @@ class Replicas:
 
 
 def capture(fn, n_steps, start):
+    """One CUDA graph holding steps start .. start + n_steps - 1 of ``fn`` (each step
+    launched once before the capture, so host-side first-call paths are warm)."""
     import torch
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for i in range(n_steps):       # warm the capture-time host paths once
+        for i in range(n_steps):
             fn(start + i)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
@@ -249,36 +256,30 @@ def capture(fn, n_steps, start):
     return g
 
 
-class GraphRunner:
-    """Launch exactly n steps of `fn` through CUDA graphs: one graph of R steps
-    (copies 0..R-1) plus single-step graphs for the remainder."""
+class StepGraphs:
+    """The warm-up steps 0 .. warmup - 1 and the timed steps warmup .. warmup + steps - 1
+    of ``fn`` (step i works on cache copy i % R inside ``fn``), each captured as ONE
+    graph, so the timed region is a single replay of exactly ``steps`` launches of the
+    hot path whatever ``steps`` is."""
 
-    def __init__(self, fn, R):
-        self.R = R
-        self.full = capture(fn, R, 0)
-        self.single = [capture(fn, 1, i) for i in range(R)]
-
-    def run(self, n, offset=0):
-        """Steps offset .. offset + n - 1 (copy index = step % R)."""
-        i = offset
-        while i % self.R and n:
-            self.single[i % self.R].replay(); i += 1; n -= 1
-        while n >= self.R:
-            self.full.replay(); i += self.R; n -= self.R
-        while n:
-            self.single[i % self.R].replay(); i += 1; n -= 1
+    def __init__(self, fn, steps, warmup, capture_fn=capture):
+        self.steps, self.warmup = steps, warmup
+        self.warm = capture_fn(fn, warmup, 0)
+        self.timed = capture_fn(fn, steps, warmup)
 
 
-def time_steps(runner, steps, warmup, world, sampler=None):
+def time_steps(graphs: StepGraphs, world, sampler=None):
+    """Replay the warm-up graph, then time one replay of the timed graph with CUDA
+    events on the current stream (barrier and synchronize on both sides); ms."""
     import torch
-    runner.run(warmup, 0)
+    graphs.warm.replay()
     torch.cuda.synchronize()
     barrier(world)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if sampler:
         sampler.start()
     start.record()
-    runner.run(steps, warmup)
+    graphs.timed.replay()
     end.record()
     torch.cuda.synchronize()
     if sampler:
@@ -306,6 +307,76 @@ def algorithmic_bytes(rep: Replicas, v_rows_read: int, n_partials: int, with_o: 
     return k_bytes + v_bytes + q_bytes + pt_bytes + part_bytes + out_bytes
 
 
+def _round(d):
+    return {k: (round(v, 6) if isinstance(v, float) else v) for k, v in d.items()}
+
+
+def n_partials(wl, inp, L, CS):
+    return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
+
+
+def measure_variant(rep, args, world, device, tau, scope, v_opt, hbm_peak, sampler=None,
+                    traffic_key=None):
+    """Counters of one launch, then the timed graph of args.steps launches; one dict per
+    variant (absent keys: the variant is unsupported for this request)."""
+    import torch
+    import quantized_kv_cache_split_b200 as K
+    wl, inp = rep.wl, rep.inp
+    st = torch.zeros(4, dtype=torch.int64, device=device)
+    try:
+        rep.decode(0, tau, st, scope=scope, v_opt=v_opt)
+        torch.cuda.synchronize()
+    except K.KvqError as e:  # e.g. the sequence-wide maximum needs every split on its own CTA
+        return {"tau": tau, "max_scope": scope, "unavailable": str(e)}
+    st = [int(x) for x in st.cpu()]
+    graphs = StepGraphs(lambda i: rep.decode(i, tau, scope=scope, v_opt=v_opt), args.steps,
+                        args.warmup)
+    ms = reduce_max(time_steps(graphs, world, sampler), world, device)
+    del graphs
+    launches = decode_launches_per_call(rep, device)
+    abytes = algorithmic_bytes(rep, st[2], n_partials(wl, inp, rep.L_sh, rep.CS_sh) if scope == "cluster"
+                               else n_partials(wl, inp, rep.L, 1),
+                               with_o=scope == "cluster" or launches == 2)
+    us_step = ms * 1e3 / args.steps
+    achieved = abytes / (us_step * 1e-6) / 1e9
+    return dict(tau=tau, max_scope=scope,
+                v_fetch={0: "auto", K.KVQ_OPT_V_KEPT_ONLY: "kept_only", K.KVQ_OPT_V_WITH_K: "with_k"}[v_opt],
+                ms_per_step=ms / args.steps, us_per_token=us_step / (wl.batch * world),
+                us_per_step=us_step, tokens_per_s=wl.batch * world / (us_step * 1e-6),
+                algorithmic_bytes=abytes, achieved_gbs=achieved, frac=achieved / hbm_peak,
+                skipped_pair_frac=st[1] / max(st[0], 1), v_rows_read=st[2], v_rows_skipped=st[3],
+                launches_per_step=launches,
+                traffic=traffic_from_profile(traffic_key) if traffic_key else None)
+
+
+def workload_table(args, world, device, name, hbm_peak):
+    """Dense and sparse (every tau of the workload), with the library's default V fetch,
+    plus the sequence-wide maximum and the two V fetch policies at args.tau."""
+    import torch
+    import quantized_kv_cache_split_b200 as K
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl)
+    rep = Replicas(wl, inp, device, 3 * L2_BYTES, 0)
+    res = {"config": {"batch": wl.batch, "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
+                      "head_dim": wl.head_dim, "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
+                      "cache_format": wl.fmt, "split_tokens": rep.L, "copies": rep.R,
+                      "l2_cold": rep.l2_cold}}
+    taus = sorted(set(wl.taus) | {0.0, args.tau})
+    for tau in taus:
+        tag = "dense" if tau == 0.0 else f"sparse_tau_{tau:g}"
+        res[tag] = _round(measure_variant(rep, args, world, device, tau, "split", 0, hbm_peak))
+    for tag, scope, v_opt in (("sparse_sequence_max", "sequence", 0),
+                              ("sparse_v_kept_only", "split", K.KVQ_OPT_V_KEPT_ONLY),
+                              ("sparse_v_with_k", "split", K.KVQ_OPT_V_WITH_K)):
+        res[tag] = _round(measure_variant(rep, args, world, device, args.tau, scope, v_opt, hbm_peak))
+    sp, de = res.get(f"sparse_tau_{args.tau:g}", {}), res["dense"]
+    if "us_per_step" in sp and "us_per_step" in de:
+        res["sparse_speedup_vs_dense"] = round(de["us_per_step"] / sp["us_per_step"], 4)
+    del rep
+    torch.cuda.empty_cache()
+    return res
+
+
 def gpu_arm(args, world, rank, local):
     import torch
     import quantized_kv_cache_split_b200 as K
@@ -315,56 +386,26 @@ def gpu_arm(args, world, rank, local):
     wl = W.WORKLOADS[args.workload]
     inp = W.generate(wl)
     rep = Replicas(wl, inp, device, 3 * L2_BYTES, args.split_tokens)
-    def n_partials(L, CS):
-        return sum(wl.num_kv_heads * (((int(n) + L - 1) // L + CS - 1) // CS) for n in inp.seq_lens)
-
-    def counters(tau, scope, v_opt):
-        st = torch.zeros(4, dtype=torch.int64, device=device)
-        rep.decode(0, tau, st, scope=scope, v_opt=v_opt)
-        torch.cuda.synchronize()
-        return [int(x) for x in st.cpu()]
-
-    res = {}
     hbm_peak, peak_kind = measured_peaks()
     sampler = ClockSampler(local)
-    # the headline leaves the V fetch to the library (V with K; nvfp4: kept rows only);
-    # the two policies are also timed on their own
+    # the headline leaves the V fetch to the library; the other variants are context
     variants = (("sparse", args.tau, "split", 0), ("dense", 0.0, "split", 0),
                 ("sparse_v_kept_only", args.tau, "split", K.KVQ_OPT_V_KEPT_ONLY),
                 ("sparse_v_with_k", args.tau, "split", K.KVQ_OPT_V_WITH_K),
                 ("sparse_cluster_max", args.tau, "cluster", 0), ("sparse_sequence_max", args.tau, "sequence", 0),
                 ("sparse_sequence_max_v_kept_only", args.tau, "sequence", K.KVQ_OPT_V_KEPT_ONLY))
+    res = {}
     for tag, tau, scope, v_opt in variants:
-        try:
-            st = counters(tau, scope, v_opt)
-        except K.KvqError as e:  # the sequence-wide maximum needs every split on its own CTA
-            res[tag] = {"max_scope": scope, "unavailable": str(e)}
-            continue
-        step = GraphRunner(lambda i: rep.decode(i, tau, scope=scope, v_opt=v_opt), rep.R)
-        ms_step = reduce_max(time_steps(step, args.steps, args.warmup, world,
-                                        sampler if tag == "sparse" else None), world, device)
-        # o partials cross HBM when clusters merge them or the combine kernel does
-        abytes = algorithmic_bytes(rep, st[2], n_partials(rep.L_sh, rep.CS_sh) if scope == "cluster"
-                                   else n_partials(rep.L, 1),
-                                   with_o=scope == "cluster" or decode_launches_per_call(rep, device) == 2)
-        us_launch = ms_step * 1e3 / args.steps
-        achieved = abytes / (us_launch * 1e-6) / 1e9
-        res[tag] = dict(tau=tau, max_scope=scope, v_fetch={0: "auto", K.KVQ_OPT_V_KEPT_ONLY: "kept_only",
-                                                           K.KVQ_OPT_V_WITH_K: "with_k"}[v_opt],
-                        ms_per_step=ms_step / args.steps,
-                        us_per_token=ms_step * 1e3 / args.steps / (wl.batch * world),
-                        us_per_launch=us_launch, algorithmic_bytes=abytes,
-                        achieved_gbs=achieved, frac=achieved / hbm_peak,
-                        skipped_pair_frac=st[1] / max(st[0], 1),
-                        v_rows_read=st[2], v_rows_skipped=st[3],
-                        traffic=traffic_from_profile(f"{args.workload}:{tag}"))
-        del step
+        res[tag] = measure_variant(rep, args, world, device, tau, scope, v_opt, hbm_peak,
+                                   sampler if tag == "sparse" else None,
+                                   traffic_key=f"{args.workload}:{tag}")
     # the two-launch path (partials, then kvq_combine) for comparison
-    two = GraphRunner(lambda i: (rep.decode(i, args.tau, fused=False), rep.combine(i)), rep.R)
-    ms_two = reduce_max(time_steps(two, args.steps, args.warmup, world), world, device)
+    two = StepGraphs(lambda i: (rep.decode(i, args.tau, fused=False), rep.combine(i)), args.steps, args.warmup)
+    ms_two = reduce_max(time_steps(two, world), world, device)
     del two
     e2e = None if args.skip_e2e else e2e_arm(args, rep, wl, inp, device, world)
     sp = res["sparse"]
+    launches = decode_launches_per_call(rep, device)
     line = {
         "metric": METRIC, "value": round(sp["us_per_token"], 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sp["ms_per_step"], 6),
@@ -374,43 +415,47 @@ def gpu_arm(args, world, rank, local):
                    "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                    "context": list(wl.seq_lens) if wl.batch > 1 else wl.seq_lens[0],
                    "cache_format": wl.fmt, "tau": args.tau, "split_tokens": rep.L,
-                   "v_fetch": "library's choice: V tiles with K (nvfp4: kept rows only)",
+                   "v_fetch": V_FETCH_DEFAULT,
                    "cluster_max_schedule": {"split_tokens": rep.L_sh, "splits_per_cluster": rep.CS_sh},
                    "l2": (f"inputs rotate over {rep.R} cache copies "
                           f"({rep.R * rep.plane_bytes / 2**20:.0f} MiB > 3x L2)" if rep.l2_cold else
                           f"inputs rotate over {rep.R} cache copies "
                           f"({rep.R * rep.plane_bytes / 2**20:.1f} MiB < L2: timed with the cache in L2)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "step": ("one kvq_decode_attn call (CUDA graph): "
-                            + ("one launch, merge in the kernel" if decode_launches_per_call(rep, device) == 1
+                   "timing": (f"warm-up and timed steps each one CUDA graph ({args.warmup} and "
+                              f"{args.steps} kvq_decode_attn calls), CUDA events around one replay"),
+                   "step": ("one kvq_decode_attn call: "
+                            + ("one launch, merge in the kernel" if launches == 1
                                else "decode launch + combine launch"))},
         "roofline": {"bound": "hbm", "achieved": round(sp["achieved_gbs"], 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(sp["frac"], 4),
                      "traffic": sp["traffic"], "peak_kind": peak_kind,
-                     "kernel": f"decode_kernel<{wl.fmt},{wl.head_dim}>",
+                     "kernel": f"decode kernel <{wl.fmt},{wl.head_dim}>",
                      "algorithmic_bytes_per_launch": sp["algorithmic_bytes"],
-                     "us_per_launch": round(sp["us_per_launch"], 3)},
+                     "us_per_launch": round(sp["us_per_step"] / launches, 3)},
         "e2e": e2e,
-        "gpu_launches": args.steps * decode_launches_per_call(rep, device),
-        "dense": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res["dense"].items()},
-        "sparse": {k: (round(v, 6) if isinstance(v, float) else v) for k, v in sp.items()},
-        "sparse_cluster_max": {k: (round(v, 6) if isinstance(v, float) else v)
-                               for k, v in res["sparse_cluster_max"].items()},
-        "sparse_sequence_max": {k: (round(v, 6) if isinstance(v, float) else v)
-                                for k, v in res["sparse_sequence_max"].items()},
-        **{tag: {k: (round(v, 6) if isinstance(v, float) else v) for k, v in res[tag].items()}
-           for tag in ("sparse_v_kept_only", "sparse_v_with_k", "sparse_sequence_max_v_kept_only")},
+        "gpu_launches": args.steps * launches,
+        **{tag: _round(v) for tag, v in res.items()},
         "two_launch_us_per_token": round(ms_two * 1e3 / args.steps / (wl.batch * world), 4),
         "clocks": sampler.report(),
     }
+    head_L = rep.L
+    del rep
+    torch.cuda.empty_cache()
+    if args.all_workloads:
+        line["workloads"] = {name: workload_table(args, world, device, name, hbm_peak)
+                             for name in W.WORKLOADS}
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        line["cpu_baseline"] = cpu_baseline(wl, inp, rep.L, args.tau, budget_s=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wl, inp, head_L, args.tau, budget_s=args.cpu_seconds)
     if world > 1:
         import torch.distributed as td
         td.barrier()
         td.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+V_FETCH_DEFAULT = "library's choice (kvq.h: KVQ_OPT_V_KEPT_ONLY / KVQ_OPT_V_WITH_K)"
 
 
 def decode_launches_per_call(rep, device):
@@ -428,7 +473,8 @@ def e2e_arm(args, rep, wl, inp, device, world):
     cache (kvq_quantize_kv), runs the decode (with its in-kernel merge) and reads the
     output back to pinned host memory.  The step is captured once per cache copy as a
     CUDA graph of those public-API calls (how a serving loop issues it) and replayed;
-    the eager form (every call from Python each step) is reported beside it."""
+    the eager form (every call from Python each step) is reported beside it, and the
+    dense (tau = 0) path is timed the same way."""
     import torch
     B, Hq, Hkv, D = wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     nq, nkv = B * Hq * D, B * Hkv * D
@@ -444,13 +490,15 @@ def e2e_arm(args, rep, wl, inp, device, world):
     d_v = d_in[nq + nkv:].view(B, Hkv, D)
     out = torch.empty((B, Hq, D), dtype=torch.float32, device=device)
 
-    def step(i):
-        c = rep.caches[i % rep.R]
-        d_in.copy_(h_in, non_blocking=True)
-        c.write(d_k, d_v, last)
-        c.attention(d_q, rep.seq, rep.max_seq, rep.pt, inp.max_pages, tau=args.tau,
-                    sm_scale=rep.sm, split_tokens=rep.L, out=out)
-        h_out.copy_(out, non_blocking=True)
+    def make_step(tau):
+        def step(i):
+            c = rep.caches[i % rep.R]
+            d_in.copy_(h_in, non_blocking=True)
+            c.write(d_k, d_v, last)
+            c.attention(d_q, rep.seq, rep.max_seq, rep.pt, inp.max_pages, tau=tau,
+                        sm_scale=rep.sm, split_tokens=rep.L, out=out)
+            h_out.copy_(out, non_blocking=True)
+        return step
 
     def timed(run):
         for i in range(args.warmup):
@@ -463,54 +511,105 @@ def e2e_arm(args, rep, wl, inp, device, world):
         torch.cuda.synchronize()
         return reduce_max(time.perf_counter() - t0, world, device)
 
-    el_eager = timed(step)
-    R = min(rep.R, args.steps)  # one graph per cache copy the timed steps use
-    graphs = [capture(step, 1, i) for i in range(R)]
-    el = timed(lambda i: graphs[i % R].replay())
+    per = lambda e: round(e * 1e6 / args.steps / (B * world), 3)  # noqa: E731
+    res = {}
+    for tag, tau in (("", args.tau), ("dense_", 0.0)):
+        step = make_step(tau)
+        el_eager = timed(step)
+        R = min(rep.R, args.steps + args.warmup)  # one graph per cache copy the steps use
+        graphs = [capture(step, 1, i) for i in range(R)]
+        el = timed(lambda i: graphs[i % R].replay())
+        del graphs
+        res[tag + "value"] = per(el)
+        res[tag + "eager_value"] = per(el_eager)
     bi = h_in.numel() * 2
     bo = h_out.numel() * 4
-    per = lambda e: round(e * 1e6 / args.steps / (B * world), 3)  # noqa: E731
-    return {"value": per(el), "unit": UNIT,
+    return {"value": res["value"], "unit": UNIT,
             "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
             "how": "public API per step: H2D(q, k, v) + QuantizedKVCache.write + .attention + "
-                   "D2H(out), captured as one CUDA graph per cache copy and replayed",
-            "eager_value": per(el_eager),
+                   "D2H(out), captured as one CUDA graph per cache copy and replayed (host-timed)",
+            "eager_value": res["eager_value"],
+            "dense_value": res["dense_value"], "dense_eager_value": res["dense_eager_value"],
             "gpu_launches_per_step": 1 + decode_launches_per_call(rep, device)}
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
 
-def _oracle_sample(wl, inp, split, tau, n_pos):
-    """One bounded sample: the oracle's sparse-V decode for the first KV head of the
-    first sequence, truncated to n_pos positions.  Returns (seconds, fraction of the
-    workload's (position, KV head) units it covers)."""
+def _oracle_group(task):
+    """One (sequence, KV head) group of the oracle's sparse-V decode step, truncated to
+    n_pos positions; runs in a worker process (spawned) or inline.  Returns seconds."""
+    name, b, h, n_pos, split, tau = task
+    from threadpoolctl import threadpool_limits
     from oracle import attention as OA
     from oracle import codebook as OC
+    wl = W.WORKLOADS[name]
+    inp = W.generate(wl) if _GEN.get(name) is None else _GEN[name]
+    _GEN[name] = inp
     cb = OC.lloyd_max_f16(16, 1.0 / math.sqrt(wl.head_dim)) if wl.fmt == "lut4" else None
-    seq = np.array([n_pos], dtype=np.int32)
+    off = int(inp.seq_offsets()[b])
+    n = min(n_pos, int(inp.seq_lens[b]))
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        OA.decode_step(wl.fmt, inp.q[b:b + 1], inp.k[off:off + n], inp.v[off:off + n],
+                       np.array([n], dtype=np.int32), wl.num_kv_heads, 1.0 / math.sqrt(wl.head_dim),
+                       tau, split, signs=inp.signs, codebook16=cb, with_dense=False, groups=[(0, h)])
+        return time.perf_counter() - t0
+
+
+_GEN = {}
+
+
+def _pool(n):
+    import multiprocessing as mp
+    return mp.get_context("spawn").Pool(n)
+
+
+def oracle_all_cores(wl, inp, split, tau, n_pos, pool, workers):
+    """Wall time of the oracle over every (sequence, KV head) group (each truncated to
+    n_pos positions), the groups spread over ``workers`` spawned processes; returns
+    (seconds, fraction of the workload's positions x KV heads covered)."""
+    tasks = [(wl.name, b, h, n_pos, split, tau) for b in range(wl.batch) for h in range(wl.num_kv_heads)]
     t0 = time.perf_counter()
-    OA.decode_step(wl.fmt, inp.q[:1], inp.k[:n_pos], inp.v[:n_pos], seq, wl.num_kv_heads,
-                   1.0 / math.sqrt(wl.head_dim), tau, split, signs=inp.signs, codebook16=cb,
-                   with_dense=False, groups=[(0, 0)])
+    pool.map(_oracle_group, tasks, chunksize=1)
     dt = time.perf_counter() - t0
-    frac = n_pos / (int(inp.seq_lens.sum()) * wl.num_kv_heads)
-    return dt, frac
+    covered = sum(min(n_pos, int(n)) for n in inp.seq_lens) * wl.num_kv_heads
+    return dt, covered / (int(inp.seq_lens.sum()) * wl.num_kv_heads)
 
 
 def cpu_baseline(wl, inp, split, tau, budget_s=15.0):
-    from threadpoolctl import threadpool_limits
+    """The fp64 oracle as it stands on the host cores: one core (one group, repeated for
+    about half the budget) and all cores (every group in parallel over spawned workers)."""
+    _GEN[wl.name] = inp
     n_pos = int(inp.seq_lens[0])
-    with threadpool_limits(limits=1):
-        times, frac = [], None
-        t_end = time.perf_counter() + budget_s
-        while time.perf_counter() < t_end or not times:
-            dt, frac = _oracle_sample(wl, inp, split, tau, n_pos)
-            times.append(dt)
-    us_per_step = statistics.median(times) / frac * 1e6
-    return {"value": round(us_per_step / wl.batch, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+    times = []
+    t_end = time.perf_counter() + budget_s / 2
+    while time.perf_counter() < t_end or not times:
+        times.append(_oracle_group((wl.name, 0, 0, n_pos, split, tau)))
+    frac1 = min(n_pos, int(inp.seq_lens[0])) / (int(inp.seq_lens.sum()) * wl.num_kv_heads)
+    us_1 = statistics.median(times) / frac1 * 1e6 / wl.batch
+    cores = len(os.sched_getaffinity(0))
+    groups = wl.batch * wl.num_kv_heads
+    workers = max(1, min(cores, groups))
+    all_cores = None
+    try:
+        with _pool(workers) as pool:
+            pool.map(_oracle_group, [(wl.name, 0, 0, 64, split, tau)] * workers)  # start-up, not timed
+            reps = []
+            t_end = time.perf_counter() + budget_s / 2
+            while time.perf_counter() < t_end or not reps:
+                dt, fr = oracle_all_cores(wl, inp, split, tau, n_pos, pool, workers)
+                reps.append(dt / fr)
+        all_cores = {"value": round(statistics.median(reps) * 1e6 / wl.batch, 1), "unit": UNIT,
+                     "cores": workers, "host_cores": cores,
+                     "sample": f"every (sequence, KV head) group ({groups}) truncated to {n_pos} positions, "
+                               f"{len(reps)} runs over {workers} spawned worker processes, scaled to the workload"}
+    except Exception as e:  # pragma: no cover - a host without process support
+        all_cores = {"unavailable": str(e)}
+    return {"value": round(us_1, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"fp64 numpy oracle (quantize + dequant + schedule-exact sparse-V attention) "
                       f"on 1 of {wl.num_kv_heads} KV heads x {n_pos} positions, {len(times)} runs, "
-                      f"scaled to the whole workload"}
+                      f"scaled to the whole workload",
+            "all_cores": all_cores}
 
 
 def reference_arm(args, world, rank):
@@ -518,20 +617,23 @@ def reference_arm(args, world, rank):
         return
     wl = W.WORKLOADS[args.workload]
     inp = W.generate(wl)
-    from threadpoolctl import threadpool_limits
-    # size one step so that warmup + steps finish in about args.ref_budget seconds
-    with threadpool_limits(limits=1):
+    _GEN[wl.name] = inp
+    split = 896
+    cores = len(os.sched_getaffinity(0))
+    workers = max(1, min(cores, wl.batch * wl.num_kv_heads))
+    with _pool(workers) as pool:
+        # size one step so that warmup + steps finish in about args.ref_budget seconds
         pilot = 1024
-        dt, _ = _oracle_sample(wl, inp, 896, args.tau, pilot)
+        dt, fr = oracle_all_cores(wl, inp, split, args.tau, pilot, pool, workers)
         per_pos = dt / pilot
-        n_pos = int(args.ref_budget / max(args.steps + args.warmup, 1) / per_pos)
-        n_pos = max(64, min(n_pos, int(inp.seq_lens[0])))
+        n_pos = int(args.ref_budget / max(args.steps + args.warmup, 1) / max(per_pos, 1e-9))
+        n_pos = max(64, min(n_pos, int(inp.seq_lens.max())))
         for _ in range(args.warmup):
-            _oracle_sample(wl, inp, 896, args.tau, n_pos)
+            oracle_all_cores(wl, inp, split, args.tau, n_pos, pool, workers)
         t = []
         frac = None
         for _ in range(args.steps):
-            dt, frac = _oracle_sample(wl, inp, 896, args.tau, n_pos)
+            dt, frac = oracle_all_cores(wl, inp, split, args.tau, n_pos, pool, workers)
             t.append(dt)
     us_step = sum(t) / len(t) / frac * 1e6
     value = us_step / wl.batch
@@ -540,10 +642,11 @@ def reference_arm(args, world, rank):
             "ms_per_step": round(us_step / 1e3, 3), "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "cache_format": wl.fmt, "tau": args.tau,
-                       "split_tokens": 896},
-            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": f"each step: fp64 oracle on 1 KV head x {n_pos} positions, "
-                                       f"scaled to the whole workload"},
+                       "split_tokens": split},
+            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": workers, "kind": "oracle",
+                             "sample": f"each step: fp64 oracle on every (sequence, KV head) group truncated "
+                                       f"to {n_pos} positions over {workers} spawned workers "
+                                       f"({cores} host cores), scaled to the whole workload"},
             "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -552,7 +655,7 @@ def reference_arm(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="gqa_32k_q4", choices=sorted(W.WORKLOADS))
@@ -562,6 +665,8 @@ def main(argv=None):
     ap.add_argument("--skip-e2e", action="store_true", help="(profiling runs) skip the e2e leg")
     ap.add_argument("--split-tokens", type=int, default=0,
                     help="positions per split (0: the library's choice, kvq_resolve_split)")
+    ap.add_argument("--headline-only", dest="all_workloads", action="store_false",
+                    help="(profiling runs) skip the per-workload table of every configuration")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -118,6 +118,9 @@ size_t kvq_scale_row_count(int32_t fmt, int32_t head_dim);
 
 /*
  * kvq_quantize -- write n_tokens K (or V) vectors into a cache plane pair.
+ *   Passage: tproger page, "Почему это работает для любой квантизации" (the q8_0, q4_0 and
+ *   Walsh-Hadamard-rotated codebook KV formats the method runs on) and "Ключевые выводы"
+ *   (NVFP4); the pages fix no block arithmetic, so the formulas above are this library's.
  *   x       device fp16 [n_tokens][num_kv_heads][head_dim]
  *   slots   device int32 [n_tokens]: physical slot of token i (NULL: slot i);
  *           every slot must lie in [0, num_pages*page_size) (not checked on device)
@@ -131,6 +134,7 @@ int kvq_quantize(const kvq_cache_desc* desc, const void* x, int32_t n_tokens,
 
 /*
  * kvq_quantize_kv -- kvq_quantize of the K vectors k into (k_codes, k_scales) and of the
+ *   (Passage: as kvq_quantize.)
  * V vectors v into (v_codes, v_scales), same slots, in one launch (the append of a
  * decode step).  Arguments, layout, results and errors are those of two kvq_quantize
  * calls.
@@ -141,6 +145,8 @@ int kvq_quantize_kv(const kvq_cache_desc* desc, const void* k, const void* v, in
 
 /*
  * kvq_resolve_split -- the split length L (positions per split-KV work unit) that
+ *   (No passage: the pages' kernel walks one sequence; splitting it across SMs is this
+ *   library's schedule, reported so that a checker can replay it.)
  * kvq_decode_attn and kvq_combine use for a request (same split_tokens and
  * options).  split_tokens > 0 is capped at KVQ_MAX_SPLIT_TOKENS and rounded up to a
  * multiple of 64; split_tokens == 0 picks one from the problem size and how many
@@ -188,6 +194,10 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
 
 /*
  * kvq_decode_attn -- split-KV decode attention with sparse V.
+ *   Passage: tproger page, "Решение — не ускорять, а пропускать" (the softmax weights come
+ *   from K before V is touched; a position whose weight is below the threshold, 1e-6 on
+ *   the page, has its V dequantization and accumulation skipped) and "FAQ" (K is always
+ *   dequantized, since it produces the weights).
  *   q            device fp16 [batch][num_q_heads][head_dim], 16-byte aligned
  *   k_codes, k_scales, v_codes, v_scales   device planes (layout above), 16-byte aligned
  *   page_table   device int32 [batch][max_pages] (NULL: sequence b uses pages
@@ -253,6 +263,8 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
 
 /*
  * kvq_combine -- log-sum-exp merge of the partials of kvq_decode_attn (same
+ *   (No passage: the pages' kernel keeps one running softmax per sequence; the merge of
+ *   split-KV partials is the standard log-sum-exp identity written out below.)
  * batch, num_q_heads, max_seq_len, split_tokens, options, seq_lens and workspace), for callers
  * that passed no output pointer to it (or that merge partials from elsewhere):
  *   M = max_s m_s,  out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s,
@@ -275,10 +287,12 @@ int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch
  *   Arguments are those of kvq_decode_attn without the workspace; `out` is required.
  *   Returns KVQ_ERR_WORKSPACE when kvq_workspace_size(...) for the request exceeds
  *   KVQ_NOALLOC_SCRATCH_BYTES.
- *   The first call on each device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.  All calls share
- *   the one array and each call clears its fault-flag word and merge counters first, so calls whose
- *   execution overlaps on the GPU (different streams, or another thread) race.
+ *   Every call looks up the array's device address with the calling thread's current
+ *   device; the first call on a device is its set-up and may load the library's device
+ *   code there, so make it before any stream capture.  All calls share the one array and
+ *   each call clears its fault-flag word and merge counters first, so calls whose
+ *   execution overlaps on the GPU (different streams, or another thread) race.  Faults
+ *   that the kernel detects (KVQ_FLAG_*) are read back with kvq_noalloc_read_flags.
  */
 int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q, int32_t batch,
                             int32_t num_q_heads, const void* k_codes, const void* k_scales,
@@ -288,7 +302,18 @@ int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q, int32_t b
                             unsigned long long* stats, float* out, void* stream);
 
 /*
+ * kvq_noalloc_read_flags -- synchronize `stream` and read the KVQ_FLAG_* bits that the last
+ * kvq_decode_attn_noalloc call on the current device left in the static scratch (each call
+ * clears them first) into *flags (host).  Like that call, it allocates nothing.  Returns
+ * KVQ_ERR_INVALID_ARG for a null `flags`, KVQ_ERR_CUDA if a CUDA call fails.
+ */
+int kvq_noalloc_read_flags(uint32_t* flags, void* stream);
+
+/*
  * kvq_lloyd_max_codebook -- the minimum-MSE `levels`-entry scalar codebook for
+ *   (Passage: the rotated codebook format of "Почему это работает для любой квантизации";
+ *   the page names no codebook, Lloyd-Max for the rotated coordinates' Gaussian is this
+ *   library's reading.)
  * N(0, sigma^2) (Lloyd's iteration in fp64, symmetric), rounded to IEEE fp16
  * (round-to-nearest-even) and written to out_fp16 (host, `levels` entries,
  * increasing).  The lut4 format uses levels = 16, sigma = 1/sqrt(head_dim).

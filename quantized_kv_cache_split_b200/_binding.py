@@ -88,6 +88,7 @@ def _load():
         "kvq_combine": (ctypes.c_int, [D, P, I32, I32, I32, I32, U32, P, P, P]),
         "kvq_decode_attn_noalloc": (ctypes.c_int, [D, P, I32, I32, P, P, P, P, P, I32, P, I32, F32,
                                                    F32, I32, U32, P, P, P]),
+        "kvq_noalloc_read_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
         "kvq_lloyd_max_codebook": (ctypes.c_int, [I32, ctypes.c_double,
                                                   ctypes.POINTER(ctypes.c_uint16)]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -255,3 +256,10 @@ def kvq_decode_attn_noalloc(desc: KvqCacheDesc, q, batch: int, num_q_heads: int,
     if check:
         _check("kvq_decode_attn_noalloc", st)
     return st
+
+
+def kvq_noalloc_read_flags(stream=None) -> int:
+    """KVQ_FLAG_* bits of the last kvq_decode_attn_noalloc call on the current device."""
+    flags = ctypes.c_uint32(0)
+    _check("kvq_noalloc_read_flags", _lib.kvq_noalloc_read_flags(ctypes.byref(flags), _stream(stream)))
+    return int(flags.value)

@@ -7,8 +7,6 @@
 // merge, as kvq_decode_attn given an output pointer, but keeps the partials and merge
 // counters in a static device array owned by the library, so the caller passes only
 // inputs and outputs.
-#include <mutex>
-
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -18,20 +16,15 @@ namespace {
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
-// Device address of the scratch array, looked up once per device with that device current.
-// (In host code the symbol name is only a host-side stand-in, never a device address.)
+// Device address of the scratch array on the current device.  In host code the symbol
+// name is only a host-side stand-in, never a device address, so it is looked up with
+// cudaGetSymbolAddress, with the device current, on every call: nothing is cached that a
+// reset or a recreated context could leave stale.  The first lookup on a device is its
+// set-up (it may load the library's device code there).
 int scratch_address(void** out) {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
+  *out = p;
   return KVQ_OK;
 }
 
@@ -68,4 +61,13 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q
   return kvq_decode_attn(desc, q, batch, num_q_heads, k_codes, k_scales, v_codes, v_scales,
                          page_table, max_pages, seq_lens, max_seq_len, sm_scale, tau, L, options,
                          ws, need, stats, out, stream);
+}
+
+extern "C" int kvq_noalloc_read_flags(uint32_t* flags, void* stream) {
+  if (!flags) return KVQ_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  const int st = scratch_address(&ws);
+  if (st != KVQ_OK) return st;
+  // the flag word is word 0 of the scratch, as of a workspace
+  return kvq_read_device_flags(ws, flags, stream);
 }

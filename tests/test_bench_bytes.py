@@ -48,3 +48,24 @@ def test_paged_bytes_include_page_table_and_o_partials():
     out = 8 * 32 * 128 * 4
     got = bench.algorithmic_bytes(rep, 466267, splits * 4, with_o=True)
     assert got == k + v + q + pt + part + out == 112549272
+
+
+def test_timed_region_is_one_graph_of_exactly_the_timed_steps():
+    # whatever --steps is (here fewer steps than cache copies, and a warm-up that is not a
+    # multiple of anything), the warm-up and the timed region are each ONE capture: steps
+    # 0 .. W-1 and W .. W+K-1
+    calls = []
+
+    def fake_capture(fn, n_steps, start):
+        calls.append((n_steps, start))
+        return ("graph", n_steps, start)
+
+    g = bench.StepGraphs(lambda i: None, steps=20, warmup=5, capture_fn=fake_capture)
+    assert calls == [(5, 0), (20, 5)]
+    assert g.warm == ("graph", 5, 0) and g.timed == ("graph", 20, 5)
+
+
+def test_cpu_oracle_group_runs_on_the_host():
+    # the CPU baseline's unit of work (one (sequence, KV head) group of the oracle, truncated)
+    dt = bench._oracle_group(("tiny_q8_d64", 0, 0, 128, 64, 1e-6))
+    assert dt > 0.0

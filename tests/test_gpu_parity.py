@@ -2,6 +2,7 @@
 the same seeded inputs.  Quantized planes must match bit for bit; attention
 outputs must satisfy the error bound of the method; skip counters must match
 the oracle's under the same split schedule within 0.1%."""
+import functools
 import math
 
 import numpy as np
@@ -303,19 +304,26 @@ def test_decode_parity_full_32k_v_fetch(v_fetch, scope):
     check_parity(inp, g, o, 1e-6)
 
 
+@functools.lru_cache(maxsize=2)
+def _paged_inputs(name):
+    return W.generate(W.WORKLOADS[name])
+
+
 @pytest.mark.parametrize("name", ["paged_b8_q4", "paged_b8_q8"])
-def test_decode_parity_full_paged(name):
+@pytest.mark.parametrize("tau", [0.0, 1e-6, 1e-4])
+def test_decode_parity_full_paged(name, tau):
+    # The 8-stream paged configuration at full size (245,760 positions, 3840 pages) over its
+    # tau sweep: every output element of all 32 (sequence, KV head) groups against the
+    # oracle, and the skip counters (pairs and V rows) within 0.1% of the oracle's under the
+    # same split schedule.
     wl = W.WORKLOADS[name]
-    inp = W.generate(wl)
-    g = run_library(inp, 1e-6, 0)
-    # full output on three (sequence, KV head) groups computed one by one by the oracle,
-    # plus the exact counters over everything
-    groups = [(3, 0), (0, 2), (7, 3)]
-    o = run_oracle(inp, 1e-6, g["split"], groups=groups)
-    check_parity(inp, g, o, 1e-6, groups=groups)
-    total = int(inp.seq_lens.sum())
-    assert g["stats"][0] == total * wl.num_q_heads
-    assert g["stats"][2] + g["stats"][3] == total * wl.num_kv_heads
+    inp = _paged_inputs(name)
+    g = run_library(inp, tau, 0)
+    o = run_oracle(inp, tau, g["split"])
+    check_parity(inp, g, o, tau)
+    assert g["flags"] == 0
+    if tau > 0:
+        assert g["stats"][1] > 0.3 * g["stats"][0]
 
 
 # ------------------------------------------------------------------ device-side fault reporting

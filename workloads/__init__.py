@@ -122,8 +122,18 @@ class Inputs:
         return np.concatenate([[0], np.cumsum(self.seq_lens)]).astype(np.int64)
 
 
+def _to_f16(x: np.ndarray) -> np.ndarray:
+    """IEEE fp32 -> fp16, round to nearest even (torch's vectorised cast when torch is
+    importable, else numpy's; both are the same IEEE conversion, bit for bit)."""
+    try:
+        import torch
+    except ImportError:  # pragma: no cover - torch is always present in this project
+        return x.astype(np.float16)
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float16).numpy()
+
+
 def _normal_f16(rng: np.random.Generator, shape) -> np.ndarray:
-    return rng.standard_normal(shape, dtype=np.float32).astype(np.float16)
+    return _to_f16(rng.standard_normal(shape, dtype=np.float32))
 
 
 def generate(wl: Workload, seed: Optional[int] = None) -> Inputs:

@@ -256,16 +256,36 @@ def capture(fn, n_steps, start):
     return g
 
 
+def upload_graph(g) -> bool:
+    """Upload an instantiated graph to the device ahead of its first replay (cuGraphUpload),
+    so that the first, timed replay does not include the upload.  False if the driver
+    call is unavailable."""
+    import ctypes
+    import torch
+    try:
+        cu = ctypes.CDLL("libcuda.so.1")
+        cu.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        cu.cuGraphUpload.restype = ctypes.c_int
+        st = cu.cuGraphUpload(ctypes.c_void_p(g.raw_cuda_graph_exec()),
+                              ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        torch.cuda.synchronize()
+        return st == 0
+    except Exception:
+        return False
+
+
 class StepGraphs:
     """The warm-up steps 0 .. warmup - 1 and the timed steps warmup .. warmup + steps - 1
     of ``fn`` (step i works on cache copy i % R inside ``fn``), each captured as ONE
     graph, so the timed region is a single replay of exactly ``steps`` launches of the
-    hot path whatever ``steps`` is."""
+    hot path whatever ``steps`` is.  The timed graph is uploaded to the device before it
+    is first replayed."""
 
-    def __init__(self, fn, steps, warmup, capture_fn=capture):
+    def __init__(self, fn, steps, warmup, capture_fn=capture, upload_fn=upload_graph):
         self.steps, self.warmup = steps, warmup
         self.warm = capture_fn(fn, warmup, 0)
         self.timed = capture_fn(fn, steps, warmup)
+        self.uploaded = upload_fn(self.timed)
 
 
 def time_steps(graphs: StepGraphs, world, sampler=None):

@@ -7,6 +7,7 @@
 #include <mutex>
 #include <vector>
 
+#include "kvq_decode2.h"
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -80,7 +81,7 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
     if (cap4 > 0) {
       ctas_per_pair = 4 * std::max<int64_t>(1, cap4 / pairs);
     } else {
-      const int cap1 = decode_cluster_capacity(desc->fmt, desc->head_dim, 1);
+      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim);
       if (cap1 <= 0) return KVQ_ERR_CUDA;
       ctas_per_pair = std::max<int64_t>(1, cap1 / pairs);
     }
@@ -245,8 +246,13 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
     return KVQ_OK;
   }
   int CS = 1, capacity = 0;
-  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
-  if (st != KVQ_OK) return st;
+  if (options & KVQ_OPT_SHARED_MAX) {
+    st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
+    if (st != KVQ_OK) return st;
+  } else {
+    capacity = decode2_capacity(desc->fmt, desc->head_dim);
+    if (capacity <= 0) return KVQ_ERR_CUDA;
+  }
   DecodeArgs a;
   a.desc = *desc;
   a.q = q;
@@ -299,8 +305,15 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   // workspace and the combine kernel merges them, one CTA per (sequence, query head),
   // which measured faster than the last finisher of each (sequence, KV head) merging alone.
   const bool combine_after = out && CS == 1 && groups > capacity;
-  if (combine_after) a.out = nullptr;
-  st = launch_decode(a, static_cast<cudaStream_t>(stream));
+  if (options & KVQ_OPT_SHARED_MAX) {
+    // clusters of splits sharing one running maximum: the cluster kernel
+    if (combine_after) a.out = nullptr;
+    st = launch_decode(a, static_cast<cudaStream_t>(stream));
+  } else {
+    // the streaming kernel merges in-kernel when every split has its own CTA, else it
+    // writes the partials for the combine kernel
+    st = launch_decode2(a, static_cast<cudaStream_t>(stream));
+  }
   if (st != KVQ_OK || !combine_after) return st;
   return launch_combine(*desc, workspace, batch, num_q_heads, max_seq_len, L, CS, a.max_splits, seq_lens,
                         out, static_cast<cudaStream_t>(stream));

@@ -1,0 +1,1015 @@
+// Split-KV decode attention with sparse V dequantization (sm_100a): the streaming kernel.
+//
+// Method (tproger.ru, "Пропуск 90% работы по деквантизации ускорил
+// декодирование LLM", section "Решение — не ускорять, а пропускать"): the softmax
+// weights come from K before any V work, so V dequantization and accumulation are
+// skipped for every position whose weight exp(s - m_running) is below tau; section
+// "FAQ": K itself is always dequantized.
+//
+// Work unit: one split (<= 1024 positions = 16 tiles of 64) of one (sequence, KV head).
+// One CTA of 16 warps per SM; CTAs loop over the units.  Per unit:
+//   copies    Warp w owns tile w.  Its lane 0 issues the tile's K codes as one tensor
+//             copy (TMA, swizzled so that the fragment loads are free of bank
+//             conflicts) and its scale rows as one bulk copy, both completing on the
+//             tile's mbarrier; with V fetched with K, the V tile the same way on a
+//             second mbarrier.  Nothing waits for the copies to be issued.
+//   query     Warp 0 builds the query fragments (lut4: the rotated query) for the CTA.
+//   K pass    Each warp scores its tile on the tensor cores (mma.sync m16n8k16,
+//             positions x heads x head_dim) once its copy lands; scores stay in
+//             registers.
+//   maximum   One CTA barrier; every warp reads the split's maximum per head (with the
+//             sequence-wide option, the splits of the (sequence, KV head) first
+//             exchange their maxima and denominators through tagged words).
+//   weights   Each warp turns its scores into weights p = 2^(s - m), adds them all
+//             into the denominator, keeps a pair iff s - m >= log2(tau), writes the
+//             kept weights (fp16) into the CTA's weight matrix and a 64-bit row mask of
+//             the rows any head keeps; with V fetched after the test, it gathers just
+//             those rows.
+//   V pass    12 warps split the head dimension into 32-dim slices and the tiles into
+//             position sets, so no warp holds the whole output: for every 16-row group
+//             with a kept row, ldmatrix.trans of the slice's codes (magic-number fp16 for
+//             q8_0 / q4_0, centroid or E2M1 lookups for lut4 / nvfp4) times the group's
+//             weights on the tensor cores.  Skipped groups cost nothing, skipped rows
+//             inside a kept group contribute zero.
+//   merge     When every unit has its own CTA, the splits publish (m, l) after the
+//             weights; one otherwise idle warp collects every split's (m, l) during the
+//             V pass and the CTA adds its normalized share into the output with vector
+//             atomics (lut4: rotated back first).  Otherwise the CTA writes its partial
+//             (o, m, l) and the combine kernel merges them.
+// Every wait (mbarriers, exchange, flags) is bounded and reports KVQ_FLAG_TIMEOUT.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "kvq_decode2.h"
+#include "kvq_decode_common.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kNW = 16;              // warps per CTA: warp w owns tile w of the unit
+constexpr int kNT = 32 * kNW;
+constexpr int kVW = 12;              // warps of the V pass (dim slices x position sets)
+constexpr int kPollWarp = kNW - 1;   // collects the exchange during the V pass
+static_assert(kNW * kTile == KVQ_MAX_SPLIT_TOKENS, "one tile per warp per split");
+
+// ------------------------------------------------------------------ mbarriers, bulk copies
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false after ~kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity))
+    if (clock64() - t0 > kWaitCycles) return false;
+  return true;
+}
+// Rows y .. y + 63 of a 2-D tensor map (x = 0) into shared memory (swizzled as the map says).
+__device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* map, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// A contiguous range (16-byte aligned, a multiple of 16 bytes) into shared memory.
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+// Generic-proxy accesses of shared memory before this point are ordered before later
+// async-proxy (bulk copy) writes to it.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void ldsm_x2_trans(const void* p, uint32_t& d0, uint32_t& d1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(d0), "=r"(d1)
+               : "r"(smem_u32(p))
+               : "memory");
+}
+__device__ __forceinline__ uint32_t hadd2u(uint32_t a, uint32_t b) {
+  return h2_as_u32(__hadd2(u32_as_h2(a), u32_as_h2(b)));
+}
+__device__ __forceinline__ uint32_t hmul2uu(uint32_t a, uint32_t b) {
+  return h2_as_u32(__hmul2(u32_as_h2(a), u32_as_h2(b)));
+}
+
+// ------------------------------------------------------------------ V slices
+// The V pass of one warp covers a 32-dim slice `dq` of the head dimension: chunk dq of a
+// q4_0 / lut4 / nvfp4 code row (16 bytes = 32 nibbles), chunks 2dq and 2dq + 1 of a
+// q8_0 row (16 dims each).  For 16 positions (rows s0 .. s0 + 15 of a staged tile) it
+// adds v_hat^T p into acc[2][4], two m16n8 tiles (rows = dims, cols = heads):
+//   q4_0 / lut4 / nvfp4: tile mt row r <-> dim 32 dq + 4 r + 2 mt, row r + 8 <-> that + 1
+//   q8_0:                tile j  row r <-> dim 16 (2 dq + j) + 2 r, row r + 8 <-> that + 1
+// (lane (r, c) holds rows r, r + 8 of heads 2c, 2c + 1).  B = the weights of rows
+// s0 + {2c, 2c + 1, 2c + 8, 2c + 9} for head r, read from the CTA's weight matrix.
+template <int FMT, int D>
+__device__ __forceinline__ int slice_dim(int dq, int mt, int r, int i) {
+  if constexpr (FMT == KVQ_FMT_Q8_0) return 16 * (2 * dq + mt) + 2 * r + (i >> 1);
+  else return 32 * dq + 4 * r + 2 * mt + (i >> 1);
+}
+
+// Per-position scale of the slice as fp16 (mag formats: the block scale d; lut4: the
+// vector norm; nvfp4: the E4M3 scale of the lane's 16-dim block times the vector scale),
+// zero for a row no head keeps (its staged bytes may be anything).
+template <int FMT, int D>
+__device__ __forceinline__ uint32_t slice_scale_bits(const uint8_t* vs, int row, int dq, int r, bool kept) {
+  using C = Cfg<FMT, D>;
+  if (!kept) return 0u;
+  const uint8_t* srow = vs + row * C::SROW;
+  if constexpr (C::kLut) return lds16(srow);
+  else if constexpr (C::kNv) {
+    const float g = *reinterpret_cast<const float*>(srow + D / 16);
+    return __half_as_ushort(__float2half_rn(e4m3_float(srow[2 * dq + (r >> 2)]) * g));
+  } else {
+    return lds16(srow + 2 * dq);  // block dq (32 dims) of q8_0 / q4_0
+  }
+}
+
+// q8_0 / q4_0: codes enter the MMA as magic-number fp16 with the offset removed by one
+// exact fp16 subtraction; the block scale rides on the weights, B = p d 2^-k (k >= 0 per
+// warp, so that p 2^14 d 2^-k stays inside fp16; acc is rescaled by 2^k at the end).
+template <int FMT, int D>
+__device__ __forceinline__ void v_slice_mag(const uint8_t* __restrict__ vc, const uint8_t* __restrict__ vs,
+                                            const __half* __restrict__ prow, int s0, uint32_t gmask,
+                                            int dq, int lane, uint32_t f2k, float (&acc)[2][4]) {
+  using C = Cfg<FMT, D>;
+  const int r = lane >> 2, c = lane & 3;
+  const int ra = s0 + 2 * c, rb = ra + 8;
+  const uint32_t d01 = slice_scale_bits<FMT, D>(vs, ra, dq, r, (gmask >> (2 * c)) & 1u) |
+                       (slice_scale_bits<FMT, D>(vs, ra + 1, dq, r, (gmask >> (2 * c + 1)) & 1u) << 16);
+  const uint32_t d89 = slice_scale_bits<FMT, D>(vs, rb, dq, r, (gmask >> (2 * c + 8)) & 1u) |
+                       (slice_scale_bits<FMT, D>(vs, rb + 1, dq, r, (gmask >> (2 * c + 9)) & 1u) << 16);
+  const uint32_t b0 = hmul2uu(lds32(prow + 2 * c), hmul2uu(d01, f2k));
+  const uint32_t b1 = hmul2uu(lds32(prow + 2 * c + 8), hmul2uu(d89, f2k));
+  constexpr uint32_t kM1032 = 0xE408E408u, kM72 = 0xD480D480u, kM1152 = 0xE480E480u;  // -offsets
+  if constexpr (C::kQ4) {
+    // matrix 0: rows s0 .. s0 + 7, matrix 1: rows s0 + 8 .. s0 + 15; chunk dq
+    const int row = s0 + (lane & 15);
+    uint32_t x0, x1;
+    ldsm_x2_trans(vc + row * C::CROW + ((dq ^ swz<FMT, D>(row)) << 4), x0, x1);
+    const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
+    mma16816(acc[0], hadd2u((x0 & 0x000F000Fu) | kMagic, kM1032), hadd2u((x0 & 0x00F000F0u) | kMagic64, kM72),
+             hadd2u((x1 & 0x000F000Fu) | kMagic, kM1032), hadd2u((x1 & 0x00F000F0u) | kMagic64, kM72), b0, b1);
+    mma16816(acc[1], hadd2u((y0 & 0x000F000Fu) | kMagic, kM1032), hadd2u((y0 & 0x00F000F0u) | kMagic64, kM72),
+             hadd2u((y1 & 0x000F000Fu) | kMagic, kM1032), hadd2u((y1 & 0x00F000F0u) | kMagic64, kM72), b0, b1);
+  } else {
+    // matrix i: rows s0 + 8 (i & 1) .., chunk 2 dq + (i >> 1)
+    const int mi = lane >> 3;
+    const int row = s0 + 8 * (mi & 1) + (lane & 7);
+    uint32_t R[2][2];
+    ldsm_x4_trans(vc + row * C::CROW + (((2 * dq + (mi >> 1)) ^ swz<FMT, D>(row)) << 4), R[0][0], R[0][1],
+                  R[1][0], R[1][1]);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t x0 = R[j][0] ^ 0x80808080u, x1 = R[j][1] ^ 0x80808080u;
+      mma16816(acc[j], hadd2u(prmt(x0, 0x64646464u, 0x4240u), kM1152), hadd2u(prmt(x0, 0x64646464u, 0x4341u), kM1152),
+               hadd2u(prmt(x1, 0x64646464u, 0x4240u), kM1152), hadd2u(prmt(x1, 0x64646464u, 0x4341u), kM1152), b0, b1);
+    }
+  }
+}
+
+// lut4 / nvfp4: the nibbles are looked up (centroids / E2M1 values) into fp16 pairs of
+// the two positions and multiplied by the positions' scales; B = p.
+template <int FMT, int D>
+__device__ __forceinline__ void v_slice_lut(const uint8_t* __restrict__ vc, const uint8_t* __restrict__ vs,
+                                            const __half* __restrict__ prow, int s0, uint32_t gmask,
+                                            int dq, int lane, const Lut& lut, float (&acc)[2][4]) {
+  using C = Cfg<FMT, D>;
+  const int r = lane >> 2, c = lane & 3;
+  const int ra = s0 + 2 * c, rb = ra + 8;
+  const uint32_t sab = slice_scale_bits<FMT, D>(vs, ra, dq, r, (gmask >> (2 * c)) & 1u) |
+                       (slice_scale_bits<FMT, D>(vs, ra + 1, dq, r, (gmask >> (2 * c + 1)) & 1u) << 16);
+  const uint32_t scd = slice_scale_bits<FMT, D>(vs, rb, dq, r, (gmask >> (2 * c + 8)) & 1u) |
+                       (slice_scale_bits<FMT, D>(vs, rb + 1, dq, r, (gmask >> (2 * c + 9)) & 1u) << 16);
+  const uint32_t b0 = lds32(prow + 2 * c), b1 = lds32(prow + 2 * c + 8);
+  const int row = s0 + (lane & 15);
+  uint32_t x[2];
+  ldsm_x2_trans(vc + row * C::CROW + ((dq ^ swz<FMT, D>(row)) << 4), x[0], x[1]);
+  // e[h][i]: dim 4r + i of positions (2c + 8h, 2c + 8h + 1) as an fp16 pair
+  uint32_t e[2][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t La, Ha, Lb, Hb;
+    lut_lookup4(lut, x[h], nib_mask_lo(x[h]), La, Ha);
+    lut_lookup4(lut, x[h] >> 16, nib_mask_hi(x[h]), Lb, Hb);
+    const uint32_t ta01 = prmt(La, Ha, 0x5140u), tb01 = prmt(Lb, Hb, 0x5140u);
+    const uint32_t ta23 = prmt(La, Ha, 0x7362u), tb23 = prmt(Lb, Hb, 0x7362u);
+    const uint32_t s = h ? scd : sab;
+    e[h][0] = hmul2uu(prmt(ta01, tb01, 0x5410u), s);
+    e[h][1] = hmul2uu(prmt(ta01, tb01, 0x7632u), s);
+    e[h][2] = hmul2uu(prmt(ta23, tb23, 0x5410u), s);
+    e[h][3] = hmul2uu(prmt(ta23, tb23, 0x7632u), s);
+  }
+  mma16816(acc[0], e[0][0], e[0][1], e[1][0], e[1][1], b0, b1);
+  mma16816(acc[1], e[0][2], e[0][3], e[1][2], e[1][3], b0, b1);
+}
+
+// ------------------------------------------------------------------ the kernel
+template <int FMT, int D>
+__global__ void __launch_bounds__(kNT, 1)
+decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv) {
+  using C = Cfg<FMT, D>;
+  const DecodeArgs& a = pr.a;
+  constexpr int NDQ = D / 32;           // 32-dim slices
+  constexpr int NPQ = kVW / NDQ;        // position sets of the V pass
+  constexpr int CODE = kTile * C::CROW; // code bytes of one staged tile
+  constexpr int SC = kTile * C::SROW;   // scale bytes of one staged tile
+  constexpr int kQfWords = 2 * C::KSTEPS + (C::kLut ? 2 * C::KSTEPS : 0) + 2 * C::NBLK;
+
+  extern __shared__ __align__(1024) uint8_t smem2_raw[];
+  __shared__ __align__(8) uint64_t kbar[kNW], vbar[kNW];
+  __shared__ float red_m[kNW][8], red_l[kNW][8];
+  __shared__ unsigned long long kmask[kNW];
+  __shared__ int cnt_skip[kNW];
+  __shared__ float mh_s[8], share_s[8];
+  __shared__ int misc[4];  // 0: clamped length, 1: exchange ok, 2: tag
+  __shared__ uint32_t qfr[kQfWords * 32];
+
+  uint8_t* sm = smem2_raw + ((1024u - (smem_u32(smem2_raw) & 1023u)) & 1023u);
+  uint8_t* kcode = sm + pr.off_kcode;
+  uint8_t* kscale = sm + pr.off_kscale;
+  uint8_t* vcode = sm + pr.off_vcode;    // == kcode when V goes into the K slots
+  uint8_t* vscale = sm + pr.off_vscale;
+  __half* pw = reinterpret_cast<__half*>(sm + pr.off_pw);       // [8][LP] weights x 2^14
+  float* red_o = reinterpret_cast<float*>(sm + pr.off_redo);   // [NPQ][8][D]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = lane >> 2, c = lane & 3;
+  uint32_t* flags = reinterpret_cast<uint32_t*>(a.workspace);
+  const int hkv = a.desc.num_kv_heads, G = a.group, P = a.desc.page_size, Ls = a.split_tokens;
+  const int B = a.batch, Hq = a.num_q_heads;
+  const int NT = Ls / kTile;            // tiles per unit
+  const int LP = pr.lp;                 // weight-matrix row stride (halves)
+  const int NCU = a.max_splits;
+  const int total = B * NCU * hkv;
+  const int cap = min(a.max_seq_len, a.max_pages * P);
+  const bool add_merge = a.out != nullptr && a.group_merge;
+  const bool v_tma = pr.v_tma != 0;     // V tiles copied whole (with K, or right after it)
+  const bool v_sep = pr.v_sep != 0;     // V tiles in their own region (copied with K)
+  const float qk_scale = a.sm_scale * kLog2e;
+  const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
+  const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNW; ++i) {
+      mbar_init(&kbar[i], 1);
+      mbar_init(&vbar[i], 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Programmatic dependent launch: the next grid may be scheduled now; nothing is read
+  // from global memory before the preceding grid has completed.
+  grid_dependents_launch();
+  grid_dependency_wait();
+  if (tid == 0) {  // every CTA takes part in the launch count that tags the exchange
+    const unsigned long long ep = epoch_read(a.epoch);
+    epoch_advance(a.epoch);
+    misc[2] = (int)epoch_tag(ep);
+  }
+  __syncthreads();  // mbarriers initialized, tag known
+  Lut lut;
+  if constexpr (C::kLut) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t e = a.desc.codebook[4 * i + j];
+        lo |= (e & 0xffu) << (8 * j);
+        hi |= (e >> 8) << (8 * j);
+      }
+      lut.lo[i] = lo;
+      lut.hi[i] = hi;
+    }
+  } else if constexpr (C::kNv) {
+    const uint32_t hi[4] = {0x3E3C3800u, 0x46444240u, 0xBEBCB880u, 0xC6C4C2C0u};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      lut.lo[i] = 0u;
+      lut.hi[i] = hi[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lut.lo[i] = lut.hi[i] = 0u;
+  }
+
+  const __half* qg = static_cast<const __half*>(a.q);
+  const uint8_t* kscales_g = static_cast<const uint8_t*>(a.k_scales);
+  const uint8_t* vcodes_g = static_cast<const uint8_t*>(a.v_codes);
+  const uint8_t* vscales_g = static_cast<const uint8_t*>(a.v_scales);
+
+#pragma unroll 1
+  for (int it = blockIdx.x, k = 0; it < total; it += gridDim.x, ++k) {
+    const uint32_t ph = (uint32_t)k & 1u;  // mbarrier phase of this unit
+    const int kvh = it % hkv;
+    const int b = (it / hkv) % B;
+    const int cu = it / (hkv * B);
+    const int t0 = cu * Ls;
+    const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;
+
+    // ---- copies: lane 0 of warp w issues tile w (positions that exist in memory)
+    int row0 = -1;
+    bool k_issued = false, v_issued = false;
+    if (warp < NT) {
+      if (lane == 0) {
+        const int tok0 = t0 + warp * kTile;
+        uint32_t kbytes = 0, vbytes = 0;
+        if (tok0 < cap) {
+          const int lp = tok0 / P, off = tok0 - lp * P;  // tiles never straddle pages (P % 64 == 0)
+          const int page = a.page_table ? __ldg(a.page_table + (size_t)b * a.max_pages + lp)
+                                        : b * a.max_pages + lp;
+          if (page >= 0 && page < a.desc.num_pages) {
+            row0 = (page * hkv + kvh) * P + off;
+            kbytes = CODE + SC;
+            if (v_sep) vbytes = CODE + SC;
+          } else {
+            set_flag(flags, KVQ_FLAG_BAD_PAGE);
+          }
+        }
+        fence_proxy_async();
+        mbar_expect_tx(&kbar[warp], kbytes);
+        if (kbytes) {
+          tma_rows(kcode + warp * CODE, &tmk, row0, &kbar[warp]);
+          bulk_copy(kscale + warp * SC, kscales_g + (size_t)row0 * C::SROW, SC, &kbar[warp]);
+        }
+        if (v_sep) {
+          mbar_expect_tx(&vbar[warp], vbytes);
+          if (vbytes) {
+            tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+            bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+          }
+        }
+      }
+      row0 = __shfl_sync(0xffffffffu, row0, 0);
+      k_issued = row0 >= 0;
+      v_issued = v_sep && k_issued;
+    }
+    // ---- the sequence length; split 0 clears the output rows the splits add into
+    if (warp == 1) {
+      if (lane == 0) {
+        const int n = __ldg(a.seq_lens + b);
+        if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
+        misc[0] = max(0, min(n, cap));
+        misc[1] = 1;
+      }
+      if (add_merge && cu == 0) {
+        float4* orow = reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D);
+        for (int i = lane; i < G * D / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
+        if (lane == 0) flag_set_release(a.zflag + (size_t)b * hkv + kvh, (uint32_t)misc[2]);
+      }
+    }
+    // ---- query fragments, built once for the CTA by warp 0
+    if (warp == 0) {
+      QRaw<D> qraw;
+      load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr, a.desc.signs, c,
+                         qraw);
+      uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
+      float corr[C::NBLK][2];
+      build_query<FMT, D>(qraw, c, qf, ql, corr);
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        qfr[(2 * ks) * 32 + lane] = qf[ks][0];
+        qfr[(2 * ks + 1) * 32 + lane] = qf[ks][1];
+        if constexpr (C::kLut) {
+          qfr[(2 * C::KSTEPS + 2 * ks) * 32 + lane] = ql[ks][0];
+          qfr[(2 * C::KSTEPS + 2 * ks + 1) * 32 + lane] = ql[ks][1];
+        }
+      }
+      if constexpr (!C::kLut) {
+#pragma unroll
+        for (int m = 0; m < C::NBLK; ++m) {
+          qfr[(2 * C::KSTEPS + 2 * m) * 32 + lane] = __float_as_uint(corr[m][0]);
+          qfr[(2 * C::KSTEPS + 2 * m + 1) * 32 + lane] = __float_as_uint(corr[m][1]);
+        }
+      }
+    }
+    __syncthreads();  // B0: query fragments, length
+    const int nb = misc[0];
+    const uint32_t tag = (uint32_t)misc[2];
+    const int n_tok = max(0, min(Ls, nb - t0));
+    const int nvalid = warp < NT ? max(0, min(kTile, n_tok - warp * kTile)) : 0;
+    const bool has_tile = nvalid > 0 && k_issued;
+    if (nvalid > 0 && !k_issued && lane == 0) set_flag(flags, KVQ_FLAG_BAD_PAGE);
+
+    // ---- K pass
+    float s[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    bool k_waited = false;
+    if (has_tile) {
+      uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
+      float corr[C::NBLK][2];
+#pragma unroll
+      for (int ks = 0; ks < C::KSTEPS; ++ks) {
+        qf[ks][0] = qfr[(2 * ks) * 32 + lane];
+        qf[ks][1] = qfr[(2 * ks + 1) * 32 + lane];
+        ql[ks][0] = C::kLut ? qfr[(2 * C::KSTEPS + 2 * ks) * 32 + lane] : 0u;
+        ql[ks][1] = C::kLut ? qfr[(2 * C::KSTEPS + 2 * ks + 1) * 32 + lane] : 0u;
+      }
+#pragma unroll
+      for (int m = 0; m < C::NBLK; ++m) {
+        corr[m][0] = C::kLut ? 0.f : __uint_as_float(qfr[(2 * C::KSTEPS + 2 * m) * 32 + lane]);
+        corr[m][1] = C::kLut ? 0.f : __uint_as_float(qfr[(2 * C::KSTEPS + 2 * m + 1) * 32 + lane]);
+      }
+      k_waited = true;
+      if (!mbar_wait(&kbar[warp], ph)) {
+        if (lane == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+        mbar_wait(&kbar[warp], ph);  // the copy must not be left in flight
+      }
+      const uint8_t* kc = kcode + warp * CODE;
+      const uint8_t* ks_ = kscale + warp * SC;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
+        if (16 * j < nvalid) {
+          float t[4];
+          k_job_scores<FMT, D>(kc, ks_, 16 * j + r, qf, ql, corr, lut, c, t);
+          const bool va = 16 * j + r < nvalid, vb = 16 * j + r + 8 < nvalid;
+          s[j][0] = va ? t[0] * qk_scale : -INFINITY;
+          s[j][1] = va ? t[1] * qk_scale : -INFINITY;
+          s[j][2] = vb ? t[2] * qk_scale : -INFINITY;
+          s[j][3] = vb ? t[3] * qk_scale : -INFINITY;
+          mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][2]));
+          mx1 = fmaxf(mx1, fmaxf(s[j][1], s[j][3]));
+        }
+      }
+    }
+    if (k_issued && !k_waited) mbar_wait(&kbar[warp], ph);  // a speculative tile past the end
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (r == 0) {
+      red_m[warp][2 * c] = mx0;
+      red_m[warp][2 * c + 1] = mx1;
+    }
+    // V into this warp's K slot right behind its K pass (V tiles copied whole but no
+    // room for a separate region)
+    if (v_tma && !v_sep && warp < NT) {
+      __syncwarp();  // every lane is done reading the K tile
+      if (lane == 0) {
+        fence_proxy_async();
+        const uint32_t vbytes = k_issued && nvalid > 0 ? CODE + SC : 0;
+        mbar_expect_tx(&vbar[warp], vbytes);
+        if (vbytes) {
+          tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+          bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+        }
+      }
+      v_issued = k_issued && nvalid > 0;
+    } else if (!v_sep && warp < NT && lane == 0) {
+      mbar_expect_tx(&vbar[warp], 0);  // every barrier completes one phase per unit
+    }
+    __syncthreads();  // B1: every warp's maxima
+
+    // ---- the split's maximum per head (log2 units)
+    float mh0, mh1;
+    {
+      float m = -INFINITY;
+      if (lane < 8)
+        for (int w = 0; w < NT; ++w) m = fmaxf(m, red_m[w][lane]);
+      mh0 = __shfl_sync(0xffffffffu, m, 2 * c);
+      mh1 = __shfl_sync(0xffffffffu, m, 2 * c + 1);
+      if (warp == 0 && lane < 8) mh_s[lane] = m;
+    }
+    float inv_L0 = 1.f, inv_L1 = 1.f;  // sequence-wide option: weights already final
+    if (a.global_max) {
+      // every split publishes (m, l relative to m); the poll warp derives the final
+      // maximum M and denominator L of every head; the weights below use M
+      float l0 = 0.f, l1 = 0.f;
+      if (has_tile) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          l0 += ex2(s[j][0] - mh0) + ex2(s[j][2] - mh0);
+          l1 += ex2(s[j][1] - mh1) + ex2(s[j][3] - mh1);
+        }
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      if (r == 0) {
+        red_l[warp][2 * c] = hl0 ? l0 : 0.f;
+        red_l[warp][2 * c + 1] = hl1 ? l1 : 0.f;
+      }
+      __syncthreads();
+      if (tid < G && n_tok > 0) {
+        float l = 0.f;
+        for (int w = 0; w < NT; ++w) l += red_l[w][tid];
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mh_s[tid], l);
+      }
+      if (warp == kPollWarp && n_tok > 0) {
+        const int nsplit = (nb + Ls - 1) / Ls;
+        const int h = lane >> 2, j = lane & 3;
+        float M, L;
+        bool ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
+                                 j, 4, nsplit, h < G, tag, M, L);
+        if (ok) {
+          xch_combine(M, L, 2);
+          if (j == 0 && h < G) {
+            mh_s[h] = M;
+            share_s[h] = 1.f / L;
+          }
+        } else if (lane == 0) {
+          set_flag(flags, KVQ_FLAG_TIMEOUT);
+          misc[1] = 0;
+        }
+      }
+      __syncthreads();
+      if (misc[1]) {
+        mh0 = mh_s[2 * c < G ? 2 * c : 0];
+        mh1 = mh_s[2 * c + 1 < G ? 2 * c + 1 : 0];
+        inv_L0 = share_s[2 * c < G ? 2 * c : 0];
+        inv_L1 = share_s[2 * c + 1 < G ? 2 * c + 1 : 0];
+      }
+    }
+    (void)inv_L0;
+    (void)inv_L1;
+
+    // ---- weights, skip test, row masks (and the gathers of kept V rows)
+    if (warp < NT) {
+      float l0 = 0.f, l1 = 0.f;
+      int nskip = 0;
+      unsigned long long tmask = 0ull;
+      __half* pcol = pw + warp * kTile;
+      if (has_tile) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (16 * j < nvalid) {
+            const int ra = 16 * j + r, rb = ra + 8;
+            const bool va = ra < nvalid, vb = rb < nvalid;
+            const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
+            const float da0 = s[j][0] - mh0, da1 = s[j][1] - mh1;
+            const float db0 = s[j][2] - mh0, db1 = s[j][3] - mh1;
+            const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
+            const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
+            l0 += ea0 + eb0;
+            l1 += ea1 + eb1;
+            const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
+            const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
+            nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
+            const __half2 pa = __floats2half2_rn(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f);
+            const __half2 pb = __floats2half2_rn(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f);
+            pcol[(2 * c) * LP + ra] = __low2half(pa);
+            pcol[(2 * c + 1) * LP + ra] = __high2half(pa);
+            pcol[(2 * c) * LP + rb] = __low2half(pb);
+            pcol[(2 * c + 1) * LP + rb] = __high2half(pb);
+            // rows any head keeps: row r from the lanes of row r, then all 16 rows of the job
+            const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
+            const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
+            const uint32_t mine = c == 0 ? ((((rows_a >> (4 * r)) & 1u) << r) | (((rows_b >> (4 * r)) & 1u) << (r + 8)))
+                                         : 0u;
+            tmask |= (unsigned long long)__reduce_or_sync(0xffffffffu, mine) << (16 * j);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      if (r == 0) {
+        red_l[warp][2 * c] = l0;
+        red_l[warp][2 * c + 1] = l1;
+      }
+      if (lane == 0) {
+        kmask[warp] = tmask;
+        cnt_skip[warp] = nskip;
+      }
+      if (!v_tma && tmask) {
+        // gather the kept rows into this tile's V slot: codes with the tile's chunk
+        // swizzle, and the rows' scales (lut4: the aligned pair holding the norm)
+        uint8_t* dst = vcode + warp * CODE;
+        uint8_t* dsc = vscale + warp * SC;
+        const uint8_t* src = vcodes_g + (size_t)row0 * C::CROW;
+        const uint8_t* ssrc = vscales_g + (size_t)row0 * C::SROW;
+        constexpr int CPR = C::CROW / 16;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = lane + 32 * h;
+          if ((tmask >> i) & 1ull) {
+#pragma unroll
+            for (int cc = 0; cc < CPR; ++cc)
+              cp_async16(dst + i * C::CROW + ((cc ^ swz<FMT, D>(i)) << 4), src + (size_t)i * C::CROW + cc * 16);
+            if constexpr (C::SROW == 16) cp_async16(dsc + i * 16, ssrc + (size_t)i * 16);
+            else if constexpr (C::SROW == 8) cp_async8(dsc + i * 8, ssrc + (size_t)i * 8);
+            else cp_async4(dsc + (i & ~1) * 2, ssrc + (size_t)(i & ~1) * 2);
+          }
+        }
+        cp_async_commit();
+      }
+    }
+    __syncthreads();  // B2: weights, row masks, denominators
+
+    // ---- publish (m, l) for the in-kernel merge, or write the partial's (m, l)
+    if (tid < G && n_tok > 0) {
+      float l = 0.f;
+      for (int w = 0; w < NT; ++w) l += red_l[w][tid];
+      if (add_merge) {
+        // the sequence-wide maximum made the weights final already
+        if (!a.global_max) xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mh_s[tid], l);
+      } else {  // (sequence-wide maximum: M, and l relative to M)
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mh_s[tid];
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+      }
+    }
+    if (tid == 32 && a.stats && n_tok > 0) {
+      int ns = 0, nk = 0;
+      for (int w = 0; w < NT; ++w) {
+        ns += cnt_skip[w];
+        nk += __popcll(kmask[w]);
+      }
+      atomicAdd(&a.stats[0], (unsigned long long)n_tok * G);
+      atomicAdd(&a.stats[1], (unsigned long long)ns);
+      atomicAdd(&a.stats[2], (unsigned long long)nk);
+      atomicAdd(&a.stats[3], (unsigned long long)(n_tok - nk));
+    }
+    if (!v_tma) {
+      cp_async_wait<0>();
+      __syncthreads();  // B3: every gathered row is in place
+    }
+
+    // ---- V pass (dim slice dq, position set pq) / exchange poll
+    if (warp < kVW && n_tok > 0) {
+      const int dq = warp % NDQ, pq = warp / NDQ;
+      float acc[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      int kcur = 0;  // mag formats: B carries d 2^-kcur
+#pragma unroll 1
+      for (int t = pq; t < NT; t += NPQ) {
+        const unsigned long long km = kmask[t];
+        if (!km) continue;
+        if (v_tma && !mbar_wait(&vbar[t], ph)) {
+          if (lane == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+          mbar_wait(&vbar[t], ph);
+          continue;
+        }
+        const uint8_t* vc = vcode + t * CODE;
+        const uint8_t* vs = vscale + t * SC;
+        const __half* prow = pw + r * LP + t * kTile;
+        if constexpr (C::kMag) {
+          // the largest kept scale of this block in the tile sets k (it only grows)
+          const uint32_t e0 = ((km >> lane) & 1ull) ? lds16(vs + lane * C::SROW + 2 * dq) & 0x7FFFu : 0u;
+          const uint32_t e1 = ((km >> (lane + 32)) & 1ull) ? lds16(vs + (lane + 32) * C::SROW + 2 * dq) & 0x7FFFu : 0u;
+          const uint32_t emax = __reduce_max_sync(0xffffffffu, max(e0, e1));
+          const int kt = min(14, max(0, (int)(emax >> 10) - 15));
+          if (kt > kcur) {
+            const float f = __int_as_float((127 + kcur - kt) << 23);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc[mt][i] *= f;
+            kcur = kt;
+          }
+          const uint32_t f2k = ((uint32_t)(15 - kcur) << 10) * 0x10001u;  // fp16 2^-kcur, both halves
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t gm = (uint32_t)(km >> (16 * g)) & 0xFFFFu;
+            if (gm) v_slice_mag<FMT, D>(vc, vs, prow + 16 * g, 16 * g, gm, dq, lane, f2k, acc);
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t gm = (uint32_t)(km >> (16 * g)) & 0xFFFFu;
+            if (gm) v_slice_lut<FMT, D>(vc, vs, prow + 16 * g, 16 * g, gm, dq, lane, lut, acc);
+          }
+        }
+      }
+      const float fin = __int_as_float((127 + kcur) << 23) * kPUnscale;
+      float* ro = red_o + (size_t)pq * 8 * D;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int h = 2 * c + (i & 1);
+          ro[h * D + slice_dim<FMT, D>(dq, mt, r, i)] = acc[mt][i] * fin;
+        }
+    } else if (warp == kPollWarp && add_merge && !a.global_max && n_tok > 0) {
+      // this split's share of each head, 2^(m_s - M) / L, once split 0 has cleared the
+      // output rows and every split of the (sequence, KV head) has published
+      bool ok = true;
+      if (lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) {
+        const int nsplit = (nb + Ls - 1) / Ls;
+        const int h = lane >> 2, j = lane & 3;
+        float M, L;
+        ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits, j, 4,
+                            nsplit, h < G, tag, M, L);
+        if (ok) {
+          xch_combine(M, L, 2);
+          if (j == 0 && h < G) share_s[h] = ex2(mh_s[h] - M) / L;
+        }
+      }
+      if (lane == 0 && !ok) {
+        set_flag(flags, KVQ_FLAG_TIMEOUT);
+        misc[1] = 0;
+      }
+    } else if (warp == kPollWarp && add_merge && a.global_max && n_tok > 0 && lane == 0) {
+      // the weights are final already; the output rows must be cleared before adding
+      if (!flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag)) {
+        set_flag(flags, KVQ_FLAG_TIMEOUT);
+        misc[1] = 0;
+      }
+    }
+    // no copy of this unit stays in flight past the end of the unit
+    if (v_issued && warp < NT && !kmask[warp]) mbar_wait(&vbar[warp], ph);
+    __syncthreads();  // B4: the slices' partial sums, the shares
+
+    // ---- this split's contribution
+    if (n_tok > 0) {
+      constexpr int Q4 = D / 4;
+      if (add_merge) {
+        if (misc[1]) {
+          if constexpr (C::kLut) {
+            // rotate back (R^T = diag(s) c H), one warp per head, then add
+            if (warp < G) {
+              constexpr int K = D / 32;
+              const float sh = share_s[warp];
+              float y[K];
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk) {
+                float v = 0.f;
+#pragma unroll
+                for (int q = 0; q < NPQ; ++q) v += red_o[((size_t)q * 8 + warp) * D + 32 * kk + lane];
+                y[kk] = v * sh;
+              }
+#pragma unroll
+              for (int hb = 1; hb < 32; hb <<= 1) {
+                const bool upper = (lane & hb) != 0;
+#pragma unroll
+                for (int kk = 0; kk < K; ++kk) {
+                  const float t = __shfl_xor_sync(0xffffffffu, y[kk], hb);
+                  y[kk] = upper ? (t - y[kk]) : (y[kk] + t);
+                }
+              }
+#pragma unroll
+              for (int hb = 1; hb < K; hb <<= 1)
+#pragma unroll
+                for (int kk = 0; kk < K; ++kk)
+                  if (!(kk & hb)) {
+                    const float u = y[kk], v = y[kk + hb];
+                    y[kk] = u + v;
+                    y[kk + hb] = u - v;
+                  }
+              const float cs = D == 64 ? 0.125f : 0.08838834764831845f;
+              float* dst = a.out + ((size_t)b * Hq + (size_t)kvh * G + warp) * D;
+#pragma unroll
+              for (int kk = 0; kk < K; ++kk)
+                atomicAdd(dst + 32 * kk + lane, y[kk] * cs * (float)a.desc.signs[32 * kk + lane]);
+            }
+          } else {
+            for (int e = tid; e < G * Q4; e += kNT) {
+              const int h = e / Q4, d4 = e - h * Q4;
+              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+              for (int q = 0; q < NPQ; ++q) {
+                const float4 x = reinterpret_cast<const float4*>(red_o + ((size_t)q * 8 + h) * D)[d4];
+                v.x += x.x;
+                v.y += x.y;
+                v.z += x.z;
+                v.w += x.w;
+              }
+              const float sh = share_s[h];
+              v.x *= sh;
+              v.y *= sh;
+              v.z *= sh;
+              v.w *= sh;
+              red_add_f32x4(a.out + ((size_t)b * Hq + (size_t)kvh * G + h) * D + 4 * d4, v);
+            }
+          }
+        }
+      } else {
+        for (int e = tid; e < G * Q4; e += kNT) {
+          const int h = e / Q4, d4 = e - h * Q4;
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int q = 0; q < NPQ; ++q) {
+            const float4 x = reinterpret_cast<const float4*>(red_o + ((size_t)q * 8 + h) * D)[d4];
+            v.x += x.x;
+            v.y += x.y;
+            v.z += x.z;
+            v.w += x.w;
+          }
+          reinterpret_cast<float4*>(a.part_o + (slot0 + (size_t)h * a.max_splits) * D)[d4] = v;
+        }
+      }
+    }
+    __syncthreads();  // B5: the unit's buffers are free
+  }
+}
+
+// ------------------------------------------------------------------ host side
+std::mutex g_mu2;
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// The codes plane as a 2-D tensor of `rows` rows of `crow` bytes; a box is one 64-row tile,
+// swizzled in 16-byte chunks across the row (128-, 64- or 32-byte rows).
+bool code_map(CUtensorMap* m, const void* base, uint64_t rows, int crow) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)crow, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)crow};
+  cuuint32_t box[2] = {(cuuint32_t)crow, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = crow == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : crow == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : CU_TENSOR_MAP_SWIZZLE_32B;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemMax = 232448;  // dynamic + static shared memory per CTA on sm_100a
+constexpr size_t kStaticReserve = 8192;
+
+template <int FMT, int D>
+struct Plan {
+  using C = Cfg<FMT, D>;
+  static constexpr size_t CODE = kTile * C::CROW, SC = kTile * C::SROW;
+  // byte offsets for a unit of nt tiles; v_sep: V tiles get their own region
+  static size_t layout(int nt, bool v_sep, Decode2Params* p) {
+    auto up = [](size_t x, size_t m) { return (x + m - 1) / m * m; };
+    size_t o = 0;
+    p->off_kcode = (uint32_t)o;
+    o += nt * CODE;
+    p->off_kscale = (uint32_t)o;
+    o = up(o + nt * SC, 1024);
+    if (v_sep) {
+      p->off_vcode = (uint32_t)o;
+      o += nt * CODE;
+      p->off_vscale = (uint32_t)o;
+      o = up(o + nt * SC, 128);
+    } else {
+      p->off_vcode = p->off_kcode;
+      p->off_vscale = p->off_kscale;
+    }
+    p->lp = nt * kTile + 8;
+    p->off_pw = (uint32_t)o;
+    o = up(o + (size_t)8 * p->lp * 2, 128);
+    p->off_redo = (uint32_t)o;
+    o += (size_t)(kVW / (D / 32)) * 8 * D * 4;
+    return o + 1024;  // slack for aligning the base to 1024
+  }
+};
+
+template <int FMT, int D>
+int configure2(int dev) {
+  static uint64_t done_mask = 0;  // guarded by g_mu2
+  if (!(done_mask >> dev & 1)) {
+    if (cudaFuncSetAttribute(decode2_kernel<FMT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(kSmemMax - kStaticReserve)) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+    done_mask |= 1ull << dev;
+  }
+  return KVQ_OK;
+}
+
+template <int FMT, int D>
+int capacity2_t() {
+  static int cache[64] = {};  // CTAs resident at once + 1, per device; guarded by g_mu2
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(g_mu2);
+  if (cache[dev] == 0) {
+    if (configure2<FMT, D>(dev) != KVQ_OK) return 0;
+    Decode2Params p{};
+    const size_t bytes = Plan<FMT, D>::layout(kNW, false, &p);
+    int n = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode2_kernel<FMT, D>, kNT, bytes) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    cache[dev] = n * sms + 1;
+  }
+  return cache[dev] - 1;
+}
+
+template <int FMT, int D>
+int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
+  using C = Cfg<FMT, D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(g_mu2);
+    if (configure2<FMT, D>(dev) != KVQ_OK) return KVQ_ERR_CUDA;
+  }
+  const int cap = capacity2_t<FMT, D>();
+  if (cap <= 0) return KVQ_ERR_CUDA;
+  Decode2Params p{};
+  p.a = a;
+  const int nt = a.split_tokens / kTile;
+  const int64_t units = (int64_t)a.batch * a.max_splits * a.desc.num_kv_heads;
+  p.a.grid = (int)std::min<int64_t>(units, cap);
+  if (p.a.grid <= 0) return KVQ_OK;
+  // every unit on its own CTA at once: the splits exchange (m, l) and add their shares
+  p.a.group_merge = a.out != nullptr && units <= cap;
+  if (a.global_max && units > cap) return KVQ_ERR_UNSUPPORTED;
+  // V tiles copied whole: tau = 0 (every row is needed) or when the launch asks; in their
+  // own region when shared memory allows, else into the K slots right after the K pass
+  const bool whole = !(a.tau > 0.f) || a.v_early;
+  size_t bytes = Plan<FMT, D>::layout(nt, whole, &p);
+  p.v_sep = whole ? 1 : 0;
+  if (bytes + kStaticReserve > kSmemMax) {
+    bytes = Plan<FMT, D>::layout(nt, false, &p);
+    p.v_sep = 0;
+  }
+  p.v_tma = whole ? 1 : 0;
+  CUtensorMap tmk, tmv;
+  const uint64_t rows = (uint64_t)a.desc.num_pages * a.desc.num_kv_heads * a.desc.page_size;
+  if (!code_map(&tmk, a.k_codes, rows, C::CROW) || !code_map(&tmv, a.v_codes, rows, C::CROW))
+    return KVQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  const bool coop = p.a.group_merge || a.global_max;
+  if (coop) {  // CTAs wait for one another: all resident together
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na].val.cooperative = 1;
+    ++na;
+  }
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  cfg.gridDim = dim3(p.a.grid, 1, 1);
+  cfg.blockDim = dim3(kNT, 1, 1);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
+  if (e != cudaSuccess && coop) {  // a driver that does not take both: cooperative alone
+    (void)cudaGetLastError();
+    cfg.numAttrs = na - 1;
+    e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
+  }
+  if (e != cudaSuccess) return KVQ_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_decode2(const DecodeArgs& a, cudaStream_t stream) {
+  const int f = a.desc.fmt, d = a.desc.head_dim;
+  if (f == KVQ_FMT_Q8_0 && d == 128) return launch2_t<KVQ_FMT_Q8_0, 128>(a, stream);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return launch2_t<KVQ_FMT_Q8_0, 64>(a, stream);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return launch2_t<KVQ_FMT_Q4_0, 128>(a, stream);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return launch2_t<KVQ_FMT_Q4_0, 64>(a, stream);
+  if (f == KVQ_FMT_LUT4 && d == 128) return launch2_t<KVQ_FMT_LUT4, 128>(a, stream);
+  if (f == KVQ_FMT_LUT4 && d == 64) return launch2_t<KVQ_FMT_LUT4, 64>(a, stream);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return launch2_t<KVQ_FMT_NVFP4, 128>(a, stream);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return launch2_t<KVQ_FMT_NVFP4, 64>(a, stream);
+  return KVQ_ERR_UNSUPPORTED;
+}
+
+int decode2_capacity(int f, int d) {
+  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity2_t<KVQ_FMT_Q8_0, 128>();
+  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity2_t<KVQ_FMT_Q8_0, 64>();
+  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity2_t<KVQ_FMT_Q4_0, 128>();
+  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity2_t<KVQ_FMT_Q4_0, 64>();
+  if (f == KVQ_FMT_LUT4 && d == 128) return capacity2_t<KVQ_FMT_LUT4, 128>();
+  if (f == KVQ_FMT_LUT4 && d == 64) return capacity2_t<KVQ_FMT_LUT4, 64>();
+  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity2_t<KVQ_FMT_NVFP4, 128>();
+  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity2_t<KVQ_FMT_NVFP4, 64>();
+  return 0;
+}
+
+}  // namespace kvq

@@ -1,0 +1,29 @@
+// Internal interface of the streaming decode kernel (kvq_decode2.cu).
+#pragma once
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+// Launch parameters: the request (DecodeArgs) plus the shared-memory plan the host
+// computed for it (byte offsets from the 1024-aligned base of dynamic shared memory).
+struct Decode2Params {
+  DecodeArgs a;
+  uint32_t off_kcode, off_kscale;  // K tiles: codes (swizzled), scale rows
+  uint32_t off_vcode, off_vscale;  // V tiles (== the K tiles' offsets when V reuses them)
+  uint32_t off_pw;                 // weights x 2^14, fp16 [8 heads][lp]
+  uint32_t off_redo;               // V-pass partial sums, fp32 [position sets][8][head_dim]
+  int lp;                          // weight row stride in halves (positions + 8)
+  int v_tma;                       // V tiles copied whole (else only the kept rows, gathered)
+  int v_sep;                       // V tiles in their own region, copied together with K
+};
+
+// The streaming decode kernel for every format and head_dim; merges in-kernel when every
+// unit has its own CTA and `out` is given, else writes the partials (the caller then
+// launches the combine kernel).  KVQ_ERR_UNSUPPORTED for the sequence-wide maximum when
+// the units do not all fit at once.
+int launch_decode2(const DecodeArgs& a, cudaStream_t stream);
+// CTAs of the streaming kernel resident at once on the current device (0 on error).
+int decode2_capacity(int fmt, int head_dim);
+
+}  // namespace kvq

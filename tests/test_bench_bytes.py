@@ -60,7 +60,8 @@ def test_timed_region_is_one_graph_of_exactly_the_timed_steps():
         calls.append((n_steps, start))
         return ("graph", n_steps, start)
 
-    g = bench.StepGraphs(lambda i: None, steps=20, warmup=5, capture_fn=fake_capture)
+    g = bench.StepGraphs(lambda i: None, steps=20, warmup=5, capture_fn=fake_capture,
+                         upload_fn=lambda graph: True)
     assert calls == [(5, 0), (20, 5)]
     assert g.warm == ("graph", 5, 0) and g.timed == ("graph", 20, 5)
 

@@ -50,7 +50,6 @@ namespace {
 
 constexpr int kNW = 16;              // warps per CTA: warp w owns tile w of the unit
 constexpr int kNT = 32 * kNW;
-constexpr int kVW = 12;              // warps of the V pass (dim slices x position sets)
 constexpr int kPollWarp = kNW - 1;   // collects the exchange during the V pass
 static_assert(kNW * kTile == KVQ_MAX_SPLIT_TOKENS, "one tile per warp per split");
 
@@ -112,115 +111,185 @@ __device__ __forceinline__ uint32_t hmul2uu(uint32_t a, uint32_t b) {
   return h2_as_u32(__hmul2(u32_as_h2(a), u32_as_h2(b)));
 }
 
-// ------------------------------------------------------------------ V slices
-// The V pass of one warp covers a 32-dim slice `dq` of the head dimension: chunk dq of a
-// q4_0 / lut4 / nvfp4 code row (16 bytes = 32 nibbles), chunks 2dq and 2dq + 1 of a
-// q8_0 row (16 dims each).  For 16 positions (rows s0 .. s0 + 15 of a staged tile) it
-// adds v_hat^T p into acc[2][4], two m16n8 tiles (rows = dims, cols = heads):
-//   q4_0 / lut4 / nvfp4: tile mt row r <-> dim 32 dq + 4 r + 2 mt, row r + 8 <-> that + 1
-//   q8_0:                tile j  row r <-> dim 16 (2 dq + j) + 2 r, row r + 8 <-> that + 1
-// (lane (r, c) holds rows r, r + 8 of heads 2c, 2c + 1).  B = the weights of rows
-// s0 + {2c, 2c + 1, 2c + 8, 2c + 9} for head r, read from the CTA's weight matrix.
+// ------------------------------------------------------------------ V groups
+// The V pass of a warp covers its own tile, all of the head dimension, one group of 16
+// staged rows (s0 .. s0 + 15, the first n_valid of them inside the sequence) at a time:
+// acc[mt] (m16n8 tiles, rows = dims, cols = heads) += v_hat^T p.  The weights enter as
+// B fragments kept in registers: p01 = (p of rows s0 + 2c, s0 + 2c + 1) and p89 = (rows
+// s0 + 2c + 8, s0 + 2c + 9) for head r, as fp16 x 2^14, zero for skipped pairs.  Rows past
+// n_valid get scale 0, so whatever bytes their slots hold contribute nothing (every
+// format decodes any bit pattern to a finite value).  Output dim of tile mt, row r (row
+// r + 8: that + 1):
+//   q4_0: 32 (mt >> 1) + 4 r + 2 (mt & 1)     q8_0: 16 mt + 2 r     lut4 / nvfp4: E r + 2 mt
 template <int FMT, int D>
-__device__ __forceinline__ int slice_dim(int dq, int mt, int r, int i) {
-  if constexpr (FMT == KVQ_FMT_Q8_0) return 16 * (2 * dq + mt) + 2 * r + (i >> 1);
-  else return 32 * dq + 4 * r + 2 * mt + (i >> 1);
-}
-
-// Per-position scale of the slice as fp16 (mag formats: the block scale d; lut4: the
-// vector norm; nvfp4: the E4M3 scale of the lane's 16-dim block times the vector scale),
-// zero for a row no head keeps (its staged bytes may be anything).
-template <int FMT, int D>
-__device__ __forceinline__ uint32_t slice_scale_bits(const uint8_t* vs, int row, int dq, int r, bool kept) {
+__device__ __forceinline__ int out_dim(int r, int mt, int i) {
   using C = Cfg<FMT, D>;
-  if (!kept) return 0u;
-  const uint8_t* srow = vs + row * C::SROW;
-  if constexpr (C::kLut) return lds16(srow);
-  else if constexpr (C::kNv) {
-    const float g = *reinterpret_cast<const float*>(srow + D / 16);
-    return __half_as_ushort(__float2half_rn(e4m3_float(srow[2 * dq + (r >> 2)]) * g));
-  } else {
-    return lds16(srow + 2 * dq);  // block dq (32 dims) of q8_0 / q4_0
-  }
+  if constexpr (C::kQ4) return 32 * (mt >> 1) + 4 * r + 2 * (mt & 1) + (i >> 1);
+  else if constexpr (C::kQ8) return 16 * mt + 2 * r + (i >> 1);
+  else return C::E * r + 2 * mt + (i >> 1);
 }
 
 // q8_0 / q4_0: codes enter the MMA as magic-number fp16 with the offset removed by one
-// exact fp16 subtraction; the block scale rides on the weights, B = p d 2^-k (k >= 0 per
-// warp, so that p 2^14 d 2^-k stays inside fp16; acc is rescaled by 2^k at the end).
+// exact fp16 subtraction; the block scale rides on the weights, B = p d' per block, with
+// d' = d 2^-k[blk] (k >= 0 per block and tile, so that p 2^14 d' stays inside fp16; the
+// tile's scale rows are rescaled in place by tile_mag_normalize and acc by mag_finish).
 template <int FMT, int D>
-__device__ __forceinline__ void v_slice_mag(const uint8_t* __restrict__ vc, const uint8_t* __restrict__ vs,
-                                            const __half* __restrict__ prow, int s0, uint32_t gmask,
-                                            int dq, int lane, uint32_t f2k, float (&acc)[2][4]) {
+__device__ __forceinline__ void vg_mag(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                       int s0, int n_valid, uint32_t p01, uint32_t p89, int lane,
+                                       float (&acc)[Cfg<FMT, D>::MT][4]) {
   using C = Cfg<FMT, D>;
-  const int r = lane >> 2, c = lane & 3;
-  const int ra = s0 + 2 * c, rb = ra + 8;
-  const uint32_t d01 = slice_scale_bits<FMT, D>(vs, ra, dq, r, (gmask >> (2 * c)) & 1u) |
-                       (slice_scale_bits<FMT, D>(vs, ra + 1, dq, r, (gmask >> (2 * c + 1)) & 1u) << 16);
-  const uint32_t d89 = slice_scale_bits<FMT, D>(vs, rb, dq, r, (gmask >> (2 * c + 8)) & 1u) |
-                       (slice_scale_bits<FMT, D>(vs, rb + 1, dq, r, (gmask >> (2 * c + 9)) & 1u) << 16);
-  const uint32_t b0 = hmul2uu(lds32(prow + 2 * c), hmul2uu(d01, f2k));
-  const uint32_t b1 = hmul2uu(lds32(prow + 2 * c + 8), hmul2uu(d89, f2k));
-  constexpr uint32_t kM1032 = 0xE408E408u, kM72 = 0xD480D480u, kM1152 = 0xE480E480u;  // -offsets
-  if constexpr (C::kQ4) {
-    // matrix 0: rows s0 .. s0 + 7, matrix 1: rows s0 + 8 .. s0 + 15; chunk dq
-    const int row = s0 + (lane & 15);
-    uint32_t x0, x1;
-    ldsm_x2_trans(vc + row * C::CROW + ((dq ^ swz<FMT, D>(row)) << 4), x0, x1);
-    const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
-    mma16816(acc[0], hadd2u((x0 & 0x000F000Fu) | kMagic, kM1032), hadd2u((x0 & 0x00F000F0u) | kMagic64, kM72),
-             hadd2u((x1 & 0x000F000Fu) | kMagic, kM1032), hadd2u((x1 & 0x00F000F0u) | kMagic64, kM72), b0, b1);
-    mma16816(acc[1], hadd2u((y0 & 0x000F000Fu) | kMagic, kM1032), hadd2u((y0 & 0x00F000F0u) | kMagic64, kM72),
-             hadd2u((y1 & 0x000F000Fu) | kMagic, kM1032), hadd2u((y1 & 0x00F000F0u) | kMagic64, kM72), b0, b1);
-  } else {
-    // matrix i: rows s0 + 8 (i & 1) .., chunk 2 dq + (i >> 1)
-    const int mi = lane >> 3;
-    const int row = s0 + 8 * (mi & 1) + (lane & 7);
+  constexpr int NCH = C::CROW / 16;  // 16-byte chunks per row
+  constexpr int NW = C::NBLK / 2;    // 32-bit scale words (two blocks each) per row
+  const int c = lane & 3;
+  uint32_t ws[4][NW];  // scale words of rows s0 + {2c, 2c + 1, 2c + 8, 2c + 9}
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int slot = 2 * c + (q & 1) + 8 * (q >> 1);
+    const uint32_t* sr = reinterpret_cast<const uint32_t*>(scales + (s0 + slot) * C::SROW);
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ws[q][w] = slot < n_valid ? sr[w] : 0u;
+  }
+  uint32_t b0[C::NBLK], b1[C::NBLK];
+#pragma unroll
+  for (int blk = 0; blk < C::NBLK; ++blk) {
+    const uint32_t sel = (blk & 1) ? 0x7632u : 0x5410u;
+    b0[blk] = h2_as_u32(__hmul2(u32_as_h2(p01), u32_as_h2(prmt(ws[0][blk >> 1], ws[1][blk >> 1], sel))));
+    b1[blk] = h2_as_u32(__hmul2(u32_as_h2(p89), u32_as_h2(prmt(ws[2][blk >> 1], ws[3][blk >> 1], sel))));
+  }
+  auto sub = [](uint32_t x, uint32_t neg) { return h2_as_u32(__hadd2(u32_as_h2(x), u32_as_h2(neg))); };
+  constexpr uint32_t kM1032 = 0xE408E408u, kM72 = 0xD480D480u, kM1152 = 0xE480E480u;  // fp16 pairs
+  // two chunks per matrix load: matrix i = (rows s0 + 8 (i & 1) .., chunk cb + (i >> 1)),
+  // so R[j][h] = chunk cb + j, rows 2c, 2c + 1 (+ 8 h)
+  const int mi = lane >> 3;
+  const int row = s0 + 8 * (mi & 1) + (lane & 7);
+  const uint8_t* rp = codes + row * C::CROW;
+  const int sw = swz<FMT, D>(row);
+#pragma unroll
+  for (int cb = 0; cb < NCH; cb += 2) {
     uint32_t R[2][2];
-    ldsm_x4_trans(vc + row * C::CROW + (((2 * dq + (mi >> 1)) ^ swz<FMT, D>(row)) << 4), R[0][0], R[0][1],
-                  R[1][0], R[1][1]);
+    ldsm_x4_trans(rp + (((cb + (mi >> 1)) ^ sw) << 4), R[0][0], R[0][1], R[1][0], R[1][1]);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-      const uint32_t x0 = R[j][0] ^ 0x80808080u, x1 = R[j][1] ^ 0x80808080u;
-      mma16816(acc[j], hadd2u(prmt(x0, 0x64646464u, 0x4240u), kM1152), hadd2u(prmt(x0, 0x64646464u, 0x4341u), kM1152),
-               hadd2u(prmt(x1, 0x64646464u, 0x4240u), kM1152), hadd2u(prmt(x1, 0x64646464u, 0x4341u), kM1152), b0, b1);
+      const int ch = cb + j;
+      if constexpr (C::kQ4) {
+        const uint32_t x0 = R[j][0], x1 = R[j][1], y0 = x0 >> 8, y1 = x1 >> 8;
+        mma16816(acc[2 * ch], sub((x0 & 0x000F000Fu) | kMagic, kM1032), sub((x0 & 0x00F000F0u) | kMagic64, kM72),
+                 sub((x1 & 0x000F000Fu) | kMagic, kM1032), sub((x1 & 0x00F000F0u) | kMagic64, kM72), b0[ch], b1[ch]);
+        mma16816(acc[2 * ch + 1], sub((y0 & 0x000F000Fu) | kMagic, kM1032), sub((y0 & 0x00F000F0u) | kMagic64, kM72),
+                 sub((y1 & 0x000F000Fu) | kMagic, kM1032), sub((y1 & 0x00F000F0u) | kMagic64, kM72), b0[ch], b1[ch]);
+      } else {
+        const uint32_t x0 = R[j][0] ^ 0x80808080u, x1 = R[j][1] ^ 0x80808080u;
+        mma16816(acc[ch], sub(prmt(x0, 0x64646464u, 0x4240u), kM1152), sub(prmt(x0, 0x64646464u, 0x4341u), kM1152),
+                 sub(prmt(x1, 0x64646464u, 0x4240u), kM1152), sub(prmt(x1, 0x64646464u, 0x4341u), kM1152),
+                 b0[ch >> 1], b1[ch >> 1]);
+      }
     }
   }
 }
 
-// lut4 / nvfp4: the nibbles are looked up (centroids / E2M1 values) into fp16 pairs of
-// the two positions and multiplied by the positions' scales; B = p.
+// Per block, k = the smallest exponent >= 0 with d 2^-k < 2 over the tile's first n rows,
+// and those scale rows multiplied by 2^-k in place (exact).  Warp-wide; every row is one
+// lane's (rows lane and lane + 32).
 template <int FMT, int D>
-__device__ __forceinline__ void v_slice_lut(const uint8_t* __restrict__ vc, const uint8_t* __restrict__ vs,
-                                            const __half* __restrict__ prow, int s0, uint32_t gmask,
-                                            int dq, int lane, const Lut& lut, float (&acc)[2][4]) {
+__device__ __forceinline__ void tile_mag_normalize(uint8_t* scales, int n, int lane, int (&k)[Cfg<FMT, D>::NBLK]) {
   using C = Cfg<FMT, D>;
-  const int r = lane >> 2, c = lane & 3;
-  const int ra = s0 + 2 * c, rb = ra + 8;
-  const uint32_t sab = slice_scale_bits<FMT, D>(vs, ra, dq, r, (gmask >> (2 * c)) & 1u) |
-                       (slice_scale_bits<FMT, D>(vs, ra + 1, dq, r, (gmask >> (2 * c + 1)) & 1u) << 16);
-  const uint32_t scd = slice_scale_bits<FMT, D>(vs, rb, dq, r, (gmask >> (2 * c + 8)) & 1u) |
-                       (slice_scale_bits<FMT, D>(vs, rb + 1, dq, r, (gmask >> (2 * c + 9)) & 1u) << 16);
-  const uint32_t b0 = lds32(prow + 2 * c), b1 = lds32(prow + 2 * c + 8);
-  const int row = s0 + (lane & 15);
-  uint32_t x[2];
-  ldsm_x2_trans(vc + row * C::CROW + ((dq ^ swz<FMT, D>(row)) << 4), x[0], x[1]);
-  // e[h][i]: dim 4r + i of positions (2c + 8h, 2c + 8h + 1) as an fp16 pair
-  uint32_t e[2][4];
+  constexpr int NW = C::NBLK / 2;
+  uint32_t mx[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mx[w] = 0u;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint32_t La, Ha, Lb, Hb;
-    lut_lookup4(lut, x[h], nib_mask_lo(x[h]), La, Ha);
-    lut_lookup4(lut, x[h] >> 16, nib_mask_hi(x[h]), Lb, Hb);
-    const uint32_t ta01 = prmt(La, Ha, 0x5140u), tb01 = prmt(Lb, Hb, 0x5140u);
-    const uint32_t ta23 = prmt(La, Ha, 0x7362u), tb23 = prmt(Lb, Hb, 0x7362u);
-    const uint32_t s = h ? scd : sab;
-    e[h][0] = hmul2uu(prmt(ta01, tb01, 0x5410u), s);
-    e[h][1] = hmul2uu(prmt(ta01, tb01, 0x7632u), s);
-    e[h][2] = hmul2uu(prmt(ta23, tb23, 0x5410u), s);
-    e[h][3] = hmul2uu(prmt(ta23, tb23, 0x7632u), s);
+    const int row = lane + 32 * h;
+    if (row < n) {
+      const uint32_t* sr = reinterpret_cast<const uint32_t*>(scales + row * C::SROW);
+#pragma unroll
+      for (int w = 0; w < NW; ++w)  // |d| (scales are >= 0 but may be -0)
+        mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(sr[w] & 0x7FFF7FFFu)));
+    }
   }
-  mma16816(acc[0], e[0][0], e[0][1], e[1][0], e[1][1], b0, b1);
-  mma16816(acc[1], e[0][2], e[0][3], e[1][2], e[1][3], b0, b1);
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(__shfl_xor_sync(0xffffffffu, mx[w], o))));
+  bool any = false;
+  uint32_t f[NW];
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int e0 = (mx[w] >> 10) & 31, e1 = (mx[w] >> 26) & 31;  // fp16 exponent fields
+    k[2 * w] = min(14, max(0, e0 - 15));
+    k[2 * w + 1] = min(14, max(0, e1 - 15));
+    any |= (k[2 * w] | k[2 * w + 1]) != 0;
+    f[w] = ((uint32_t)(15 - k[2 * w]) << 10) | ((uint32_t)(15 - k[2 * w + 1]) << 26);  // 2^-k
+  }
+  if (any) {  // (warp-uniform) typical data needs no rescaling
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int row = lane + 32 * h;
+      if (row < n) {
+        uint32_t* sr = reinterpret_cast<uint32_t*>(scales + row * C::SROW);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) sr[w] = h2_as_u32(__hmul2(u32_as_h2(sr[w]), u32_as_h2(f[w])));
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// lut4 / nvfp4: thread (r, c) dequantizes dims E r .. E r + E - 1 of rows 2c, 2c + 1 and
+// 2c + 8, 2c + 9 into fp16 pairs (centroid / E2M1 lookups) times the rows' scales; B = p.
+template <int FMT, int D>
+__device__ __forceinline__ void vg_lut(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                       int s0, int n_valid, uint32_t p01, uint32_t p89, int lane, const Lut& lut,
+                                       float (&acc)[Cfg<FMT, D>::MT][4]) {
+  using C = Cfg<FMT, D>;
+  const int r = lane >> 2, c = lane & 3;
+  const int sa = 2 * c, sc = sa + 8;
+  auto code = [&](int slot) -> const uint8_t* {
+    const int row = s0 + slot, o = C::RAWB * r;
+    return codes + row * C::CROW + (((o >> 4) ^ swz<FMT, D>(row)) << 4) + (o & 15);
+  };
+  auto scale = [&](int slot) -> __half {
+    if (slot >= n_valid) return __ushort_as_half(0);
+    const uint8_t* srow = scales + (s0 + slot) * C::SROW;
+    if constexpr (C::kNv)  // E4M3 block scale of this thread's dims times the vector scale
+      return __float2half_rn(e4m3_float(srow[(C::E * r) / 16]) * *reinterpret_cast<const float*>(srow + D / 16));
+    return *reinterpret_cast<const __half*>(srow);
+  };
+  const __half2 dab = __halves2half2(scale(sa), scale(sa + 1));
+  const __half2 dcd = __halves2half2(scale(sc), scale(sc + 1));
+  uint32_t wa[C::NWORD], wb[C::NWORD], wc[C::NWORD], wd[C::NWORD];
+  v_raw<FMT, D>(code(sa), wa);
+  v_raw<FMT, D>(code(sa + 1), wb);
+  v_raw<FMT, D>(code(sc), wc);
+  v_raw<FMT, D>(code(sc + 1), wd);
+  uint32_t eab[C::E], ecd[C::E];
+  v_dequant_pair<FMT, D>(wa, wb, lut, eab);
+  v_dequant_pair<FMT, D>(wc, wd, lut, ecd);
+#pragma unroll
+  for (int e = 0; e < C::E; ++e) {
+    eab[e] = h2_as_u32(__hmul2(u32_as_h2(eab[e]), dab));
+    ecd[e] = h2_as_u32(__hmul2(u32_as_h2(ecd[e]), dcd));
+  }
+#pragma unroll
+  for (int mt = 0; mt < C::MT; ++mt)
+    mma16816(acc[mt], eab[2 * mt], eab[2 * mt + 1], ecd[2 * mt], ecd[2 * mt + 1], p01, p89);
+}
+
+// An 8x8 matrix of 16-bit elements held one row pair per lane (lane (r, c): row r,
+// columns 2c, 2c + 1), transposed: lane (r, c) gets row 2c and 2c + 1 of column r.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Named barrier among `count` threads (a multiple of 32): arrive without waiting / wait.
+__device__ __forceinline__ void named_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -230,8 +299,6 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
                const __grid_constant__ CUtensorMap tmv) {
   using C = Cfg<FMT, D>;
   const DecodeArgs& a = pr.a;
-  constexpr int NDQ = D / 32;           // 32-dim slices
-  constexpr int NPQ = kVW / NDQ;        // position sets of the V pass
   constexpr int CODE = kTile * C::CROW; // code bytes of one staged tile
   constexpr int SC = kTile * C::SROW;   // scale bytes of one staged tile
   constexpr int kQfWords = 2 * C::KSTEPS + (C::kLut ? 2 * C::KSTEPS : 0) + 2 * C::NBLK;
@@ -239,10 +306,9 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   extern __shared__ __align__(1024) uint8_t smem2_raw[];
   __shared__ __align__(8) uint64_t kbar[kNW], vbar[kNW];
   __shared__ float red_m[kNW][8], red_l[kNW][8];
-  __shared__ unsigned long long kmask[kNW];
-  __shared__ int cnt_skip[kNW];
+  __shared__ int cnt_skip[kNW], cnt_keep[kNW];
   __shared__ float mh_s[8], share_s[8];
-  __shared__ int misc[4];  // 0: clamped length, 1: exchange ok, 2: tag
+  __shared__ int misc[4];  // 0: clamped length, 1: exchange ok, 2: tag, 3: warps holding accumulators
   __shared__ uint32_t qfr[kQfWords * 32];
 
   uint8_t* sm = smem2_raw + ((1024u - (smem_u32(smem2_raw) & 1023u)) & 1023u);
@@ -250,8 +316,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   uint8_t* kscale = sm + pr.off_kscale;
   uint8_t* vcode = sm + pr.off_vcode;    // == kcode when V goes into the K slots
   uint8_t* vscale = sm + pr.off_vscale;
-  __half* pw = reinterpret_cast<__half*>(sm + pr.off_pw);       // [8][LP] weights x 2^14
-  float* red_o = reinterpret_cast<float*>(sm + pr.off_redo);   // [NPQ][8][D]
+  float* ostage = reinterpret_cast<float*>(sm + pr.off_ostage);  // [8][D] this unit's output rows
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
@@ -259,7 +324,6 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   const int hkv = a.desc.num_kv_heads, G = a.group, P = a.desc.page_size, Ls = a.split_tokens;
   const int B = a.batch, Hq = a.num_q_heads;
   const int NT = Ls / kTile;            // tiles per unit
-  const int LP = pr.lp;                 // weight-matrix row stride (halves)
   const int NCU = a.max_splits;
   const int total = B * NCU * hkv;
   const int cap = min(a.max_seq_len, a.max_pages * P);
@@ -281,12 +345,14 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   // from global memory before the preceding grid has completed.
   grid_dependents_launch();
   grid_dependency_wait();
-  if (tid == 0) {  // every CTA takes part in the launch count that tags the exchange
-    const unsigned long long ep = epoch_read(a.epoch);
+  // every CTA takes part in the launch count that tags the exchange; the read is in
+  // flight while the first unit's copies are issued (its value is stored before B0)
+  unsigned long long ep_raw = 0;
+  if (tid == 32) {
+    ep_raw = epoch_read(a.epoch);
     epoch_advance(a.epoch);
-    misc[2] = (int)epoch_tag(ep);
   }
-  __syncthreads();  // mbarriers initialized, tag known
+  __syncthreads();  // mbarriers initialized
   Lut lut;
   if constexpr (C::kLut) {
 #pragma unroll
@@ -327,23 +393,29 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     const int t0 = cu * Ls;
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;
 
-    // ---- copies: lane 0 of warp w issues tile w (positions that exist in memory)
+    // ---- small loads first (a load issued behind the bulk copies waits for them): the
+    //      query words (warp 0) and the sequence length (warp 1)
+    QRaw<D> qraw;
+    if (warp == 0)
+      load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr, a.desc.signs, c,
+                         qraw);
+    int n_raw = 0;
+    if (warp == 1 && lane == 0) n_raw = __ldg(a.seq_lens + b);
+    // ---- K copies: lane 0 of warp w issues tile w (positions that exist in memory; a
+    //      tile past the sequence's end is copied speculatively and left unused)
     int row0 = -1;
     bool k_issued = false, v_issued = false;
     if (warp < NT) {
       if (lane == 0) {
         const int tok0 = t0 + warp * kTile;
-        uint32_t kbytes = 0, vbytes = 0;
+        uint32_t kbytes = 0;
         if (tok0 < cap) {
           const int lp = tok0 / P, off = tok0 - lp * P;  // tiles never straddle pages (P % 64 == 0)
           const int page = a.page_table ? __ldg(a.page_table + (size_t)b * a.max_pages + lp)
                                         : b * a.max_pages + lp;
-          if (page >= 0 && page < a.desc.num_pages) {
+          if (page >= 0 && page < a.desc.num_pages) {  // else flagged below if it holds positions
             row0 = (page * hkv + kvh) * P + off;
             kbytes = CODE + SC;
-            if (v_sep) vbytes = CODE + SC;
-          } else {
-            set_flag(flags, KVQ_FLAG_BAD_PAGE);
           }
         }
         fence_proxy_async();
@@ -352,38 +424,20 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
           tma_rows(kcode + warp * CODE, &tmk, row0, &kbar[warp]);
           bulk_copy(kscale + warp * SC, kscales_g + (size_t)row0 * C::SROW, SC, &kbar[warp]);
         }
-        if (v_sep) {
-          mbar_expect_tx(&vbar[warp], vbytes);
-          if (vbytes) {
-            tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
-            bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
-          }
-        }
       }
       row0 = __shfl_sync(0xffffffffu, row0, 0);
       k_issued = row0 >= 0;
       v_issued = v_sep && k_issued;
     }
-    // ---- the sequence length; split 0 clears the output rows the splits add into
-    if (warp == 1) {
-      if (lane == 0) {
-        const int n = __ldg(a.seq_lens + b);
-        if (n < 0 || n > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
-        misc[0] = max(0, min(n, cap));
-        misc[1] = 1;
-      }
-      if (add_merge && cu == 0) {
-        float4* orow = reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D);
-        for (int i = lane; i < G * D / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        __syncwarp();
-        if (lane == 0) flag_set_release(a.zflag + (size_t)b * hkv + kvh, (uint32_t)misc[2]);
-      }
+    if (warp == 1 && lane == 0) {
+      if (n_raw < 0 || n_raw > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
+      misc[0] = max(0, min(n_raw, cap));
+      misc[1] = 1;
+      misc[3] = 0;
+      if (k == 0) misc[2] = (int)epoch_tag(ep_raw);
     }
     // ---- query fragments, built once for the CTA by warp 0
     if (warp == 0) {
-      QRaw<D> qraw;
-      load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr, a.desc.signs, c,
-                         qraw);
       uint32_t qf[C::KSTEPS][2], ql[C::KSTEPS][2];
       float corr[C::NBLK][2];
       build_query<FMT, D>(qraw, c, qf, ql, corr);
@@ -405,6 +459,23 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
     }
     __syncthreads();  // B0: query fragments, length
+    // ---- V copies when V tiles come with K: issued after every K copy of the CTA, so the
+    //      K tiles land first
+    if (v_sep && warp < NT && lane == 0) {
+      const uint32_t vbytes = k_issued ? CODE + SC : 0;
+      mbar_expect_tx(&vbar[warp], vbytes);
+      if (vbytes) {
+        tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+        bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+      }
+    }
+    // ---- split 0 clears the output rows that the splits add their shares into
+    if (warp == 1 && add_merge && cu == 0) {
+      float4* orow = reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D);
+      for (int i = lane; i < G * D / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncwarp();
+      if (lane == 0) flag_set_release(a.zflag + (size_t)b * hkv + kvh, (uint32_t)misc[2]);
+    }
     const int nb = misc[0];
     const uint32_t tag = (uint32_t)misc[2];
     const int n_tok = max(0, min(Ls, nb - t0));
@@ -495,10 +566,10 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       mh1 = __shfl_sync(0xffffffffu, m, 2 * c + 1);
       if (warp == 0 && lane < 8) mh_s[lane] = m;
     }
-    float inv_L0 = 1.f, inv_L1 = 1.f;  // sequence-wide option: weights already final
     if (a.global_max) {
       // every split publishes (m, l relative to m); the poll warp derives the final
-      // maximum M and denominator L of every head; the weights below use M
+      // maximum M and denominator L of every head; the weights below use M, and this
+      // split's share of the output is 1 / L
       float l0 = 0.f, l1 = 0.f;
       if (has_tile) {
 #pragma unroll
@@ -543,52 +614,50 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (misc[1]) {
         mh0 = mh_s[2 * c < G ? 2 * c : 0];
         mh1 = mh_s[2 * c + 1 < G ? 2 * c + 1 : 0];
-        inv_L0 = share_s[2 * c < G ? 2 * c : 0];
-        inv_L1 = share_s[2 * c + 1 < G ? 2 * c + 1 : 0];
       }
     }
-    (void)inv_L0;
-    (void)inv_L1;
+    // In-kernel merge without the sequence-wide maximum: the tile owners hand their
+    // denominators to the poll warp through a named barrier and go on with their V pass;
+    // the poll warp publishes (m, l) and collects every split's while they work.
+    const bool publish = add_merge && !a.global_max && n_tok > 0;
+    const int pub_count = 32 * (NT == kNW ? kNW : NT + 1);
 
-    // ---- weights, skip test, row masks (and the gathers of kept V rows)
+    // ---- weights, skip test and V pass of this warp's own tile
     if (warp < NT) {
       float l0 = 0.f, l1 = 0.f;
       int nskip = 0;
-      unsigned long long tmask = 0ull;
-      __half* pcol = pw + warp * kTile;
+      uint32_t gk = 0;          // groups (16-row jobs) with a kept pair
+      uint32_t p01[4], p89[4];  // B fragments of the weights (fp16 x 2^14), per group
+      unsigned long long rows = 0ull;
       if (has_tile) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (16 * j < nvalid) {
-            const int ra = 16 * j + r, rb = ra + 8;
-            const bool va = ra < nvalid, vb = rb < nvalid;
-            const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
-            const float da0 = s[j][0] - mh0, da1 = s[j][1] - mh1;
-            const float db0 = s[j][2] - mh0, db1 = s[j][3] - mh1;
-            const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
-            const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
-            l0 += ea0 + eb0;
-            l1 += ea1 + eb1;
-            const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
-            const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
-            nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
-            const __half2 pa = __floats2half2_rn(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f);
-            const __half2 pb = __floats2half2_rn(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f);
-            pcol[(2 * c) * LP + ra] = __low2half(pa);
-            pcol[(2 * c + 1) * LP + ra] = __high2half(pa);
-            pcol[(2 * c) * LP + rb] = __low2half(pb);
-            pcol[(2 * c + 1) * LP + rb] = __high2half(pb);
-            // rows any head keeps: row r from the lanes of row r, then all 16 rows of the job
+          const int ra = 16 * j + r, rb = ra + 8;
+          const bool va = ra < nvalid, vb = rb < nvalid;
+          const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
+          const float da0 = s[j][0] - mh0, da1 = s[j][1] - mh1;
+          const float db0 = s[j][2] - mh0, db1 = s[j][3] - mh1;
+          const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
+          const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
+          l0 += ea0 + eb0;
+          l1 += ea1 + eb1;
+          const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
+          const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
+          nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
+          // the kept weights as the V MMA's B fragments: rows 0-7 / 8-15 of the group,
+          // transposed from (row r, heads 2c, 2c + 1) to (rows 2c, 2c + 1, head r)
+          p01[j] = movmatrix_trans(pack_h2(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f));
+          p89[j] = movmatrix_trans(pack_h2(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f));
+          gk |= (__any_sync(0xffffffffu, ka0 || ka1 || kb0 || kb1) ? 1u : 0u) << j;
+          if (!v_tma || a.stats) {  // rows any head keeps (the rows to gather; V rows needed)
             const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
             const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
-            const uint32_t mine = c == 0 ? ((((rows_a >> (4 * r)) & 1u) << r) | (((rows_b >> (4 * r)) & 1u) << (r + 8)))
-                                         : 0u;
-            tmask |= (unsigned long long)__reduce_or_sync(0xffffffffu, mine) << (16 * j);
+            const uint32_t mine =
+                c == 0 ? ((((rows_a >> (4 * r)) & 1u) << r) | (((rows_b >> (4 * r)) & 1u) << (r + 8))) : 0u;
+            rows |= (unsigned long long)__reduce_or_sync(0xffffffffu, mine) << (16 * j);
           }
         }
       }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -598,122 +667,96 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         red_l[warp][2 * c] = l0;
         red_l[warp][2 * c + 1] = l1;
       }
-      if (lane == 0) {
-        kmask[warp] = tmask;
-        cnt_skip[warp] = nskip;
+      if (a.stats) {
+#pragma unroll
+        for (int o = 16; o; o >>= 1) nskip += __shfl_xor_sync(0xffffffffu, nskip, o);
+        if (lane == 0) {
+          cnt_skip[warp] = nskip;
+          cnt_keep[warp] = __popcll(rows);
+        }
       }
-      if (!v_tma && tmask) {
-        // gather the kept rows into this tile's V slot: codes with the tile's chunk
-        // swizzle, and the rows' scales (lut4: the aligned pair holding the norm)
-        uint8_t* dst = vcode + warp * CODE;
-        uint8_t* dsc = vscale + warp * SC;
+      if (publish && warp != kPollWarp) named_arrive(1, pub_count);  // l is in shared memory
+
+      uint8_t* vc = (v_sep ? vcode : kcode) + warp * CODE;
+      uint8_t* vs = (v_sep ? vscale : kscale) + warp * SC;
+      if (!v_tma && rows) {
+        // gather the kept rows into this warp's (now free) K slot: codes with the tile's
+        // chunk swizzle, and the rows' scales (lut4: the aligned pair holding the norm)
         const uint8_t* src = vcodes_g + (size_t)row0 * C::CROW;
         const uint8_t* ssrc = vscales_g + (size_t)row0 * C::SROW;
         constexpr int CPR = C::CROW / 16;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int i = lane + 32 * h;
-          if ((tmask >> i) & 1ull) {
+          if ((rows >> i) & 1ull) {
 #pragma unroll
             for (int cc = 0; cc < CPR; ++cc)
-              cp_async16(dst + i * C::CROW + ((cc ^ swz<FMT, D>(i)) << 4), src + (size_t)i * C::CROW + cc * 16);
-            if constexpr (C::SROW == 16) cp_async16(dsc + i * 16, ssrc + (size_t)i * 16);
-            else if constexpr (C::SROW == 8) cp_async8(dsc + i * 8, ssrc + (size_t)i * 8);
-            else cp_async4(dsc + (i & ~1) * 2, ssrc + (size_t)(i & ~1) * 2);
+              cp_async16(vc + i * C::CROW + ((cc ^ swz<FMT, D>(i)) << 4), src + (size_t)i * C::CROW + cc * 16);
+            if constexpr (C::SROW == 16) cp_async16(vs + i * 16, ssrc + (size_t)i * 16);
+            else if constexpr (C::SROW == 8) cp_async8(vs + i * 8, ssrc + (size_t)i * 8);
+            else if constexpr (C::SROW == 4) cp_async4(vs + i * 4, ssrc + (size_t)i * 4);
+            else cp_async4(vs + (i & ~1) * 2, ssrc + (size_t)(i & ~1) * 2);  // 2-byte rows: the pair
+            static_assert(C::SROW == 16 || C::SROW == 8 || C::SROW == 4 || C::SROW == 2, "scale row");
           }
         }
         cp_async_commit();
+        cp_async_wait<0>();
+        __syncwarp();
       }
-    }
-    __syncthreads();  // B2: weights, row masks, denominators
-
-    // ---- publish (m, l) for the in-kernel merge, or write the partial's (m, l)
-    if (tid < G && n_tok > 0) {
-      float l = 0.f;
-      for (int w = 0; w < NT; ++w) l += red_l[w][tid];
-      if (add_merge) {
-        // the sequence-wide maximum made the weights final already
-        if (!a.global_max) xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mh_s[tid], l);
-      } else {  // (sequence-wide maximum: M, and l relative to M)
-        a.part_m[slot0 + (size_t)tid * a.max_splits] = mh_s[tid];
-        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
-      }
-    }
-    if (tid == 32 && a.stats && n_tok > 0) {
-      int ns = 0, nk = 0;
-      for (int w = 0; w < NT; ++w) {
-        ns += cnt_skip[w];
-        nk += __popcll(kmask[w]);
-      }
-      atomicAdd(&a.stats[0], (unsigned long long)n_tok * G);
-      atomicAdd(&a.stats[1], (unsigned long long)ns);
-      atomicAdd(&a.stats[2], (unsigned long long)nk);
-      atomicAdd(&a.stats[3], (unsigned long long)(n_tok - nk));
-    }
-    if (!v_tma) {
-      cp_async_wait<0>();
-      __syncthreads();  // B3: every gathered row is in place
-    }
-
-    // ---- V pass (dim slice dq, position set pq) / exchange poll
-    if (warp < kVW && n_tok > 0) {
-      const int dq = warp % NDQ, pq = warp / NDQ;
-      float acc[2][4];
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      int kcur = 0;  // mag formats: B carries d 2^-kcur
-#pragma unroll 1
-      for (int t = pq; t < NT; t += NPQ) {
-        const unsigned long long km = kmask[t];
-        if (!km) continue;
-        if (v_tma && !mbar_wait(&vbar[t], ph)) {
-          if (lane == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
-          mbar_wait(&vbar[t], ph);
-          continue;
-        }
-        const uint8_t* vc = vcode + t * CODE;
-        const uint8_t* vs = vscale + t * SC;
-        const __half* prow = pw + r * LP + t * kTile;
-        if constexpr (C::kMag) {
-          // the largest kept scale of this block in the tile sets k (it only grows)
-          const uint32_t e0 = ((km >> lane) & 1ull) ? lds16(vs + lane * C::SROW + 2 * dq) & 0x7FFFu : 0u;
-          const uint32_t e1 = ((km >> (lane + 32)) & 1ull) ? lds16(vs + (lane + 32) * C::SROW + 2 * dq) & 0x7FFFu : 0u;
-          const uint32_t emax = __reduce_max_sync(0xffffffffu, max(e0, e1));
-          const int kt = min(14, max(0, (int)(emax >> 10) - 15));
-          if (kt > kcur) {
-            const float f = __int_as_float((127 + kcur - kt) << 23);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) acc[mt][i] *= f;
-            kcur = kt;
+      bool v_waited = false;
+      if (gk) {
+        if (v_tma) {
+          v_waited = true;
+          if (!mbar_wait(&vbar[warp], ph)) {
+            if (lane == 0) set_flag(flags, KVQ_FLAG_TIMEOUT);
+            mbar_wait(&vbar[warp], ph);  // the copy must not be left in flight
           }
-          const uint32_t f2k = ((uint32_t)(15 - kcur) << 10) * 0x10001u;  // fp16 2^-kcur, both halves
+        }
+        float acc[C::MT][4];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t gm = (uint32_t)(km >> (16 * g)) & 0xFFFFu;
-            if (gm) v_slice_mag<FMT, D>(vc, vs, prow + 16 * g, 16 * g, gm, dq, lane, f2k, acc);
+        for (int mt = 0; mt < C::MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        if constexpr (C::kMag) {
+          int kx[C::NBLK];
+          tile_mag_normalize<FMT, D>(vs, nvalid, lane, kx);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if ((gk >> j) & 1u) vg_mag<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), p01[j], p89[j], lane, acc);
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt) {
+            const float f = __int_as_float((127 + kx[mt >> 1]) << 23) * kPUnscale;  // undo 2^-k, 2^14
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][i] *= f;
           }
         } else {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t gm = (uint32_t)(km >> (16 * g)) & 0xFFFFu;
-            if (gm) v_slice_lut<FMT, D>(vc, vs, prow + 16 * g, 16 * g, gm, dq, lane, lut, acc);
-          }
+          for (int j = 0; j < 4; ++j)
+            if ((gk >> j) & 1u)
+              vg_lut<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), p01[j], p89[j], lane, lut, acc);
+#pragma unroll
+          for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][i] *= kPUnscale;
         }
+        // the accumulators go to this warp's K code slot (its V data is read: same warp)
+        __syncwarp();
+        float* accw = reinterpret_cast<float*>(kcode + warp * CODE);
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) accw[(mt * 4 + i) * 32 + lane] = acc[mt][i];
+        if (lane == 0) atomicOr(&misc[3], 1 << warp);
       }
-      const float fin = __int_as_float((127 + kcur) << 23) * kPUnscale;
-      float* ro = red_o + (size_t)pq * 8 * D;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int h = 2 * c + (i & 1);
-          ro[h * D + slice_dim<FMT, D>(dq, mt, r, i)] = acc[mt][i] * fin;
-        }
-    } else if (warp == kPollWarp && add_merge && !a.global_max && n_tok > 0) {
-      // this split's share of each head, 2^(m_s - M) / L, once split 0 has cleared the
-      // output rows and every split of the (sequence, KV head) has published
+      if (v_issued && !v_waited) mbar_wait(&vbar[warp], ph);  // no copy stays in flight
+    }
+    if (warp == kPollWarp && publish) {
+      // publish this split's (m, l), then wait for split 0's cleared output rows and for
+      // every split's (m, l): this split's share of each head is 2^(m_s - M) / L
+      named_sync(1, pub_count);
+      if (lane < G) {
+        float l = 0.f;
+        for (int w = 0; w < NT; ++w) l += red_l[w][lane];
+        xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, mh_s[lane], l);
+      }
       bool ok = true;
       if (lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -739,11 +782,53 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         misc[1] = 0;
       }
     }
-    // no copy of this unit stays in flight past the end of the unit
-    if (v_issued && warp < NT && !kmask[warp]) mbar_wait(&vbar[warp], ph);
-    __syncthreads();  // B4: the slices' partial sums, the shares
+    __syncthreads();  // B4: accumulators, denominators, shares
 
-    // ---- this split's contribution
+    // ---- this split's contribution: the warps' accumulators summed (four consecutive
+    //      lanes' entries per thread), scaled by the share, staged as [head][dim]
+    if (n_tok > 0) {
+      if (!add_merge && tid < G) {
+        float l = 0.f;
+        for (int w = 0; w < NT; ++w) l += red_l[w][tid];
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mh_s[tid];  // (sequence-wide maximum: M)
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+      }
+      if (tid == 32 && a.stats) {
+        int ns = 0, nk = 0;
+        for (int w = 0; w < NT; ++w) {
+          if (w * kTile < n_tok) {
+            ns += cnt_skip[w];
+            nk += cnt_keep[w];
+          }
+        }
+        atomicAdd(&a.stats[0], (unsigned long long)n_tok * G);
+        atomicAdd(&a.stats[1], (unsigned long long)ns);
+        atomicAdd(&a.stats[2], (unsigned long long)nk);
+        atomicAdd(&a.stats[3], (unsigned long long)(n_tok - nk));
+      }
+      const uint32_t wk = (uint32_t)misc[3];
+      for (int q4 = tid; q4 < 8 * C::NE; q4 += kNT) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int w = 0; w < NT; ++w)
+          if ((wk >> w) & 1u) {
+            const float4 x = reinterpret_cast<const float4*>(kcode + w * CODE)[q4];
+            v[0] += x.x;
+            v[1] += x.y;
+            v[2] += x.z;
+            v[3] += x.w;
+          }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int q = 4 * q4 + t;
+          const int ln = q & 31, e = q >> 5;
+          const int mt = e >> 2, i = e & 3;
+          const int h = 2 * (ln & 3) + (i & 1);
+          ostage[h * D + out_dim<FMT, D>(ln >> 2, mt, i)] = add_merge && h < G ? v[t] * share_s[h] : v[t];
+        }
+      }
+    }
+    __syncthreads();
     if (n_tok > 0) {
       constexpr int Q4 = D / 4;
       if (add_merge) {
@@ -752,15 +837,9 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
             // rotate back (R^T = diag(s) c H), one warp per head, then add
             if (warp < G) {
               constexpr int K = D / 32;
-              const float sh = share_s[warp];
               float y[K];
 #pragma unroll
-              for (int kk = 0; kk < K; ++kk) {
-                float v = 0.f;
-#pragma unroll
-                for (int q = 0; q < NPQ; ++q) v += red_o[((size_t)q * 8 + warp) * D + 32 * kk + lane];
-                y[kk] = v * sh;
-              }
+              for (int kk = 0; kk < K; ++kk) y[kk] = ostage[warp * D + 32 * kk + lane];
 #pragma unroll
               for (int hb = 1; hb < 32; hb <<= 1) {
                 const bool upper = (lane & hb) != 0;
@@ -786,39 +865,16 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
                 atomicAdd(dst + 32 * kk + lane, y[kk] * cs * (float)a.desc.signs[32 * kk + lane]);
             }
           } else {
-            for (int e = tid; e < G * Q4; e += kNT) {
-              const int h = e / Q4, d4 = e - h * Q4;
-              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-              for (int q = 0; q < NPQ; ++q) {
-                const float4 x = reinterpret_cast<const float4*>(red_o + ((size_t)q * 8 + h) * D)[d4];
-                v.x += x.x;
-                v.y += x.y;
-                v.z += x.z;
-                v.w += x.w;
-              }
-              const float sh = share_s[h];
-              v.x *= sh;
-              v.y *= sh;
-              v.z *= sh;
-              v.w *= sh;
-              red_add_f32x4(a.out + ((size_t)b * Hq + (size_t)kvh * G + h) * D + 4 * d4, v);
-            }
+            for (int e = tid; e < G * Q4; e += kNT)
+              red_add_f32x4(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D + 4 * e,
+                            reinterpret_cast<const float4*>(ostage)[e]);
           }
         }
       } else {
         for (int e = tid; e < G * Q4; e += kNT) {
           const int h = e / Q4, d4 = e - h * Q4;
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int q = 0; q < NPQ; ++q) {
-            const float4 x = reinterpret_cast<const float4*>(red_o + ((size_t)q * 8 + h) * D)[d4];
-            v.x += x.x;
-            v.y += x.y;
-            v.z += x.z;
-            v.w += x.w;
-          }
-          reinterpret_cast<float4*>(a.part_o + (slot0 + (size_t)h * a.max_splits) * D)[d4] = v;
+          reinterpret_cast<float4*>(a.part_o + (slot0 + (size_t)h * a.max_splits) * D)[d4] =
+              reinterpret_cast<const float4*>(ostage)[e];
         }
       }
     }
@@ -865,6 +921,7 @@ constexpr size_t kStaticReserve = 8192;
 template <int FMT, int D>
 struct Plan {
   using C = Cfg<FMT, D>;
+  static_assert(kTile * C::CROW >= C::NE * 32 * 4, "a warp's accumulators fit its K code slot");
   static constexpr size_t CODE = kTile * C::CROW, SC = kTile * C::SROW;
   // byte offsets for a unit of nt tiles; v_sep: V tiles get their own region
   static size_t layout(int nt, bool v_sep, Decode2Params* p) {
@@ -883,11 +940,8 @@ struct Plan {
       p->off_vcode = p->off_kcode;
       p->off_vscale = p->off_kscale;
     }
-    p->lp = nt * kTile + 8;
-    p->off_pw = (uint32_t)o;
-    o = up(o + (size_t)8 * p->lp * 2, 128);
-    p->off_redo = (uint32_t)o;
-    o += (size_t)(kVW / (D / 32)) * 8 * D * 4;
+    p->off_ostage = (uint32_t)o;
+    o += (size_t)8 * D * 4;
     return o + 1024;  // slack for aligning the base to 1024
   }
 };

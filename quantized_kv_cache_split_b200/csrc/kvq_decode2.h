@@ -11,9 +11,7 @@ struct Decode2Params {
   DecodeArgs a;
   uint32_t off_kcode, off_kscale;  // K tiles: codes (swizzled), scale rows
   uint32_t off_vcode, off_vscale;  // V tiles (== the K tiles' offsets when V reuses them)
-  uint32_t off_pw;                 // weights x 2^14, fp16 [8 heads][lp]
-  uint32_t off_redo;               // V-pass partial sums, fp32 [position sets][8][head_dim]
-  int lp;                          // weight row stride in halves (positions + 8)
+  uint32_t off_ostage;             // one unit's output rows, fp32 [8 heads][head_dim]
   int v_tma;                       // V tiles copied whole (else only the kept rows, gathered)
   int v_sep;                       // V tiles in their own region, copied together with K
 };

@@ -51,6 +51,7 @@ namespace {
 constexpr int kNW = 16;              // warps per CTA: warp w owns tile w of the unit
 constexpr int kNT = 32 * kNW;
 constexpr int kPollWarp = kNW - 1;   // collects the exchange during the V pass
+constexpr int kPollSleepNs = 32;     // back-off between polls of the exchange
 static_assert(kNW * kTile == KVQ_MAX_SPLIT_TOKENS, "one tile per warp per split");
 
 // ------------------------------------------------------------------ mbarriers, bulk copies
@@ -429,6 +430,19 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       k_issued = row0 >= 0;
       v_issued = v_sep && k_issued;
     }
+    // ---- V copies when V tiles come with K: issued after every K copy of the CTA, so the
+    //      K tiles land first
+    if (v_sep) {
+      __syncthreads();
+      if (warp < NT && lane == 0) {
+        const uint32_t vbytes = k_issued ? CODE + SC : 0;
+        mbar_expect_tx(&vbar[warp], vbytes);
+        if (vbytes) {
+          tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+          bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+        }
+      }
+    }
     if (warp == 1 && lane == 0) {
       if (n_raw < 0 || n_raw > cap) set_flag(flags, KVQ_FLAG_BAD_SEQLEN);
       misc[0] = max(0, min(n_raw, cap));
@@ -459,17 +473,9 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
     }
     __syncthreads();  // B0: query fragments, length
-    // ---- V copies when V tiles come with K: issued after every K copy of the CTA, so the
-    //      K tiles land first
-    if (v_sep && warp < NT && lane == 0) {
-      const uint32_t vbytes = k_issued ? CODE + SC : 0;
-      mbar_expect_tx(&vbar[warp], vbytes);
-      if (vbytes) {
-        tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
-        bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
-      }
-    }
-    // ---- split 0 clears the output rows that the splits add their shares into
+    // ---- split 0 clears the output rows that the splits add their shares into and raises
+    //      their flag with release semantics; whoever adds waits for it with acquire
+    //      semantics (a wait that is long over by then)
     if (warp == 1 && add_merge && cu == 0) {
       float4* orow = reinterpret_cast<float4*>(a.out + ((size_t)b * Hq + (size_t)kvh * G) * D);
       for (int i = lane; i < G * D / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -598,7 +604,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         const int h = lane >> 2, j = lane & 3;
         float M, L;
         bool ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
-                                 j, 4, nsplit, h < G, tag, M, L);
+                                 j, 4, nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {
           xch_combine(M, L, 2);
           if (j == 0 && h < G) {
@@ -765,7 +771,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         const int h = lane >> 2, j = lane & 3;
         float M, L;
         ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits, j, 4,
-                            nsplit, h < G, tag, M, L);
+                            nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {
           xch_combine(M, L, 2);
           if (j == 0 && h < G) share_s[h] = ex2(mh_s[h] - M) / L;

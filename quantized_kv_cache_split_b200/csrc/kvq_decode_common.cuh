@@ -298,7 +298,8 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
 template <int T>
 __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int step, int n,
                                            bool active, uint32_t tag, float& M, float& L,
-                                           long long limit = kWaitCycles) {
+                                           long long limit = kWaitCycles, int sleep_ns = 32,
+                                           bool acquire_first = false) {
   M = -INFINITY;
   L = 0.f;
   for (int ub = 0; ub < n; ub += T * step) {
@@ -311,11 +312,13 @@ __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int s
         const int u = ub + first + step * t;
         mv[t] = -INFINITY;
         lv[t] = 0.f;
-        if (active && u < n) all &= xch_load(e + u, tag, mv[t], lv[t]);
+        if (active && u < n)
+          all &= (acquire_first && u == 0) ? xch_load_acquire(e, tag, mv[t], lv[t])
+                                           : xch_load(e + u, tag, mv[t], lv[t]);
       }
       if (__all_sync(0xffffffffu, all)) break;
       if (__any_sync(0xffffffffu, clock64() - t0 > limit)) return false;
-      __nanosleep(32);
+      __nanosleep(sleep_ns);
     }
     float bm = M;
 #pragma unroll

@@ -44,7 +44,7 @@ METRIC = "decode-attn µs/token & achieved KV HBM GB/s at 32K ctx, sparse-V vs d
 UNIT = "us/token"
 L2_BYTES = 126 * 1024 * 1024
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_traffic.json")
-DECODE_SRC = os.path.join(ROOT, "quantized_kv_cache_split_b200", "csrc", "kvq_decode.cu")
+DECODE_SRC = os.path.join(ROOT, "quantized_kv_cache_split_b200", "csrc", "kvq_decode2.cu")
 
 
 # ------------------------------------------------------------------ distributed plumbing

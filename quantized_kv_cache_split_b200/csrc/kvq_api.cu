@@ -76,12 +76,12 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
     // about one split per CTA slot of the device if every sequence were max_seq_len
     // long (clusters of 4 CTAs when the splits share their running maximum)
     const int64_t pairs = (int64_t)std::max(batch, 1) * desc->num_kv_heads;
-    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode_cluster_capacity(desc->fmt, desc->head_dim, 4) : 0;
+    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode2_capacity(desc->fmt, desc->head_dim, 4) : 0;
     int64_t ctas_per_pair;  // splits of one (sequence, KV head) that run at once
     if (cap4 > 0) {
       ctas_per_pair = 4 * std::max<int64_t>(1, cap4 / pairs);
     } else {
-      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim);
+      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim, 1);
       if (cap1 <= 0) return KVQ_ERR_CUDA;
       ctas_per_pair = std::max<int64_t>(1, cap1 / pairs);
     }
@@ -100,7 +100,7 @@ int resolve_cluster(const kvq_cache_desc* desc, int max_seq_len, int L, uint32_t
                     int* cs_out, int* cap_out) {
   int CS = (options & KVQ_OPT_SHARED_MAX) ? cluster_for(max_splits_for(std::max(max_seq_len, 1), L)) : 1;
   for (; CS >= 1; CS >>= 1) {
-    const int cap = decode_cluster_capacity(desc->fmt, desc->head_dim, CS);
+    const int cap = decode2_capacity(desc->fmt, desc->head_dim, CS);
     if (cap > 0) {
       *cs_out = CS;
       *cap_out = cap;
@@ -246,13 +246,8 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
     return KVQ_OK;
   }
   int CS = 1, capacity = 0;
-  if (options & KVQ_OPT_SHARED_MAX) {
-    st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
-    if (st != KVQ_OK) return st;
-  } else {
-    capacity = decode2_capacity(desc->fmt, desc->head_dim);
-    if (capacity <= 0) return KVQ_ERR_CUDA;
-  }
+  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
+  if (st != KVQ_OK) return st;
   DecodeArgs a;
   a.desc = *desc;
   a.q = q;
@@ -299,24 +294,16 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.v_early = (options & KVQ_OPT_V_WITH_K)      ? 1
               : (options & KVQ_OPT_V_KEPT_ONLY) ? 0
                                                 : desc->fmt != KVQ_FMT_NVFP4;
-  // The merge: inside the decode kernel when every split has its own CTA (the splits add
-  // their shares) or splits share a cluster (the cluster merges, the last one to finish
-  // a (sequence, KV head) merges the clusters' partials); otherwise the partials go to the
-  // workspace and the combine kernel merges them, one CTA per (sequence, query head),
-  // which measured faster than the last finisher of each (sequence, KV head) merging alone.
-  const bool combine_after = out && CS == 1 && groups > capacity;
-  if (options & KVQ_OPT_SHARED_MAX) {
-    // clusters of splits sharing one running maximum: the cluster kernel
-    if (combine_after) a.out = nullptr;
-    st = launch_decode(a, static_cast<cudaStream_t>(stream));
-  } else {
-    // the streaming kernel merges in-kernel when every split has its own CTA, else it
-    // writes the partials for the combine kernel
-    st = launch_decode2(a, static_cast<cudaStream_t>(stream));
-  }
+  // The merge: inside the decode kernel when every group of splits has its own CTAs at
+  // once (the splits exchange (m, l) and add their shares into the output); otherwise every
+  // split writes its partial to the workspace and the combine kernel merges them, one CTA
+  // per (sequence, query head), which measured faster than the last finisher of each
+  // (sequence, KV head) merging alone.
+  const bool combine_after = out && groups > capacity;
+  st = launch_decode2(a, static_cast<cudaStream_t>(stream));
   if (st != KVQ_OK || !combine_after) return st;
-  return launch_combine(*desc, workspace, batch, num_q_heads, max_seq_len, L, CS, a.max_splits, seq_lens,
-                        out, static_cast<cudaStream_t>(stream));
+  return launch_combine(*desc, workspace, batch, num_q_heads, max_seq_len, L, a.max_splits, seq_lens, out,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch,
@@ -332,10 +319,7 @@ int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch
   if (st != KVQ_OK) return st;
   if (max_splits_for(max_seq_len, L) > KVQ_MAX_SPLITS) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;
-  int CS = 1, capacity = 0;
-  st = resolve_cluster(desc, max_seq_len, L, options, &CS, &capacity);
-  if (st != KVQ_OK) return st;
-  return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L, CS,
+  return launch_combine(*desc, workspace, batch, num_q_heads, std::max(max_seq_len, 0), L,
                         max_splits_for(max_seq_len, L), seq_lens, out,
                         static_cast<cudaStream_t>(stream));
 }

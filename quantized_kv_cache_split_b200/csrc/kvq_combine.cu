@@ -2,8 +2,7 @@
 //   M = max_s m_s,  out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
 // (m is kept in log2 units by the decode kernel).  For the rotated lut4 format
 // the merged vector is rotated back: out = s .* (c * H * out').
-// The decode kernel leaves one partial per cluster of `cluster` consecutive splits, so
-// sequence b has ceil(ceil(n_b / L) / cluster) partials.
+// The decode kernel leaves one partial per split, so sequence b has ceil(n_b / L) of them.
 // One CTA of 512 threads per (sequence, query head): the partial maxima and weights
 // are computed one partial per thread, then 512/head_dim thread groups each sum a
 // share of the partials with several loads in flight, and the groups are added.
@@ -20,7 +19,7 @@ constexpr int kMaxCombineSplits = KVQ_MAX_SPLITS;  // splits per sequence merged
 template <int D, bool ROT>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_kernel(const uint8_t* __restrict__ ws, int batch, int hq, int max_seq_len,
-               int split_tokens, int cluster, int max_splits, const int32_t* __restrict__ seq_lens,
+               int split_tokens, int max_splits, const int32_t* __restrict__ seq_lens,
                const int8_t* __restrict__ signs, float* __restrict__ out) {
   constexpr int kGroups = kCombineThreads / D;  // thread groups splitting the split range
   __shared__ float wsh[kMaxCombineSplits];
@@ -36,7 +35,7 @@ combine_kernel(const uint8_t* __restrict__ ws, int batch, int hq, int max_seq_le
   const float* m = o + n_part * D;
   const float* l = m + n_part;
   const int n = max(0, min(seq_lens[b], max_seq_len));
-  const int ns = ((n + split_tokens - 1) / split_tokens + cluster - 1) / cluster;
+  const int ns = (n + split_tokens - 1) / split_tokens;
   const size_t u0 = (size_t)bh * max_splits;
   // 1. maxima and weights: one split per thread (strided), loads all in flight
   float M = -INFINITY;
@@ -123,8 +122,7 @@ combine_kernel(const uint8_t* __restrict__ ws, int batch, int hq, int max_seq_le
 }  // namespace
 
 int launch_combine(const kvq_cache_desc& desc, const void* workspace, int batch, int num_q_heads,
-                   int max_seq_len, int split_tokens, int cluster, int max_splits,
-                   const int32_t* seq_lens, float* out, cudaStream_t stream) {
+                   int max_seq_len, int split_tokens, int max_splits, const int32_t* seq_lens, float* out, cudaStream_t stream) {
   const int64_t blocks = (int64_t)batch * num_q_heads;
   if (blocks <= 0) return KVQ_OK;
   if (blocks > 0x7fffffffLL) return KVQ_ERR_UNSUPPORTED;
@@ -133,7 +131,7 @@ int launch_combine(const kvq_cache_desc& desc, const void* workspace, int batch,
   const bool rot = desc.fmt == KVQ_FMT_LUT4;
 #define KVQ_COMBINE(DIM, ROT)                                                            \
   combine_kernel<DIM, ROT><<<(unsigned)blocks, kCombineThreads, 0, stream>>>(            \
-      ws, batch, num_q_heads, max_seq_len, split_tokens, cluster, max_splits, seq_lens,  \
+      ws, batch, num_q_heads, max_seq_len, split_tokens, max_splits, seq_lens,           \
       desc.signs, out)
   if (desc.head_dim == 128) {
     if (rot) KVQ_COMBINE(128, true); else KVQ_COMBINE(128, false);

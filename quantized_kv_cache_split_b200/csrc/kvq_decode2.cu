@@ -99,18 +99,6 @@ __device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-__device__ __forceinline__ void ldsm_x2_trans(const void* p, uint32_t& d0, uint32_t& d1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(d0), "=r"(d1)
-               : "r"(smem_u32(p))
-               : "memory");
-}
-__device__ __forceinline__ uint32_t hadd2u(uint32_t a, uint32_t b) {
-  return h2_as_u32(__hadd2(u32_as_h2(a), u32_as_h2(b)));
-}
-__device__ __forceinline__ uint32_t hmul2uu(uint32_t a, uint32_t b) {
-  return h2_as_u32(__hmul2(u32_as_h2(a), u32_as_h2(b)));
-}
 
 // ------------------------------------------------------------------ V groups
 // The V pass of a warp covers its own tile, all of the head dimension, one group of 16
@@ -308,7 +296,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   __shared__ __align__(8) uint64_t kbar[kNW], vbar[kNW];
   __shared__ float red_m[kNW][8], red_l[kNW][8];
   __shared__ int cnt_skip[kNW], cnt_keep[kNW];
-  __shared__ float mh_s[8], share_s[8];
+  __shared__ float mh_s[8], mc_s[8], share_s[8];  // split maximum, the one the skip test uses
   __shared__ int misc[4];  // 0: clamped length, 1: exchange ok, 2: tag, 3: warps holding accumulators
   __shared__ uint32_t qfr[kQfWords * 32];
 
@@ -318,6 +306,9 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   uint8_t* vcode = sm + pr.off_vcode;    // == kcode when V goes into the K slots
   uint8_t* vscale = sm + pr.off_vscale;
   float* ostage = reinterpret_cast<float*>(sm + pr.off_ostage);  // [8][D] this unit's output rows
+  float4* sscore = reinterpret_cast<float4*>(sm + pr.off_score);  // [warps][4 jobs][32 lanes] scores
+  uint32_t* pword = reinterpret_cast<uint32_t*>(sm + pr.off_pword);  // [warps][4 groups][2][32] B fragments
+  int* s_pre = reinterpret_cast<int*>(sm + pr.off_units);  // [batch + 1] units before sequence b
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = lane >> 2, c = lane & 3;
@@ -326,7 +317,14 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   const int B = a.batch, Hq = a.num_q_heads;
   const int NT = Ls / kTile;            // tiles per unit
   const int NCU = a.max_splits;
-  const int total = B * NCU * hkv;
+  // Thread-block clusters of CS consecutive splits of one (sequence, KV head) share one
+  // running maximum (the skip test and the weights of every split of the group use the
+  // maximum over the group's scores); CTA `rank` of the cluster takes split g CS + rank of
+  // the group g it is on.  CS = 1: every split on its own.
+  const int CS = a.cluster;
+  const int rank = CS > 1 ? (int)cluster_rank() : 0;
+  const int NG = (NCU + CS - 1) / CS;  // groups of splits per (sequence, KV head)
+  const int total = B * NG * hkv;
   const int cap = min(a.max_seq_len, a.max_pages * P);
   const bool add_merge = a.out != nullptr && a.group_merge;
   const bool v_tma = pr.v_tma != 0;     // V tiles copied whole (with K, or right after it)
@@ -380,17 +378,59 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     for (int i = 0; i < 4; ++i) lut.lo[i] = lut.hi[i] = 0u;
   }
 
+  // Multi-round launches take only the units that exist (sequence-major: the splits of
+  // sequence 0, then of sequence 1, ...; every KV head of a split in turn), so that every
+  // CTA gets the same number of them; a single-round launch has one unit per CTA in the
+  // static order (split-major) and a unit past its sequence's end exits at once.
+  int total_units = total;
+  if (pr.dense_units) {
+    if (warp == 0) {
+      int carry = 0;
+      for (int b0 = 0; b0 < B; b0 += 32) {
+        const int bb = b0 + lane;
+        const int n = bb < B ? max(0, min(__ldg(a.seq_lens + bb), cap)) : 0;
+        int v = (n + Ls - 1) / Ls * hkv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += y;
+        }
+        if (bb < B) s_pre[bb + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) s_pre[0] = 0;
+    }
+    __syncthreads();
+    total_units = s_pre[B];
+  }
+
   const __half* qg = static_cast<const __half*>(a.q);
   const uint8_t* kscales_g = static_cast<const uint8_t*>(a.k_scales);
   const uint8_t* vcodes_g = static_cast<const uint8_t*>(a.v_codes);
   const uint8_t* vscales_g = static_cast<const uint8_t*>(a.v_scales);
 
+  const int it0 = CS > 1 ? (int)blockIdx.x / CS : (int)blockIdx.x;
+  const int it_step = CS > 1 ? (int)gridDim.x / CS : (int)gridDim.x;
 #pragma unroll 1
-  for (int it = blockIdx.x, k = 0; it < total; it += gridDim.x, ++k) {
+  for (int it = it0, k = 0; it < total_units; it += it_step, ++k) {
     const uint32_t ph = (uint32_t)k & 1u;  // mbarrier phase of this unit
-    const int kvh = it % hkv;
-    const int b = (it / hkv) % B;
-    const int cu = it / (hkv * B);
+    int kvh, b, cu;
+    if (pr.dense_units) {
+      int lo = 0, hi = B;  // the sequence b with s_pre[b] <= it < s_pre[b + 1]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_pre[mid] <= it) lo = mid;
+        else hi = mid;
+      }
+      b = lo;
+      const int rem = it - s_pre[b];
+      cu = rem / hkv;
+      kvh = rem - cu * hkv;
+    } else {
+      kvh = it % hkv;
+      b = (it / hkv) % B;
+      cu = (it / (hkv * B)) * CS + rank;
+    }
     const int t0 = cu * Ls;
     const size_t slot0 = ((size_t)b * Hq + (size_t)kvh * G) * a.max_splits + cu;
 
@@ -489,10 +529,10 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     const bool has_tile = nvalid > 0 && k_issued;
     if (nvalid > 0 && !k_issued && lane == 0) set_flag(flags, KVQ_FLAG_BAD_PAGE);
 
-    // ---- K pass
-    float s[4][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
+    // ---- K pass (the four 16-row jobs in a loop, not unrolled: every warp runs this code
+    //      once per unit, so its size is what the instruction cache sees); the scores go
+    //      to the warp's scratch, invalid rows as -inf
+    float4* scw = sscore + warp * 4 * 32 + lane;
     float mx0 = -INFINITY, mx1 = -INFINITY;
     bool k_waited = false;
     if (has_tile) {
@@ -517,20 +557,19 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
       const uint8_t* kc = kcode + warp * CODE;
       const uint8_t* ks_ = kscale + warp * SC;
-#pragma unroll
+#pragma unroll 1
       for (int j = 0; j < 4; ++j) {
-        s[j][0] = s[j][1] = s[j][2] = s[j][3] = -INFINITY;
+        float4 sv = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
         if (16 * j < nvalid) {
           float t[4];
           k_job_scores<FMT, D>(kc, ks_, 16 * j + r, qf, ql, corr, lut, c, t);
           const bool va = 16 * j + r < nvalid, vb = 16 * j + r + 8 < nvalid;
-          s[j][0] = va ? t[0] * qk_scale : -INFINITY;
-          s[j][1] = va ? t[1] * qk_scale : -INFINITY;
-          s[j][2] = vb ? t[2] * qk_scale : -INFINITY;
-          s[j][3] = vb ? t[3] * qk_scale : -INFINITY;
-          mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][2]));
-          mx1 = fmaxf(mx1, fmaxf(s[j][1], s[j][3]));
+          sv = make_float4(va ? t[0] * qk_scale : -INFINITY, va ? t[1] * qk_scale : -INFINITY,
+                           vb ? t[2] * qk_scale : -INFINITY, vb ? t[3] * qk_scale : -INFINITY);
+          mx0 = fmaxf(mx0, fmaxf(sv.x, sv.z));
+          mx1 = fmaxf(mx1, fmaxf(sv.y, sv.w));
         }
+        scw[j * 32] = sv;
       }
     }
     if (k_issued && !k_waited) mbar_wait(&kbar[warp], ph);  // a speculative tile past the end
@@ -571,6 +610,21 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       mh0 = __shfl_sync(0xffffffffu, m, 2 * c);
       mh1 = __shfl_sync(0xffffffffu, m, 2 * c + 1);
       if (warp == 0 && lane < 8) mh_s[lane] = m;
+      if (CS > 1) {
+        // the maximum over the cluster's splits: every CTA's maxima are written before the
+        // cluster barrier, read from distributed shared memory after it; the arrive after
+        // the reads lets each CTA know, at the end of the unit, that nobody reads its
+        // maxima any more
+        cluster_sync();
+        for (int rk = 0; rk < CS; ++rk) {
+          if (rk == rank) continue;
+          mh0 = fmaxf(mh0, dsmem_ld(dsmem_addr(mh_s + 2 * c, rk)));
+          mh1 = fmaxf(mh1, dsmem_ld(dsmem_addr(mh_s + 2 * c + 1, rk)));
+          if (lane < 8) m = fmaxf(m, dsmem_ld(dsmem_addr(mh_s + lane, rk)));
+        }
+        cluster_arrive();
+      }
+      if (warp == 0 && lane < 8) mc_s[lane] = m;
     }
     if (a.global_max) {
       // every split publishes (m, l relative to m); the poll warp derives the final
@@ -578,10 +632,11 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       // split's share of the output is 1 / L
       float l0 = 0.f, l1 = 0.f;
       if (has_tile) {
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < 4; ++j) {
-          l0 += ex2(s[j][0] - mh0) + ex2(s[j][2] - mh0);
-          l1 += ex2(s[j][1] - mh1) + ex2(s[j][3] - mh1);
+          const float4 sv = scw[j * 32];  // invalid rows hold -inf
+          l0 += ex2(sv.x - mh0) + ex2(sv.z - mh0);
+          l1 += ex2(sv.y - mh1) + ex2(sv.w - mh1);
         }
       }
 #pragma unroll
@@ -597,7 +652,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (tid < G && n_tok > 0) {
         float l = 0.f;
         for (int w = 0; w < NT; ++w) l += red_l[w][tid];
-        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mh_s[tid], l);
+        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mc_s[tid], l);
       }
       if (warp == kPollWarp && n_tok > 0) {
         const int nsplit = (nb + Ls - 1) / Ls;
@@ -608,7 +663,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         if (ok) {
           xch_combine(M, L, 2);
           if (j == 0 && h < G) {
-            mh_s[h] = M;
+            mc_s[h] = M;
             share_s[h] = 1.f / L;
           }
         } else if (lane == 0) {
@@ -618,8 +673,8 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
       __syncthreads();
       if (misc[1]) {
-        mh0 = mh_s[2 * c < G ? 2 * c : 0];
-        mh1 = mh_s[2 * c + 1 < G ? 2 * c + 1 : 0];
+        mh0 = mc_s[2 * c < G ? 2 * c : 0];
+        mh1 = mc_s[2 * c + 1 < G ? 2 * c + 1 : 0];
       }
     }
     // In-kernel merge without the sequence-wide maximum: the tile owners hand their
@@ -632,17 +687,18 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     if (warp < NT) {
       float l0 = 0.f, l1 = 0.f;
       int nskip = 0;
-      uint32_t gk = 0;          // groups (16-row jobs) with a kept pair
-      uint32_t p01[4], p89[4];  // B fragments of the weights (fp16 x 2^14), per group
+      uint32_t gk = 0;  // groups (16-row jobs) with a kept pair
+      uint32_t* pww = pword + warp * 4 * 64 + lane;  // B fragments of the weights, per group
       unsigned long long rows = 0ull;
       if (has_tile) {
-#pragma unroll
+#pragma unroll 1
         for (int j = 0; j < 4; ++j) {
           const int ra = 16 * j + r, rb = ra + 8;
           const bool va = ra < nvalid, vb = rb < nvalid;
           const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
-          const float da0 = s[j][0] - mh0, da1 = s[j][1] - mh1;
-          const float db0 = s[j][2] - mh0, db1 = s[j][3] - mh1;
+          const float4 sv = scw[j * 32];
+          const float da0 = sv.x - mh0, da1 = sv.y - mh1;
+          const float db0 = sv.z - mh0, db1 = sv.w - mh1;
           const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
           const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
           l0 += ea0 + eb0;
@@ -652,8 +708,8 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
           nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
           // the kept weights as the V MMA's B fragments: rows 0-7 / 8-15 of the group,
           // transposed from (row r, heads 2c, 2c + 1) to (rows 2c, 2c + 1, head r)
-          p01[j] = movmatrix_trans(pack_h2(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f));
-          p89[j] = movmatrix_trans(pack_h2(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f));
+          pww[j * 64] = movmatrix_trans(pack_h2(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f));
+          pww[j * 64 + 32] = movmatrix_trans(pack_h2(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f));
           gk |= (__any_sync(0xffffffffu, ka0 || ka1 || kb0 || kb1) ? 1u : 0u) << j;
           if (!v_tma || a.stats) {  // rows any head keeps (the rows to gather; V rows needed)
             const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
@@ -724,9 +780,10 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         if constexpr (C::kMag) {
           int kx[C::NBLK];
           tile_mag_normalize<FMT, D>(vs, nvalid, lane, kx);
-#pragma unroll
+#pragma unroll 1
           for (int j = 0; j < 4; ++j)
-            if ((gk >> j) & 1u) vg_mag<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), p01[j], p89[j], lane, acc);
+            if ((gk >> j) & 1u)
+              vg_mag<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), pww[j * 64], pww[j * 64 + 32], lane, acc);
 #pragma unroll
           for (int mt = 0; mt < C::MT; ++mt) {
             const float f = __int_as_float((127 + kx[mt >> 1]) << 23) * kPUnscale;  // undo 2^-k, 2^14
@@ -734,10 +791,10 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
             for (int i = 0; i < 4; ++i) acc[mt][i] *= f;
           }
         } else {
-#pragma unroll
+#pragma unroll 1
           for (int j = 0; j < 4; ++j)
             if ((gk >> j) & 1u)
-              vg_lut<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), p01[j], p89[j], lane, lut, acc);
+              vg_lut<FMT, D>(vc, vs, 16 * j, min(16, nvalid - 16 * j), pww[j * 64], pww[j * 64 + 32], lane, lut, acc);
 #pragma unroll
           for (int mt = 0; mt < C::MT; ++mt)
 #pragma unroll
@@ -761,7 +818,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (lane < G) {
         float l = 0.f;
         for (int w = 0; w < NT; ++w) l += red_l[w][lane];
-        xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, mh_s[lane], l);
+        xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, mc_s[lane], l);
       }
       bool ok = true;
       if (lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
@@ -774,7 +831,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
                             nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {
           xch_combine(M, L, 2);
-          if (j == 0 && h < G) share_s[h] = ex2(mh_s[h] - M) / L;
+          if (j == 0 && h < G) share_s[h] = ex2(mc_s[h] - M) / L;
         }
       }
       if (lane == 0 && !ok) {
@@ -796,7 +853,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (!add_merge && tid < G) {
         float l = 0.f;
         for (int w = 0; w < NT; ++w) l += red_l[w][tid];
-        a.part_m[slot0 + (size_t)tid * a.max_splits] = mh_s[tid];  // (sequence-wide maximum: M)
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mc_s[tid];  // (the maximum the weights use)
         a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
       }
       if (tid == 32 && a.stats) {
@@ -885,6 +942,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
     }
     __syncthreads();  // B5: the unit's buffers are free
+    if (CS > 1) cluster_wait();  // every CTA of the cluster is done reading this one's maxima
   }
 }
 
@@ -948,6 +1006,12 @@ struct Plan {
     }
     p->off_ostage = (uint32_t)o;
     o += (size_t)8 * D * 4;
+    p->off_score = (uint32_t)o;  // per warp: 4 jobs x 32 lanes x float4
+    o += (size_t)kNW * 4 * 32 * 16;
+    p->off_pword = (uint32_t)o;  // per warp: 4 groups x 2 x 32 lanes x u32
+    o += (size_t)kNW * 4 * 64 * 4;
+    p->off_units = (uint32_t)o;  // prefix of the units per sequence
+    o += (size_t)(KVQ_MAX_BATCH + 1) * 4;
     return o + 1024;  // slack for aligning the base to 1024
   }
 };
@@ -964,23 +1028,46 @@ int configure2(int dev) {
   return KVQ_OK;
 }
 
+// CTAs (CS = 1) or clusters of CS CTAs of the streaming kernel resident at once on the
+// current device, cached per device and cluster size.
 template <int FMT, int D>
-int capacity2_t() {
-  static int cache[64] = {};  // CTAs resident at once + 1, per device; guarded by g_mu2
+int capacity2_t(int CS) {
+  static int cache[64][4] = {};  // [device][log2 CS] = count + 1; guarded by g_mu2
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int ci = CS == 8 ? 3 : CS == 4 ? 2 : CS == 2 ? 1 : 0;
   std::lock_guard<std::mutex> lock(g_mu2);
-  if (cache[dev] == 0) {
+  if (cache[dev][ci] == 0) {
     if (configure2<FMT, D>(dev) != KVQ_OK) return 0;
     Decode2Params p{};
     const size_t bytes = Plan<FMT, D>::layout(kNW, false, &p);
-    int n = 0, sms = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode2_kernel<FMT, D>, kNT, bytes) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return 0;
-    cache[dev] = n * sms + 1;
+    int n = 0;
+    if (CS == 1) {
+      int sms = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode2_kernel<FMT, D>, kNT, bytes) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+      n *= sms;
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = CS;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(CS * 64, 1, 1);
+      cfg.blockDim = dim3(kNT, 1, 1);
+      cfg.dynamicSmemBytes = bytes;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, decode2_kernel<FMT, D>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+    }
+    cache[dev][ci] = n + 1;
   }
-  return cache[dev] - 1;
+  return cache[dev][ci] - 1;
 }
 
 template <int FMT, int D>
@@ -992,17 +1079,20 @@ int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_mu2);
     if (configure2<FMT, D>(dev) != KVQ_OK) return KVQ_ERR_CUDA;
   }
-  const int cap = capacity2_t<FMT, D>();
+  const int CS = a.cluster;
+  const int cap = capacity2_t<FMT, D>(CS);  // CTAs, or clusters of CS CTAs
   if (cap <= 0) return KVQ_ERR_CUDA;
   Decode2Params p{};
   p.a = a;
   const int nt = a.split_tokens / kTile;
-  const int64_t units = (int64_t)a.batch * a.max_splits * a.desc.num_kv_heads;
-  p.a.grid = (int)std::min<int64_t>(units, cap);
+  const int64_t groups = (int64_t)a.batch * a.desc.num_kv_heads * ((a.max_splits + CS - 1) / CS);
+  p.a.grid = (int)std::min<int64_t>(groups, cap) * CS;
   if (p.a.grid <= 0) return KVQ_OK;
-  // every unit on its own CTA at once: the splits exchange (m, l) and add their shares
-  p.a.group_merge = a.out != nullptr && units <= cap;
-  if (a.global_max && units > cap) return KVQ_ERR_UNSUPPORTED;
+  // every group on its own CTAs at once: the splits exchange (m, l) and add their shares;
+  // otherwise CTAs loop over the units (those that exist, when splits are independent)
+  p.a.group_merge = a.out != nullptr && groups <= cap;
+  p.dense_units = (CS == 1 && groups > cap) ? 1 : 0;
+  if (a.global_max && groups > cap) return KVQ_ERR_UNSUPPORTED;
   // V tiles copied whole: tau = 0 (every row is needed) or when the launch asks; in their
   // own region when shared memory allows, else into the K slots right after the K pass
   const bool whole = !(a.tau > 0.f) || a.v_early;
@@ -1018,8 +1108,15 @@ int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
   if (!code_map(&tmk, a.k_codes, rows, C::CROW) || !code_map(&tmv, a.v_codes, rows, C::CROW))
     return KVQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   int na = 0;
+  if (CS > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = CS;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   const bool coop = p.a.group_merge || a.global_max;
   if (coop) {  // CTAs wait for one another: all resident together
     attr[na].id = cudaLaunchAttributeCooperative;
@@ -1036,7 +1133,7 @@ int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = na;
   cudaError_t e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
-  if (e != cudaSuccess && coop) {  // a driver that does not take both: cooperative alone
+  if (e != cudaSuccess && coop) {  // a driver that does not take both: without PDL
     (void)cudaGetLastError();
     cfg.numAttrs = na - 1;
     e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
@@ -1060,16 +1157,40 @@ int launch_decode2(const DecodeArgs& a, cudaStream_t stream) {
   return KVQ_ERR_UNSUPPORTED;
 }
 
-int decode2_capacity(int f, int d) {
-  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity2_t<KVQ_FMT_Q8_0, 128>();
-  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity2_t<KVQ_FMT_Q8_0, 64>();
-  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity2_t<KVQ_FMT_Q4_0, 128>();
-  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity2_t<KVQ_FMT_Q4_0, 64>();
-  if (f == KVQ_FMT_LUT4 && d == 128) return capacity2_t<KVQ_FMT_LUT4, 128>();
-  if (f == KVQ_FMT_LUT4 && d == 64) return capacity2_t<KVQ_FMT_LUT4, 64>();
-  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity2_t<KVQ_FMT_NVFP4, 128>();
-  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity2_t<KVQ_FMT_NVFP4, 64>();
+int decode2_capacity(int f, int d, int cluster) {
+  if (cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8) return 0;
+  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity2_t<KVQ_FMT_Q8_0, 128>(cluster);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity2_t<KVQ_FMT_Q8_0, 64>(cluster);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity2_t<KVQ_FMT_Q4_0, 128>(cluster);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity2_t<KVQ_FMT_Q4_0, 64>(cluster);
+  if (f == KVQ_FMT_LUT4 && d == 128) return capacity2_t<KVQ_FMT_LUT4, 128>(cluster);
+  if (f == KVQ_FMT_LUT4 && d == 64) return capacity2_t<KVQ_FMT_LUT4, 64>(cluster);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity2_t<KVQ_FMT_NVFP4, 128>(cluster);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity2_t<KVQ_FMT_NVFP4, 64>(cluster);
   return 0;
+}
+
+namespace {
+// The exchange's bounded waits against entries that never become this launch's: the
+// (m, l) poll and the cleared-rows flag wait each give up after `limit` cycles and set
+// KVQ_FLAG_TIMEOUT, as a decode that lost a split would.  The entries are four exchange
+// entries and one flag word in the workspace header's spare bytes (64..143), read only.
+__global__ void selftest_wait_kernel(uint8_t* ws, long long limit) {
+  uint32_t* flags = reinterpret_cast<uint32_t*>(ws);
+  const ulonglong2* e = reinterpret_cast<const ulonglong2*>(ws + 64);
+  const unsigned long long* f = reinterpret_cast<const unsigned long long*>(ws + 128);
+  const uint32_t never = 0xffffffffu;  // no launch reaches this tag
+  float M, L;
+  const bool ok1 = xch_reduce<4>(e, threadIdx.x & 31, 32, 4, true, never, M, L, limit);
+  bool ok2 = true;
+  if ((threadIdx.x & 31) == 0) ok2 = flag_wait_acquire(f, never, limit);
+  if ((threadIdx.x & 31) == 0 && (!ok1 || !ok2)) set_flag(flags, KVQ_FLAG_TIMEOUT);
+}
+}  // namespace
+
+int launch_selftest_wait(void* workspace, long long max_cycles, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(static_cast<uint8_t*>(workspace), max_cycles);
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 }  // namespace kvq

@@ -37,7 +37,7 @@ struct DecodeArgs {
                       // [batch][num_q_heads][max_splits]
   unsigned long long* stats;
   float* out;         // non-null: merge in the same kernel and write the output
-  int cluster;        // consecutive splits per thread-block cluster (1, 2 or 4)
+  int cluster;        // consecutive splits per thread-block cluster (1, 2, 4 or 8)
   int shared_max;     // the splits of a cluster share one running maximum
   int global_max;     // every split of a (sequence, KV head) uses the maximum over all of them
   int grid;           // CTAs launched (a multiple of cluster)
@@ -51,8 +51,7 @@ struct DecodeArgs {
 // Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch
 // counter that tags the exchange entries); the merge flags and counters (u64 flags
 // "output rows cleared" [batch][num_q_heads], then int32 last-arrival counters
-// [batch][num_q_heads], together rounded up to 256 bytes); then, one slot per cluster of
-// splits:
+// [batch][num_q_heads], together rounded up to 256 bytes); then, one slot per split:
 //   (m, l) exchange [batch][num_q_heads][max_splits] 2 x u64, each word a fp32 value
 //   under a 32-bit launch tag (what the splits of a (sequence, KV head) publish to one
 //   another)
@@ -69,13 +68,9 @@ __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
 int launch_quantize(const kvq_cache_desc& desc, const void* x, const void* x2, int n_tok,
                     const int32_t* slots, void* codes, void* scales, void* codes2, void* scales2,
                     cudaStream_t stream);
-int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 int launch_selftest_wait(void* workspace, long long max_cycles, cudaStream_t stream);
-// Clusters of `cluster` CTAs of the decode kernel for (fmt, head_dim) that fit on the
-// current device at once (0 if none); cached per device.
-int decode_cluster_capacity(int fmt, int head_dim, int cluster);
 int launch_combine(const kvq_cache_desc& desc, const void* workspace, int batch, int num_q_heads,
-                   int max_seq_len, int split_tokens, int cluster, int max_splits, const int32_t* seq_lens,
+                   int max_seq_len, int split_tokens, int max_splits, const int32_t* seq_lens,
                    float* out, cudaStream_t stream);
 
 int device_sm_count();

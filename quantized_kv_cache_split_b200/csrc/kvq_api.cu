@@ -76,17 +76,24 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
     // about one split per CTA slot of the device if every sequence were max_seq_len
     // long (clusters of 4 CTAs when the splits share their running maximum)
     const int64_t pairs = (int64_t)std::max(batch, 1) * desc->num_kv_heads;
-    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode2_capacity(desc->fmt, desc->head_dim, 4) : 0;
+    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode2_capacity(desc->fmt, desc->head_dim, 4, KVQ_MAX_SPLIT_TOKENS) : 0;
     int64_t ctas_per_pair;  // splits of one (sequence, KV head) that run at once
     if (cap4 > 0) {
       ctas_per_pair = 4 * std::max<int64_t>(1, cap4 / pairs);
     } else {
-      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim, 1);
+      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim, 1, KVQ_MAX_SPLIT_TOKENS);
       if (cap1 <= 0) return KVQ_ERR_CUDA;
       ctas_per_pair = std::max<int64_t>(1, cap1 / pairs);
     }
     L = (int)std::min<int64_t>((std::max(max_seq_len, 1) + ctas_per_pair - 1) / ctas_per_pair,
                                KVQ_MAX_SPLIT_TOKENS);
+    // More splits than CTAs even at the longest split: the CTAs loop over the units, and
+    // two CTAs of half the size per SM (splits of 8 tiles) overlap one's copies with the
+    // other's arithmetic (measured faster than one CTA of 16 warps looping)
+    const int64_t units = pairs * ((std::max(max_seq_len, 1) + L - 1) / L);
+    if (!(options & (KVQ_OPT_SHARED_MAX | KVQ_OPT_GLOBAL_MAX)) && units > ctas_per_pair * pairs &&
+        L == KVQ_MAX_SPLIT_TOKENS)
+      L = KVQ_MAX_SPLIT_TOKENS / 2;
   }
   L = (L + kTile - 1) / kTile * kTile;
   *L_out = std::max(kTile, std::min(L, KVQ_MAX_SPLIT_TOKENS));
@@ -100,7 +107,7 @@ int resolve_cluster(const kvq_cache_desc* desc, int max_seq_len, int L, uint32_t
                     int* cs_out, int* cap_out) {
   int CS = (options & KVQ_OPT_SHARED_MAX) ? cluster_for(max_splits_for(std::max(max_seq_len, 1), L)) : 1;
   for (; CS >= 1; CS >>= 1) {
-    const int cap = decode2_capacity(desc->fmt, desc->head_dim, CS);
+    const int cap = decode2_capacity(desc->fmt, desc->head_dim, CS, L);
     if (cap > 0) {
       *cs_out = CS;
       *cap_out = cap;

@@ -48,11 +48,11 @@
 namespace kvq {
 namespace {
 
-constexpr int kNW = 16;              // warps per CTA: warp w owns tile w of the unit
-constexpr int kNT = 32 * kNW;
-constexpr int kPollWarp = kNW - 1;   // collects the exchange during the V pass
+// NW warps per CTA (16, 8 or 4): warp w owns tile w of the unit, so a unit holds at most
+// NW tiles, and 16 / NW CTAs share an SM (the register file holds 16 warps of 128).
+constexpr int kMaxNW = 16;
 constexpr int kPollSleepNs = 32;     // back-off between polls of the exchange
-static_assert(kNW * kTile == KVQ_MAX_SPLIT_TOKENS, "one tile per warp per split");
+static_assert(kMaxNW * kTile == KVQ_MAX_SPLIT_TOKENS, "one tile per warp per split");
 
 // ------------------------------------------------------------------ mbarriers, bulk copies
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -62,24 +62,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+// True once the phase with the given parity has completed; a thread whose phase is not complete yet may be suspended (it takes no
+// issue slots) until the phase completes or about `ns` nanoseconds have passed.
+__device__ __forceinline__ bool mbar_try_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
       : "memory");
   return ok != 0;
 }
+constexpr uint32_t kSuspendNs = 1000000;  // one suspension at most (the loop bounds the wait)
 // Wait for the phase with the given parity to complete; false after ~kWaitCycles.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
+  if (mbar_try_suspend(bar, parity, kSuspendNs)) return true;
   const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
+  while (!mbar_try_suspend(bar, parity, kSuspendNs))
     if (clock64() - t0 > kWaitCycles) return false;
   return true;
 }
+
 // Rows y .. y + 63 of a 2-D tensor map (x = 0) into shared memory (swizzled as the map says).
 __device__ __forceinline__ void tma_rows(void* dst, const CUtensorMap* map, int y, uint64_t* bar) {
   asm volatile(
@@ -282,11 +286,14 @@ __device__ __forceinline__ void named_sync(int id, int count) {
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int FMT, int D>
-__global__ void __launch_bounds__(kNT, 1)
+template <int FMT, int D, int NW>
+__global__ void __launch_bounds__(32 * NW, 16 / NW)
 decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__ CUtensorMap tmk,
                const __grid_constant__ CUtensorMap tmv) {
   using C = Cfg<FMT, D>;
+  constexpr int kNW = NW;
+  constexpr int kNT = 32 * NW;
+  constexpr int kPollWarp = NW - 1;  // collects the exchange during the V pass
   const DecodeArgs& a = pr.a;
   constexpr int CODE = kTile * C::CROW; // code bytes of one staged tile
   constexpr int SC = kTile * C::SROW;   // scale bytes of one staged tile
@@ -897,12 +904,13 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (add_merge) {
         if (misc[1]) {
           if constexpr (C::kLut) {
-            // rotate back (R^T = diag(s) c H), one warp per head, then add
-            if (warp < G) {
+            // rotate back (R^T = diag(s) c H), one warp per head in turn, then add
+#pragma unroll 1
+            for (int hh = warp; hh < G; hh += kNW) {
               constexpr int K = D / 32;
               float y[K];
 #pragma unroll
-              for (int kk = 0; kk < K; ++kk) y[kk] = ostage[warp * D + 32 * kk + lane];
+              for (int kk = 0; kk < K; ++kk) y[kk] = ostage[hh * D + 32 * kk + lane];
 #pragma unroll
               for (int hb = 1; hb < 32; hb <<= 1) {
                 const bool upper = (lane & hb) != 0;
@@ -922,7 +930,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
                     y[kk + hb] = u - v;
                   }
               const float cs = D == 64 ? 0.125f : 0.08838834764831845f;
-              float* dst = a.out + ((size_t)b * Hq + (size_t)kvh * G + warp) * D;
+              float* dst = a.out + ((size_t)b * Hq + (size_t)kvh * G + hh) * D;
 #pragma unroll
               for (int kk = 0; kk < K; ++kk)
                 atomicAdd(dst + 32 * kk + lane, y[kk] * cs * (float)a.desc.signs[32 * kk + lane]);
@@ -979,8 +987,11 @@ bool code_map(CUtensorMap* m, const void* base, uint64_t rows, int crow) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemMax = 232448;  // dynamic + static shared memory per CTA on sm_100a
+constexpr size_t kSmemSM = 233472;   // shared memory per SM (1 KB of it reserved per CTA)
 constexpr size_t kStaticReserve = 8192;
+// dynamic + static shared memory of one CTA when 16 / NW CTAs share an SM (a plan that
+// does not fit is still launched, with fewer CTAs per SM: the capacity counts them)
+constexpr size_t smem_budget(int nw) { return kSmemSM / (16 / nw) - 1024; }
 
 template <int FMT, int D>
 struct Plan {
@@ -988,7 +999,7 @@ struct Plan {
   static_assert(kTile * C::CROW >= C::NE * 32 * 4, "a warp's accumulators fit its K code slot");
   static constexpr size_t CODE = kTile * C::CROW, SC = kTile * C::SROW;
   // byte offsets for a unit of nt tiles; v_sep: V tiles get their own region
-  static size_t layout(int nt, bool v_sep, Decode2Params* p) {
+  static size_t layout(int nw, int nt, bool v_sep, Decode2Params* p) {
     auto up = [](size_t x, size_t m) { return (x + m - 1) / m * m; };
     size_t o = 0;
     p->off_kcode = (uint32_t)o;
@@ -1007,21 +1018,21 @@ struct Plan {
     p->off_ostage = (uint32_t)o;
     o += (size_t)8 * D * 4;
     p->off_score = (uint32_t)o;  // per warp: 4 jobs x 32 lanes x float4
-    o += (size_t)kNW * 4 * 32 * 16;
+    o += (size_t)nw * 4 * 32 * 16;
     p->off_pword = (uint32_t)o;  // per warp: 4 groups x 2 x 32 lanes x u32
-    o += (size_t)kNW * 4 * 64 * 4;
+    o += (size_t)nw * 4 * 64 * 4;
     p->off_units = (uint32_t)o;  // prefix of the units per sequence
     o += (size_t)(KVQ_MAX_BATCH + 1) * 4;
     return o + 1024;  // slack for aligning the base to 1024
   }
 };
 
-template <int FMT, int D>
+template <int FMT, int D, int NW>
 int configure2(int dev) {
   static uint64_t done_mask = 0;  // guarded by g_mu2
   if (!(done_mask >> dev & 1)) {
-    if (cudaFuncSetAttribute(decode2_kernel<FMT, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(kSmemMax - kStaticReserve)) != cudaSuccess)
+    if (cudaFuncSetAttribute(decode2_kernel<FMT, D, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(smem_budget(16) - kStaticReserve)) != cudaSuccess)
       return KVQ_ERR_CUDA;
     done_mask |= 1ull << dev;
   }
@@ -1030,7 +1041,7 @@ int configure2(int dev) {
 
 // CTAs (CS = 1) or clusters of CS CTAs of the streaming kernel resident at once on the
 // current device, cached per device and cluster size.
-template <int FMT, int D>
+template <int FMT, int D, int NW>
 int capacity2_t(int CS) {
   static int cache[64][4] = {};  // [device][log2 CS] = count + 1; guarded by g_mu2
   int dev = 0;
@@ -1038,13 +1049,14 @@ int capacity2_t(int CS) {
   const int ci = CS == 8 ? 3 : CS == 4 ? 2 : CS == 2 ? 1 : 0;
   std::lock_guard<std::mutex> lock(g_mu2);
   if (cache[dev][ci] == 0) {
-    if (configure2<FMT, D>(dev) != KVQ_OK) return 0;
+    if (configure2<FMT, D, NW>(dev) != KVQ_OK) return 0;
     Decode2Params p{};
-    const size_t bytes = Plan<FMT, D>::layout(kNW, false, &p);
+    const size_t bytes = Plan<FMT, D>::layout(NW, NW, false, &p);
     int n = 0;
     if (CS == 1) {
       int sms = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode2_kernel<FMT, D>, kNT, bytes) != cudaSuccess ||
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode2_kernel<FMT, D, NW>, 32 * NW, bytes) !=
+              cudaSuccess ||
           cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 0;
       n *= sms;
@@ -1056,11 +1068,11 @@ int capacity2_t(int CS) {
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(CS * 64, 1, 1);
-      cfg.blockDim = dim3(kNT, 1, 1);
+      cfg.blockDim = dim3(32 * NW, 1, 1);
       cfg.dynamicSmemBytes = bytes;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, decode2_kernel<FMT, D>, &cfg) != cudaSuccess) {
+      if (cudaOccupancyMaxActiveClusters(&n, decode2_kernel<FMT, D, NW>, &cfg) != cudaSuccess) {
         (void)cudaGetLastError();
         n = 0;
       }
@@ -1070,17 +1082,17 @@ int capacity2_t(int CS) {
   return cache[dev][ci] - 1;
 }
 
-template <int FMT, int D>
+template <int FMT, int D, int NW>
 int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
   using C = Cfg<FMT, D>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KVQ_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lock(g_mu2);
-    if (configure2<FMT, D>(dev) != KVQ_OK) return KVQ_ERR_CUDA;
+    if (configure2<FMT, D, NW>(dev) != KVQ_OK) return KVQ_ERR_CUDA;
   }
   const int CS = a.cluster;
-  const int cap = capacity2_t<FMT, D>(CS);  // CTAs, or clusters of CS CTAs
+  const int cap = capacity2_t<FMT, D, NW>(CS);  // CTAs, or clusters of CS CTAs
   if (cap <= 0) return KVQ_ERR_CUDA;
   Decode2Params p{};
   p.a = a;
@@ -1096,10 +1108,10 @@ int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
   // V tiles copied whole: tau = 0 (every row is needed) or when the launch asks; in their
   // own region when shared memory allows, else into the K slots right after the K pass
   const bool whole = !(a.tau > 0.f) || a.v_early;
-  size_t bytes = Plan<FMT, D>::layout(nt, whole, &p);
+  size_t bytes = Plan<FMT, D>::layout(NW, nt, whole, &p);
   p.v_sep = whole ? 1 : 0;
-  if (bytes + kStaticReserve > kSmemMax) {
-    bytes = Plan<FMT, D>::layout(nt, false, &p);
+  if (bytes + kStaticReserve > smem_budget(NW)) {
+    bytes = Plan<FMT, D>::layout(NW, nt, false, &p);
     p.v_sep = 0;
   }
   p.v_tma = whole ? 1 : 0;
@@ -1127,46 +1139,66 @@ int launch2_t(const DecodeArgs& a, cudaStream_t stream) {
   attr[na].val.programmaticStreamSerializationAllowed = 1;
   ++na;
   cfg.gridDim = dim3(p.a.grid, 1, 1);
-  cfg.blockDim = dim3(kNT, 1, 1);
+  cfg.blockDim = dim3(32 * NW, 1, 1);
   cfg.dynamicSmemBytes = bytes;
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D, NW>, p, tmk, tmv);
   if (e != cudaSuccess && coop) {  // a driver that does not take both: without PDL
     (void)cudaGetLastError();
     cfg.numAttrs = na - 1;
-    e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D>, p, tmk, tmv);
+    e = cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, D, NW>, p, tmk, tmv);
   }
   if (e != cudaSuccess) return KVQ_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+// Warps per CTA for a split of L positions: one tile per warp, the smallest CTA that
+// holds the split.
+int warps_for(int split_tokens) { return split_tokens <= 4 * kTile ? 4 : split_tokens <= 8 * kTile ? 8 : 16; }
+
+template <int FMT, int D>
+int launch_nw(const DecodeArgs& a, cudaStream_t stream) {
+  const int nw = warps_for(a.split_tokens);
+  if (nw == 4) return launch2_t<FMT, D, 4>(a, stream);
+  if (nw == 8) return launch2_t<FMT, D, 8>(a, stream);
+  return launch2_t<FMT, D, 16>(a, stream);
+}
+
+template <int FMT, int D>
+int capacity_nw(int cluster, int split_tokens) {
+  const int nw = warps_for(split_tokens);
+  if (nw == 4) return capacity2_t<FMT, D, 4>(cluster);
+  if (nw == 8) return capacity2_t<FMT, D, 8>(cluster);
+  return capacity2_t<FMT, D, 16>(cluster);
 }
 
 }  // namespace
 
 int launch_decode2(const DecodeArgs& a, cudaStream_t stream) {
   const int f = a.desc.fmt, d = a.desc.head_dim;
-  if (f == KVQ_FMT_Q8_0 && d == 128) return launch2_t<KVQ_FMT_Q8_0, 128>(a, stream);
-  if (f == KVQ_FMT_Q8_0 && d == 64) return launch2_t<KVQ_FMT_Q8_0, 64>(a, stream);
-  if (f == KVQ_FMT_Q4_0 && d == 128) return launch2_t<KVQ_FMT_Q4_0, 128>(a, stream);
-  if (f == KVQ_FMT_Q4_0 && d == 64) return launch2_t<KVQ_FMT_Q4_0, 64>(a, stream);
-  if (f == KVQ_FMT_LUT4 && d == 128) return launch2_t<KVQ_FMT_LUT4, 128>(a, stream);
-  if (f == KVQ_FMT_LUT4 && d == 64) return launch2_t<KVQ_FMT_LUT4, 64>(a, stream);
-  if (f == KVQ_FMT_NVFP4 && d == 128) return launch2_t<KVQ_FMT_NVFP4, 128>(a, stream);
-  if (f == KVQ_FMT_NVFP4 && d == 64) return launch2_t<KVQ_FMT_NVFP4, 64>(a, stream);
+  if (f == KVQ_FMT_Q8_0 && d == 128) return launch_nw<KVQ_FMT_Q8_0, 128>(a, stream);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return launch_nw<KVQ_FMT_Q8_0, 64>(a, stream);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return launch_nw<KVQ_FMT_Q4_0, 128>(a, stream);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return launch_nw<KVQ_FMT_Q4_0, 64>(a, stream);
+  if (f == KVQ_FMT_LUT4 && d == 128) return launch_nw<KVQ_FMT_LUT4, 128>(a, stream);
+  if (f == KVQ_FMT_LUT4 && d == 64) return launch_nw<KVQ_FMT_LUT4, 64>(a, stream);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return launch_nw<KVQ_FMT_NVFP4, 128>(a, stream);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return launch_nw<KVQ_FMT_NVFP4, 64>(a, stream);
   return KVQ_ERR_UNSUPPORTED;
 }
 
-int decode2_capacity(int f, int d, int cluster) {
+int decode2_capacity(int f, int d, int cluster, int split_tokens) {
   if (cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8) return 0;
-  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity2_t<KVQ_FMT_Q8_0, 128>(cluster);
-  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity2_t<KVQ_FMT_Q8_0, 64>(cluster);
-  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity2_t<KVQ_FMT_Q4_0, 128>(cluster);
-  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity2_t<KVQ_FMT_Q4_0, 64>(cluster);
-  if (f == KVQ_FMT_LUT4 && d == 128) return capacity2_t<KVQ_FMT_LUT4, 128>(cluster);
-  if (f == KVQ_FMT_LUT4 && d == 64) return capacity2_t<KVQ_FMT_LUT4, 64>(cluster);
-  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity2_t<KVQ_FMT_NVFP4, 128>(cluster);
-  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity2_t<KVQ_FMT_NVFP4, 64>(cluster);
+  if (f == KVQ_FMT_Q8_0 && d == 128) return capacity_nw<KVQ_FMT_Q8_0, 128>(cluster, split_tokens);
+  if (f == KVQ_FMT_Q8_0 && d == 64) return capacity_nw<KVQ_FMT_Q8_0, 64>(cluster, split_tokens);
+  if (f == KVQ_FMT_Q4_0 && d == 128) return capacity_nw<KVQ_FMT_Q4_0, 128>(cluster, split_tokens);
+  if (f == KVQ_FMT_Q4_0 && d == 64) return capacity_nw<KVQ_FMT_Q4_0, 64>(cluster, split_tokens);
+  if (f == KVQ_FMT_LUT4 && d == 128) return capacity_nw<KVQ_FMT_LUT4, 128>(cluster, split_tokens);
+  if (f == KVQ_FMT_LUT4 && d == 64) return capacity_nw<KVQ_FMT_LUT4, 64>(cluster, split_tokens);
+  if (f == KVQ_FMT_NVFP4 && d == 128) return capacity_nw<KVQ_FMT_NVFP4, 128>(cluster, split_tokens);
+  if (f == KVQ_FMT_NVFP4 && d == 64) return capacity_nw<KVQ_FMT_NVFP4, 64>(cluster, split_tokens);
   return 0;
 }
 

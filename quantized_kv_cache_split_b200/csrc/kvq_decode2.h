@@ -26,8 +26,9 @@ struct Decode2Params {
 // launches the combine kernel).  KVQ_ERR_UNSUPPORTED for the sequence-wide maximum when
 // the units do not all fit at once.
 int launch_decode2(const DecodeArgs& a, cudaStream_t stream);
-// CTAs (cluster = 1) or clusters of `cluster` (2, 4 or 8) CTAs of the streaming kernel
-// resident at once on the current device (0 on error or if none fits).
-int decode2_capacity(int fmt, int head_dim, int cluster);
+// CTAs (cluster = 1) or clusters of `cluster` (2, 4 or 8) CTAs of the streaming kernel for
+// splits of split_tokens positions resident at once on the current device (0 on error or
+// if none fits).
+int decode2_capacity(int fmt, int head_dim, int cluster, int split_tokens);
 
 }  // namespace kvq

@@ -150,8 +150,11 @@ int kvq_quantize_kv(const kvq_cache_desc* desc, const void* k, const void* v, in
  * kvq_decode_attn and kvq_combine use for a request (same split_tokens and
  * options).  split_tokens > 0 is capped at KVQ_MAX_SPLIT_TOKENS and rounded up to a
  * multiple of 64; split_tokens == 0 picks one from the problem size and how many
- * CTAs (or CTA clusters) of the decode kernel fit on the current device (about one
- * split per CTA slot).
+ * CTAs (or CTA clusters) of the decode kernel fit on the current device: at least 32
+ * splits per (sequence, KV head), more when that leaves SMs idle, splits of at least
+ * 128 positions, and the shortest such length whose splits all run at once (one CTA
+ * each, CTAs of 4, 8 or 16 warps, one per 64-position tile); when even the longest
+ * split leaves more splits than CTAs, splits of 512 positions that the CTAs loop over.
  * Returns L (> 0) or a KVQ_ERR_* code.
  * Sequence b is cut into splits [k*L, min((k+1)*L, seq_len_b)), k = 0, 1, ...
  */
@@ -163,8 +166,8 @@ int32_t kvq_resolve_split(const kvq_cache_desc* desc, int32_t batch, int32_t num
  * head) that one thread-block cluster processes together (same arguments as
  * kvq_resolve_split).  CS = 1 without KVQ_OPT_SHARED_MAX; with it CS is 2 or 4
  * (when sequences are long enough), splits kCS .. kCS + CS - 1 form cluster group k,
- * and the CTAs of a group share one running maximum and merge their partials on
- * chip, so the workspace holds one partial per group.
+ * and the CTAs of a group share one running maximum (exchanged on chip); the
+ * workspace still holds one partial per split.
  */
 int32_t kvq_resolve_cluster(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
                             int32_t max_seq_len, int32_t split_tokens, uint32_t options);
@@ -221,11 +224,11 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                skip test is done (fewest bytes; a second DRAM round trip); with
  *                KVQ_OPT_V_WITH_K every V tile is copied together with its K tile and
  *                the skipped rows are left out of the contraction only (more bytes, no
- *                second round trip).  Neither: V_WITH_K, except KVQ_FMT_NVFP4 (kept rows
- *                only); both measured on B200, where these steps are bound by latency
- *                and the MMA pipe rather than by HBM bytes.  tau = 0 always copies V
- *                with K.  Formats whose staging does not fit shared memory twice
- *                (q8_0 at head_dim 128) copy kept rows only.
+ *                second round trip).  Neither: V_WITH_K (measured faster on B200, where
+ *                these steps are bound by latency and instruction issue rather than by
+ *                HBM bytes).  tau = 0 always copies V with K.  Where K and V tiles do not
+ *                both fit in shared memory (q8_0 at head_dim 128), each V tile is copied
+ *                into its K tile's place as soon as that tile's scores are taken.
  *                KVQ_OPT_GLOBAL_MAX needs every split of the request on its own
  *                CTA at once (KVQ_ERR_UNSUPPORTED otherwise): the CTAs of a (sequence, KV
  *                head) exchange their maxima through the workspace between the K pass
@@ -244,11 +247,8 @@ int kvq_read_device_flags(const void* workspace, uint32_t* flags, void* stream);
  *                log-sum-exp rule of kvq_combine): when every split of the request runs
  *                on its own CTA at once, inside the decode kernel, each split adding its
  *                normalized share into the output with floating-point atomics (so the
- *                last bits of the output may differ from run to run); otherwise, with
- *                clusters of splits (KVQ_OPT_SHARED_MAX and kvq_resolve_cluster > 1),
- *                inside the kernel too, the last cluster to finish a (sequence, KV head)
- *                merging it; otherwise by a second launch on the same stream, the
- *                combine kernel of kvq_combine.  Calls that share a workspace
+ *                last bits of the output may differ from run to run); otherwise by a
+ *                second launch on the same stream, the combine kernel of kvq_combine.  Calls that share a workspace
  *                must not overlap on the GPU.
  * Query head h attends with KV head h / (num_q_heads / num_kv_heads).
  * The group size num_q_heads / num_kv_heads must be 1..KVQ_MAX_GROUP.

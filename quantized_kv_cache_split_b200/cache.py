@@ -87,8 +87,8 @@ class QuantizedKVCache:
         splits of a thread-block cluster) or "sequence" (over all splits of the
         sequence and KV head).  ``v_fetch``: how V rows reach the SM when tau > 0:
         "kept" (only the kept rows, after the skip test), "with_k" (every V tile with its
-        K tile; skipped rows are left out of the contraction only) or "auto" (with_k,
-        except nvfp4: kept); the result is the same."""
+        K tile; skipped rows are left out of the contraction only) or "auto" (with_k);
+        the result is the same."""
         scopes = {"split": 0, "cluster": kb.KVQ_OPT_SHARED_MAX, "sequence": kb.KVQ_OPT_GLOBAL_MAX}
         fetches = {"auto": 0, "kept": kb.KVQ_OPT_V_KEPT_ONLY, "with_k": kb.KVQ_OPT_V_WITH_K}
         if max_scope not in scopes:

@@ -56,6 +56,9 @@ int max_splits_for(int max_seq_len, int split_tokens) {
   return (max_seq_len + split_tokens - 1) / split_tokens;
 }
 
+constexpr int kMinSplits = 32;         // splits per (sequence, KV head) at the least
+constexpr int kMinSplitTokens = 128;   // positions per split at the least (automatic choice)
+
 int cluster_for(int max_splits) { return max_splits >= 4 ? 4 : max_splits >= 2 ? 2 : 1; }
 
 // Split length L of a request (the device is queried only when split_tokens == 0).
@@ -72,28 +75,42 @@ int resolve_split_len(const kvq_cache_desc* desc, int batch, int num_q_heads, in
   int L;
   if (split_tokens > 0) {
     L = std::min(split_tokens, KVQ_MAX_SPLIT_TOKENS);
-  } else {
-    // about one split per CTA slot of the device if every sequence were max_seq_len
-    // long (clusters of 4 CTAs when the splits share their running maximum)
+  } else if (options & KVQ_OPT_SHARED_MAX) {
+    // clusters of 4 splits sharing their running maximum: about one split per CTA slot of
+    // the device if every sequence were max_seq_len long
     const int64_t pairs = (int64_t)std::max(batch, 1) * desc->num_kv_heads;
-    const int cap4 = (options & KVQ_OPT_SHARED_MAX) ? decode2_capacity(desc->fmt, desc->head_dim, 4, KVQ_MAX_SPLIT_TOKENS) : 0;
-    int64_t ctas_per_pair;  // splits of one (sequence, KV head) that run at once
-    if (cap4 > 0) {
-      ctas_per_pair = 4 * std::max<int64_t>(1, cap4 / pairs);
-    } else {
-      const int cap1 = decode2_capacity(desc->fmt, desc->head_dim, 1, KVQ_MAX_SPLIT_TOKENS);
-      if (cap1 <= 0) return KVQ_ERR_CUDA;
-      ctas_per_pair = std::max<int64_t>(1, cap1 / pairs);
-    }
+    const int cap4 = decode2_capacity(desc->fmt, desc->head_dim, 4, KVQ_MAX_SPLIT_TOKENS);
+    const int cap1 = decode2_capacity(desc->fmt, desc->head_dim, 1, KVQ_MAX_SPLIT_TOKENS);
+    if (cap1 <= 0) return KVQ_ERR_CUDA;
+    const int64_t ctas_per_pair = cap4 > 0 ? 4 * std::max<int64_t>(1, cap4 / pairs)
+                                           : std::max<int64_t>(1, cap1 / pairs);
     L = (int)std::min<int64_t>((std::max(max_seq_len, 1) + ctas_per_pair - 1) / ctas_per_pair,
                                KVQ_MAX_SPLIT_TOKENS);
+  } else {
+    // Splits per (sequence, KV head): enough to give every SM a CTA of 16 warps, and at
+    // least kMinSplits (short contexts: more and smaller CTAs, each a shorter chain; the
+    // kernel's CTA follows the split, one warp per tile).  Then the shortest length from
+    // there whose units all fit on the device at once, so that the splits merge inside
+    // the kernel.
+    const int64_t pairs = (int64_t)std::max(batch, 1) * desc->num_kv_heads;
+    const int64_t n = std::max(max_seq_len, 1);
+    const int cap16 = decode2_capacity(desc->fmt, desc->head_dim, 1, KVQ_MAX_SPLIT_TOKENS);
+    if (cap16 <= 0) return KVQ_ERR_CUDA;
+    const int64_t S = std::max<int64_t>(cap16 / pairs, kMinSplits);
+    int64_t l = (n + S - 1) / S;
+    l = std::min<int64_t>(std::max<int64_t>((l + kTile - 1) / kTile * kTile, kMinSplitTokens),
+                          KVQ_MAX_SPLIT_TOKENS);
+    bool fits = false;
+    for (;; l += kTile) {
+      const int cap = decode2_capacity(desc->fmt, desc->head_dim, 1, (int)l);
+      if (cap <= 0) return KVQ_ERR_CUDA;
+      fits = pairs * ((n + l - 1) / l) <= cap;
+      if (fits || l >= KVQ_MAX_SPLIT_TOKENS) break;
+    }
     // More splits than CTAs even at the longest split: the CTAs loop over the units, and
     // two CTAs of half the size per SM (splits of 8 tiles) overlap one's copies with the
     // other's arithmetic (measured faster than one CTA of 16 warps looping)
-    const int64_t units = pairs * ((std::max(max_seq_len, 1) + L - 1) / L);
-    if (!(options & (KVQ_OPT_SHARED_MAX | KVQ_OPT_GLOBAL_MAX)) && units > ctas_per_pair * pairs &&
-        L == KVQ_MAX_SPLIT_TOKENS)
-      L = KVQ_MAX_SPLIT_TOKENS / 2;
+    L = fits ? (int)l : KVQ_MAX_SPLIT_TOKENS / 2;
   }
   L = (L + kTile - 1) / kTile * kTile;
   *L_out = std::max(kTile, std::min(L, KVQ_MAX_SPLIT_TOKENS));
@@ -295,12 +312,9 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   // the maximum over all splits needs every split on its own CTA at once
   if (a.global_max && groups > capacity) return KVQ_ERR_UNSUPPORTED;
   a.grid = (int)std::min<int64_t>(groups, capacity) * CS;
-  // At these sizes the step is bound by latency and the legacy MMA pipe, not by bytes, so
-  // by default V comes with K (no second DRAM round trip); nvfp4 gathers its kept rows
-  // instead (its V pass over a partly kept staged tile measured slower than the gather)
-  a.v_early = (options & KVQ_OPT_V_WITH_K)      ? 1
-              : (options & KVQ_OPT_V_KEPT_ONLY) ? 0
-                                                : desc->fmt != KVQ_FMT_NVFP4;
+  // At these sizes the step is bound by latency and instruction issue, not by bytes, so
+  // by default V comes with K (no second DRAM round trip)
+  a.v_early = (options & KVQ_OPT_V_KEPT_ONLY) ? 0 : 1;
   // The merge: inside the decode kernel when every group of splits has its own CTAs at
   // once (the splits exchange (m, l) and add their shares into the output); otherwise every
   // split writes its partial to the workspace and the combine kernel merges them, one CTA

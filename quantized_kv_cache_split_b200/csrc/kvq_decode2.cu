@@ -7,39 +7,41 @@
 // "FAQ": K itself is always dequantized.
 //
 // Work unit: one split (<= 1024 positions = 16 tiles of 64) of one (sequence, KV head).
-// One CTA of 16 warps per SM; CTAs loop over the units.  Per unit:
-//   copies    Warp w owns tile w.  Its lane 0 issues the tile's K codes as one tensor
-//             copy (TMA, swizzled so that the fragment loads are free of bank
-//             conflicts) and its scale rows as one bulk copy, both completing on the
-//             tile's mbarrier; with V fetched with K, the V tile the same way on a
-//             second mbarrier.  Nothing waits for the copies to be issued.
+// A CTA has one warp per tile of a split (4, 8 or 16 warps, so 4, 2 or 1 CTAs per SM);
+// when there are more units than CTAs, the CTAs loop over the units.  Per unit:
+//   copies    Lane 0 of warp w issues K tile w as one tensor copy (TMA, swizzled so that
+//             the fragment loads are free of bank conflicts) and its scale rows as one
+//             bulk copy, both completing on the warp's mbarrier.  V tiles copied whole go
+//             into their own region when shared memory allows: right behind the K copy,
+//             or, when every split has its own CTA and the split is long, after the K
+//             pass, so that the launch's K copies have the memory system to themselves;
+//             else into the K tile's place once its scores are taken.
 //   query     Warp 0 builds the query fragments (lut4: the rotated query) for the CTA.
 //   K pass    Each warp scores its tile on the tensor cores (mma.sync m16n8k16,
-//             positions x heads x head_dim) once its copy lands; scores stay in
-//             registers.
+//             positions x heads x head_dim) once its copy lands, keeps the scores in
+//             its shared-memory scratch, and folds them into its (max, denominator).
 //   maximum   One CTA barrier; every warp reads the split's maximum per head (with the
-//             sequence-wide option, the splits of the (sequence, KV head) first
-//             exchange their maxima and denominators through tagged words).
-//   weights   Each warp turns its scores into weights p = 2^(s - m), adds them all
-//             into the denominator, keeps a pair iff s - m >= log2(tau), writes the
-//             kept weights (fp16) into the CTA's weight matrix and a 64-bit row mask of
-//             the rows any head keeps; with V fetched after the test, it gathers just
-//             those rows.
-//   V pass    12 warps split the head dimension into 32-dim slices and the tiles into
-//             position sets, so no warp holds the whole output: for every 16-row group
-//             with a kept row, ldmatrix.trans of the slice's codes (magic-number fp16 for
-//             q8_0 / q4_0, centroid or E2M1 lookups for lut4 / nvfp4) times the group's
-//             weights on the tensor cores.  Skipped groups cost nothing, skipped rows
-//             inside a kept group contribute zero.
-//   merge     When every unit has its own CTA, the splits publish (m, l) after the
-//             weights; one otherwise idle warp collects every split's (m, l) during the
-//             V pass and the CTA adds its normalized share into the output with vector
-//             atomics (lut4: rotated back first).  Otherwise the CTA writes its partial
-//             (o, m, l) and the combine kernel merges them.
+//             cluster option, the maximum over a thread-block cluster of splits, through
+//             distributed shared memory; with the sequence-wide option, the splits of the
+//             (sequence, KV head) first exchange their (m, l) through tagged words).
+//   weights   Each warp turns its scores into weights p = 2^(s - m), keeps a pair iff
+//             s - m >= log2(tau), and turns the kept weights (fp16) into the B fragments
+//             of its V pass (movmatrix); a 16-row group with no kept pair is skipped.
+//   V pass    The tile's warp: per kept group, ldmatrix.trans of the V codes (magic-number
+//             fp16 for q8_0 / q4_0, centroid or E2M1 lookups for lut4 / nvfp4) times the
+//             group's weights on the tensor cores; skipped rows inside a kept group
+//             contribute zero.  With V fetched after the test, the kept rows alone are
+//             gathered first.
+//   merge     When every unit has its own CTA, a poll warp publishes the split's (m, l)
+//             right after the maximum and collects every split's during the V pass; the
+//             CTA adds its normalized share into the output with vector atomics (lut4:
+//             rotated back first) once split 0 has cleared the output rows.  Otherwise the
+//             CTA writes its partial (o, m, l) and the combine kernel merges them.
 // Every wait (mbarriers, exchange, flags) is bounded and reports KVQ_FLAG_TIMEOUT.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cfloat>
 #include <mutex>
 
 #include "kvq_decode2.h"
@@ -201,29 +203,32 @@ __device__ __forceinline__ void tile_mag_normalize(uint8_t* scales, int n, int l
     }
   }
 #pragma unroll
+  for (int b = 0; b < C::NBLK; ++b) k[b] = 0;
+  // typical data: every |d| < 2 (fp16 exponent field < 16), nothing to rescale
+  bool big = false;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) big |= (mx[w] & 0x7C00u) >= 0x4000u || (mx[w] & 0x7C000000u) >= 0x40000000u;
+  if (!__any_sync(0xffffffffu, big)) return;
+#pragma unroll
   for (int o = 16; o; o >>= 1)
 #pragma unroll
     for (int w = 0; w < NW; ++w)
       mx[w] = h2_as_u32(__hmax2(u32_as_h2(mx[w]), u32_as_h2(__shfl_xor_sync(0xffffffffu, mx[w], o))));
-  bool any = false;
   uint32_t f[NW];
 #pragma unroll
   for (int w = 0; w < NW; ++w) {
     const int e0 = (mx[w] >> 10) & 31, e1 = (mx[w] >> 26) & 31;  // fp16 exponent fields
     k[2 * w] = min(14, max(0, e0 - 15));
     k[2 * w + 1] = min(14, max(0, e1 - 15));
-    any |= (k[2 * w] | k[2 * w + 1]) != 0;
     f[w] = ((uint32_t)(15 - k[2 * w]) << 10) | ((uint32_t)(15 - k[2 * w + 1]) << 26);  // 2^-k
   }
-  if (any) {  // (warp-uniform) typical data needs no rescaling
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int row = lane + 32 * h;
-      if (row < n) {
-        uint32_t* sr = reinterpret_cast<uint32_t*>(scales + row * C::SROW);
+  for (int h = 0; h < 2; ++h) {
+    const int row = lane + 32 * h;
+    if (row < n) {
+      uint32_t* sr = reinterpret_cast<uint32_t*>(scales + row * C::SROW);
 #pragma unroll
-        for (int w = 0; w < NW; ++w) sr[w] = h2_as_u32(__hmul2(u32_as_h2(sr[w]), u32_as_h2(f[w])));
-      }
+      for (int w = 0; w < NW; ++w) sr[w] = h2_as_u32(__hmul2(u32_as_h2(sr[w]), u32_as_h2(f[w])));
     }
   }
   __syncwarp();
@@ -277,14 +282,6 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-// Named barrier among `count` threads (a multiple of 32): arrive without waiting / wait.
-__device__ __forceinline__ void named_arrive(int id, int count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D, int NW>
 __global__ void __launch_bounds__(32 * NW, 16 / NW)
@@ -304,6 +301,8 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   __shared__ float red_m[kNW][8], red_l[kNW][8];
   __shared__ int cnt_skip[kNW], cnt_keep[kNW];
   __shared__ float mh_s[8], mc_s[8], share_s[8];  // split maximum, the one the skip test uses
+  __shared__ float ls_s[8];                        // split denominator relative to mh_s
+  __shared__ float mg_s[8];                        // sequence-wide maximum (that option)
   __shared__ int misc[4];  // 0: clamped length, 1: exchange ok, 2: tag, 3: warps holding accumulators
   __shared__ uint32_t qfr[kQfWords * 32];
 
@@ -336,29 +335,27 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
   const bool add_merge = a.out != nullptr && a.group_merge;
   const bool v_tma = pr.v_tma != 0;     // V tiles copied whole (with K, or right after it)
   const bool v_sep = pr.v_sep != 0;     // V tiles in their own region (copied with K)
+  // ... after the K pass when the split is long (measured: short splits gain nothing)
+  const bool v_late = v_sep && add_merge && NT >= 8;
   const float qk_scale = a.sm_scale * kLog2e;
-  const float thr = a.tau > 0.f ? log2f(a.tau) : -INFINITY;  // keep iff s - m >= log2(tau)
+  // keep iff s - m >= log2(tau); tau = 0 keeps every position in the sequence (a row
+  // past the end holds s = -inf, below any finite threshold)
+  const float thr = a.tau > 0.f ? log2f(a.tau) : -FLT_MAX;
   const bool hl0 = 2 * c < G, hl1 = 2 * c + 1 < G;
 
-  if (tid == 0) {
-    for (int i = 0; i < kNW; ++i) {
-      mbar_init(&kbar[i], 1);
-      mbar_init(&vbar[i], 1);
-    }
+  // every warp's lane 0 initializes the warp's own barriers (it alone issues their copies;
+  // the warp's lanes wait on them after a warp barrier), so no CTA barrier is needed here
+  if (lane == 0) {
+    mbar_init(&kbar[warp], 1);
+    mbar_init(&vbar[warp], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  __syncwarp();
   // Programmatic dependent launch: the next grid may be scheduled now; nothing is read
   // from global memory before the preceding grid has completed.
   grid_dependents_launch();
   grid_dependency_wait();
-  // every CTA takes part in the launch count that tags the exchange; the read is in
-  // flight while the first unit's copies are issued (its value is stored before B0)
   unsigned long long ep_raw = 0;
-  if (tid == 32) {
-    ep_raw = epoch_read(a.epoch);
-    epoch_advance(a.epoch);
-  }
-  __syncthreads();  // mbarriers initialized
   Lut lut;
   if constexpr (C::kLut) {
 #pragma unroll
@@ -448,7 +445,15 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       load_query<FMT, D>(r < G ? qg + ((size_t)b * Hq + (size_t)kvh * G + r) * D : nullptr, a.desc.signs, c,
                          qraw);
     int n_raw = 0;
-    if (warp == 1 && lane == 0) n_raw = __ldg(a.seq_lens + b);
+    if (warp == 1 && lane == 0) {
+      n_raw = __ldg(a.seq_lens + b);
+      // every CTA takes part in the launch count that tags the exchange (its value is
+      // stored before B0)
+      if (k == 0) {
+        ep_raw = epoch_read(a.epoch);
+        epoch_advance(a.epoch);
+      }
+    }
     // ---- K copies: lane 0 of warp w issues tile w (positions that exist in memory; a
     //      tile past the sequence's end is copied speculatively and left unused)
     int row0 = -1;
@@ -475,19 +480,18 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
       row0 = __shfl_sync(0xffffffffu, row0, 0);
       k_issued = row0 >= 0;
-      v_issued = v_sep && k_issued;
-    }
-    // ---- V copies when V tiles come with K: issued after every K copy of the CTA, so the
-    //      K tiles land first
-    if (v_sep) {
-      __syncthreads();
-      if (warp < NT && lane == 0) {
-        const uint32_t vbytes = k_issued ? CODE + SC : 0;
-        mbar_expect_tx(&vbar[warp], vbytes);
-        if (vbytes) {
-          tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
-          bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+      // V tiles copied whole into their own region, CTAs looping over units or writing
+      // partials: each V copy goes out right behind its K copy
+      if (v_sep && !v_late) {
+        if (lane == 0) {
+          const uint32_t vbytes = k_issued ? CODE + SC : 0;
+          mbar_expect_tx(&vbar[warp], vbytes);
+          if (vbytes) {
+            tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+            bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+          }
         }
+        v_issued = k_issued;
       }
     }
     if (warp == 1 && lane == 0) {
@@ -585,9 +589,29 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
     }
-    if (r == 0) {
-      red_m[warp][2 * c] = mx0;
-      red_m[warp][2 * c + 1] = mx1;
+    {
+      // the tile's denominators relative to its own maxima (rows past the end hold -inf),
+      // so that the split's (m, l) is known at the CTA barrier that follows
+      float lw0 = 0.f, lw1 = 0.f;
+      if (has_tile) {
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+          const float4 sv = scw[j * 32];
+          lw0 += ex2(sv.x - mx0) + ex2(sv.z - mx0);
+          lw1 += ex2(sv.y - mx1) + ex2(sv.w - mx1);
+        }
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lw0 += __shfl_xor_sync(0xffffffffu, lw0, o);
+        lw1 += __shfl_xor_sync(0xffffffffu, lw1, o);
+      }
+      if (r == 0) {
+        red_m[warp][2 * c] = mx0;
+        red_m[warp][2 * c + 1] = mx1;
+        red_l[warp][2 * c] = lw0;
+        red_l[warp][2 * c + 1] = lw1;
+      }
     }
     // V into this warp's K slot right behind its K pass (V tiles copied whole but no
     // room for a separate region)
@@ -607,16 +631,53 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       mbar_expect_tx(&vbar[warp], 0);  // every barrier completes one phase per unit
     }
     __syncthreads();  // B1: every warp's maxima
+    // V tiles copied whole into their own region, every split on its own CTA (the step is
+    // one round of copies): the V copies go out once all K tiles of the CTA have landed, so
+    // that the K copies of the launch have the memory system first
+    if (v_sep && v_late && warp < NT) {
+      if (lane == 0) {
+        fence_proxy_async();
+        mbar_expect_tx(&vbar[warp], has_tile ? CODE + SC : 0);
+        if (has_tile) {
+          tma_rows(vcode + warp * CODE, &tmv, row0, &vbar[warp]);
+          bulk_copy(vscale + warp * SC, vscales_g + (size_t)row0 * C::SROW, SC, &vbar[warp]);
+        }
+      }
+      v_issued = has_tile;
+    }
 
-    // ---- the split's maximum per head (log2 units)
+    // ---- the split's maximum per head (log2 units); warp 0 and the poll warp also fold
+    //      the tiles' denominators into the split's (lane h: head h)
     float mh0, mh1;
+    float m_own = -INFINITY, l_own = 0.f;  // lanes < 8 of warp 0 and of the poll warp
+    float m_use = -INFINITY;               // the maximum the weights use (lanes < 8)
     {
+      // lane (head h = lane & 7, quarter q = lane >> 3) folds the tiles of warps q, q + 4,
+      // ...; the quarters are combined by shuffles, so every lane holds head lane & 7
+      const int hh = lane & 7, q = lane >> 3;
       float m = -INFINITY;
-      if (lane < 8)
-        for (int w = 0; w < NT; ++w) m = fmaxf(m, red_m[w][lane]);
+      for (int w = q; w < NT; w += 4) m = fmaxf(m, red_m[w][hh]);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      m_own = m;
+      if (warp == 0 || warp == kPollWarp) {
+        float l = 0.f;
+        if (m > -INFINITY) {
+          for (int w = q; w < NT; w += 4) {
+            const float mw = red_m[w][hh];
+            if (mw > -INFINITY) l = fmaf(red_l[w][hh], ex2(mw - m), l);
+          }
+        }
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        l_own = l;
+      }
       mh0 = __shfl_sync(0xffffffffu, m, 2 * c);
       mh1 = __shfl_sync(0xffffffffu, m, 2 * c + 1);
-      if (warp == 0 && lane < 8) mh_s[lane] = m;
+      if (warp == 0 && lane < 8) {
+        mh_s[lane] = m;
+        ls_s[lane] = l_own;
+      }
       if (CS > 1) {
         // the maximum over the cluster's splits: every CTA's maxima are written before the
         // cluster barrier, read from distributed shared memory after it; the arrive after
@@ -632,35 +693,13 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         cluster_arrive();
       }
       if (warp == 0 && lane < 8) mc_s[lane] = m;
+      m_use = m;
     }
     if (a.global_max) {
       // every split publishes (m, l relative to m); the poll warp derives the final
       // maximum M and denominator L of every head; the weights below use M, and this
       // split's share of the output is 1 / L
-      float l0 = 0.f, l1 = 0.f;
-      if (has_tile) {
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-          const float4 sv = scw[j * 32];  // invalid rows hold -inf
-          l0 += ex2(sv.x - mh0) + ex2(sv.z - mh0);
-          l1 += ex2(sv.y - mh1) + ex2(sv.w - mh1);
-        }
-      }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-      }
-      if (r == 0) {
-        red_l[warp][2 * c] = hl0 ? l0 : 0.f;
-        red_l[warp][2 * c + 1] = hl1 ? l1 : 0.f;
-      }
-      __syncthreads();
-      if (tid < G && n_tok > 0) {
-        float l = 0.f;
-        for (int w = 0; w < NT; ++w) l += red_l[w][tid];
-        xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, mc_s[tid], l);
-      }
+      if (tid < G && n_tok > 0) xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, m_own, l_own);
       if (warp == kPollWarp && n_tok > 0) {
         const int nsplit = (nb + Ls - 1) / Ls;
         const int h = lane >> 2, j = lane & 3;
@@ -670,7 +709,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
         if (ok) {
           xch_combine(M, L, 2);
           if (j == 0 && h < G) {
-            mc_s[h] = M;
+            mg_s[h] = M;
             share_s[h] = 1.f / L;
           }
         } else if (lane == 0) {
@@ -680,45 +719,55 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       }
       __syncthreads();
       if (misc[1]) {
-        mh0 = mc_s[2 * c < G ? 2 * c : 0];
-        mh1 = mc_s[2 * c + 1 < G ? 2 * c + 1 : 0];
+        mh0 = mg_s[2 * c < G ? 2 * c : 0];
+        mh1 = mg_s[2 * c + 1 < G ? 2 * c + 1 : 0];
+        if (warp == 0 && lane < G) mc_s[lane] = mg_s[lane];  // (read after the next CTA barrier)
       }
     }
-    // In-kernel merge without the sequence-wide maximum: the tile owners hand their
-    // denominators to the poll warp through a named barrier and go on with their V pass;
-    // the poll warp publishes (m, l) and collects every split's while they work.
+    // In-kernel merge without the sequence-wide maximum: the poll warp publishes the
+    // split's (m, l) at once (l relative to the maximum the weights use) and, after its own
+    // tile if it has one, collects every split's while the others work; a warp without a
+    // tile, if there is one besides, waits for split 0's cleared output rows meanwhile.
     const bool publish = add_merge && !a.global_max && n_tok > 0;
-    const int pub_count = 32 * (NT == kNW ? kNW : NT + 1);
+    const int zwarp = NT < kNW - 1 ? NT : kPollWarp;
+    if (warp == kPollWarp && publish && lane < G)
+      xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, m_use, l_own * ex2(m_own - m_use));
+    if (warp == zwarp && zwarp != kPollWarp && publish && lane == 0) {
+      if (!flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag)) {
+        set_flag(flags, KVQ_FLAG_TIMEOUT);
+        misc[1] = 0;
+      }
+    }
+
+    // a head past the group (G < 8) gets m = +inf: every one of its weights is 0 and none
+    // of its positions is kept
+    if (!hl0) mh0 = INFINITY;
+    if (!hl1) mh1 = INFINITY;
 
     // ---- weights, skip test and V pass of this warp's own tile
     if (warp < NT) {
-      float l0 = 0.f, l1 = 0.f;
       int nskip = 0;
       uint32_t gk = 0;  // groups (16-row jobs) with a kept pair
       uint32_t* pww = pword + warp * 4 * 64 + lane;  // B fragments of the weights, per group
       unsigned long long rows = 0ull;
+      const bool count = !v_tma || a.stats;  // the kept rows wanted (to gather them, or counted)
       if (has_tile) {
 #pragma unroll 1
         for (int j = 0; j < 4; ++j) {
-          const int ra = 16 * j + r, rb = ra + 8;
-          const bool va = ra < nvalid, vb = rb < nvalid;
-          const bool la0 = va && hl0, la1 = va && hl1, lb0 = vb && hl0, lb1 = vb && hl1;
+          // rows past the end hold s = -inf: weight 0, never kept
           const float4 sv = scw[j * 32];
           const float da0 = sv.x - mh0, da1 = sv.y - mh1;
           const float db0 = sv.z - mh0, db1 = sv.w - mh1;
-          const float ea0 = la0 ? ex2(da0) : 0.f, ea1 = la1 ? ex2(da1) : 0.f;
-          const float eb0 = lb0 ? ex2(db0) : 0.f, eb1 = lb1 ? ex2(db1) : 0.f;
-          l0 += ea0 + eb0;
-          l1 += ea1 + eb1;
-          const bool ka0 = la0 && da0 >= thr, ka1 = la1 && da1 >= thr;
-          const bool kb0 = lb0 && db0 >= thr, kb1 = lb1 && db1 >= thr;
-          nskip += (la0 && !ka0) + (la1 && !ka1) + (lb0 && !kb0) + (lb1 && !kb1);
+          const float ea0 = ex2(da0), ea1 = ex2(da1), eb0 = ex2(db0), eb1 = ex2(db1);
+          const bool ka0 = da0 >= thr, ka1 = da1 >= thr, kb0 = db0 >= thr, kb1 = db1 >= thr;
           // the kept weights as the V MMA's B fragments: rows 0-7 / 8-15 of the group,
           // transposed from (row r, heads 2c, 2c + 1) to (rows 2c, 2c + 1, head r)
           pww[j * 64] = movmatrix_trans(pack_h2(ka0 ? ea0 * kPScale : 0.f, ka1 ? ea1 * kPScale : 0.f));
           pww[j * 64 + 32] = movmatrix_trans(pack_h2(kb0 ? eb0 * kPScale : 0.f, kb1 ? eb1 * kPScale : 0.f));
           gk |= (__any_sync(0xffffffffu, ka0 || ka1 || kb0 || kb1) ? 1u : 0u) << j;
-          if (!v_tma || a.stats) {  // rows any head keeps (the rows to gather; V rows needed)
+          if (count) {  // rows any head keeps (the rows to gather; V rows needed), skip count
+            const bool va = 16 * j + r < nvalid, vb = 16 * j + r + 8 < nvalid;
+            nskip += (va && hl0 && !ka0) + (va && hl1 && !ka1) + (vb && hl0 && !kb0) + (vb && hl1 && !kb1);
             const uint32_t rows_a = rows_of(__ballot_sync(0xffffffffu, ka0 || ka1));
             const uint32_t rows_b = rows_of(__ballot_sync(0xffffffffu, kb0 || kb1));
             const uint32_t mine =
@@ -726,15 +775,6 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
             rows |= (unsigned long long)__reduce_or_sync(0xffffffffu, mine) << (16 * j);
           }
         }
-      }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-      }
-      if (r == 0) {
-        red_l[warp][2 * c] = l0;
-        red_l[warp][2 * c + 1] = l1;
       }
       if (a.stats) {
 #pragma unroll
@@ -744,7 +784,6 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
           cnt_keep[warp] = __popcll(rows);
         }
       }
-      if (publish && warp != kPollWarp) named_arrive(1, pub_count);  // l is in shared memory
 
       uint8_t* vc = (v_sep ? vcode : kcode) + warp * CODE;
       uint8_t* vs = (v_sep ? vscale : kscale) + warp * SC;
@@ -819,26 +858,21 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (v_issued && !v_waited) mbar_wait(&vbar[warp], ph);  // no copy stays in flight
     }
     if (warp == kPollWarp && publish) {
-      // publish this split's (m, l), then wait for split 0's cleared output rows and for
-      // every split's (m, l): this split's share of each head is 2^(m_s - M) / L
-      named_sync(1, pub_count);
-      if (lane < G) {
-        float l = 0.f;
-        for (int w = 0; w < NT; ++w) l += red_l[w][lane];
-        xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, mc_s[lane], l);
-      }
+      // wait for every split's (m, l) (and, with no other warp to do it, for split 0's
+      // cleared output rows): this split's share of each head is 2^(m_s - M) / L
       bool ok = true;
-      if (lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
+      if (zwarp == kPollWarp && lane == 0) ok = flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int h = lane >> 2, j = lane & 3;
+      const float mine = __shfl_sync(0xffffffffu, m_use, h & 7);  // this split's maximum of head h
       if (ok) {
         const int nsplit = (nb + Ls - 1) / Ls;
-        const int h = lane >> 2, j = lane & 3;
         float M, L;
         ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits, j, 4,
                             nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {
           xch_combine(M, L, 2);
-          if (j == 0 && h < G) share_s[h] = ex2(mc_s[h] - M) / L;
+          if (j == 0 && h < G) share_s[h] = ex2(mine - M) / L;
         }
       }
       if (lane == 0 && !ok) {
@@ -858,10 +892,9 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     //      lanes' entries per thread), scaled by the share, staged as [head][dim]
     if (n_tok > 0) {
       if (!add_merge && tid < G) {
-        float l = 0.f;
-        for (int w = 0; w < NT; ++w) l += red_l[w][tid];
-        a.part_m[slot0 + (size_t)tid * a.max_splits] = mc_s[tid];  // (the maximum the weights use)
-        a.part_l[slot0 + (size_t)tid * a.max_splits] = l;
+        // (the maximum the weights used, and the denominator relative to it)
+        a.part_m[slot0 + (size_t)tid * a.max_splits] = mc_s[tid];
+        a.part_l[slot0 + (size_t)tid * a.max_splits] = ls_s[tid] * ex2(mh_s[tid] - mc_s[tid]);
       }
       if (tid == 32 && a.stats) {
         int ns = 0, nk = 0;

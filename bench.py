@@ -414,6 +414,8 @@ def gpu_arm(args, world, rank, local):
                 ("sparse_v_with_k", args.tau, "split", K.KVQ_OPT_V_WITH_K),
                 ("sparse_cluster_max", args.tau, "cluster", 0), ("sparse_sequence_max", args.tau, "sequence", 0),
                 ("sparse_sequence_max_v_kept_only", args.tau, "sequence", K.KVQ_OPT_V_KEPT_ONLY))
+    if not args.cluster_variant:
+        variants = tuple(v for v in variants if v[2] != "cluster")
     res = {}
     for tag, tau, scope, v_opt in variants:
         res[tag] = measure_variant(rep, args, world, device, tau, scope, v_opt, hbm_peak,
@@ -687,6 +689,9 @@ def main(argv=None):
                     help="positions per split (0: the library's choice, kvq_resolve_split)")
     ap.add_argument("--headline-only", dest="all_workloads", action="store_false",
                     help="(profiling runs) skip the per-workload table of every configuration")
+    ap.add_argument("--no-cluster", dest="cluster_variant", action="store_false",
+                    help="(profiling runs) skip the cluster-shared-maximum variant, whose "
+                         "cooperative cluster launch ncu's injection does not run")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

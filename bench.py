@@ -288,6 +288,20 @@ class StepGraphs:
         self.uploaded = upload_fn(self.timed)
 
 
+def prewarm(fn, seconds: float = 0.3, n_steps: int = 50):
+    """Untimed: replay a graph of ``n_steps`` steps of ``fn`` for about ``seconds``, so that
+    the first timed variant does not meet a GPU still leaving its idle clocks (measured:
+    without it the first variant of a run came out ~1 us per step slower than the same
+    variant timed later in the run)."""
+    import torch
+    g = capture(fn, n_steps, 0)
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        g.replay()
+        torch.cuda.synchronize()
+    del g
+
+
 def time_steps(graphs: StepGraphs, world, sampler=None):
     """Replay the warm-up graph, then time one replay of the timed graph with CUDA
     events on the current stream (barrier and synchronize on both sides); ms."""
@@ -416,6 +430,7 @@ def gpu_arm(args, world, rank, local):
                 ("sparse_sequence_max_v_kept_only", args.tau, "sequence", K.KVQ_OPT_V_KEPT_ONLY))
     if not args.cluster_variant:
         variants = tuple(v for v in variants if v[2] != "cluster")
+    prewarm(lambda i: rep.decode(i, args.tau))
     res = {}
     for tag, tau, scope, v_opt in variants:
         res[tag] = measure_variant(rep, args, world, device, tau, scope, v_opt, hbm_peak,

@@ -27,7 +27,7 @@ struct DecodeArgs {
   int split_tokens;   // resolved, multiple of kTile
   int max_splits;     // ceil(max_seq_len / split_tokens)
   void* workspace;
-  int* counters;      // [batch][num_kv_heads] arrival counters of the last-arrival merge
+  int* counters;      // [batch][num_q_heads] int32 words reserved in the workspace (unused)
   unsigned long long* zflag;  // [batch][num_kv_heads] output rows cleared (launch tag)
   unsigned long long* epoch;  // launch counter in the workspace header (exchange tags)
   float* part_o;      // partials, see below
@@ -49,9 +49,9 @@ struct DecodeArgs {
 };
 
 // Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch
-// counter that tags the exchange entries); the merge flags and counters (u64 flags
-// "output rows cleared" [batch][num_q_heads], then int32 last-arrival counters
-// [batch][num_q_heads], together rounded up to 256 bytes); then, one slot per split:
+// counter that tags the exchange entries); the merge flags (u64 "output rows cleared"
+// [batch][num_q_heads], then int32 words [batch][num_q_heads] that are reserved,
+// together rounded up to 256 bytes); then, one slot per split:
 //   (m, l) exchange [batch][num_q_heads][max_splits] 2 x u64, each word a fp32 value
 //   under a 32-bit launch tag (what the splits of a (sequence, KV head) publish to one
 //   another)

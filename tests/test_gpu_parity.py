@@ -138,9 +138,9 @@ def test_combine_kernel_matches_in_kernel_merge(name, tau):
 
 @pytest.mark.parametrize("scope", ["split", "cluster"])
 def test_in_kernel_merge_resets_its_counters(scope):
-    # back-to-back multi-round calls on one workspace: each must merge exactly once (the
-    # clusters' last finisher counts arrivals in the workspace; split scope merges with the
-    # combine kernel after the decode; the additive merge may change the last bits)
+    # back-to-back multi-round calls on one workspace: each must merge exactly once (both
+    # scopes merge with the combine kernel after the decode; the additive merge of a
+    # single-round launch may change the last bits)
     import quantized_kv_cache_split_b200 as K
     wl = W.shrink(W.WORKLOADS["paged_b8_q4"], [3000, 64, 0, 1500, 777], n_planted=8)
     inp = W.generate(wl)

@@ -293,7 +293,7 @@ int kvq_decode_attn(const kvq_cache_desc* desc, const void* q, int32_t batch,
   a.workspace = workspace;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   a.zflag = reinterpret_cast<unsigned long long*>(ws + kWorkspaceHeader);
-  a.counters = reinterpret_cast<int*>(a.zflag + (size_t)batch * num_q_heads);
+  a.arrive = a.zflag + (size_t)batch * num_q_heads;
   a.epoch = reinterpret_cast<unsigned long long*>(ws + kEpochOffset);
   a.group_merge = 0;  // decided at launch
   const size_t n_part = (size_t)batch * num_q_heads * a.max_splits;

@@ -29,7 +29,7 @@ combine_kernel(const uint8_t* __restrict__ ws, int batch, int hq, int max_seq_le
   const int b = bh / hq;
   const int tid = threadIdx.x;
   const size_t n_part = (size_t)batch * hq * max_splits;
-  // the partials follow the header, the merge counters and the (m, l) exchange entries
+  // the partials follow the header, the merge words and the (m, l) exchange entries
   const float* o = reinterpret_cast<const float*>(ws + kWorkspaceHeader + counters_bytes(batch, hq) +
                                                   16 * n_part);
   const float* m = o + n_part * D;

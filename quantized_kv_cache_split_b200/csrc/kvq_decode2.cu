@@ -282,6 +282,37 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// ------------------------------------------------------------------ exchange publication
+// The split's (m, l) of every head (lane h holds head h) stored by lane 0, then its
+// arrival on the (sequence, KV head)'s arrival word; returns (in lane 0) the count that
+// word reaches once every split of the (sequence, KV head) has arrived.  Warp-uniform.
+__device__ __forceinline__ unsigned long long publish_split(const DecodeArgs& a, size_t slot0, uint32_t tag,
+                                                            float m, float l, int G, int lane, int pair,
+                                                            bool first, int nsplit) {
+  float mv[8], lv[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    mv[h] = __shfl_sync(0xffffffffu, m, h);
+    lv[h] = __shfl_sync(0xffffffffu, l, h);
+  }
+  unsigned long long target = 0;
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < G) xch_store(a.xch + slot0 + (size_t)h * a.max_splits, tag, mv[h], lv[h]);
+    target = arrive_add(a.arrive + pair, first, nsplit);
+  }
+  return target;
+}
+// Before polling the exchange words: lane 0 waits (briefly bounded) until every split of
+// the (sequence, KV head) has arrived, so that the poll reads the entries about once instead
+// of hammering them; the poll still checks every entry's tag and keeps the full bound.
+constexpr long long kArriveWaitCycles = 1ll << 15;
+__device__ __forceinline__ void arrivals_await(const DecodeArgs& a, int pair, unsigned long long target, int lane) {
+  if (lane == 0) (void)arrivals_wait(a.arrive + pair, target, kArriveWaitCycles, kPollSleepNs);
+  __syncwarp();
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int FMT, int D, int NW>
 __global__ void __launch_bounds__(32 * NW, 16 / NW)
@@ -699,11 +730,13 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       // every split publishes (m, l relative to m); the poll warp derives the final
       // maximum M and denominator L of every head; the weights below use M, and this
       // split's share of the output is 1 / L
-      if (tid < G && n_tok > 0) xch_store(a.xch + slot0 + (size_t)tid * a.max_splits, tag, m_own, l_own);
       if (warp == kPollWarp && n_tok > 0) {
         const int nsplit = (nb + Ls - 1) / Ls;
+        const unsigned long long target =
+            publish_split(a, slot0, tag, m_own, l_own, G, lane, b * hkv + kvh, cu == 0, nsplit);
         const int h = lane >> 2, j = lane & 3;
         float M, L;
+        arrivals_await(a, b * hkv + kvh, target, lane);
         bool ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits,
                                  j, 4, nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {
@@ -730,8 +763,10 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
     // tile, if there is one besides, waits for split 0's cleared output rows meanwhile.
     const bool publish = add_merge && !a.global_max && n_tok > 0;
     const int zwarp = NT < kNW - 1 ? NT : kPollWarp;
-    if (warp == kPollWarp && publish && lane < G)
-      xch_store(a.xch + slot0 + (size_t)lane * a.max_splits, tag, m_use, l_own * ex2(m_own - m_use));
+    unsigned long long arrive_target = 0;  // (lane 0 of the poll warp)
+    if (warp == kPollWarp && publish)
+      arrive_target = publish_split(a, slot0, tag, m_use, l_own * ex2(m_own - m_use), G, lane, b * hkv + kvh,
+                                    cu == 0, (nb + Ls - 1) / Ls);
     if (warp == zwarp && zwarp != kPollWarp && publish && lane == 0) {
       if (!flag_wait_acquire(a.zflag + (size_t)b * hkv + kvh, tag)) {
         set_flag(flags, KVQ_FLAG_TIMEOUT);
@@ -868,6 +903,7 @@ decode2_kernel(const __grid_constant__ Decode2Params pr, const __grid_constant__
       if (ok) {
         const int nsplit = (nb + Ls - 1) / Ls;
         float M, L;
+        arrivals_await(a, b * hkv + kvh, arrive_target, lane);
         ok = xch_reduce<16>(a.xch + ((size_t)b * Hq + (size_t)kvh * G + (h < G ? h : 0)) * a.max_splits, j, 4,
                             nsplit, h < G, tag, M, L, kWaitCycles, kPollSleepNs);
         if (ok) {

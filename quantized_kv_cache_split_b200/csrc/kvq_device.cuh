@@ -165,6 +165,31 @@ __device__ __forceinline__ bool flag_wait_acquire(const unsigned long long* p, u
   }
 }
 
+// Arrival word of one (sequence, KV head): every launch adds exactly kArriveStep to it
+// over the splits that publish (split 0: kArriveStep - (n - 1), the others 1), so a split
+// that reads v before its own add knows that the word reaches (v / kArriveStep + 1) *
+// kArriveStep once every split has arrived.  A relaxed add: the count is only a hint that
+// the exchange entries are there (a reader still checks every entry's tag).
+constexpr unsigned long long kArriveStep = 1ull << 16;  // > any number of splits
+__device__ __forceinline__ unsigned long long arrive_add(unsigned long long* p, bool first, int n) {
+  unsigned long long old;
+  asm volatile("atom.relaxed.gpu.global.add.u64 %0, [%1], %2;"
+               : "=l"(old)
+               : "l"(p), "l"(first ? kArriveStep - (unsigned long long)(n - 1) : 1ull)
+               : "memory");
+  return (old / kArriveStep + 1) * kArriveStep;
+}
+// Wait (at most `limit` SM cycles) until the arrival word reaches `target`.
+__device__ __forceinline__ bool arrivals_wait(const unsigned long long* p, unsigned long long target,
+                                              long long limit, int sleep_ns) {
+  const long long t0 = clock64();
+  for (;;) {
+    if (ld_relaxed_u64(p) >= target) return true;
+    if (clock64() - t0 > limit) return false;
+    __nanosleep(sleep_ns);
+  }
+}
+
 __device__ __forceinline__ unsigned long long tag_word(uint32_t tag, float v) {
   return ((unsigned long long)tag << 32) | __float_as_uint(v);
 }

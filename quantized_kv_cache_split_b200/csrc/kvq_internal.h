@@ -27,7 +27,7 @@ struct DecodeArgs {
   int split_tokens;   // resolved, multiple of kTile
   int max_splits;     // ceil(max_seq_len / split_tokens)
   void* workspace;
-  int* counters;      // [batch][num_q_heads] int32 words reserved in the workspace (unused)
+  unsigned long long* arrive;  // [batch][num_kv_heads] exchange arrival words (kArriveStep per launch)
   unsigned long long* zflag;  // [batch][num_kv_heads] output rows cleared (launch tag)
   unsigned long long* epoch;  // launch counter in the workspace header (exchange tags)
   float* part_o;      // partials, see below
@@ -49,9 +49,10 @@ struct DecodeArgs {
 };
 
 // Workspace: a 256-byte header (word 0: KVQ_FLAG_* bits; bytes 8..15: the launch
-// counter that tags the exchange entries); the merge flags (u64 "output rows cleared"
-// [batch][num_q_heads], then int32 words [batch][num_q_heads] that are reserved,
-// together rounded up to 256 bytes); then, one slot per split:
+// counter that tags the exchange entries); the merge words (u64 "output rows cleared"
+// flags, then u64 exchange arrival counts, each
+// [batch][num_q_heads] of which [batch][num_kv_heads] are used, together rounded up to 256
+// bytes); then, one slot per split:
 //   (m, l) exchange [batch][num_q_heads][max_splits] 2 x u64, each word a fp32 value
 //   under a 32-bit launch tag (what the splits of a (sequence, KV head) publish to one
 //   another)
@@ -60,7 +61,7 @@ struct DecodeArgs {
 //   l [batch][num_q_heads][max_splits] fp32
 size_t partials_bytes(int batch, int num_q_heads, int head_dim, int max_splits);
 __host__ __device__ inline size_t counters_bytes(int batch, int num_q_heads) {
-  return ((size_t)batch * num_q_heads * (sizeof(uint64_t) + sizeof(int32_t)) + 255) / 256 * 256;
+  return ((size_t)batch * num_q_heads * (2 * sizeof(uint64_t)) + 255) / 256 * 256;
 }
 
 // x2 == nullptr: one plane pair; otherwise the second pair (x2, codes2, scales2) in the

@@ -5,7 +5,7 @@
 // forbids new allocations, or a host that calls in from a context where cudaMalloc is
 // not permitted.  This entry point runs the same split-KV kernel, with its in-kernel
 // merge, as kvq_decode_attn given an output pointer, but keeps the partials and merge
-// counters in a static device array owned by the library, so the caller passes only
+// words in a static device array owned by the library, so the caller passes only
 // inputs and outputs.
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -50,7 +50,7 @@ extern "C" int kvq_decode_attn_noalloc(const kvq_cache_desc* desc, const void* q
   int st = scratch_address(&ws);
   if (st != KVQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the flag word and the merge counters start at zero for every call; the launch
+  // the flag word and the merge words start at zero for every call; the launch
   // counter in the header (bytes 8..15) keeps counting, so that no exchange entry left
   // by an earlier call carries the tag of this one
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s) != cudaSuccess ||

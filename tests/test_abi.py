@@ -76,10 +76,10 @@ def test_split_resolution_and_workspace_size():
     assert K.kvq_resolve_split(d, 1, 32, 4096, 5000) == K.KVQ_MAX_SPLIT_TOKENS
     assert K.kvq_resolve_split(d, 1, 32, 4096, 1) == 64
     ws = K.kvq_workspace_size(2, 32, 128, 1000, 128)
-    # header, merge flags (u64) and counters (int32) per (sequence, head) rounded to 256,
-    # then per partial the tagged (m, l) exchange entry and (o, m, l)
-    assert ws == 256 + 768 + 2 * 32 * 8 * (16 + (128 + 2) * 4)
-    assert K.kvq_workspace_size(3, 32, 128, 1000, 128) == 256 + 1280 + 3 * 32 * 8 * (16 + (128 + 2) * 4)
+    # header, cleared-rows flags and exchange arrival words (u64 each) per (sequence,
+    # head) rounded to 256, then per partial the tagged (m, l) exchange entry and (o, m, l)
+    assert ws == 256 + 1024 + 2 * 32 * 8 * (16 + (128 + 2) * 4)
+    assert K.kvq_workspace_size(3, 32, 128, 1000, 128) == 256 + 1536 + 3 * 32 * 8 * (16 + (128 + 2) * 4)
 
 
 @pytest.mark.parametrize("kw,code", [

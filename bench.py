@@ -312,6 +312,10 @@ def time_steps(graphs: StepGraphs, world, sampler=None):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if sampler:
         sampler.start()
+    # the device first spins ~1 ms, so that the timed region starts with the graph already
+    # queued behind the start event: host-side delays (the sampler thread's NVML calls, the
+    # replay call itself) then never appear as idle time between the events
+    torch.cuda._sleep(2_000_000)
     start.record()
     graphs.timed.replay()
     end.record()

@@ -177,7 +177,7 @@ size_t kvq_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                           int32_t max_seq_len, int32_t split_tokens);
 
 /* Zero the workspace (its device flag word, the launch counter that tags the (m, l)
- * exchange and the merge counters); call once after allocating it.  A workspace whose
+ * exchange, the cleared-rows flags and the arrival counts); call once after allocating it.  A workspace whose
  * call to kvq_decode_attn completed is ready for the next call without another init,
  * whatever the next call's shape; after KVQ_FLAG_TIMEOUT, init it again. */
 int kvq_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
@@ -290,7 +290,7 @@ int kvq_combine(const kvq_cache_desc* desc, const void* workspace, int32_t batch
  *   Every call looks up the array's device address with the calling thread's current
  *   device; the first call on a device is its set-up and may load the library's device
  *   code there, so make it before any stream capture.  All calls share the one array and
- *   each call clears its fault-flag word and merge counters first, so calls whose
+ *   each call clears its fault-flag word and merge words first, so calls whose
  *   execution overlaps on the GPU (different streams, or another thread) race.  Faults
  *   that the kernel detects (KVQ_FLAG_*) are read back with kvq_noalloc_read_flags.
  */

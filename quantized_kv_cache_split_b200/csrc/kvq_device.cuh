@@ -213,10 +213,6 @@ __device__ __forceinline__ bool xch_load_acquire(const ulonglong2* p, uint32_t t
   return (uint32_t)(a >> 32) == tag && (uint32_t)(b >> 32) == tag;
 }
 
-// Every earlier write of this thread (and, cumulatively, the writes it has observed, e.g.
-// through a CTA barrier) is ordered before its later writes, at GPU scope.
-__device__ __forceinline__ void fence_release_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-
 // Read an entry; false while it is not this launch's (tag mismatch in either word).
 __device__ __forceinline__ bool xch_load(const ulonglong2* p, uint32_t tag, float& m, float& l) {
   unsigned long long a, b;

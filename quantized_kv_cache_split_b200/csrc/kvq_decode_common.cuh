@@ -21,10 +21,7 @@ constexpr float kPUnscale = 1.0f / 16384.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kMagic = 0x64006400u;    // fp16 1024 in both halves (unit mantissa step 1)
 constexpr uint32_t kMagic64 = 0x54005400u;  // fp16 64: mantissa bits 4..7 then count in units of 1
-constexpr size_t kSmemLimit = 232448;       // dynamic shared memory per CTA on sm_100a
 
-constexpr int round128(int x) { return (x + 127) / 128 * 128; }
-constexpr int cmax3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
 
 template <int FMT, int D>
 struct Cfg {
@@ -36,12 +33,8 @@ struct Cfg {
   // fp16 slots per scale row (nvfp4: E4M3 bytes, fp32 vector scale, padding)
   static constexpr int NSC = kLut ? 1 : kNv ? (D / 16 + 4 + 7) / 8 * 4 : D / 32;
   static constexpr int SROW = 2 * NSC;                   // scale bytes per row
-  static constexpr int RPW = 16 / SROW;                  // rows per 16-byte scale window
   static constexpr int NBLK = D / 32;
   static constexpr int KSTEPS = D / 16;
-  static constexpr int STAGE_CODE = kTile * CROW;        // one tile: codes ...
-  static constexpr int STAGE_SC = kTile * SROW;          // ... then scales
-  static constexpr int TILE = STAGE_CODE + STAGE_SC;
   // XOR swizzle of 16-byte chunks within a K code row: chunk ^= (row >> SWZ_SHIFT) & SWZ_MASK
   static constexpr int SWZ_SHIFT = CROW == 128 ? 0 : CROW == 64 ? 1 : 2;
   static constexpr int SWZ_MASK = CROW / 16 - 1;
@@ -52,29 +45,10 @@ struct Cfg {
   static constexpr int RAWB = kQ8 ? E : E / 2;           // code bytes per position per thread
   static constexpr int NWORD = RAWB / 4;
   // q8_0 / q4_0 V pass: codes enter the MMA as magic-number fp16 (code + offset) read
-  // with transposing matrix loads, the scale rides on the weights (see v_group_mag)
+  // with transposing matrix loads, the scale rides on the weights (see vg_mag)
   static constexpr bool kMag = kQ8 || kQ4;
-  // V staging (a whole tile or gathered rows): codes at row stride CROW with the same
-  // chunk swizzle as K, then a tile's scale rows (SROW each) or, for gathered rows, the
-  // 16-byte window of the scales plane that holds each row's scales
-  static constexpr int GSC = STAGE_CODE;                  // gathered rows' scale windows
-  // per-warp buffer: its K tile, then its staged V rows, then its accumulators for the
-  // block-wide sum
-  static constexpr int KBUF = round128(cmax3(TILE, STAGE_CODE + kTile * 16, NE * 32 * 4));
-  static constexpr int VT = round128(TILE);              // per-warp V tile copied with K
   static_assert(CROW % 16 == 0 && (CROW == 128 || CROW == 64 || CROW == 32), "row size");
 };
-
-// cp.async.wait_group with a count known only after unrolling
-__device__ __forceinline__ void cp_async_wait_n(int n) {
-  switch (n) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    case 2: cp_async_wait<2>(); break;
-    case 3: cp_async_wait<3>(); break;
-    default: cp_async_wait<4>(); break;
-  }
-}
 
 // ------------------------------------------------------------------ LUT lookups
 // 16 fp16 centroids held as 4 registers of low bytes and 4 of high bytes; a
@@ -298,8 +272,7 @@ __device__ __forceinline__ void v_raw(const uint8_t* p, uint32_t (&w)[Cfg<FMT, D
 template <int T>
 __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int step, int n,
                                            bool active, uint32_t tag, float& M, float& L,
-                                           long long limit = kWaitCycles, int sleep_ns = 32,
-                                           bool acquire_first = false) {
+                                           long long limit = kWaitCycles, int sleep_ns = 32) {
   M = -INFINITY;
   L = 0.f;
   for (int ub = 0; ub < n; ub += T * step) {
@@ -313,8 +286,7 @@ __device__ __forceinline__ bool xch_reduce(const ulonglong2* e, int first, int s
         mv[t] = -INFINITY;
         lv[t] = 0.f;
         if (active && u < n)
-          all &= (acquire_first && u == 0) ? xch_load_acquire(e, tag, mv[t], lv[t])
-                                           : xch_load(e + u, tag, mv[t], lv[t]);
+          all &= xch_load(e + u, tag, mv[t], lv[t]);
       }
       if (__all_sync(0xffffffffu, all)) break;
       if (__any_sync(0xffffffffu, clock64() - t0 > limit)) return false;

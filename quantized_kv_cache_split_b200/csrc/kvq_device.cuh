@@ -201,18 +201,6 @@ __device__ __forceinline__ void xch_store(ulonglong2* p, uint32_t tag, float m, 
                : "memory");
 }
 
-// Read an entry with acquire semantics (two single-word acquire loads): the writes its
-// publisher made before publishing with release semantics are visible afterwards.
-__device__ __forceinline__ bool xch_load_acquire(const ulonglong2* p, uint32_t tag, float& m, float& l) {
-  unsigned long long a, b;
-  const unsigned long long* w = reinterpret_cast<const unsigned long long*>(p);
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(a) : "l"(w) : "memory");
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(b) : "l"(w + 1) : "memory");
-  m = __uint_as_float((uint32_t)a);
-  l = __uint_as_float((uint32_t)b);
-  return (uint32_t)(a >> 32) == tag && (uint32_t)(b >> 32) == tag;
-}
-
 // Read an entry; false while it is not this launch's (tag mismatch in either word).
 __device__ __forceinline__ bool xch_load(const ulonglong2* p, uint32_t tag, float& m, float& l) {
   unsigned long long a, b;
